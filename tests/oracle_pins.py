@@ -1,0 +1,381 @@
+"""Pins for the CPU oracle: checks against facts that do not come from the oracle itself.
+
+Each pin takes an ``oracle.Oracle`` and raises AssertionError when the oracle disagrees with:
+  * brute force: contiguous attention straight from the generator's logical K/V streams (no
+    block table, no max subtraction, numpy long double);
+  * a library routine: torch's scaled_dot_product_attention in float64 on the CPU;
+  * closed forms: one token, constant values, zero query, a dominant key, two tokens, and a
+    three-token example evaluated with Python's decimal module;
+  * invariants the sources fix: placement of physical blocks, block size, unread slots and
+    block-table entries, shared blocks, and the split-context merge.
+The same pins run against deliberately broken copies of the oracle (test_oracle_mutants.py);
+each broken copy must fail at least one of them.
+
+Sources (vLLM tutorials): [P2] "vLLM core features: PagedAttention, Continuous Batching,
+quantization support, distributed inference" 4.1; [P3] "Core inference engine (part 1): vLLM
+architecture, PagedAttention principle, Continuous Batching mechanism" 2.2; [P4] "vLLM core
+architecture: model loading, PagedAttention principle, KV cache management" 2.2.1, 2.2.2.
+"""
+from __future__ import annotations
+
+import math
+from decimal import Decimal, getcontext
+
+import numpy as np
+
+from paged_kv_cache_427_b200 import workloads as W
+
+REL_TOL_F64 = 1e-12
+
+
+def _rel_err(a, b) -> float:
+    a = np.asarray(a, dtype=np.float64)
+    b = np.asarray(b, dtype=np.float64)
+    scale = max(1e-300, float(np.max(np.abs(b))) if b.size else 1.0)
+    return float(np.max(np.abs(a - b))) / scale if a.size else 0.0
+
+
+def _step(orc, batch: W.PagedBatch):
+    """Run the oracle's step on copies of the pool: copies, writes, then decode."""
+    kc = batch.key_cache.copy()
+    vc = batch.value_cache.copy()
+    if batch.block_mapping is not None and len(batch.block_mapping):
+        assert orc.copy_blocks(kc, vc, batch.block_mapping, batch.dtype) == 0
+    assert orc.reshape_and_cache(batch.key, batch.value, kc, vc, batch.slot_mapping,
+                                 batch.dtype) == 0
+    out = orc.decode(batch.query, kc, vc, batch.block_tables, batch.context_lens, batch.scale,
+                     batch.dtype)
+    return out, kc, vc
+
+
+def brute_force(batch: W.PagedBatch) -> np.ndarray:
+    """Attention over the logical streams, long double, no max subtraction, no paging."""
+    S, Hq, D = batch.query.shape
+    G = Hq // batch.num_kv_heads
+    out = np.zeros((S, Hq, D), dtype=np.longdouble)
+    for s in range(S):
+        L = int(batch.context_lens[s])
+        if L <= 0:
+            continue
+        K = W.decode_to_f64(batch.logical_key[s][:L], batch.dtype).astype(np.longdouble)
+        V = W.decode_to_f64(batch.logical_value[s][:L], batch.dtype).astype(np.longdouble)
+        q = W.decode_to_f64(batch.query[s], batch.dtype).astype(np.longdouble)
+        for h in range(Hq):
+            g = h // G
+            z = np.longdouble(batch.scale) * np.einsum("td,d->t", K[:, g, :], q[h])
+            w = np.exp(z)
+            out[s, h] = np.einsum("t,td->d", w, V[:, g, :]) / w.sum()
+    return out
+
+
+def _small_batches():
+    """Tiny structured cases: several G, D, block sizes and element types."""
+    cases = []
+    rng = np.random.default_rng([W.BASE_SEED, 99])
+    specs = [  # (Hq, Hkv, D, bs, dtype)
+        (4, 4, 64, 16, "f32"),
+        (8, 2, 64, 8, "bf16"),
+        (8, 2, 128, 32, "bf16"),
+        (4, 1, 128, 16, "f32"),
+        (6, 3, 64, 8, "f16"),
+    ]
+    for i, (hq, hkv, d, bs, dt) in enumerate(specs):
+        lens = rng.integers(1, 100, size=5).astype(np.int32)
+        lens[0] = 1
+        lens[1] = bs          # exactly one full block
+        lens[2] = bs + 1      # one token into the second block
+        cases.append(W.build_batch(f"small{i}", lens, num_heads=hq, num_kv_heads=hkv,
+                                   head_dim=d, block_size=bs, dtype=dt,
+                                   seed=W.BASE_SEED + 100 + i, keep_logical=True))
+    cases.append(W.tiny_fp32())
+    return cases
+
+
+# ---------------------------------------------------------------------------------------------
+# pins
+# ---------------------------------------------------------------------------------------------
+
+def pin_brute_force(orc):
+    """The paged oracle equals contiguous long-double attention on the logical streams."""
+    for batch in _small_batches():
+        out, _, _ = _step(orc, batch)
+        ref = brute_force(batch)
+        err = _rel_err(out, ref.astype(np.float64))
+        assert err < REL_TOL_F64, f"{batch.name}: brute-force rel err {err:.3e}"
+
+
+def pin_torch_sdpa(orc):
+    """The oracle equals torch.nn.functional.scaled_dot_product_attention (float64, CPU)."""
+    import torch
+
+    for batch in _small_batches():
+        out, _, _ = _step(orc, batch)
+        S, Hq, D = batch.query.shape
+        for s in range(S):
+            L = int(batch.context_lens[s])
+            K = torch.from_numpy(W.decode_to_f64(batch.logical_key[s][:L], batch.dtype))
+            V = torch.from_numpy(W.decode_to_f64(batch.logical_value[s][:L], batch.dtype))
+            q = torch.from_numpy(W.decode_to_f64(batch.query[s], batch.dtype))
+            ref = torch.nn.functional.scaled_dot_product_attention(
+                q[:, None, :], K.permute(1, 0, 2), V.permute(1, 0, 2), scale=batch.scale,
+                enable_gqa=True)[:, 0, :].numpy()
+            err = _rel_err(out[s], ref)
+            assert err < REL_TOL_F64, f"{batch.name} seq {s}: sdpa rel err {err:.3e}"
+
+
+def _custom(context_lens, key_rows, value_rows, query, *, Hq, Hkv, D, bs=16, dtype="f32",
+            scale=None):
+    """A batch from explicit logical rows ([S] lists of [L, Hkv, D] float arrays)."""
+    b = W.build_batch("custom", context_lens, num_heads=Hq, num_kv_heads=Hkv, head_dim=D,
+                      block_size=bs, dtype=dtype, seed=W.BASE_SEED + 500, keep_logical=True)
+    kc = W._fill_pool(b.key_cache.shape, dtype, "nan")
+    vc = W._fill_pool(b.value_cache.shape, dtype, "nan")
+    for s, L in enumerate(context_lens):
+        kr = W.encode(np.asarray(key_rows[s], np.float32), dtype)
+        vr = W.encode(np.asarray(value_rows[s], np.float32), dtype)
+        W._place(kc, b.block_tables[s], 0, kr[:L - 1], bs)
+        W._place(vc, b.block_tables[s], 0, vr[:L - 1], bs)
+        b.key[s], b.value[s] = kr[L - 1], vr[L - 1]
+        b.logical_key[s], b.logical_value[s] = kr, vr
+    b.key_cache, b.value_cache = kc, vc
+    b.query = W.encode(np.asarray(query, np.float32), dtype)
+    if scale is not None:
+        b.scale = scale
+    return b
+
+
+def pin_closed_forms(orc):
+    """One token -> its value row; equal values -> that value; zero query or equal keys -> mean;
+    a dominant key -> its value row; two tokens -> the logistic mix."""
+    rng = np.random.default_rng(7)
+    Hq, Hkv, D = 4, 2, 64
+    # (a) context of one token: the output is that token's value row, exactly.
+    k1 = [rng.standard_normal((1, Hkv, D)).astype(np.float32) for _ in range(3)]
+    v1 = [rng.standard_normal((1, Hkv, D)).astype(np.float32) for _ in range(3)]
+    q = rng.standard_normal((3, Hq, D)).astype(np.float32)
+    b = _custom([1, 1, 1], k1, v1, q, Hq=Hq, Hkv=Hkv, D=D)
+    out, _, _ = _step(orc, b)
+    for s in range(3):
+        for h in range(Hq):
+            assert np.array_equal(out[s, h], v1[s][0, h // 2].astype(np.float64)), "L=1"
+    # (b) all value rows equal c -> output c.
+    L = 41
+    kk = [rng.standard_normal((L, Hkv, D)).astype(np.float32)]
+    c = rng.standard_normal((Hkv, D)).astype(np.float32)
+    vv = [np.broadcast_to(c, (L, Hkv, D)).copy()]
+    b = _custom([L], kk, vv, rng.standard_normal((1, Hq, D)), Hq=Hq, Hkv=Hkv, D=D)
+    out, _, _ = _step(orc, b)
+    for h in range(Hq):
+        assert _rel_err(out[0, h], c[h // 2]) < 1e-15, "constant V"
+    # (c) zero query -> mean of V; (d) equal keys -> mean of V.
+    vv = [rng.standard_normal((L, Hkv, D)).astype(np.float32)]
+    mean = vv[0].astype(np.float64).mean(axis=0)
+    b = _custom([L], kk, vv, np.zeros((1, Hq, D)), Hq=Hq, Hkv=Hkv, D=D)
+    out, _, _ = _step(orc, b)
+    for h in range(Hq):
+        assert _rel_err(out[0, h], mean[h // 2]) < 1e-13, "zero query"
+    keq = [np.broadcast_to(rng.standard_normal((1, Hkv, D)).astype(np.float32),
+                           (L, Hkv, D)).copy()]
+    b = _custom([L], keq, vv, rng.standard_normal((1, Hq, D)), Hq=Hq, Hkv=Hkv, D=D)
+    out, _, _ = _step(orc, b)
+    for h in range(Hq):
+        assert _rel_err(out[0, h], mean[h // 2]) < 1e-13, "equal keys"
+    # (e) one key whose logit leads every other by more than 60 -> its value row.
+    qd = np.zeros((1, Hq, D), np.float32)
+    qd[0, :, 0] = 1.0
+    kd = np.zeros((L, Hkv, D), np.float32)
+    kd[:, :, 1:] = rng.standard_normal((L, Hkv, D - 1))
+    j = 29
+    kd[j, :, 0] = 512.0  # scale 1/8 -> logit 64, others 0
+    b = _custom([L], [kd], vv, qd, Hq=Hq, Hkv=Hkv, D=D, scale=1.0 / 8)
+    out, _, _ = _step(orc, b)
+    for h in range(Hq):
+        assert _rel_err(out[0, h], vv[0][j, h // 2]) < 1e-20 * L + 1e-26, "dominant key"
+    # (f) two tokens: out = s(z0 - z1) v0 + s(z1 - z0) v1 with s the logistic function.
+    q2 = np.zeros((1, Hq, D), np.float32)
+    q2[0, :, 0] = 2.0
+    k2 = np.zeros((2, Hkv, D), np.float32)
+    k2[0, :, 0] = 0.75
+    k2[1, :, 0] = -1.25
+    v2 = rng.standard_normal((2, Hkv, D)).astype(np.float32)
+    b = _custom([2], [k2], [v2], q2, Hq=Hq, Hkv=Hkv, D=D, scale=0.5)
+    out, _, _ = _step(orc, b)
+    z0, z1 = 0.5 * 2.0 * 0.75, 0.5 * 2.0 * -1.25
+    s01 = 1.0 / (1.0 + math.exp(z1 - z0))
+    for h in range(Hq):
+        ref = s01 * v2[0, h // 2].astype(np.float64) + (1 - s01) * v2[1, h // 2].astype(np.float64)
+        assert _rel_err(out[0, h], ref) < 1e-15, "two tokens"
+
+
+def pin_decimal_example(orc):
+    """Three tokens with logits {0, 1, -2} (exact in binary), values evaluated with 40-digit
+    decimal arithmetic; the context straddles a block boundary (block_size 2)."""
+    getcontext().prec = 40
+    Hq = Hkv = 1
+    D = 64
+    q = np.zeros((1, 1, D), np.float32)
+    q[0, 0, 0] = 1.0
+    k = np.zeros((3, 1, D), np.float32)
+    k[:, 0, 0] = [0.0, 1.0, -2.0]
+    v = np.zeros((3, 1, D), np.float32)
+    v[:, 0, 0] = [1.0, 2.0, 4.0]
+    v[:, 0, 1] = [-3.0, 0.5, 8.0]
+    b = _custom([3], [k], [v], q, Hq=Hq, Hkv=Hkv, D=D, bs=8, scale=1.0)
+    b2 = W.build_batch("custom", [3], num_heads=1, num_kv_heads=1, head_dim=D, block_size=2,
+                       dtype="f32", seed=1, keep_logical=True)
+    kc = W._fill_pool(b2.key_cache.shape, "f32", "nan")
+    vc = W._fill_pool(b2.value_cache.shape, "f32", "nan")
+    W._place(kc, b2.block_tables[0], 0, k, 2)
+    W._place(vc, b2.block_tables[0], 0, v, 2)
+    for batch, caches in ((b, None), (b2, (kc, vc))):
+        if caches is None:
+            out, _, _ = _step(orc, batch)
+        else:
+            out = orc.decode(q, caches[0], caches[1], b2.block_tables, np.array([3], np.int32),
+                             1.0, "f32")
+        e = [Decimal(z).exp() for z in (0, 1, -2)]
+        den = sum(e)
+        exp0 = (e[0] * 1 + e[1] * 2 + e[2] * 4) / den
+        exp1 = (e[0] * Decimal(-3) + e[1] * Decimal("0.5") + e[2] * 8) / den
+        assert abs(Decimal(float(out[0, 0, 0])) - exp0) < Decimal("1e-15"), "decimal d0"
+        assert abs(Decimal(float(out[0, 0, 1])) - exp1) < Decimal("1e-15"), "decimal d1"
+        assert np.all(out[0, 0, 2:] == 0.0), "decimal zeros"
+
+
+def pin_placement_invariance(orc):
+    """[P4] 2.2.1: physical blocks may sit anywhere.  Same logical values, other permutation or
+    other block size (8/16/32), unread slots poisoned or zeroed -> bit-identical output."""
+    lens = np.array([1, 7, 8, 9, 33, 70], np.int32)
+    outs = []
+    for bs in (8, 16, 32):
+        for salt in (0, 1):
+            for fill in ("nan", "zero"):
+                b = W.build_batch("inv", lens, num_heads=8, num_kv_heads=2, head_dim=64,
+                                  block_size=bs, dtype="bf16", seed=W.BASE_SEED + 700,
+                                  perm_salt=salt, fill=fill, pool_factor=2.0)
+                outs.append(_step(orc, b)[0])
+    for o in outs[1:]:
+        assert np.array_equal(o, outs[0]), "placement / block size changed the output"
+
+
+def pin_unread_table_entries(orc):
+    """Block-table entries past a sequence's last block are never read, however invalid."""
+    b = W.build_batch("tab", [5, 17, 40], num_heads=4, num_kv_heads=2, head_dim=64,
+                      block_size=16, dtype="bf16", seed=W.BASE_SEED + 701, max_blocks=6)
+    ref, _, _ = _step(orc, b)
+    t = b.block_tables.copy()
+    t[t < 0] = 2 ** 30
+    b.block_tables = t
+    out, _, _ = _step(orc, b)
+    assert np.array_equal(out, ref), "entries past the context changed the output"
+
+
+def pin_cache_write(orc):
+    """[P2] 4.1: a new token lands at offset slot % bs of block slot / bs.  Reading every
+    sequence back through its block table gives its logical stream; nothing else changes;
+    negative slots store nothing; slots outside the pool are refused."""
+    for batch in _small_batches() + [W.shared_prefix(num_groups=3, suffix_range=(16, 60),
+                                                     keep_logical=True)]:
+        _, kc, vc = _step(orc, batch)
+        bs = batch.block_size
+        for s in range(batch.num_seqs):
+            L = int(batch.context_lens[s])
+            t = np.arange(L)
+            phys = batch.block_tables[s][t // bs]
+            got_k = kc[phys, :, t % bs, :]
+            got_v = vc[phys, :, t % bs, :]
+            assert np.array_equal(got_k.view(np.uint8), batch.logical_key[s][:L].view(np.uint8))
+            assert np.array_equal(got_v.view(np.uint8), batch.logical_value[s][:L].view(np.uint8))
+        # bytes outside the written slots and the copied blocks are untouched
+        touched = np.zeros(kc.shape[:1] + kc.shape[2:3], bool)
+        for sl in batch.slot_mapping:
+            touched[sl // bs, sl % bs] = True
+        if batch.block_mapping is not None:
+            for _, dst in batch.block_mapping:
+                touched[dst, :] = True
+        keep = ~touched
+        a = kc.transpose(0, 2, 1, 3)[keep]
+        b0 = batch.key_cache.transpose(0, 2, 1, 3)[keep]
+        assert np.array_equal(a.view(np.uint8), b0.view(np.uint8)), "untouched slots changed"
+    b = W.tiny_fp32()
+    kc, vc = b.key_cache.copy(), b.value_cache.copy()
+    slots = b.slot_mapping.copy()
+    slots[1] = -1                               # padding token: stores nothing
+    slots[2] = b.num_blocks * b.block_size      # first slot past the pool: refused
+    skipped = orc.reshape_and_cache(b.key, b.value, kc, vc, slots, "f32")
+    assert skipped == 1, "out-of-pool slot not refused"
+    expect_k = b.key_cache.copy()
+    expect_v = b.value_cache.copy()
+    for s in (0, 3):                            # only these two tokens are stored
+        blk, off = divmod(int(b.slot_mapping[s]), b.block_size)
+        expect_k[blk, :, off] = b.key[s]
+        expect_v[blk, :, off] = b.value[s]
+    assert np.array_equal(kc.view(np.uint8), expect_k.view(np.uint8)), "skip/refuse broke K"
+    assert np.array_equal(vc.view(np.uint8), expect_v.view(np.uint8)), "skip/refuse broke V"
+
+
+def pin_copy_blocks(orc):
+    """Copy-on-write of shared blocks ([P2] 4.1, [P3] 2.2): every dst block equals its src in
+    both caches afterwards, other blocks keep their bytes, ids outside the pool are refused."""
+    b = W.build_batch("cow", [30, 50], num_heads=4, num_kv_heads=2, head_dim=64, block_size=8,
+                      dtype="bf16", seed=W.BASE_SEED + 702, fill="zero", pool_factor=3.0)
+    rng = np.random.default_rng(3)
+    kc = W.encode(rng.standard_normal(b.key_cache.shape).astype(np.float32), "bf16")
+    vc = W.encode(rng.standard_normal(b.value_cache.shape).astype(np.float32), "bf16")
+    k0, v0 = kc.copy(), vc.copy()
+    pairs = np.array([[0, 5], [3, 1], [7, 2], [0, 9]], np.int64)
+    assert orc.copy_blocks(kc, vc, pairs, "bf16") == 0
+    for src, dst in pairs:
+        assert np.array_equal(kc[dst], k0[src]) and np.array_equal(vc[dst], v0[src])
+    dsts = set(pairs[:, 1].tolist())
+    for blk in range(kc.shape[0]):
+        if blk not in dsts:
+            assert np.array_equal(kc[blk], k0[blk]) and np.array_equal(vc[blk], v0[blk])
+    bad = np.array([[0, kc.shape[0]], [-1, 4]], np.int64)
+    k1 = kc.copy()
+    assert orc.copy_blocks(kc, vc, bad, "bf16") == 2
+    assert np.array_equal(kc, k1)
+
+
+def pin_shared_prefix(orc):
+    """Sequences sharing prefix blocks read the same bytes: the paged result over the shared
+    pool equals brute force on each member's own logical stream."""
+    b = W.shared_prefix(num_groups=2, prefix_len=64, suffix_range=(16, 40), keep_logical=True)
+    out, _, _ = _step(orc, b)
+    err = _rel_err(out, brute_force(b).astype(np.float64))
+    assert err < REL_TOL_F64, f"shared prefix rel err {err:.3e}"
+
+
+def pin_split_merge(orc):
+    """Split-context partitions merged with the log-sum-exp rule reproduce the unsplit
+    result; empty partitions are neutral."""
+    b = W.build_batch("split", [1, 20, 64, 100], num_heads=8, num_kv_heads=2, head_dim=128,
+                      block_size=16, dtype="bf16", seed=W.BASE_SEED + 703)
+    full, kc, vc = _step(orc, b)
+    for bounds in ([0, 16, 48, 10 ** 6], [0, 1, 2, 3, 99, 10 ** 6], [0, 64, 64, 200, 10 ** 6]):
+        parts = [orc.decode_range(b.query, kc, vc, b.block_tables, b.context_lens, b.scale,
+                                  "bf16", lo, hi) for lo, hi in zip(bounds[:-1], bounds[1:])]
+        for s in range(b.num_seqs):
+            for h in range(b.num_heads):
+                o = np.stack([p[0][s, h] for p in parts])
+                m = np.array([p[1][s, h] for p in parts])
+                l = np.array([p[2][s, h] for p in parts])
+                merged = orc.lse_combine(o, m, l)
+                assert _rel_err(merged, full[s, h]) < REL_TOL_F64, f"merge {bounds} s{s} h{h}"
+
+
+def pin_zero_context(orc):
+    """A sequence with no context gives a zero row; its neighbours are unaffected."""
+    b = W.build_batch("zero", [0, 5, 0, 9], num_heads=4, num_kv_heads=1, head_dim=64,
+                      block_size=8, dtype="f32", seed=W.BASE_SEED + 704, keep_logical=True)
+    out, _, _ = _step(orc, b)
+    assert np.all(out[0] == 0) and np.all(out[2] == 0), "empty context not zero"
+    ref = brute_force(b).astype(np.float64)
+    assert _rel_err(out[1], ref[1]) < REL_TOL_F64 and _rel_err(out[3], ref[3]) < REL_TOL_F64
+
+
+ALL_PINS = [
+    pin_brute_force, pin_torch_sdpa, pin_closed_forms, pin_decimal_example,
+    pin_placement_invariance, pin_unread_table_entries, pin_cache_write, pin_copy_blocks,
+    pin_shared_prefix, pin_split_merge, pin_zero_context,
+]
