@@ -1,0 +1,493 @@
+"""Benchmark of the paged-attention decode step on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+A step is one pass of the whole hot path over one batch: the new tokens' cache write
+(pa_reshape_and_cache; plus pa_copy_blocks for the shared-prefix workload) followed by the
+decode (pa_decode).  The default workload is the Llama-3-8B-shaped decode step: 64 sequences,
+32 query / 8 KV heads, head_dim 128, bf16, block_size 16, contexts U[128, 2048].
+
+`value` is the whole-job throughput in algorithmic GB/s: the bytes a step must move (every
+attended K/V row once, Q and out, block-table entries, context lengths, the written rows), with
+inputs resident in HBM.  To keep L2 (126 MB) from serving repeated reads, consecutive steps
+rotate over several copies of the KV pool whose attended bytes each exceed L2.  `e2e` is the
+same metric measured through the same public calls with the step's inputs copied from pinned
+host memory and the output read back every step.  `roofline` relates the decode kernel's
+algorithmic bytes per launch to its mean CUDA-event duration and the measured HBM copy
+bandwidth.  `cpu_baseline` times the CPU oracle on a bounded sample of the same workload.
+
+With --gpus N (launched under torchrun) every rank runs an independent replica of the step on
+its own GPU: the path has no exchange step, so there is no collective on the data path.
+--impl reference times the CPU oracle as the reference arm.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from paged_kv_cache_427_b200 import workloads as W  # noqa: E402
+
+METRIC = "paged decode attention KV GB/s (% of B200 HBM peak), attended tokens/s"
+NOMINAL_HBM_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+L2_BYTES = 126 * 2 ** 20
+ELT = {"f32": 4, "bf16": 2, "f16": 2}
+
+
+# ----------------------------------------------------------------------------------------------
+# byte accounting
+# ----------------------------------------------------------------------------------------------
+
+def decode_bytes(b: W.PagedBatch, out_elt: int, unique: bool = True) -> int:
+    """Algorithmic bytes of one decode: each attended K/V row once (a physical slot shared by
+    several sequences counts once when `unique`), Q and out rows, the block-table entries of
+    each context and the context lengths."""
+    e = ELT[b.dtype]
+    lens = np.maximum(b.context_lens.astype(np.int64), 0)
+    row = b.num_kv_heads * b.head_dim * e * 2  # K and V of one token, all kv heads
+    if unique:
+        slots = []
+        for s, L in enumerate(lens):
+            if L:
+                t = np.arange(L)
+                slots.append(b.block_tables[s, t // b.block_size].astype(np.int64) * b.block_size
+                             + t % b.block_size)
+        kv = (len(np.unique(np.concatenate(slots))) if slots else 0) * row
+    else:
+        kv = int(lens.sum()) * row
+    qo = b.num_seqs * b.num_heads * b.head_dim * (e + out_elt)
+    tables = int(((lens + b.block_size - 1) // b.block_size).sum()) * 4 + b.num_seqs * 4
+    return int(kv + qo + tables)
+
+
+def write_bytes(b: W.PagedBatch) -> int:
+    """New K/V rows read and stored, their slots, and whole-block copies (read + write)."""
+    e = ELT[b.dtype]
+    t = int((b.slot_mapping >= 0).sum())
+    rows = t * b.num_kv_heads * b.head_dim * e * 2 * 2 + len(b.slot_mapping) * 8
+    copies = 0
+    if b.block_mapping is not None:
+        copies = len(b.block_mapping) * (b.num_kv_heads * b.block_size * b.head_dim * e * 2 * 2 + 16)
+    return int(rows + copies)
+
+
+def attended_bytes(b: W.PagedBatch) -> int:
+    lens = np.maximum(b.context_lens.astype(np.int64), 0)
+    return int(lens.sum()) * b.num_kv_heads * b.head_dim * ELT[b.dtype] * 2
+
+
+# ----------------------------------------------------------------------------------------------
+# environment facts
+# ----------------------------------------------------------------------------------------------
+
+def hbm_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_sources_digest() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "paged_kv_cache_427_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        if f.endswith((".cu", ".cuh", ".h")):
+            with open(os.path.join(csrc, f), "rb") as fh:
+                h.update(f.encode() + fh.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload: str):
+    """DRAM bytes per decode launch from the committed ncu summary, if it was taken on the
+    current kernel sources; else None."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)
+        entry = rec.get(workload)
+        if entry and entry.get("sources") == kernel_sources_digest():
+            return float(entry["dram_bytes_per_launch"])
+    except Exception:
+        pass
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons while the GPU works."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str | None):
+        self.proc = None
+        self.gpu_id = gpu_id
+
+    def start(self):
+        cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "100"]
+        if self.gpu_id:
+            cmd += ["-i", self.gpu_id]
+        try:
+            self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+        return self
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=10)
+        except Exception:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, smax, power, reasons = [], [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            p = [x.strip() for x in line.split(",")]
+            if len(p) < 9:
+                continue
+            try:
+                sm.append(float(p[1]))
+                smax.append(float(p[2]))
+                power.append(float(p[3]))
+            except ValueError:
+                continue
+            for n, v in zip(names, p[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return None
+        # samples under load: the upper half by power draw
+        cut = statistics.median(power)
+        loaded = [s for s, pw in zip(sm, power) if pw >= cut] or sm
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": max(smax),
+                "reasons": sorted(reasons), "samples": len(sm),
+                "power_w_max": max(power)}
+
+
+# ----------------------------------------------------------------------------------------------
+# the oracle (CPU baseline and reference arm)
+# ----------------------------------------------------------------------------------------------
+
+def oracle_sample_run(b: W.PagedBatch, budget_s: float, orc):
+    """Time the oracle's step on the first n sequences, n grown until one run takes about
+    budget_s.  Returns (seconds, n, algorithmic bytes of the sample, attended tokens)."""
+    kc, vc = b.key_cache, b.value_cache
+    n = 1
+    while True:
+        sub = W.sub_batch(b, np.arange(n))
+        t0 = time.perf_counter()
+        orc.decode(sub["query"], kc, vc, sub["block_tables"], sub["context_lens"], b.scale, b.dtype)
+        dt = time.perf_counter() - t0
+        if dt >= budget_s or n == b.num_seqs:
+            break
+        n = min(b.num_seqs, max(n + 1, int(n * min(8.0, budget_s / max(dt, 1e-4)))))
+    sb = W.PagedBatch(**{**b.__dict__, "query": sub["query"], "block_tables": sub["block_tables"],
+                          "context_lens": sub["context_lens"]})
+    return dt, n, decode_bytes(sb, ELT[b.dtype], unique=False), int(sub["context_lens"].sum())
+
+
+def cpu_baseline(b: W.PagedBatch, budget_s: float = 10.0):
+    import oracle
+
+    orc = oracle.load()
+    dt, n, nbytes, toks = oracle_sample_run(b, budget_s, orc)
+    return {"value": round(nbytes / dt / 1e9, 4), "unit": "GB/s", "cores": orc.max_threads(),
+            "kind": "oracle",
+            "sample": f"oracle decode (fp64, OpenMP) of the first {n} of {b.num_seqs} sequences "
+                      f"({toks} attended tokens), one run of {dt:.2f} s",
+            "attended_tokens_per_s": round(toks / dt, 1)}
+
+
+def run_reference(args, b: W.PagedBatch, config: dict):
+    import oracle
+
+    orc = oracle.load()
+    steps, warmup = args.steps, args.warmup
+    # each step decodes a bounded sample, sized so the whole run takes about two minutes
+    per_step = max(0.005, 120.0 / max(1, steps + warmup))
+    _, n, nbytes, toks = oracle_sample_run(b, per_step, orc)
+    sub = W.sub_batch(b, np.arange(n))
+    kc, vc = b.key_cache.copy(), b.value_cache.copy()
+
+    def step():
+        orc.reshape_and_cache(b.key[:n], b.value[:n], kc, vc, b.slot_mapping[:n], b.dtype)
+        orc.decode(sub["query"], kc, vc, sub["block_tables"], sub["context_lens"], b.scale, b.dtype)
+
+    for _ in range(warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(steps):
+        step()
+    dt = (time.perf_counter() - t0) / max(1, steps)
+    e = ELT[b.dtype]
+    step_bytes = nbytes + n * b.num_kv_heads * b.head_dim * e * 4 + n * 8
+    value = step_bytes / dt / 1e9
+    line = {"impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s",
+            "n_gpus": args.gpus, "steps": steps, "warmup": warmup, "ms_per_step": round(dt * 1e3, 4),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": config,
+            "attended_tokens_per_s": round(toks / dt, 1),
+            "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": orc.max_threads(),
+                             "kind": "oracle",
+                             "sample": f"each step: oracle cache write + decode of the first {n} of "
+                                       f"{b.num_seqs} sequences ({toks} attended tokens)"},
+            "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ----------------------------------------------------------------------------------------------
+# the CUDA path
+# ----------------------------------------------------------------------------------------------
+
+def make_batch(name: str) -> W.PagedBatch:
+    return W.workload(name)
+
+
+def run_ours(args, b: W.PagedBatch, config: dict, rank: int, world: int, local_rank: int):
+    import torch
+    import torch.distributed as dist
+
+    import paged_kv_cache_427_b200 as pa
+
+    pa.load()
+    dev = torch.device("cuda", local_rank)
+    tdt = {"bf16": torch.bfloat16, "f16": torch.float16, "f32": torch.float32}[b.dtype]
+    out_dtype = tdt
+
+    def dev_t(a, dt=None):
+        if dt == "bf16":
+            return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
+        return torch.from_numpy(np.ascontiguousarray(a)).to(dev)
+
+    # rotating pools: enough copies that each step's attended bytes push the previous step's
+    # rows out of L2 before they are read again
+    att = attended_bytes(b)
+    rot = args.rotations or max(2, min(8, math.ceil(3 * L2_BYTES / max(att, 1)) + 1))
+    kc0 = dev_t(b.key_cache, b.dtype)
+    vc0 = dev_t(b.value_cache, b.dtype)
+    pools = [(kc0, vc0)] + [(kc0.clone(), vc0.clone()) for _ in range(rot - 1)]
+    q = dev_t(b.query, b.dtype)
+    key = dev_t(b.key, b.dtype)
+    value = dev_t(b.value, b.dtype)
+    slots = dev_t(b.slot_mapping)
+    tables = dev_t(b.block_tables)
+    lens = dev_t(b.context_lens)
+    mapping = dev_t(b.block_mapping) if b.block_mapping is not None and len(b.block_mapping) else None
+    out = torch.empty(q.shape, dtype=out_dtype, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step(i, ev=None):
+        kc, vc = pools[i % rot]
+        if mapping is not None:
+            pa.pa_copy_blocks(kc, vc, mapping)
+        pa.pa_reshape_and_cache(key, value, kc, vc, slots)
+        if ev is not None:
+            ev[0].record(stream)
+        pa.pa_decode(out, q, kc, vc, tables, lens, b.scale, b.block_size, b.num_kv_heads)
+        if ev is not None:
+            ev[1].record(stream)
+
+    launches_per_step = 2 + (1 if mapping is not None else 0)
+    gpu_uuid = None
+    try:
+        gpu_uuid = str(torch.cuda.get_device_properties(dev).uuid)
+        if not gpu_uuid.startswith("GPU-"):
+            gpu_uuid = "GPU-" + gpu_uuid
+    except Exception:
+        pass
+    sampler = ClockSampler(gpu_uuid).start()
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    # a short soak so the clock sampler sees the GPU under this load even when K is small
+    t_soak = time.perf_counter()
+    i = 0
+    while time.perf_counter() - t_soak < args.soak:
+        for _ in range(200):
+            step(i)
+            i += 1
+        torch.cuda.synchronize()
+
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    start.record(stream)
+    for i in range(args.steps):
+        step(i, evs[i])
+    end.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    elapsed_ms = start.elapsed_time(end)
+    decode_ms = [s.elapsed_time(e) for s, e in evs]
+
+    # end to end through the same calls: inputs from pinned host memory, output read back
+    def host_t(a, dt=None):
+        a = np.ascontiguousarray(a)
+        t = torch.from_numpy(a.view(np.int16) if dt == "bf16" else a)
+        return (t.view(torch.bfloat16) if dt == "bf16" else t).pin_memory()
+
+    h_q = host_t(b.query, b.dtype)
+    h_in = {"key": host_t(b.key, b.dtype), "value": host_t(b.value, b.dtype),
+            "slots": host_t(b.slot_mapping), "tables": host_t(b.block_tables),
+            "lens": host_t(b.context_lens)}
+    h_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    d_in = {k: torch.empty_like(v, device=dev) for k, v in h_in.items()}
+    d_q = torch.empty_like(h_q, device=dev)
+    h2d = sum(v.numel() * v.element_size() for v in h_in.values()) + h_q.numel() * h_q.element_size()
+    d2h = h_out.numel() * h_out.element_size()
+
+    def e2e_step(i):
+        d_q.copy_(h_q, non_blocking=True)
+        for k in d_in:
+            d_in[k].copy_(h_in[k], non_blocking=True)
+        kc, vc = pools[i % rot]
+        if mapping is not None:
+            pa.pa_copy_blocks(kc, vc, mapping)
+        pa.pa_reshape_and_cache(d_in["key"], d_in["value"], kc, vc, d_in["slots"])
+        pa.pa_decode(out, d_q, kc, vc, d_in["tables"], d_in["lens"], b.scale, b.block_size, b.num_kv_heads)
+        h_out.copy_(out, non_blocking=True)
+        stream.synchronize()
+
+    e2e_steps = args.steps
+    for i in range(min(args.warmup, 50)):
+        e2e_step(i)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e_start, e_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e_start.record(stream)
+    for i in range(e2e_steps):
+        e2e_step(i)
+    e_end.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e_start.elapsed_time(e_end)
+    clocks = sampler.stop()
+
+    if world > 1:
+        t = torch.tensor([elapsed_ms, e2e_ms, float(np.mean(decode_ms))], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        elapsed_ms, e2e_ms, dec_mean = t.tolist()
+    else:
+        dec_mean = float(np.mean(decode_ms))
+    flags = pa.pa_get_device_error(clear=True)
+    if rank != 0:
+        return
+    if flags:
+        print(f"warning: device error word 0x{flags:x}", file=sys.stderr)
+
+    out_elt = torch.tensor([], dtype=out_dtype).element_size()
+    dec_unique = decode_bytes(b, out_elt, unique=True)
+    dec_logical = decode_bytes(b, out_elt, unique=False)
+    step_bytes = dec_unique + write_bytes(b)
+    ms = elapsed_ms / args.steps
+    value = world * step_bytes / (ms * 1e-3) / 1e9
+    e2e_ms_step = e2e_ms / e2e_steps
+    peak, peak_src = hbm_peak()
+    achieved = dec_unique / (dec_mean * 1e-3) / 1e9
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": b.dtype,
+        "data": "synthetic", "config": config,
+        "attended_tokens_per_s": round(world * b.attended_tokens / (ms * 1e-3), 1),
+        "seq_steps_per_s": round(world * b.num_seqs / (ms * 1e-3), 1),
+        "pct_of_8TBs": round(100 * value / world / NOMINAL_HBM_GBS, 2),
+        f"pct_of_{peak_src}_hbm": round(100 * value / world / peak, 2),
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak, "unit": "GB/s",
+                     "frac": round(achieved / peak, 4), "traffic": recorded_traffic(config["workload"]),
+                     "kernel": "paged_decode_kernel", "peak_source": peak_src,
+                     "algorithmic_bytes_per_launch": dec_unique,
+                     "mean_launch_us": round(dec_mean * 1e3, 3)},
+        "e2e": {"value": round(world * step_bytes / (e2e_ms_step * 1e-3) / 1e9, 2), "unit": "GB/s",
+                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+                "ms_per_step": round(e2e_ms_step, 5)},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clocks,
+    }
+    if dec_logical != dec_unique:
+        line["logical_GBps"] = round(world * (dec_logical + write_bytes(b)) / (ms * 1e-3) / 1e9, 2)
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(b, args.cpu_seconds)
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--workload", default="llama3_8b_decode",
+                    help="llama3_8b_decode | short_chat_bs{8,16,32} | shared_prefix | long_mixed | tiny_fp32")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--rotations", type=int, default=0, help="copies of the KV pool (0 = enough to defeat L2)")
+    ap.add_argument("--soak", type=float, default=1.0, help="seconds of untimed load for the clock sampler")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("at least 3 warm-up steps")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        args.gpus = world if world > 1 else args.gpus
+    b = make_batch(args.workload)
+    config = {"workload": args.workload, "num_seqs": b.num_seqs, "num_heads": b.num_heads,
+              "num_kv_heads": b.num_kv_heads, "head_dim": b.head_dim, "block_size": b.block_size,
+              "kv_dtype": b.dtype, "attended_tokens": b.attended_tokens,
+              "num_blocks": b.num_blocks, "max_blocks_per_seq": b.max_blocks,
+              "seed": b.meta.get("seed"),
+              "l2": "inputs larger than L2: steps rotate over copies of the KV pool",
+              "pool_rotations": args.rotations or "auto",
+              "parallelism": f"replicas x{world}" if world > 1 else "single GPU"}
+
+    if args.impl == "reference":
+        if rank == 0:
+            run_reference(args, b, config)
+        return
+
+    import torch
+
+    torch.cuda.set_device(local_rank)
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        run_ours(args, b, config, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

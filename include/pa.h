@@ -1,0 +1,214 @@
+/*
+ * pa.h - C ABI of a paged KV-cache decode-attention library for NVIDIA B200 (sm_100a).
+ *
+ * Sources (web tutorials on vLLM, cited by page and section):
+ *   [P2] "vLLM core features: PagedAttention, Continuous Batching, quantization support,
+ *        distributed inference", section 4.1: the KV cache is cut into fixed-size blocks; a
+ *        block table records the physical block behind each logical block; generating a token
+ *        appends one mapping; several sequences may share physical blocks.
+ *   [P3] "Core inference engine (part 1): vLLM architecture, PagedAttention principle,
+ *        Continuous Batching mechanism", section 2.2: pages of a fixed number of tokens (e.g.
+ *        16) scattered through memory and found through a page table; shared prompt pages;
+ *        page size is a tuning parameter (8 vs 32).
+ *   [P4] "vLLM core architecture: model loading, PagedAttention principle, KV cache
+ *        management", section 2.2.1 (logical block, physical block of the same size, block
+ *        table; block size 16 by default, 8 or 32 as alternatives) and section 2.2.2
+ *        (attention assembles each sequence's complete KV sequence through its block table).
+ *
+ * Conventions shared by every call
+ *   - Tensors are described by pa_tensor: a device pointer, an element type, a shape and
+ *     strides counted in elements.  The caller owns every buffer; the library never frees or
+ *     keeps a caller pointer beyond the call.  All buffers of one call live on the current CUDA
+ *     device.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = the legacy default stream).  Every
+ *     call only enqueues work on that stream and returns; none reads device data on the host
+ *     or synchronises, except pa_get_device_error, which says so.  Launch sizes come from
+ *     shapes only, never from the values in context_lens.
+ *   - Host-side checks (shapes, element types, strides, 16-byte alignment, that every tensor
+ *     lies inside one device allocation) reject bad arguments before anything is enqueued;
+ *     the call then returns a negative pa_status and pa_last_error() describes the problem.
+ *   - Values that only the device sees (block ids, slots, context lengths) are checked by the
+ *     kernels: a bad value sets a bit in the per-device error word (pa_get_device_error) and
+ *     the offending access is redirected or skipped, never performed out of bounds.  The
+ *     result for the affected sequence is then unspecified.
+ *
+ * Layouts
+ *   key_cache, value_cache  [num_blocks, num_kv_heads, block_size, head_dim]; the innermost
+ *                           two dimensions contiguous (so one (block, kv head) tile is one
+ *                           contiguous run of block_size * head_dim elements); the two caches
+ *                           share shape, element type and strides.  Physical-block-major order
+ *                           follows [P4] 2.2.2; head before token is this library's choice.
+ *   query, out              [num_seqs, num_heads, head_dim], head_dim contiguous.
+ *   key, value (new tokens) [num_tokens, num_kv_heads, head_dim], head_dim contiguous.
+ *   block_tables            [num_seqs, max_blocks] int32, row-major with unit inner stride.
+ *   context_lens            [num_seqs] int32, contiguous; counts every token of the sequence,
+ *                           including the one written in this step.
+ *   slot_mapping            [num_tokens] int64, contiguous; slot = block * block_size + offset,
+ *                           negative = padding token (nothing stored).
+ *   block_mapping           [num_pairs, 2] int64, contiguous (src, dst) block ids.
+ * Query head h reads kv head h / (num_heads / num_kv_heads).
+ *
+ * Supported: element types fp32, bf16, fp16 (query and caches of one type; out either that
+ * type or fp32); head_dim 64 or 128; block_size 8, 16 or 32; num_heads / num_kv_heads in
+ * {1, 2, 4, 8}.  Other combinations return PA_ERR_UNSUPPORTED.
+ */
+#ifndef PA_H_
+#define PA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define PA_VERSION 1
+
+/* Symbols of this ABI are the only ones the shared library exports. */
+#if defined(__GNUC__)
+#define PA_API __attribute__((visibility("default")))
+#else
+#define PA_API
+#endif
+
+typedef enum pa_dtype { PA_F32 = 0, PA_BF16 = 1, PA_F16 = 2, PA_I32 = 3, PA_I64 = 4 } pa_dtype;
+
+#define PA_MAX_DIMS 5
+
+typedef struct pa_tensor {
+  void *data;                  /* device pointer of element [0, 0, ...] */
+  int32_t dtype;               /* pa_dtype */
+  int32_t ndim;                /* 1 .. PA_MAX_DIMS */
+  int64_t shape[PA_MAX_DIMS];  /* sizes; entries past ndim are ignored */
+  int64_t stride[PA_MAX_DIMS]; /* strides in elements; entries past ndim are ignored */
+} pa_tensor;
+
+typedef enum pa_status {
+  PA_OK = 0,
+  PA_ERR_INVALID_ARG = -1, /* NULL pointer, negative size, unknown flag, ... */
+  PA_ERR_SHAPE = -2,       /* shapes disagree with each other or with block_size/num_kv_heads */
+  PA_ERR_DTYPE = -3,       /* element type not allowed for this argument */
+  PA_ERR_UNSUPPORTED = -4, /* valid but not built: head_dim, block_size or group size */
+  PA_ERR_CUDA = -5,        /* a CUDA runtime call or a launch failed; see pa_last_error() */
+  PA_ERR_WORKSPACE = -6,   /* workspace missing, too small or misaligned */
+  PA_ERR_LAYOUT = -7       /* stride or alignment requirement not met, or tensor not inside
+                              one device allocation of the current device */
+} pa_status;
+
+/* Bits of the per-device error word set by kernels (see pa_get_device_error). */
+#define PA_DEVERR_BLOCK_ID 0x1u    /* a block-table entry needed for a context lay outside
+                                      [0, num_blocks); block 0 was read instead */
+#define PA_DEVERR_CONTEXT_LEN 0x2u /* context_len < 0 (treated as 0) or > max_blocks *
+                                      block_size (clamped) */
+#define PA_DEVERR_SLOT 0x4u        /* slot >= num_blocks * block_size; the token was skipped */
+#define PA_DEVERR_COPY_PAIR 0x8u   /* a copy pair held an id outside [0, num_blocks); skipped */
+#define PA_DEVERR_TIMEOUT 0x10u    /* an asynchronous copy did not complete within about one
+                                      second; the kernel abandoned its work and returned.  The
+                                      decode workspace must be re-initialised afterwards */
+
+/* Flags of pa_decode_ex. */
+#define PA_DECODE_SEPARATE_REDUCE 0x1u /* merge split contexts in a second kernel instead of
+                                          in the last warp to finish each (sequence, kv head) */
+
+/*
+ * pa_reshape_and_cache - store this step's new keys and values into their cache slots.
+ * [P2] 4.1: each generated token appends one logical->physical mapping; the scheduler hands
+ * the token a slot, and its K/V rows go to offset slot % block_size of physical block
+ * slot / block_size, for every kv head:
+ *   key_cache[slot / bs, h, slot % bs, :] = key[i, h, :]   (value alike), for slot >= 0.
+ * key, value: [T, Hkv, D]; caches as above; slot_mapping: [T] int64.  Copies are bit-exact.
+ * Slots must be distinct within a call (otherwise which token lands is unspecified).
+ * A slot >= num_blocks * block_size sets PA_DEVERR_SLOT and that token is skipped.
+ */
+PA_API int pa_reshape_and_cache(const pa_tensor *key, const pa_tensor *value,
+                         const pa_tensor *key_cache, const pa_tensor *value_cache,
+                         const pa_tensor *slot_mapping, void *stream);
+
+/*
+ * pa_copy_blocks - copy whole physical blocks (all kv heads, all slots, both caches):
+ *   key_cache[dst] = key_cache[src], value_cache[dst] = value_cache[src]
+ * for each (src, dst) row of block_mapping [N, 2] int64.  This is the copy-on-write a block
+ * shared by several sequences ([P2] 4.1 parallel sampling, [P3] 2.2 shared prompt pages,
+ * [P4] 2.2.1 beam search) needs before one sharer writes into it.  Bit-exact.
+ * Preconditions: dst ids distinct, and no dst is also a src in the same call.  A pair with an
+ * id outside [0, num_blocks) sets PA_DEVERR_COPY_PAIR and is skipped.
+ */
+PA_API int pa_copy_blocks(const pa_tensor *key_cache, const pa_tensor *value_cache,
+                   const pa_tensor *block_mapping, void *stream);
+
+/*
+ * pa_decode - one decode step of paged attention.  For every sequence s and query head h,
+ * with g = h / (num_heads / num_kv_heads) and L = context_lens[s], the context is assembled
+ * through the block table ([P4] 2.2.2):
+ *   K_t = key_cache[block_tables[s, t / bs], g, t % bs, :]   (V alike),  0 <= t < L,
+ * and   out[s, h, :] = softmax_t(scale * q[s, h, :] . K_t) . V_t,
+ * accumulated in fp32.  L = 0 gives a zero row.  Block-table entries past ceil(L / bs) are
+ * never read.  The per-block loop printed in [P4] 2.2.2 states only the principle; this is the
+ * full-context softmax it stands for.
+ *
+ * Long contexts are split across warps; partial results are merged with the log-sum-exp rule.
+ * pa_decode uses a library-owned workspace per device, allocated (cudaMalloc, then zeroed on
+ * `stream`) the first time a call needs more than the current one holds: such a first call
+ * must not happen during stream capture, and concurrent pa_decode calls on different streams
+ * of one device must not overlap on the GPU (they share that workspace); use pa_decode_ex
+ * with a workspace per stream for that.
+ */
+PA_API int pa_decode(const pa_tensor *out, const pa_tensor *query, const pa_tensor *key_cache,
+              const pa_tensor *value_cache, const pa_tensor *block_tables,
+              const pa_tensor *context_lens, float scale, int32_t block_size,
+              int32_t num_kv_heads, void *stream);
+
+/*
+ * pa_decode_ex - pa_decode with caller-chosen parallel split and caller-owned workspace.
+ *   num_workers   number of warps that split the step's work, each taking an equal share of
+ *                 the (sequence, kv head, 16-row chunk) list; 0 = one full wave of the device.
+ *                 1 computes every sequence in a single warp (no merging at all).
+ *   flags         0 or PA_DECODE_SEPARATE_REDUCE.
+ *   workspace     device memory of at least pa_decode_workspace_bytes(...) bytes, 256-byte
+ *                 aligned, zero-filled before its first use (pa_workspace_init).  Every call
+ *                 that completes leaves it ready for the next call.  Calls sharing one
+ *                 workspace must not overlap on the GPU.
+ */
+PA_API int pa_decode_ex(const pa_tensor *out, const pa_tensor *query, const pa_tensor *key_cache,
+                 const pa_tensor *value_cache, const pa_tensor *block_tables,
+                 const pa_tensor *context_lens, float scale, int32_t block_size,
+                 int32_t num_kv_heads, int32_t num_workers, uint32_t flags, void *workspace,
+                 size_t workspace_bytes, void *stream);
+
+/*
+ * Bytes of workspace pa_decode_ex needs for num_seqs sequences of the given head counts and
+ * head_dim with num_workers warps (0 = the largest default of the current device).  Returns
+ * 0 on invalid arguments.
+ */
+PA_API size_t pa_decode_workspace_bytes(int64_t num_seqs, int32_t num_heads, int32_t num_kv_heads,
+                                 int32_t head_dim, int32_t num_workers);
+
+/* The number of warps pa_decode uses for a configuration on the current device (0 on error). */
+PA_API int32_t pa_decode_default_workers(int32_t dtype, int32_t head_dim, int32_t block_size,
+                                  int32_t group_size);
+
+/* Zero-fill a decode workspace on `stream` (before its first use, or after a
+ * PA_DEVERR_TIMEOUT). */
+PA_API int pa_workspace_init(void *workspace, size_t workspace_bytes, void *stream);
+
+/* Free the library-owned decode workspaces of every device (synchronises each device). */
+PA_API int pa_release_workspaces(void);
+
+/* Message for the last non-OK return of a pa_* call on this host thread ("" if none). */
+PA_API const char *pa_last_error(void);
+
+/*
+ * Read the current device's error word into *flags (a mask of PA_DEVERR_* bits), after
+ * waiting for `stream` to finish; clear it afterwards when `clear` is non-zero.  This call
+ * synchronises `stream`.
+ */
+PA_API int pa_get_device_error(void *stream, uint32_t *flags, int32_t clear);
+
+/* PA_VERSION of the library actually loaded. */
+PA_API int32_t pa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PA_H_ */

@@ -1,1 +1,202 @@
-"""B200-native paged KV-cache decode attention (placeholder; the binding lands with the library)."""
+"""B200-native paged KV-cache decode attention.
+
+Python binding of the C ABI declared in ``include/pa.h`` (library ``libpa.so`` in this
+directory, built by ``python -m paged_kv_cache_427_b200.build``).  The binding only marshals
+torch tensors into ``pa_tensor`` descriptors and passes the current CUDA stream: every step of
+the computation runs in the library's sm_100a kernels.  There is no CPU fallback: if the
+library is missing or fails to load, every call raises.
+
+Calls (same names as the C ABI):
+  pa_reshape_and_cache(key, value, key_cache, value_cache, slot_mapping)
+  pa_copy_blocks(key_cache, value_cache, block_mapping)
+  pa_decode(out, query, key_cache, value_cache, block_tables, context_lens, scale,
+            block_size, num_kv_heads)
+  pa_decode_ex(..., num_workers=0, flags=0, workspace=None)
+  pa_decode_workspace_bytes, pa_decode_default_workers, pa_workspace_init,
+  pa_release_workspaces, pa_last_error, pa_get_device_error, pa_version
+Seeded synthetic workloads live in ``paged_kv_cache_427_b200.workloads`` (no torch, no CUDA).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIBRARY = os.path.join(_HERE, "libpa.so")
+HEADER = os.path.join(os.path.dirname(_HERE), "include", "pa.h")
+
+PA_F32, PA_BF16, PA_F16, PA_I32, PA_I64 = 0, 1, 2, 3, 4
+PA_OK = 0
+PA_DECODE_SEPARATE_REDUCE = 0x1
+PA_DEVERR_BLOCK_ID = 0x1
+PA_DEVERR_CONTEXT_LEN = 0x2
+PA_DEVERR_SLOT = 0x4
+PA_DEVERR_COPY_PAIR = 0x8
+PA_DEVERR_TIMEOUT = 0x10
+STATUS_NAMES = {0: "PA_OK", -1: "PA_ERR_INVALID_ARG", -2: "PA_ERR_SHAPE", -3: "PA_ERR_DTYPE",
+                -4: "PA_ERR_UNSUPPORTED", -5: "PA_ERR_CUDA", -6: "PA_ERR_WORKSPACE",
+                -7: "PA_ERR_LAYOUT"}
+
+
+class PaTensor(ctypes.Structure):
+    _fields_ = [("data", ctypes.c_void_p), ("dtype", ctypes.c_int32), ("ndim", ctypes.c_int32),
+                ("shape", ctypes.c_int64 * 5), ("stride", ctypes.c_int64 * 5)]
+
+
+class PagedAttentionError(RuntimeError):
+    def __init__(self, call: str, status: int, message: str):
+        super().__init__(f"{call} failed: {STATUS_NAMES.get(status, status)}: {message}")
+        self.status = status
+
+
+_lib = None
+_P = ctypes.c_void_p
+_T = ctypes.POINTER(PaTensor)
+
+
+def load(path: str = LIBRARY) -> ctypes.CDLL:
+    """Load libpa.so (once).  Raises ImportError when it has not been built."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise ImportError(f"{path} is missing: build it with `python -m paged_kv_cache_427_b200.build`")
+    lib = ctypes.CDLL(path)
+    i32, u32, i64, sz, f32 = ctypes.c_int32, ctypes.c_uint32, ctypes.c_int64, ctypes.c_size_t, ctypes.c_float
+    lib.pa_reshape_and_cache.argtypes = [_T, _T, _T, _T, _T, _P]
+    lib.pa_copy_blocks.argtypes = [_T, _T, _T, _P]
+    lib.pa_decode.argtypes = [_T, _T, _T, _T, _T, _T, f32, i32, i32, _P]
+    lib.pa_decode_ex.argtypes = [_T, _T, _T, _T, _T, _T, f32, i32, i32, i32, u32, _P, sz, _P]
+    lib.pa_decode_workspace_bytes.argtypes = [i64, i32, i32, i32, i32]
+    lib.pa_decode_workspace_bytes.restype = sz
+    lib.pa_decode_default_workers.argtypes = [i32, i32, i32, i32]
+    lib.pa_decode_default_workers.restype = i32
+    lib.pa_workspace_init.argtypes = [_P, sz, _P]
+    lib.pa_release_workspaces.argtypes = []
+    lib.pa_last_error.argtypes = []
+    lib.pa_last_error.restype = ctypes.c_char_p
+    lib.pa_get_device_error.argtypes = [_P, ctypes.POINTER(u32), i32]
+    lib.pa_version.argtypes = []
+    lib.pa_version.restype = i32
+    for name in ("pa_reshape_and_cache", "pa_copy_blocks", "pa_decode", "pa_decode_ex",
+                 "pa_workspace_init", "pa_release_workspaces", "pa_get_device_error"):
+        getattr(lib, name).restype = ctypes.c_int
+    _lib = lib
+    return lib
+
+
+def _torch_dtype_code(t) -> int:
+    import torch
+
+    codes = {torch.float32: PA_F32, torch.bfloat16: PA_BF16, torch.float16: PA_F16,
+             torch.int32: PA_I32, torch.int64: PA_I64}
+    if t.dtype not in codes:
+        raise TypeError(f"unsupported tensor dtype {t.dtype}")
+    return codes[t.dtype]
+
+
+def describe(t) -> PaTensor:
+    """pa_tensor descriptor of a torch tensor (no copy; the tensor must outlive the call)."""
+    d = PaTensor()
+    d.data = t.data_ptr()
+    d.dtype = _torch_dtype_code(t)
+    d.ndim = t.dim()
+    if t.dim() > 5:
+        raise ValueError("at most 5 dimensions")
+    for i, (n, s) in enumerate(zip(t.shape, t.stride())):
+        d.shape[i] = n
+        d.stride[i] = s
+    return d
+
+
+def _stream(stream) -> int | None:
+    if stream is None:
+        import torch
+
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _check(call: str, rc: int):
+    if rc != PA_OK:
+        raise PagedAttentionError(call, rc, (load().pa_last_error() or b"").decode())
+
+
+def pa_reshape_and_cache(key, value, key_cache, value_cache, slot_mapping, stream=None):
+    """Store each new token's K/V rows at its slot (see include/pa.h)."""
+    lib = load()
+    d = [describe(x) for x in (key, value, key_cache, value_cache, slot_mapping)]
+    _check("pa_reshape_and_cache", lib.pa_reshape_and_cache(*[ctypes.byref(x) for x in d], _stream(stream)))
+
+
+def pa_copy_blocks(key_cache, value_cache, block_mapping, stream=None):
+    """Copy whole blocks dst <- src for each (src, dst) row of block_mapping."""
+    lib = load()
+    d = [describe(x) for x in (key_cache, value_cache, block_mapping)]
+    _check("pa_copy_blocks", lib.pa_copy_blocks(*[ctypes.byref(x) for x in d], _stream(stream)))
+
+
+def pa_decode(out, query, key_cache, value_cache, block_tables, context_lens, scale, block_size,
+              num_kv_heads, stream=None):
+    """One decode step of paged attention into `out` (library-owned workspace)."""
+    lib = load()
+    d = [describe(x) for x in (out, query, key_cache, value_cache, block_tables, context_lens)]
+    _check("pa_decode", lib.pa_decode(*[ctypes.byref(x) for x in d], float(scale), int(block_size),
+                                      int(num_kv_heads), _stream(stream)))
+
+
+def pa_decode_ex(out, query, key_cache, value_cache, block_tables, context_lens, scale,
+                 block_size, num_kv_heads, num_workers=0, flags=0, workspace=None, stream=None):
+    """pa_decode with an explicit warp count, flags and a caller-owned workspace (a CUDA uint8
+    tensor of at least pa_decode_workspace_bytes bytes, zeroed by pa_workspace_init once)."""
+    lib = load()
+    d = [describe(x) for x in (out, query, key_cache, value_cache, block_tables, context_lens)]
+    ws_ptr = workspace.data_ptr() if workspace is not None else None
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check("pa_decode_ex", lib.pa_decode_ex(*[ctypes.byref(x) for x in d], float(scale),
+                                            int(block_size), int(num_kv_heads), int(num_workers),
+                                            int(flags), ws_ptr, ws_bytes, _stream(stream)))
+
+
+def pa_decode_workspace_bytes(num_seqs, num_heads, num_kv_heads, head_dim, num_workers=0) -> int:
+    return int(load().pa_decode_workspace_bytes(num_seqs, num_heads, num_kv_heads, head_dim, num_workers))
+
+
+def pa_decode_default_workers(dtype: int, head_dim: int, block_size: int, group_size: int) -> int:
+    return int(load().pa_decode_default_workers(dtype, head_dim, block_size, group_size))
+
+
+def pa_workspace_init(workspace, stream=None):
+    lib = load()
+    _check("pa_workspace_init", lib.pa_workspace_init(
+        workspace.data_ptr(), workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
+def pa_release_workspaces():
+    _check("pa_release_workspaces", load().pa_release_workspaces())
+
+
+def pa_last_error() -> str:
+    return (load().pa_last_error() or b"").decode()
+
+
+def pa_get_device_error(clear: bool = False, stream=None) -> int:
+    """The device error word (PA_DEVERR_* bits); synchronises the stream."""
+    flags = ctypes.c_uint32(0)
+    _check("pa_get_device_error", load().pa_get_device_error(_stream(stream), ctypes.byref(flags), int(clear)))
+    return int(flags.value)
+
+
+def pa_version() -> int:
+    return int(load().pa_version())
+
+
+def header_functions(path: str = HEADER) -> list[str]:
+    """Names of the functions include/pa.h declares."""
+    import re
+
+    with open(path) as f:
+        text = f.read()
+    return sorted(set(re.findall(r"^\s*PA_API\s+(?:const\s+)?\w+\s*\*?\s*(pa_\w+)\s*\(", text, re.M)))

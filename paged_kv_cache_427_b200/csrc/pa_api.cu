@@ -1,0 +1,560 @@
+// pa_api.cu - the C ABI of the paged-attention library (declared in include/pa.h): argument
+// validation, kernel selection, workspaces and the per-device error word.
+//
+// No call reads device data on the host or synchronises (pa_get_device_error and
+// pa_release_workspaces excepted, as documented); launch sizes come from shapes only.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <mutex>
+#include <string>
+#include <vector>
+
+#include "pa.h"
+#include "pa_internal.h"
+
+namespace {
+
+// The error word of the device that loaded this module (one instance per device).
+__device__ unsigned int g_pa_error_word;
+
+thread_local std::string g_last_error;
+
+int fail(int code, const char *fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return code;
+}
+
+int cuda_fail(cudaError_t e, const char *what) {
+  return fail(PA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+typedef CUresult (*MemGetAddressRangeFn)(CUdeviceptr *, size_t *, CUdeviceptr);
+
+struct DeviceState {
+  bool ready = false;
+  int num_sms = 0;
+  unsigned int *err = nullptr;
+  void *ws = nullptr;  // library-owned decode workspace
+  size_t ws_bytes = 0;
+};
+
+std::mutex g_mu;
+std::vector<DeviceState> g_devices;
+MemGetAddressRangeFn g_mem_range = nullptr;
+bool g_mem_range_tried = false;
+
+// Per-device set-up on first use: SM count and the address of the error word.
+int device_state(DeviceState **out, int *dev_out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  std::lock_guard<std::mutex> lock(g_mu);
+  if ((int)g_devices.size() <= dev) g_devices.resize(dev + 1);
+  DeviceState &st = g_devices[dev];
+  if (!st.ready) {
+    e = cudaDeviceGetAttribute(&st.num_sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
+    e = cudaGetSymbolAddress(reinterpret_cast<void **>(&st.err), g_pa_error_word);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(error word)");
+    st.ready = true;
+  }
+  if (!g_mem_range_tried) {
+    g_mem_range_tried = true;
+    void *fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuMemGetAddressRange", &fn, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_mem_range = reinterpret_cast<MemGetAddressRangeFn>(fn);
+  }
+  *out = &st;
+  if (dev_out) *dev_out = dev;
+  return PA_OK;
+}
+
+size_t elt_size(int dtype) {
+  switch (dtype) {
+    case PA_F32:
+    case PA_I32:
+      return 4;
+    case PA_BF16:
+    case PA_F16:
+      return 2;
+    case PA_I64:
+      return 8;
+    default:
+      return 0;
+  }
+}
+
+const char *dtype_name(int d) {
+  switch (d) {
+    case PA_F32: return "fp32";
+    case PA_BF16: return "bf16";
+    case PA_F16: return "fp16";
+    case PA_I32: return "int32";
+    case PA_I64: return "int64";
+    default: return "unknown";
+  }
+}
+
+int check_tensor(const pa_tensor *t, const char *name, int ndim) {
+  if (!t) return fail(PA_ERR_INVALID_ARG, "%s: NULL descriptor", name);
+  if (t->ndim != ndim) return fail(PA_ERR_SHAPE, "%s: expected %d dims, got %d", name, ndim, t->ndim);
+  if (elt_size(t->dtype) == 0) return fail(PA_ERR_DTYPE, "%s: unknown element type %d", name, t->dtype);
+  for (int i = 0; i < ndim; ++i) {
+    if (t->shape[i] < 0) return fail(PA_ERR_SHAPE, "%s: negative size in dim %d", name, i);
+    if (t->stride[i] < 0) return fail(PA_ERR_LAYOUT, "%s: negative stride in dim %d", name, i);
+  }
+  return PA_OK;
+}
+
+int64_t numel(const pa_tensor *t) {
+  int64_t n = 1;
+  for (int i = 0; i < t->ndim; ++i) n *= t->shape[i];
+  return n;
+}
+
+// The bytes from data to one past the last element the tensor addresses.
+uint64_t extent_bytes(const pa_tensor *t) {
+  if (numel(t) == 0) return 0;
+  uint64_t last = 0;
+  for (int i = 0; i < t->ndim; ++i) last += (uint64_t)(t->shape[i] - 1) * (uint64_t)t->stride[i];
+  return (last + 1) * elt_size(t->dtype);
+}
+
+// Every byte the tensor addresses lies in one allocation of the current device.
+int check_device_memory(const pa_tensor *t, const char *name, int dev) {
+  const uint64_t ext = extent_bytes(t);
+  if (ext == 0) return PA_OK;
+  if (!t->data) return fail(PA_ERR_INVALID_ARG, "%s: NULL data pointer", name);
+  cudaPointerAttributes attr;
+  cudaError_t e = cudaPointerGetAttributes(&attr, t->data);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return fail(PA_ERR_LAYOUT, "%s: not a CUDA pointer (%s)", name, cudaGetErrorString(e));
+  }
+  if (attr.type != cudaMemoryTypeDevice && attr.type != cudaMemoryTypeManaged)
+    return fail(PA_ERR_LAYOUT, "%s: not device memory", name);
+  if (attr.type == cudaMemoryTypeDevice && attr.device != dev)
+    return fail(PA_ERR_LAYOUT, "%s: lives on device %d, current device is %d", name, attr.device, dev);
+  if (g_mem_range) {
+    CUdeviceptr base = 0;
+    size_t size = 0;
+    // When the driver cannot name the allocation the pointer check above stands alone.
+    const uint64_t p = (uint64_t)(uintptr_t)t->data;
+    if (g_mem_range(&base, &size, (CUdeviceptr)(uintptr_t)t->data) == CUDA_SUCCESS &&
+        p + ext > (uint64_t)base + size)
+      return fail(PA_ERR_LAYOUT, "%s: addresses %llu bytes but its allocation ends after %llu", name,
+                  (unsigned long long)ext, (unsigned long long)((uint64_t)base + size - p));
+  }
+  return PA_OK;
+}
+
+bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
+
+// Strides of the dims [0, upto) multiplied by the element size are multiples of 16 bytes.
+bool strides16(const pa_tensor *t, int upto) {
+  const size_t e = elt_size(t->dtype);
+  for (int i = 0; i < upto; ++i)
+    if (((size_t)t->stride[i] * e) % 16 != 0) return false;
+  return true;
+}
+
+struct CacheShape {
+  int64_t num_blocks;
+  int num_kv_heads, block_size, head_dim, dtype;
+};
+
+int check_caches(const pa_tensor *kc, const pa_tensor *vc, CacheShape *cs) {
+  int rc;
+  if ((rc = check_tensor(kc, "key_cache", 4)) || (rc = check_tensor(vc, "value_cache", 4))) return rc;
+  for (int i = 0; i < 4; ++i)
+    if (kc->shape[i] != vc->shape[i] || kc->stride[i] != vc->stride[i])
+      return fail(PA_ERR_SHAPE, "key_cache and value_cache differ in shape or strides (dim %d)", i);
+  if (kc->dtype != vc->dtype) return fail(PA_ERR_DTYPE, "key_cache and value_cache element types differ");
+  if (kc->dtype != PA_F32 && kc->dtype != PA_BF16 && kc->dtype != PA_F16)
+    return fail(PA_ERR_DTYPE, "caches must be fp32, bf16 or fp16 (got %s)", dtype_name(kc->dtype));
+  if (kc->stride[3] != 1 || kc->stride[2] != kc->shape[3])
+    return fail(PA_ERR_LAYOUT, "caches: each (block, kv head) tile [block_size, head_dim] must be contiguous");
+  if (!aligned16(kc->data) || !aligned16(vc->data) || !strides16(kc, 2))
+    return fail(PA_ERR_LAYOUT, "caches: data and block/head strides must be 16-byte aligned");
+  if (kc->shape[1] <= 0 || kc->shape[2] <= 0 || kc->shape[3] <= 0)
+    return fail(PA_ERR_SHAPE, "caches: num_kv_heads, block_size and head_dim must be positive");
+  if (kc->shape[1] > 0x7fffffff || kc->shape[2] > 0x7fffffff || kc->shape[3] > 0x7fffffff)
+    return fail(PA_ERR_SHAPE, "caches: dimension too large");
+  cs->num_blocks = kc->shape[0];
+  cs->num_kv_heads = (int)kc->shape[1];
+  cs->block_size = (int)kc->shape[2];
+  cs->head_dim = (int)kc->shape[3];
+  cs->dtype = kc->dtype;
+  return PA_OK;
+}
+
+bool get_kernel(int dtype, int head_dim, int block_size, int group, pa::DecodeKernel *k) {
+  switch (dtype) {
+    case PA_F32: return pa::decode_kernel_f32(head_dim, block_size, group, k);
+    case PA_BF16: return pa::decode_kernel_bf16(head_dim, block_size, group, k);
+    case PA_F16: return pa::decode_kernel_f16(head_dim, block_size, group, k);
+    default: return false;
+  }
+}
+
+// Warps of one full wave of the device for a kernel (CTAs per SM x SMs x warps per CTA).
+int default_workers(const pa::DecodeKernel &k, int num_sms) {
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k.kernel, k.warps_per_cta * 32,
+                                                    k.smem_bytes) != cudaSuccess ||
+      per_sm < 1) {
+    cudaGetLastError();
+    per_sm = 1;
+  }
+  return per_sm * num_sms * k.warps_per_cta;
+}
+
+// Workspace layout: counters [S*Hkv] u32 | pair_meta [S*Hkv] int2 | part_ml [(S*Hkv+W)*G*2] f32
+//                   | part_o [(S*Hkv+W)*G*D] f32, each region 256-byte aligned.
+struct WsLayout {
+  size_t counters, pair_meta, part_ml, part_o, total;
+};
+
+size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+WsLayout ws_layout(int64_t S, int Hq, int Hkv, int D, int W) {
+  WsLayout L;
+  const size_t pairs = (size_t)S * (size_t)Hkv;
+  const size_t segs = pairs + (size_t)W;
+  const size_t G = (size_t)(Hq / Hkv);
+  L.counters = 0;
+  L.pair_meta = align256(pairs * 4);
+  L.part_ml = L.pair_meta + align256(pairs * 8);
+  L.part_o = L.part_ml + align256(segs * G * 2 * 4);
+  L.total = L.part_o + align256(segs * G * (size_t)D * 4);
+  return L;
+}
+
+int decode_impl(const pa_tensor *out, const pa_tensor *query, const pa_tensor *key_cache,
+                const pa_tensor *value_cache, const pa_tensor *block_tables,
+                const pa_tensor *context_lens, float scale, int32_t block_size,
+                int32_t num_kv_heads, int32_t num_workers, uint32_t flags, void *workspace,
+                size_t workspace_bytes, bool library_workspace, void *stream) {
+  int rc;
+  CacheShape cs;
+  if ((rc = check_caches(key_cache, value_cache, &cs))) return rc;
+  if ((rc = check_tensor(query, "query", 3)) || (rc = check_tensor(out, "out", 3)) ||
+      (rc = check_tensor(block_tables, "block_tables", 2)) ||
+      (rc = check_tensor(context_lens, "context_lens", 1)))
+    return rc;
+  if (flags & ~PA_DECODE_SEPARATE_REDUCE) return fail(PA_ERR_INVALID_ARG, "unknown flags 0x%x", flags);
+  if (num_workers < 0) return fail(PA_ERR_INVALID_ARG, "num_workers must be >= 0");
+  if (block_size != cs.block_size)
+    return fail(PA_ERR_SHAPE, "block_size %d does not match the cache's %d", block_size, cs.block_size);
+  if (num_kv_heads != cs.num_kv_heads)
+    return fail(PA_ERR_SHAPE, "num_kv_heads %d does not match the cache's %d", num_kv_heads, cs.num_kv_heads);
+  const int64_t S = query->shape[0];
+  const int64_t Hq = query->shape[1];
+  const int D = cs.head_dim;
+  if (query->shape[2] != D) return fail(PA_ERR_SHAPE, "query head_dim %lld != cache head_dim %d", (long long)query->shape[2], D);
+  if (out->shape[0] != S || out->shape[1] != Hq || out->shape[2] != D)
+    return fail(PA_ERR_SHAPE, "out must be [num_seqs, num_heads, head_dim] like query");
+  if (block_tables->shape[0] != S || context_lens->shape[0] != S)
+    return fail(PA_ERR_SHAPE, "block_tables and context_lens need one row per sequence");
+  if (query->dtype != cs.dtype) return fail(PA_ERR_DTYPE, "query must have the caches' element type");
+  if (out->dtype != PA_F32 && out->dtype != cs.dtype)
+    return fail(PA_ERR_DTYPE, "out must be fp32 or the caches' element type");
+  if (block_tables->dtype != PA_I32 || context_lens->dtype != PA_I32)
+    return fail(PA_ERR_DTYPE, "block_tables and context_lens must be int32");
+  if (Hq <= 0 && S > 0) return fail(PA_ERR_SHAPE, "num_heads must be positive");
+  if (Hq % num_kv_heads != 0) return fail(PA_ERR_SHAPE, "num_heads %lld is not a multiple of num_kv_heads %d", (long long)Hq, num_kv_heads);
+  const int G = (int)(Hq / num_kv_heads);
+  if (D != 64 && D != 128) return fail(PA_ERR_UNSUPPORTED, "head_dim %d (built: 64, 128)", D);
+  if (block_size != 8 && block_size != 16 && block_size != 32)
+    return fail(PA_ERR_UNSUPPORTED, "block_size %d (built: 8, 16, 32)", block_size);
+  if (G != 1 && G != 2 && G != 4 && G != 8)
+    return fail(PA_ERR_UNSUPPORTED, "query heads per kv head %d (built: 1, 2, 4, 8)", G);
+  if (query->stride[2] != 1 || out->stride[2] != 1)
+    return fail(PA_ERR_LAYOUT, "query and out need a contiguous head_dim");
+  if (!aligned16(query->data) || !strides16(query, 2) || !aligned16(out->data) || !strides16(out, 2))
+    return fail(PA_ERR_LAYOUT, "query/out: data and sequence/head strides must be 16-byte aligned");
+  if (block_tables->stride[1] != 1 && block_tables->shape[1] > 1)
+    return fail(PA_ERR_LAYOUT, "block_tables rows must be contiguous");
+  if (context_lens->stride[0] != 1 && S > 1) return fail(PA_ERR_LAYOUT, "context_lens must be contiguous");
+  if (S > 0x7fffffff || block_tables->shape[1] * block_size > 0x7fffffff)
+    return fail(PA_ERR_SHAPE, "too many sequences or too long a block table");
+  if (!std::isfinite(scale)) return fail(PA_ERR_INVALID_ARG, "scale must be finite");
+  if (S == 0) return PA_OK;
+  DeviceState *ds;
+  int dev;
+  if ((rc = device_state(&ds, &dev))) return rc;
+  if ((rc = check_device_memory(key_cache, "key_cache", dev)) ||
+      (rc = check_device_memory(value_cache, "value_cache", dev)) ||
+      (rc = check_device_memory(query, "query", dev)) || (rc = check_device_memory(out, "out", dev)) ||
+      (rc = check_device_memory(block_tables, "block_tables", dev)) ||
+      (rc = check_device_memory(context_lens, "context_lens", dev)))
+    return rc;
+
+  pa::DecodeKernel k;
+  if (!get_kernel(cs.dtype, D, block_size, G, &k))
+    return fail(PA_ERR_CUDA, "could not prepare the decode kernel: %s", cudaGetErrorString(cudaGetLastError()));
+  const int W = num_workers > 0 ? num_workers : default_workers(k, ds->num_sms);
+  // worker_of() multiplies a chunk index by W in 64 bits
+  const double chunks = (double)S * num_kv_heads * ((double)block_tables->shape[1] * block_size / k.chunk_tokens + 1);
+  if (chunks * (double)W > 4.0e18) return fail(PA_ERR_SHAPE, "step too large for the work split");
+  const WsLayout L = ws_layout(S, (int)Hq, num_kv_heads, D, W);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (library_workspace) {
+    std::lock_guard<std::mutex> lock(g_mu);
+    if (ds->ws_bytes < L.total) {
+      cudaError_t e;
+      if (ds->ws) {
+        e = cudaDeviceSynchronize();
+        if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceSynchronize (workspace growth)");
+        cudaFree(ds->ws);
+        ds->ws = nullptr;
+        ds->ws_bytes = 0;
+      }
+      const size_t want = L.total + L.total / 4;
+      e = cudaMalloc(&ds->ws, want);
+      if (e != cudaSuccess) return cuda_fail(e, "cudaMalloc(decode workspace)");
+      e = cudaMemsetAsync(ds->ws, 0, want, st);
+      if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(decode workspace)");
+      ds->ws_bytes = want;
+    }
+    workspace = ds->ws;
+    workspace_bytes = ds->ws_bytes;
+  } else {
+    if (!workspace || workspace_bytes < L.total)
+      return fail(PA_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", L.total, workspace_bytes);
+    if (((uintptr_t)workspace & 255u) != 0) return fail(PA_ERR_WORKSPACE, "workspace must be 256-byte aligned");
+  }
+
+  pa::DecodeArgs a;
+  a.out = out->data;
+  a.out_dtype = out->dtype;
+  a.out_s = out->stride[0];
+  a.out_h = out->stride[1];
+  a.query = query->data;
+  a.q_s = query->stride[0];
+  a.q_h = query->stride[1];
+  a.q_heads_contiguous = (query->stride[1] == D) ? 1 : 0;
+  a.key_cache = key_cache->data;
+  a.value_cache = value_cache->data;
+  a.kv_blk = key_cache->stride[0];
+  a.kv_head = key_cache->stride[1];
+  a.block_tables = static_cast<const int32_t *>(block_tables->data);
+  a.bt_s = block_tables->stride[0];
+  a.context_lens = static_cast<const int32_t *>(context_lens->data);
+  a.num_seqs = (int)S;
+  a.num_kv_heads = num_kv_heads;
+  a.max_blocks = (int)block_tables->shape[1];
+  a.num_blocks = cs.num_blocks;
+  a.scale_log2 = (float)((double)scale * 1.4426950408889634);
+  a.num_workers = W;
+  char *ws = static_cast<char *>(workspace);
+  a.counters = reinterpret_cast<unsigned int *>(ws + L.counters);
+  a.pair_meta = reinterpret_cast<int2 *>(ws + L.pair_meta);
+  a.part_ml = reinterpret_cast<float *>(ws + L.part_ml);
+  a.part_o = reinterpret_cast<float *>(ws + L.part_o);
+  a.err = ds->err;
+  a.separate_reduce = (flags & PA_DECODE_SEPARATE_REDUCE) ? 1 : 0;
+  const int ctas = (W + k.warps_per_cta - 1) / k.warps_per_cta;
+  cudaError_t e = k.launch(a, ctas, st);
+  if (e != cudaSuccess) return cuda_fail(e, "decode launch");
+  if (a.separate_reduce) {
+    e = k.launch_reduce(a, st);
+    if (e != cudaSuccess) return cuda_fail(e, "merge launch");
+  }
+  return PA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int pa_reshape_and_cache(const pa_tensor *key, const pa_tensor *value, const pa_tensor *key_cache,
+                         const pa_tensor *value_cache, const pa_tensor *slot_mapping, void *stream) {
+  int rc;
+  CacheShape cs;
+  if ((rc = check_caches(key_cache, value_cache, &cs))) return rc;
+  if ((rc = check_tensor(key, "key", 3)) || (rc = check_tensor(value, "value", 3)) ||
+      (rc = check_tensor(slot_mapping, "slot_mapping", 1)))
+    return rc;
+  const int64_t T = key->shape[0];
+  for (int i = 0; i < 3; ++i)
+    if (value->shape[i] != key->shape[i]) return fail(PA_ERR_SHAPE, "key and value shapes differ");
+  if (key->shape[1] != cs.num_kv_heads || key->shape[2] != cs.head_dim)
+    return fail(PA_ERR_SHAPE, "key/value must be [num_tokens, num_kv_heads, head_dim] of the cache");
+  if (slot_mapping->shape[0] != T) return fail(PA_ERR_SHAPE, "slot_mapping needs one slot per token");
+  if (key->dtype != cs.dtype || value->dtype != cs.dtype)
+    return fail(PA_ERR_DTYPE, "key/value must have the caches' element type");
+  if (slot_mapping->dtype != PA_I64) return fail(PA_ERR_DTYPE, "slot_mapping must be int64");
+  if (key->stride[2] != 1 || value->stride[2] != 1 || (slot_mapping->stride[0] != 1 && T > 1))
+    return fail(PA_ERR_LAYOUT, "key/value need a contiguous head_dim and slot_mapping unit stride");
+  if (!aligned16(key->data) || !aligned16(value->data) || !strides16(key, 2) || !strides16(value, 2))
+    return fail(PA_ERR_LAYOUT, "key/value: data and token/head strides must be 16-byte aligned");
+  if (T == 0) return PA_OK;
+  DeviceState *ds;
+  int dev;
+  if ((rc = device_state(&ds, &dev))) return rc;
+  if ((rc = check_device_memory(key_cache, "key_cache", dev)) ||
+      (rc = check_device_memory(value_cache, "value_cache", dev)) ||
+      (rc = check_device_memory(key, "key", dev)) || (rc = check_device_memory(value, "value", dev)) ||
+      (rc = check_device_memory(slot_mapping, "slot_mapping", dev)))
+    return rc;
+  const size_t e = elt_size(cs.dtype);
+  pa::CacheWriteArgs a;
+  a.key = static_cast<const char *>(key->data);
+  a.value = static_cast<const char *>(value->data);
+  a.k_tok = key->stride[0] * (int64_t)e;
+  a.k_head = key->stride[1] * (int64_t)e;
+  a.v_tok = value->stride[0] * (int64_t)e;
+  a.v_head = value->stride[1] * (int64_t)e;
+  a.key_cache = static_cast<char *>(key_cache->data);
+  a.value_cache = static_cast<char *>(value_cache->data);
+  a.c_blk = key_cache->stride[0] * (int64_t)e;
+  a.c_head = key_cache->stride[1] * (int64_t)e;
+  a.row_bytes = (int)(cs.head_dim * e);
+  a.slots = static_cast<const int64_t *>(slot_mapping->data);
+  a.num_tokens = T;
+  a.num_kv_heads = cs.num_kv_heads;
+  a.block_size = cs.block_size;
+  a.num_slots = cs.num_blocks * cs.block_size;
+  a.err = ds->err;
+  if (a.row_bytes % 16 != 0) return fail(PA_ERR_UNSUPPORTED, "head_dim * element size must be a multiple of 16 bytes");
+  cudaError_t err = pa::launch_reshape_and_cache(a, ds->num_sms, static_cast<cudaStream_t>(stream));
+  return err == cudaSuccess ? PA_OK : cuda_fail(err, "reshape_and_cache launch");
+}
+
+int pa_copy_blocks(const pa_tensor *key_cache, const pa_tensor *value_cache,
+                   const pa_tensor *block_mapping, void *stream) {
+  int rc;
+  CacheShape cs;
+  if ((rc = check_caches(key_cache, value_cache, &cs))) return rc;
+  if ((rc = check_tensor(block_mapping, "block_mapping", 2))) return rc;
+  if (block_mapping->dtype != PA_I64) return fail(PA_ERR_DTYPE, "block_mapping must be int64");
+  if (block_mapping->shape[1] != 2) return fail(PA_ERR_SHAPE, "block_mapping must be [num_pairs, 2]");
+  const int64_t N = block_mapping->shape[0];
+  if (N > 1 && block_mapping->stride[0] != 2) return fail(PA_ERR_LAYOUT, "block_mapping must be contiguous");
+  if (block_mapping->stride[1] != 1) return fail(PA_ERR_LAYOUT, "block_mapping must be contiguous");
+  if (N == 0) return PA_OK;
+  DeviceState *ds;
+  int dev;
+  if ((rc = device_state(&ds, &dev))) return rc;
+  if ((rc = check_device_memory(key_cache, "key_cache", dev)) ||
+      (rc = check_device_memory(value_cache, "value_cache", dev)) ||
+      (rc = check_device_memory(block_mapping, "block_mapping", dev)))
+    return rc;
+  const size_t e = elt_size(cs.dtype);
+  pa::CopyBlocksArgs a;
+  a.key_cache = static_cast<char *>(key_cache->data);
+  a.value_cache = static_cast<char *>(value_cache->data);
+  a.c_blk = key_cache->stride[0] * (int64_t)e;
+  a.c_head = key_cache->stride[1] * (int64_t)e;
+  a.tile_bytes = (int)(cs.block_size * cs.head_dim * e);
+  a.pairs = static_cast<const int64_t *>(block_mapping->data);
+  a.num_pairs = N;
+  a.num_kv_heads = cs.num_kv_heads;
+  a.num_blocks = cs.num_blocks;
+  a.err = ds->err;
+  if (a.tile_bytes % 16 != 0) return fail(PA_ERR_UNSUPPORTED, "block tile must be a multiple of 16 bytes");
+  cudaError_t err = pa::launch_copy_blocks(a, ds->num_sms, static_cast<cudaStream_t>(stream));
+  return err == cudaSuccess ? PA_OK : cuda_fail(err, "copy_blocks launch");
+}
+
+int pa_decode(const pa_tensor *out, const pa_tensor *query, const pa_tensor *key_cache,
+              const pa_tensor *value_cache, const pa_tensor *block_tables,
+              const pa_tensor *context_lens, float scale, int32_t block_size,
+              int32_t num_kv_heads, void *stream) {
+  return decode_impl(out, query, key_cache, value_cache, block_tables, context_lens, scale,
+                     block_size, num_kv_heads, 0, 0u, nullptr, 0, true, stream);
+}
+
+int pa_decode_ex(const pa_tensor *out, const pa_tensor *query, const pa_tensor *key_cache,
+                 const pa_tensor *value_cache, const pa_tensor *block_tables,
+                 const pa_tensor *context_lens, float scale, int32_t block_size,
+                 int32_t num_kv_heads, int32_t num_workers, uint32_t flags, void *workspace,
+                 size_t workspace_bytes, void *stream) {
+  return decode_impl(out, query, key_cache, value_cache, block_tables, context_lens, scale,
+                     block_size, num_kv_heads, num_workers, flags, workspace, workspace_bytes,
+                     false, stream);
+}
+
+size_t pa_decode_workspace_bytes(int64_t num_seqs, int32_t num_heads, int32_t num_kv_heads,
+                                 int32_t head_dim, int32_t num_workers) {
+  if (num_seqs < 0 || num_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 || num_workers < 0 ||
+      num_heads % num_kv_heads != 0)
+    return 0;
+  int W = num_workers;
+  if (W == 0) {
+    DeviceState *ds;
+    if (device_state(&ds, nullptr) != PA_OK) return 0;
+    W = ds->num_sms * 16;  // at most 4 CTAs of 4 warps per SM for any built configuration
+  }
+  return ws_layout(num_seqs, num_heads, num_kv_heads, head_dim, W).total;
+}
+
+int32_t pa_decode_default_workers(int32_t dtype, int32_t head_dim, int32_t block_size,
+                                  int32_t group_size) {
+  DeviceState *ds;
+  if (device_state(&ds, nullptr) != PA_OK) return 0;
+  pa::DecodeKernel k;
+  if (!get_kernel(dtype, head_dim, block_size, group_size, &k)) return 0;
+  return default_workers(k, ds->num_sms);
+}
+
+int pa_workspace_init(void *workspace, size_t workspace_bytes, void *stream) {
+  if (!workspace && workspace_bytes) return fail(PA_ERR_INVALID_ARG, "NULL workspace");
+  if (!workspace_bytes) return PA_OK;
+  cudaError_t e = cudaMemsetAsync(workspace, 0, workspace_bytes, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? PA_OK : cuda_fail(e, "cudaMemsetAsync(workspace)");
+}
+
+int pa_release_workspaces(void) {
+  int cur = 0;
+  if (cudaGetDevice(&cur) != cudaSuccess) return fail(PA_ERR_CUDA, "cudaGetDevice failed");
+  std::lock_guard<std::mutex> lock(g_mu);
+  for (size_t d = 0; d < g_devices.size(); ++d) {
+    if (!g_devices[d].ws) continue;
+    cudaSetDevice((int)d);
+    cudaDeviceSynchronize();
+    cudaFree(g_devices[d].ws);
+    g_devices[d].ws = nullptr;
+    g_devices[d].ws_bytes = 0;
+  }
+  cudaSetDevice(cur);
+  return PA_OK;
+}
+
+const char *pa_last_error(void) { return g_last_error.c_str(); }
+
+int pa_get_device_error(void *stream, uint32_t *flags, int32_t clear) {
+  if (!flags) return fail(PA_ERR_INVALID_ARG, "flags is NULL");
+  DeviceState *ds;
+  int rc = device_state(&ds, nullptr);
+  if (rc) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  unsigned int host = 0;
+  cudaError_t e = cudaMemcpyAsync(&host, ds->err, sizeof(host), cudaMemcpyDeviceToHost, st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return cuda_fail(e, "reading the error word");
+  *flags = host;
+  if (clear) {
+    e = cudaMemsetAsync(ds->err, 0, sizeof(unsigned int), st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) return cuda_fail(e, "clearing the error word");
+  }
+  return PA_OK;
+}
+
+int32_t pa_version(void) { return PA_VERSION; }
+
+}  // extern "C"

@@ -1,0 +1,84 @@
+// pa_internal.h - host-side interface between the C ABI (pa_api.cu) and the kernel files.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace pa {
+
+// Everything a decode launch needs, already validated.  Strides are in elements.
+struct DecodeArgs {
+  void *out;
+  int out_dtype;
+  int64_t out_s, out_h;
+  const void *query;
+  int64_t q_s, q_h;
+  int q_heads_contiguous;  // query heads of one group form one contiguous run
+  const void *key_cache;
+  const void *value_cache;
+  int64_t kv_blk, kv_head;
+  const int32_t *block_tables;
+  int64_t bt_s;
+  const int32_t *context_lens;
+  int num_seqs;
+  int num_kv_heads;
+  int max_blocks;
+  int64_t num_blocks;
+  float scale_log2;  // scale * log2(e): logits are kept in base-2 units
+  int num_workers;   // warps sharing the work
+  // workspace (see pa_api.cu for the layout)
+  unsigned int *counters;
+  int2 *pair_meta;
+  float *part_ml;
+  float *part_o;
+  unsigned int *err;
+  int separate_reduce;
+};
+
+struct DecodeKernel {
+  cudaError_t (*launch)(const DecodeArgs &, int num_ctas, cudaStream_t);
+  cudaError_t (*launch_reduce)(const DecodeArgs &, cudaStream_t);
+  const void *kernel;  // for occupancy queries
+  int warps_per_cta;
+  int smem_bytes;
+  int chunk_tokens;
+};
+
+// Kernel tables, one per element type.  Return false when the (head_dim, block_size, group)
+// combination is not built.
+bool decode_kernel_f32(int head_dim, int block_size, int group, DecodeKernel *k);
+bool decode_kernel_bf16(int head_dim, int block_size, int group, DecodeKernel *k);
+bool decode_kernel_f16(int head_dim, int block_size, int group, DecodeKernel *k);
+
+struct CacheWriteArgs {
+  const char *key;
+  const char *value;
+  int64_t k_tok, k_head, v_tok, v_head;  // bytes
+  char *key_cache;
+  char *value_cache;
+  int64_t c_blk, c_head;  // bytes
+  int row_bytes;
+  const int64_t *slots;
+  int64_t num_tokens;
+  int num_kv_heads;
+  int block_size;
+  int64_t num_slots;
+  unsigned int *err;
+};
+
+struct CopyBlocksArgs {
+  char *key_cache;
+  char *value_cache;
+  int64_t c_blk, c_head;  // bytes
+  int tile_bytes;         // block_size * row bytes: one (block, kv head) tile
+  const int64_t *pairs;
+  int64_t num_pairs;
+  int num_kv_heads;
+  int64_t num_blocks;
+  unsigned int *err;
+};
+
+cudaError_t launch_reshape_and_cache(const CacheWriteArgs &a, int num_sms, cudaStream_t st);
+cudaError_t launch_copy_blocks(const CopyBlocksArgs &a, int num_sms, cudaStream_t st);
+
+}  // namespace pa

@@ -1,0 +1,148 @@
+"""The C-ABI library builds, loads and exports what include/pa.h declares; host-side argument
+checks run before any CUDA call, so they are exercised here without a GPU."""
+import ctypes
+import re
+import subprocess
+
+import pytest
+
+import paged_kv_cache_427_b200 as pa
+from paged_kv_cache_427_b200 import build as pa_build
+
+
+@pytest.fixture(scope="module")
+def lib():
+    pa_build.build()
+    return pa.load()
+
+
+def test_every_declared_function_is_exported(lib):
+    declared = pa.header_functions()
+    assert {"pa_reshape_and_cache", "pa_copy_blocks", "pa_decode", "pa_decode_ex"} <= set(declared)
+    out = subprocess.run(["nm", "-D", "--defined-only", pa.LIBRARY], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(re.findall(r"\sT\s(pa_\w+)$", out, re.M))
+    missing = [f for f in declared if f not in exported]
+    assert not missing, f"declared but not exported: {missing}"
+    for f in declared:
+        assert hasattr(lib, f)
+    # nothing but the C ABI leaks out of the library
+    assert not [s for s in re.findall(r"\sT\s(\S+)$", out, re.M) if not s.startswith("pa_")
+                and not s.startswith("_init") and not s.startswith("_fini")]
+
+
+def test_version_matches_header(lib):
+    with open(pa.HEADER) as f:
+        v = int(re.search(r"#define PA_VERSION (\d+)", f.read()).group(1))
+    assert pa.pa_version() == v
+
+
+def test_workspace_bytes_layout(lib):
+    # counters [S*Hkv] u32 | pair_meta [S*Hkv] int2 | part_ml [(S*Hkv+W)*G*2] f32 |
+    # part_o [(S*Hkv+W)*G*D] f32, each region rounded up to 256 bytes
+    def up(x):
+        return (x + 255) // 256 * 256
+
+    S, Hq, Hkv, D, W = 64, 32, 8, 128, 1184
+    pairs, segs, G = S * Hkv, S * Hkv + W, Hq // Hkv
+    expect = up(pairs * 4) + up(pairs * 8) + up(segs * G * 2 * 4) + up(segs * G * D * 4)
+    assert pa.pa_decode_workspace_bytes(S, Hq, Hkv, D, W) == expect
+    assert pa.pa_decode_workspace_bytes(S, 30, 8, D, W) == 0  # heads not a multiple
+    assert pa.pa_decode_workspace_bytes(-1, Hq, Hkv, D, W) == 0
+
+
+def _t(shape, dtype, data=0x10000, stride=None):
+    d = pa.PaTensor()
+    d.data = data
+    d.dtype = dtype
+    d.ndim = len(shape)
+    if stride is None:
+        stride, acc = [], 1
+        for n in reversed(shape):
+            stride.insert(0, acc)
+            acc *= n
+    for i, (n, s) in enumerate(zip(shape, stride)):
+        d.shape[i] = n
+        d.stride[i] = s
+    return d
+
+
+def _decode_args(S=4, Hq=8, Hkv=2, D=128, bs=16, NB=32, MB=4, dt=pa.PA_BF16, out_dt=None,
+                 q_data=0x10000):
+    return dict(out=_t([S, Hq, D], out_dt if out_dt is not None else dt),
+                query=_t([S, Hq, D], dt, data=q_data),
+                kc=_t([NB, Hkv, bs, D], dt), vc=_t([NB, Hkv, bs, D], dt),
+                bt=_t([S, MB], pa.PA_I32), cl=_t([S], pa.PA_I32))
+
+
+def _decode(lib, a, bs=16, hkv=2, flags=0, workers=0, scale=0.1):
+    r = ctypes.byref
+    return lib.pa_decode_ex(r(a["out"]), r(a["query"]), r(a["kc"]), r(a["vc"]), r(a["bt"]),
+                            r(a["cl"]), scale, bs, hkv, workers, flags, None, 0, None)
+
+
+@pytest.mark.parametrize("case,expect", [
+    (dict(D=96), -4),                        # head_dim not built
+    (dict(bs=64), -4),                       # block_size not built
+    (dict(Hq=24, Hkv=2), -4),                # group of 12 not built
+    (dict(Hq=7, Hkv=2), -2),                 # heads not a multiple of kv heads
+    (dict(out_dt=pa.PA_F16), -3),            # out neither fp32 nor the cache type
+    (dict(q_data=0x10008), -7),              # query misaligned
+])
+def test_decode_rejects_bad_arguments_before_cuda(lib, case, expect):
+    kw = dict(case)
+    a = _decode_args(**kw)
+    assert _decode(lib, a, bs=kw.get("bs", 16), hkv=kw.get("Hkv", 2)) == expect
+    assert pa.pa_last_error()
+
+
+def test_decode_rejects_mismatches(lib):
+    a = _decode_args()
+    assert _decode(lib, a, bs=8) == -2          # block_size disagrees with the cache
+    assert _decode(lib, a, hkv=4) == -2         # num_kv_heads disagrees with the cache
+    assert _decode(lib, a, flags=0x80) == -1    # unknown flag
+    assert _decode(lib, a, workers=-1) == -1
+    assert _decode(lib, a, scale=float("nan")) == -1
+    b = _decode_args()
+    b["vc"] = _t([32, 2, 16, 128], pa.PA_F16)
+    assert _decode(lib, b) == -3                 # caches of different types
+    c = _decode_args()
+    c["bt"] = _t([4, 4], pa.PA_I64)
+    assert _decode(lib, c) == -3                 # block table must be int32
+    d = _decode_args()
+    d["kc"] = _t([32, 2, 16, 128], pa.PA_BF16, stride=[4096, 2048, 256, 1])
+    d["vc"] = _t([32, 2, 16, 128], pa.PA_BF16, stride=[4096, 2048, 256, 1])
+    assert _decode(lib, d) == -7                 # tile rows not contiguous
+    e = _decode_args()
+    e["cl"] = _t([3], pa.PA_I32)
+    assert _decode(lib, e) == -2                 # one context length per sequence
+
+
+def test_zero_sequences_is_a_no_op(lib):
+    a = _decode_args(S=0)
+    assert _decode(lib, a) == 0
+
+
+def test_reshape_and_cache_rejects_bad_arguments(lib):
+    r = ctypes.byref
+    kc = _t([32, 2, 16, 128], pa.PA_BF16)
+    vc = _t([32, 2, 16, 128], pa.PA_BF16)
+    key = _t([5, 2, 128], pa.PA_BF16)
+    val = _t([5, 2, 128], pa.PA_BF16)
+    slots32 = _t([5], pa.PA_I32)
+    assert lib.pa_reshape_and_cache(r(key), r(val), r(kc), r(vc), r(slots32), None) == -3
+    slots = _t([4], pa.PA_I64)
+    assert lib.pa_reshape_and_cache(r(key), r(val), r(kc), r(vc), r(slots), None) == -2
+    key3 = _t([5, 3, 128], pa.PA_BF16)
+    assert lib.pa_reshape_and_cache(r(key3), r(key3), r(kc), r(vc), r(_t([5], pa.PA_I64)), None) == -2
+    empty = _t([0, 2, 128], pa.PA_BF16)
+    assert lib.pa_reshape_and_cache(r(empty), r(empty), r(kc), r(vc), r(_t([0], pa.PA_I64)), None) == 0
+
+
+def test_copy_blocks_rejects_bad_arguments(lib):
+    r = ctypes.byref
+    kc = _t([32, 2, 16, 128], pa.PA_BF16)
+    vc = _t([32, 2, 16, 128], pa.PA_BF16)
+    assert lib.pa_copy_blocks(r(kc), r(vc), r(_t([3, 3], pa.PA_I64)), None) == -2
+    assert lib.pa_copy_blocks(r(kc), r(vc), r(_t([3, 2], pa.PA_I32)), None) == -3
+    assert lib.pa_copy_blocks(r(kc), r(vc), r(_t([0, 2], pa.PA_I64)), None) == 0
