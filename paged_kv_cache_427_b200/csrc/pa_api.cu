@@ -9,6 +9,7 @@
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
+#include <cstdlib>
 #include <mutex>
 #include <string>
 #include <vector>
@@ -38,6 +39,26 @@ int cuda_fail(cudaError_t e, const char *what) {
 }
 
 typedef CUresult (*MemGetAddressRangeFn)(CUdeviceptr *, size_t *, CUdeviceptr);
+
+// Test hooks, read once per process: PA_TEST_WAIT_LIMIT_CYCLES shortens every wait on a copy,
+// PA_TEST_STALL_COPIES=1 makes each decode warp's first stage wait for 16 bytes that no copy
+// delivers, so that the wait runs out, the kernel records PA_DEVERR_TIMEOUT and returns.
+struct TestHooks {
+  long long wait_cycles = 2000000000ll;  // about one second at the 1965 MHz maximum SM clock
+  int stall = 0;
+  TestHooks() {
+    if (const char *v = std::getenv("PA_TEST_WAIT_LIMIT_CYCLES")) {
+      const long long x = std::atoll(v);
+      if (x > 0) wait_cycles = x;
+    }
+    if (const char *v = std::getenv("PA_TEST_STALL_COPIES")) stall = std::atoi(v) != 0;
+  }
+};
+
+const TestHooks &test_hooks() {
+  static TestHooks h;
+  return h;
+}
 
 struct DeviceState {
   bool ready = false;
@@ -366,6 +387,8 @@ int decode_impl(const pa_tensor *out, const pa_tensor *query, const pa_tensor *k
   a.part_o = reinterpret_cast<float *>(ws + L.part_o);
   a.err = ds->err;
   a.separate_reduce = (flags & PA_DECODE_SEPARATE_REDUCE) ? 1 : 0;
+  a.wait_cycles = test_hooks().wait_cycles;
+  a.test_stall = test_hooks().stall;
   const int ctas = (W + k.warps_per_cta - 1) / k.warps_per_cta;
   cudaError_t e = k.launch(a, ctas, st);
   if (e != cudaSuccess) return cuda_fail(e, "decode launch");

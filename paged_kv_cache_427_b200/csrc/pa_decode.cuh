@@ -333,8 +333,9 @@ __global__ void __launch_bounds__(128, 1) paged_decode_kernel(const DecodeArgs a
       int ncopy = 0;
 #pragma unroll
       for (int k = 0; k < Tr::kCopies; ++k) ncopy += (c_i * CH + k * Tr::kCopyRows < c_len);
-      const uint32_t bytes =
-          2u * ncopy * Tr::kCopyBytes + ((flags & kFirst) ? (uint32_t)Tr::kQBytes : 0u);
+      const uint32_t bytes = 2u * ncopy * Tr::kCopyBytes +
+                             ((flags & kFirst) ? (uint32_t)Tr::kQBytes : 0u) +
+                             ((a.test_stall && issued == 0) ? 16u : 0u);
       fence_proxy_async_smem();
       mbar_arrive_expect_tx(bars + slot, bytes);
 #pragma unroll
@@ -408,11 +409,11 @@ __global__ void __launch_bounds__(128, 1) paged_decode_kernel(const DecodeArgs a
   for (long long c = 0; c < n; ++c) {
     const int slot = (int)(c % ST);
     const uint32_t parity = (uint32_t)((c / ST) & 1);
-    if (!mbar_wait_bounded(bars + slot, parity, kWaitLimitCycles)) {
+    if (!mbar_wait_bounded(bars + slot, parity, a.wait_cycles)) {
       // a copy never completed: record it, let the copies already issued land, and stop.
       if (lane == 0) set_error(a.err, PA_DEVERR_TIMEOUT);
       for (long long k = c; k < issued; ++k)
-        mbar_wait_bounded(bars + (int)(k % ST), (uint32_t)((k / ST) & 1), kWaitLimitCycles);
+        mbar_wait_bounded(bars + (int)(k % ST), (uint32_t)((k / ST) & 1), a.wait_cycles);
       return;
     }
     const ChunkMeta m = meta[slot];

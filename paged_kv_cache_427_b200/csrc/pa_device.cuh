@@ -169,7 +169,4 @@ __device__ __forceinline__ void set_error(unsigned int *err, unsigned int bits) 
   if (err) atomicOr(err, bits);
 }
 
-// About one second at the B200's 1965 MHz maximum SM clock.
-constexpr long long kWaitLimitCycles = 2000000000ll;
-
 }  // namespace pa

@@ -33,6 +33,8 @@ struct DecodeArgs {
   float *part_o;
   unsigned int *err;
   int separate_reduce;
+  long long wait_cycles;  // limit of every wait on a copy (about one second by default)
+  int test_stall;         // test hook: each warp's first stage expects 16 bytes nobody sends
 };
 
 struct DecodeKernel {

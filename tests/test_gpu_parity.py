@@ -11,7 +11,8 @@ import torch
 import paged_kv_cache_427_b200 as pa
 from paged_kv_cache_427_b200 import workloads as W
 from tests.gpu_helpers import (DeviceBatch, assert_bf16_output, assert_close,
-                               assert_no_device_error, oracle_step, require_gpu, to_host)
+                               assert_no_device_error, assert_rounded_from, oracle_step,
+                               require_gpu, to_host)
 
 pytestmark = pytest.mark.gpu
 
@@ -58,10 +59,11 @@ def test_llama_small_workers(llama_small, workers, flags):
     db = DeviceBatch(b)
     db.write()
     _check_caches(db, kc, vc, "bf16")
-    out = db.decode("f32", num_workers=workers, flags=flags)
-    assert_close(to_host(out, "f32"), ref, "bf16", f"W={workers} flags={flags}")
-    outb = db.decode("bf16", num_workers=workers, flags=flags)
-    assert_bf16_output(to_host(outb, "bf16"), ref, f"bf16 out W={workers}")
+    out = to_host(db.decode("f32", num_workers=workers, flags=flags), "f32")
+    assert_close(out, ref, "bf16", f"W={workers} flags={flags}")
+    outb = to_host(db.decode("bf16", num_workers=workers, flags=flags), "bf16")
+    assert_bf16_output(outb, ref, f"bf16 out W={workers}")
+    assert_rounded_from(outb, out, f"bf16 out W={workers}")
     assert_no_device_error()
 
 
