@@ -293,6 +293,17 @@ def run_ours(args, b: W.PagedBatch, config: dict, rank: int, world: int, local_r
     mapping = dev_t(b.block_mapping) if b.block_mapping is not None and len(b.block_mapping) else None
     out = torch.empty(q.shape, dtype=out_dtype, device=dev)
     stream = torch.cuda.current_stream()
+    ws = None
+    if args.decode_flags:
+        ws = torch.zeros(pa.pa_decode_workspace_bytes(b.num_seqs, b.num_heads, b.num_kv_heads,
+                                                      b.head_dim, 0), dtype=torch.uint8, device=dev)
+
+    def decode(qq, kc, vc, tt, ll):
+        if ws is None:
+            pa.pa_decode(out, qq, kc, vc, tt, ll, b.scale, b.block_size, b.num_kv_heads)
+        else:
+            pa.pa_decode_ex(out, qq, kc, vc, tt, ll, b.scale, b.block_size, b.num_kv_heads,
+                            flags=args.decode_flags, workspace=ws)
 
     def step(i, ev=None):
         kc, vc = pools[i % rot]
@@ -301,11 +312,11 @@ def run_ours(args, b: W.PagedBatch, config: dict, rank: int, world: int, local_r
         pa.pa_reshape_and_cache(key, value, kc, vc, slots)
         if ev is not None:
             ev[0].record(stream)
-        pa.pa_decode(out, q, kc, vc, tables, lens, b.scale, b.block_size, b.num_kv_heads)
+        decode(q, kc, vc, tables, lens)
         if ev is not None:
             ev[1].record(stream)
 
-    launches_per_step = 2 + (1 if mapping is not None else 0)
+    launches_per_step = 2 + (1 if mapping is not None else 0) + (1 if args.decode_flags & 1 else 0)
     gpu_uuid = None
     try:
         gpu_uuid = str(torch.cuda.get_device_properties(dev).uuid)
@@ -367,7 +378,7 @@ def run_ours(args, b: W.PagedBatch, config: dict, rank: int, world: int, local_r
         if mapping is not None:
             pa.pa_copy_blocks(kc, vc, mapping)
         pa.pa_reshape_and_cache(d_in["key"], d_in["value"], kc, vc, d_in["slots"])
-        pa.pa_decode(out, d_q, kc, vc, d_in["tables"], d_in["lens"], b.scale, b.block_size, b.num_kv_heads)
+        decode(d_q, kc, vc, d_in["tables"], d_in["lens"])
         h_out.copy_(out, non_blocking=True)
         stream.synchronize()
 
@@ -418,7 +429,10 @@ def run_ours(args, b: W.PagedBatch, config: dict, rank: int, world: int, local_r
         f"pct_of_{peak_src}_hbm": round(100 * value / world / peak, 2),
         "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 4), "traffic": recorded_traffic(config["workload"]),
-                     "kernel": "paged_decode_kernel", "peak_source": peak_src,
+                     "kernel": ("paged_decode_kernel (CUDA cores)"
+                                if (args.decode_flags & 2 or b.dtype == "f32")
+                                else "paged_decode_mma_kernel (mma.sync + TMA)"),
+                     "peak_source": peak_src,
                      "algorithmic_bytes_per_launch": dec_unique,
                      "mean_launch_us": round(dec_mean * 1e3, 3)},
         "e2e": {"value": round(world * step_bytes / (e2e_ms_step * 1e-3) / 1e9, 2), "unit": "GB/s",
@@ -442,6 +456,8 @@ def main():
     ap.add_argument("--workload", default="llama3_8b_decode",
                     help="llama3_8b_decode | short_chat_bs{8,16,32} | shared_prefix | long_mixed | tiny_fp32")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--decode-flags", type=int, default=0,
+                    help="pa_decode_ex flags (2 = CUDA-core kernel, 1 = separate merge kernel)")
     ap.add_argument("--rotations", type=int, default=0, help="copies of the KV pool (0 = enough to defeat L2)")
     ap.add_argument("--soak", type=float, default=1.0, help="seconds of untimed load for the clock sampler")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
@@ -463,6 +479,7 @@ def main():
               "seed": b.meta.get("seed"),
               "l2": "inputs larger than L2: steps rotate over copies of the KV pool",
               "pool_rotations": args.rotations or "auto",
+              "decode_flags": args.decode_flags,
               "parallelism": f"replicas x{world}" if world > 1 else "single GPU"}
 
     if args.impl == "reference":

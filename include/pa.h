@@ -109,6 +109,9 @@ typedef enum pa_status {
 /* Flags of pa_decode_ex. */
 #define PA_DECODE_SEPARATE_REDUCE 0x1u /* merge split contexts in a second kernel instead of
                                           in the last warp to finish each (sequence, kv head) */
+#define PA_DECODE_CUDA_CORES 0x2u      /* 16-bit caches: use the CUDA-core kernel instead of the
+                                          tensor-core (mma.sync + TMA) one; fp32 caches always
+                                          use the CUDA-core kernel */
 
 /*
  * pa_reshape_and_cache - store this step's new keys and values into their cache slots.

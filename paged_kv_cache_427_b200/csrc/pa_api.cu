@@ -39,6 +39,10 @@ int cuda_fail(cudaError_t e, const char *what) {
 }
 
 typedef CUresult (*MemGetAddressRangeFn)(CUdeviceptr *, size_t *, CUdeviceptr);
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
 // Test hooks, read once per process: PA_TEST_WAIT_LIMIT_CYCLES shortens every wait on a copy,
 // PA_TEST_STALL_COPIES=1 makes each decode warp's first stage wait for 16 bytes that no copy
@@ -71,6 +75,7 @@ struct DeviceState {
 std::mutex g_mu;
 std::vector<DeviceState> g_devices;
 MemGetAddressRangeFn g_mem_range = nullptr;
+EncodeTiledFn g_encode_tiled = nullptr;
 bool g_mem_range_tried = false;
 
 // Per-device set-up on first use: SM count and the address of the error word.
@@ -96,6 +101,11 @@ int device_state(DeviceState **out, int *dev_out) {
             cudaSuccess &&
         q == cudaDriverEntryPointSuccess)
       g_mem_range = reinterpret_cast<MemGetAddressRangeFn>(fn);
+    fn = nullptr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode_tiled = reinterpret_cast<EncodeTiledFn>(fn);
   }
   *out = &st;
   if (dev_out) *dev_out = dev;
@@ -221,13 +231,77 @@ int check_caches(const pa_tensor *kc, const pa_tensor *vc, CacheShape *cs) {
   return PA_OK;
 }
 
-bool get_kernel(int dtype, int head_dim, int block_size, int group, pa::DecodeKernel *k) {
+bool get_kernel(int dtype, int head_dim, int block_size, int group, bool tensor_cores,
+                pa::DecodeKernel *k) {
   switch (dtype) {
-    case PA_F32: return pa::decode_kernel_f32(head_dim, block_size, group, k);
-    case PA_BF16: return pa::decode_kernel_bf16(head_dim, block_size, group, k);
-    case PA_F16: return pa::decode_kernel_f16(head_dim, block_size, group, k);
+    case PA_F32: return pa::decode_kernel_f32(head_dim, block_size, group, false, k);
+    case PA_BF16: return pa::decode_kernel_bf16(head_dim, block_size, group, tensor_cores, k);
+    case PA_F16: return pa::decode_kernel_f16(head_dim, block_size, group, tensor_cores, k);
     default: return false;
   }
+}
+
+// TMA descriptors of a cache, cached by everything they encode (the pools of a process are few).
+struct MapKey {
+  const void *ptr;
+  int dtype, rows;
+  int64_t shape[4], stride[4];
+  bool operator==(const MapKey &o) const {
+    if (ptr != o.ptr || dtype != o.dtype || rows != o.rows) return false;
+    for (int i = 0; i < 4; ++i)
+      if (shape[i] != o.shape[i] || stride[i] != o.stride[i]) return false;
+    return true;
+  }
+};
+struct MapEntry {
+  MapKey key;
+  CUtensorMap map;
+  uint64_t used;
+};
+std::vector<MapEntry> g_maps;
+uint64_t g_map_clock = 0;
+
+// The cache as a 4-D tensor (head_dim, block_size, kv heads, blocks) read in 128-byte swizzled
+// boxes of 64 elements x `rows` rows (one 128-byte column half of `rows` consecutive tokens).
+int cache_map(const pa_tensor *t, int rows, CUtensorMap *out) {
+  MapKey key;
+  key.ptr = t->data;
+  key.dtype = t->dtype;
+  key.rows = rows;
+  for (int i = 0; i < 4; ++i) {
+    key.shape[i] = t->shape[i];
+    key.stride[i] = t->stride[i];
+  }
+  std::lock_guard<std::mutex> lock(g_mu);
+  for (auto &e : g_maps)
+    if (e.key == key) {
+      e.used = ++g_map_clock;
+      *out = e.map;
+      return PA_OK;
+    }
+  if (!g_encode_tiled) return fail(PA_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
+  const cuuint64_t dims[4] = {(cuuint64_t)t->shape[3], (cuuint64_t)t->shape[2],
+                              (cuuint64_t)t->shape[1], (cuuint64_t)t->shape[0]};
+  const cuuint64_t strides[3] = {(cuuint64_t)t->stride[2] * 2, (cuuint64_t)t->stride[1] * 2,
+                                 (cuuint64_t)t->stride[0] * 2};
+  const cuuint32_t box[4] = {64, (cuuint32_t)rows, 1, 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUtensorMap map;
+  const CUresult r = g_encode_tiled(
+      &map, t->dtype == PA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
+      4, t->data, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+      CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(PA_ERR_LAYOUT, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  if (g_maps.size() >= 16) {
+    size_t old = 0;
+    for (size_t i = 1; i < g_maps.size(); ++i)
+      if (g_maps[i].used < g_maps[old].used) old = i;
+    g_maps.erase(g_maps.begin() + old);
+  }
+  g_maps.push_back(MapEntry{key, map, ++g_map_clock});
+  *out = map;
+  return PA_OK;
 }
 
 // Warps of one full wave of the device for a kernel (CTAs per SM x SMs x warps per CTA).
@@ -275,7 +349,8 @@ int decode_impl(const pa_tensor *out, const pa_tensor *query, const pa_tensor *k
       (rc = check_tensor(block_tables, "block_tables", 2)) ||
       (rc = check_tensor(context_lens, "context_lens", 1)))
     return rc;
-  if (flags & ~PA_DECODE_SEPARATE_REDUCE) return fail(PA_ERR_INVALID_ARG, "unknown flags 0x%x", flags);
+  if (flags & ~(PA_DECODE_SEPARATE_REDUCE | PA_DECODE_CUDA_CORES))
+    return fail(PA_ERR_INVALID_ARG, "unknown flags 0x%x", flags);
   if (num_workers < 0) return fail(PA_ERR_INVALID_ARG, "num_workers must be >= 0");
   if (block_size != cs.block_size)
     return fail(PA_ERR_SHAPE, "block_size %d does not match the cache's %d", block_size, cs.block_size);
@@ -324,8 +399,14 @@ int decode_impl(const pa_tensor *out, const pa_tensor *query, const pa_tensor *k
     return rc;
 
   pa::DecodeKernel k;
-  if (!get_kernel(cs.dtype, D, block_size, G, &k))
+  const bool tensor_cores = cs.dtype != PA_F32 && !(flags & PA_DECODE_CUDA_CORES);
+  if (!get_kernel(cs.dtype, D, block_size, G, tensor_cores, &k))
     return fail(PA_ERR_CUDA, "could not prepare the decode kernel: %s", cudaGetErrorString(cudaGetLastError()));
+  pa::TmaMaps maps;
+  if (k.tma_rows > 0) {
+    if ((rc = cache_map(key_cache, k.tma_rows, &maps.k)) || (rc = cache_map(value_cache, k.tma_rows, &maps.v)))
+      return rc;
+  }
   const int W = num_workers > 0 ? num_workers : default_workers(k, ds->num_sms);
   // worker_of() multiplies a chunk index by W in 64 bits
   const double chunks = (double)S * num_kv_heads * ((double)block_tables->shape[1] * block_size / k.chunk_tokens + 1);
@@ -390,7 +471,7 @@ int decode_impl(const pa_tensor *out, const pa_tensor *query, const pa_tensor *k
   a.wait_cycles = test_hooks().wait_cycles;
   a.test_stall = test_hooks().stall;
   const int ctas = (W + k.warps_per_cta - 1) / k.warps_per_cta;
-  cudaError_t e = k.launch(a, ctas, st);
+  cudaError_t e = k.launch(a, &maps, ctas, st);
   if (e != cudaSuccess) return cuda_fail(e, "decode launch");
   if (a.separate_reduce) {
     e = k.launch_reduce(a, st);
@@ -530,7 +611,7 @@ int32_t pa_decode_default_workers(int32_t dtype, int32_t head_dim, int32_t block
   DeviceState *ds;
   if (device_state(&ds, nullptr) != PA_OK) return 0;
   pa::DecodeKernel k;
-  if (!get_kernel(dtype, head_dim, block_size, group_size, &k)) return 0;
+  if (!get_kernel(dtype, head_dim, block_size, group_size, dtype != PA_F32, &k)) return 0;
   return default_workers(k, ds->num_sms);
 }
 

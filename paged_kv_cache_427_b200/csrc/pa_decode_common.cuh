@@ -1,0 +1,364 @@
+// pa_decode_common.cuh - parts shared by the decode kernels: the stream-K work split over
+// warps, the chunk cursor that walks a warp's share, and the log-sum-exp merge of pieces.
+//
+// What decode computes ([P4] "vLLM core architecture: model loading, PagedAttention
+// principle, KV cache management", 2.2.2): for every sequence s and query head h the keys and
+// values are assembled through the block table and
+//     out[s,h] = softmax_t(scale * q[s,h] . K_t) . V_t  over the positions t < L_s.
+// The per-block loop printed on that page adds per-block outputs and only states the principle;
+// the kernels compute the full-context softmax with running rescaling and merge split contexts
+// with the log-sum-exp rule.  Block tables and physical blocks follow [P2] "vLLM core
+// features: PagedAttention, Continuous Batching, quantization support, distributed inference"
+// 4.1 and [P4] 2.2.1.
+//
+// Work split (B200 design, not from the sources): the step's work is the list of chunks
+// (sequence, kv head, a fixed number of key rows) in sequence-major order, C chunks in all.  A
+// persistent grid of W warps gives warp w the chunks [floor(wC/W), floor((w+1)C/W)) (W is
+// clamped to C so that no share is empty).  No launch size depends on context lengths and every
+// warp moves the same number of bytes, whatever the mix of lengths.  A (sequence, kv head)
+// inside one share is written directly; otherwise each share's piece stores (o, m, l) in the
+// workspace and the last piece to finish (atomic ticket, no waiting) merges them.
+#pragma once
+
+#include "pa_device.cuh"
+#include "pa_internal.h"
+
+namespace pa {
+
+// Per-stage description written by the issuing lane before the stage's barrier arrives.
+struct ChunkMeta {
+  int s, kvh, chunk, len;
+  int flags, first_worker, npieces, pair;
+};
+constexpr int kFirst = 1;      // first chunk of this warp's piece of a (sequence, kv head)
+constexpr int kLast = 2;       // last chunk of the piece
+constexpr int kPairStart = 4;  // chunk 0 of the (sequence, kv head)
+
+__device__ __forceinline__ int clamp_len(int len, int max_len) {
+  return len < 0 ? 0 : (len > max_len ? max_len : len);
+}
+
+// The warp whose share [floor(w*C/W), floor((w+1)*C/W)) contains chunk c.
+__device__ __forceinline__ int worker_of(long long c, long long C, int W) {
+  return (int)(((c + 1) * (long long)W + C - 1) / C - 1);
+}
+
+// Where one warp's share starts and how long it is.
+struct WarpShare {
+  long long C;  // chunks in the step
+  int W;        // effective number of workers
+  long long g0, n;
+  int s, rem, len;  // first chunk: sequence, index among that sequence's Hkv*nch chunks, length
+};
+
+// Block-wide prologue, called by every thread of the CTA: zero rows of empty contexts, count
+// the chunks, and locate each warp's first chunk with an exclusive scan over sequences.
+// `scratch` holds 256 bytes of shared memory.  Returns false when this warp has no work.
+template <int CH, int kWarps, int G, int D>
+__device__ bool split_prologue(const DecodeArgs &a, unsigned char *scratch, int max_len,
+                               WarpShare &ws) {
+  const int lane = threadIdx.x & 31;
+  const int wid = threadIdx.x >> 5;
+  const int S = a.num_seqs;
+  const int Hkv = a.num_kv_heads;
+  long long *red = reinterpret_cast<long long *>(scratch);  // [kWarps]
+  int4 *loc = reinterpret_cast<int4 *>(scratch + 64);       // [kWarps]
+  long long local = 0;
+  for (int s = threadIdx.x; s < S; s += blockDim.x) {
+    const int raw = __ldg(a.context_lens + s);
+    const int len = clamp_len(raw, max_len);
+    if (raw != len && blockIdx.x == 0) set_error(a.err, PA_DEVERR_CONTEXT_LEN);
+    local += (len + CH - 1) / CH;
+    if (len == 0 && (s % gridDim.x) == blockIdx.x) {
+      const int out_elt = a.out_dtype == PA_F32 ? 4 : 2;
+      const float z[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      for (int h = 0; h < Hkv * G; ++h)
+        for (int d = 0; d < D; d += 8)
+          store_row_piece(static_cast<char *>(a.out) +
+                              ((long long)s * a.out_s + (long long)h * a.out_h + d) * out_elt,
+                          a.out_dtype, z, 8);
+    }
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) local += __shfl_xor_sync(FULL_MASK, local, off);
+  if (lane == 0) red[wid] = local;
+  if (threadIdx.x < kWarps) loc[threadIdx.x] = make_int4(-1, 0, 0, 0);
+  __syncthreads();
+  long long C = 0;
+#pragma unroll
+  for (int w = 0; w < kWarps; ++w) C += red[w];
+  C *= Hkv;
+  __syncthreads();
+  const int W = (int)(C < (long long)a.num_workers ? C : (long long)a.num_workers);
+  ws.C = C;
+  ws.W = W;
+  if (W == 0) return false;
+
+  long long my_g0[kWarps];
+  long long last_needed = -1;
+#pragma unroll
+  for (int w = 0; w < kWarps; ++w) {
+    long long gw = (long long)blockIdx.x * kWarps + w;
+    if (gw > W) gw = W;
+    my_g0[w] = gw * C / W;
+    const long long g1 = (gw + 1 > W ? W : gw + 1) * C / W;
+    if (my_g0[w] < g1) last_needed = my_g0[w];
+  }
+  long long running = 0;
+  for (int base = 0; base < S && running <= last_needed; base += 8 * 32 * kWarps) {
+    long long cnt[8];
+    long long tsum = 0;
+    int lens8[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const int s = base + threadIdx.x * 8 + k;
+      lens8[k] = s < S ? clamp_len(__ldg(a.context_lens + s), max_len) : 0;
+      cnt[k] = (long long)((lens8[k] + CH - 1) / CH) * Hkv;
+      tsum += cnt[k];
+    }
+    long long x = tsum;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const long long y = __shfl_up_sync(FULL_MASK, x, off);
+      if (lane >= off) x += y;
+    }
+    if (lane == 31) red[wid] = x;
+    __syncthreads();
+    long long ex = running;
+    long long tile_total = 0;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) {
+      if (w < wid) ex += red[w];
+      tile_total += red[w];
+    }
+    ex += x - tsum;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+#pragma unroll
+      for (int w = 0; w < kWarps; ++w)
+        if (my_g0[w] <= last_needed && my_g0[w] >= ex && my_g0[w] < ex + cnt[k])
+          loc[w] = make_int4(base + threadIdx.x * 8 + k, (int)(my_g0[w] - ex), lens8[k], 0);
+      ex += cnt[k];
+    }
+    running += tile_total;
+    __syncthreads();
+  }
+
+  const int gw = blockIdx.x * kWarps + wid;
+  if (gw >= W) return false;
+  ws.g0 = (long long)gw * C / W;
+  ws.n = (long long)(gw + 1) * C / W - ws.g0;
+  const int4 st = loc[wid];
+  ws.s = st.x;
+  ws.rem = st.y;
+  ws.len = st.z;
+  return ws.n > 0 && st.x >= 0;
+}
+
+// Walks one warp's share chunk by chunk in issue order.  Every lane keeps the same state.
+// A chunk is CH key rows; it touches COPIES physical blocks of COPY_ROWS rows each.  The block
+// ids of the next chunk to issue are loaded one chunk ahead.
+template <int CH, int BS, int COPIES, int COPY_ROWS>
+struct ChunkCursor {
+  int s, len, nch, kvh, i, next_len;
+  long long base;  // global index of chunk 0 of the current (sequence, kv head)
+  int first_worker, npieces;
+  long long issued, n, C;
+  int W, S, Hkv, max_len;
+  int blk[COPIES];
+
+  __device__ __forceinline__ void fetch_blocks(const DecodeArgs &a) {
+#pragma unroll
+    for (int k = 0; k < COPIES; ++k) {
+      const int t = i * CH + k * COPY_ROWS;
+      blk[k] = (t < len) ? __ldg(a.block_tables + (long long)s * a.bt_s + t / BS) : 0;
+    }
+  }
+
+  __device__ __forceinline__ void pieces() {
+    first_worker = worker_of(base, C, W);
+    npieces = worker_of(base + nch - 1, C, W) - first_worker + 1;
+  }
+
+  __device__ __forceinline__ void init(const DecodeArgs &a, const WarpShare &ws, int max_len_) {
+    S = a.num_seqs;
+    Hkv = a.num_kv_heads;
+    max_len = max_len_;
+    C = ws.C;
+    W = ws.W;
+    n = ws.n;
+    issued = 0;
+    s = ws.s;
+    len = ws.len;
+    nch = (len + CH - 1) / CH;
+    kvh = ws.rem / nch;
+    i = ws.rem % nch;
+    base = ws.g0 - ws.rem + (long long)kvh * nch;
+    next_len = (s + 1 < S) ? clamp_len(__ldg(a.context_lens + s + 1), max_len) : 0;
+    fetch_blocks(a);
+    pieces();
+  }
+
+  __device__ __forceinline__ int flags() const {
+    int f = 0;
+    if (i == 0 || issued == 0) f |= kFirst;
+    if (i == nch - 1 || issued == n - 1) f |= kLast;
+    if (i == 0) f |= kPairStart;
+    return f;
+  }
+
+  __device__ __forceinline__ ChunkMeta meta(int f) const {
+    ChunkMeta m;
+    m.s = s;
+    m.kvh = kvh;
+    m.chunk = i;
+    m.len = len;
+    m.flags = f;
+    m.first_worker = first_worker;
+    m.npieces = npieces;
+    m.pair = s * Hkv + kvh;
+    return m;
+  }
+
+  // Copies of this chunk that hold context rows (the others are past the context).
+  __device__ __forceinline__ int valid_copies() const {
+    int v = 0;
+#pragma unroll
+    for (int k = 0; k < COPIES; ++k) v += (i * CH + k * COPY_ROWS < len);
+    return v;
+  }
+
+  // Move to the next chunk of the share (call after issuing the current one).
+  __device__ __forceinline__ void advance(const DecodeArgs &a) {
+    ++issued;
+    if (issued >= n) return;
+    if (++i == nch) {
+      i = 0;
+      base += nch;
+      if (++kvh == Hkv) {
+        kvh = 0;
+        ++s;
+        len = next_len;
+        while (len == 0 && s + 1 < S) {
+          ++s;
+          len = clamp_len(__ldg(a.context_lens + s), max_len);
+        }
+        nch = (len + CH - 1) / CH;
+        next_len = (s + 1 < S) ? clamp_len(__ldg(a.context_lens + s + 1), max_len) : 0;
+      }
+      pieces();
+    }
+    fetch_blocks(a);
+  }
+};
+
+// Merge the pieces (o, m, l) of one (sequence, kv head) and write its G output rows.  Called by
+// a whole warp; pieces live in workspace slots pair + first_worker + k, k < npieces; lane j
+// handles dims [4j, 4j+4) of every head.  m is in base-2 logit units.
+template <int G, int D>
+__device__ __forceinline__ void merge_pieces(const DecodeArgs &a, int pair, int first_worker,
+                                             int npieces, int s, int kvh, int lane) {
+  float M[G];
+#pragma unroll
+  for (int h = 0; h < G; ++h) M[h] = -INFINITY;
+  for (int k = 0; k < npieces; ++k) {
+    const long long seg = (long long)pair + first_worker + k;
+#pragma unroll
+    for (int h = 0; h < G; ++h) M[h] = fmaxf(M[h], __ldcg(a.part_ml + (seg * G + h) * 2));
+  }
+  const bool active = lane < D / 4;
+  float4 num[G];
+  float den[G];
+#pragma unroll
+  for (int h = 0; h < G; ++h) {
+    den[h] = 0.f;
+    num[h] = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+  for (int k = 0; k < npieces; ++k) {
+    const long long seg = (long long)pair + first_worker + k;
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+      const float m = __ldcg(a.part_ml + (seg * G + h) * 2);
+      const float l = __ldcg(a.part_ml + (seg * G + h) * 2 + 1);
+      const float w = l * fast_exp2(m - M[h]);
+      den[h] += w;
+      if (active) {
+        const float4 x = __ldcg(reinterpret_cast<const float4 *>(a.part_o + (seg * G + h) * D) + lane);
+        num[h].x += w * x.x;
+        num[h].y += w * x.y;
+        num[h].z += w * x.z;
+        num[h].w += w * x.w;
+      }
+    }
+  }
+  if (!active) return;
+  const int out_elt = a.out_dtype == PA_F32 ? 4 : 2;
+#pragma unroll
+  for (int h = 0; h < G; ++h) {
+    const float inv = 1.f / den[h];
+    const float v[4] = {num[h].x * inv, num[h].y * inv, num[h].z * inv, num[h].w * inv};
+    char *dst = static_cast<char *>(a.out) +
+                ((long long)s * a.out_s + (long long)(kvh * G + h) * a.out_h + lane * 4) * out_elt;
+    if (a.out_dtype == PA_F32) {
+      *reinterpret_cast<float4 *>(dst) = make_float4(v[0], v[1], v[2], v[3]);
+    } else if (a.out_dtype == PA_BF16) {
+      __nv_bfloat162 lo = __floats2bfloat162_rn(v[0], v[1]), hi = __floats2bfloat162_rn(v[2], v[3]);
+      uint2 u;
+      u.x = *reinterpret_cast<uint32_t *>(&lo);
+      u.y = *reinterpret_cast<uint32_t *>(&hi);
+      *reinterpret_cast<uint2 *>(dst) = u;
+    } else {
+      __half2 lo = __floats2half2_rn(v[0], v[1]), hi = __floats2half2_rn(v[2], v[3]);
+      uint2 u;
+      u.x = *reinterpret_cast<uint32_t *>(&lo);
+      u.y = *reinterpret_cast<uint32_t *>(&hi);
+      *reinterpret_cast<uint2 *>(dst) = u;
+    }
+  }
+}
+
+// After a piece's (o, m, l) are stored: publish them, take a ticket, and merge when this is the
+// last piece of its (sequence, kv head).  Called by a whole warp.
+template <int G, int D>
+__device__ __forceinline__ void finish_piece(const DecodeArgs &a, const ChunkMeta &m, int lane) {
+  if (a.separate_reduce) return;
+  __threadfence();
+  __syncwarp();
+  unsigned int ticket = 0;
+  if (lane == 0) ticket = atomicAdd(a.counters + m.pair, 1u);
+  ticket = __shfl_sync(FULL_MASK, ticket, 0);
+  if (ticket == (unsigned int)(m.npieces - 1)) {
+    __threadfence();
+    merge_pieces<G, D>(a, m.pair, m.first_worker, m.npieces, m.s, m.kvh, lane);
+    if (lane == 0) a.counters[m.pair] = 0u;
+  }
+}
+
+// Separate merge: one warp per (sequence, kv head) that has more than one piece.
+template <int G, int D, int BS>
+__global__ void __launch_bounds__(128) paged_decode_merge_kernel(const DecodeArgs a) {
+  const int lane = threadIdx.x & 31;
+  const long long pairs = (long long)a.num_seqs * a.num_kv_heads;
+  const int max_len = a.max_blocks * BS;
+  for (long long p = (long long)blockIdx.x * 4 + (threadIdx.x >> 5); p < pairs;
+       p += (long long)gridDim.x * 4) {
+    const int s = (int)(p / a.num_kv_heads);
+    const int kvh = (int)(p % a.num_kv_heads);
+    if (clamp_len(__ldg(a.context_lens + s), max_len) == 0) continue;
+    const int2 pm = a.pair_meta[p];
+    if (pm.y <= 1) continue;
+    merge_pieces<G, D>(a, (int)p, pm.x, pm.y, s, kvh, lane);
+  }
+}
+
+template <int G, int D, int BS>
+cudaError_t launch_decode_merge(const DecodeArgs &a, cudaStream_t st) {
+  const long long pairs = (long long)a.num_seqs * a.num_kv_heads;
+  long long blocks = (pairs + 3) / 4;
+  if (blocks > 4096) blocks = 4096;
+  if (blocks < 1) blocks = 1;
+  paged_decode_merge_kernel<G, D, BS><<<(int)blocks, 128, 0, st>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace pa

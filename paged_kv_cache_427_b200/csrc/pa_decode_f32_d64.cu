@@ -1,8 +1,9 @@
-// Decode kernels for f32 caches with head_dim 64 (block sizes 8/16/32, groups 1/2/4/8).
-#include "pa_decode.cuh"
+// Decode kernels for fp32 caches with head_dim 64 (CUDA-core; block sizes 8/16/32, 1/2/4/8
+// query heads per kv head).
+#include "pa_decode_mma.cuh"
 
 namespace pa {
-bool decode_kernel_f32_d64(int block_size, int group, DecodeKernel *k) {
-  return decode_kernel_table<float, 64>(block_size, group, k);
+bool decode_kernel_f32_d64(int block_size, int group, bool, DecodeKernel *k) {
+  return decode_table_f32<64>(block_size, group, k);
 }
 }  // namespace pa

@@ -1,0 +1,465 @@
+// pa_decode_mma.cuh - the tensor-core decode kernel for 16-bit caches (bf16 or fp16).
+//
+// Same work split, cursor and merge as the CUDA-core kernel (pa_decode_common.cuh); what
+// changes is how a chunk of 16 key/value rows is consumed:
+//   * Loads: each chunk's key and value tiles arrive by TMA tensor copies (the caches are
+//     described as 4-D tensors head_dim x block_size x kv_heads x blocks) in the 128-byte
+//     swizzled layout, one box of 64 elements x 16 rows (8 at block_size 8) per 128-byte column
+//     half; the block id of each box comes from the block table, fetched a chunk ahead.  The
+//     swizzle makes every ldmatrix below free of shared-memory bank conflicts.
+//   * q.K: mma.sync m16n8k16 with the 16 tokens as M, the query heads of the GQA group as N
+//     (padded to 8 with zeros) and head_dim as K; A comes from the key tile by ldmatrix, B (the
+//     group's query rows) is loaded once per piece into registers.  Products of two 16-bit
+//     values are exact in the fp32 accumulator; the scale is applied to the fp32 result.
+//   * softmax: base-2 logits, per-head chunk maxima over 8 lanes by shuffles, the running
+//     maximum moved only when a chunk exceeds it by more than 2^8 (weights stay <= 256).
+//   * P.V: mma.sync with head_dim as M (V tile read transposed by ldmatrix.trans), the tokens as
+//     K and the heads as N.  P is split into two 16-bit terms (P = hi + lo, hi = round(P),
+//     lo = round(P - hi)) so the weights keep about 16 significant bits: one 16-bit rounding of P
+//     alone would cost ~2^-9 relative error per weight.
+// An instruction count of about 200 per 16-token chunk (against about 1000 for the CUDA-core
+// kernel) leaves the kernel bound by HBM bandwidth.
+#pragma once
+
+#include "pa_decode.cuh"
+
+namespace pa {
+
+template <typename T>
+struct MmaType;
+template <>
+struct MmaType<__nv_bfloat16> {
+  static __device__ __forceinline__ void mma(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                             uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+        "{%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+  }
+  // p -> (hi, lo) as 16-bit patterns with hi + lo ~= p to about 16 significant bits
+  static __device__ __forceinline__ void split(float p, uint16_t &hi, uint16_t &lo) {
+    const __nv_bfloat16 h = __float2bfloat16_rn(p);
+    const __nv_bfloat16 l = __float2bfloat16_rn(p - __bfloat162float(h));
+    hi = *reinterpret_cast<const uint16_t *>(&h);
+    lo = *reinterpret_cast<const uint16_t *>(&l);
+  }
+  static constexpr CUtensorMapDataType kTmaType = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+};
+template <>
+struct MmaType<__half> {
+  static __device__ __forceinline__ void mma(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                             uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+        "{%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+  }
+  static __device__ __forceinline__ void split(float p, uint16_t &hi, uint16_t &lo) {
+    const __half h = __float2half_rn(p);
+    const __half l = __float2half_rn(p - __half2float(h));
+    hi = *reinterpret_cast<const uint16_t *>(&h);
+    lo = *reinterpret_cast<const uint16_t *>(&l);
+  }
+  static constexpr CUtensorMapDataType kTmaType = CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+};
+
+__device__ __forceinline__ void ldmatrix_x4(uint32_t (&r)[4], uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+
+__device__ __forceinline__ void ldmatrix_x4_trans(uint32_t (&r)[4], uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+
+// TMA tensor copy of one box (x = element column, y = row in block, z = kv head, w = block)
+// into shared memory, completion counted on `bar`.
+__device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap *map, int x, int y,
+                                            int z, int w, uint64_t *bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes "
+      "[%0], [%1, {%2, %3, %4, %5}], [%6];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(w), "r"(smem_u32(bar))
+      : "memory");
+}
+
+template <int D, int BS, int G>
+struct MmaTraits {
+  static constexpr int kChunk = 16;                     // tokens per chunk (M of q.K)
+  static constexpr int kHalves = D / 64;                // 128-byte column halves of a row
+  static constexpr int kBoxRows = BS < 16 ? BS : 16;    // rows per TMA box
+  static constexpr int kCopies = 16 / kBoxRows;         // blocks touched per chunk
+  static constexpr int kTileBytes = 16 * D * 2;         // key (or value) bytes of a chunk
+  static constexpr int kQBytes = G * D * 2;
+  static constexpr int kStageBytes = 2 * kTileBytes + (kQBytes + 1023) / 1024 * 1024;
+  static constexpr int kWarps = 4;
+  static constexpr int kStages = (kWarps * 3 * kStageBytes <= 110 * 1024) ? 3 : 2;
+  static constexpr int kRingBytes = kWarps * kStages * kStageBytes;
+  static constexpr int kPbufBytes = 2 * 8 * 16 * 2;    // [hi, lo][8 heads][16 tokens]
+  static constexpr int kSmallBytes = (kStages * 32 + kStages * 8 + 127) / 128 * 128 + kPbufBytes;
+  static constexpr int kPrologueOff = kRingBytes + kWarps * kSmallBytes;
+  static constexpr int kSmemBytes = kPrologueOff + 256 + 1024;  // + slack to align to 1 KB
+  static constexpr int kKSteps = D / 16;                // k-steps of q.K
+  static constexpr int kMTiles = D / 16;                // m-tiles of P.V
+  static_assert(D == 64 || D == 128, "head_dim 64 or 128");
+  static_assert(G <= 8, "at most 8 query heads per kv head");
+};
+
+template <typename T, int D, int BS, int G>
+__global__ void __launch_bounds__(128, 2)
+    paged_decode_mma_kernel(const DecodeArgs a, const __grid_constant__ TmaMaps maps) {
+  using Tr = MmaTraits<D, BS, G>;
+  using M = MmaType<T>;
+  constexpr int ST = Tr::kStages;
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  // 128-byte swizzled boxes must start on 1 KB boundaries
+  unsigned char *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+
+  const int lane = threadIdx.x & 31;
+  const int wid = threadIdx.x >> 5;
+  const int max_len = a.max_blocks * BS;
+
+  WarpShare share;
+  if (!split_prologue<16, Tr::kWarps, G, D>(a, smem + Tr::kPrologueOff, max_len, share)) return;
+  const int gw = blockIdx.x * Tr::kWarps + wid;
+
+  unsigned char *ring = smem + wid * ST * Tr::kStageBytes;
+  unsigned char *small = smem + Tr::kRingBytes + wid * Tr::kSmallBytes;
+  ChunkMeta *meta = reinterpret_cast<ChunkMeta *>(small);
+  uint64_t *bars = reinterpret_cast<uint64_t *>(small + ST * 32);
+  unsigned char *pbuf = small + (ST * 32 + ST * 8 + 127) / 128 * 128;
+  if (lane == 0) {
+#pragma unroll
+    for (int i = 0; i < ST; ++i) mbar_init(bars + i, 1);
+    fence_barrier_init();
+  }
+  __syncwarp();
+
+  ChunkCursor<16, BS, Tr::kCopies, Tr::kBoxRows> cur;
+  cur.init(a, share, max_len);
+  const long long n = share.n;
+
+  auto issue = [&](int slot) {
+    const int f = cur.flags();
+    unsigned char *stage = ring + slot * Tr::kStageBytes;
+    if (lane == 0) {
+      meta[slot] = cur.meta(f);
+      const uint32_t bytes = 2u * cur.valid_copies() * Tr::kHalves * Tr::kBoxRows * 128u +
+                             ((f & kFirst) ? (uint32_t)Tr::kQBytes : 0u) +
+                             ((a.test_stall && cur.issued == 0) ? 16u : 0u);
+      fence_proxy_async_smem();
+      mbar_arrive_expect_tx(bars + slot, bytes);
+#pragma unroll
+      for (int k = 0; k < Tr::kCopies; ++k) {
+        const int t = cur.i * 16 + k * Tr::kBoxRows;
+        if (t < cur.len) {
+          int blk = cur.blk[k];
+          if (blk < 0 || (long long)blk >= a.num_blocks) {
+            set_error(a.err, PA_DEVERR_BLOCK_ID);
+            blk = 0;
+          }
+#pragma unroll
+          for (int hf = 0; hf < Tr::kHalves; ++hf) {
+            const uint32_t off = hf * 2048 + k * Tr::kBoxRows * 128;
+            tma_load_4d(smem_u32(stage + off), &maps.k, hf * 64, t % BS, cur.kvh, blk, bars + slot);
+            tma_load_4d(smem_u32(stage + Tr::kTileBytes + off), &maps.v, hf * 64, t % BS, cur.kvh,
+                        blk, bars + slot);
+          }
+        }
+      }
+      if (f & kFirst) {
+        const char *q = static_cast<const char *>(a.query) +
+                        ((long long)cur.s * a.q_s + (long long)cur.kvh * G * a.q_h) * 2;
+        if (a.q_heads_contiguous) {
+          bulk_copy_g2s(stage + 2 * Tr::kTileBytes, q, Tr::kQBytes, bars + slot);
+        } else {
+#pragma unroll
+          for (int h = 0; h < G; ++h)
+            bulk_copy_g2s(stage + 2 * Tr::kTileBytes + h * D * 2, q + (long long)h * a.q_h * 2, D * 2,
+                          bars + slot);
+        }
+      }
+    }
+    cur.advance(a);
+  };
+
+  const long long prime = n < ST ? n : ST;
+  for (long long i = 0; i < prime; ++i) issue((int)i);
+
+  const int g = lane >> 2;  // fragment row group
+  const int c = lane & 3;   // fragment column pair
+  const int h0 = 2 * c, h1 = 2 * c + 1;  // heads of this lane's logits / output columns
+  // ldmatrix row addressing (constant per lane)
+  const int lm = lane >> 3;         // which 8x8 matrix this lane addresses
+  const int lr = lane & 7;          // row within it
+  uint32_t qb[Tr::kKSteps][2];
+  float o[Tr::kMTiles][4];
+  float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
+
+  for (long long cc = 0; cc < n; ++cc) {
+    const int slot = (int)(cc % ST);
+    const uint32_t parity = (uint32_t)((cc / ST) & 1);
+    if (!mbar_wait_bounded(bars + slot, parity, a.wait_cycles)) {
+      if (lane == 0) set_error(a.err, PA_DEVERR_TIMEOUT);
+      for (long long k = cc; k < cur.issued; ++k)
+        mbar_wait_bounded(bars + (int)(k % ST), (uint32_t)((k / ST) & 1), a.wait_cycles);
+      return;
+    }
+    const ChunkMeta m = meta[slot];
+    unsigned char *stage = ring + slot * Tr::kStageBytes;
+    const uint32_t kbase = smem_u32(stage);
+    const uint32_t vbase = kbase + Tr::kTileBytes;
+    if (m.flags & kFirst) {
+      const unsigned char *qs = stage + 2 * Tr::kTileBytes;
+#pragma unroll
+      for (int ks = 0; ks < Tr::kKSteps; ++ks) {
+        if (g < G) {
+          qb[ks][0] = *reinterpret_cast<const uint32_t *>(qs + (g * D + 16 * ks + 2 * c) * 2);
+          qb[ks][1] = *reinterpret_cast<const uint32_t *>(qs + (g * D + 16 * ks + 8 + 2 * c) * 2);
+        } else {
+          qb[ks][0] = 0u;
+          qb[ks][1] = 0u;
+        }
+      }
+#pragma unroll
+      for (int mt = 0; mt < Tr::kMTiles; ++mt) o[mt][0] = o[mt][1] = o[mt][2] = o[mt][3] = 0.f;
+      m0 = m1 = -INFINITY;
+      l0 = l1 = 0.f;
+    }
+
+    // ---- q.K on tensor cores: s = S[token g | g+8][head 2c | 2c+1] ----
+    float s[4] = {0.f, 0.f, 0.f, 0.f};
+    {
+      const int row = ((lm & 1) << 3) | lr;
+#pragma unroll
+      for (int ks = 0; ks < Tr::kKSteps; ++ks) {
+        const int c16 = ((ks & 3) << 1) | (lm >> 1);
+        const uint32_t addr = kbase + (ks >> 2) * 2048 + row * 128 + ((c16 ^ lr) << 4);
+        uint32_t af[4];
+        ldmatrix_x4(af, addr);
+        M::mma(s, af, qb[ks][0], qb[ks][1]);
+      }
+    }
+#pragma unroll
+    for (int e = 0; e < 4; ++e) s[e] *= a.scale_log2;
+    const int tok0 = m.chunk * 16;
+    const bool tail = tok0 + 16 > m.len;
+    if (tail) {
+      if (tok0 + g >= m.len) s[0] = s[1] = -INFINITY;
+      if (tok0 + g + 8 >= m.len) s[2] = s[3] = -INFINITY;
+    }
+
+    // ---- online softmax ----
+    float cm0 = fmaxf(s[0], s[2]), cm1 = fmaxf(s[1], s[3]);
+#pragma unroll
+    for (int off = 4; off < 32; off <<= 1) {
+      cm0 = fmaxf(cm0, __shfl_xor_sync(FULL_MASK, cm0, off));
+      cm1 = fmaxf(cm1, __shfl_xor_sync(FULL_MASK, cm1, off));
+    }
+    if (__any_sync(FULL_MASK, (cm0 > m0 + 8.f) || (cm1 > m1 + 8.f))) {
+      const float n0 = fmaxf(m0, cm0), n1 = fmaxf(m1, cm1);
+      const float a0 = fast_exp2(m0 - n0), a1 = fast_exp2(m1 - n1);
+      m0 = n0;
+      m1 = n1;
+      l0 *= a0;
+      l1 *= a1;
+#pragma unroll
+      for (int mt = 0; mt < Tr::kMTiles; ++mt) {
+        o[mt][0] *= a0;
+        o[mt][1] *= a1;
+        o[mt][2] *= a0;
+        o[mt][3] *= a1;
+      }
+    }
+    const float p0 = fast_exp2(s[0] - m0), p1 = fast_exp2(s[1] - m1);
+    const float p2 = fast_exp2(s[2] - m0), p3 = fast_exp2(s[3] - m1);
+    l0 += p0 + p2;
+    l1 += p1 + p3;
+    {
+      // P transposed to [hi|lo][head][token] for the B operand of P.V
+      uint16_t *pb = reinterpret_cast<uint16_t *>(pbuf);
+      uint16_t hi, lo;
+      M::split(p0, hi, lo);
+      pb[h0 * 16 + g] = hi;
+      pb[128 + h0 * 16 + g] = lo;
+      M::split(p1, hi, lo);
+      pb[h1 * 16 + g] = hi;
+      pb[128 + h1 * 16 + g] = lo;
+      M::split(p2, hi, lo);
+      pb[h0 * 16 + g + 8] = hi;
+      pb[128 + h0 * 16 + g + 8] = lo;
+      M::split(p3, hi, lo);
+      pb[h1 * 16 + g + 8] = hi;
+      pb[128 + h1 * 16 + g + 8] = lo;
+    }
+    __syncwarp();
+    uint32_t pf[4];  // B fragments: hi (tokens 0-7, 8-15), lo (tokens 0-7, 8-15)
+    ldmatrix_x4(pf, smem_u32(pbuf) + (lm >> 1) * 256 + lr * 32 + (lm & 1) * 16);
+
+    // ---- P.V on tensor cores: o[mt] = O^T[dim 16mt+g | +8][head 2c | 2c+1] ----
+    {
+      const int row = ((lm >> 1) << 3) | lr;  // token row of the V tile
+      const bool mask_lo = tail && (tok0 + 2 * c >= m.len);
+      const bool mask_hi = tail && (tok0 + 2 * c + 1 >= m.len);
+      const bool mask_lo8 = tail && (tok0 + 2 * c + 8 >= m.len);
+      const bool mask_hi8 = tail && (tok0 + 2 * c + 9 >= m.len);
+#pragma unroll
+      for (int mt = 0; mt < Tr::kMTiles; ++mt) {
+        const int c16g = (mt << 1) | (lm & 1);
+        const uint32_t addr =
+            vbase + (c16g >> 3) * 2048 + row * 128 + (((c16g & 7) ^ lr) << 4);
+        uint32_t vf[4];
+        ldmatrix_x4_trans(vf, addr);
+        if (tail) {
+          // rows past the context may hold anything (NaN included): zero them
+          if (mask_lo) { vf[0] &= 0xffff0000u; vf[1] &= 0xffff0000u; }
+          if (mask_hi) { vf[0] &= 0x0000ffffu; vf[1] &= 0x0000ffffu; }
+          if (mask_lo8) { vf[2] &= 0xffff0000u; vf[3] &= 0xffff0000u; }
+          if (mask_hi8) { vf[2] &= 0x0000ffffu; vf[3] &= 0x0000ffffu; }
+        }
+        M::mma(o[mt], vf, pf[0], pf[1]);
+        M::mma(o[mt], vf, pf[2], pf[3]);
+      }
+    }
+
+    // ---- end of a piece ----
+    if (m.flags & kLast) {
+      float t0 = l0, t1 = l1;
+#pragma unroll
+      for (int off = 4; off < 32; off <<= 1) {
+        t0 += __shfl_xor_sync(FULL_MASK, t0, off);
+        t1 += __shfl_xor_sync(FULL_MASK, t1, off);
+      }
+      const float inv0 = 1.f / t0, inv1 = 1.f / t1;
+      if (a.separate_reduce && (m.flags & kPairStart) && lane == 0)
+        a.pair_meta[m.pair] = make_int2(m.first_worker, m.npieces);
+      if (m.npieces == 1) {
+        const int out_elt = a.out_dtype == PA_F32 ? 4 : 2;
+        char *row0 = static_cast<char *>(a.out) +
+                     ((long long)m.s * a.out_s + (long long)(m.kvh * G + h0) * a.out_h) * out_elt;
+        char *row1 = row0 + (long long)a.out_h * out_elt;
+#pragma unroll
+        for (int mt = 0; mt < Tr::kMTiles; ++mt) {
+          const int d0 = 16 * mt + g, d1 = d0 + 8;
+          if (a.out_dtype == PA_F32) {
+            if (h0 < G) {
+              reinterpret_cast<float *>(row0)[d0] = o[mt][0] * inv0;
+              reinterpret_cast<float *>(row0)[d1] = o[mt][2] * inv0;
+            }
+            if (h1 < G) {
+              reinterpret_cast<float *>(row1)[d0] = o[mt][1] * inv1;
+              reinterpret_cast<float *>(row1)[d1] = o[mt][3] * inv1;
+            }
+          } else if (a.out_dtype == PA_BF16) {
+            if (h0 < G) {
+              reinterpret_cast<__nv_bfloat16 *>(row0)[d0] = __float2bfloat16_rn(o[mt][0] * inv0);
+              reinterpret_cast<__nv_bfloat16 *>(row0)[d1] = __float2bfloat16_rn(o[mt][2] * inv0);
+            }
+            if (h1 < G) {
+              reinterpret_cast<__nv_bfloat16 *>(row1)[d0] = __float2bfloat16_rn(o[mt][1] * inv1);
+              reinterpret_cast<__nv_bfloat16 *>(row1)[d1] = __float2bfloat16_rn(o[mt][3] * inv1);
+            }
+          } else {
+            if (h0 < G) {
+              reinterpret_cast<__half *>(row0)[d0] = __float2half_rn(o[mt][0] * inv0);
+              reinterpret_cast<__half *>(row0)[d1] = __float2half_rn(o[mt][2] * inv0);
+            }
+            if (h1 < G) {
+              reinterpret_cast<__half *>(row1)[d0] = __float2half_rn(o[mt][1] * inv1);
+              reinterpret_cast<__half *>(row1)[d1] = __float2half_rn(o[mt][3] * inv1);
+            }
+          }
+        }
+      } else {
+        const long long seg = (long long)m.pair + gw;
+        float *o0 = a.part_o + (seg * G + h0) * D;
+        float *o1 = o0 + D;
+#pragma unroll
+        for (int mt = 0; mt < Tr::kMTiles; ++mt) {
+          const int d0 = 16 * mt + g, d1 = d0 + 8;
+          if (h0 < G) {
+            o0[d0] = o[mt][0] * inv0;
+            o0[d1] = o[mt][2] * inv0;
+          }
+          if (h1 < G) {
+            o1[d0] = o[mt][1] * inv1;
+            o1[d1] = o[mt][3] * inv1;
+          }
+        }
+        if (g == 0) {
+          if (h0 < G) *reinterpret_cast<float2 *>(a.part_ml + (seg * G + h0) * 2) = make_float2(m0, t0);
+          if (h1 < G) *reinterpret_cast<float2 *>(a.part_ml + (seg * G + h1) * 2) = make_float2(m1, t1);
+        }
+        finish_piece<G, D>(a, m, lane);
+      }
+    }
+    __syncwarp();
+    if (cur.issued < n) issue(slot);
+  }
+}
+
+template <typename T, int D, int BS, int G>
+cudaError_t launch_decode_mma(const DecodeArgs &a, const TmaMaps *maps, int num_ctas,
+                              cudaStream_t st) {
+  using Tr = MmaTraits<D, BS, G>;
+  paged_decode_mma_kernel<T, D, BS, G><<<num_ctas, Tr::kWarps * 32, Tr::kSmemBytes, st>>>(a, *maps);
+  return cudaGetLastError();
+}
+
+template <typename T, int D, int BS, int G>
+bool make_decode_mma(DecodeKernel *k) {
+  using Tr = MmaTraits<D, BS, G>;
+  static bool configured[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
+  if (!configured[dev]) {
+    if (cudaFuncSetAttribute(paged_decode_mma_kernel<T, D, BS, G>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             Tr::kSmemBytes) != cudaSuccess)
+      return false;
+    configured[dev] = true;
+  }
+  k->launch = &launch_decode_mma<T, D, BS, G>;
+  k->launch_reduce = &launch_decode_merge<G, D, BS>;
+  k->kernel = reinterpret_cast<const void *>(&paged_decode_mma_kernel<T, D, BS, G>);
+  k->warps_per_cta = Tr::kWarps;
+  k->smem_bytes = Tr::kSmemBytes;
+  k->chunk_tokens = 16;
+  k->tma_rows = Tr::kBoxRows;
+  return true;
+}
+
+// Tables over block_size {8, 16, 32} x group {1, 2, 4, 8} for one element type and head_dim.
+template <typename T, int D>
+bool decode_table(int block_size, int group, bool tensor_cores, DecodeKernel *k) {
+#define PA_CASE(BB, GG)                                                            \
+  if (block_size == BB && group == GG)                                             \
+    return tensor_cores ? make_decode_mma<T, D, BB, GG>(k) : make_decode_simt<T, D, BB, GG>(k);
+#define PA_GROUPS(BB) PA_CASE(BB, 1) PA_CASE(BB, 2) PA_CASE(BB, 4) PA_CASE(BB, 8)
+  PA_GROUPS(8)
+  PA_GROUPS(16)
+  PA_GROUPS(32)
+#undef PA_GROUPS
+#undef PA_CASE
+  return false;
+}
+
+template <int D>
+bool decode_table_f32(int block_size, int group, DecodeKernel *k) {
+#define PA_CASE(BB, GG) \
+  if (block_size == BB && group == GG) return make_decode_simt<float, D, BB, GG>(k);
+#define PA_GROUPS(BB) PA_CASE(BB, 1) PA_CASE(BB, 2) PA_CASE(BB, 4) PA_CASE(BB, 8)
+  PA_GROUPS(8)
+  PA_GROUPS(16)
+  PA_GROUPS(32)
+#undef PA_GROUPS
+#undef PA_CASE
+  return false;
+}
+
+}  // namespace pa

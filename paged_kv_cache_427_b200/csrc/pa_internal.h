@@ -1,6 +1,7 @@
 // pa_internal.h - host-side interface between the C ABI (pa_api.cu) and the kernel files.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -37,20 +38,28 @@ struct DecodeArgs {
   int test_stall;         // test hook: each warp's first stage expects 16 bytes nobody sends
 };
 
+// TMA descriptors of the two caches, viewed as 4-D tensors (head_dim, block_size, kv heads,
+// blocks), 128-byte swizzled boxes of 64 elements x tma_rows rows.
+struct TmaMaps {
+  CUtensorMap k;
+  CUtensorMap v;
+};
+
 struct DecodeKernel {
-  cudaError_t (*launch)(const DecodeArgs &, int num_ctas, cudaStream_t);
+  cudaError_t (*launch)(const DecodeArgs &, const TmaMaps *, int num_ctas, cudaStream_t);
   cudaError_t (*launch_reduce)(const DecodeArgs &, cudaStream_t);
   const void *kernel;  // for occupancy queries
   int warps_per_cta;
   int smem_bytes;
   int chunk_tokens;
+  int tma_rows;  // 0: the kernel reads the caches with 1-D bulk copies; else TMA box rows
 };
 
-// Kernel tables, one per element type.  Return false when the (head_dim, block_size, group)
-// combination is not built.
-bool decode_kernel_f32(int head_dim, int block_size, int group, DecodeKernel *k);
-bool decode_kernel_bf16(int head_dim, int block_size, int group, DecodeKernel *k);
-bool decode_kernel_f16(int head_dim, int block_size, int group, DecodeKernel *k);
+// Kernel tables, one per element type.  `tensor_cores` selects the mma.sync kernel (16-bit
+// types only).  Return false when the combination is not built.
+bool decode_kernel_f32(int head_dim, int block_size, int group, bool tensor_cores, DecodeKernel *k);
+bool decode_kernel_bf16(int head_dim, int block_size, int group, bool tensor_cores, DecodeKernel *k);
+bool decode_kernel_f16(int head_dim, int block_size, int group, bool tensor_cores, DecodeKernel *k);
 
 struct CacheWriteArgs {
   const char *key;

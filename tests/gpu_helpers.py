@@ -72,6 +72,7 @@ class DeviceBatch:
         if out is None:
             out = torch.empty(q.shape, dtype=TORCH_DTYPE[out_dtype], device=q.device)
         if num_workers is None and not flags and workspace is None:
+            # pa_decode: library-owned workspace, default kernel and worker count
             pa.pa_decode(out, q, self.key_cache, self.value_cache, self.block_tables,
                          self.context_lens, b.scale, b.block_size, b.num_kv_heads)
         else:

@@ -53,7 +53,8 @@ def llama_small(oracle):
 
 
 @pytest.mark.parametrize("workers,flags", [(None, 0), (1, 0), (7, 0), (33, 0), (512, 0),
-                                           (5000, 0), (7, 1), (512, 1), (None, 1)])
+                                           (5000, 0), (7, 1), (512, 1), (None, 1),
+                                           (None, 2), (1, 2), (33, 2), (512, 3)])
 def test_llama_small_workers(llama_small, workers, flags):
     b, ref, kc, vc = llama_small
     db = DeviceBatch(b)
@@ -124,6 +125,7 @@ def test_long_mixed_full_size(oracle):
     out = db.decode("f32")
     outb = db.decode("bf16")
     outs = db.decode("f32", flags=pa.PA_DECODE_SEPARATE_REDUCE)
+    outc = db.decode("f32", flags=pa.PA_DECODE_CUDA_CORES)
     torch.cuda.synchronize()
     lens = b.context_lens
     longest = list(np.argsort(lens)[-4:])
@@ -134,6 +136,7 @@ def test_long_mixed_full_size(oracle):
     _check_caches(db, kc, vc, "bf16")
     assert_close(to_host(out, "f32")[seqs], ref, "bf16", "long mixed (sampled)")
     assert_close(to_host(outs, "f32")[seqs], ref, "bf16", "long mixed separate reduce")
+    assert_close(to_host(outc, "f32")[seqs], ref, "bf16", "long mixed CUDA-core kernel")
     assert_bf16_output(to_host(outb, "bf16")[seqs], ref, "long mixed bf16 (sampled)")
     assert_no_device_error()
 
@@ -152,16 +155,17 @@ def test_placement_and_poison_invariance():
     """Same logical values: other permutation, zero instead of NaN in unread slots, garbage in
     unread block-table entries -> bit-identical output (the kernel walks logical order)."""
     base = dict(num_seqs=10, min_len=1, max_len=200)
-    ref = _gpu_out(W.llama3_8b_decode(**base), num_workers=97)
-    b = W.llama3_8b_decode(**base, fill="zero")
-    assert np.array_equal(_gpu_out(b, num_workers=97), ref)
-    b = W.llama3_8b_decode(**base)
-    b.block_tables = np.where(b.block_tables < 0, np.int32(2 ** 30), b.block_tables)
-    assert np.array_equal(_gpu_out(b, num_workers=97), ref)
-    b = W.build_batch("perm", W.llama3_8b_decode(**base).context_lens, num_heads=32,
-                      num_kv_heads=8, head_dim=128, block_size=16, dtype="bf16",
-                      seed=W.BASE_SEED + 2, perm_salt=5, max_blocks=13)
-    assert np.array_equal(_gpu_out(b, num_workers=97), ref)
+    for flags in (0, pa.PA_DECODE_CUDA_CORES):
+        ref = _gpu_out(W.llama3_8b_decode(**base), num_workers=97, flags=flags)
+        b = W.llama3_8b_decode(**base, fill="zero")
+        assert np.array_equal(_gpu_out(b, num_workers=97, flags=flags), ref)
+        b = W.llama3_8b_decode(**base)
+        b.block_tables = np.where(b.block_tables < 0, np.int32(2 ** 30), b.block_tables)
+        assert np.array_equal(_gpu_out(b, num_workers=97, flags=flags), ref)
+        b = W.build_batch("perm", W.llama3_8b_decode(**base).context_lens, num_heads=32,
+                          num_kv_heads=8, head_dim=128, block_size=16, dtype="bf16",
+                          seed=W.BASE_SEED + 2, perm_salt=5, max_blocks=13)
+        assert np.array_equal(_gpu_out(b, num_workers=97, flags=flags), ref)
     assert_no_device_error()
 
 
@@ -194,18 +198,21 @@ def test_configuration_coverage(oracle, dtype, D, bs, hq, hkv):
     b = W.build_batch("cov", lens, num_heads=hq, num_kv_heads=hkv, head_dim=D, block_size=bs,
                       dtype=dtype, seed=W.BASE_SEED + 900 + D + bs)
     ref, kc, vc = oracle_step(oracle, b)
-    for workers in (None, 5):
+    variants = [(None, 0), (5, 0)] + ([(None, pa.PA_DECODE_CUDA_CORES), (5, pa.PA_DECODE_CUDA_CORES)]
+                                      if dtype != "f32" else [])
+    for workers, flags in variants:
         db = DeviceBatch(b)
         db.write()
         _check_caches(db, kc, vc, dtype)
-        assert_close(to_host(db.decode("f32", num_workers=workers), "f32"), ref, dtype,
-                     f"{dtype} D{D} bs{bs} G{hq // hkv}")
+        what = f"{dtype} D{D} bs{bs} G{hq // hkv} W={workers} flags={flags}"
+        assert_close(to_host(db.decode("f32", num_workers=workers, flags=flags), "f32"), ref,
+                     dtype, what)
         if dtype != "f32":
-            got = to_host(db.decode(dtype, num_workers=workers), dtype)
+            got = to_host(db.decode(dtype, num_workers=workers, flags=flags), dtype)
             if dtype == "bf16":
-                assert_bf16_output(got, ref, "bf16 out")
+                assert_bf16_output(got, ref, "bf16 out " + what)
             else:
-                assert_close(got.astype(np.float64), ref, dtype, "fp16 out")
+                assert_close(got.astype(np.float64), ref, dtype, "fp16 out " + what)
     assert_no_device_error()
 
 
@@ -215,9 +222,10 @@ def test_empty_and_extreme_contexts(oracle):
                       dtype="bf16", seed=W.BASE_SEED + 950, max_blocks=13)
     ref, _, _ = oracle_step(oracle, b)
     for workers in (None, 1, 4, 50):
-        got = _gpu_out(b, num_workers=workers)
-        assert np.all(got[[0, 2, 5]] == 0)
-        assert_close(got, ref, "bf16", f"edge W={workers}")
+        for flags in (0, pa.PA_DECODE_CUDA_CORES):
+            got = _gpu_out(b, num_workers=workers, flags=flags)
+            assert np.all(got[[0, 2, 5]] == 0)
+            assert_close(got, ref, "bf16", f"edge W={workers} flags={flags}")
     b0 = W.build_batch("allzero", [0, 0, 0], num_heads=8, num_kv_heads=2, head_dim=64,
                        block_size=8, dtype="bf16", seed=1, max_blocks=2)
     assert np.all(_gpu_out(b0) == 0)
@@ -229,7 +237,7 @@ def test_single_very_long_sequence(oracle):
     b = W.build_batch("long1", [32768], num_heads=32, num_kv_heads=8, head_dim=128,
                       block_size=16, dtype="bf16", seed=W.BASE_SEED + 960)
     ref, _, _ = oracle_step(oracle, b)
-    for flags in (0, pa.PA_DECODE_SEPARATE_REDUCE):
+    for flags in (0, pa.PA_DECODE_SEPARATE_REDUCE, pa.PA_DECODE_CUDA_CORES):
         assert_close(_gpu_out(b, flags=flags), ref, "bf16", f"32k tokens flags={flags}")
     assert_no_device_error()
 
@@ -242,11 +250,12 @@ def test_strided_query_and_out(oracle):
     big = torch.zeros((5, 32, 256), dtype=torch.bfloat16, device="cuda")
     big[:, :, 64:192] = db.query
     q = big[:, :, 64:192]                          # heads not contiguous: one copy per head
-    outbig = torch.zeros((5, 40, 128), dtype=torch.float32, device="cuda")
-    out = outbig[:, 4:36, :]
-    db.decode("f32", query=q, out=out)
-    assert_close(to_host(out, "f32"), ref, "bf16", "strided")
-    assert torch.all(outbig[:, :4] == 0) and torch.all(outbig[:, 36:] == 0)
+    for flags in (0, pa.PA_DECODE_CUDA_CORES):
+        outbig = torch.zeros((5, 40, 128), dtype=torch.float32, device="cuda")
+        out = outbig[:, 4:36, :]
+        db.decode("f32", query=q, out=out, flags=flags)
+        assert_close(to_host(out, "f32"), ref, "bf16", f"strided flags={flags}")
+        assert torch.all(outbig[:, :4] == 0) and torch.all(outbig[:, 36:] == 0)
     assert_no_device_error()
 
 
