@@ -74,6 +74,25 @@ struct DeviceState {
 
 std::mutex g_mu;
 std::vector<DeviceState> g_devices;
+
+// Merge counters sit at the start of a decode workspace, one per (sequence, kv head), and every
+// completed call leaves them zero.  The regions after them move with the number of sequences,
+// so a call with fewer sequences may write partial results where a later, larger call keeps
+// counters.  For each workspace the library remembers how many leading bytes are known to hold
+// zero counters and zeroes the rest (on the call's stream) before a call that needs more.
+struct CleanRecord {
+  const void *ws;
+  size_t clean;
+};
+std::vector<CleanRecord> g_clean;  // guarded by g_mu
+
+CleanRecord &clean_record(const void *ws) {
+  for (auto &r : g_clean)
+    if (r.ws == ws) return r;
+  if (g_clean.size() >= 64) g_clean.erase(g_clean.begin());
+  g_clean.push_back(CleanRecord{ws, 0});
+  return g_clean.back();
+}
 MemGetAddressRangeFn g_mem_range = nullptr;
 EncodeTiledFn g_encode_tiled = nullptr;
 bool g_mem_range_tried = false;
@@ -421,6 +440,7 @@ int decode_impl(const pa_tensor *out, const pa_tensor *query, const pa_tensor *k
         e = cudaDeviceSynchronize();
         if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceSynchronize (workspace growth)");
         cudaFree(ds->ws);
+        clean_record(ds->ws).clean = 0;
         ds->ws = nullptr;
         ds->ws_bytes = 0;
       }
@@ -430,6 +450,7 @@ int decode_impl(const pa_tensor *out, const pa_tensor *query, const pa_tensor *k
       e = cudaMemsetAsync(ds->ws, 0, want, st);
       if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(decode workspace)");
       ds->ws_bytes = want;
+      clean_record(ds->ws).clean = want;
     }
     workspace = ds->ws;
     workspace_bytes = ds->ws_bytes;
@@ -437,6 +458,17 @@ int decode_impl(const pa_tensor *out, const pa_tensor *query, const pa_tensor *k
     if (!workspace || workspace_bytes < L.total)
       return fail(PA_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", L.total, workspace_bytes);
     if (((uintptr_t)workspace & 255u) != 0) return fail(PA_ERR_WORKSPACE, "workspace must be 256-byte aligned");
+  }
+  {
+    const size_t counter_bytes = (size_t)S * (size_t)num_kv_heads * 4;
+    std::lock_guard<std::mutex> lock(g_mu);
+    CleanRecord &rec = clean_record(workspace);
+    if (rec.clean < counter_bytes) {
+      cudaError_t e = cudaMemsetAsync(static_cast<char *>(workspace) + rec.clean, 0,
+                                      counter_bytes - rec.clean, st);
+      if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(merge counters)");
+    }
+    rec.clean = counter_bytes;
   }
 
   pa::DecodeArgs a;
@@ -619,7 +651,10 @@ int pa_workspace_init(void *workspace, size_t workspace_bytes, void *stream) {
   if (!workspace && workspace_bytes) return fail(PA_ERR_INVALID_ARG, "NULL workspace");
   if (!workspace_bytes) return PA_OK;
   cudaError_t e = cudaMemsetAsync(workspace, 0, workspace_bytes, static_cast<cudaStream_t>(stream));
-  return e == cudaSuccess ? PA_OK : cuda_fail(e, "cudaMemsetAsync(workspace)");
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(workspace)");
+  std::lock_guard<std::mutex> lock(g_mu);
+  clean_record(workspace).clean = workspace_bytes;
+  return PA_OK;
 }
 
 int pa_release_workspaces(void) {
@@ -631,6 +666,8 @@ int pa_release_workspaces(void) {
     cudaSetDevice((int)d);
     cudaDeviceSynchronize();
     cudaFree(g_devices[d].ws);
+    for (auto &r : g_clean)
+      if (r.ws == g_devices[d].ws) r.clean = 0;
     g_devices[d].ws = nullptr;
     g_devices[d].ws_bytes = 0;
   }

@@ -156,6 +156,7 @@ __global__ void __launch_bounds__(128, 1) paged_decode_kernel(const DecodeArgs a
   float2 acc[G][EPL / 2];
   float m_ref = -INFINITY;
   float lsum = 0.f;
+  bool piece_at_start = false;  // this piece begins at chunk 0 of its (sequence, kv head)
 
   for (long long c = 0; c < n; ++c) {
     const int slot = (int)(c % ST);
@@ -182,6 +183,7 @@ __global__ void __launch_bounds__(128, 1) paged_decode_kernel(const DecodeArgs a
       }
       m_ref = -INFINITY;
       lsum = 0.f;
+      piece_at_start = (m.flags & kPairStart) != 0;
     }
 
     // ---- logits: one (row, head) per lane after the reduce ----
@@ -300,7 +302,7 @@ __global__ void __launch_bounds__(128, 1) paged_decode_kernel(const DecodeArgs a
         lh[h] = __shfl_sync(FULL_MASK, lt, h * HL);
         mh[h] = __shfl_sync(FULL_MASK, m_ref, h * HL);
       }
-      if (a.separate_reduce && (m.flags & kPairStart) && lane == 0)
+      if (a.separate_reduce && piece_at_start && lane == 0)
         a.pair_meta[m.pair] = make_int2(m.first_worker, m.npieces);
       if (m.npieces == 1) {
         if (r == 0) {

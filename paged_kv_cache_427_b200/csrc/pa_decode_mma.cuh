@@ -200,6 +200,7 @@ __global__ void __launch_bounds__(128, 2)
   uint32_t qb[Tr::kKSteps][2];
   float o[Tr::kMTiles][4];
   float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
+  bool piece_at_start = false;  // this piece begins at chunk 0 of its (sequence, kv head)
 
   for (long long cc = 0; cc < n; ++cc) {
     const int slot = (int)(cc % ST);
@@ -230,6 +231,7 @@ __global__ void __launch_bounds__(128, 2)
       for (int mt = 0; mt < Tr::kMTiles; ++mt) o[mt][0] = o[mt][1] = o[mt][2] = o[mt][3] = 0.f;
       m0 = m1 = -INFINITY;
       l0 = l1 = 0.f;
+      piece_at_start = (m.flags & kPairStart) != 0;
     }
 
     // ---- q.K on tensor cores: s = S[token g | g+8][head 2c | 2c+1] ----
@@ -336,7 +338,7 @@ __global__ void __launch_bounds__(128, 2)
         t1 += __shfl_xor_sync(FULL_MASK, t1, off);
       }
       const float inv0 = 1.f / t0, inv1 = 1.f / t1;
-      if (a.separate_reduce && (m.flags & kPairStart) && lane == 0)
+      if (a.separate_reduce && piece_at_start && lane == 0)
         a.pair_meta[m.pair] = make_int2(m.first_worker, m.npieces);
       if (m.npieces == 1) {
         const int out_elt = a.out_dtype == PA_F32 ? 4 : 2;

@@ -282,7 +282,7 @@ def test_copy_blocks_bit_exact_and_bad_pairs(oracle):
     rng = np.random.default_rng(11)
     b.key_cache = W.encode(rng.standard_normal(b.key_cache.shape, dtype=np.float32), "bf16")
     b.value_cache = W.encode(rng.standard_normal(b.value_cache.shape, dtype=np.float32), "bf16")
-    pairs = np.array([[3, 100], [7, 5], [3, 9]], np.int64)
+    pairs = np.array([[3, 60], [7, 5], [3, 9]], np.int64)
     db = DeviceBatch(b)
     pa.pa_copy_blocks(db.key_cache, db.value_cache, torch.from_numpy(pairs).cuda())
     kc, vc = b.key_cache.copy(), b.value_cache.copy()
@@ -311,7 +311,8 @@ def test_bad_block_ids_and_lengths_are_flagged():
     b.slot_mapping[[1, 3]] = -1
     out = _gpu_out(b)
     assert np.all(out[3] == 0)
-    assert pa.pa_get_device_error(clear=True) == pa.PA_DEVERR_CONTEXT_LEN
+    # the clamped context of sequence 1 also reaches block-table entries past its blocks
+    assert pa.pa_get_device_error(clear=True) & pa.PA_DEVERR_CONTEXT_LEN
 
 
 def test_decode_and_decode_ex_agree():
