@@ -207,6 +207,33 @@ PA_API const char *pa_last_error(void);
  */
 PA_API int pa_get_device_error(void *stream, uint32_t *flags, int32_t clear);
 
+/*
+ * pa_decode_noalloc - pa_decode for callers that cannot allocate device memory.
+ *
+ * The vLLM tutorials have no counterpart to this call; it exists for users of this library.
+ * Some callers may not call cudaMalloc: code that runs while a stream is being captured into a
+ * CUDA graph, engines that reserve all device memory up front for their own pool and forbid
+ * later allocations, and latency-critical loops that cannot afford the implicit device
+ * synchronisation an allocation or a free may cause.  pa_decode allocates its workspace on
+ * first use and pa_decode_ex needs one from the caller; this call needs neither.
+ *
+ * Same arguments, semantics and tolerances as pa_decode.  Its scratch (merge counters and
+ * partial results) is a fixed device array of PA_NOALLOC_SCRATCH_BYTES inside the library,
+ * which every GPU that loads the library holds until the process exits.  A call whose shapes
+ * need more scratch than that (roughly: more than about 3,000 (sequence, kv head) pairs at
+ * head_dim 128 and 4 query heads per kv head) returns PA_ERR_WORKSPACE without launching.
+ * The first call on a device looks up the array's device address and clears it on `stream`;
+ * make that first call before any stream capture.  The call itself allocates nothing: no
+ * cudaMalloc, no cudaFree, no allocating library routine.  All calls share the one array, so
+ * calls that overlap on the GPU (for instance on two streams) race and give wrong results;
+ * issue them in one stream or one after another.
+ */
+#define PA_NOALLOC_SCRATCH_BYTES (8u * 1024u * 1024u)
+PA_API int pa_decode_noalloc(const pa_tensor *out, const pa_tensor *query,
+                             const pa_tensor *key_cache, const pa_tensor *value_cache,
+                             const pa_tensor *block_tables, const pa_tensor *context_lens,
+                             float scale, int32_t block_size, int32_t num_kv_heads, void *stream);
+
 /* PA_VERSION of the library actually loaded. */
 PA_API int32_t pa_version(void);
 

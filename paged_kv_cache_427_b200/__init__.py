@@ -34,6 +34,8 @@ PA_DEVERR_CONTEXT_LEN = 0x2
 PA_DEVERR_SLOT = 0x4
 PA_DEVERR_COPY_PAIR = 0x8
 PA_DEVERR_TIMEOUT = 0x10
+PA_NOALLOC_SCRATCH_BYTES = 8 * 1024 * 1024
+PA_ERR_WORKSPACE = -6
 STATUS_NAMES = {0: "PA_OK", -1: "PA_ERR_INVALID_ARG", -2: "PA_ERR_SHAPE", -3: "PA_ERR_DTYPE",
                 -4: "PA_ERR_UNSUPPORTED", -5: "PA_ERR_CUDA", -6: "PA_ERR_WORKSPACE",
                 -7: "PA_ERR_LAYOUT"}
@@ -77,9 +79,11 @@ def load(path: str = LIBRARY) -> ctypes.CDLL:
     lib.pa_last_error.argtypes = []
     lib.pa_last_error.restype = ctypes.c_char_p
     lib.pa_get_device_error.argtypes = [_P, ctypes.POINTER(u32), i32]
+    lib.pa_decode_noalloc.argtypes = [_T, _T, _T, _T, _T, _T, f32, i32, i32, _P]
     lib.pa_version.argtypes = []
     lib.pa_version.restype = i32
     for name in ("pa_reshape_and_cache", "pa_copy_blocks", "pa_decode", "pa_decode_ex",
+                 "pa_decode_noalloc",
                  "pa_workspace_init", "pa_release_workspaces", "pa_get_device_error"):
         getattr(lib, name).restype = ctypes.c_int
     _lib = lib
@@ -159,6 +163,18 @@ def pa_decode_ex(out, query, key_cache, value_cache, block_tables, context_lens,
     _check("pa_decode_ex", lib.pa_decode_ex(*[ctypes.byref(x) for x in d], float(scale),
                                             int(block_size), int(num_kv_heads), int(num_workers),
                                             int(flags), ws_ptr, ws_bytes, _stream(stream)))
+
+
+def pa_decode_noalloc(out, query, key_cache, value_cache, block_tables, context_lens, scale,
+                      block_size, num_kv_heads, stream=None):
+    """pa_decode for callers that cannot allocate device memory: the scratch is a fixed
+    8 MiB device array inside the library (see include/pa.h); shapes that need more are
+    refused with PA_ERR_WORKSPACE; calls overlapping on the GPU race on that array."""
+    lib = load()
+    d = [describe(x) for x in (out, query, key_cache, value_cache, block_tables, context_lens)]
+    _check("pa_decode_noalloc", lib.pa_decode_noalloc(*[ctypes.byref(x) for x in d], float(scale),
+                                                      int(block_size), int(num_kv_heads),
+                                                      _stream(stream)))
 
 
 def pa_decode_workspace_bytes(num_seqs, num_heads, num_kv_heads, head_dim, num_workers=0) -> int:

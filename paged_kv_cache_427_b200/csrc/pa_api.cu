@@ -514,6 +514,36 @@ int decode_impl(const pa_tensor *out, const pa_tensor *query, const pa_tensor *k
 
 }  // namespace
 
+namespace pa {
+
+// Helpers for the allocation-free entry point (pa_noalloc.cu).
+void set_last_error(const char *msg) { g_last_error = msg; }
+
+size_t decode_scratch_need(const pa_tensor *query, const pa_tensor *key_cache, int32_t block_size,
+                           int32_t num_kv_heads) {
+  if (!query || !key_cache || query->ndim != 3 || key_cache->ndim != 4 || num_kv_heads <= 0 ||
+      query->shape[1] % num_kv_heads != 0)
+    return 0;
+  DeviceState *ds;
+  if (device_state(&ds, nullptr) != PA_OK) return 0;
+  DecodeKernel k;
+  const int D = (int)key_cache->shape[3];
+  const int G = (int)(query->shape[1] / num_kv_heads);
+  if (!get_kernel(key_cache->dtype, D, block_size, G, key_cache->dtype != PA_F32, &k)) return 0;
+  return ws_layout(query->shape[0], (int)query->shape[1], num_kv_heads, D,
+                   default_workers(k, ds->num_sms)).total;
+}
+
+int decode_into(const pa_tensor *out, const pa_tensor *query, const pa_tensor *key_cache,
+                const pa_tensor *value_cache, const pa_tensor *block_tables,
+                const pa_tensor *context_lens, float scale, int32_t block_size,
+                int32_t num_kv_heads, void *workspace, size_t workspace_bytes, void *stream) {
+  return decode_impl(out, query, key_cache, value_cache, block_tables, context_lens, scale,
+                     block_size, num_kv_heads, 0, 0u, workspace, workspace_bytes, false, stream);
+}
+
+}  // namespace pa
+
 extern "C" {
 
 int pa_reshape_and_cache(const pa_tensor *key, const pa_tensor *value, const pa_tensor *key_cache,

@@ -5,6 +5,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "pa.h"
+
 namespace pa {
 
 // Everything a decode launch needs, already validated.  Strides are in elements.
@@ -90,6 +92,17 @@ struct CopyBlocksArgs {
 };
 
 cudaError_t launch_reshape_and_cache(const CacheWriteArgs &a, int num_sms, cudaStream_t st);
+
+// For the allocation-free entry point: the scratch bytes a pa_decode call with these shapes
+// needs (0 when the arguments are invalid), decode into a given scratch buffer, and set the
+// message pa_last_error() returns.
+size_t decode_scratch_need(const pa_tensor *query, const pa_tensor *key_cache, int32_t block_size,
+                           int32_t num_kv_heads);
+int decode_into(const pa_tensor *out, const pa_tensor *query, const pa_tensor *key_cache,
+                const pa_tensor *value_cache, const pa_tensor *block_tables,
+                const pa_tensor *context_lens, float scale, int32_t block_size,
+                int32_t num_kv_heads, void *workspace, size_t workspace_bytes, void *stream);
+void set_last_error(const char *msg);
 cudaError_t launch_copy_blocks(const CopyBlocksArgs &a, int num_sms, cudaStream_t st);
 
 }  // namespace pa
