@@ -456,8 +456,9 @@ def main():
     ap.add_argument("--workload", default="llama3_8b_decode",
                     help="llama3_8b_decode | short_chat_bs{8,16,32} | shared_prefix | long_mixed | tiny_fp32")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--decode-flags", type=int, default=0,
-                    help="pa_decode_ex flags (2 = CUDA-core kernel, 1 = separate merge kernel)")
+    ap.add_argument("--decode-flags", type=int, default=4,
+                    help="pa_decode_ex flags: 4 = start while the cache write runs (default), "
+                         "2 = CUDA-core kernel, 1 = separate merge kernel, 0 = plain pa_decode")
     ap.add_argument("--rotations", type=int, default=0, help="copies of the KV pool (0 = enough to defeat L2)")
     ap.add_argument("--soak", type=float, default=1.0, help="seconds of untimed load for the clock sampler")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)

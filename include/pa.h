@@ -112,6 +112,14 @@ typedef enum pa_status {
 #define PA_DECODE_CUDA_CORES 0x2u      /* 16-bit caches: use the CUDA-core kernel instead of the
                                           tensor-core (mma.sync + TMA) one; fp32 caches always
                                           use the CUDA-core kernel */
+#define PA_DECODE_OVERLAP_PREVIOUS 0x4u /* let the decode kernel start while the kernel launched
+                                          just before it on `stream` is still running
+                                          (programmatic dependent launch): it reads context_lens
+                                          and block_tables and zeroes the out rows of empty
+                                          contexts before it waits for that kernel, and reads
+                                          the caches and the query only after.  Use it only when
+                                          that kernel writes none of context_lens, block_tables
+                                          and out, e.g. right after pa_reshape_and_cache */
 
 /*
  * pa_reshape_and_cache - store this step's new keys and values into their cache slots.

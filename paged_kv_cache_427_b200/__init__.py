@@ -29,6 +29,7 @@ PA_F32, PA_BF16, PA_F16, PA_I32, PA_I64 = 0, 1, 2, 3, 4
 PA_OK = 0
 PA_DECODE_SEPARATE_REDUCE = 0x1
 PA_DECODE_CUDA_CORES = 0x2
+PA_DECODE_OVERLAP_PREVIOUS = 0x4
 PA_DEVERR_BLOCK_ID = 0x1
 PA_DEVERR_CONTEXT_LEN = 0x2
 PA_DEVERR_SLOT = 0x4

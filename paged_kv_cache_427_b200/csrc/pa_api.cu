@@ -368,7 +368,7 @@ int decode_impl(const pa_tensor *out, const pa_tensor *query, const pa_tensor *k
       (rc = check_tensor(block_tables, "block_tables", 2)) ||
       (rc = check_tensor(context_lens, "context_lens", 1)))
     return rc;
-  if (flags & ~(PA_DECODE_SEPARATE_REDUCE | PA_DECODE_CUDA_CORES))
+  if (flags & ~(PA_DECODE_SEPARATE_REDUCE | PA_DECODE_CUDA_CORES | PA_DECODE_OVERLAP_PREVIOUS))
     return fail(PA_ERR_INVALID_ARG, "unknown flags 0x%x", flags);
   if (num_workers < 0) return fail(PA_ERR_INVALID_ARG, "num_workers must be >= 0");
   if (block_size != cs.block_size)
@@ -503,7 +503,7 @@ int decode_impl(const pa_tensor *out, const pa_tensor *query, const pa_tensor *k
   a.wait_cycles = test_hooks().wait_cycles;
   a.test_stall = test_hooks().stall;
   const int ctas = (W + k.warps_per_cta - 1) / k.warps_per_cta;
-  cudaError_t e = k.launch(a, &maps, ctas, st);
+  cudaError_t e = k.launch(a, &maps, ctas, (flags & PA_DECODE_OVERLAP_PREVIOUS) != 0, st);
   if (e != cudaSuccess) return cuda_fail(e, "decode launch");
   if (a.separate_reduce) {
     e = k.launch_reduce(a, st);

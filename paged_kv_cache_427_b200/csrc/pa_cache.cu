@@ -17,6 +17,9 @@ namespace pa {
 
 // One thread per 16-byte piece of one (token, kv head) row, keys and values together.
 __global__ void __launch_bounds__(256) reshape_and_cache_kernel(CacheWriteArgs a) {
+  // A decode launched to overlap this grid may start now; it waits for this grid's writes
+  // before it reads the caches.
+  allow_next_grid();
   const int vec_per_row = a.row_bytes >> 4;
   const int64_t total = a.num_tokens * a.num_kv_heads * vec_per_row;
   for (int64_t idx = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; idx < total;

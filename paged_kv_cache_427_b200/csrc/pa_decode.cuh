@@ -146,6 +146,9 @@ __global__ void __launch_bounds__(128, 1) paged_decode_kernel(const DecodeArgs a
     cur.advance(a);
   };
 
+  // Everything above read only context_lens and block_tables; the caches and the query may
+  // still be written by the previous grid when this one was launched to overlap it.
+  wait_for_previous_grid();
   const long long prime = n < ST ? n : ST;
   for (long long i = 0; i < prime; ++i) issue((int)i);
 
@@ -350,11 +353,29 @@ __global__ void __launch_bounds__(128, 1) paged_decode_kernel(const DecodeArgs a
   }
 }
 
+// Launch with or without programmatic dependent launch on the previous grid of the stream.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_overlapping(void (*kernel)(KArgs...), int ctas, int threads, int smem,
+                               bool overlap_previous, cudaStream_t st, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(ctas);
+  cfg.blockDim = dim3(threads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = overlap_previous ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
 template <typename T, int D, int BS, int G>
-cudaError_t launch_decode_simt(const DecodeArgs &a, const TmaMaps *, int num_ctas, cudaStream_t st) {
+cudaError_t launch_decode_simt(const DecodeArgs &a, const TmaMaps *, int num_ctas,
+                               bool overlap_previous, cudaStream_t st) {
   using Tr = SimtTraits<T, D, BS, G>;
-  paged_decode_kernel<T, D, BS, G><<<num_ctas, Tr::kWarps * 32, Tr::kSmemBytes, st>>>(a);
-  return cudaGetLastError();
+  return launch_overlapping(paged_decode_kernel<T, D, BS, G>, num_ctas, Tr::kWarps * 32,
+                            Tr::kSmemBytes, overlap_previous, st, a);
 }
 
 template <typename T, int D, int BS, int G>

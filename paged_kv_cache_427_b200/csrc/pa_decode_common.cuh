@@ -57,18 +57,21 @@ struct WarpShare {
 template <int CH, int kWarps, int G, int D>
 __device__ bool split_prologue(const DecodeArgs &a, unsigned char *scratch, int max_len,
                                WarpShare &ws) {
+  constexpr int kTile = 8 * 32 * kWarps;  // sequences per scan tile, 8 per thread
   const int lane = threadIdx.x & 31;
   const int wid = threadIdx.x >> 5;
   const int S = a.num_seqs;
   const int Hkv = a.num_kv_heads;
   long long *red = reinterpret_cast<long long *>(scratch);  // [kWarps]
   int4 *loc = reinterpret_cast<int4 *>(scratch + 64);       // [kWarps]
-  long long local = 0;
-  for (int s = threadIdx.x; s < S; s += blockDim.x) {
+  if (threadIdx.x < kWarps) loc[threadIdx.x] = make_int4(-1, 0, 0, 0);
+
+  // Clamped length of sequence s (s < S); flags a bad length (CTA 0 only) and writes the zero
+  // rows of an empty context (one CTA per sequence).  Idempotent, so a tile may see it twice.
+  auto seq_len = [&](int s) -> int {
     const int raw = __ldg(a.context_lens + s);
     const int len = clamp_len(raw, max_len);
     if (raw != len && blockIdx.x == 0) set_error(a.err, PA_DEVERR_CONTEXT_LEN);
-    local += (len + CH - 1) / CH;
     if (len == 0 && (s % gridDim.x) == blockIdx.x) {
       const int out_elt = a.out_dtype == PA_F32 ? 4 : 2;
       const float z[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
@@ -78,17 +81,61 @@ __device__ bool split_prologue(const DecodeArgs &a, unsigned char *scratch, int 
                               ((long long)s * a.out_s + (long long)h * a.out_h + d) * out_elt,
                           a.out_dtype, z, 8);
     }
+    return len;
+  };
+
+  // Load one tile of sequences: this thread's chunk counts and the tile-wide exclusive prefix
+  // of its first count.
+  long long cnt[8];
+  int lens8[8];
+  auto load_tile = [&](int base, long long &tile_total) -> long long {
+    long long tsum = 0;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const int s = base + threadIdx.x * 8 + k;
+      lens8[k] = s < S ? seq_len(s) : 0;
+      cnt[k] = (long long)((lens8[k] + CH - 1) / CH) * Hkv;
+      tsum += cnt[k];
+    }
+    long long x = tsum;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const long long y = __shfl_up_sync(FULL_MASK, x, off);
+      if (lane >= off) x += y;
+    }
+    __syncthreads();  // red[] free
+    if (lane == 31) red[wid] = x;
+    __syncthreads();
+    long long ex = 0;
+    tile_total = 0;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) {
+      if (w < wid) ex += red[w];
+      tile_total += red[w];
+    }
+    return ex + x - tsum;
+  };
+
+  long long tile_total = 0;
+  long long ex0 = load_tile(0, tile_total);
+  long long C = tile_total;
+  if (S > kTile) {
+    // more than one tile: count the rest first (the first tile stays in registers for S <= kTile)
+    for (int base = kTile; base < S; base += kTile) {
+      long long t = 0;
+      long long local = 0;
+      for (int s = base + threadIdx.x; s < base + kTile && s < S; s += blockDim.x)
+        local += (long long)((seq_len(s) + CH - 1) / CH) * Hkv;
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) local += __shfl_xor_sync(FULL_MASK, local, off);
+      __syncthreads();
+      if (lane == 0) red[wid] = local;
+      __syncthreads();
+#pragma unroll
+      for (int w = 0; w < kWarps; ++w) t += red[w];
+      C += t;
+    }
   }
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) local += __shfl_xor_sync(FULL_MASK, local, off);
-  if (lane == 0) red[wid] = local;
-  if (threadIdx.x < kWarps) loc[threadIdx.x] = make_int4(-1, 0, 0, 0);
-  __syncthreads();
-  long long C = 0;
-#pragma unroll
-  for (int w = 0; w < kWarps; ++w) C += red[w];
-  C *= Hkv;
-  __syncthreads();
   const int W = (int)(C < (long long)a.num_workers ? C : (long long)a.num_workers);
   ws.C = C;
   ws.W = W;
@@ -105,33 +152,12 @@ __device__ bool split_prologue(const DecodeArgs &a, unsigned char *scratch, int 
     if (my_g0[w] < g1) last_needed = my_g0[w];
   }
   long long running = 0;
-  for (int base = 0; base < S && running <= last_needed; base += 8 * 32 * kWarps) {
-    long long cnt[8];
-    long long tsum = 0;
-    int lens8[8];
-#pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      const int s = base + threadIdx.x * 8 + k;
-      lens8[k] = s < S ? clamp_len(__ldg(a.context_lens + s), max_len) : 0;
-      cnt[k] = (long long)((lens8[k] + CH - 1) / CH) * Hkv;
-      tsum += cnt[k];
+  for (int base = 0; base < S && running <= last_needed; base += kTile) {
+    long long ex = ex0;
+    if (base > 0) {
+      ex = load_tile(base, tile_total);
     }
-    long long x = tsum;
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-      const long long y = __shfl_up_sync(FULL_MASK, x, off);
-      if (lane >= off) x += y;
-    }
-    if (lane == 31) red[wid] = x;
-    __syncthreads();
-    long long ex = running;
-    long long tile_total = 0;
-#pragma unroll
-    for (int w = 0; w < kWarps; ++w) {
-      if (w < wid) ex += red[w];
-      tile_total += red[w];
-    }
-    ex += x - tsum;
+    ex += running;
 #pragma unroll
     for (int k = 0; k < 8; ++k) {
 #pragma unroll
@@ -141,8 +167,8 @@ __device__ bool split_prologue(const DecodeArgs &a, unsigned char *scratch, int 
       ex += cnt[k];
     }
     running += tile_total;
-    __syncthreads();
   }
+  __syncthreads();
 
   const int gw = blockIdx.x * kWarps + wid;
   if (gw >= W) return false;

@@ -31,8 +31,7 @@ template <>
 struct MmaType<__nv_bfloat16> {
   static __device__ __forceinline__ void mma(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
                                              uint32_t b1) {
-    asm volatile(
-        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
         "{%8,%9}, {%0,%1,%2,%3};"
         : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
@@ -50,8 +49,7 @@ template <>
 struct MmaType<__half> {
   static __device__ __forceinline__ void mma(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
                                              uint32_t b1) {
-    asm volatile(
-        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
         "{%8,%9}, {%0,%1,%2,%3};"
         : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
@@ -188,6 +186,9 @@ __global__ void __launch_bounds__(128, 2)
     cur.advance(a);
   };
 
+  // Everything above read only context_lens and block_tables; the caches and the query may
+  // still be written by the previous grid when this one was launched to overlap it.
+  wait_for_previous_grid();
   const long long prime = n < ST ? n : ST;
   for (long long i = 0; i < prime; ++i) issue((int)i);
 
@@ -235,8 +236,10 @@ __global__ void __launch_bounds__(128, 2)
     }
 
     // ---- q.K on tensor cores: s = S[token g | g+8][head 2c | 2c+1] ----
-    float s[4] = {0.f, 0.f, 0.f, 0.f};
+    float s[4];
     {
+      // two accumulators (even / odd k-steps) halve the chain of dependent mma
+      float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f};
       const int row = ((lm & 1) << 3) | lr;
 #pragma unroll
       for (int ks = 0; ks < Tr::kKSteps; ++ks) {
@@ -244,11 +247,14 @@ __global__ void __launch_bounds__(128, 2)
         const uint32_t addr = kbase + (ks >> 2) * 2048 + row * 128 + ((c16 ^ lr) << 4);
         uint32_t af[4];
         ldmatrix_x4(af, addr);
-        M::mma(s, af, qb[ks][0], qb[ks][1]);
+        if (ks & 1)
+          M::mma(sb, af, qb[ks][0], qb[ks][1]);
+        else
+          M::mma(sa, af, qb[ks][0], qb[ks][1]);
       }
-    }
 #pragma unroll
-    for (int e = 0; e < 4; ++e) s[e] *= a.scale_log2;
+      for (int e = 0; e < 4; ++e) s[e] = (sa[e] + sb[e]) * a.scale_log2;
+    }
     const int tok0 = m.chunk * 16;
     const bool tail = tok0 + 16 > m.len;
     if (tail) {
@@ -256,14 +262,15 @@ __global__ void __launch_bounds__(128, 2)
       if (tok0 + g + 8 >= m.len) s[2] = s[3] = -INFINITY;
     }
 
-    // ---- online softmax ----
+    // ---- online softmax: the reference maximum moves only when some logit passes it by
+    // more than 8 (base 2); only then are the chunk maxima gathered across lanes ----
     float cm0 = fmaxf(s[0], s[2]), cm1 = fmaxf(s[1], s[3]);
-#pragma unroll
-    for (int off = 4; off < 32; off <<= 1) {
-      cm0 = fmaxf(cm0, __shfl_xor_sync(FULL_MASK, cm0, off));
-      cm1 = fmaxf(cm1, __shfl_xor_sync(FULL_MASK, cm1, off));
-    }
     if (__any_sync(FULL_MASK, (cm0 > m0 + 8.f) || (cm1 > m1 + 8.f))) {
+#pragma unroll
+      for (int off = 4; off < 32; off <<= 1) {
+        cm0 = fmaxf(cm0, __shfl_xor_sync(FULL_MASK, cm0, off));
+        cm1 = fmaxf(cm1, __shfl_xor_sync(FULL_MASK, cm1, off));
+      }
       const float n0 = fmaxf(m0, cm0), n1 = fmaxf(m1, cm1);
       const float a0 = fast_exp2(m0 - n0), a1 = fast_exp2(m1 - n1);
       m0 = n0;
@@ -407,10 +414,10 @@ __global__ void __launch_bounds__(128, 2)
 
 template <typename T, int D, int BS, int G>
 cudaError_t launch_decode_mma(const DecodeArgs &a, const TmaMaps *maps, int num_ctas,
-                              cudaStream_t st) {
+                              bool overlap_previous, cudaStream_t st) {
   using Tr = MmaTraits<D, BS, G>;
-  paged_decode_mma_kernel<T, D, BS, G><<<num_ctas, Tr::kWarps * 32, Tr::kSmemBytes, st>>>(a, *maps);
-  return cudaGetLastError();
+  return launch_overlapping(paged_decode_mma_kernel<T, D, BS, G>, num_ctas, Tr::kWarps * 32,
+                            Tr::kSmemBytes, overlap_previous, st, a, *maps);
 }
 
 template <typename T, int D, int BS, int G>

@@ -165,6 +165,14 @@ __device__ __forceinline__ float fast_exp2(float x) {
 // Packed fp32x2 FMA (sm_100): d = a * b + c on both halves.
 __device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
 
+// Programmatic dependent launch: wait until the grid this one depends on has completed and its
+// memory is visible (returns at once when the launch had no such dependency) ...
+__device__ __forceinline__ void wait_for_previous_grid() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+// ... and let the grid launched after this one start early.
+__device__ __forceinline__ void allow_next_grid() { asm volatile("griddepcontrol.launch_dependents;"); }
+
 __device__ __forceinline__ void set_error(unsigned int *err, unsigned int bits) {
   if (err) atomicOr(err, bits);
 }

@@ -48,7 +48,8 @@ struct TmaMaps {
 };
 
 struct DecodeKernel {
-  cudaError_t (*launch)(const DecodeArgs &, const TmaMaps *, int num_ctas, cudaStream_t);
+  cudaError_t (*launch)(const DecodeArgs &, const TmaMaps *, int num_ctas, bool overlap_previous,
+                        cudaStream_t);
   cudaError_t (*launch_reduce)(const DecodeArgs &, cudaStream_t);
   const void *kernel;  // for occupancy queries
   int warps_per_cta;
