@@ -280,8 +280,9 @@ struct MapEntry {
 std::vector<MapEntry> g_maps;
 uint64_t g_map_clock = 0;
 
-// The cache as a 4-D tensor (head_dim, block_size, kv heads, blocks) read in 128-byte swizzled
-// boxes of 64 elements x `rows` rows (one 128-byte column half of `rows` consecutive tokens).
+// The cache as a 5-D tensor (64 elements, block_size rows, head_dim / 64 column halves, kv heads,
+// blocks) read in 128-byte swizzled boxes of 64 x `rows` x head_dim/64: one box brings a whole
+// (rows x head_dim) tile, laid out in shared memory as [half][row][128 bytes].
 int cache_map(const pa_tensor *t, int rows, CUtensorMap *out) {
   MapKey key;
   key.ptr = t->data;
@@ -299,16 +300,17 @@ int cache_map(const pa_tensor *t, int rows, CUtensorMap *out) {
       return PA_OK;
     }
   if (!g_encode_tiled) return fail(PA_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
-  const cuuint64_t dims[4] = {(cuuint64_t)t->shape[3], (cuuint64_t)t->shape[2],
-                              (cuuint64_t)t->shape[1], (cuuint64_t)t->shape[0]};
-  const cuuint64_t strides[3] = {(cuuint64_t)t->stride[2] * 2, (cuuint64_t)t->stride[1] * 2,
+  const cuuint64_t halves = (cuuint64_t)t->shape[3] / 64;
+  const cuuint64_t dims[5] = {64, (cuuint64_t)t->shape[2], halves, (cuuint64_t)t->shape[1],
+                              (cuuint64_t)t->shape[0]};
+  const cuuint64_t strides[4] = {(cuuint64_t)t->stride[2] * 2, 128, (cuuint64_t)t->stride[1] * 2,
                                  (cuuint64_t)t->stride[0] * 2};
-  const cuuint32_t box[4] = {64, (cuuint32_t)rows, 1, 1};
-  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  const cuuint32_t box[5] = {64, (cuuint32_t)rows, (cuuint32_t)halves, 1, 1};
+  const cuuint32_t estr[5] = {1, 1, 1, 1, 1};
   CUtensorMap map;
   const CUresult r = g_encode_tiled(
       &map, t->dtype == PA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
-      4, t->data, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+      5, t->data, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
       CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
       CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(PA_ERR_LAYOUT, "cuTensorMapEncodeTiled failed (%d)", (int)r);
@@ -326,7 +328,7 @@ int cache_map(const pa_tensor *t, int rows, CUtensorMap *out) {
 // Warps of one full wave of the device for a kernel (CTAs per SM x SMs x warps per CTA).
 int default_workers(const pa::DecodeKernel &k, int num_sms) {
   int per_sm = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k.kernel, k.warps_per_cta * 32,
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k.kernel, k.threads_per_cta,
                                                     k.smem_bytes) != cudaSuccess ||
       per_sm < 1) {
     cudaGetLastError();
@@ -502,7 +504,7 @@ int decode_impl(const pa_tensor *out, const pa_tensor *query, const pa_tensor *k
   a.separate_reduce = (flags & PA_DECODE_SEPARATE_REDUCE) ? 1 : 0;
   a.wait_cycles = test_hooks().wait_cycles;
   a.test_stall = test_hooks().stall;
-  const int ctas = (W + k.warps_per_cta - 1) / k.warps_per_cta;
+  const int ctas = (W + k.warps_per_cta - 1) / k.warps_per_cta;  // warps_per_cta workers each
   cudaError_t e = k.launch(a, &maps, ctas, (flags & PA_DECODE_OVERLAP_PREVIOUS) != 0, st);
   if (e != cudaSuccess) return cuda_fail(e, "decode launch");
   if (a.separate_reduce) {

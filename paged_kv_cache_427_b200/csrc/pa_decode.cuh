@@ -85,7 +85,7 @@ __global__ void __launch_bounds__(128, 1) paged_decode_kernel(const DecodeArgs a
   const int max_len = a.max_blocks * BS;
 
   WarpShare share;
-  if (!split_prologue<CH, Tr::kWarps, G, D>(a, smem + Tr::kPrologueOff, max_len, share)) return;
+  if (!split_prologue<CH, Tr::kWarps, G, D>(a, max_len, share)) return;
   const int gw = blockIdx.x * Tr::kWarps + wid;
 
   unsigned char *wsm = smem + wid * Tr::kWarpBytes;
@@ -396,6 +396,7 @@ bool make_decode_simt(DecodeKernel *k) {
   k->launch_reduce = &launch_decode_merge<G, D, BS>;
   k->kernel = reinterpret_cast<const void *>(&paged_decode_kernel<T, D, BS, G>);
   k->warps_per_cta = Tr::kWarps;
+  k->threads_per_cta = Tr::kWarps * 32;
   k->smem_bytes = Tr::kSmemBytes;
   k->chunk_tokens = Tr::kChunk;
   k->tma_rows = 0;

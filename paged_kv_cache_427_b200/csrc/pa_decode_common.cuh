@@ -51,134 +51,78 @@ struct WarpShare {
   int s, rem, len;  // first chunk: sequence, index among that sequence's Hkv*nch chunks, length
 };
 
-// Block-wide prologue, called by every thread of the CTA: zero rows of empty contexts, count
-// the chunks, and locate each warp's first chunk with an exclusive scan over sequences.
-// `scratch` holds 256 bytes of shared memory.  Returns false when this warp has no work.
+// Zero the `heads` output rows of a sequence with an empty context (kept out of line: rare;
+// plain arguments, so the kernel parameters need no local copy).
+template <int D>
+__device__ __noinline__ void zero_rows(char *row0, long long out_h, int out_dtype, int heads) {
+  const int out_elt = out_dtype == PA_F32 ? 4 : 2;
+  const float z[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+  for (int h = 0; h < heads; ++h)
+    for (int d = 0; d < D; d += 8)
+      store_row_piece(row0 + ((long long)h * out_h + d) * out_elt, out_dtype, z, 8);
+}
+
+__device__ __forceinline__ long long warp_sum(long long x) {
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) x += __shfl_xor_sync(FULL_MASK, x, off);
+  return x;
+}
+
+// Warp-level prologue: every warp counts the step's chunks itself (reading context_lens
+// coalesced), takes its share, and finds the sequence holding its first chunk with a scan over
+// 32 sequences at a time.  No shared memory and no block-wide barrier, so warps start as soon
+// as they are scheduled.  Warp gw also flags bad lengths (warp 0) and zeroes the rows of empty
+// contexts s with s % (warps launched) == gw.  Returns false when this warp has no work.
 template <int CH, int kWarps, int G, int D>
-__device__ bool split_prologue(const DecodeArgs &a, unsigned char *scratch, int max_len,
-                               WarpShare &ws) {
-  constexpr int kTile = 8 * 32 * kWarps;  // sequences per scan tile, 8 per thread
+__device__ __forceinline__ bool split_prologue(const DecodeArgs &a, int max_len, WarpShare &ws) {
   const int lane = threadIdx.x & 31;
-  const int wid = threadIdx.x >> 5;
+  const int gw = blockIdx.x * kWarps + (threadIdx.x >> 5);
+  const int launched = gridDim.x * kWarps;
   const int S = a.num_seqs;
   const int Hkv = a.num_kv_heads;
-  long long *red = reinterpret_cast<long long *>(scratch);  // [kWarps]
-  int4 *loc = reinterpret_cast<int4 *>(scratch + 64);       // [kWarps]
-  if (threadIdx.x < kWarps) loc[threadIdx.x] = make_int4(-1, 0, 0, 0);
-
-  // Clamped length of sequence s (s < S); flags a bad length (CTA 0 only) and writes the zero
-  // rows of an empty context (one CTA per sequence).  Idempotent, so a tile may see it twice.
-  auto seq_len = [&](int s) -> int {
-    const int raw = __ldg(a.context_lens + s);
-    const int len = clamp_len(raw, max_len);
-    if (raw != len && blockIdx.x == 0) set_error(a.err, PA_DEVERR_CONTEXT_LEN);
-    if (len == 0 && (s % gridDim.x) == blockIdx.x) {
-      const int out_elt = a.out_dtype == PA_F32 ? 4 : 2;
-      const float z[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-      for (int h = 0; h < Hkv * G; ++h)
-        for (int d = 0; d < D; d += 8)
-          store_row_piece(static_cast<char *>(a.out) +
-                              ((long long)s * a.out_s + (long long)h * a.out_h + d) * out_elt,
-                          a.out_dtype, z, 8);
-    }
-    return len;
-  };
-
-  // Load one tile of sequences: this thread's chunk counts and the tile-wide exclusive prefix
-  // of its first count.
-  long long cnt[8];
-  int lens8[8];
-  auto load_tile = [&](int base, long long &tile_total) -> long long {
-    long long tsum = 0;
-#pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      const int s = base + threadIdx.x * 8 + k;
-      lens8[k] = s < S ? seq_len(s) : 0;
-      cnt[k] = (long long)((lens8[k] + CH - 1) / CH) * Hkv;
-      tsum += cnt[k];
-    }
-    long long x = tsum;
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-      const long long y = __shfl_up_sync(FULL_MASK, x, off);
-      if (lane >= off) x += y;
-    }
-    __syncthreads();  // red[] free
-    if (lane == 31) red[wid] = x;
-    __syncthreads();
-    long long ex = 0;
-    tile_total = 0;
-#pragma unroll
-    for (int w = 0; w < kWarps; ++w) {
-      if (w < wid) ex += red[w];
-      tile_total += red[w];
-    }
-    return ex + x - tsum;
-  };
-
-  long long tile_total = 0;
-  long long ex0 = load_tile(0, tile_total);
-  long long C = tile_total;
-  if (S > kTile) {
-    // more than one tile: count the rest first (the first tile stays in registers for S <= kTile)
-    for (int base = kTile; base < S; base += kTile) {
-      long long t = 0;
-      long long local = 0;
-      for (int s = base + threadIdx.x; s < base + kTile && s < S; s += blockDim.x)
-        local += (long long)((seq_len(s) + CH - 1) / CH) * Hkv;
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) local += __shfl_xor_sync(FULL_MASK, local, off);
-      __syncthreads();
-      if (lane == 0) red[wid] = local;
-      __syncthreads();
-#pragma unroll
-      for (int w = 0; w < kWarps; ++w) t += red[w];
-      C += t;
+  long long mine = 0;
+  for (int base = 0; base < S; base += 32) {
+    const int s = base + lane;
+    if (s < S) {
+      const int raw = __ldg(a.context_lens + s);
+      const int len = clamp_len(raw, max_len);
+      if (raw != len && gw == 0) set_error(a.err, PA_DEVERR_CONTEXT_LEN);
+      if (len == 0 && s % launched == gw)
+        zero_rows<D>(static_cast<char *>(a.out) + (long long)s * a.out_s * (a.out_dtype == PA_F32 ? 4 : 2),
+                     a.out_h, a.out_dtype, Hkv * G);
+      mine += (len + CH - 1) / CH;
     }
   }
+  const long long C = warp_sum(mine) * Hkv;
   const int W = (int)(C < (long long)a.num_workers ? C : (long long)a.num_workers);
   ws.C = C;
   ws.W = W;
-  if (W == 0) return false;
-
-  long long my_g0[kWarps];
-  long long last_needed = -1;
-#pragma unroll
-  for (int w = 0; w < kWarps; ++w) {
-    long long gw = (long long)blockIdx.x * kWarps + w;
-    if (gw > W) gw = W;
-    my_g0[w] = gw * C / W;
-    const long long g1 = (gw + 1 > W ? W : gw + 1) * C / W;
-    if (my_g0[w] < g1) last_needed = my_g0[w];
-  }
+  if (W == 0 || gw >= W) return false;
+  ws.g0 = (long long)gw * C / W;
+  ws.n = (long long)(gw + 1) * C / W - ws.g0;  // >= 1 because W <= C
   long long running = 0;
-  for (int base = 0; base < S && running <= last_needed; base += kTile) {
-    long long ex = ex0;
-    if (base > 0) {
-      ex = load_tile(base, tile_total);
+  for (int base = 0; base < S; base += 32) {
+    const int s = base + lane;
+    const int len = s < S ? clamp_len(__ldg(a.context_lens + s), max_len) : 0;
+    const long long cnt = (long long)((len + CH - 1) / CH) * Hkv;
+    long long incl = cnt;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const long long y = __shfl_up_sync(FULL_MASK, incl, off);
+      if (lane >= off) incl += y;
     }
-    ex += running;
-#pragma unroll
-    for (int k = 0; k < 8; ++k) {
-#pragma unroll
-      for (int w = 0; w < kWarps; ++w)
-        if (my_g0[w] <= last_needed && my_g0[w] >= ex && my_g0[w] < ex + cnt[k])
-          loc[w] = make_int4(base + threadIdx.x * 8 + k, (int)(my_g0[w] - ex), lens8[k], 0);
-      ex += cnt[k];
+    const long long tile_total = __shfl_sync(FULL_MASK, incl, 31);
+    if (running + tile_total > ws.g0) {
+      const bool hit = (running + incl - cnt <= ws.g0) && (ws.g0 < running + incl);
+      const int src = __ffs(__ballot_sync(FULL_MASK, hit)) - 1;
+      ws.s = base + src;
+      ws.rem = (int)(ws.g0 - running - __shfl_sync(FULL_MASK, incl - cnt, src));
+      ws.len = __shfl_sync(FULL_MASK, len, src);
+      return true;
     }
     running += tile_total;
   }
-  __syncthreads();
-
-  const int gw = blockIdx.x * kWarps + wid;
-  if (gw >= W) return false;
-  ws.g0 = (long long)gw * C / W;
-  ws.n = (long long)(gw + 1) * C / W - ws.g0;
-  const int4 st = loc[wid];
-  ws.s = st.x;
-  ws.rem = st.y;
-  ws.len = st.z;
-  return ws.n > 0 && st.x >= 0;
+  return false;  // not reached: g0 < C always lies in some sequence
 }
 
 // Walks one warp's share chunk by chunk in issue order.  Every lane keeps the same state.

@@ -2,11 +2,12 @@
 //
 // Same work split, cursor and merge as the CUDA-core kernel (pa_decode_common.cuh); what
 // changes is how a chunk of 16 key/value rows is consumed:
-//   * Loads: each chunk's key and value tiles arrive by TMA tensor copies (the caches are
-//     described as 4-D tensors head_dim x block_size x kv_heads x blocks) in the 128-byte
-//     swizzled layout, one box of 64 elements x 16 rows (8 at block_size 8) per 128-byte column
-//     half; the block id of each box comes from the block table, fetched a chunk ahead.  The
-//     swizzle makes every ldmatrix below free of shared-memory bank conflicts.
+//   * Loads: each chunk's key and value tiles arrive by TMA tensor copies in the 128-byte
+//     swizzled layout, one box per tile (the caches are described as 5-D tensors 64 elements x
+//     block_size rows x head_dim/64 column halves x kv_heads x blocks, so a box holds 16 rows
+//     (8 at block_size 8) of a whole head row); the block id of each box comes from the block
+//     table, fetched a chunk ahead.  The swizzle makes every ldmatrix below free of
+//     shared-memory bank conflicts.
 //   * q.K: mma.sync m16n8k16 with the 16 tokens as M, the query heads of the GQA group as N
 //     (padded to 8 with zeros) and head_dim as K; A comes from the key tile by ldmatrix, B (the
 //     group's query rows) is loaded once per piece into registers.  Products of two 16-bit
@@ -17,8 +18,8 @@
 //     K and the heads as N.  P is split into two 16-bit terms (P = hi + lo, hi = round(P),
 //     lo = round(P - hi)) so the weights keep about 16 significant bits: one 16-bit rounding of P
 //     alone would cost ~2^-9 relative error per weight.
-// An instruction count of about 200 per 16-token chunk (against about 1000 for the CUDA-core
-// kernel) leaves the kernel bound by HBM bandwidth.
+// Warp specialization keeps the copies off the critical path: four worker warps per CTA
+// consume chunks from their own rings, one producer warp issues all copies (see the kernel).
 #pragma once
 
 #include "pa_decode.cuh"
@@ -75,15 +76,33 @@ __device__ __forceinline__ void ldmatrix_x4_trans(uint32_t (&r)[4], uint32_t add
                : "r"(addr));
 }
 
-// TMA tensor copy of one box (x = element column, y = row in block, z = kv head, w = block)
-// into shared memory, completion counted on `bar`.
-__device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap *map, int x, int y,
-                                            int z, int w, uint64_t *bar) {
+// TMA tensor copy of one box of the 5-D cache view (row in block y, kv head z, block w) into
+// shared memory, completion counted on `bar`.
+__device__ __forceinline__ void tma_load_tile(uint32_t dst, const CUtensorMap *map, int y, int z,
+                                              int w, uint64_t *bar) {
   asm volatile(
-      "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes "
-      "[%0], [%1, {%2, %3, %4, %5}], [%6];" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(w), "r"(smem_u32(bar))
+      "cp.async.bulk.tensor.5d.shared::cluster.global.tile.mbarrier::complete_tx::bytes "
+      "[%0], [%1, {%2, %3, %4, %5, %6}], [%7];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(0), "r"(y), "r"(0), "r"(z), "r"(w),
+      "r"(smem_u32(bar))
       : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+// Non-blocking test of a barrier phase.
+__device__ __forceinline__ bool mbar_test(uint64_t *bar, uint32_t parity) {
+  uint32_t done;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(done)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return done != 0;
 }
 
 template <int D, int BS, int G>
@@ -92,28 +111,52 @@ struct MmaTraits {
   static constexpr int kHalves = D / 64;                // 128-byte column halves of a row
   static constexpr int kBoxRows = BS < 16 ? BS : 16;    // rows per TMA box
   static constexpr int kCopies = 16 / kBoxRows;         // blocks touched per chunk
+  static constexpr int kBoxBytes = kBoxRows * D * 2;    // one box: [half][row][128 B]
   static constexpr int kTileBytes = 16 * D * 2;         // key (or value) bytes of a chunk
   static constexpr int kQBytes = G * D * 2;
   static constexpr int kStageBytes = 2 * kTileBytes + (kQBytes + 1023) / 1024 * 1024;
-  static constexpr int kWarps = 4;
-  static constexpr int kStages = (kWarps * 3 * kStageBytes <= 110 * 1024) ? 3 : 2;
-  static constexpr int kRingBytes = kWarps * kStages * kStageBytes;
+  static constexpr int kWorkers = 4;                    // consumer warps; one producer warp more
+  static constexpr int kThreads = (kWorkers + 1) * 32;
+  static constexpr int kStages = (kWorkers * 3 * kStageBytes <= 110 * 1024) ? 3 : 2;
+  static constexpr int kRingBytes = kWorkers * kStages * kStageBytes;
   static constexpr int kPbufBytes = 2 * 8 * 16 * 2;    // [hi, lo][8 heads][16 tokens]
-  static constexpr int kSmallBytes = (kStages * 32 + kStages * 8 + 127) / 128 * 128 + kPbufBytes;
-  static constexpr int kPrologueOff = kRingBytes + kWarps * kSmallBytes;
-  static constexpr int kSmemBytes = kPrologueOff + 256 + 1024;  // + slack to align to 1 KB
+  static constexpr int kMetaOff = 0;
+  static constexpr int kFullOff = kStages * 32;
+  static constexpr int kEmptyOff = kFullOff + kStages * 8;
+  static constexpr int kPbufOff = (kEmptyOff + kStages * 8 + 127) / 128 * 128;
+  static constexpr int kSmallBytes = kPbufOff + kPbufBytes;
+  static constexpr int kShareOff = kRingBytes + kWorkers * kSmallBytes;
+  static constexpr int kSmemBytes = kShareOff + kWorkers * 32 + 16 + 1024;  // + 1 KB alignment
   static constexpr int kKSteps = D / 16;                // k-steps of q.K
   static constexpr int kMTiles = D / 16;                // m-tiles of P.V
   static_assert(D == 64 || D == 128, "head_dim 64 or 128");
   static_assert(G <= 8, "at most 8 query heads per kv head");
 };
 
+// Shared-memory record of one worker's share, written by the worker for the producer.
+struct ShareRecord {
+  int s, rem, len, pad;
+  long long g0, n;
+};
+
+// Offset in a tile of row r (0..15), column half h: boxes of kBoxRows rows, each [half][row].
+template <typename Tr>
+__device__ __forceinline__ uint32_t tile_offset(int r, int h) {
+  return (r / Tr::kBoxRows) * Tr::kBoxBytes + h * (Tr::kBoxRows * 128) + (r % Tr::kBoxRows) * 128;
+}
+
+// Warp specialization: warps 0..3 are workers (each consumes its own share of the chunk list
+// from its own ring of stages), warp 4 is the producer: its lane k walks worker k's share and
+// issues that worker's copies (one TMA box per key tile and per value tile, plus the query rows
+// when a new (sequence, kv head) starts) as soon as the worker releases a stage.  The workers
+// never issue copies, so TMA issue latency stays off their critical path.
 template <typename T, int D, int BS, int G>
-__global__ void __launch_bounds__(128, 2)
+__global__ void __launch_bounds__(MmaTraits<D, BS, G>::kThreads, 2)
     paged_decode_mma_kernel(const DecodeArgs a, const __grid_constant__ TmaMaps maps) {
   using Tr = MmaTraits<D, BS, G>;
   using M = MmaType<T>;
   constexpr int ST = Tr::kStages;
+  constexpr int NW = Tr::kWorkers;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   // 128-byte swizzled boxes must start on 1 KB boundaries
   unsigned char *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
@@ -121,83 +164,151 @@ __global__ void __launch_bounds__(128, 2)
   const int lane = threadIdx.x & 31;
   const int wid = threadIdx.x >> 5;
   const int max_len = a.max_blocks * BS;
+  ShareRecord *shares = reinterpret_cast<ShareRecord *>(smem + Tr::kShareOff);
+  long long *step_C = reinterpret_cast<long long *>(smem + Tr::kShareOff + NW * 32);
+  int *step_W = reinterpret_cast<int *>(smem + Tr::kShareOff + NW * 32 + 8);
 
-  WarpShare share;
-  if (!split_prologue<16, Tr::kWarps, G, D>(a, smem + Tr::kPrologueOff, max_len, share)) return;
-  const int gw = blockIdx.x * Tr::kWarps + wid;
-
-  unsigned char *ring = smem + wid * ST * Tr::kStageBytes;
-  unsigned char *small = smem + Tr::kRingBytes + wid * Tr::kSmallBytes;
-  ChunkMeta *meta = reinterpret_cast<ChunkMeta *>(small);
-  uint64_t *bars = reinterpret_cast<uint64_t *>(small + ST * 32);
-  unsigned char *pbuf = small + (ST * 32 + ST * 8 + 127) / 128 * 128;
-  if (lane == 0) {
-#pragma unroll
-    for (int i = 0; i < ST; ++i) mbar_init(bars + i, 1);
-    fence_barrier_init();
-  }
-  __syncwarp();
-
-  ChunkCursor<16, BS, Tr::kCopies, Tr::kBoxRows> cur;
-  cur.init(a, share, max_len);
-  const long long n = share.n;
-
-  auto issue = [&](int slot) {
-    const int f = cur.flags();
-    unsigned char *stage = ring + slot * Tr::kStageBytes;
+  // ---- set-up: barriers, then every worker finds its share and publishes it ----
+  if (wid < NW) {
+    unsigned char *small = smem + Tr::kRingBytes + wid * Tr::kSmallBytes;
     if (lane == 0) {
-      meta[slot] = cur.meta(f);
-      const uint32_t bytes = 2u * cur.valid_copies() * Tr::kHalves * Tr::kBoxRows * 128u +
-                             ((f & kFirst) ? (uint32_t)Tr::kQBytes : 0u) +
-                             ((a.test_stall && cur.issued == 0) ? 16u : 0u);
-      fence_proxy_async_smem();
-      mbar_arrive_expect_tx(bars + slot, bytes);
 #pragma unroll
-      for (int k = 0; k < Tr::kCopies; ++k) {
-        const int t = cur.i * 16 + k * Tr::kBoxRows;
-        if (t < cur.len) {
-          int blk = cur.blk[k];
-          if (blk < 0 || (long long)blk >= a.num_blocks) {
-            set_error(a.err, PA_DEVERR_BLOCK_ID);
-            blk = 0;
-          }
-#pragma unroll
-          for (int hf = 0; hf < Tr::kHalves; ++hf) {
-            const uint32_t off = hf * 2048 + k * Tr::kBoxRows * 128;
-            tma_load_4d(smem_u32(stage + off), &maps.k, hf * 64, t % BS, cur.kvh, blk, bars + slot);
-            tma_load_4d(smem_u32(stage + Tr::kTileBytes + off), &maps.v, hf * 64, t % BS, cur.kvh,
-                        blk, bars + slot);
-          }
-        }
+      for (int i = 0; i < ST; ++i) {
+        mbar_init(reinterpret_cast<uint64_t *>(small + Tr::kFullOff) + i, 1);
+        mbar_init(reinterpret_cast<uint64_t *>(small + Tr::kEmptyOff) + i, 1);
       }
-      if (f & kFirst) {
-        const char *q = static_cast<const char *>(a.query) +
-                        ((long long)cur.s * a.q_s + (long long)cur.kvh * G * a.q_h) * 2;
-        if (a.q_heads_contiguous) {
-          bulk_copy_g2s(stage + 2 * Tr::kTileBytes, q, Tr::kQBytes, bars + slot);
-        } else {
-#pragma unroll
-          for (int h = 0; h < G; ++h)
-            bulk_copy_g2s(stage + 2 * Tr::kTileBytes + h * D * 2, q + (long long)h * a.q_h * 2, D * 2,
-                          bars + slot);
-        }
+      fence_barrier_init();
+    }
+    WarpShare ws;
+    ws.n = 0;
+    const bool has = split_prologue<16, NW, G, D>(a, max_len, ws);
+    if (lane == 0) {
+      ShareRecord r;
+      r.s = has ? ws.s : -1;
+      r.rem = has ? ws.rem : 0;
+      r.len = has ? ws.len : 0;
+      r.pad = 0;
+      r.g0 = has ? ws.g0 : 0;
+      r.n = has ? ws.n : 0;
+      shares[wid] = r;
+      if (wid == 0) {
+        *step_C = ws.C;
+        *step_W = ws.W;
       }
     }
-    cur.advance(a);
-  };
+  } else if (lane == 0) {
+    // bring the two descriptors into the TMA unit while the workers run their prologue
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&maps.k)) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&maps.v)) : "memory");
+  }
+  __syncthreads();
 
-  // Everything above read only context_lens and block_tables; the caches and the query may
-  // still be written by the previous grid when this one was launched to overlap it.
-  wait_for_previous_grid();
-  const long long prime = n < ST ? n : ST;
-  for (long long i = 0; i < prime; ++i) issue((int)i);
+  if (wid == NW) {
+    // ================================ producer ================================
+    const int k = lane;  // the worker this lane feeds
+    bool active = false;
+    ChunkCursor<16, BS, Tr::kCopies, Tr::kBoxRows> cur;
+    unsigned char *ring = smem + k * ST * Tr::kStageBytes;
+    unsigned char *small = smem + Tr::kRingBytes + k * Tr::kSmallBytes;
+    ChunkMeta *meta = reinterpret_cast<ChunkMeta *>(small + Tr::kMetaOff);
+    uint64_t *full = reinterpret_cast<uint64_t *>(small + Tr::kFullOff);
+    uint64_t *empty = reinterpret_cast<uint64_t *>(small + Tr::kEmptyOff);
+    if (k < NW) {
+      const ShareRecord r = shares[k];
+      if (r.n > 0 && r.s >= 0) {
+        WarpShare ws;
+        ws.C = *step_C;
+        ws.W = *step_W;
+        ws.g0 = r.g0;
+        ws.n = r.n;
+        ws.s = r.s;
+        ws.rem = r.rem;
+        ws.len = r.len;
+        cur.init(a, ws, max_len);
+        active = true;
+      }
+    }
+    // Everything above read only context_lens and block_tables; the caches and the query may
+    // still be written by the previous grid when this one was launched to overlap it.
+    wait_for_previous_grid();
+    long long last_progress = clock64();
+    while (__any_sync(FULL_MASK, active)) {
+      bool can = false;
+      int slot = 0;
+      if (active) {
+        slot = (int)(cur.issued % ST);
+        can = cur.issued < ST ||
+              mbar_test(empty + slot, (uint32_t)(((cur.issued / ST) - 1) & 1));
+      }
+      if (can) {
+        const int f = cur.flags();
+        unsigned char *stage = ring + slot * Tr::kStageBytes;
+        meta[slot] = cur.meta(f);
+        const uint32_t bytes = 2u * cur.valid_copies() * Tr::kBoxBytes +
+                               ((f & kFirst) ? (uint32_t)Tr::kQBytes : 0u) +
+                               ((a.test_stall && cur.issued == 0) ? 16u : 0u);
+        mbar_arrive_expect_tx(full + slot, bytes);
+#pragma unroll
+        for (int c = 0; c < Tr::kCopies; ++c) {
+          const int t = cur.i * 16 + c * Tr::kBoxRows;
+          if (t < cur.len) {
+            int blk = cur.blk[c];
+            if (blk < 0 || (long long)blk >= a.num_blocks) {
+              set_error(a.err, PA_DEVERR_BLOCK_ID);
+              blk = 0;
+            }
+            const uint32_t off = c * Tr::kBoxBytes;
+            tma_load_tile(smem_u32(stage + off), &maps.k, t % BS, cur.kvh, blk, full + slot);
+            tma_load_tile(smem_u32(stage + Tr::kTileBytes + off), &maps.v, t % BS, cur.kvh, blk,
+                          full + slot);
+          }
+        }
+        if (f & kFirst) {
+          const char *q = static_cast<const char *>(a.query) +
+                          ((long long)cur.s * a.q_s + (long long)cur.kvh * G * a.q_h) * 2;
+          if (a.q_heads_contiguous) {
+            bulk_copy_g2s(stage + 2 * Tr::kTileBytes, q, Tr::kQBytes, full + slot);
+          } else {
+#pragma unroll
+            for (int h = 0; h < G; ++h)
+              bulk_copy_g2s(stage + 2 * Tr::kTileBytes + h * D * 2, q + (long long)h * a.q_h * 2,
+                            D * 2, full + slot);
+          }
+        }
+        cur.advance(a);
+        if (cur.issued >= cur.n) active = false;
+      }
+      if (__any_sync(FULL_MASK, can)) {
+        last_progress = clock64();
+      } else {
+        if (clock64() - last_progress > a.wait_cycles) {
+          // a worker stopped releasing stages: give up (the worker reports its own timeout)
+          if (active) set_error(a.err, PA_DEVERR_TIMEOUT);
+          break;
+        }
+        __nanosleep(64);
+      }
+    }
+    return;
+  }
+
+  // ================================ workers ================================
+  const ShareRecord share = shares[wid];
+  if (share.n <= 0 || share.s < 0) return;
+  const int gw = blockIdx.x * NW + wid;
+  const long long n = share.n;
+  unsigned char *ring = smem + wid * ST * Tr::kStageBytes;
+  unsigned char *small = smem + Tr::kRingBytes + wid * Tr::kSmallBytes;
+  const ChunkMeta *meta = reinterpret_cast<const ChunkMeta *>(small + Tr::kMetaOff);
+  uint64_t *full = reinterpret_cast<uint64_t *>(small + Tr::kFullOff);
+  uint64_t *empty = reinterpret_cast<uint64_t *>(small + Tr::kEmptyOff);
+  unsigned char *pbuf = small + Tr::kPbufOff;
 
   const int g = lane >> 2;  // fragment row group
   const int c = lane & 3;   // fragment column pair
   const int h0 = 2 * c, h1 = 2 * c + 1;  // heads of this lane's logits / output columns
-  // ldmatrix row addressing (constant per lane)
-  const int lm = lane >> 3;         // which 8x8 matrix this lane addresses
-  const int lr = lane & 7;          // row within it
+  const int lm = lane >> 3;  // which 8x8 matrix this lane addresses for ldmatrix
+  const int lr = lane & 7;   // row within it
   uint32_t qb[Tr::kKSteps][2];
   float o[Tr::kMTiles][4];
   float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
@@ -206,10 +317,11 @@ __global__ void __launch_bounds__(128, 2)
   for (long long cc = 0; cc < n; ++cc) {
     const int slot = (int)(cc % ST);
     const uint32_t parity = (uint32_t)((cc / ST) & 1);
-    if (!mbar_wait_bounded(bars + slot, parity, a.wait_cycles)) {
+    if (!mbar_wait_bounded(full + slot, parity, a.wait_cycles)) {
+      // a copy never completed: record it, let the copies that may be in flight land, stop.
       if (lane == 0) set_error(a.err, PA_DEVERR_TIMEOUT);
-      for (long long k = cc; k < cur.issued; ++k)
-        mbar_wait_bounded(bars + (int)(k % ST), (uint32_t)((k / ST) & 1), a.wait_cycles);
+      for (long long j = cc; j < cc + ST && j < n; ++j)
+        mbar_wait_bounded(full + (int)(j % ST), (uint32_t)((j / ST) & 1), a.wait_cycles);
       return;
     }
     const ChunkMeta m = meta[slot];
@@ -244,7 +356,7 @@ __global__ void __launch_bounds__(128, 2)
 #pragma unroll
       for (int ks = 0; ks < Tr::kKSteps; ++ks) {
         const int c16 = ((ks & 3) << 1) | (lm >> 1);
-        const uint32_t addr = kbase + (ks >> 2) * 2048 + row * 128 + ((c16 ^ lr) << 4);
+        const uint32_t addr = kbase + tile_offset<Tr>(row, ks >> 2) + ((c16 ^ lr) << 4);
         uint32_t af[4];
         ldmatrix_x4(af, addr);
         if (ks & 1)
@@ -320,8 +432,7 @@ __global__ void __launch_bounds__(128, 2)
 #pragma unroll
       for (int mt = 0; mt < Tr::kMTiles; ++mt) {
         const int c16g = (mt << 1) | (lm & 1);
-        const uint32_t addr =
-            vbase + (c16g >> 3) * 2048 + row * 128 + (((c16g & 7) ^ lr) << 4);
+        const uint32_t addr = vbase + tile_offset<Tr>(row, c16g >> 3) + (((c16g & 7) ^ lr) << 4);
         uint32_t vf[4];
         ldmatrix_x4_trans(vf, addr);
         if (tail) {
@@ -335,6 +446,9 @@ __global__ void __launch_bounds__(128, 2)
         M::mma(o[mt], vf, pf[2], pf[3]);
       }
     }
+    // the stage is no longer needed: hand it back to the producer
+    __syncwarp();
+    if (lane == 0) mbar_arrive(empty + slot);
 
     // ---- end of a piece ----
     if (m.flags & kLast) {
@@ -407,8 +521,6 @@ __global__ void __launch_bounds__(128, 2)
         finish_piece<G, D>(a, m, lane);
       }
     }
-    __syncwarp();
-    if (cur.issued < n) issue(slot);
   }
 }
 
@@ -416,7 +528,7 @@ template <typename T, int D, int BS, int G>
 cudaError_t launch_decode_mma(const DecodeArgs &a, const TmaMaps *maps, int num_ctas,
                               bool overlap_previous, cudaStream_t st) {
   using Tr = MmaTraits<D, BS, G>;
-  return launch_overlapping(paged_decode_mma_kernel<T, D, BS, G>, num_ctas, Tr::kWarps * 32,
+  return launch_overlapping(paged_decode_mma_kernel<T, D, BS, G>, num_ctas, Tr::kThreads,
                             Tr::kSmemBytes, overlap_previous, st, a, *maps);
 }
 
@@ -436,7 +548,8 @@ bool make_decode_mma(DecodeKernel *k) {
   k->launch = &launch_decode_mma<T, D, BS, G>;
   k->launch_reduce = &launch_decode_merge<G, D, BS>;
   k->kernel = reinterpret_cast<const void *>(&paged_decode_mma_kernel<T, D, BS, G>);
-  k->warps_per_cta = Tr::kWarps;
+  k->warps_per_cta = Tr::kWorkers;
+  k->threads_per_cta = Tr::kThreads;
   k->smem_bytes = Tr::kSmemBytes;
   k->chunk_tokens = 16;
   k->tma_rows = Tr::kBoxRows;

@@ -40,8 +40,10 @@ struct DecodeArgs {
   int test_stall;         // test hook: each warp's first stage expects 16 bytes nobody sends
 };
 
-// TMA descriptors of the two caches, viewed as 4-D tensors (head_dim, block_size, kv heads,
-// blocks), 128-byte swizzled boxes of 64 elements x tma_rows rows.
+// TMA descriptors of the two caches, viewed as 5-D tensors (64 elements, block_size rows,
+// head_dim / 64 column halves, kv heads, blocks) read in 128-byte swizzled boxes of
+// 64 x tma_rows x head_dim/64: one box holds a whole (rows x head_dim) tile as
+// [half][row][128 bytes].
 struct TmaMaps {
   CUtensorMap k;
   CUtensorMap v;
@@ -52,7 +54,8 @@ struct DecodeKernel {
                         cudaStream_t);
   cudaError_t (*launch_reduce)(const DecodeArgs &, cudaStream_t);
   const void *kernel;  // for occupancy queries
-  int warps_per_cta;
+  int warps_per_cta;    // worker warps per CTA (each takes one share of the chunk list)
+  int threads_per_cta;  // all threads of a CTA (workers plus any helper warp)
   int smem_bytes;
   int chunk_tokens;
   int tma_rows;  // 0: the kernel reads the caches with 1-D bulk copies; else TMA box rows
