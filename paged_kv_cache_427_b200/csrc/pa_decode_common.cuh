@@ -223,42 +223,84 @@ struct ChunkCursor {
 };
 
 // Merge the pieces (o, m, l) of one (sequence, kv head) and write its G output rows.  Called by
-// a whole warp; pieces live in workspace slots pair + first_worker + k, k < npieces; lane j
-// handles dims [4j, 4j+4) of every head.  m is in base-2 logit units.
+// a whole warp; pieces live in workspace slots pair + first_worker + k, k < npieces.  Loads are
+// issued for many pieces at once (lane k fetches piece k's (m, l); then 4 pieces' outputs per
+// round) so a merge costs a few memory round trips, not two per piece.  m is in base-2 units.
 template <int G, int D>
 __device__ __forceinline__ void merge_pieces(const DecodeArgs &a, int pair, int first_worker,
                                              int npieces, int s, int kvh, int lane) {
-  float M[G];
-#pragma unroll
-  for (int h = 0; h < G; ++h) M[h] = -INFINITY;
-  for (int k = 0; k < npieces; ++k) {
-    const long long seg = (long long)pair + first_worker + k;
-#pragma unroll
-    for (int h = 0; h < G; ++h) M[h] = fmaxf(M[h], __ldcg(a.part_ml + (seg * G + h) * 2));
-  }
-  const bool active = lane < D / 4;
+  const long long seg0 = (long long)pair + first_worker;
+  const bool active = lane < D / 4;  // lane j handles dims [4j, 4j+4) of every head
+  float M[G], den[G];
   float4 num[G];
-  float den[G];
 #pragma unroll
   for (int h = 0; h < G; ++h) {
+    M[h] = -INFINITY;
     den[h] = 0.f;
     num[h] = make_float4(0.f, 0.f, 0.f, 0.f);
   }
-  for (int k = 0; k < npieces; ++k) {
-    const long long seg = (long long)pair + first_worker + k;
+  for (int base = 0; base < npieces; base += 32) {
+    const int cnt = npieces - base < 32 ? npieces - base : 32;
+    // lane k < cnt: (m, l) of piece base + k for every head
+    float mk[G], lk[G];
 #pragma unroll
     for (int h = 0; h < G; ++h) {
-      const float m = __ldcg(a.part_ml + (seg * G + h) * 2);
-      const float l = __ldcg(a.part_ml + (seg * G + h) * 2 + 1);
-      const float w = l * fast_exp2(m - M[h]);
-      den[h] += w;
-      if (active) {
-        const float4 x = __ldcg(reinterpret_cast<const float4 *>(a.part_o + (seg * G + h) * D) + lane);
-        num[h].x += w * x.x;
-        num[h].y += w * x.y;
-        num[h].z += w * x.z;
-        num[h].w += w * x.w;
+      mk[h] = -INFINITY;
+      lk[h] = 0.f;
+    }
+    if (lane < cnt) {
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        const float2 ml = __ldcg(reinterpret_cast<const float2 *>(a.part_ml + ((seg0 + base + lane) * G + h) * 2));
+        mk[h] = ml.x;
+        lk[h] = ml.y;
       }
+    }
+    // fold this group into the running maximum and rescale what is already accumulated
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+      float gm = mk[h];
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) gm = fmaxf(gm, __shfl_xor_sync(FULL_MASK, gm, off));
+      const float newM = fmaxf(M[h], gm);
+      const float r = (M[h] == -INFINITY) ? 0.f : fast_exp2(M[h] - newM);
+      den[h] *= r;
+      num[h].x *= r;
+      num[h].y *= r;
+      num[h].z *= r;
+      num[h].w *= r;
+      M[h] = newM;
+      // this lane's weight for its piece
+      const float w = (lane < cnt) ? lk[h] * fast_exp2(mk[h] - newM) : 0.f;
+      float ws = w;
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) ws += __shfl_xor_sync(FULL_MASK, ws, off);
+      den[h] += ws;
+      mk[h] = w;  // reuse: the weight of piece base + lane
+    }
+    // outputs: U pieces per round (U*G float4 in flight per lane), loads issued together
+    constexpr int U = G >= 8 ? 1 : 8 / G;
+    for (int k = 0; k < cnt; k += U) {
+      float4 x[U][G];
+#pragma unroll
+      for (int u = 0; u < U; ++u)
+#pragma unroll
+        for (int h = 0; h < G; ++h)
+          x[u][h] = (active && k + u < cnt)
+                        ? __ldcg(reinterpret_cast<const float4 *>(a.part_o + ((seg0 + base + k + u) * G + h) * D) + lane)
+                        : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int u = 0; u < U; ++u)
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+          const float w = __shfl_sync(FULL_MASK, mk[h], (k + u) & 31);
+          if (k + u < cnt) {
+            num[h].x += w * x[u][h].x;
+            num[h].y += w * x[u][h].y;
+            num[h].z += w * x[u][h].z;
+            num[h].w += w * x[u][h].w;
+          }
+        }
     }
   }
   if (!active) return;
@@ -287,6 +329,25 @@ __device__ __forceinline__ void merge_pieces(const DecodeArgs &a, int pair, int 
   }
 }
 
+// What a worker needs to take a split piece's ticket after its (o, m, l) are stored.
+struct PieceInfo {
+  int pair, first_worker, npieces, s, kvh;
+};
+
+// Take the ticket of a published piece and merge when it is the last of its (sequence, kv
+// head).  The caller has made the piece's stores visible GPU-wide.  Called by a whole warp.
+template <int G, int D>
+__device__ __forceinline__ void take_ticket(const DecodeArgs &a, const PieceInfo &p, int lane) {
+  unsigned int ticket = 0;
+  if (lane == 0) ticket = atomicAdd(a.counters + p.pair, 1u);
+  ticket = __shfl_sync(FULL_MASK, ticket, 0);
+  if (ticket == (unsigned int)(p.npieces - 1)) {
+    __threadfence();
+    merge_pieces<G, D>(a, p.pair, p.first_worker, p.npieces, p.s, p.kvh, lane);
+    if (lane == 0) a.counters[p.pair] = 0u;
+  }
+}
+
 // After a piece's (o, m, l) are stored: publish them, take a ticket, and merge when this is the
 // last piece of its (sequence, kv head).  Called by a whole warp.
 template <int G, int D>
@@ -304,10 +365,12 @@ __device__ __forceinline__ void finish_piece(const DecodeArgs &a, const ChunkMet
   }
 }
 
-// Separate merge: one warp per (sequence, kv head) that has more than one piece.
+// Separate merge: one warp per (sequence, kv head) that has more than one piece.  Launched to
+// overlap the decode grid; it waits for that grid's pieces before reading them.
 template <int G, int D, int BS>
 __global__ void __launch_bounds__(128) paged_decode_merge_kernel(const DecodeArgs a) {
   const int lane = threadIdx.x & 31;
+  wait_for_previous_grid();
   const long long pairs = (long long)a.num_seqs * a.num_kv_heads;
   const int max_len = a.max_blocks * BS;
   for (long long p = (long long)blockIdx.x * 4 + (threadIdx.x >> 5); p < pairs;
@@ -327,8 +390,16 @@ cudaError_t launch_decode_merge(const DecodeArgs &a, cudaStream_t st) {
   long long blocks = (pairs + 3) / 4;
   if (blocks > 4096) blocks = 4096;
   if (blocks < 1) blocks = 1;
-  paged_decode_merge_kernel<G, D, BS><<<(int)blocks, 128, 0, st>>>(a);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)blocks);
+  cfg.blockDim = dim3(128);
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, paged_decode_merge_kernel<G, D, BS>, a);
 }
 
 }  // namespace pa

@@ -88,6 +88,15 @@ __device__ __forceinline__ void tma_load_tile(uint32_t dst, const CUtensorMap *m
       : "memory");
 }
 
+// Prefetch one box of the 5-D cache view into L2 (no shared memory, no completion to wait for).
+__device__ __forceinline__ void tma_prefetch_tile(const CUtensorMap *map, int y, int z, int w) {
+  asm volatile(
+      "cp.async.bulk.prefetch.tensor.5d.L2.global.tile [%0, {%1, %2, %3, %4, %5}];" ::"l"(
+          reinterpret_cast<uint64_t>(map)),
+      "r"(0), "r"(y), "r"(0), "r"(z), "r"(w)
+      : "memory");
+}
+
 __device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
@@ -226,8 +235,21 @@ __global__ void __launch_bounds__(MmaTraits<D, BS, G>::kThreads, 2)
         ws.len = r.len;
         cur.init(a, ws, max_len);
         active = true;
+        // Warm L2 with the first chunk while the previous grid may still run: L2 is the point
+        // of coherence, so a line that grid writes afterwards is read fresh by the copies below.
+#pragma unroll
+        for (int c = 0; c < Tr::kCopies; ++c) {
+          const int t = cur.i * 16 + c * Tr::kBoxRows;
+          const int blk = cur.blk[c];
+          if (t < cur.len && blk >= 0 && (long long)blk < a.num_blocks) {
+            tma_prefetch_tile(&maps.k, t % BS, cur.kvh, blk);
+            tma_prefetch_tile(&maps.v, t % BS, cur.kvh, blk);
+          }
+        }
       }
     }
+    // A grid launched after this one (the separate merge) may start now and wait for us.
+    if (lane == 0) allow_next_grid();
     // Everything above read only context_lens and block_tables; the caches and the query may
     // still be written by the previous grid when this one was launched to overlap it.
     wait_for_previous_grid();
