@@ -62,7 +62,7 @@
 extern "C" {
 #endif
 
-#define PA_VERSION 1
+#define PA_VERSION 2
 
 /* Symbols of this ABI are the only ones the shared library exports. */
 #if defined(__GNUC__)
@@ -134,6 +134,29 @@ typedef enum pa_status {
 PA_API int pa_reshape_and_cache(const pa_tensor *key, const pa_tensor *value,
                          const pa_tensor *key_cache, const pa_tensor *value_cache,
                          const pa_tensor *slot_mapping, void *stream);
+
+/*
+ * pa_decode_step - one whole decode step: pa_reshape_and_cache(key, value, key_cache,
+ * value_cache, slot_mapping) followed by pa_decode_ex(out, query, key_cache, value_cache,
+ * block_tables, context_lens, ..., num_workers = 0, PA_DECODE_OVERLAP_PREVIOUS, workspace),
+ * i.e. the write side of [P2] 4.1 and the attention of [P4] 2.2.2 for the same step.  The
+ * decode is launched as a programmatic dependent of the write: its prologue (context_lens,
+ * block_tables, the split of the work) runs while the write finishes, and it reads the caches
+ * only after.  Both halves are validated before either is launched, so a refused call launches
+ * nothing.  workspace: as for pa_decode_ex, or NULL for the library-owned one of pa_decode.
+ * With a caller workspace initialised beforehand (pa_workspace_init) the call allocates
+ * nothing and can be captured into a CUDA graph (one graph node per kernel, the programmatic
+ * dependency kept as a graph edge); the graph is valid as long as the tensors it was captured
+ * with stay where they are.  Errors as for the two calls; on PA_ERR_CUDA from the decode launch
+ * the cache write may already have been launched.
+ */
+PA_API int pa_decode_step(const pa_tensor *key, const pa_tensor *value,
+                          const pa_tensor *key_cache, const pa_tensor *value_cache,
+                          const pa_tensor *slot_mapping, const pa_tensor *out,
+                          const pa_tensor *query, const pa_tensor *block_tables,
+                          const pa_tensor *context_lens, float scale, int32_t block_size,
+                          int32_t num_kv_heads, void *workspace, size_t workspace_bytes,
+                          void *stream);
 
 /*
  * pa_copy_blocks - copy whole physical blocks (all kv heads, all slots, both caches):

@@ -36,7 +36,13 @@ PA_DEVERR_SLOT = 0x4
 PA_DEVERR_COPY_PAIR = 0x8
 PA_DEVERR_TIMEOUT = 0x10
 PA_NOALLOC_SCRATCH_BYTES = 8 * 1024 * 1024
+PA_ERR_INVALID_ARG = -1
+PA_ERR_SHAPE = -2
+PA_ERR_DTYPE = -3
+PA_ERR_UNSUPPORTED = -4
+PA_ERR_CUDA = -5
 PA_ERR_WORKSPACE = -6
+PA_ERR_LAYOUT = -7
 STATUS_NAMES = {0: "PA_OK", -1: "PA_ERR_INVALID_ARG", -2: "PA_ERR_SHAPE", -3: "PA_ERR_DTYPE",
                 -4: "PA_ERR_UNSUPPORTED", -5: "PA_ERR_CUDA", -6: "PA_ERR_WORKSPACE",
                 -7: "PA_ERR_LAYOUT"}
@@ -81,6 +87,7 @@ def load(path: str = LIBRARY) -> ctypes.CDLL:
     lib.pa_last_error.restype = ctypes.c_char_p
     lib.pa_get_device_error.argtypes = [_P, ctypes.POINTER(u32), i32]
     lib.pa_decode_noalloc.argtypes = [_T, _T, _T, _T, _T, _T, f32, i32, i32, _P]
+    lib.pa_decode_step.argtypes = [_T, _T, _T, _T, _T, _T, _T, _T, _T, f32, i32, i32, _P, sz, _P]
     lib.pa_version.argtypes = []
     lib.pa_version.restype = i32
     for name in ("pa_reshape_and_cache", "pa_copy_blocks", "pa_decode", "pa_decode_ex",
@@ -164,6 +171,21 @@ def pa_decode_ex(out, query, key_cache, value_cache, block_tables, context_lens,
     _check("pa_decode_ex", lib.pa_decode_ex(*[ctypes.byref(x) for x in d], float(scale),
                                             int(block_size), int(num_kv_heads), int(num_workers),
                                             int(flags), ws_ptr, ws_bytes, _stream(stream)))
+
+
+def pa_decode_step(key, value, key_cache, value_cache, slot_mapping, out, query, block_tables,
+                   context_lens, scale, block_size, num_kv_heads, workspace=None, stream=None):
+    """One whole step: the cache write, then the decode launched to overlap it (see
+    include/pa.h).  workspace: a CUDA uint8 tensor as for pa_decode_ex, or None for the
+    library-owned one."""
+    lib = load()
+    d = [describe(x) for x in (key, value, key_cache, value_cache, slot_mapping, out, query,
+                               block_tables, context_lens)]
+    ws_ptr = workspace.data_ptr() if workspace is not None else None
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check("pa_decode_step", lib.pa_decode_step(*[ctypes.byref(x) for x in d], float(scale),
+                                                int(block_size), int(num_kv_heads), ws_ptr,
+                                                ws_bytes, _stream(stream)))
 
 
 def pa_decode_noalloc(out, query, key_cache, value_cache, block_tables, context_lens, scale,

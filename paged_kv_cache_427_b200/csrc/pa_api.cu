@@ -80,6 +80,10 @@ std::vector<DeviceState> g_devices;
 // so a call with fewer sequences may write partial results where a later, larger call keeps
 // counters.  For each workspace the library remembers how many leading bytes are known to hold
 // zero counters and zeroes the rest (on the call's stream) before a call that needs more.
+// How far a call goes: host-side argument checks only, every check (device memory, workspace
+// size) without launching, or the whole call.
+enum class CallMode { kHostChecks, kAllChecks, kLaunch };
+
 struct CleanRecord {
   const void *ws;
   size_t clean;
@@ -362,7 +366,8 @@ int decode_impl(const pa_tensor *out, const pa_tensor *query, const pa_tensor *k
                 const pa_tensor *value_cache, const pa_tensor *block_tables,
                 const pa_tensor *context_lens, float scale, int32_t block_size,
                 int32_t num_kv_heads, int32_t num_workers, uint32_t flags, void *workspace,
-                size_t workspace_bytes, bool library_workspace, void *stream) {
+                size_t workspace_bytes, bool library_workspace, void *stream,
+                CallMode mode = CallMode::kLaunch) {
   int rc;
   CacheShape cs;
   if ((rc = check_caches(key_cache, value_cache, &cs))) return rc;
@@ -408,7 +413,7 @@ int decode_impl(const pa_tensor *out, const pa_tensor *query, const pa_tensor *k
   if (S > 0x7fffffff || block_tables->shape[1] * block_size > 0x7fffffff)
     return fail(PA_ERR_SHAPE, "too many sequences or too long a block table");
   if (!std::isfinite(scale)) return fail(PA_ERR_INVALID_ARG, "scale must be finite");
-  if (S == 0) return PA_OK;
+  if (S == 0 || mode == CallMode::kHostChecks) return PA_OK;
   DeviceState *ds;
   int dev;
   if ((rc = device_state(&ds, &dev))) return rc;
@@ -434,6 +439,13 @@ int decode_impl(const pa_tensor *out, const pa_tensor *query, const pa_tensor *k
   if (chunks * (double)W > 4.0e18) return fail(PA_ERR_SHAPE, "step too large for the work split");
   const WsLayout L = ws_layout(S, (int)Hq, num_kv_heads, D, W);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (mode == CallMode::kAllChecks) {  // everything a launch would check, nothing launched
+    if (!library_workspace && (!workspace || workspace_bytes < L.total))
+      return fail(PA_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", L.total, workspace_bytes);
+    if (!library_workspace && ((uintptr_t)workspace & 255u) != 0)
+      return fail(PA_ERR_WORKSPACE, "workspace must be 256-byte aligned");
+    return PA_OK;
+  }
   if (library_workspace) {
     std::lock_guard<std::mutex> lock(g_mu);
     if (ds->ws_bytes < L.total) {
@@ -546,10 +558,11 @@ int decode_into(const pa_tensor *out, const pa_tensor *query, const pa_tensor *k
 
 }  // namespace pa
 
-extern "C" {
+namespace {
 
-int pa_reshape_and_cache(const pa_tensor *key, const pa_tensor *value, const pa_tensor *key_cache,
-                         const pa_tensor *value_cache, const pa_tensor *slot_mapping, void *stream) {
+int write_impl(const pa_tensor *key, const pa_tensor *value, const pa_tensor *key_cache,
+               const pa_tensor *value_cache, const pa_tensor *slot_mapping, void *stream,
+               CallMode mode) {
   int rc;
   CacheShape cs;
   if ((rc = check_caches(key_cache, value_cache, &cs))) return rc;
@@ -569,7 +582,7 @@ int pa_reshape_and_cache(const pa_tensor *key, const pa_tensor *value, const pa_
     return fail(PA_ERR_LAYOUT, "key/value need a contiguous head_dim and slot_mapping unit stride");
   if (!aligned16(key->data) || !aligned16(value->data) || !strides16(key, 2) || !strides16(value, 2))
     return fail(PA_ERR_LAYOUT, "key/value: data and token/head strides must be 16-byte aligned");
-  if (T == 0) return PA_OK;
+  if (T == 0 || mode == CallMode::kHostChecks) return PA_OK;
   DeviceState *ds;
   int dev;
   if ((rc = device_state(&ds, &dev))) return rc;
@@ -598,8 +611,39 @@ int pa_reshape_and_cache(const pa_tensor *key, const pa_tensor *value, const pa_
   a.num_slots = cs.num_blocks * cs.block_size;
   a.err = ds->err;
   if (a.row_bytes % 16 != 0) return fail(PA_ERR_UNSUPPORTED, "head_dim * element size must be a multiple of 16 bytes");
+  if (mode == CallMode::kAllChecks) return PA_OK;
   cudaError_t err = pa::launch_reshape_and_cache(a, ds->num_sms, static_cast<cudaStream_t>(stream));
   return err == cudaSuccess ? PA_OK : cuda_fail(err, "reshape_and_cache launch");
+}
+
+}  // namespace
+
+extern "C" {
+
+int pa_reshape_and_cache(const pa_tensor *key, const pa_tensor *value, const pa_tensor *key_cache,
+                         const pa_tensor *value_cache, const pa_tensor *slot_mapping, void *stream) {
+  return write_impl(key, value, key_cache, value_cache, slot_mapping, stream, CallMode::kLaunch);
+}
+
+int pa_decode_step(const pa_tensor *key, const pa_tensor *value, const pa_tensor *key_cache,
+                   const pa_tensor *value_cache, const pa_tensor *slot_mapping,
+                   const pa_tensor *out, const pa_tensor *query, const pa_tensor *block_tables,
+                   const pa_tensor *context_lens, float scale, int32_t block_size,
+                   int32_t num_kv_heads, void *workspace, size_t workspace_bytes, void *stream) {
+  const bool lib_ws = workspace == nullptr;
+  int rc;
+  // both halves are checked (host-side checks of both first) before either is launched
+  for (CallMode m : {CallMode::kHostChecks, CallMode::kAllChecks})
+    if ((rc = write_impl(key, value, key_cache, value_cache, slot_mapping, stream, m)) ||
+        (rc = decode_impl(out, query, key_cache, value_cache, block_tables, context_lens, scale,
+                          block_size, num_kv_heads, 0, PA_DECODE_OVERLAP_PREVIOUS, workspace,
+                          workspace_bytes, lib_ws, stream, m)))
+      return rc;
+  if ((rc = write_impl(key, value, key_cache, value_cache, slot_mapping, stream, CallMode::kLaunch)))
+    return rc;
+  return decode_impl(out, query, key_cache, value_cache, block_tables, context_lens, scale,
+                     block_size, num_kv_heads, 0, PA_DECODE_OVERLAP_PREVIOUS, workspace,
+                     workspace_bytes, lib_ws, stream);
 }
 
 int pa_copy_blocks(const pa_tensor *key_cache, const pa_tensor *value_cache,

@@ -146,3 +146,28 @@ def test_copy_blocks_rejects_bad_arguments(lib):
     assert lib.pa_copy_blocks(r(kc), r(vc), r(_t([3, 3], pa.PA_I64)), None) == -2
     assert lib.pa_copy_blocks(r(kc), r(vc), r(_t([3, 2], pa.PA_I32)), None) == -3
     assert lib.pa_copy_blocks(r(kc), r(vc), r(_t([0, 2], pa.PA_I64)), None) == 0
+
+
+def test_decode_step_checks_both_halves_first(lib):
+    r = ctypes.byref
+    a = _decode_args()
+    key = _t([4, 2, 128], pa.PA_BF16)
+    slots = _t([4], pa.PA_I64)
+
+    def step(key=key, slots=slots, a=a, bs=16):
+        return lib.pa_decode_step(r(key), r(key), r(a["kc"]), r(a["vc"]), r(slots), r(a["out"]),
+                                  r(a["query"]), r(a["bt"]), r(a["cl"]), 0.1, bs, 2, None, 0, None)
+
+    assert step(slots=_t([4], pa.PA_I32)) == -3        # write half: slots must be int64
+    assert step(key=_t([4, 3, 128], pa.PA_BF16)) == -2  # write half: kv heads of the cache
+    assert step(bs=8) == -2                             # decode half: block_size mismatch
+    b = _decode_args(D=96)
+    assert step(key=_t([4, 2, 96], pa.PA_BF16), a=b) == -4  # decode half: head_dim not built
+    assert pa.pa_last_error()
+
+
+def test_status_constants_match_header():
+    with open(pa.HEADER) as f:
+        text = f.read()
+    for name, value in re.findall(r"\b(PA_ERR_[A-Z_]+)\s*=\s*(-\d+)", text):
+        assert getattr(pa, name) == int(value), name
