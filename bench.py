@@ -512,6 +512,79 @@ def run_ours(args, b: W.PagedBatch, config: dict, rank: int, world: int, local_r
     print(json.dumps(line), flush=True)
 
 
+def run_swap(args, b, config):
+    """Block swap between the device cache and a pinned host cache: every block the batch's
+    sequences use goes out (device -> host, scattered host ids) and back in (host -> device,
+    scattered device ids), each direction one pa_swap_blocks call timed with CUDA events.  The
+    roofline is the host link as one plain cudaMemcpyAsync of the same bytes between one
+    contiguous pinned buffer and device memory moves them, measured in the same run."""
+    import torch
+
+    import paged_kv_cache_427_b200 as pa
+
+    pa.load()
+    dev = torch.device("cuda", 0)
+    t = {"bf16": torch.bfloat16, "f16": torch.float16, "f32": torch.float32}[b.dtype]
+
+    def dev_t(a, dt=None):
+        if dt == "bf16":
+            return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
+        return torch.from_numpy(np.ascontiguousarray(a)).to(dev)
+
+    kc, vc = dev_t(b.key_cache, b.dtype), dev_t(b.value_cache, b.dtype)
+    ids = []
+    for s in range(b.num_seqs):
+        ids.extend(b.block_tables[s, :-(-int(b.context_lens[s]) // b.block_size)].tolist())
+    ids = np.array(sorted(set(ids)), np.int64)
+    n = len(ids)
+    rng = np.random.default_rng(0)
+    host_ids = rng.permutation(n).astype(np.int64)
+    hk = torch.empty((n,) + tuple(kc.shape[1:]), dtype=t).pin_memory()
+    hv = torch.empty_like(hk).pin_memory()
+    out_pairs = torch.from_numpy(np.stack([ids, host_ids], 1)).to(dev)
+    in_pairs = torch.from_numpy(np.stack([host_ids, rng.permutation(ids)], 1)).to(dev)
+    block_bytes = kc[0].numel() * kc.element_size() * 2  # K and V of one block
+    total = n * block_bytes
+    flat_h = torch.empty(total, dtype=torch.uint8).pin_memory()
+    flat_d = torch.empty(total, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def timed(fn, reps):
+        for _ in range(args.warmup):
+            fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / reps
+
+    reps = max(3, min(args.steps, 50))
+    out_ms = timed(lambda: pa.pa_swap_blocks(kc, vc, hk, hv, out_pairs), reps)
+    in_ms = timed(lambda: pa.pa_swap_blocks(hk, hv, kc, vc, in_pairs), reps)
+    d2h_ms = timed(lambda: flat_h.copy_(flat_d, non_blocking=True), reps)
+    h2d_ms = timed(lambda: flat_d.copy_(flat_h, non_blocking=True), reps)
+    gbs = lambda ms: total / (ms * 1e-3) / 1e9
+    flags = pa.pa_get_device_error(clear=True)
+    if flags:
+        print(f"warning: device error word 0x{flags:x}", file=sys.stderr)
+    line = {"metric": "block swap GB/s (device <-> pinned host, pa_swap_blocks)",
+            "value": round(gbs((out_ms + in_ms) / 2), 2), "unit": "GB/s", "n_gpus": 1,
+            "steps": reps, "warmup": args.warmup, "higher_is_better": True,
+            "dtype": b.dtype, "data": "synthetic",
+            "config": dict(config, swapped_blocks=n, bytes_per_direction=total),
+            "swap_out": {"ms": round(out_ms, 4), "GBps": round(gbs(out_ms), 2),
+                         "link_GBps": round(gbs(d2h_ms), 2), "frac": round(d2h_ms / out_ms, 4)},
+            "swap_in": {"ms": round(in_ms, 4), "GBps": round(gbs(in_ms), 2),
+                        "link_GBps": round(gbs(h2d_ms), 2), "frac": round(h2d_ms / in_ms, 4)},
+            "roofline": {"bound": "host link", "peak_source": "cudaMemcpyAsync of one contiguous "
+                         "pinned buffer of the same bytes, same run"},
+            "gpu_launches": 2 * reps}
+    print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -527,6 +600,8 @@ def main():
     ap.add_argument("--soak", type=float, default=1.0, help="seconds of untimed load for the clock sampler")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--swap", action="store_true",
+                    help="measure block swap (pa_swap_blocks) of the workload's blocks instead")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("at least 3 warm-up steps")
@@ -555,6 +630,10 @@ def main():
     import torch
 
     torch.cuda.set_device(local_rank)
+    if args.swap:
+        if rank == 0:
+            run_swap(args, b, config)
+        return
     if world > 1:
         import datetime
 

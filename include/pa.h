@@ -62,7 +62,7 @@
 extern "C" {
 #endif
 
-#define PA_VERSION 2
+#define PA_VERSION 3
 
 /* Symbols of this ABI are the only ones the shared library exports. */
 #if defined(__GNUC__)
@@ -169,6 +169,25 @@ PA_API int pa_decode_step(const pa_tensor *key, const pa_tensor *value,
  */
 PA_API int pa_copy_blocks(const pa_tensor *key_cache, const pa_tensor *value_cache,
                    const pa_tensor *block_mapping, void *stream);
+
+/*
+ * pa_swap_blocks - move whole physical blocks between two caches, typically the device cache
+ * and a swap cache in pinned host memory ([P4] 2.3.2: blocks, not whole requests, are swapped
+ * out to CPU memory and back):
+ *   dst_key_cache[dst] = src_key_cache[src], dst_value_cache[dst] = src_value_cache[src]
+ * for each (src, dst) row of block_mapping [N, 2] int64 (src indexes the source caches, dst the
+ * destination caches).  Both cache pairs have the element type, kv heads, block_size and
+ * head_dim of the other; their block counts may differ.  Each tensor (the mapping included) is
+ * device memory of the current device or pinned host memory mapped into its address space
+ * (cudaHostAlloc / cudaMallocHost; the extent of host memory is not checked); pageable host
+ * memory returns PA_ERR_LAYOUT.  One kernel moves every block, 16 bytes per thread, so host
+ * memory is read or written directly over the host link.  Bit-exact.  Preconditions: dst ids
+ * distinct; the source and destination blocks do not overlap.  A pair with an id outside its
+ * cache sets PA_DEVERR_COPY_PAIR and is skipped.
+ */
+PA_API int pa_swap_blocks(const pa_tensor *src_key_cache, const pa_tensor *src_value_cache,
+                          const pa_tensor *dst_key_cache, const pa_tensor *dst_value_cache,
+                          const pa_tensor *block_mapping, void *stream);
 
 /*
  * pa_decode - one decode step of paged attention.  For every sequence s and query head h,

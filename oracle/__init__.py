@@ -69,6 +69,8 @@ class Oracle:
         lib.pao_reshape_and_cache.restype = _I32
         lib.pao_copy_blocks.argtypes = [_P, _P, _P, _I64, _I64, _I32, _I32, _I32, _I32]
         lib.pao_copy_blocks.restype = _I32
+        lib.pao_swap_blocks.argtypes = [_P, _P, _I64, _P, _P, _I64, _P, _I64, _I32, _I32, _I32, _I32]
+        lib.pao_swap_blocks.restype = _I32
         lib.pao_decode_range.argtypes = [
             _P, _P, _P, _P, _I32, _P, _P, _I32, _P, _I64, _P, _I64, _I32, _I32, _I32, _I32, _I64,
             _D, _I64, _I64, _I32,
@@ -103,6 +105,17 @@ class Oracle:
         return int(self._lib.pao_copy_blocks(
             _ptr(key_cache), _ptr(value_cache), _ptr(bm), bm.shape[0], nb, hkv, bs, d,
             DTYPE_CODE[dtype]))
+
+    def swap_blocks(self, src_key, src_value, dst_key, dst_value, block_mapping, dtype: str) -> int:
+        """Move whole blocks dst pool[dst] <- src pool[src].  Returns skipped-pair count."""
+        snb, hkv, bs, d = src_key.shape
+        dnb = dst_key.shape[0]
+        if dst_key.shape[1:] != src_key.shape[1:]:
+            raise ValueError("pools differ in block shape")
+        bm = np.ascontiguousarray(block_mapping, dtype=np.int64).reshape(-1, 2)
+        return int(self._lib.pao_swap_blocks(
+            _ptr(src_key), _ptr(src_value), snb, _ptr(dst_key), _ptr(dst_value), dnb, _ptr(bm),
+            bm.shape[0], hkv, bs, d, DTYPE_CODE[dtype]))
 
     def decode_range(self, query, key_cache, value_cache, block_tables, context_lens, scale,
                      dtype: str, t_begin: int, t_end: int, q_dtype: str | None = None,

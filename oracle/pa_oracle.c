@@ -154,6 +154,37 @@ int pao_copy_blocks(void *key_cache, void *value_cache, const int64_t *block_map
 }
 
 /*
+ * Move whole physical blocks between two pools of the same block shape: dst pool block dst <-
+ * src pool block src, keys and values, for each (src, dst) pair ([P4] 2.3.2: the scheduler
+ * swaps KV cache out block by block, to CPU memory, and back in).  src_blocks and dst_blocks
+ * are the two pools' block counts.  Returns the number of pairs skipped because an id lies
+ * outside its pool.
+ */
+int pao_swap_blocks(const void *src_key, const void *src_value, int64_t src_blocks,
+                    void *dst_key, void *dst_value, int64_t dst_blocks,
+                    const int64_t *block_mapping, int64_t num_pairs, int num_kv_heads,
+                    int block_size, int head_dim, int dtype) {
+  if (num_pairs < 0 || src_blocks < 0 || dst_blocks < 0 || num_kv_heads <= 0 || block_size <= 0 ||
+      head_dim <= 0)
+    return PAO_BAD_ARG;
+  const size_t block_bytes =
+      (size_t)num_kv_heads * (size_t)block_size * (size_t)head_dim * elt_size(dtype);
+  int skipped = 0;
+  for (int64_t p = 0; p < num_pairs; ++p) {
+    const int64_t src = block_mapping[2 * p], dst = block_mapping[2 * p + 1];
+    if (src < 0 || src >= src_blocks || dst < 0 || dst >= dst_blocks) {
+      ++skipped;
+      continue;
+    }
+    memcpy((char *)dst_key + (size_t)dst * block_bytes,
+           (const char *)src_key + (size_t)src * block_bytes, block_bytes);
+    memcpy((char *)dst_value + (size_t)dst * block_bytes,
+           (const char *)src_value + (size_t)src * block_bytes, block_bytes);
+  }
+  return skipped;
+}
+
+/*
  * Assemble the first `len` tokens of one sequence's keys and values for kv head g into
  * contiguous rows kc[t][d], vc[t][d] ([P4] 2.2.2: look up the physical block of each logical
  * block in the block table, then read K/V from the physical cache).

@@ -75,6 +75,7 @@ def load(path: str = LIBRARY) -> ctypes.CDLL:
     i32, u32, i64, sz, f32 = ctypes.c_int32, ctypes.c_uint32, ctypes.c_int64, ctypes.c_size_t, ctypes.c_float
     lib.pa_reshape_and_cache.argtypes = [_T, _T, _T, _T, _T, _P]
     lib.pa_copy_blocks.argtypes = [_T, _T, _T, _P]
+    lib.pa_swap_blocks.argtypes = [_T, _T, _T, _T, _T, _P]
     lib.pa_decode.argtypes = [_T, _T, _T, _T, _T, _T, f32, i32, i32, _P]
     lib.pa_decode_ex.argtypes = [_T, _T, _T, _T, _T, _T, f32, i32, i32, i32, u32, _P, sz, _P]
     lib.pa_decode_workspace_bytes.argtypes = [i64, i32, i32, i32, i32]
@@ -149,6 +150,16 @@ def pa_copy_blocks(key_cache, value_cache, block_mapping, stream=None):
     lib = load()
     d = [describe(x) for x in (key_cache, value_cache, block_mapping)]
     _check("pa_copy_blocks", lib.pa_copy_blocks(*[ctypes.byref(x) for x in d], _stream(stream)))
+
+
+def pa_swap_blocks(src_key_cache, src_value_cache, dst_key_cache, dst_value_cache, block_mapping,
+                   stream=None):
+    """Move whole blocks dst <- src between two caches, e.g. device memory and pinned host
+    memory (torch tensors created with pin_memory=True)."""
+    lib = load()
+    d = [describe(x) for x in (src_key_cache, src_value_cache, dst_key_cache, dst_value_cache,
+                               block_mapping)]
+    _check("pa_swap_blocks", lib.pa_swap_blocks(*[ctypes.byref(x) for x in d], _stream(stream)))
 
 
 def pa_decode(out, query, key_cache, value_cache, block_tables, context_lens, scale, block_size,

@@ -616,6 +616,81 @@ int write_impl(const pa_tensor *key, const pa_tensor *value, const pa_tensor *ke
   return err == cudaSuccess ? PA_OK : cuda_fail(err, "reshape_and_cache launch");
 }
 
+// Device address through which a kernel on `dev` reaches t's data: device (or managed) memory
+// of that device, or pinned host memory mapped into the device's address space.  Pageable
+// host memory is refused.  The extent is checked for device allocations only.
+int device_address(const pa_tensor *t, const char *name, int dev, void **addr) {
+  *addr = t->data;
+  if (extent_bytes(t) == 0) return PA_OK;
+  if (!t->data) return fail(PA_ERR_INVALID_ARG, "%s: NULL data pointer", name);
+  cudaPointerAttributes attr;
+  cudaError_t e = cudaPointerGetAttributes(&attr, t->data);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return fail(PA_ERR_LAYOUT, "%s: not a CUDA pointer (%s)", name, cudaGetErrorString(e));
+  }
+  if (attr.type == cudaMemoryTypeHost) {
+    if (!attr.devicePointer)
+      return fail(PA_ERR_LAYOUT, "%s: pinned host memory not mapped into the device", name);
+    *addr = attr.devicePointer;
+    return PA_OK;
+  }
+  return check_device_memory(t, name, dev);
+}
+
+int copy_blocks_impl(const pa_tensor *src_k, const pa_tensor *src_v, const pa_tensor *dst_k,
+                     const pa_tensor *dst_v, const pa_tensor *block_mapping, bool host_allowed,
+                     void *stream) {
+  int rc;
+  CacheShape s, d;
+  if ((rc = check_caches(src_k, src_v, &s))) return rc;
+  if ((rc = check_caches(dst_k, dst_v, &d))) return rc;
+  if (s.dtype != d.dtype || s.num_kv_heads != d.num_kv_heads || s.block_size != d.block_size ||
+      s.head_dim != d.head_dim)
+    return fail(PA_ERR_SHAPE, "source and destination caches differ in element type or block shape");
+  if ((rc = check_tensor(block_mapping, "block_mapping", 2))) return rc;
+  if (block_mapping->dtype != PA_I64) return fail(PA_ERR_DTYPE, "block_mapping must be int64");
+  if (block_mapping->shape[1] != 2) return fail(PA_ERR_SHAPE, "block_mapping must be [num_pairs, 2]");
+  const int64_t N = block_mapping->shape[0];
+  if (N > 1 && block_mapping->stride[0] != 2) return fail(PA_ERR_LAYOUT, "block_mapping must be contiguous");
+  if (block_mapping->stride[1] != 1) return fail(PA_ERR_LAYOUT, "block_mapping must be contiguous");
+  const size_t e = elt_size(s.dtype);
+  if ((s.block_size * s.head_dim * e) % 16 != 0)
+    return fail(PA_ERR_UNSUPPORTED, "block tile must be a multiple of 16 bytes");
+  if (N == 0) return PA_OK;
+  DeviceState *ds;
+  int dev;
+  if ((rc = device_state(&ds, &dev))) return rc;
+  void *p[5];
+  const pa_tensor *ts[5] = {src_k, src_v, dst_k, dst_v, block_mapping};
+  const char *names[5] = {"source key cache", "source value cache", "destination key cache",
+                          "destination value cache", "block_mapping"};
+  for (int i = 0; i < 5; ++i) {
+    rc = host_allowed ? device_address(ts[i], names[i], dev, &p[i])
+                      : check_device_memory(ts[i], names[i], dev);
+    if (!host_allowed) p[i] = ts[i]->data;
+    if (rc) return rc;
+  }
+  pa::CopyBlocksArgs a;
+  a.src_key = static_cast<const char *>(p[0]);
+  a.src_value = static_cast<const char *>(p[1]);
+  a.dst_key = static_cast<char *>(p[2]);
+  a.dst_value = static_cast<char *>(p[3]);
+  a.src_blk = src_k->stride[0] * (int64_t)e;
+  a.src_head = src_k->stride[1] * (int64_t)e;
+  a.dst_blk = dst_k->stride[0] * (int64_t)e;
+  a.dst_head = dst_k->stride[1] * (int64_t)e;
+  a.tile_bytes = (int)(s.block_size * s.head_dim * e);
+  a.pairs = static_cast<const int64_t *>(p[4]);
+  a.num_pairs = N;
+  a.num_kv_heads = s.num_kv_heads;
+  a.src_blocks = s.num_blocks;
+  a.dst_blocks = d.num_blocks;
+  a.err = ds->err;
+  cudaError_t err = pa::launch_copy_blocks(a, ds->num_sms, static_cast<cudaStream_t>(stream));
+  return err == cudaSuccess ? PA_OK : cuda_fail(err, host_allowed ? "swap_blocks launch" : "copy_blocks launch");
+}
+
 }  // namespace
 
 extern "C" {
@@ -648,38 +723,15 @@ int pa_decode_step(const pa_tensor *key, const pa_tensor *value, const pa_tensor
 
 int pa_copy_blocks(const pa_tensor *key_cache, const pa_tensor *value_cache,
                    const pa_tensor *block_mapping, void *stream) {
-  int rc;
-  CacheShape cs;
-  if ((rc = check_caches(key_cache, value_cache, &cs))) return rc;
-  if ((rc = check_tensor(block_mapping, "block_mapping", 2))) return rc;
-  if (block_mapping->dtype != PA_I64) return fail(PA_ERR_DTYPE, "block_mapping must be int64");
-  if (block_mapping->shape[1] != 2) return fail(PA_ERR_SHAPE, "block_mapping must be [num_pairs, 2]");
-  const int64_t N = block_mapping->shape[0];
-  if (N > 1 && block_mapping->stride[0] != 2) return fail(PA_ERR_LAYOUT, "block_mapping must be contiguous");
-  if (block_mapping->stride[1] != 1) return fail(PA_ERR_LAYOUT, "block_mapping must be contiguous");
-  if (N == 0) return PA_OK;
-  DeviceState *ds;
-  int dev;
-  if ((rc = device_state(&ds, &dev))) return rc;
-  if ((rc = check_device_memory(key_cache, "key_cache", dev)) ||
-      (rc = check_device_memory(value_cache, "value_cache", dev)) ||
-      (rc = check_device_memory(block_mapping, "block_mapping", dev)))
-    return rc;
-  const size_t e = elt_size(cs.dtype);
-  pa::CopyBlocksArgs a;
-  a.key_cache = static_cast<char *>(key_cache->data);
-  a.value_cache = static_cast<char *>(value_cache->data);
-  a.c_blk = key_cache->stride[0] * (int64_t)e;
-  a.c_head = key_cache->stride[1] * (int64_t)e;
-  a.tile_bytes = (int)(cs.block_size * cs.head_dim * e);
-  a.pairs = static_cast<const int64_t *>(block_mapping->data);
-  a.num_pairs = N;
-  a.num_kv_heads = cs.num_kv_heads;
-  a.num_blocks = cs.num_blocks;
-  a.err = ds->err;
-  if (a.tile_bytes % 16 != 0) return fail(PA_ERR_UNSUPPORTED, "block tile must be a multiple of 16 bytes");
-  cudaError_t err = pa::launch_copy_blocks(a, ds->num_sms, static_cast<cudaStream_t>(stream));
-  return err == cudaSuccess ? PA_OK : cuda_fail(err, "copy_blocks launch");
+  return copy_blocks_impl(key_cache, value_cache, key_cache, value_cache, block_mapping, false,
+                          stream);
+}
+
+int pa_swap_blocks(const pa_tensor *src_key_cache, const pa_tensor *src_value_cache,
+                   const pa_tensor *dst_key_cache, const pa_tensor *dst_value_cache,
+                   const pa_tensor *block_mapping, void *stream) {
+  return copy_blocks_impl(src_key_cache, src_value_cache, dst_key_cache, dst_value_cache,
+                          block_mapping, true, stream);
 }
 
 int pa_decode(const pa_tensor *out, const pa_tensor *query, const pa_tensor *key_cache,

@@ -45,7 +45,9 @@ __global__ void __launch_bounds__(256) reshape_and_cache_kernel(CacheWriteArgs a
   }
 }
 
-// One thread per 16-byte piece of one (pair, kv head) tile, keys and values together.
+// One thread per 16-byte piece of one (pair, kv head) tile, keys and values together.  Source
+// and destination caches may be the same tensors (copy-on-write) or live in different memory
+// (swap between device memory and pinned host memory mapped into the device's address space).
 __global__ void __launch_bounds__(256) copy_blocks_kernel(CopyBlocksArgs a) {
   const int vec_per_tile = a.tile_bytes >> 4;
   const int64_t total = a.num_pairs * a.num_kv_heads * vec_per_tile;
@@ -57,16 +59,16 @@ __global__ void __launch_bounds__(256) copy_blocks_kernel(CopyBlocksArgs a) {
     const int64_t p = ph / a.num_kv_heads;
     const int64_t src = __ldg(a.pairs + 2 * p);
     const int64_t dst = __ldg(a.pairs + 2 * p + 1);
-    if (src < 0 || src >= a.num_blocks || dst < 0 || dst >= a.num_blocks) {
+    if (src < 0 || src >= a.src_blocks || dst < 0 || dst >= a.dst_blocks) {
       if (h == 0 && v == 0) set_error(a.err, PA_DEVERR_COPY_PAIR);
       continue;
     }
-    const int64_t so = src * a.c_blk + h * a.c_head + (int64_t)v * 16;
-    const int64_t d = dst * a.c_blk + h * a.c_head + (int64_t)v * 16;
-    const uint4 kv = *reinterpret_cast<const uint4 *>(a.key_cache + so);
-    const uint4 vv = *reinterpret_cast<const uint4 *>(a.value_cache + so);
-    *reinterpret_cast<uint4 *>(a.key_cache + d) = kv;
-    *reinterpret_cast<uint4 *>(a.value_cache + d) = vv;
+    const int64_t so = src * a.src_blk + h * a.src_head + (int64_t)v * 16;
+    const int64_t d = dst * a.dst_blk + h * a.dst_head + (int64_t)v * 16;
+    const uint4 kv = *reinterpret_cast<const uint4 *>(a.src_key + so);
+    const uint4 vv = *reinterpret_cast<const uint4 *>(a.src_value + so);
+    *reinterpret_cast<uint4 *>(a.dst_key + d) = kv;
+    *reinterpret_cast<uint4 *>(a.dst_value + d) = vv;
   }
 }
 

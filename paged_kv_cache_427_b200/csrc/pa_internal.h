@@ -83,15 +83,18 @@ struct CacheWriteArgs {
   unsigned int *err;
 };
 
+// Whole-block copies from one pair of caches to another (the same pair for copy-on-write,
+// device and pinned host memory for swapping).
 struct CopyBlocksArgs {
-  char *key_cache;
-  char *value_cache;
-  int64_t c_blk, c_head;  // bytes
-  int tile_bytes;         // block_size * row bytes: one (block, kv head) tile
+  const char *src_key, *src_value;
+  char *dst_key, *dst_value;
+  int64_t src_blk, src_head;  // bytes
+  int64_t dst_blk, dst_head;  // bytes
+  int tile_bytes;             // block_size * row bytes: one (block, kv head) tile
   const int64_t *pairs;
   int64_t num_pairs;
   int num_kv_heads;
-  int64_t num_blocks;
+  int64_t src_blocks, dst_blocks;
   unsigned int *err;
 };
 

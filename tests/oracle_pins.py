@@ -337,6 +337,54 @@ def pin_copy_blocks(orc):
     assert np.array_equal(kc, k1)
 
 
+def pin_swap_blocks(orc):
+    """Block-level swap ([P4] 2.3.2): blocks copied to a second pool equal their sources and
+    nothing else there changes; a sequence swapped out, its device blocks overwritten, and
+    swapped back into other free blocks (table updated) decodes to the same bits; ids outside
+    either pool are refused."""
+    b = W.build_batch("swap", [30, 50, 17], num_heads=8, num_kv_heads=2, head_dim=64,
+                      block_size=8, dtype="bf16", seed=W.BASE_SEED + 705, pool_factor=3.0)
+    orc.reshape_and_cache(b.key, b.value, b.key_cache, b.value_cache, b.slot_mapping, b.dtype)
+    kc, vc = b.key_cache, b.value_cache
+    nb = kc.shape[0]
+    rng = np.random.default_rng(11)
+    nh = nb + 16  # host pool larger than the device pool: every id below stays inside both
+    hk = W.encode(rng.standard_normal((nh,) + kc.shape[1:]).astype(np.float32), "bf16")
+    hv = W.encode(rng.standard_normal((nh,) + kc.shape[1:]).astype(np.float32), "bf16")
+    before = orc.decode(b.query, kc, vc, b.block_tables, b.context_lens, b.scale, b.dtype)
+
+    s = 1
+    nblk = -(-int(b.context_lens[s]) // b.block_size)
+    dev_ids = b.block_tables[s, :nblk].astype(np.int64)
+    host_ids = rng.permutation(nb)[:nblk].astype(np.int64)  # below nb
+    hk0, hv0 = hk.copy(), hv.copy()
+    out_pairs = np.stack([dev_ids, host_ids], 1)
+    assert orc.swap_blocks(kc, vc, hk, hv, out_pairs, "bf16") == 0
+    for src, dst in out_pairs:
+        assert np.array_equal(hk[dst], kc[src]) and np.array_equal(hv[dst], vc[src])
+    for blk in set(range(nh)) - set(host_ids.tolist()):
+        assert np.array_equal(hk[blk], hk0[blk]) and np.array_equal(hv[blk], hv0[blk])
+
+    # the device blocks are reused by someone else; the sequence comes back elsewhere
+    kc[dev_ids] = W.encode(np.full(kc[dev_ids].shape, np.nan, np.float32), "bf16")
+    vc[dev_ids] = W.encode(np.full(vc[dev_ids].shape, np.nan, np.float32), "bf16")
+    used = set()
+    for q in range(b.num_seqs):
+        used |= set(b.block_tables[q, :-(-int(b.context_lens[q]) // b.block_size)].tolist())
+    free = np.array(sorted(set(range(nb)) - used), np.int64)
+    new_ids = rng.permutation(free)[:nblk]
+    assert orc.swap_blocks(hk, hv, kc, vc, np.stack([host_ids, new_ids], 1), "bf16") == 0
+    tables = b.block_tables.copy()
+    tables[s, :nblk] = new_ids
+    after = orc.decode(b.query, kc, vc, tables, b.context_lens, b.scale, b.dtype)
+    assert np.array_equal(after, before)
+
+    k1, h1 = kc.copy(), hk.copy()
+    bad_out = np.array([[0, nh], [nb, 0], [-1, 3]], np.int64)
+    assert orc.swap_blocks(kc, vc, hk, hv, bad_out, "bf16") == 3
+    assert np.array_equal(hk, h1) and np.array_equal(kc, k1)
+
+
 def pin_shared_prefix(orc):
     """Sequences sharing prefix blocks read the same bytes: the paged result over the shared
     pool equals brute force on each member's own logical stream."""
@@ -377,5 +425,5 @@ def pin_zero_context(orc):
 ALL_PINS = [
     pin_brute_force, pin_torch_sdpa, pin_closed_forms, pin_decimal_example,
     pin_placement_invariance, pin_unread_table_entries, pin_cache_write, pin_copy_blocks,
-    pin_shared_prefix, pin_split_merge, pin_zero_context,
+    pin_swap_blocks, pin_shared_prefix, pin_split_merge, pin_zero_context,
 ]

@@ -41,6 +41,13 @@ MUTANTS = {
         "           (const char *)key_cache + (size_t)src * block_bytes, block_bytes);",
         "memcpy((char *)key_cache + (size_t)src * block_bytes,\n"
         "           (const char *)key_cache + (size_t)dst * block_bytes, block_bytes);"),
+    "swap_value_from_key": (
+        "memcpy((char *)dst_value + (size_t)dst * block_bytes,\n"
+        "           (const char *)src_value + (size_t)src * block_bytes, block_bytes);",
+        "memcpy((char *)dst_value + (size_t)dst * block_bytes,\n"
+        "           (const char *)src_key + (size_t)src * block_bytes, block_bytes);"),
+    "swap_dst_index": ("memcpy((char *)dst_key + (size_t)dst * block_bytes,",
+                       "memcpy((char *)dst_key + (size_t)src * block_bytes,"),
     "bf16_shift": ("uint32_t u = (uint32_t)h << 16;", "uint32_t u = (uint32_t)h << 15;"),
     "f16_bias": ("v = ldexp((double)(m | 0x400), e - 25);", "v = ldexp((double)(m | 0x400), e - 24);"),
     "merge_sign": ("const double w = l[p] * exp(m[p] - big_m);",
