@@ -25,8 +25,8 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 SOURCE = os.path.join(_HERE, "pa_oracle.c")
 LIBRARY = os.path.join(_HERE, "libpa_oracle.so")
 
-DTYPE_CODE = {"f32": 0, "bf16": 1, "f16": 2}
-ELT_BYTES = {"f32": 4, "bf16": 2, "f16": 2}
+DTYPE_CODE = {"f32": 0, "bf16": 1, "f16": 2, "fp8": 3}
+ELT_BYTES = {"f32": 4, "bf16": 2, "f16": 2, "fp8": 1}
 
 _P = ctypes.c_void_p
 _I64 = ctypes.c_int64
@@ -76,6 +76,15 @@ class Oracle:
             _D, _I64, _I64, _I32,
         ]
         lib.pao_decode_range.restype = _I32
+        lib.pao_decode_range_scaled.argtypes = lib.pao_decode_range.argtypes + [_P, _P]
+        lib.pao_decode_range_scaled.restype = _I32
+        lib.pao_fp8_encode.argtypes = [_P, _I32, _I64, ctypes.c_float, _P]
+        lib.pao_fp8_encode.restype = None
+        lib.pao_fp8_decode.argtypes = [_P, _I64, _P]
+        lib.pao_fp8_decode.restype = None
+        lib.pao_reshape_and_cache_fp8.argtypes = [_P, _P, _I32, _P, _P, _P, _I64, _I64, _I32, _I32,
+                                                  _I32, _P, _P]
+        lib.pao_reshape_and_cache_fp8.restype = _I32
         lib.pao_lse_combine.argtypes = [_P, _P, _P, _P, _I64, _I32]
         lib.pao_lse_combine.restype = None
         lib.pao_max_threads.argtypes = []
@@ -117,10 +126,41 @@ class Oracle:
             _ptr(src_key), _ptr(src_value), snb, _ptr(dst_key), _ptr(dst_value), dnb, _ptr(bm),
             bm.shape[0], hkv, bs, d, DTYPE_CODE[dtype]))
 
+    def fp8_encode(self, x, dtype: str, scale: float) -> np.ndarray:
+        """FP8 E4M3 codes of x / scale (x of element type dtype, divided in fp32)."""
+        raw = _raw(x, dtype)
+        out = np.empty(raw.shape, dtype=np.uint8)
+        self._lib.pao_fp8_encode(_ptr(raw), DTYPE_CODE[dtype], raw.size, float(scale), _ptr(out))
+        return out
+
+    def fp8_decode(self, codes) -> np.ndarray:
+        c = np.ascontiguousarray(codes, dtype=np.uint8)
+        out = np.empty(c.shape, dtype=np.float64)
+        self._lib.pao_fp8_decode(_ptr(c), c.size, _ptr(out))
+        return out
+
+    def reshape_and_cache_fp8(self, key, value, dtype: str, key_cache, value_cache, slot_mapping,
+                              k_scale, v_scale) -> int:
+        """Quantise new tokens' K/V rows (element type dtype) into FP8 caches in place, kv head
+        h with k_scale[h] / v_scale[h].  Returns skipped-token count."""
+        nb, hkv, bs, d = key_cache.shape
+        for c in (key_cache, value_cache):
+            if not c.flags.c_contiguous or c.dtype != np.uint8:
+                raise ValueError("FP8 caches must be C-contiguous uint8 (written in place)")
+        key = _raw(key, dtype)
+        value = _raw(value, dtype)
+        slots = np.ascontiguousarray(slot_mapping, dtype=np.int64)
+        ks = np.ascontiguousarray(k_scale, dtype=np.float32)
+        vs = np.ascontiguousarray(v_scale, dtype=np.float32)
+        return int(self._lib.pao_reshape_and_cache_fp8(
+            _ptr(key), _ptr(value), DTYPE_CODE[dtype], _ptr(key_cache), _ptr(value_cache),
+            _ptr(slots), slots.shape[0], nb, hkv, bs, d, _ptr(ks), _ptr(vs)))
+
     def decode_range(self, query, key_cache, value_cache, block_tables, context_lens, scale,
                      dtype: str, t_begin: int, t_end: int, q_dtype: str | None = None,
-                     num_threads: int = 0):
-        """Attention restricted to context positions [t_begin, t_end).
+                     num_threads: int = 0, k_scale=None, v_scale=None):
+        """Attention restricted to context positions [t_begin, t_end).  With k_scale/v_scale
+        ([Hkv] fp32) the keys and values of kv head g are multiplied by them (FP8 caches).
 
         Returns (out [S,Hq,D] float64, m [S,Hq] float64, l [S,Hq] float64).
         """
@@ -137,20 +177,24 @@ class Oracle:
         out = np.empty((s, hq, d), dtype=np.float64)
         m = np.empty((s, hq), dtype=np.float64)
         l = np.empty((s, hq), dtype=np.float64)
-        rc = self._lib.pao_decode_range(
+        ks = None if k_scale is None else np.ascontiguousarray(k_scale, dtype=np.float32)
+        vs = None if v_scale is None else np.ascontiguousarray(v_scale, dtype=np.float32)
+        rc = self._lib.pao_decode_range_scaled(
             _ptr(out), _ptr(m), _ptr(l), _ptr(q), DTYPE_CODE[q_dtype], _ptr(kc), _ptr(vc),
             DTYPE_CODE[dtype], _ptr(bt), bt.shape[1] if bt.ndim == 2 else 0, _ptr(cl), s, hq, hkv,
-            d, bs, nb, float(scale), int(t_begin), int(t_end), int(num_threads))
+            d, bs, nb, float(scale), int(t_begin), int(t_end), int(num_threads),
+            None if ks is None else _ptr(ks), None if vs is None else _ptr(vs))
         if rc != 0:
             raise ValueError(f"oracle decode failed with status {rc}")
         return out, m, l
 
     def decode(self, query, key_cache, value_cache, block_tables, context_lens, scale,
-               dtype: str, q_dtype: str | None = None, num_threads: int = 0) -> np.ndarray:
+               dtype: str, q_dtype: str | None = None, num_threads: int = 0, k_scale=None,
+               v_scale=None) -> np.ndarray:
         """softmax(scale * q K^T) V over each sequence's whole context: [S, Hq, D] float64."""
         out, _, _ = self.decode_range(query, key_cache, value_cache, block_tables, context_lens,
                                       scale, dtype, 0, np.iinfo(np.int64).max, q_dtype,
-                                      num_threads)
+                                      num_threads, k_scale, v_scale)
         return out
 
     def lse_combine(self, o_parts, m, l) -> np.ndarray:

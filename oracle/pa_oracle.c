@@ -36,8 +36,16 @@
  *   - A context length of 0 gives an all-zero output row.
  *   - A negative slot in slot_mapping means "store nothing" (a padding token).
  *
- * Element types: 0 = fp32, 1 = bf16 (upper half of an fp32), 2 = IEEE binary16.  Elements are
- * widened exactly to double before any arithmetic; all arithmetic is in double.
+ * Element types: 0 = fp32, 1 = bf16 (upper half of an fp32), 2 = IEEE binary16, 3 = FP8 E4M3
+ * (cache only).  Elements are widened exactly to double before any arithmetic; all arithmetic
+ * is in double, except the quantisation to FP8, which divides in fp32 (the precision the write
+ * kernel decides the code in).
+ *
+ * FP8 KV cache ([P2] 4.3 lists FP8 E4M3, 8-bit floating point, ~50 % memory, as a supported
+ * storage format; using it for the KV cache with one fp32 scale per kv head is this build's
+ * reading): the cache holds code(x / scale[h]) and the attention reads decode(code) * scale[h].
+ * E4M3: 1 sign bit, 4 exponent bits (bias 7), 3 fraction bits; exponent 0 is subnormal
+ * (m * 2^-9); S.1111.111 is NaN; no infinities; the largest finite magnitude is 448.
  */
 #include <math.h>
 #include <stdint.h>
@@ -47,7 +55,7 @@
 #include <omp.h>
 #endif
 
-enum { PAO_F32 = 0, PAO_BF16 = 1, PAO_F16 = 2 };
+enum { PAO_F32 = 0, PAO_BF16 = 1, PAO_F16 = 2, PAO_FP8 = 3 };
 
 enum {
   PAO_OK = 0,
@@ -57,7 +65,45 @@ enum {
   PAO_NO_MEMORY = -4
 };
 
-static size_t elt_size(int dtype) { return dtype == PAO_F32 ? 4u : 2u; }
+static size_t elt_size(int dtype) { return dtype == PAO_F32 ? 4u : (dtype == PAO_FP8 ? 1u : 2u); }
+
+/* Value of one FP8 E4M3 code. */
+static double fp8_to_double(uint8_t c) {
+  const int sign = c >> 7, e = (c >> 3) & 0xf, m = c & 7;
+  double v;
+  if (e == 15 && m == 7)
+    v = NAN;
+  else if (e == 0)
+    v = ldexp((double)m, -9); /* subnormal: m/8 * 2^(1-7) */
+  else
+    v = ldexp((double)(8 + m), e - 10); /* (1 + m/8) * 2^(e-7) */
+  return sign ? -v : v;
+}
+
+/* The E4M3 code nearest to x, ties to the even code, magnitudes of 448 and above saturated to
+ * 448, NaN to the NaN code 0x7f. */
+static uint8_t double_to_fp8(double x) {
+  if (isnan(x)) return 0x7f;
+  const uint8_t sign = signbit(x) ? 0x80 : 0;
+  const double a = fabs(x);
+  if (a >= 448.0) return sign | 0x7e;
+  int code;
+  if (a < ldexp(1.0, -6)) {
+    code = (int)rint(a * 512.0); /* subnormal lattice m * 2^-9; 8 is the smallest normal */
+  } else {
+    int ex;
+    frexp(a, &ex); /* a = f * 2^ex, f in [0.5, 1): exponent of the leading bit ex - 1 */
+    const int e = ex - 1;
+    int m = (int)rint((ldexp(a, -e) - 1.0) * 8.0);
+    int be = e + 7;
+    if (m == 8) {
+      m = 0;
+      ++be;
+    }
+    code = (be << 3) | m; /* at most 0x7e: a < 448 */
+  }
+  return sign | (uint8_t)code;
+}
 
 /* Widen element idx of a buffer of the given element type to double (exact for all three). */
 static double elt_to_double(const void *base, size_t idx, int dtype) {
@@ -66,6 +112,7 @@ static double elt_to_double(const void *base, size_t idx, int dtype) {
     memcpy(&f, (const char *)base + idx * 4u, 4u);
     return (double)f;
   }
+  if (dtype == PAO_FP8) return fp8_to_double(((const uint8_t *)base)[idx]);
   uint16_t h;
   memcpy(&h, (const char *)base + idx * 2u, 2u);
   if (dtype == PAO_BF16) {
@@ -119,6 +166,57 @@ int pao_reshape_and_cache(const void *key, const void *value, void *key_cache, v
           row;
       memcpy((char *)key_cache + dst, (const char *)key + src, row);
       memcpy((char *)value_cache + dst, (const char *)value + src, row);
+    }
+  }
+  return skipped;
+}
+
+/*
+ * FP8 codes of n elements of src (element type src_dtype), each divided by `scale` in fp32
+ * first: out[i] = code((float)src[i] / scale).
+ */
+void pao_fp8_encode(const void *src, int src_dtype, int64_t n, float scale, uint8_t *out) {
+  for (int64_t i = 0; i < n; ++i) {
+    const float x = (float)elt_to_double(src, (size_t)i, src_dtype);
+    const float q = x / scale;
+    out[i] = double_to_fp8((double)q);
+  }
+}
+
+/* The values of n FP8 codes. */
+void pao_fp8_decode(const uint8_t *codes, int64_t n, double *out) {
+  for (int64_t i = 0; i < n; ++i) out[i] = fp8_to_double(codes[i]);
+}
+
+/*
+ * Write side of an FP8 cache: like pao_reshape_and_cache, the rows of kv head h quantised
+ * with k_scale[h] (keys) and v_scale[h] (values) on the way in.  key, value have element type
+ * src_dtype; the caches hold one code per element.
+ */
+int pao_reshape_and_cache_fp8(const void *key, const void *value, int src_dtype, uint8_t *key_cache,
+                              uint8_t *value_cache, const int64_t *slot_mapping, int64_t num_tokens,
+                              int64_t num_blocks, int num_kv_heads, int block_size, int head_dim,
+                              const float *k_scale, const float *v_scale) {
+  if (num_tokens < 0 || num_blocks < 0 || num_kv_heads <= 0 || block_size <= 0 || head_dim <= 0)
+    return PAO_BAD_ARG;
+  const size_t es = elt_size(src_dtype);
+  int skipped = 0;
+  for (int64_t i = 0; i < num_tokens; ++i) {
+    const int64_t slot = slot_mapping[i];
+    if (slot < 0) continue; /* a padding token stores nothing */
+    if (slot >= num_blocks * (int64_t)block_size) {
+      ++skipped;
+      continue;
+    }
+    const int64_t blk = slot / block_size, off = slot % block_size;
+    for (int h = 0; h < num_kv_heads; ++h) {
+      const size_t srow = ((size_t)i * (size_t)num_kv_heads + (size_t)h) * (size_t)head_dim;
+      const size_t drow =
+          (((size_t)blk * (size_t)num_kv_heads + (size_t)h) * (size_t)block_size + (size_t)off) *
+          (size_t)head_dim;
+      pao_fp8_encode((const char *)key + srow * es, src_dtype, head_dim, k_scale[h], key_cache + drow);
+      pao_fp8_encode((const char *)value + srow * es, src_dtype, head_dim, v_scale[h],
+                     value_cache + drow);
     }
   }
   return skipped;
@@ -256,12 +354,17 @@ static void attend_rows(double *o, double *m_out, double *l_out, const double *q
  *   query    [num_seqs][num_heads][head_dim]  q_dtype
  *   block_tables [num_seqs][max_blocks] int32, context_lens [num_seqs] int32
  */
-int pao_decode_range(double *out, double *m_out, double *l_out, const void *query, int q_dtype,
-                     const void *key_cache, const void *value_cache, int kv_dtype,
-                     const int32_t *block_tables, int64_t max_blocks, const int32_t *context_lens,
-                     int64_t num_seqs, int num_heads, int num_kv_heads, int head_dim,
-                     int block_size, int64_t num_blocks, double scale, int64_t t_begin,
-                     int64_t t_end, int num_threads) {
+/*
+ * As pao_decode_range, with the keys and values of kv head g multiplied by k_scale[g] and
+ * v_scale[g] (either may be NULL: 1) after they are read: the attention of an FP8 cache.
+ */
+int pao_decode_range_scaled(double *out, double *m_out, double *l_out, const void *query,
+                            int q_dtype, const void *key_cache, const void *value_cache,
+                            int kv_dtype, const int32_t *block_tables, int64_t max_blocks,
+                            const int32_t *context_lens, int64_t num_seqs, int num_heads,
+                            int num_kv_heads, int head_dim, int block_size, int64_t num_blocks,
+                            double scale, int64_t t_begin, int64_t t_end, int num_threads,
+                            const float *k_scale, const float *v_scale) {
   if (num_seqs < 0 || num_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0 ||
       max_blocks < 0 || num_heads % num_kv_heads != 0)
     return PAO_BAD_ARG;
@@ -304,6 +407,12 @@ int pao_decode_range(double *out, double *m_out, double *l_out, const void *quer
             status = rc;
             for (int d = 0; d < head_dim; ++d) o[d] = NAN;
           } else {
+            const double ks = k_scale ? (double)k_scale[g] : 1.0;
+            const double vs = v_scale ? (double)v_scale[g] : 1.0;
+            for (size_t i = 0; i < (size_t)t1 * (size_t)head_dim; ++i) {
+              kc[i] *= ks;
+              vc[i] *= vs;
+            }
             const size_t qrow = ((size_t)s * (size_t)num_heads + (size_t)h) * (size_t)head_dim;
             for (int d = 0; d < head_dim; ++d) q[d] = elt_to_double(query, qrow + (size_t)d, q_dtype);
             attend_rows(o, &m, &l, q, kc, vc, t0, t1, head_dim, scale, z);
@@ -319,6 +428,18 @@ int pao_decode_range(double *out, double *m_out, double *l_out, const void *quer
     }
   }
   return status;
+}
+
+int pao_decode_range(double *out, double *m_out, double *l_out, const void *query, int q_dtype,
+                     const void *key_cache, const void *value_cache, int kv_dtype,
+                     const int32_t *block_tables, int64_t max_blocks, const int32_t *context_lens,
+                     int64_t num_seqs, int num_heads, int num_kv_heads, int head_dim,
+                     int block_size, int64_t num_blocks, double scale, int64_t t_begin,
+                     int64_t t_end, int num_threads) {
+  return pao_decode_range_scaled(out, m_out, l_out, query, q_dtype, key_cache, value_cache,
+                                 kv_dtype, block_tables, max_blocks, context_lens, num_seqs,
+                                 num_heads, num_kv_heads, head_dim, block_size, num_blocks, scale,
+                                 t_begin, t_end, num_threads, NULL, NULL);
 }
 
 /* The whole decode step: softmax(scale * q K^T) V over each sequence's full context. */

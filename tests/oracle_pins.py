@@ -385,6 +385,95 @@ def pin_swap_blocks(orc):
     assert np.array_equal(hk, h1) and np.array_equal(kc, k1)
 
 
+def _torch_fp8_values():
+    """The 256 E4M3 code values from torch's float8_e4m3fn type (a library decoder)."""
+    import torch
+    return torch.arange(256, dtype=torch.uint8).view(torch.float8_e4m3fn).double().numpy()
+
+
+def pin_fp8_codec(orc):
+    """FP8 E4M3 ([P2] 4.3 lists the format): the oracle's decoder agrees with torch's
+    float8_e4m3fn on all 256 codes; its encoder agrees with torch's round-to-nearest-even cast
+    on every finite bf16 value divided by several scales wherever torch's cast stays finite,
+    saturates to +-448 beyond, keeps NaN as 0x7f, and decodes back to the same value."""
+    import torch
+    codes = np.arange(256, dtype=np.uint8)
+    ref = _torch_fp8_values()
+    got = orc.fp8_decode(codes)
+    assert np.array_equal(np.isnan(got), np.isnan(ref))
+    fin = ~np.isnan(ref)
+    assert np.array_equal(got[fin], ref[fin])
+    assert got[0x7e] == 448.0 and got[0x08] == 2.0 ** -6 and got[0x01] == 2.0 ** -9
+    assert np.all(np.diff(got[:0x7f]) > 0)  # codes 0..0x7e increase strictly
+    bits = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    vals = (bits.astype(np.uint32) << 16).view(np.float32)
+    bits = bits[np.isfinite(vals)]
+    for scale in (1.0, 0.0078125, 0.37, 3.0):
+        enc = orc.fp8_encode(bits, "bf16", scale)
+        q = torch.from_numpy((bits.astype(np.uint32) << 16).view(np.float32)) / scale
+        tq = q.to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+        inside = np.abs(q.numpy()) <= 464.0  # torch's cast is finite here
+        assert np.array_equal(enc[inside], tq[inside]), scale
+        big = ~inside
+        assert np.all((enc[big] & 0x7f) == 0x7e)
+        assert np.array_equal(enc[big] >> 7, (q.numpy()[big] < 0).astype(np.uint8))
+    nan_bf16 = np.array([0x7fc0, 0xffc0], np.uint16)
+    assert np.all(orc.fp8_encode(nan_bf16, "bf16", 1.0) == 0x7f)
+    roundtrip = orc.fp8_encode(got[fin].astype(np.float32), "f32", 1.0)
+    assert np.array_equal(orc.fp8_decode(roundtrip), got[fin])
+
+
+def pin_fp8_cache(orc):
+    """FP8 cache write and attention: each written slot holds the codes of its row divided by
+    its kv head's scale, untouched and padding slots keep their bytes; the attention over an FP8
+    cache equals long-double brute force over the decoded values times the per-head scales
+    (keys and values scaled differently)."""
+    b = W.build_batch("fp8", [1, 15, 16, 37, 60], num_heads=8, num_kv_heads=2, head_dim=64,
+                      block_size=8, dtype="bf16", seed=W.BASE_SEED + 706, fill="zero",
+                      keep_logical=True)
+    nb, hkv, bs, d = b.key_cache.shape
+    ks = np.array([0.011, 0.023], np.float32)
+    vs = np.array([0.017, 0.0041], np.float32)
+    kc = np.zeros((nb, hkv, bs, d), np.uint8)
+    vc = np.zeros((nb, hkv, bs, d), np.uint8)
+    # every token of every sequence through the write path
+    for s in range(b.num_seqs):
+        L = int(b.context_lens[s])
+        t = np.arange(L)
+        slots = b.block_tables[s, t // bs].astype(np.int64) * bs + t % bs
+        k_rows = np.ascontiguousarray(b.logical_key[s][:L])  # [L, Hkv, D]
+        v_rows = np.ascontiguousarray(b.logical_value[s][:L])
+        assert orc.reshape_and_cache_fp8(k_rows, v_rows, "bf16", kc, vc, slots, ks, vs) == 0
+        for i in range(L):
+            blk, off = slots[i] // bs, slots[i] % bs
+            for h in range(hkv):
+                assert np.array_equal(kc[blk, h, off], orc.fp8_encode(k_rows[i, h], "bf16", ks[h]))
+                assert np.array_equal(vc[blk, h, off], orc.fp8_encode(v_rows[i, h], "bf16", vs[h]))
+    k1, v1 = kc.copy(), vc.copy()
+    pad = np.array([-1, nb * bs + 3], np.int64)
+    rows = np.ones((2, hkv, d), np.uint16) * 0x3f80
+    assert orc.reshape_and_cache_fp8(rows, rows, "bf16", kc, vc, pad, ks, vs) == 1
+    assert np.array_equal(kc, k1) and np.array_equal(vc, v1)
+
+    got = orc.decode(b.query, kc, vc, b.block_tables, b.context_lens, b.scale, "fp8",
+                     q_dtype="bf16", k_scale=ks, v_scale=vs)
+    table = _torch_fp8_values()
+    q = W.decode_to_f64(b.query, "bf16").astype(np.longdouble)
+    group = b.num_heads // hkv
+    for s in range(b.num_seqs):
+        L = int(b.context_lens[s])
+        t = np.arange(L)
+        blk, off = b.block_tables[s, t // bs], t % bs
+        for h in range(b.num_heads):
+            g = h // group
+            K = table[kc[blk, g, off]].astype(np.longdouble) * np.longdouble(ks[g])
+            V = table[vc[blk, g, off]].astype(np.longdouble) * np.longdouble(vs[g])
+            z = np.longdouble(b.scale) * (K @ q[s, h])
+            w = np.exp(z - z.max())
+            ref = (w @ V) / w.sum()
+            assert np.allclose(got[s, h], ref.astype(np.float64), rtol=1e-12, atol=1e-15), (s, h)
+
+
 def pin_shared_prefix(orc):
     """Sequences sharing prefix blocks read the same bytes: the paged result over the shared
     pool equals brute force on each member's own logical stream."""
@@ -425,5 +514,5 @@ def pin_zero_context(orc):
 ALL_PINS = [
     pin_brute_force, pin_torch_sdpa, pin_closed_forms, pin_decimal_example,
     pin_placement_invariance, pin_unread_table_entries, pin_cache_write, pin_copy_blocks,
-    pin_swap_blocks, pin_shared_prefix, pin_split_merge, pin_zero_context,
+    pin_swap_blocks, pin_fp8_codec, pin_fp8_cache, pin_shared_prefix, pin_split_merge, pin_zero_context,
 ]

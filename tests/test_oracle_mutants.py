@@ -48,6 +48,17 @@ MUTANTS = {
         "           (const char *)src_key + (size_t)src * block_bytes, block_bytes);"),
     "swap_dst_index": ("memcpy((char *)dst_key + (size_t)dst * block_bytes,",
                        "memcpy((char *)dst_key + (size_t)src * block_bytes,"),
+    "fp8_exponent_bias": ("v = ldexp((double)(8 + m), e - 10);", "v = ldexp((double)(8 + m), e - 11);"),
+    "fp8_subnormal_scale": ("v = ldexp((double)m, -9);", "v = ldexp((double)m, -10);"),
+    "fp8_subnormal_floor": ("code = (int)rint(a * 512.0);", "code = (int)floor(a * 512.0);"),
+    "fp8_normal_floor": ("int m = (int)rint((ldexp(a, -e) - 1.0) * 8.0);",
+                         "int m = (int)floor((ldexp(a, -e) - 1.0) * 8.0);"),
+    "fp8_late_saturation": ("if (a >= 448.0) return sign | 0x7e;", "if (a >= 480.0) return sign | 0x7e;"),
+    "fp8_quantise_multiplies": ("const float q = x / scale;", "const float q = x * scale;"),
+    "fp8_padding_counted": ("if (slot < 0) continue; /* a padding token stores nothing */",
+                            "if (slot < 0) { ++skipped; continue; }"),
+    "fp8_v_scaled_by_k": ("const double vs = v_scale ? (double)v_scale[g] : 1.0;",
+                          "const double vs = k_scale ? (double)k_scale[g] : 1.0;"),
     "bf16_shift": ("uint32_t u = (uint32_t)h << 16;", "uint32_t u = (uint32_t)h << 15;"),
     "f16_bias": ("v = ldexp((double)(m | 0x400), e - 25);", "v = ldexp((double)(m | 0x400), e - 24);"),
     "merge_sign": ("const double w = l[p] * exp(m[p] - big_m);",
