@@ -62,7 +62,7 @@
 extern "C" {
 #endif
 
-#define PA_VERSION 3
+#define PA_VERSION 4
 
 /* Symbols of this ABI are the only ones the shared library exports. */
 #if defined(__GNUC__)
@@ -71,7 +71,14 @@ extern "C" {
 #define PA_API
 #endif
 
-typedef enum pa_dtype { PA_F32 = 0, PA_BF16 = 1, PA_F16 = 2, PA_I32 = 3, PA_I64 = 4 } pa_dtype;
+typedef enum pa_dtype {
+  PA_F32 = 0,
+  PA_BF16 = 1,
+  PA_F16 = 2,
+  PA_I32 = 3,
+  PA_I64 = 4,
+  PA_FP8_E4M3 = 5 /* KV caches only, with per-kv-head fp32 scales: see pa_decode_fp8 */
+} pa_dtype;
 
 #define PA_MAX_DIMS 5
 
@@ -157,6 +164,43 @@ PA_API int pa_decode_step(const pa_tensor *key, const pa_tensor *value,
                           const pa_tensor *context_lens, float scale, int32_t block_size,
                           int32_t num_kv_heads, void *workspace, size_t workspace_bytes,
                           void *stream);
+
+/*
+ * FP8 KV cache ([P2] 4.3 lists FP8 E4M3, 8-bit floating point, about half the memory of 16-bit,
+ * among the supported storage formats; storing the KV cache in it with one fp32 scale per kv
+ * head is this library's reading).  E4M3: 1 sign bit, 4 exponent bits (bias 7), 3 fraction
+ * bits, subnormals below 2^-6, no infinities, largest finite magnitude 448, NaN = S.1111.111.
+ * The cache holds code(x / scale[h]); attention reads decode(code) * scale[h].
+ *
+ * pa_reshape_and_cache_fp8 - pa_reshape_and_cache into FP8 caches: for each element x of
+ * key[i, h, :] (value alike) the code of x / k_scale[h] is stored, the division in fp32
+ * (correctly rounded), the code the nearest E4M3 value (ties to the even code), magnitudes
+ * beyond 448 saturated to 448, NaN kept.  key, value: [T, Hkv, D] fp32, bf16 or fp16;
+ * caches: fp8_e4m3 [NB, Hkv, bs, D]; k_scale, v_scale: fp32 [Hkv] device memory.  Slots as for
+ * pa_reshape_and_cache.  The codes equal the oracle's bit for bit.
+ */
+PA_API int pa_reshape_and_cache_fp8(const pa_tensor *key, const pa_tensor *value,
+                                    const pa_tensor *key_cache, const pa_tensor *value_cache,
+                                    const pa_tensor *slot_mapping, const pa_tensor *k_scale,
+                                    const pa_tensor *v_scale, void *stream);
+
+/*
+ * pa_decode_fp8 - pa_decode_ex over FP8 caches: K_t = decode(code) * k_scale[g] and V_t =
+ * decode(code) * v_scale[g] for kv head g, then the same attention.  query: bf16 or fp16;
+ * out: fp32 or the query's type.  head_dim 128 (other sizes PA_ERR_UNSUPPORTED); block_size
+ * 8/16/32; 1/2/4/8 query heads per kv head.  The tensor-core kernel widens each tile to fp16
+ * (exact) and scales each query head by a power of two into the fp16 range (1/alpha folded
+ * into its logit scale), so the accuracy is that of the 16-bit caches.  workspace NULL: the
+ * library-owned workspace of pa_decode; otherwise as for pa_decode_ex.  Flags as for
+ * pa_decode_ex except PA_DECODE_CUDA_CORES (PA_ERR_UNSUPPORTED).  pa_copy_blocks and
+ * pa_swap_blocks move FP8 blocks as bytes.
+ */
+PA_API int pa_decode_fp8(const pa_tensor *out, const pa_tensor *query, const pa_tensor *key_cache,
+                         const pa_tensor *value_cache, const pa_tensor *block_tables,
+                         const pa_tensor *context_lens, const pa_tensor *k_scale,
+                         const pa_tensor *v_scale, float scale, int32_t block_size,
+                         int32_t num_kv_heads, int32_t num_workers, uint32_t flags,
+                         void *workspace, size_t workspace_bytes, void *stream);
 
 /*
  * pa_copy_blocks - copy whole physical blocks (all kv heads, all slots, both caches):

@@ -25,7 +25,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIBRARY = os.path.join(_HERE, "libpa.so")
 HEADER = os.path.join(os.path.dirname(_HERE), "include", "pa.h")
 
-PA_F32, PA_BF16, PA_F16, PA_I32, PA_I64 = 0, 1, 2, 3, 4
+PA_F32, PA_BF16, PA_F16, PA_I32, PA_I64, PA_FP8_E4M3 = 0, 1, 2, 3, 4, 5
 PA_OK = 0
 PA_DECODE_SEPARATE_REDUCE = 0x1
 PA_DECODE_CUDA_CORES = 0x2
@@ -76,6 +76,8 @@ def load(path: str = LIBRARY) -> ctypes.CDLL:
     lib.pa_reshape_and_cache.argtypes = [_T, _T, _T, _T, _T, _P]
     lib.pa_copy_blocks.argtypes = [_T, _T, _T, _P]
     lib.pa_swap_blocks.argtypes = [_T, _T, _T, _T, _T, _P]
+    lib.pa_reshape_and_cache_fp8.argtypes = [_T, _T, _T, _T, _T, _T, _T, _P]
+    lib.pa_decode_fp8.argtypes = [_T, _T, _T, _T, _T, _T, _T, _T, f32, i32, i32, i32, u32, _P, sz, _P]
     lib.pa_decode.argtypes = [_T, _T, _T, _T, _T, _T, f32, i32, i32, _P]
     lib.pa_decode_ex.argtypes = [_T, _T, _T, _T, _T, _T, f32, i32, i32, i32, u32, _P, sz, _P]
     lib.pa_decode_workspace_bytes.argtypes = [i64, i32, i32, i32, i32]
@@ -103,7 +105,7 @@ def _torch_dtype_code(t) -> int:
     import torch
 
     codes = {torch.float32: PA_F32, torch.bfloat16: PA_BF16, torch.float16: PA_F16,
-             torch.int32: PA_I32, torch.int64: PA_I64}
+             torch.int32: PA_I32, torch.int64: PA_I64, torch.float8_e4m3fn: PA_FP8_E4M3}
     if t.dtype not in codes:
         raise TypeError(f"unsupported tensor dtype {t.dtype}")
     return codes[t.dtype]
@@ -160,6 +162,30 @@ def pa_swap_blocks(src_key_cache, src_value_cache, dst_key_cache, dst_value_cach
     d = [describe(x) for x in (src_key_cache, src_value_cache, dst_key_cache, dst_value_cache,
                                block_mapping)]
     _check("pa_swap_blocks", lib.pa_swap_blocks(*[ctypes.byref(x) for x in d], _stream(stream)))
+
+
+def pa_reshape_and_cache_fp8(key, value, key_cache, value_cache, slot_mapping, k_scale, v_scale,
+                             stream=None):
+    """Quantise new tokens' K/V rows into FP8 E4M3 caches (torch.float8_e4m3fn tensors) with
+    one fp32 scale per kv head (see include/pa.h)."""
+    lib = load()
+    d = [describe(x) for x in (key, value, key_cache, value_cache, slot_mapping, k_scale, v_scale)]
+    _check("pa_reshape_and_cache_fp8",
+           lib.pa_reshape_and_cache_fp8(*[ctypes.byref(x) for x in d], _stream(stream)))
+
+
+def pa_decode_fp8(out, query, key_cache, value_cache, block_tables, context_lens, k_scale, v_scale,
+                  scale, block_size, num_kv_heads, num_workers=0, flags=0, workspace=None,
+                  stream=None):
+    """Decode over FP8 E4M3 caches with per-kv-head scales; workspace None = library-owned."""
+    lib = load()
+    d = [describe(x) for x in (out, query, key_cache, value_cache, block_tables, context_lens,
+                               k_scale, v_scale)]
+    ws_ptr = workspace.data_ptr() if workspace is not None else None
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check("pa_decode_fp8", lib.pa_decode_fp8(*[ctypes.byref(x) for x in d], float(scale),
+                                              int(block_size), int(num_kv_heads), int(num_workers),
+                                              int(flags), ws_ptr, ws_bytes, _stream(stream)))
 
 
 def pa_decode(out, query, key_cache, value_cache, block_tables, context_lens, scale, block_size,

@@ -145,6 +145,8 @@ size_t elt_size(int dtype) {
       return 2;
     case PA_I64:
       return 8;
+    case PA_FP8_E4M3:
+      return 1;
     default:
       return 0;
   }
@@ -157,6 +159,7 @@ const char *dtype_name(int d) {
     case PA_F16: return "fp16";
     case PA_I32: return "int32";
     case PA_I64: return "int64";
+    case PA_FP8_E4M3: return "fp8_e4m3";
     default: return "unknown";
   }
 }
@@ -229,15 +232,17 @@ struct CacheShape {
   int num_kv_heads, block_size, head_dim, dtype;
 };
 
-int check_caches(const pa_tensor *kc, const pa_tensor *vc, CacheShape *cs) {
+int check_caches(const pa_tensor *kc, const pa_tensor *vc, CacheShape *cs, bool allow_fp8 = false) {
   int rc;
   if ((rc = check_tensor(kc, "key_cache", 4)) || (rc = check_tensor(vc, "value_cache", 4))) return rc;
   for (int i = 0; i < 4; ++i)
     if (kc->shape[i] != vc->shape[i] || kc->stride[i] != vc->stride[i])
       return fail(PA_ERR_SHAPE, "key_cache and value_cache differ in shape or strides (dim %d)", i);
   if (kc->dtype != vc->dtype) return fail(PA_ERR_DTYPE, "key_cache and value_cache element types differ");
-  if (kc->dtype != PA_F32 && kc->dtype != PA_BF16 && kc->dtype != PA_F16)
-    return fail(PA_ERR_DTYPE, "caches must be fp32, bf16 or fp16 (got %s)", dtype_name(kc->dtype));
+  if (kc->dtype == PA_FP8_E4M3 && !allow_fp8)
+    return fail(PA_ERR_DTYPE, "FP8 caches need their scales: use the _fp8 entry points");
+  if (kc->dtype != PA_F32 && kc->dtype != PA_BF16 && kc->dtype != PA_F16 && kc->dtype != PA_FP8_E4M3)
+    return fail(PA_ERR_DTYPE, "caches must be fp32, bf16, fp16 or fp8_e4m3 (got %s)", dtype_name(kc->dtype));
   if (kc->stride[3] != 1 || kc->stride[2] != kc->shape[3])
     return fail(PA_ERR_LAYOUT, "caches: each (block, kv head) tile [block_size, head_dim] must be contiguous");
   if (!aligned16(kc->data) || !aligned16(vc->data) || !strides16(kc, 2))
@@ -304,16 +309,21 @@ int cache_map(const pa_tensor *t, int rows, CUtensorMap *out) {
       return PA_OK;
     }
   if (!g_encode_tiled) return fail(PA_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
-  const cuuint64_t halves = (cuuint64_t)t->shape[3] / 64;
-  const cuuint64_t dims[5] = {64, (cuuint64_t)t->shape[2], halves, (cuuint64_t)t->shape[1],
+  const cuuint64_t e = (cuuint64_t)elt_size(t->dtype);
+  const cuuint64_t per128 = 128 / e;  // elements in one 128-byte swizzle span
+  const cuuint64_t spans = (cuuint64_t)t->shape[3] / per128;
+  const cuuint64_t dims[5] = {per128, (cuuint64_t)t->shape[2], spans, (cuuint64_t)t->shape[1],
                               (cuuint64_t)t->shape[0]};
-  const cuuint64_t strides[4] = {(cuuint64_t)t->stride[2] * 2, 128, (cuuint64_t)t->stride[1] * 2,
-                                 (cuuint64_t)t->stride[0] * 2};
-  const cuuint32_t box[5] = {64, (cuuint32_t)rows, (cuuint32_t)halves, 1, 1};
+  const cuuint64_t strides[4] = {(cuuint64_t)t->stride[2] * e, 128, (cuuint64_t)t->stride[1] * e,
+                                 (cuuint64_t)t->stride[0] * e};
+  const cuuint32_t box[5] = {(cuuint32_t)per128, (cuuint32_t)rows, (cuuint32_t)spans, 1, 1};
   const cuuint32_t estr[5] = {1, 1, 1, 1, 1};
   CUtensorMap map;
+  const CUtensorMapDataType type = t->dtype == PA_FP8_E4M3 ? CU_TENSOR_MAP_DATA_TYPE_UINT8
+                                   : t->dtype == PA_BF16   ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                                           : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
   const CUresult r = g_encode_tiled(
-      &map, t->dtype == PA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
+      &map, type,
       5, t->data, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
       CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
       CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -367,10 +377,13 @@ int decode_impl(const pa_tensor *out, const pa_tensor *query, const pa_tensor *k
                 const pa_tensor *context_lens, float scale, int32_t block_size,
                 int32_t num_kv_heads, int32_t num_workers, uint32_t flags, void *workspace,
                 size_t workspace_bytes, bool library_workspace, void *stream,
-                CallMode mode = CallMode::kLaunch) {
+                CallMode mode = CallMode::kLaunch, const pa_tensor *k_scale = nullptr,
+                const pa_tensor *v_scale = nullptr) {
   int rc;
   CacheShape cs;
-  if ((rc = check_caches(key_cache, value_cache, &cs))) return rc;
+  const bool fp8 = k_scale != nullptr;
+  if ((rc = check_caches(key_cache, value_cache, &cs, fp8))) return rc;
+  if (fp8 && cs.dtype != PA_FP8_E4M3) return fail(PA_ERR_DTYPE, "pa_decode_fp8 needs fp8_e4m3 caches");
   if ((rc = check_tensor(query, "query", 3)) || (rc = check_tensor(out, "out", 3)) ||
       (rc = check_tensor(block_tables, "block_tables", 2)) ||
       (rc = check_tensor(context_lens, "context_lens", 1)))
@@ -390,9 +403,27 @@ int decode_impl(const pa_tensor *out, const pa_tensor *query, const pa_tensor *k
     return fail(PA_ERR_SHAPE, "out must be [num_seqs, num_heads, head_dim] like query");
   if (block_tables->shape[0] != S || context_lens->shape[0] != S)
     return fail(PA_ERR_SHAPE, "block_tables and context_lens need one row per sequence");
-  if (query->dtype != cs.dtype) return fail(PA_ERR_DTYPE, "query must have the caches' element type");
-  if (out->dtype != PA_F32 && out->dtype != cs.dtype)
-    return fail(PA_ERR_DTYPE, "out must be fp32 or the caches' element type");
+  if (fp8) {
+    if (query->dtype != PA_BF16 && query->dtype != PA_F16)
+      return fail(PA_ERR_DTYPE, "with FP8 caches the query must be bf16 or fp16");
+    if (out->dtype != PA_F32 && out->dtype != query->dtype)
+      return fail(PA_ERR_DTYPE, "out must be fp32 or the query's element type");
+    if ((rc = check_tensor(k_scale, "k_scale", 1)) || (rc = check_tensor(v_scale, "v_scale", 1)))
+      return rc;
+    if (k_scale->dtype != PA_F32 || v_scale->dtype != PA_F32)
+      return fail(PA_ERR_DTYPE, "k_scale and v_scale must be fp32");
+    if (k_scale->shape[0] != num_kv_heads || v_scale->shape[0] != num_kv_heads)
+      return fail(PA_ERR_SHAPE, "k_scale and v_scale need one value per kv head");
+    if ((k_scale->stride[0] != 1 || v_scale->stride[0] != 1) && num_kv_heads > 1)
+      return fail(PA_ERR_LAYOUT, "k_scale and v_scale must be contiguous");
+    if (flags & PA_DECODE_CUDA_CORES)
+      return fail(PA_ERR_UNSUPPORTED, "FP8 caches are read by the tensor-core kernel only");
+    if (cs.head_dim != 128) return fail(PA_ERR_UNSUPPORTED, "FP8 caches: head_dim %d (built: 128)", cs.head_dim);
+  } else {
+    if (query->dtype != cs.dtype) return fail(PA_ERR_DTYPE, "query must have the caches' element type");
+    if (out->dtype != PA_F32 && out->dtype != cs.dtype)
+      return fail(PA_ERR_DTYPE, "out must be fp32 or the caches' element type");
+  }
   if (block_tables->dtype != PA_I32 || context_lens->dtype != PA_I32)
     return fail(PA_ERR_DTYPE, "block_tables and context_lens must be int32");
   if (Hq <= 0 && S > 0) return fail(PA_ERR_SHAPE, "num_heads must be positive");
@@ -423,10 +454,15 @@ int decode_impl(const pa_tensor *out, const pa_tensor *query, const pa_tensor *k
       (rc = check_device_memory(block_tables, "block_tables", dev)) ||
       (rc = check_device_memory(context_lens, "context_lens", dev)))
     return rc;
+  if (fp8 && ((rc = check_device_memory(k_scale, "k_scale", dev)) ||
+              (rc = check_device_memory(v_scale, "v_scale", dev))))
+    return rc;
 
   pa::DecodeKernel k;
   const bool tensor_cores = cs.dtype != PA_F32 && !(flags & PA_DECODE_CUDA_CORES);
-  if (!get_kernel(cs.dtype, D, block_size, G, tensor_cores, &k))
+  const bool got = fp8 ? pa::decode_kernel_fp8(query->dtype, D, block_size, G, &k)
+                       : get_kernel(cs.dtype, D, block_size, G, tensor_cores, &k);
+  if (!got)
     return fail(PA_ERR_CUDA, "could not prepare the decode kernel: %s", cudaGetErrorString(cudaGetLastError()));
   pa::TmaMaps maps;
   if (k.tma_rows > 0) {
@@ -513,6 +549,8 @@ int decode_impl(const pa_tensor *out, const pa_tensor *query, const pa_tensor *k
   a.part_ml = reinterpret_cast<float *>(ws + L.part_ml);
   a.part_o = reinterpret_cast<float *>(ws + L.part_o);
   a.err = ds->err;
+  a.k_scale = fp8 ? static_cast<const float *>(k_scale->data) : nullptr;
+  a.v_scale = fp8 ? static_cast<const float *>(v_scale->data) : nullptr;
   a.separate_reduce = (flags & PA_DECODE_SEPARATE_REDUCE) ? 1 : 0;
   a.wait_cycles = test_hooks().wait_cycles;
   a.test_stall = test_hooks().stall;
@@ -643,8 +681,8 @@ int copy_blocks_impl(const pa_tensor *src_k, const pa_tensor *src_v, const pa_te
                      void *stream) {
   int rc;
   CacheShape s, d;
-  if ((rc = check_caches(src_k, src_v, &s))) return rc;
-  if ((rc = check_caches(dst_k, dst_v, &d))) return rc;
+  if ((rc = check_caches(src_k, src_v, &s, true))) return rc;
+  if ((rc = check_caches(dst_k, dst_v, &d, true))) return rc;
   if (s.dtype != d.dtype || s.num_kv_heads != d.num_kv_heads || s.block_size != d.block_size ||
       s.head_dim != d.head_dim)
     return fail(PA_ERR_SHAPE, "source and destination caches differ in element type or block shape");
@@ -691,9 +729,96 @@ int copy_blocks_impl(const pa_tensor *src_k, const pa_tensor *src_v, const pa_te
   return err == cudaSuccess ? PA_OK : cuda_fail(err, host_allowed ? "swap_blocks launch" : "copy_blocks launch");
 }
 
+int write_fp8_impl(const pa_tensor *key, const pa_tensor *value, const pa_tensor *key_cache,
+                   const pa_tensor *value_cache, const pa_tensor *slot_mapping,
+                   const pa_tensor *k_scale, const pa_tensor *v_scale, void *stream) {
+  int rc;
+  CacheShape cs;
+  if ((rc = check_caches(key_cache, value_cache, &cs, true))) return rc;
+  if (cs.dtype != PA_FP8_E4M3) return fail(PA_ERR_DTYPE, "pa_reshape_and_cache_fp8 needs fp8_e4m3 caches");
+  if ((rc = check_tensor(key, "key", 3)) || (rc = check_tensor(value, "value", 3)) ||
+      (rc = check_tensor(slot_mapping, "slot_mapping", 1)) ||
+      (rc = check_tensor(k_scale, "k_scale", 1)) || (rc = check_tensor(v_scale, "v_scale", 1)))
+    return rc;
+  const int64_t T = key->shape[0];
+  for (int i = 0; i < 3; ++i)
+    if (value->shape[i] != key->shape[i]) return fail(PA_ERR_SHAPE, "key and value shapes differ");
+  if (key->shape[1] != cs.num_kv_heads || key->shape[2] != cs.head_dim)
+    return fail(PA_ERR_SHAPE, "key/value must be [num_tokens, num_kv_heads, head_dim] of the cache");
+  if (slot_mapping->shape[0] != T) return fail(PA_ERR_SHAPE, "slot_mapping needs one slot per token");
+  if (key->dtype != value->dtype || (key->dtype != PA_F32 && key->dtype != PA_BF16 && key->dtype != PA_F16))
+    return fail(PA_ERR_DTYPE, "key/value must both be fp32, bf16 or fp16");
+  if (slot_mapping->dtype != PA_I64) return fail(PA_ERR_DTYPE, "slot_mapping must be int64");
+  if (k_scale->dtype != PA_F32 || v_scale->dtype != PA_F32)
+    return fail(PA_ERR_DTYPE, "k_scale and v_scale must be fp32");
+  if (k_scale->shape[0] != cs.num_kv_heads || v_scale->shape[0] != cs.num_kv_heads)
+    return fail(PA_ERR_SHAPE, "k_scale and v_scale need one value per kv head");
+  if ((k_scale->stride[0] != 1 || v_scale->stride[0] != 1) && cs.num_kv_heads > 1)
+    return fail(PA_ERR_LAYOUT, "k_scale and v_scale must be contiguous");
+  if (key->stride[2] != 1 || value->stride[2] != 1 || (slot_mapping->stride[0] != 1 && T > 1))
+    return fail(PA_ERR_LAYOUT, "key/value need a contiguous head_dim and slot_mapping unit stride");
+  if (!aligned16(key->data) || !aligned16(value->data) || !strides16(key, 2) || !strides16(value, 2))
+    return fail(PA_ERR_LAYOUT, "key/value: data and token/head strides must be 16-byte aligned");
+  if (cs.head_dim % 16 != 0) return fail(PA_ERR_UNSUPPORTED, "FP8 caches: head_dim must be a multiple of 16");
+  if (T == 0) return PA_OK;
+  DeviceState *ds;
+  int dev;
+  if ((rc = device_state(&ds, &dev))) return rc;
+  if ((rc = check_device_memory(key_cache, "key_cache", dev)) ||
+      (rc = check_device_memory(value_cache, "value_cache", dev)) ||
+      (rc = check_device_memory(key, "key", dev)) || (rc = check_device_memory(value, "value", dev)) ||
+      (rc = check_device_memory(slot_mapping, "slot_mapping", dev)) ||
+      (rc = check_device_memory(k_scale, "k_scale", dev)) ||
+      (rc = check_device_memory(v_scale, "v_scale", dev)))
+    return rc;
+  const size_t se = elt_size(key->dtype);
+  pa::CacheWriteFp8Args a;
+  a.key = static_cast<const char *>(key->data);
+  a.value = static_cast<const char *>(value->data);
+  a.src_dtype = key->dtype;
+  a.k_tok = key->stride[0] * (int64_t)se;
+  a.k_head = key->stride[1] * (int64_t)se;
+  a.v_tok = value->stride[0] * (int64_t)se;
+  a.v_head = value->stride[1] * (int64_t)se;
+  a.key_cache = static_cast<unsigned char *>(key_cache->data);
+  a.value_cache = static_cast<unsigned char *>(value_cache->data);
+  a.c_blk = key_cache->stride[0];
+  a.c_head = key_cache->stride[1];
+  a.head_dim = cs.head_dim;
+  a.slots = static_cast<const int64_t *>(slot_mapping->data);
+  a.num_tokens = T;
+  a.num_kv_heads = cs.num_kv_heads;
+  a.block_size = cs.block_size;
+  a.num_slots = cs.num_blocks * cs.block_size;
+  a.k_scale = static_cast<const float *>(k_scale->data);
+  a.v_scale = static_cast<const float *>(v_scale->data);
+  a.err = ds->err;
+  cudaError_t err = pa::launch_reshape_and_cache_fp8(a, ds->num_sms, static_cast<cudaStream_t>(stream));
+  return err == cudaSuccess ? PA_OK : cuda_fail(err, "reshape_and_cache_fp8 launch");
+}
+
 }  // namespace
 
 extern "C" {
+
+int pa_reshape_and_cache_fp8(const pa_tensor *key, const pa_tensor *value,
+                             const pa_tensor *key_cache, const pa_tensor *value_cache,
+                             const pa_tensor *slot_mapping, const pa_tensor *k_scale,
+                             const pa_tensor *v_scale, void *stream) {
+  return write_fp8_impl(key, value, key_cache, value_cache, slot_mapping, k_scale, v_scale, stream);
+}
+
+int pa_decode_fp8(const pa_tensor *out, const pa_tensor *query, const pa_tensor *key_cache,
+                  const pa_tensor *value_cache, const pa_tensor *block_tables,
+                  const pa_tensor *context_lens, const pa_tensor *k_scale,
+                  const pa_tensor *v_scale, float scale, int32_t block_size, int32_t num_kv_heads,
+                  int32_t num_workers, uint32_t flags, void *workspace, size_t workspace_bytes,
+                  void *stream) {
+  if (!k_scale || !v_scale) return fail(PA_ERR_INVALID_ARG, "k_scale and v_scale are required");
+  return decode_impl(out, query, key_cache, value_cache, block_tables, context_lens, scale,
+                     block_size, num_kv_heads, num_workers, flags, workspace, workspace_bytes,
+                     workspace == nullptr, stream, CallMode::kLaunch, k_scale, v_scale);
+}
 
 int pa_reshape_and_cache(const pa_tensor *key, const pa_tensor *value, const pa_tensor *key_cache,
                          const pa_tensor *value_cache, const pa_tensor *slot_mapping, void *stream) {

@@ -72,6 +72,74 @@ __global__ void __launch_bounds__(256) copy_blocks_kernel(CopyBlocksArgs a) {
   }
 }
 
+// Two fp32 values -> two FP8 E4M3 codes (round to nearest even, saturated to +-448, NaN kept),
+// x0 in the low byte.
+__device__ __forceinline__ uint16_t f32x2_to_fp8x2(float x0, float x1) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(x1), "f"(x0));
+  return r;
+}
+
+template <typename S>
+__device__ __forceinline__ void load_row16(const char *p, float (&f)[16]) {
+  if constexpr (sizeof(S) == 4) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint4 v = __ldg(reinterpret_cast<const uint4 *>(p) + i);
+      f[4 * i] = __uint_as_float(v.x);
+      f[4 * i + 1] = __uint_as_float(v.y);
+      f[4 * i + 2] = __uint_as_float(v.z);
+      f[4 * i + 3] = __uint_as_float(v.w);
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      float g[8];
+      Elem<S>::unpack(__ldg(reinterpret_cast<const uint4 *>(p) + i), g);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) f[8 * i + j] = g[j];
+    }
+  }
+}
+
+// One thread per 16 codes (16 elements) of one (token, kv head) row, keys and values together.
+// Each element is divided by its head's scale in fp32 (IEEE division) before the conversion.
+template <typename S>
+__global__ void __launch_bounds__(256) reshape_and_cache_fp8_kernel(CacheWriteFp8Args a) {
+  allow_next_grid();
+  const int vec_per_row = a.head_dim >> 4;
+  const int64_t total = a.num_tokens * a.num_kv_heads * vec_per_row;
+  for (int64_t idx = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; idx < total;
+       idx += (int64_t)gridDim.x * blockDim.x) {
+    const int v = (int)(idx % vec_per_row);
+    const int64_t th = idx / vec_per_row;
+    const int h = (int)(th % a.num_kv_heads);
+    const int64_t t = th / a.num_kv_heads;
+    const int64_t slot = __ldg(a.slots + t);
+    if (slot < 0) continue;  // padding token
+    if (slot >= a.num_slots) {
+      if (h == 0 && v == 0) set_error(a.err, PA_DEVERR_SLOT);
+      continue;
+    }
+    const int64_t dst = (slot / a.block_size) * a.c_blk + h * a.c_head +
+                        (slot % a.block_size) * a.head_dim + v * 16;
+    const float ks = __ldg(a.k_scale + h), vs = __ldg(a.v_scale + h);
+    float fk[16], fv[16];
+    load_row16<S>(a.key + t * a.k_tok + h * a.k_head + (int64_t)v * 16 * sizeof(S), fk);
+    load_row16<S>(a.value + t * a.v_tok + h * a.v_head + (int64_t)v * 16 * sizeof(S), fv);
+    uint32_t ck[4], cv[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      ck[i] = (uint32_t)f32x2_to_fp8x2(__fdiv_rn(fk[4 * i], ks), __fdiv_rn(fk[4 * i + 1], ks)) |
+              ((uint32_t)f32x2_to_fp8x2(__fdiv_rn(fk[4 * i + 2], ks), __fdiv_rn(fk[4 * i + 3], ks)) << 16);
+      cv[i] = (uint32_t)f32x2_to_fp8x2(__fdiv_rn(fv[4 * i], vs), __fdiv_rn(fv[4 * i + 1], vs)) |
+              ((uint32_t)f32x2_to_fp8x2(__fdiv_rn(fv[4 * i + 2], vs), __fdiv_rn(fv[4 * i + 3], vs)) << 16);
+    }
+    *reinterpret_cast<uint4 *>(a.key_cache + dst) = make_uint4(ck[0], ck[1], ck[2], ck[3]);
+    *reinterpret_cast<uint4 *>(a.value_cache + dst) = make_uint4(cv[0], cv[1], cv[2], cv[3]);
+  }
+}
+
 static int grid_for(int64_t items, int num_sms) {
   const int64_t blocks = (items + 255) / 256;
   const int64_t cap = (int64_t)num_sms * 8;
@@ -89,6 +157,19 @@ cudaError_t launch_copy_blocks(const CopyBlocksArgs &a, int num_sms, cudaStream_
   const int64_t items = a.num_pairs * a.num_kv_heads * (a.tile_bytes / 16);
   if (items == 0) return cudaSuccess;
   copy_blocks_kernel<<<grid_for(items, num_sms), 256, 0, st>>>(a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_reshape_and_cache_fp8(const CacheWriteFp8Args &a, int num_sms, cudaStream_t st) {
+  const int64_t items = a.num_tokens * a.num_kv_heads * (a.head_dim / 16);
+  if (items == 0) return cudaSuccess;
+  const int grid = grid_for(items, num_sms);
+  if (a.src_dtype == PA_F32)
+    reshape_and_cache_fp8_kernel<float><<<grid, 256, 0, st>>>(a);
+  else if (a.src_dtype == PA_BF16)
+    reshape_and_cache_fp8_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(a);
+  else
+    reshape_and_cache_fp8_kernel<__half><<<grid, 256, 0, st>>>(a);
   return cudaGetLastError();
 }
 

@@ -64,6 +64,15 @@ struct MmaType<__half> {
   static constexpr CUtensorMapDataType kTmaType = CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
 };
 
+// Four FP8 E4M3 values (bytes 0..3 of w) -> two f16x2: lo = (byte 0, byte 1), hi = (byte 2,
+// byte 3), the lower byte in the lower half.  Exact: every E4M3 value is an f16.
+__device__ __forceinline__ void fp8x4_to_f16x2(uint32_t w, uint32_t &lo, uint32_t &hi) {
+  asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %2;\n\t"
+      "cvt.rn.f16x2.e4m3x2 %0, l;\n\tcvt.rn.f16x2.e4m3x2 %1, h;\n\t}"
+      : "=r"(lo), "=r"(hi)
+      : "r"(w));
+}
+
 __device__ __forceinline__ void ldmatrix_x4(uint32_t (&r)[4], uint32_t addr) {
   asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
                : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
@@ -114,14 +123,15 @@ __device__ __forceinline__ bool mbar_test(uint64_t *bar, uint32_t parity) {
   return done != 0;
 }
 
-template <int D, int BS, int G>
+// KVB: bytes per cache element (2: bf16/fp16, 1: FP8 E4M3).  The query is 16-bit either way.
+template <int D, int BS, int G, int KVB = 2>
 struct MmaTraits {
   static constexpr int kChunk = 16;                     // tokens per chunk (M of q.K)
-  static constexpr int kHalves = D / 64;                // 128-byte column halves of a row
+  static constexpr int kHalves = D * KVB / 128;         // 128-byte column blocks of a row
   static constexpr int kBoxRows = BS < 16 ? BS : 16;    // rows per TMA box
   static constexpr int kCopies = 16 / kBoxRows;         // blocks touched per chunk
-  static constexpr int kBoxBytes = kBoxRows * D * 2;    // one box: [half][row][128 B]
-  static constexpr int kTileBytes = 16 * D * 2;         // key (or value) bytes of a chunk
+  static constexpr int kBoxBytes = kBoxRows * D * KVB;  // one box: [block][row][128 B]
+  static constexpr int kTileBytes = 16 * D * KVB;       // key (or value) bytes of a chunk
   static constexpr int kQBytes = G * D * 2;
   static constexpr int kStageBytes = 2 * kTileBytes + (kQBytes + 1023) / 1024 * 1024;
   static constexpr int kWorkers = 4;                    // consumer warps
@@ -130,7 +140,7 @@ struct MmaTraits {
   // in flight than HBM needs to run at full rate; the longer queues only raise the latency
   // every worker sees and widen the spread of finishing times (measured: the Llama-shaped
   // decode 60 -> 58 us, the long mixed batch 275 -> 259 us).
-  static constexpr int kStages = 2;
+  static constexpr int kStages = KVB == 2 ? 2 : 3;  // FP8 stages hold half the bytes
   static constexpr int kRingBytes = kWorkers * kStages * kStageBytes;
   static constexpr int kPbufBytes = 2 * 8 * 16 * 2;    // [hi, lo][8 heads][16 tokens]
   static constexpr int kMetaOff = 0;
@@ -146,6 +156,7 @@ struct MmaTraits {
   static constexpr int kKSteps = D / 16;                // k-steps of q.K
   static constexpr int kMTiles = D / 16;                // m-tiles of P.V
   static_assert(D == 64 || D == 128, "head_dim 64 or 128");
+  static_assert(D * KVB >= 128, "rows of at least one 128-byte swizzle span");
   static_assert(G <= 8, "at most 8 query heads per kv head");
 };
 
@@ -197,11 +208,14 @@ __device__ __forceinline__ uint32_t tile_offset(int r, int h) {
 // issues that worker's copies (one TMA box per key tile and per value tile, plus the query rows
 // when a new (sequence, kv head) starts) as soon as the worker releases a stage.  The workers
 // never issue copies, so TMA issue latency stays off their critical path.
-template <typename T, int D, int BS, int G>
-__global__ void __launch_bounds__(MmaTraits<D, BS, G>::kThreads, 2)
+// T: the query's element type (and the MMA's, for 16-bit caches).  KV: the caches' element
+// type; with FP8 E4M3 caches the tiles are widened to f16 in registers and the MMAs run in f16.
+template <typename T, int D, int BS, int G, typename KV = T>
+__global__ void __launch_bounds__(MmaTraits<D, BS, G, (int)sizeof(KV)>::kThreads, 2)
     paged_decode_mma_kernel(const DecodeArgs a, const __grid_constant__ TmaMaps maps) {
-  using Tr = MmaTraits<D, BS, G>;
-  using M = MmaType<T>;
+  constexpr bool kFp8 = sizeof(KV) == 1;
+  using Tr = MmaTraits<D, BS, G, (int)sizeof(KV)>;
+  using M = MmaType<typename std::conditional<kFp8, __half, T>::type>;
   constexpr int ST = Tr::kStages;
   constexpr int NW = Tr::kWorkers;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -422,6 +436,8 @@ __global__ void __launch_bounds__(MmaTraits<D, BS, G>::kThreads, 2)
   float o[Tr::kMTiles][4];
   float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
   bool piece_at_start = false;  // this piece begins at chunk 0 of its (sequence, kv head)
+  // logit scale of this lane's two heads (base 2) and the output scale (FP8 value scale)
+  float sc0 = a.scale_log2, sc1 = a.scale_log2, vsc = 1.f;
 
   for (long long cc = 0; cc < n; ++cc) {
     const int slot = (int)(cc % ST);
@@ -441,14 +457,50 @@ __global__ void __launch_bounds__(MmaTraits<D, BS, G>::kThreads, 2)
     const uint32_t vbase = kbase + Tr::kTileBytes;
     if (m.flags & kFirst) {
       const unsigned char *qs = stage + 2 * Tr::kTileBytes;
+      if constexpr (kFp8) {
+        // f16 B fragments in the dim order of the FP8 key fragments below (k-step ks holds the
+        // dims 32(ks/2) + 16(ks%2) + 4c + {0,1 | 2,3}), each head scaled by a power of two
+        // alpha that keeps |q * alpha| < 2^15; 1/alpha goes into that head's logit scale.
+        const T *q = reinterpret_cast<const T *>(qs);
+        float qv[Tr::kKSteps][4];
+        float mx = 0.f;
 #pragma unroll
-      for (int ks = 0; ks < Tr::kKSteps; ++ks) {
-        if (g < G) {
-          qb[ks][0] = *reinterpret_cast<const uint32_t *>(qs + (g * D + 16 * ks + 2 * c) * 2);
-          qb[ks][1] = *reinterpret_cast<const uint32_t *>(qs + (g * D + 16 * ks + 8 + 2 * c) * 2);
-        } else {
-          qb[ks][0] = 0u;
-          qb[ks][1] = 0u;
+        for (int ks = 0; ks < Tr::kKSteps; ++ks) {
+          const int base = 32 * (ks >> 1) + 16 * (ks & 1) + 4 * c;
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            qv[ks][e] = g < G ? Elem<T>::to_float(q[g * D + base + e]) : 0.f;
+            mx = fmaxf(mx, fabsf(qv[ks][e]));
+          }
+        }
+        mx = fmaxf(mx, __shfl_xor_sync(FULL_MASK, mx, 1));
+        mx = fmaxf(mx, __shfl_xor_sync(FULL_MASK, mx, 2));
+        // biased exponent of mx (0 for zero or subnormal), alpha = 2^(14 - unbiased)
+        const int be = (int)((__float_as_uint(mx) >> 23) & 0xffu);
+        const int ae = min(253, max(1, 127 + 14 - (be == 0 ? -126 : be - 127)));
+        const float alpha = __uint_as_float((uint32_t)ae << 23);
+        const float inv_alpha = __uint_as_float((uint32_t)(254 - ae) << 23);
+#pragma unroll
+        for (int ks = 0; ks < Tr::kKSteps; ++ks) {
+          const __half2 lo = __floats2half2_rn(qv[ks][0] * alpha, qv[ks][1] * alpha);
+          const __half2 hi = __floats2half2_rn(qv[ks][2] * alpha, qv[ks][3] * alpha);
+          qb[ks][0] = *reinterpret_cast<const uint32_t *>(&lo);
+          qb[ks][1] = *reinterpret_cast<const uint32_t *>(&hi);
+        }
+        const float ks_ = a.scale_log2 * __ldg(a.k_scale + m.kvh);
+        sc0 = ks_ * __shfl_sync(FULL_MASK, inv_alpha, 4 * h0);
+        sc1 = ks_ * __shfl_sync(FULL_MASK, inv_alpha, 4 * h1);
+        vsc = __ldg(a.v_scale + m.kvh);
+      } else {
+#pragma unroll
+        for (int ks = 0; ks < Tr::kKSteps; ++ks) {
+          if (g < G) {
+            qb[ks][0] = *reinterpret_cast<const uint32_t *>(qs + (g * D + 16 * ks + 2 * c) * 2);
+            qb[ks][1] = *reinterpret_cast<const uint32_t *>(qs + (g * D + 16 * ks + 8 + 2 * c) * 2);
+          } else {
+            qb[ks][0] = 0u;
+            qb[ks][1] = 0u;
+          }
         }
       }
 #pragma unroll
@@ -464,19 +516,40 @@ __global__ void __launch_bounds__(MmaTraits<D, BS, G>::kThreads, 2)
       // two accumulators (even / odd k-steps) halve the chain of dependent mma
       float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f};
       const int row = ((lm & 1) << 3) | lr;
+      if constexpr (kFp8) {
+        // One ldmatrix per 32 dims (two k-steps): matrix j holds tokens 8(j&1).. of the 16-byte
+        // chunk 2*s2 + (j>>1); each lane gets 4 consecutive dims of one token and widens them
+        // to (a0 | a2) or (a1 | a3) of the m16n8k16 A fragment.
 #pragma unroll
-      for (int ks = 0; ks < Tr::kKSteps; ++ks) {
-        const int c16 = ((ks & 3) << 1) | (lm >> 1);
-        const uint32_t addr = kbase + tile_offset<Tr>(row, ks >> 2) + ((c16 ^ lr) << 4);
-        uint32_t af[4];
-        ldmatrix_x4(af, addr);
-        if (ks & 1)
-          M::mma(sb, af, qb[ks][0], qb[ks][1]);
-        else
-          M::mma(sa, af, qb[ks][0], qb[ks][1]);
+        for (int s2 = 0; s2 < D / 32; ++s2) {
+          const int c16 = 2 * s2 + (lm >> 1);
+          const uint32_t addr = kbase + tile_offset<Tr>(row, 0) + ((c16 ^ lr) << 4);
+          uint32_t r[4], af[4];
+          ldmatrix_x4(r, addr);
+          fp8x4_to_f16x2(r[0], af[0], af[2]);
+          fp8x4_to_f16x2(r[1], af[1], af[3]);
+          M::mma(sa, af, qb[2 * s2][0], qb[2 * s2][1]);
+          fp8x4_to_f16x2(r[2], af[0], af[2]);
+          fp8x4_to_f16x2(r[3], af[1], af[3]);
+          M::mma(sb, af, qb[2 * s2 + 1][0], qb[2 * s2 + 1][1]);
+        }
+      } else {
+#pragma unroll
+        for (int ks = 0; ks < Tr::kKSteps; ++ks) {
+          const int c16 = ((ks & 3) << 1) | (lm >> 1);
+          const uint32_t addr = kbase + tile_offset<Tr>(row, ks >> 2) + ((c16 ^ lr) << 4);
+          uint32_t af[4];
+          ldmatrix_x4(af, addr);
+          if (ks & 1)
+            M::mma(sb, af, qb[ks][0], qb[ks][1]);
+          else
+            M::mma(sa, af, qb[ks][0], qb[ks][1]);
+        }
       }
-#pragma unroll
-      for (int e = 0; e < 4; ++e) s[e] = (sa[e] + sb[e]) * a.scale_log2;
+      s[0] = (sa[0] + sb[0]) * sc0;
+      s[1] = (sa[1] + sb[1]) * sc1;
+      s[2] = (sa[2] + sb[2]) * sc0;
+      s[3] = (sa[3] + sb[3]) * sc1;
     }
     const int tok0 = m.chunk * 16;
     const bool tail = tok0 + 16 > m.len;
@@ -533,13 +606,41 @@ __global__ void __launch_bounds__(MmaTraits<D, BS, G>::kThreads, 2)
     uint32_t pf[4];  // B fragments: hi (tokens 0-7, 8-15), lo (tokens 0-7, 8-15)
     ldmatrix_x4(pf, smem_u32(pbuf) + (lm >> 1) * 256 + lr * 32 + (lm & 1) * 16);
 
-    // ---- P.V on tensor cores: o[mt] = O^T[dim 16mt+g | +8][head 2c | 2c+1] ----
+    // ---- P.V on tensor cores: o[mt] = O^T[dim 16mt+g | +8][head 2c | 2c+1] (FP8 caches:
+    // dims 16mt+2g | 16mt+2g+1) ----
     {
-      const int row = ((lm >> 1) << 3) | lr;  // token row of the V tile
       const bool mask_lo = tail && (tok0 + 2 * c >= m.len);
       const bool mask_hi = tail && (tok0 + 2 * c + 1 >= m.len);
       const bool mask_lo8 = tail && (tok0 + 2 * c + 8 >= m.len);
       const bool mask_hi8 = tail && (tok0 + 2 * c + 9 >= m.len);
+      if constexpr (kFp8) {
+        // ldmatrix.trans of 16-bit pairs: matrix j (tokens 8(j&1).., 16-byte chunk 2mp + (j>>1))
+        // gives each lane tokens 2c, 2c+1 of dims 2g, 2g+1; a byte permute regroups them by dim
+        // (one register per dim, the two tokens as its halves) before widening to f16.
+        const int row = ((lm & 1) << 3) | lr;
+#pragma unroll
+        for (int mp = 0; mp < D / 32; ++mp) {
+          const int c16 = 2 * mp + (lm >> 1);
+          const uint32_t addr = vbase + tile_offset<Tr>(row, 0) + ((c16 ^ lr) << 4);
+          uint32_t r[4];
+          ldmatrix_x4_trans(r, addr);
+#pragma unroll
+          for (int t2 = 0; t2 < 2; ++t2) {
+            uint32_t vf[4];
+            fp8x4_to_f16x2(__byte_perm(r[2 * t2], 0u, 0x3120u), vf[0], vf[1]);
+            fp8x4_to_f16x2(__byte_perm(r[2 * t2 + 1], 0u, 0x3120u), vf[2], vf[3]);
+            if (tail) {
+              if (mask_lo) { vf[0] &= 0xffff0000u; vf[1] &= 0xffff0000u; }
+              if (mask_hi) { vf[0] &= 0x0000ffffu; vf[1] &= 0x0000ffffu; }
+              if (mask_lo8) { vf[2] &= 0xffff0000u; vf[3] &= 0xffff0000u; }
+              if (mask_hi8) { vf[2] &= 0x0000ffffu; vf[3] &= 0x0000ffffu; }
+            }
+            M::mma(o[2 * mp + t2], vf, pf[0], pf[1]);
+            M::mma(o[2 * mp + t2], vf, pf[2], pf[3]);
+          }
+        }
+      } else {
+      const int row = ((lm >> 1) << 3) | lr;  // token row of the V tile
 #pragma unroll
       for (int mt = 0; mt < Tr::kMTiles; ++mt) {
         const int c16g = (mt << 1) | (lm & 1);
@@ -556,6 +657,7 @@ __global__ void __launch_bounds__(MmaTraits<D, BS, G>::kThreads, 2)
         M::mma(o[mt], vf, pf[0], pf[1]);
         M::mma(o[mt], vf, pf[2], pf[3]);
       }
+      }
     }
     // the stage is no longer needed: hand it back to the producer
     __syncwarp();
@@ -569,7 +671,11 @@ __global__ void __launch_bounds__(MmaTraits<D, BS, G>::kThreads, 2)
         t0 += __shfl_xor_sync(FULL_MASK, t0, off);
         t1 += __shfl_xor_sync(FULL_MASK, t1, off);
       }
-      const float inv0 = 1.f / t0, inv1 = 1.f / t1;
+      float inv0 = 1.f / t0, inv1 = 1.f / t1;
+      if constexpr (kFp8) {
+        inv0 *= vsc;
+        inv1 *= vsc;
+      }
       if (a.separate_reduce && piece_at_start && lane == 0)
         a.pair_meta[m.pair] = make_int2(m.first_worker, m.npieces);
       if (m.npieces == 1) {
@@ -579,7 +685,7 @@ __global__ void __launch_bounds__(MmaTraits<D, BS, G>::kThreads, 2)
         char *row1 = row0 + (long long)a.out_h * out_elt;
 #pragma unroll
         for (int mt = 0; mt < Tr::kMTiles; ++mt) {
-          const int d0 = 16 * mt + g, d1 = d0 + 8;
+          const int d0 = kFp8 ? 16 * mt + 2 * g : 16 * mt + g, d1 = kFp8 ? d0 + 1 : d0 + 8;
           if (a.out_dtype == PA_F32) {
             if (h0 < G) {
               reinterpret_cast<float *>(row0)[d0] = o[mt][0] * inv0;
@@ -615,7 +721,7 @@ __global__ void __launch_bounds__(MmaTraits<D, BS, G>::kThreads, 2)
         float *o1 = o0 + D;
 #pragma unroll
         for (int mt = 0; mt < Tr::kMTiles; ++mt) {
-          const int d0 = 16 * mt + g, d1 = d0 + 8;
+          const int d0 = kFp8 ? 16 * mt + 2 * g : 16 * mt + g, d1 = kFp8 ? d0 + 1 : d0 + 8;
           if (h0 < G) {
             o0[d0] = o[mt][0] * inv0;
             o0[d1] = o[mt][2] * inv0;
@@ -653,30 +759,30 @@ __global__ void __launch_bounds__(MmaTraits<D, BS, G>::kThreads, 2)
   mail_post(box, mcount + wid, posted, done_msg, lane);
 }
 
-template <typename T, int D, int BS, int G>
+template <typename T, int D, int BS, int G, typename KV = T>
 cudaError_t launch_decode_mma(const DecodeArgs &a, const TmaMaps *maps, int num_ctas,
                               bool overlap_previous, cudaStream_t st) {
-  using Tr = MmaTraits<D, BS, G>;
-  return launch_overlapping(paged_decode_mma_kernel<T, D, BS, G>, num_ctas, Tr::kThreads,
+  using Tr = MmaTraits<D, BS, G, (int)sizeof(KV)>;
+  return launch_overlapping(paged_decode_mma_kernel<T, D, BS, G, KV>, num_ctas, Tr::kThreads,
                             Tr::kSmemBytes, overlap_previous, st, a, *maps);
 }
 
-template <typename T, int D, int BS, int G>
+template <typename T, int D, int BS, int G, typename KV = T>
 bool make_decode_mma(DecodeKernel *k) {
-  using Tr = MmaTraits<D, BS, G>;
+  using Tr = MmaTraits<D, BS, G, (int)sizeof(KV)>;
   static bool configured[64] = {};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
   if (!configured[dev]) {
-    if (cudaFuncSetAttribute(paged_decode_mma_kernel<T, D, BS, G>,
+    if (cudaFuncSetAttribute(paged_decode_mma_kernel<T, D, BS, G, KV>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                              Tr::kSmemBytes) != cudaSuccess)
       return false;
     configured[dev] = true;
   }
-  k->launch = &launch_decode_mma<T, D, BS, G>;
+  k->launch = &launch_decode_mma<T, D, BS, G, KV>;
   k->launch_reduce = &launch_decode_merge<G, D, BS>;
-  k->kernel = reinterpret_cast<const void *>(&paged_decode_mma_kernel<T, D, BS, G>);
+  k->kernel = reinterpret_cast<const void *>(&paged_decode_mma_kernel<T, D, BS, G, KV>);
   k->warps_per_cta = Tr::kWorkers;
   k->threads_per_cta = Tr::kThreads;
   k->smem_bytes = Tr::kSmemBytes;
@@ -704,6 +810,25 @@ template <int D>
 bool decode_table_f32(int block_size, int group, DecodeKernel *k) {
 #define PA_CASE(BB, GG) \
   if (block_size == BB && group == GG) return make_decode_simt<float, D, BB, GG>(k);
+#define PA_GROUPS(BB) PA_CASE(BB, 1) PA_CASE(BB, 2) PA_CASE(BB, 4) PA_CASE(BB, 8)
+  PA_GROUPS(8)
+  PA_GROUPS(16)
+  PA_GROUPS(32)
+#undef PA_GROUPS
+#undef PA_CASE
+  return false;
+}
+
+}  // namespace pa
+
+namespace pa {
+
+// FP8 E4M3 caches (head_dim 128) with a query of element type T: block_size {8, 16, 32} x
+// group {1, 2, 4, 8}.
+template <typename T>
+bool decode_table_fp8(int block_size, int group, DecodeKernel *k) {
+#define PA_CASE(BB, GG) \
+  if (block_size == BB && group == GG) return make_decode_mma<T, 128, BB, GG, __nv_fp8_e4m3>(k);
 #define PA_GROUPS(BB) PA_CASE(BB, 1) PA_CASE(BB, 2) PA_CASE(BB, 4) PA_CASE(BB, 8)
   PA_GROUPS(8)
   PA_GROUPS(16)

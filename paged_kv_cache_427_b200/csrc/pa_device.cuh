@@ -5,7 +5,10 @@
 
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
+#include <cuda_fp8.h>
 #include <stdint.h>
+
+#include <type_traits>
 
 #include "pa.h"
 
@@ -34,6 +37,7 @@ struct Elem<float> {
 template <>
 struct Elem<__nv_bfloat16> {
   static constexpr int kPerVec = 8;
+  static __device__ __forceinline__ float to_float(__nv_bfloat16 x) { return __bfloat162float(x); }
   // A bf16 is the upper half of an fp32: widening is a shift (low element) or a mask (high).
   static __device__ __forceinline__ void unpack(const uint4 &v, float (&f)[8]) {
     const uint32_t w[4] = {v.x, v.y, v.z, v.w};
@@ -48,6 +52,7 @@ struct Elem<__nv_bfloat16> {
 template <>
 struct Elem<__half> {
   static constexpr int kPerVec = 8;
+  static __device__ __forceinline__ float to_float(__half x) { return __half2float(x); }
   static __device__ __forceinline__ void unpack(const uint4 &v, float (&f)[8]) {
     const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll

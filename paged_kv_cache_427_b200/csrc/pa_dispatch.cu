@@ -9,6 +9,15 @@ bool decode_kernel_bf16_d64(int block_size, int group, bool tensor_cores, Decode
 bool decode_kernel_bf16_d128(int block_size, int group, bool tensor_cores, DecodeKernel *k);
 bool decode_kernel_f16_d64(int block_size, int group, bool tensor_cores, DecodeKernel *k);
 bool decode_kernel_f16_d128(int block_size, int group, bool tensor_cores, DecodeKernel *k);
+bool decode_kernel_fp8_bf16q(int block_size, int group, DecodeKernel *k);
+bool decode_kernel_fp8_f16q(int block_size, int group, DecodeKernel *k);
+
+bool decode_kernel_fp8(int q_dtype, int head_dim, int block_size, int group, DecodeKernel *k) {
+  if (head_dim != 128) return false;
+  if (q_dtype == PA_BF16) return decode_kernel_fp8_bf16q(block_size, group, k);
+  if (q_dtype == PA_F16) return decode_kernel_fp8_f16q(block_size, group, k);
+  return false;
+}
 
 bool decode_kernel_f32(int head_dim, int block_size, int group, bool tensor_cores, DecodeKernel *k) {
   if (head_dim == 64) return decode_kernel_f32_d64(block_size, group, tensor_cores, k);

@@ -35,6 +35,8 @@ struct DecodeArgs {
   float *part_ml;
   float *part_o;
   unsigned int *err;
+  const float *k_scale;   // FP8 caches: per kv head, the key/value of a code is code * scale
+  const float *v_scale;
   int separate_reduce;
   long long wait_cycles;  // limit of every wait on a copy (about one second by default)
   int test_stall;         // test hook: each warp's first stage expects 16 bytes nobody sends
@@ -99,6 +101,32 @@ struct CopyBlocksArgs {
 };
 
 cudaError_t launch_reshape_and_cache(const CacheWriteArgs &a, int num_sms, cudaStream_t st);
+
+// Quantising write into FP8 E4M3 caches: code(x / scale[h]) per element, x of element type
+// src_dtype (fp32, bf16 or fp16).
+struct CacheWriteFp8Args {
+  const char *key;
+  const char *value;
+  int src_dtype;
+  int64_t k_tok, k_head, v_tok, v_head;  // bytes
+  unsigned char *key_cache;
+  unsigned char *value_cache;
+  int64_t c_blk, c_head;  // bytes
+  int head_dim;
+  const int64_t *slots;
+  int64_t num_tokens;
+  int num_kv_heads;
+  int block_size;
+  int64_t num_slots;
+  const float *k_scale;
+  const float *v_scale;
+  unsigned int *err;
+};
+
+cudaError_t launch_reshape_and_cache_fp8(const CacheWriteFp8Args &a, int num_sms, cudaStream_t st);
+
+// Tensor-core decode for FP8 E4M3 caches with a bf16 or fp16 query (head_dim 128 only).
+bool decode_kernel_fp8(int q_dtype, int head_dim, int block_size, int group, DecodeKernel *k);
 
 // For the allocation-free entry point: the scratch bytes a pa_decode call with these shapes
 // needs (0 when the arguments are invalid), decode into a given scratch buffer, and set the
