@@ -50,13 +50,15 @@ ELT = {"f32": 4, "bf16": 2, "f16": 2}
 # byte accounting
 # ----------------------------------------------------------------------------------------------
 
-def decode_bytes(b: W.PagedBatch, out_elt: int, unique: bool = True) -> int:
+def decode_bytes(b: W.PagedBatch, out_elt: int, unique: bool = True, kv_elt: int | None = None) -> int:
     """Algorithmic bytes of one decode: each attended K/V row once (a physical slot shared by
     several sequences counts once when `unique`), Q and out rows, the block-table entries of
-    each context and the context lengths."""
+    each context and the context lengths.  kv_elt: bytes per cache element when the cache is
+    stored in another type than the batch's (FP8: 1), plus the per-head scales."""
     e = ELT[b.dtype]
+    ekv = e if kv_elt is None else kv_elt
     lens = np.maximum(b.context_lens.astype(np.int64), 0)
-    row = b.num_kv_heads * b.head_dim * e * 2  # K and V of one token, all kv heads
+    row = b.num_kv_heads * b.head_dim * ekv * 2  # K and V of one token, all kv heads
     if unique:
         slots = []
         for s, L in enumerate(lens):
@@ -69,7 +71,8 @@ def decode_bytes(b: W.PagedBatch, out_elt: int, unique: bool = True) -> int:
         kv = int(lens.sum()) * row
     qo = b.num_seqs * b.num_heads * b.head_dim * (e + out_elt)
     tables = int(((lens + b.block_size - 1) // b.block_size).sum()) * 4 + b.num_seqs * 4
-    return int(kv + qo + tables)
+    scales = 0 if kv_elt is None else b.num_kv_heads * 4 * 2
+    return int(kv + qo + tables + scales)
 
 
 def write_bytes(b: W.PagedBatch) -> int:
@@ -512,6 +515,122 @@ def run_ours(args, b: W.PagedBatch, config: dict, rank: int, world: int, local_r
     print(json.dumps(line), flush=True)
 
 
+def run_fp8(args, b, config):
+    """The same decode step over an FP8 E4M3 cache: the pool is the workload's pool quantised
+    (per-kv-head scales: largest magnitude of the head's rows / 240), each step writes the new
+    tokens with pa_reshape_and_cache_fp8 and decodes with pa_decode_fp8 launched to overlap the
+    write.  Timed like the 16-bit step: K steps with nothing between launches (`value`), then
+    the same K steps with events around each decode (the roofline)."""
+    import torch
+
+    import paged_kv_cache_427_b200 as pa
+
+    pa.load()
+    dev = torch.device("cuda", 0)
+    FP8 = torch.float8_e4m3fn
+
+    def dev_t(a, dt=None):
+        if dt == "bf16":
+            return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
+        return torch.from_numpy(np.ascontiguousarray(a)).to(dev)
+
+    kc16, vc16 = dev_t(b.key_cache, b.dtype), dev_t(b.value_cache, b.dtype)
+    # every slot the step's contexts use, except the new tokens' (the step writes those)
+    used = []
+    for s in range(b.num_seqs):
+        L = int(b.context_lens[s])
+        t = np.arange(max(L - 1, 0))
+        used.append(b.block_tables[s, t // b.block_size].astype(np.int64) * b.block_size
+                    + t % b.block_size)
+    used = np.unique(np.concatenate(used))
+    su = torch.from_numpy(used).to(dev)
+    rows_k = kc16[su // b.block_size, :, su % b.block_size, :].contiguous()  # [n, Hkv, D]
+    rows_v = vc16[su // b.block_size, :, su % b.block_size, :].contiguous()
+    key, value = dev_t(b.key, b.dtype), dev_t(b.value, b.dtype)
+    ks = (torch.cat([rows_k, key]).float().abs().amax(dim=(0, 2)) / 240.0).clamp_min(1e-8).contiguous()
+    vs = (torch.cat([rows_v, value]).float().abs().amax(dim=(0, 2)) / 240.0).clamp_min(1e-8).contiguous()
+    att = attended_bytes(b) // 2
+    rot = args.rotations or max(2, min(8, math.ceil(3 * L2_BYTES / max(att, 1)) + 1))
+    pools = []
+    for _ in range(rot):
+        kc = torch.full(kc16.shape, 0x7f, dtype=torch.uint8, device=dev).view(FP8)
+        vc = torch.full(vc16.shape, 0x7f, dtype=torch.uint8, device=dev).view(FP8)
+        pa.pa_reshape_and_cache_fp8(rows_k, rows_v, kc, vc, su, ks, vs)
+        pools.append((kc, vc))
+    del kc16, vc16, rows_k, rows_v
+    q = dev_t(b.query, b.dtype)
+    slots, tables, lens = dev_t(b.slot_mapping), dev_t(b.block_tables), dev_t(b.context_lens)
+    out = torch.empty(q.shape, dtype=q.dtype, device=dev)
+    ws = torch.zeros(pa.pa_decode_workspace_bytes(b.num_seqs, b.num_heads, b.num_kv_heads,
+                                                  b.head_dim, 0), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step(i, ev=None):
+        kc, vc = pools[i % rot]
+        pa.pa_reshape_and_cache_fp8(key, value, kc, vc, slots, ks, vs)
+        if ev is not None:
+            ev[0].record(stream)
+        pa.pa_decode_fp8(out, q, kc, vc, tables, lens, ks, vs, b.scale, b.block_size,
+                         b.num_kv_heads, 0, pa.PA_DECODE_OVERLAP_PREVIOUS, ws)
+        if ev is not None:
+            ev[1].record(stream)
+
+    sampler = ClockSampler(None).start()
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    t_soak = time.perf_counter()
+    i = 0
+    while time.perf_counter() - t_soak < args.soak:
+        for _ in range(200):
+            step(i)
+            i += 1
+        torch.cuda.synchronize()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    start.record(stream)
+    for i in range(args.steps):
+        step(i)
+    end.record(stream)
+    torch.cuda.synchronize()
+    elapsed_ms = start.elapsed_time(end)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    for i in range(args.steps):
+        step(i, evs[i])
+    torch.cuda.synchronize()
+    dec_mean = float(np.mean([s_.elapsed_time(e_) for s_, e_ in evs]))
+    clocks = sampler.stop()
+    flags = pa.pa_get_device_error(clear=True)
+    if flags:
+        print(f"warning: device error word 0x{flags:x}", file=sys.stderr)
+    dec = decode_bytes(b, ELT[b.dtype], unique=True, kv_elt=1)
+    t_new = int((b.slot_mapping >= 0).sum())
+    wbytes = t_new * b.num_kv_heads * b.head_dim * (ELT[b.dtype] + 1) * 2 + len(b.slot_mapping) * 8
+    ms = elapsed_ms / args.steps
+    value = (dec + wbytes) / (ms * 1e-3) / 1e9
+    peak, peak_src = hbm_peak()
+    achieved = dec / (dec_mean * 1e-3) / 1e9
+    line = {"metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": 1,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 5),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "fp8_e4m3 cache, bf16 query", "data": "synthetic",
+            "config": dict(config, kv_dtype="fp8_e4m3", pool_rotations=rot,
+                           kv_scales="per kv head: max |x| / 240"),
+            "attended_tokens_per_s": round(b.attended_tokens / (ms * 1e-3), 1),
+            "seq_steps_per_s": round(b.num_seqs / (ms * 1e-3), 1),
+            "pct_of_8TBs": round(100 * value / NOMINAL_HBM_GBS, 2),
+            "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak,
+                         "unit": "GB/s", "frac": round(achieved / peak, 4), "traffic": None,
+                         "kernel": "paged_decode_mma_kernel (fp8 e4m3 cache)",
+                         "peak_source": peak_src, "algorithmic_bytes_per_launch": dec,
+                         "mean_launch_us": round(dec_mean * 1e3, 3),
+                         "launch_timing": "CUDA events around each decode launch, in a second "
+                                          "timed region of the same K steps"},
+            "gpu_launches": 2 * args.steps, "clocks": clocks}
+    print(json.dumps(line), flush=True)
+
+
 def run_swap(args, b, config):
     """Block swap between the device cache and a pinned host cache: every block the batch's
     sequences use goes out (device -> host, scattered host ids) and back in (host -> device,
@@ -600,6 +719,8 @@ def main():
     ap.add_argument("--soak", type=float, default=1.0, help="seconds of untimed load for the clock sampler")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--kv", default="native", choices=["native", "fp8"],
+                    help="fp8: the same step over an FP8 E4M3 cache (pa_decode_fp8)")
     ap.add_argument("--swap", action="store_true",
                     help="measure block swap (pa_swap_blocks) of the workload's blocks instead")
     args = ap.parse_args()
@@ -633,6 +754,10 @@ def main():
     if args.swap:
         if rank == 0:
             run_swap(args, b, config)
+        return
+    if args.kv == "fp8":
+        if rank == 0:
+            run_fp8(args, b, config)
         return
     if world > 1:
         import datetime
