@@ -78,6 +78,9 @@ class Oracle:
         lib.pao_decode_range.restype = _I32
         lib.pao_decode_range_scaled.argtypes = lib.pao_decode_range.argtypes + [_P, _P]
         lib.pao_decode_range_scaled.restype = _I32
+        lib.pao_prefill.argtypes = [_P, _P, _I32, _P, _P, _I32, _P, _I64, _P, _P, _I64, _I32,
+                                    _I32, _I32, _I32, _I64, _D, _I32]
+        lib.pao_prefill.restype = _I32
         lib.pao_fp8_encode.argtypes = [_P, _I32, _I64, ctypes.c_float, _P]
         lib.pao_fp8_encode.restype = None
         lib.pao_fp8_decode.argtypes = [_P, _I64, _P]
@@ -195,6 +198,28 @@ class Oracle:
         out, _, _ = self.decode_range(query, key_cache, value_cache, block_tables, context_lens,
                                       scale, dtype, 0, np.iinfo(np.int64).max, q_dtype,
                                       num_threads, k_scale, v_scale)
+        return out
+
+    def prefill(self, query, key_cache, value_cache, block_tables, context_lens, query_start,
+                scale, dtype: str, q_dtype: str | None = None, num_threads: int = 0) -> np.ndarray:
+        """Causal attention of each sequence's new tokens (query rows query_start[s] ..
+        query_start[s+1]-1, the last positions of its context): [total new, Hq, D] float64."""
+        q_dtype = q_dtype or dtype
+        nb, hkv, bs, d = key_cache.shape
+        tq, hq, dq = query.shape
+        q = _raw(query, q_dtype)
+        kc = _raw(key_cache, dtype)
+        vc = _raw(value_cache, dtype)
+        bt = np.ascontiguousarray(block_tables, dtype=np.int32)
+        cl = np.ascontiguousarray(context_lens, dtype=np.int32)
+        qs = np.ascontiguousarray(query_start, dtype=np.int32)
+        out = np.zeros((tq, hq, d), dtype=np.float64)
+        rc = self._lib.pao_prefill(
+            _ptr(out), _ptr(q), DTYPE_CODE[q_dtype], _ptr(kc), _ptr(vc), DTYPE_CODE[dtype], _ptr(bt),
+            bt.shape[1] if bt.ndim == 2 else 0, _ptr(cl), _ptr(qs), cl.shape[0], hq, hkv, d, bs,
+            nb, float(scale), int(num_threads))
+        if rc != 0:
+            raise ValueError(f"oracle prefill failed with status {rc}")
         return out
 
     def lse_combine(self, o_parts, m, l) -> np.ndarray:

@@ -430,6 +430,79 @@ int pao_decode_range_scaled(double *out, double *m_out, double *l_out, const voi
   return status;
 }
 
+/*
+ * Prefill (several new tokens per sequence) over a paged cache.  [P2] 4.2: at each iteration
+ * requests join the running batch; a joining request's prompt tokens (or a chunk of them) are
+ * the step's new tokens, already written into the sequence's blocks.  Sequence s has
+ * q_len = query_start[s+1] - query_start[s] new tokens, the last q_len of its context_len
+ * positions; new token j (position p = context_len - q_len + j) attends causally, to positions
+ * 0 .. p of the context assembled through the block table ([P4] 2.2.2).
+ *
+ *   out    [total new tokens][num_heads][head_dim] double, row query_start[s] + j
+ *   query  [total new tokens][num_heads][head_dim] q_dtype
+ * A sequence with q_len > context_len is an error (PAO_BAD_ARG).
+ */
+int pao_prefill(double *out, const void *query, int q_dtype, const void *key_cache,
+                const void *value_cache, int kv_dtype, const int32_t *block_tables,
+                int64_t max_blocks, const int32_t *context_lens, const int32_t *query_start,
+                int64_t num_seqs, int num_heads, int num_kv_heads, int head_dim, int block_size,
+                int64_t num_blocks, double scale, int num_threads) {
+  if (num_seqs < 0 || num_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0 ||
+      max_blocks < 0 || num_heads % num_kv_heads != 0)
+    return PAO_BAD_ARG;
+  for (int64_t s = 0; s < num_seqs; ++s) {
+    const int64_t q_len = (int64_t)query_start[s + 1] - query_start[s];
+    if (q_len < 0 || q_len > context_lens[s]) return PAO_BAD_ARG;
+    if (context_lens[s] > max_blocks * (int64_t)block_size) return PAO_BAD_CONTEXT_LEN;
+  }
+  const int group = num_heads / num_kv_heads;
+  int status = PAO_OK;
+#ifdef _OPENMP
+  if (num_threads <= 0) num_threads = omp_get_max_threads();
+#pragma omp parallel for collapse(2) schedule(dynamic, 1) num_threads(num_threads)
+#endif
+  for (int64_t s = 0; s < num_seqs; ++s) {
+    for (int h = 0; h < num_heads; ++h) {
+      const int64_t len = context_lens[s];
+      const int64_t q0 = query_start[s], q_len = (int64_t)query_start[s + 1] - q0;
+      if (q_len == 0) continue;
+      const int g = h / group;
+      double *kc = (double *)malloc((size_t)len * (size_t)head_dim * sizeof(double));
+      double *vc = (double *)malloc((size_t)len * (size_t)head_dim * sizeof(double));
+      double *q = (double *)malloc((size_t)head_dim * sizeof(double));
+      double *z = (double *)malloc((size_t)len * sizeof(double));
+      int rc = (!kc || !vc || !q || !z) ? PAO_NO_MEMORY : PAO_OK;
+      if (rc == PAO_OK)
+        rc = assemble_context(kc, vc, key_cache, value_cache, kv_dtype,
+                              block_tables + (size_t)s * (size_t)max_blocks, num_blocks,
+                              num_kv_heads, block_size, head_dim, g, len);
+      for (int64_t j = 0; j < q_len; ++j) {
+        double *o = out + ((size_t)(q0 + j) * (size_t)num_heads + (size_t)h) * (size_t)head_dim;
+        if (rc != PAO_OK) {
+          for (int d = 0; d < head_dim; ++d) o[d] = NAN;
+          continue;
+        }
+        const int64_t p = len - q_len + j; /* this token's position: it sees 0 .. p */
+        const size_t qrow = ((size_t)(q0 + j) * (size_t)num_heads + (size_t)h) * (size_t)head_dim;
+        for (int d = 0; d < head_dim; ++d) q[d] = elt_to_double(query, qrow + (size_t)d, q_dtype);
+        double m, l;
+        attend_rows(o, &m, &l, q, kc, vc, 0, p + 1, head_dim, scale, z);
+      }
+      if (rc != PAO_OK) {
+#ifdef _OPENMP
+#pragma omp atomic write
+#endif
+        status = rc;
+      }
+      free(kc);
+      free(vc);
+      free(q);
+      free(z);
+    }
+  }
+  return status;
+}
+
 int pao_decode_range(double *out, double *m_out, double *l_out, const void *query, int q_dtype,
                      const void *key_cache, const void *value_cache, int kv_dtype,
                      const int32_t *block_tables, int64_t max_blocks, const int32_t *context_lens,

@@ -97,10 +97,14 @@ class PagedBatch:
     logical_key: list | None = None
     logical_value: list | None = None
     meta: dict = field(default_factory=dict)
+    # Prefill steps: the new tokens of sequence s are query rows query_start[s] ..
+    # query_start[s+1]-1 (and key/value/slot_mapping rows alike), the last positions of its
+    # context.  None for decode steps (one new token per sequence).
+    query_start: np.ndarray | None = None
 
     @property
     def num_seqs(self) -> int:
-        return int(self.query.shape[0])
+        return int(self.context_lens.shape[0])
 
     @property
     def num_blocks(self) -> int:
@@ -192,6 +196,66 @@ def build_batch(name: str, context_lens, *, num_heads: int, num_kv_heads: int, h
                       slot_mapping=slots, block_tables=tables, context_lens=lens,
                       logical_key=lk, logical_value=lv,
                       meta={"seed": seed, "perm_salt": perm_salt, "fill": fill})
+
+
+def build_prefill_batch(name: str, context_lens, q_lens, *, num_heads: int, num_kv_heads: int,
+                        head_dim: int, block_size: int, dtype: str, seed: int,
+                        pool_factor: float = 1.25, max_blocks: int | None = None,
+                        fill: str = "nan", keep_logical: bool = False) -> PagedBatch:
+    """A step in which sequence s brings q_lens[s] new tokens (a prompt chunk; 1 = a decode
+    token): positions context_lens[s] - q_lens[s] .. context_lens[s] - 1.  The pool holds each
+    sequence's earlier tokens; the new tokens' rows and slots are the step's write, and their
+    query rows are concatenated in sequence order.  Values as in build_batch."""
+    lens = np.asarray(context_lens, dtype=np.int32)
+    ql = np.asarray(q_lens, dtype=np.int32)
+    if np.any(ql < 0) or np.any(ql > lens):
+        raise ValueError("0 <= q_len <= context_len")
+    S = len(lens)
+    tables, nb = _assign_blocks(lens, block_size, None, pool_factor,
+                                np.random.default_rng([seed, 3, 0]), max_blocks)
+    kc = _fill_pool((nb, num_kv_heads, block_size, head_dim), dtype, fill)
+    vc = _fill_pool((nb, num_kv_heads, block_size, head_dim), dtype, fill)
+    keys, values, slots = [], [], []
+    lk, lv = ([], []) if keep_logical else (None, None)
+    for s in range(S):
+        L, q = int(lens[s]), int(ql[s])
+        rng = np.random.default_rng([seed, 1, s])
+        ks = _normal(rng, (L, num_kv_heads, head_dim), dtype)
+        vs = _normal(rng, (L, num_kv_heads, head_dim), dtype)
+        _place(kc, tables[s], 0, ks[:L - q], block_size)
+        _place(vc, tables[s], 0, vs[:L - q], block_size)
+        t = np.arange(L - q, L)
+        keys.append(ks[L - q:])
+        values.append(vs[L - q:])
+        slots.append(tables[s, t // block_size].astype(np.int64) * block_size + t % block_size)
+        if keep_logical:
+            lk.append(ks)
+            lv.append(vs)
+    total = int(ql.sum())
+    query = _normal(np.random.default_rng([seed, 2]), (total, num_heads, head_dim), dtype)
+    qs = np.zeros(S + 1, dtype=np.int32)
+    qs[1:] = np.cumsum(ql)
+    return PagedBatch(name=name, dtype=dtype, num_heads=num_heads, num_kv_heads=num_kv_heads,
+                      head_dim=head_dim, block_size=block_size, scale=1.0 / math.sqrt(head_dim),
+                      query=query, key_cache=kc, value_cache=vc,
+                      key=np.concatenate(keys) if keys else np.zeros((0, num_kv_heads, head_dim), STORAGE[dtype]),
+                      value=np.concatenate(values) if values else np.zeros((0, num_kv_heads, head_dim), STORAGE[dtype]),
+                      slot_mapping=np.concatenate(slots) if slots else np.zeros(0, np.int64),
+                      block_tables=tables, context_lens=lens, logical_key=lk,
+                      logical_value=lv, meta={"seed": seed, "fill": fill}, query_start=qs)
+
+
+def chunked_prefill(num_seqs: int = 8, chunk: int = 256, max_context: int = 2048,
+                    seed: int = BASE_SEED + 6) -> PagedBatch:
+    """Chunked prefill on Llama-3-8B shapes (32/8 heads, head_dim 128, bf16, block_size 16):
+    each sequence brings a prompt chunk of `chunk` tokens on top of an earlier prefix of
+    U[0, max_context - chunk] tokens (rounded to whole chunks)."""
+    rng = np.random.default_rng([seed, 0])
+    prefix = rng.integers(0, (max_context - chunk) // chunk + 1, num_seqs) * chunk
+    lens = (prefix + chunk).astype(np.int32)
+    return build_prefill_batch("chunked_prefill", lens, np.full(num_seqs, chunk, np.int32),
+                               num_heads=32, num_kv_heads=8, head_dim=128, block_size=16,
+                               dtype="bf16", seed=seed)
 
 
 # ----------------------------------------------------------------------------------------------
@@ -376,6 +440,8 @@ def workload(name: str, **kw) -> PagedBatch:
         return shared_prefix(**kw)
     if name == "long_mixed":
         return long_mixed(**kw)
+    if name == "chunked_prefill":
+        return chunked_prefill(**kw)
     raise KeyError(name)
 
 

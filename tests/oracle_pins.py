@@ -474,6 +474,44 @@ def pin_fp8_cache(orc):
             assert np.allclose(got[s, h], ref.astype(np.float64), rtol=1e-12, atol=1e-15), (s, h)
 
 
+def pin_prefill(orc):
+    """Causal prefill ([P2] 4.2: requests join the batch with their prompt): every new token's
+    row equals the decode oracle's attention of that query over the context positions 0 .. p
+    (bit for bit: the same sum), torch's float64 scaled_dot_product_attention with a causal mask
+    on the contiguous K/V agrees, and a 1-token chunk is exactly the decode step."""
+    import torch
+    b = W.build_prefill_batch("prefill", [5, 40, 17, 64, 9], [5, 13, 1, 30, 0], num_heads=8,
+                              num_kv_heads=2, head_dim=64, block_size=8, dtype="bf16",
+                              seed=W.BASE_SEED + 707, keep_logical=True)
+    kc, vc = b.key_cache.copy(), b.value_cache.copy()
+    assert orc.reshape_and_cache(b.key, b.value, kc, vc, b.slot_mapping, b.dtype) == 0
+    got = orc.prefill(b.query, kc, vc, b.block_tables, b.context_lens, b.query_start, b.scale, b.dtype)
+    qs = b.query_start
+    group = b.num_heads // b.num_kv_heads
+    for s in range(b.num_seqs):
+        L, q0, q1 = int(b.context_lens[s]), int(qs[s]), int(qs[s + 1])
+        for j in range(q1 - q0):
+            p = L - (q1 - q0) + j
+            one = orc.decode(b.query[q0 + j][None], kc, vc, b.block_tables[s][None],
+                             np.array([p + 1], np.int32), b.scale, b.dtype)
+            assert np.array_equal(got[q0 + j], one[0]), (s, j)
+        if q1 == q0:
+            continue
+        K = torch.from_numpy(W.decode_to_f64(b.logical_key[s][:L], "bf16")).permute(1, 0, 2)
+        V = torch.from_numpy(W.decode_to_f64(b.logical_value[s][:L], "bf16")).permute(1, 0, 2)
+        Q = torch.from_numpy(W.decode_to_f64(b.query[q0:q1], "bf16")).permute(1, 0, 2)
+        K = K.repeat_interleave(group, dim=0)
+        V = V.repeat_interleave(group, dim=0)
+        pos = torch.arange(L - (q1 - q0), L)[:, None]
+        mask = torch.arange(L)[None, :] <= pos
+        ref = torch.nn.functional.scaled_dot_product_attention(Q, K, V, attn_mask=mask,
+                                                               scale=b.scale)
+        assert np.allclose(got[q0:q1], ref.permute(1, 0, 2).numpy(), rtol=1e-12, atol=1e-14)
+    last = orc.decode(b.query[qs[2]:qs[3]], kc, vc, b.block_tables[2:3], b.context_lens[2:3],
+                      b.scale, b.dtype)
+    assert np.array_equal(got[qs[2]:qs[3]], last)
+
+
 def pin_shared_prefix(orc):
     """Sequences sharing prefix blocks read the same bytes: the paged result over the shared
     pool equals brute force on each member's own logical stream."""
@@ -514,5 +552,5 @@ def pin_zero_context(orc):
 ALL_PINS = [
     pin_brute_force, pin_torch_sdpa, pin_closed_forms, pin_decimal_example,
     pin_placement_invariance, pin_unread_table_entries, pin_cache_write, pin_copy_blocks,
-    pin_swap_blocks, pin_fp8_codec, pin_fp8_cache, pin_shared_prefix, pin_split_merge, pin_zero_context,
+    pin_swap_blocks, pin_fp8_codec, pin_fp8_cache, pin_prefill, pin_shared_prefix, pin_split_merge, pin_zero_context,
 ]

@@ -59,6 +59,13 @@ MUTANTS = {
                             "if (slot < 0) { ++skipped; continue; }"),
     "fp8_v_scaled_by_k": ("const double vs = v_scale ? (double)v_scale[g] : 1.0;",
                           "const double vs = k_scale ? (double)k_scale[g] : 1.0;"),
+    "prefill_causal_limit": ("attend_rows(o, &m, &l, q, kc, vc, 0, p + 1, head_dim, scale, z);",
+                             "attend_rows(o, &m, &l, q, kc, vc, 0, p, head_dim, scale, z);"),
+    "prefill_query_row": (
+        "const size_t qrow = ((size_t)(q0 + j) * (size_t)num_heads + (size_t)h) * (size_t)head_dim;",
+        "const size_t qrow = ((size_t)(q0 + q_len - 1 - j) * (size_t)num_heads + (size_t)h) * (size_t)head_dim;"),
+    "prefill_positions": ("const int64_t p = len - q_len + j; /* this token's position: it sees 0 .. p */",
+                          "const int64_t p = j; /* this token's position: it sees 0 .. p */"),
     "bf16_shift": ("uint32_t u = (uint32_t)h << 16;", "uint32_t u = (uint32_t)h << 15;"),
     "f16_bias": ("v = ldexp((double)(m | 0x400), e - 25);", "v = ldexp((double)(m | 0x400), e - 24);"),
     "merge_sign": ("const double w = l[p] * exp(m[p] - big_m);",
