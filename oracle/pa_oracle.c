@@ -466,7 +466,7 @@ int pao_prefill(double *out, const void *query, int q_dtype, const void *key_cac
       const int64_t len = context_lens[s];
       const int64_t q0 = query_start[s], q_len = (int64_t)query_start[s + 1] - q0;
       if (q_len == 0) continue;
-      const int g = h / group;
+      const int kvh = h / group; /* the kv head query head h reads */
       double *kc = (double *)malloc((size_t)len * (size_t)head_dim * sizeof(double));
       double *vc = (double *)malloc((size_t)len * (size_t)head_dim * sizeof(double));
       double *q = (double *)malloc((size_t)head_dim * sizeof(double));
@@ -475,7 +475,7 @@ int pao_prefill(double *out, const void *query, int q_dtype, const void *key_cac
       if (rc == PAO_OK)
         rc = assemble_context(kc, vc, key_cache, value_cache, kv_dtype,
                               block_tables + (size_t)s * (size_t)max_blocks, num_blocks,
-                              num_kv_heads, block_size, head_dim, g, len);
+                              num_kv_heads, block_size, head_dim, kvh, len);
       for (int64_t j = 0; j < q_len; ++j) {
         double *o = out + ((size_t)(q0 + j) * (size_t)num_heads + (size_t)h) * (size_t)head_dim;
         if (rc != PAO_OK) {

@@ -59,6 +59,8 @@ MUTANTS = {
                             "if (slot < 0) { ++skipped; continue; }"),
     "fp8_v_scaled_by_k": ("const double vs = v_scale ? (double)v_scale[g] : 1.0;",
                           "const double vs = k_scale ? (double)k_scale[g] : 1.0;"),
+    "prefill_gqa_mapping": ("const int kvh = h / group; /* the kv head query head h reads */",
+                            "const int kvh = h % num_kv_heads;"),
     "prefill_causal_limit": ("attend_rows(o, &m, &l, q, kc, vc, 0, p + 1, head_dim, scale, z);",
                              "attend_rows(o, &m, &l, q, kc, vc, 0, p, head_dim, scale, z);"),
     "prefill_query_row": (
