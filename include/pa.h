@@ -62,7 +62,7 @@
 extern "C" {
 #endif
 
-#define PA_VERSION 4
+#define PA_VERSION 5
 
 /* Symbols of this ABI are the only ones the shared library exports. */
 #if defined(__GNUC__)
@@ -201,6 +201,29 @@ PA_API int pa_decode_fp8(const pa_tensor *out, const pa_tensor *query, const pa_
                          const pa_tensor *v_scale, float scale, int32_t block_size,
                          int32_t num_kv_heads, int32_t num_workers, uint32_t flags,
                          void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * pa_prefill - causal attention of a step's new tokens (a prompt, or a chunk of one, of each
+ * sequence joining or continuing in the batch: [P2] 4.2) over the paged cache.  Sequence s
+ * brings q_len = query_start[s+1] - query_start[s] new tokens, already written into its blocks
+ * (pa_reshape_and_cache); they are its last q_len positions, and new token j (query row
+ * query_start[s] + j, position p = context_lens[s] - q_len + j) attends to positions 0 .. p:
+ *   out[r, h, :] = softmax_{t <= p}(scale * q[r, h, :] . K_t) . V_t,
+ * K_t, V_t assembled through the block table as in pa_decode ([P4] 2.2.2).
+ *   query, out: [T, Hq, D] (T = query_start[S]); out fp32 or the caches' type.
+ *   query_start: [S + 1] int32, non-decreasing from 0; block_tables [S, max_blocks];
+ *   context_lens [S].  Caches bf16 or fp16 (fp32 / FP8: PA_ERR_UNSUPPORTED), head_dim 64 or
+ *   128, block_size 8/16/32, 1/2/4/8 query heads per kv head.
+ * A sequence with q_len > context_len, or whose rows fall outside [0, T), sets
+ * PA_DEVERR_CONTEXT_LEN and its rows are not written.  Rows of tokens past query_start[S] are not written.  One kernel: a persistent grid
+ * of 4-warp CTAs, each taking tiles of 64 query rows (64/G tokens x G heads) of one (sequence,
+ * kv head) and streaming that sequence's K/V tiles up to the tile's last position through a
+ * TMA ring; the tensor cores (mma.sync) compute S = QK^T and O = PV with P kept to ~16 bits.
+ */
+PA_API int pa_prefill(const pa_tensor *out, const pa_tensor *query, const pa_tensor *key_cache,
+                      const pa_tensor *value_cache, const pa_tensor *block_tables,
+                      const pa_tensor *context_lens, const pa_tensor *query_start, float scale,
+                      int32_t block_size, int32_t num_kv_heads, void *stream);
 
 /*
  * pa_copy_blocks - copy whole physical blocks (all kv heads, all slots, both caches):

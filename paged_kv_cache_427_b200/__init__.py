@@ -76,6 +76,7 @@ def load(path: str = LIBRARY) -> ctypes.CDLL:
     lib.pa_reshape_and_cache.argtypes = [_T, _T, _T, _T, _T, _P]
     lib.pa_copy_blocks.argtypes = [_T, _T, _T, _P]
     lib.pa_swap_blocks.argtypes = [_T, _T, _T, _T, _T, _P]
+    lib.pa_prefill.argtypes = [_T, _T, _T, _T, _T, _T, _T, f32, i32, i32, _P]
     lib.pa_reshape_and_cache_fp8.argtypes = [_T, _T, _T, _T, _T, _T, _T, _P]
     lib.pa_decode_fp8.argtypes = [_T, _T, _T, _T, _T, _T, _T, _T, f32, i32, i32, i32, u32, _P, sz, _P]
     lib.pa_decode.argtypes = [_T, _T, _T, _T, _T, _T, f32, i32, i32, _P]
@@ -162,6 +163,17 @@ def pa_swap_blocks(src_key_cache, src_value_cache, dst_key_cache, dst_value_cach
     d = [describe(x) for x in (src_key_cache, src_value_cache, dst_key_cache, dst_value_cache,
                                block_mapping)]
     _check("pa_swap_blocks", lib.pa_swap_blocks(*[ctypes.byref(x) for x in d], _stream(stream)))
+
+
+def pa_prefill(out, query, key_cache, value_cache, block_tables, context_lens, query_start, scale,
+               block_size, num_kv_heads, stream=None):
+    """Causal attention of each sequence's new tokens (rows query_start[s] ..
+    query_start[s+1]-1, its last positions) over the paged cache (see include/pa.h)."""
+    lib = load()
+    d = [describe(x) for x in (out, query, key_cache, value_cache, block_tables, context_lens,
+                               query_start)]
+    _check("pa_prefill", lib.pa_prefill(*[ctypes.byref(x) for x in d], float(scale),
+                                        int(block_size), int(num_kv_heads), _stream(stream)))
 
 
 def pa_reshape_and_cache_fp8(key, value, key_cache, value_cache, slot_mapping, k_scale, v_scale,

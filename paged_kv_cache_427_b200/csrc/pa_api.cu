@@ -801,6 +801,108 @@ int write_fp8_impl(const pa_tensor *key, const pa_tensor *value, const pa_tensor
 
 extern "C" {
 
+int pa_prefill(const pa_tensor *out, const pa_tensor *query, const pa_tensor *key_cache,
+               const pa_tensor *value_cache, const pa_tensor *block_tables,
+               const pa_tensor *context_lens, const pa_tensor *query_start, float scale,
+               int32_t block_size, int32_t num_kv_heads, void *stream) {
+  int rc;
+  CacheShape cs;
+  if ((rc = check_caches(key_cache, value_cache, &cs))) return rc;
+  if ((rc = check_tensor(query, "query", 3)) || (rc = check_tensor(out, "out", 3)) ||
+      (rc = check_tensor(block_tables, "block_tables", 2)) ||
+      (rc = check_tensor(context_lens, "context_lens", 1)) ||
+      (rc = check_tensor(query_start, "query_start", 1)))
+    return rc;
+  if (block_size != cs.block_size)
+    return fail(PA_ERR_SHAPE, "block_size %d does not match the cache's %d", block_size, cs.block_size);
+  if (num_kv_heads != cs.num_kv_heads)
+    return fail(PA_ERR_SHAPE, "num_kv_heads %d does not match the cache's %d", num_kv_heads, cs.num_kv_heads);
+  const int64_t S = context_lens->shape[0];
+  const int64_t T = query->shape[0];
+  const int64_t Hq = query->shape[1];
+  const int D = cs.head_dim;
+  if (query->shape[2] != D) return fail(PA_ERR_SHAPE, "query head_dim %lld != cache head_dim %d", (long long)query->shape[2], D);
+  if (out->shape[0] != T || out->shape[1] != Hq || out->shape[2] != D)
+    return fail(PA_ERR_SHAPE, "out must be [num_tokens, num_heads, head_dim] like query");
+  if (block_tables->shape[0] != S || query_start->shape[0] != S + 1)
+    return fail(PA_ERR_SHAPE, "block_tables needs one row and query_start S + 1 entries for S sequences");
+  if (cs.dtype != PA_BF16 && cs.dtype != PA_F16)
+    return fail(PA_ERR_UNSUPPORTED, "prefill is built for bf16 and fp16 caches");
+  if (query->dtype != cs.dtype) return fail(PA_ERR_DTYPE, "query must have the caches' element type");
+  if (out->dtype != PA_F32 && out->dtype != cs.dtype)
+    return fail(PA_ERR_DTYPE, "out must be fp32 or the caches' element type");
+  if (block_tables->dtype != PA_I32 || context_lens->dtype != PA_I32 || query_start->dtype != PA_I32)
+    return fail(PA_ERR_DTYPE, "block_tables, context_lens and query_start must be int32");
+  if (Hq <= 0 && T > 0) return fail(PA_ERR_SHAPE, "num_heads must be positive");
+  if (Hq % num_kv_heads != 0) return fail(PA_ERR_SHAPE, "num_heads %lld is not a multiple of num_kv_heads %d", (long long)Hq, num_kv_heads);
+  const int G = (int)(Hq / num_kv_heads);
+  if (D != 64 && D != 128) return fail(PA_ERR_UNSUPPORTED, "head_dim %d (built: 64, 128)", D);
+  if (block_size != 8 && block_size != 16 && block_size != 32)
+    return fail(PA_ERR_UNSUPPORTED, "block_size %d (built: 8, 16, 32)", block_size);
+  if (G != 1 && G != 2 && G != 4 && G != 8)
+    return fail(PA_ERR_UNSUPPORTED, "query heads per kv head %d (built: 1, 2, 4, 8)", G);
+  if (query->stride[2] != 1 || out->stride[2] != 1)
+    return fail(PA_ERR_LAYOUT, "query and out need a contiguous head_dim");
+  if (!aligned16(query->data) || !strides16(query, 2) || !aligned16(out->data) || !strides16(out, 2))
+    return fail(PA_ERR_LAYOUT, "query/out: data and token/head strides must be 16-byte aligned");
+  if (block_tables->stride[1] != 1 && block_tables->shape[1] > 1)
+    return fail(PA_ERR_LAYOUT, "block_tables rows must be contiguous");
+  if ((context_lens->stride[0] != 1 && S > 1) || query_start->stride[0] != 1)
+    return fail(PA_ERR_LAYOUT, "context_lens and query_start must be contiguous");
+  if (S > 0x7fffffff || T > 0x7fffffff || block_tables->shape[1] * block_size > 0x7fffffff)
+    return fail(PA_ERR_SHAPE, "too many sequences or tokens, or too long a block table");
+  if (!std::isfinite(scale)) return fail(PA_ERR_INVALID_ARG, "scale must be finite");
+  if (S == 0 || T == 0) return PA_OK;
+  DeviceState *ds;
+  int dev;
+  if ((rc = device_state(&ds, &dev))) return rc;
+  if ((rc = check_device_memory(key_cache, "key_cache", dev)) ||
+      (rc = check_device_memory(value_cache, "value_cache", dev)) ||
+      (rc = check_device_memory(query, "query", dev)) || (rc = check_device_memory(out, "out", dev)) ||
+      (rc = check_device_memory(block_tables, "block_tables", dev)) ||
+      (rc = check_device_memory(context_lens, "context_lens", dev)) ||
+      (rc = check_device_memory(query_start, "query_start", dev)))
+    return rc;
+  pa::PrefillKernel k;
+  const bool got = cs.dtype == PA_BF16 ? pa::prefill_kernel_bf16(D, block_size, G, &k)
+                                       : pa::prefill_kernel_f16(D, block_size, G, &k);
+  if (!got)
+    return fail(PA_ERR_CUDA, "could not prepare the prefill kernel: %s", cudaGetErrorString(cudaGetLastError()));
+  pa::TmaMaps maps;
+  if ((rc = cache_map(key_cache, k.tma_rows, &maps.k)) || (rc = cache_map(value_cache, k.tma_rows, &maps.v)))
+    return rc;
+  // enough CTAs for every tile of any split of T tokens among S sequences, at most one wave
+  const int64_t tiles = ((T + k.tokens_per_tile - 1) / k.tokens_per_tile + S) * num_kv_heads;
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k.kernel, k.threads_per_cta,
+                                                    k.smem_bytes) != cudaSuccess || per_sm < 1)
+    per_sm = 1;
+  const int64_t wave = (int64_t)per_sm * ds->num_sms;
+  const int ctas = (int)(tiles < wave ? tiles : wave);
+  pa::PrefillArgs a;
+  a.out = out->data;
+  a.out_dtype = out->dtype;
+  a.out_t = out->stride[0];
+  a.out_h = out->stride[1];
+  a.query = query->data;
+  a.q_t = query->stride[0];
+  a.q_h = query->stride[1];
+  a.block_tables = static_cast<const int32_t *>(block_tables->data);
+  a.bt_s = block_tables->stride[0];
+  a.context_lens = static_cast<const int32_t *>(context_lens->data);
+  a.query_start = static_cast<const int32_t *>(query_start->data);
+  a.num_seqs = (int)S;
+  a.num_kv_heads = num_kv_heads;
+  a.max_blocks = (int)block_tables->shape[1];
+  a.num_blocks = cs.num_blocks;
+  a.num_tokens = T;
+  a.scale_log2 = (float)((double)scale * 1.4426950408889634);
+  a.err = ds->err;
+  a.wait_cycles = test_hooks().wait_cycles;
+  cudaError_t e = k.launch(a, &maps, ctas, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? PA_OK : cuda_fail(e, "prefill launch");
+}
+
 int pa_reshape_and_cache_fp8(const pa_tensor *key, const pa_tensor *value,
                              const pa_tensor *key_cache, const pa_tensor *value_cache,
                              const pa_tensor *slot_mapping, const pa_tensor *k_scale,

@@ -1,0 +1,123 @@
+"""pa_prefill: causal attention of each sequence's new tokens over the paged cache, compared
+with the oracle (fp32 out within the 16-bit tolerance, 16-bit out against the rounding of the
+fp64 result) on a mixed continuously batched step (whole prompts, prompt chunks on top of a
+prefix, single decode tokens, a sequence with no new token), for every built configuration, on
+the full-size chunked-prefill workload (sampled), and on its error cases."""
+import numpy as np
+import pytest
+import torch
+
+import paged_kv_cache_427_b200 as pa
+from paged_kv_cache_427_b200 import workloads as W
+from tests.gpu_helpers import (TORCH_DTYPE, assert_bf16_output, assert_close,
+                               assert_no_device_error, require_gpu, to_host, to_torch)
+
+pytestmark = pytest.mark.gpu
+
+
+class PrefillStep:
+    def __init__(self, b):
+        self.b = b
+        dt = b.dtype
+        self.query = to_torch(b.query, dt)
+        self.key_cache = to_torch(b.key_cache, dt)
+        self.value_cache = to_torch(b.value_cache, dt)
+        self.key, self.value = to_torch(b.key, dt), to_torch(b.value, dt)
+        self.slots = to_torch(b.slot_mapping)
+        self.tables = to_torch(b.block_tables)
+        self.lens = to_torch(b.context_lens)
+        self.qs = to_torch(b.query_start)
+        pa.pa_reshape_and_cache(self.key, self.value, self.key_cache, self.value_cache, self.slots)
+
+    def run(self, out_dtype):
+        b = self.b
+        out = torch.full(self.query.shape, float("nan"), dtype=TORCH_DTYPE[out_dtype], device="cuda")
+        pa.pa_prefill(out, self.query, self.key_cache, self.value_cache, self.tables, self.lens,
+                      self.qs, b.scale, b.block_size, b.num_kv_heads)
+        return to_host(out, out_dtype)
+
+
+def _oracle(orc, b):
+    kc, vc = b.key_cache.copy(), b.value_cache.copy()
+    assert orc.reshape_and_cache(b.key, b.value, kc, vc, b.slot_mapping, b.dtype) == 0
+    ref = orc.prefill(b.query, kc, vc, b.block_tables, b.context_lens, b.query_start, b.scale, b.dtype)
+    return ref, kc, vc
+
+
+def test_prefill_mixed_batch(oracle):
+    require_gpu()
+    b = W.build_prefill_batch("pf", [300, 77, 16, 1, 640, 33, 200, 95],
+                              [300, 13, 16, 1, 128, 0, 1, 95], num_heads=32, num_kv_heads=8,
+                              head_dim=128, block_size=16, dtype="bf16", seed=W.BASE_SEED + 740)
+    ref, kc, vc = _oracle(oracle, b)
+    st = PrefillStep(b)
+    assert np.array_equal(to_host(st.key_cache, "bf16"), kc)
+    assert np.array_equal(to_host(st.value_cache, "bf16"), vc)
+    assert_close(st.run("f32"), ref, "bf16", "prefill mixed batch")
+    assert_bf16_output(st.run("bf16"), ref, "prefill bf16 out")
+    assert_no_device_error()
+
+
+@pytest.mark.parametrize("dtype,D,bs,hq,hkv", [
+    ("bf16", 64, 8, 8, 8), ("bf16", 64, 32, 16, 8), ("bf16", 128, 8, 16, 2),
+    ("bf16", 128, 32, 32, 4), ("f16", 128, 16, 32, 8), ("f16", 64, 16, 8, 1),
+    ("bf16", 128, 16, 64, 8), ("f16", 128, 8, 16, 16),
+])
+def test_prefill_configurations(oracle, dtype, D, bs, hq, hkv):
+    require_gpu()
+    b = W.build_prefill_batch("pfcfg", [70, 5, 129, 40], [70, 5, 41, 1], num_heads=hq,
+                              num_kv_heads=hkv, head_dim=D, block_size=bs, dtype=dtype,
+                              seed=W.BASE_SEED + 741 + D + bs + hq)
+    ref, _, _ = _oracle(oracle, b)
+    st = PrefillStep(b)
+    assert_close(st.run("f32"), ref, dtype, f"prefill {dtype} D{D} bs{bs} G{hq // hkv}")
+    assert_no_device_error()
+
+
+def test_prefill_chunked_workload_sampled(oracle):
+    """The full-size chunked-prefill step on the GPU; the oracle recomputes three of its
+    sequences (their rows of the output)."""
+    require_gpu()
+    b = W.chunked_prefill()
+    st = PrefillStep(b)
+    got = st.run("f32")
+    pick = [0, 3, 6]
+    qs = b.query_start
+    sub = W.build_prefill_batch("sub", b.context_lens[pick], qs[1:][pick] - qs[:-1][pick],
+                                num_heads=32, num_kv_heads=8, head_dim=128, block_size=16,
+                                dtype="bf16", seed=0)  # shapes only
+    rows = np.concatenate([np.arange(qs[s], qs[s + 1]) for s in pick])
+    kc, vc = b.key_cache.copy(), b.value_cache.copy()
+    assert oracle.reshape_and_cache(b.key, b.value, kc, vc, b.slot_mapping, b.dtype) == 0
+    ref = oracle.prefill(b.query[rows], kc, vc, b.block_tables[pick], b.context_lens[pick],
+                         sub.query_start, b.scale, b.dtype)
+    assert_close(got[rows], ref, "bf16", "chunked prefill (sampled sequences)")
+    assert_no_device_error()
+
+
+def test_prefill_single_tokens_match_decode():
+    """One new token per sequence is a decode step: pa_prefill and pa_decode agree (two
+    kernels, so within the tolerance rather than bit for bit)."""
+    require_gpu()
+    b = W.build_prefill_batch("pfdec", [17, 300, 1, 64], [1, 1, 1, 1], num_heads=32,
+                              num_kv_heads=8, head_dim=128, block_size=16, dtype="bf16",
+                              seed=W.BASE_SEED + 742)
+    st = PrefillStep(b)
+    got = st.run("f32")
+    out = torch.empty(st.query.shape, dtype=torch.float32, device="cuda")
+    pa.pa_decode(out, st.query, st.key_cache, st.value_cache, st.tables, st.lens, b.scale,
+                 b.block_size, b.num_kv_heads)
+    assert_close(got, to_host(out, "f32"), "bf16", "prefill vs decode")
+
+
+def test_prefill_more_new_tokens_than_context_is_flagged():
+    require_gpu()
+    b = W.build_prefill_batch("pfbad", [40, 40], [10, 10], num_heads=8, num_kv_heads=2,
+                              head_dim=64, block_size=16, dtype="bf16", seed=W.BASE_SEED + 743)
+    st = PrefillStep(b)
+    st.lens.copy_(torch.tensor([40, 5], dtype=torch.int32))  # sequence 1: 10 new tokens, context 5
+    pa.pa_get_device_error(clear=True)
+    got = st.run("f32")
+    assert pa.pa_get_device_error(clear=True) & pa.PA_DEVERR_CONTEXT_LEN
+    assert np.all(np.isnan(got[10:20]))      # rows of the bad sequence untouched
+    assert np.all(np.isfinite(got[:10]))
