@@ -631,6 +631,108 @@ def run_fp8(args, b, config):
     print(json.dumps(line), flush=True)
 
 
+def prefill_flops(b: W.PagedBatch) -> int:
+    """Algorithmic FLOPs of a prefill step: each new token's row of each query head takes
+    2*D FLOPs per attended position for q.K and 2*D for P.V (causal: positions 0 .. p)."""
+    qs = b.query_start
+    tot = 0
+    for s in range(b.num_seqs):
+        L, q = int(b.context_lens[s]), int(qs[s + 1] - qs[s])
+        p = np.arange(L - q, L, dtype=np.int64)
+        tot += int((p + 1).sum())
+    return 4 * b.head_dim * b.num_heads * tot
+
+
+def run_prefill(args, b, config):
+    """A chunked-prefill step: the new tokens' K/V written (pa_reshape_and_cache), then
+    pa_prefill.  Timed like the decode step; the roofline is tensor-bound, against the measured
+    bf16 dense GEMM rate (the burst figure: the kernel is timed alone per launch)."""
+    import torch
+
+    import paged_kv_cache_427_b200 as pa
+
+    pa.load()
+    dev = torch.device("cuda", 0)
+
+    def dev_t(a, dt=None):
+        if dt == "bf16":
+            return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
+        return torch.from_numpy(np.ascontiguousarray(a)).to(dev)
+
+    kc0, vc0 = dev_t(b.key_cache, b.dtype), dev_t(b.value_cache, b.dtype)
+    att = attended_bytes(b)
+    rot = args.rotations or max(2, min(8, math.ceil(3 * L2_BYTES / max(att, 1)) + 1))
+    pools = [(kc0, vc0)] + [(kc0.clone(), vc0.clone()) for _ in range(rot - 1)]
+    q = dev_t(b.query, b.dtype)
+    key, value = dev_t(b.key, b.dtype), dev_t(b.value, b.dtype)
+    slots, tables = dev_t(b.slot_mapping), dev_t(b.block_tables)
+    lens, qs = dev_t(b.context_lens), dev_t(b.query_start)
+    out = torch.empty(q.shape, dtype=q.dtype, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step(i, ev=None):
+        kc, vc = pools[i % rot]
+        pa.pa_reshape_and_cache(key, value, kc, vc, slots)
+        if ev is not None:
+            ev[0].record(stream)
+        pa.pa_prefill(out, q, kc, vc, tables, lens, qs, b.scale, b.block_size, b.num_kv_heads)
+        if ev is not None:
+            ev[1].record(stream)
+
+    sampler = ClockSampler(None).start()
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    t_soak = time.perf_counter()
+    i = 0
+    while time.perf_counter() - t_soak < args.soak:
+        for _ in range(50):
+            step(i)
+            i += 1
+        torch.cuda.synchronize()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    start.record(stream)
+    for i in range(args.steps):
+        step(i)
+    end.record(stream)
+    torch.cuda.synchronize()
+    elapsed_ms = start.elapsed_time(end)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    for i in range(args.steps):
+        step(i, evs[i])
+    torch.cuda.synchronize()
+    k_ms = float(np.mean([s_.elapsed_time(e_) for s_, e_ in evs]))
+    clocks = sampler.stop()
+    flags = pa.pa_get_device_error(clear=True)
+    if flags:
+        print(f"warning: device error word 0x{flags:x}", file=sys.stderr)
+    flops = prefill_flops(b)
+    ms = elapsed_ms / args.steps
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            peak, src = float(json.load(f)["bf16_tflops"]), "measured"
+    except Exception:
+        peak, src = 1590.0, "fallback"
+    tflops = flops / (k_ms * 1e-3) / 1e12
+    new_tokens = int(b.query_start[-1])
+    line = {"metric": "paged prefill attention TFLOP/s, new tokens/s", "value": round(flops / (ms * 1e-3) / 1e12, 2),
+            "unit": "TFLOP/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(ms, 5), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": b.dtype, "data": "synthetic",
+            "config": dict(config, new_tokens=new_tokens, pool_rotations=rot,
+                           query_lens=[int(x) for x in np.diff(b.query_start)]),
+            "new_tokens_per_s": round(new_tokens / (ms * 1e-3), 1),
+            "roofline": {"bound": "tensor", "achieved": round(tflops, 2), "peak": peak,
+                         "unit": "TFLOP/s", "frac": round(tflops / peak, 4), "traffic": None,
+                         "kernel": "paged_prefill_kernel (mma.sync + TMA)", "peak_source": src,
+                         "algorithmic_flops_per_launch": flops,
+                         "mean_launch_us": round(k_ms * 1e3, 3)},
+            "gpu_launches": 2 * args.steps, "clocks": clocks}
+    print(json.dumps(line), flush=True)
+
+
 def run_swap(args, b, config):
     """Block swap between the device cache and a pinned host cache: every block the batch's
     sequences use goes out (device -> host, scattered host ids) and back in (host -> device,
@@ -710,7 +812,8 @@ def main():
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--workload", default="llama3_8b_decode",
-                    help="llama3_8b_decode | short_chat_bs{8,16,32} | shared_prefix | long_mixed | tiny_fp32")
+                    help="llama3_8b_decode | short_chat_bs{8,16,32} | shared_prefix | long_mixed | "
+                         "tiny_fp32 | chunked_prefill (pa_prefill)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--decode-flags", type=int, default=4,
                     help="pa_decode_ex flags: 4 = start while the cache write runs (default), "
@@ -758,6 +861,10 @@ def main():
     if args.kv == "fp8":
         if rank == 0:
             run_fp8(args, b, config)
+        return
+    if b.query_start is not None:
+        if rank == 0:
+            run_prefill(args, b, config)
         return
     if world > 1:
         import datetime

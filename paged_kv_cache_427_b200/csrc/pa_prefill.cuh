@@ -252,19 +252,27 @@ __global__ void __launch_bounds__(PrefillTraits<D, BS, G>::kThreads)
       const int t0 = i * 16;
 
       // ---- S = Q K^T (rows g | g+8, positions t0 + 8nt + 2c | +1) ----
-      float sc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+      float sc[2][4];
       {
+        // four independent accumulator chains (n-tile x even/odd k-step), summed at the end
+        float sx[2][2][4] = {};
         const int row = ((lm >> 1) << 3) | lr;
 #pragma unroll
         for (int ks = 0; ks < Tr::kKSteps; ++ks) {
           const int c16 = ((ks & 3) << 1) | (lm & 1);
           uint32_t r[4];
           ldmatrix_x4(r, kb + tile_offset<Tr>(row, ks >> 2) + ((c16 ^ lr) << 4));
-          M::mma(sc[0], qa[ks], r[0], r[1]);
-          M::mma(sc[1], qa[ks], r[2], r[3]);
+          M::mma(sx[0][ks & 1], qa[ks], r[0], r[1]);
+          M::mma(sx[1][ks & 1], qa[ks], r[2], r[3]);
         }
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) sc[nt][e] = sx[nt][0][e] + sx[nt][1][e];
       }
-      // ---- causal mask, online softmax per row ----
+      // ---- causal mask, online softmax per row: the reference maximum of a row moves only
+      // when a logit passes it by more than 8 (base 2), so weights stay <= 256 and most
+      // chunks skip the rescale of O ----
       float cmax[2] = {-INFINITY, -INFINITY};
 #pragma unroll
       for (int nt = 0; nt < 2; ++nt)
@@ -275,25 +283,24 @@ __global__ void __launch_bounds__(PrefillTraits<D, BS, G>::kThreads)
           sc[nt][e] = t <= prow[ri] ? sc[nt][e] * a.scale_log2 : -INFINITY;
           cmax[ri] = fmaxf(cmax[ri], sc[nt][e]);
         }
+      if (__any_sync(FULL_MASK, cmax[0] > mrow[0] + 8.f || cmax[1] > mrow[1] + 8.f)) {
+        float alpha[2];
 #pragma unroll
-      for (int ri = 0; ri < 2; ++ri) {
-        cmax[ri] = fmaxf(cmax[ri], __shfl_xor_sync(FULL_MASK, cmax[ri], 1));
-        cmax[ri] = fmaxf(cmax[ri], __shfl_xor_sync(FULL_MASK, cmax[ri], 2));
-      }
-      float mnew[2], alpha[2];
+        for (int ri = 0; ri < 2; ++ri) {
+          cmax[ri] = fmaxf(cmax[ri], __shfl_xor_sync(FULL_MASK, cmax[ri], 1));
+          cmax[ri] = fmaxf(cmax[ri], __shfl_xor_sync(FULL_MASK, cmax[ri], 2));
+          const float mnew = fmaxf(mrow[ri], cmax[ri]);
+          alpha[ri] = mnew == -INFINITY ? 1.f : fast_exp2(mrow[ri] - mnew);
+          mrow[ri] = mnew;
+          lrow[ri] *= alpha[ri];
+        }
 #pragma unroll
-      for (int ri = 0; ri < 2; ++ri) {
-        mnew[ri] = fmaxf(mrow[ri], cmax[ri]);
-        alpha[ri] = mnew[ri] == -INFINITY ? 1.f : exp2f(mrow[ri] - mnew[ri]);
-        mrow[ri] = mnew[ri];
-        lrow[ri] *= alpha[ri];
-      }
-#pragma unroll
-      for (int nt = 0; nt < Tr::kNTiles; ++nt) {
-        o[nt][0] *= alpha[0];
-        o[nt][1] *= alpha[0];
-        o[nt][2] *= alpha[1];
-        o[nt][3] *= alpha[1];
+        for (int nt = 0; nt < Tr::kNTiles; ++nt) {
+          o[nt][0] *= alpha[0];
+          o[nt][1] *= alpha[0];
+          o[nt][2] *= alpha[1];
+          o[nt][3] *= alpha[1];
+        }
       }
       float p[2][4];
 #pragma unroll
@@ -301,7 +308,7 @@ __global__ void __launch_bounds__(PrefillTraits<D, BS, G>::kThreads)
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const int ri = e >> 1;
-          p[nt][e] = mnew[ri] == -INFINITY ? 0.f : exp2f(sc[nt][e] - mnew[ri]);
+          p[nt][e] = mrow[ri] == -INFINITY ? 0.f : fast_exp2(sc[nt][e] - mrow[ri]);
           lrow[ri] += p[nt][e];
         }
       // ---- O += P V: P (16 rows x 16 positions) as the A fragment, hi and lo terms ----
@@ -335,8 +342,8 @@ __global__ void __launch_bounds__(PrefillTraits<D, BS, G>::kThreads)
             }
           }
           M::mma(o[2 * j2], ph, r[0], r[1]);
-          M::mma(o[2 * j2], pl, r[0], r[1]);
           M::mma(o[2 * j2 + 1], ph, r[2], r[3]);
+          M::mma(o[2 * j2], pl, r[0], r[1]);
           M::mma(o[2 * j2 + 1], pl, r[2], r[3]);
         }
       }
