@@ -104,13 +104,17 @@ def hbm_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
+DECODE_SOURCES = ("pa_decode_mma.cuh", "pa_decode_common.cuh", "pa_decode.cuh", "pa_device.cuh",
+                  "pa_internal.h", "pa_decode_bf16_d128.cu")
+
+
 def kernel_sources_digest() -> str:
-    """Digest of the files the decode kernels are compiled from (device code and the argument
-    block), not the host-side API."""
+    """Digest of the files the 16-bit decode kernels are compiled from (device code and the
+    argument block), not the host-side API or the other kernels."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "paged_kv_cache_427_b200", "csrc")
     for f in sorted(os.listdir(csrc)):
-        if f.endswith((".cuh", ".h")) or (f.startswith("pa_decode_") and f.endswith(".cu")):
+        if f in DECODE_SOURCES:
             with open(os.path.join(csrc, f), "rb") as fh:
                 h.update(f.encode() + fh.read())
     return h.hexdigest()[:16]
