@@ -224,6 +224,58 @@ def cpu_baseline(b: W.PagedBatch, budget_s: float = 10.0):
             "attended_tokens_per_s": round(toks / dt, 1)}
 
 
+def cpu_baseline_fp8(b: W.PagedBatch, kc8, vc8, ks, vs, budget_s: float = 10.0):
+    """The oracle's decode over the FP8 pool (codes copied from the device), first n sequences."""
+    import oracle
+
+    orc = oracle.load()
+    n = 1
+    while True:
+        sub = W.sub_batch(b, np.arange(n))
+        t0 = time.perf_counter()
+        orc.decode(sub["query"], kc8, vc8, sub["block_tables"], sub["context_lens"], b.scale,
+                   "fp8", q_dtype=b.dtype, k_scale=ks, v_scale=vs)
+        dt = time.perf_counter() - t0
+        if dt >= budget_s or n == b.num_seqs:
+            break
+        n = min(b.num_seqs, max(n + 1, int(n * min(8.0, budget_s / max(dt, 1e-4)))))
+    sb = W.PagedBatch(**{**b.__dict__, "query": sub["query"], "block_tables": sub["block_tables"],
+                          "context_lens": sub["context_lens"]})
+    nbytes = decode_bytes(sb, ELT[b.dtype], unique=False, kv_elt=1)
+    toks = int(sub["context_lens"].sum())
+    return {"value": round(nbytes / dt / 1e9, 4), "unit": "GB/s", "cores": orc.max_threads(),
+            "kind": "oracle",
+            "sample": f"oracle decode over the FP8 pool (fp64, OpenMP) of the first {n} of "
+                      f"{b.num_seqs} sequences ({toks} attended tokens), one run of {dt:.2f} s",
+            "attended_tokens_per_s": round(toks / dt, 1)}
+
+
+def cpu_baseline_prefill(b: W.PagedBatch, budget_s: float = 10.0):
+    """The oracle's prefill of the first n sequences (their new tokens' rows)."""
+    import oracle
+
+    orc = oracle.load()
+    kc, vc = b.key_cache.copy(), b.value_cache.copy()
+    orc.reshape_and_cache(b.key, b.value, kc, vc, b.slot_mapping, b.dtype)
+    qs = b.query_start
+    n = 1
+    while True:
+        t0 = time.perf_counter()
+        orc.prefill(b.query[:qs[n]], kc, vc, b.block_tables[:n], b.context_lens[:n], qs[:n + 1],
+                    b.scale, b.dtype)
+        dt = time.perf_counter() - t0
+        if dt >= budget_s or n == b.num_seqs:
+            break
+        n = min(b.num_seqs, max(n + 1, int(n * min(8.0, budget_s / max(dt, 1e-4)))))
+    sb = W.PagedBatch(**{**b.__dict__, "context_lens": b.context_lens[:n], "query_start": qs[:n + 1]})
+    flops = prefill_flops(sb)
+    return {"value": round(flops / dt / 1e12, 6), "unit": "TFLOP/s", "cores": orc.max_threads(),
+            "kind": "oracle",
+            "sample": f"oracle prefill (fp64, OpenMP) of the first {n} of {b.num_seqs} sequences "
+                      f"({int(qs[n])} new tokens), one run of {dt:.2f} s",
+            "new_tokens_per_s": round(int(qs[n]) / dt, 1)}
+
+
 def run_reference(args, b: W.PagedBatch, config: dict):
     import oracle
 
@@ -632,6 +684,11 @@ def run_fp8(args, b, config):
                          "launch_timing": "CUDA events around each decode launch, in a second "
                                           "timed region of the same K steps"},
             "gpu_launches": 2 * args.steps, "clocks": clocks}
+    if not args.no_cpu_baseline:
+        kc8, vc8 = pools[0]
+        line["cpu_baseline"] = cpu_baseline_fp8(
+            b, kc8.view(torch.uint8).cpu().numpy(), vc8.view(torch.uint8).cpu().numpy(),
+            ks.cpu().numpy(), vs.cpu().numpy(), args.cpu_seconds)
     print(json.dumps(line), flush=True)
 
 
@@ -734,6 +791,8 @@ def run_prefill(args, b, config):
                          "algorithmic_flops_per_launch": flops,
                          "mean_launch_us": round(k_ms * 1e3, 3)},
             "gpu_launches": 2 * args.steps, "clocks": clocks}
+    if not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline_prefill(b, args.cpu_seconds)
     print(json.dumps(line), flush=True)
 
 
@@ -807,6 +866,22 @@ def run_swap(args, b, config):
             "roofline": {"bound": "host link", "peak_source": "cudaMemcpyAsync of one contiguous "
                          "pinned buffer of the same bytes, same run"},
             "gpu_launches": 2 * reps}
+    if not args.no_cpu_baseline:
+        import oracle
+
+        orc = oracle.load()
+        hk_o = np.empty((n,) + b.key_cache.shape[1:], dtype=b.key_cache.dtype)
+        hv_o = np.empty_like(hk_o)
+        pairs = np.stack([ids, host_ids], 1)
+        t0, k = time.perf_counter(), 0
+        while time.perf_counter() - t0 < min(args.cpu_seconds, 5.0) or k == 0:
+            orc.swap_blocks(b.key_cache, b.value_cache, hk_o, hv_o, pairs, b.dtype)
+            k += 1
+        dt = (time.perf_counter() - t0) / k
+        line["cpu_baseline"] = {"value": round(total / dt / 1e9, 4), "unit": "GB/s", "cores": 1,
+                                "kind": "oracle",
+                                "sample": f"oracle swap-out of the same {n} blocks (host memory to "
+                                          f"host memory), {k} runs"}
     print(json.dumps(line), flush=True)
 
 
