@@ -21,8 +21,14 @@
 //   * O += P V: the S accumulators are already laid out as the A fragment of the next MMA
 //     (16 rows x 16 positions); P is split into two 16-bit terms (hi + lo) as in the decode
 //     kernel; V fragments come from the value tile by ldmatrix.trans, head_dim as N.
-// Tiles are spread over a persistent grid (x = blockIdx.x, += gridDim.x); warp 0 finds the
-// (sequence, tile) of a tile index by a scan of query_start, 32 sequences per step.
+// Tiles differ in cost (a tile's causal prefix), so they are spread longest first: every CTA
+// builds the same list of (sequence, tile) pairs sorted by cost (a histogram of costs in shared
+// memory, a prefix over it, a scatter) and takes positions of the list in snake order (round r
+// gives CTA i position r*P + i, or r*P + P-1-i when r is odd), which keeps the heaviest tiles on
+// different CTAs and evens out the sums.  Ties land in any order: each tile's rows are computed
+// by one CTA alone, so the order changes no result.  Steps too large for the shared list fall
+// back to tiles in sequence order, x = blockIdx.x, += gridDim.x, warp 0 finding the (sequence,
+// tile) of x by a scan of query_start.
 #pragma once
 
 #include "pa_decode_mma.cuh"
@@ -45,7 +51,12 @@ struct PrefillTraits {
   static constexpr int kNTiles = D / 8;
   static constexpr int kBarOff = kStages * kStageBytes;
   static constexpr int kInfoOff = kBarOff + kStages * 16;
-  static constexpr int kSmemBytes = kInfoOff + 32 + 1024;  // + 1 KB alignment
+  // longest-first schedule: a histogram of tile costs (chunks) and the sorted tile list
+  static constexpr int kMaxBins = 2048;  // costs 0 .. 2047 chunks (contexts up to 32K tokens)
+  static constexpr int kMaxList = 4096;  // (sequence, tile) pairs
+  static constexpr int kBinsOff = kInfoOff + 32;
+  static constexpr int kListOff = kBinsOff + kMaxBins * 4;
+  static constexpr int kSmemBytes = kListOff + kMaxList * 4 + 1024;  // + 1 KB alignment
   static_assert(D == 64 || D == 128, "head_dim 64 or 128");
   static_assert(G == 1 || G == 2 || G == 4 || G == 8, "1, 2, 4 or 8 query heads per kv head");
 };
@@ -116,7 +127,7 @@ __global__ void __launch_bounds__(PrefillTraits<D, BS, G>::kThreads)
   unsigned char *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   uint64_t *full = reinterpret_cast<uint64_t *>(smem + Tr::kBarOff);
   uint64_t *empty = full + ST;
-  int *info = reinterpret_cast<int *>(smem + Tr::kInfoOff);  // [s, tau, abort]
+  int *info = reinterpret_cast<int *>(smem + Tr::kInfoOff);  // [s, tau, abort, tile count]
 
   const int lane = threadIdx.x & 31;
   const int wid = threadIdx.x >> 5;
@@ -139,22 +150,107 @@ __global__ void __launch_bounds__(PrefillTraits<D, BS, G>::kThreads)
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&maps.v)) : "memory");
   }
 
-  long long pos = 0;  // ring items used so far by this CTA (every thread keeps the same count)
-  for (long long x = blockIdx.x;; x += gridDim.x) {
-    if (wid == 0) {
-      int s, tau;
-      locate_tile<Tr::kTokens>(a, x / Hkv, s, tau);
-      if (lane == 0) {
-        info[0] = s;
-        info[1] = tau;
+  // ---- the longest-first schedule ----
+  int *bins = reinterpret_cast<int *>(smem + Tr::kBinsOff);
+  int *list = reinterpret_cast<int *>(smem + Tr::kListOff);
+  const int nbins = (max_len + 15) / 16 + 1;
+  bool sorted = nbins <= Tr::kMaxBins && a.num_seqs < (1 << 19);
+  if (sorted) {
+    for (int i = threadIdx.x; i < nbins; i += Tr::kThreads) bins[i] = 0;
+    if (threadIdx.x == 0) info[3] = 0;
+  }
+  __syncthreads();
+  auto seq_tiles = [&](int sq, int &len_out, int &q_out) {
+    const int q0s = __ldg(a.query_start + sq);
+    const int qn = __ldg(a.query_start + sq + 1) - q0s;
+    const int raw = __ldg(a.context_lens + sq);
+    const int Ls = raw < 0 ? 0 : (raw > max_len ? max_len : raw);
+    len_out = Ls;
+    q_out = qn;
+    if (qn > Ls || q0s < 0 || (long long)q0s + qn > a.num_tokens) return -1;  // invalid
+    return qn > 0 ? (qn + Tr::kTokens - 1) / Tr::kTokens : 0;
+  };
+  auto tile_cost = [&](int Ls, int qn, int t) {
+    const int last = min((t + 1) * Tr::kTokens, qn);  // tokens up to this tile's last one
+    return (Ls - qn + last + 15) / 16;
+  };
+  if (sorted) {
+    for (int sq = threadIdx.x; sq < a.num_seqs; sq += Tr::kThreads) {
+      int Ls, qn;
+      const int nt = seq_tiles(sq, Ls, qn);
+      if (nt < 0) {
+        // new tokens outside the context, or query rows outside the query tensor: report
+        set_error(a.err, PA_DEVERR_CONTEXT_LEN);
+        continue;
       }
+      for (int t = 0; t < nt && t < Tr::kMaxList; ++t) atomicAdd(bins + tile_cost(Ls, qn, t), 1);
+      atomicAdd(info + 3, nt);
     }
-    __syncthreads();
-    const int s = info[0], tau = info[1];
-    const bool aborted = info[2] != 0;
-    __syncthreads();  // info is rewritten for the next tile only after every thread read it
-    if (s < 0 || aborted) break;
-    const int kvh = (int)(x % Hkv);
+  }
+  __syncthreads();
+  const int ntiles = sorted ? info[3] : 0;
+  sorted = sorted && ntiles <= Tr::kMaxList;
+  if (sorted && wid == 0) {
+    // bins[c] <- number of tiles costing more than c: where the tiles of cost c start
+    const int seg = (nbins + 31) / 32;
+    const int hi = nbins - 1 - lane * seg;  // this lane's costs: hi, hi-1, .., hi-seg+1
+    int sum = 0;
+    for (int i = 0; i < seg; ++i)
+      if (hi - i >= 0) sum += bins[hi - i];
+    int incl = sum;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int v = __shfl_up_sync(FULL_MASK, incl, off);
+      if (lane >= off) incl += v;
+    }
+    int run = incl - sum;
+    for (int i = 0; i < seg; ++i)
+      if (hi - i >= 0) {
+        const int n = bins[hi - i];
+        bins[hi - i] = run;
+        run += n;
+      }
+  }
+  __syncthreads();
+  if (sorted) {
+    for (int sq = threadIdx.x; sq < a.num_seqs; sq += Tr::kThreads) {
+      int Ls, qn;
+      const int nt = seq_tiles(sq, Ls, qn);
+      for (int t = 0; t < nt; ++t) list[atomicAdd(bins + tile_cost(Ls, qn, t), 1)] = (sq << 12) | t;
+    }
+  }
+  __syncthreads();
+
+  long long pos = 0;  // ring items used so far by this CTA (every thread keeps the same count)
+  const long long total = (long long)ntiles * Hkv;
+  for (long long round = 0;; ++round) {
+    int s, tau, kvh;
+    if (sorted) {
+      const long long k = round * gridDim.x +
+                          ((round & 1) ? (long long)gridDim.x - 1 - blockIdx.x : (long long)blockIdx.x);
+      if (k >= total || info[2] != 0) break;
+      const int e = list[k / Hkv];
+      s = e >> 12;
+      tau = e & 4095;
+      kvh = (int)(k % Hkv);
+    } else {
+      const long long x = blockIdx.x + round * gridDim.x;
+      if (wid == 0) {
+        int ls, lt_;
+        locate_tile<Tr::kTokens>(a, x / Hkv, ls, lt_);
+        if (lane == 0) {
+          info[0] = ls;
+          info[1] = lt_;
+        }
+      }
+      __syncthreads();
+      s = info[0];
+      tau = info[1];
+      const bool aborted = info[2] != 0;
+      __syncthreads();  // info is rewritten for the next tile only after every thread read it
+      if (s < 0 || aborted) break;
+      kvh = (int)(x % Hkv);
+    }
     const int q0 = __ldg(a.query_start + s);
     const int q_len = __ldg(a.query_start + s + 1) - q0;
     const int raw_len = __ldg(a.context_lens + s);
