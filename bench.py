@@ -832,7 +832,7 @@ def run_prefill(args, b, config):
             "new_tokens_per_s": round(new_tokens / (ms * 1e-3), 1),
             "roofline": {"bound": "tensor", "achieved": round(tflops, 2), "peak": peak,
                          "unit": "TFLOP/s", "frac": round(tflops / peak, 4), "traffic": None,
-                         "kernel": "paged_prefill_kernel (mma.sync + TMA)", "peak_source": src,
+                         "kernel": "paged_prefill_tc_kernel (tcgen05 + TMEM + TMA)", "peak_source": src,
                          "algorithmic_flops_per_launch": flops,
                          "mean_launch_us": round(k_ms * 1e3, 3)},
             "gpu_launches": 2 * args.steps, "clocks": clocks}

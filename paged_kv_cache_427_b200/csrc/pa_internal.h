@@ -152,7 +152,7 @@ struct PrefillKernel {
   const void *kernel;
   int threads_per_cta;
   int smem_bytes;
-  int tokens_per_tile;  // query tokens of one tile (64 rows / query heads per kv head)
+  int tokens_per_tile;  // query tokens of one tile (128 rows / query heads per kv head)
   int tma_rows;
 };
 

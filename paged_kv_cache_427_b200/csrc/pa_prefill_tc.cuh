@@ -1,0 +1,683 @@
+// pa_prefill_tc.cuh - causal attention of a step's new tokens over the paged cache (prefill, or
+// a chunk of a prompt in a continuously batched step) on the fifth-generation tensor cores:
+// tcgen05 MMAs from shared memory into tensor memory.
+//
+// Sources: [P2] "vLLM core features: PagedAttention, Continuous Batching, quantization
+// support, distributed inference" 4.2 (at each iteration requests join the running batch: a
+// joining request's prompt tokens are that step's new tokens) and [P4] "vLLM core
+// architecture: model loading, PagedAttention principle, KV cache management" 2.2.2 (attention
+// assembles the whole KV sequence through the block table).  Token j of sequence s's q_len new
+// tokens sits at position p = context_len - q_len + j and attends to positions 0 .. p.
+//
+// A tile is 128 query rows of one (sequence, kv head): 128 / G new tokens times the G query
+// heads that read that kv head (head fastest), one row per tensor-memory lane.  The context is
+// walked in kv tiles of 128 positions.  One persistent CTA per SM, six warps:
+//   * warp 4 (one lane) streams the key and value tiles of 128 positions through two-slot rings
+//     by TMA: 8-position boxes of the paged cache (both 64-element spans of the head, 128-byte
+//     swizzle) placed one after another, which is the operand layout of the MMAs;
+//   * warp 5 (one lane) issues the MMAs: S = Q K^T (M = 128 rows, N = 128 positions, K = head
+//     dim) into one of two S buffers in tensor memory, and O += P V (N = head dim, K = 128
+//     positions) into the O accumulator, P split into two 16-bit terms (hi + lo) as in the
+//     decode kernels so the weights keep about 16 significant bits;
+//   * warps 0-3 (one thread per row) copy the tile's query rows into shared memory, read S from
+//     tensor memory, apply the causal mask (which also hides positions past the context), keep
+//     the online softmax per row in base 2 with a lazy reference maximum (moved only when a
+//     logit passes it by 2^8, when O is rescaled in tensor memory), write P to shared memory and
+//     finally read O, divide by the row sums and store the rows.
+// The MMA warp issues S of kv tile j + 1 before O += P V of tile j, so the tensor cores compute
+// the next scores while the softmax warps work on the current ones.  Barriers between the roles
+// are mbarriers (copies: transaction bytes; MMAs: tcgen05.commit; threads: arrival counts);
+// every wait is bounded and a timeout sets an error bit and winds the CTA down.
+//
+// Tiles differ in cost (a tile's causal prefix), so they are spread longest first: every CTA
+// builds the same list of (sequence, tile) pairs sorted by cost (a histogram of costs in shared
+// memory, a prefix over it, a scatter) and takes positions of the list in snake order (round r
+// gives CTA i position r*P + i, or r*P + P-1-i when r is odd).  Ties land in any order: each
+// tile's rows are computed by one CTA alone, so the order changes no result.  Steps too large
+// for the shared list fall back to tiles in sequence order, x = blockIdx.x, += gridDim.x, each
+// warp finding the (sequence, tile) of x by a scan of query_start.
+#pragma once
+
+#include "pa_decode_mma.cuh"
+#include "pa_tc.cuh"
+
+namespace pa {
+
+template <int D, int BS, int G>
+struct PrefillTcTraits {
+  static constexpr int kThreads = 192;
+  static constexpr int kRows = 128;             // query rows of a tile (MMA M)
+  static constexpr int kTokens = kRows / G;     // new tokens of a tile
+  static constexpr int kKv = 128;               // context positions of a kv tile
+  static constexpr int kSpans = D / 64;
+  static constexpr int kGroup = kSpans * 1024;  // bytes between 8-row groups of Q, K, V tiles
+  static constexpr int kQBytes = kRows * D * 2;
+  static constexpr int kKvBytes = kKv * D * 2;
+  static constexpr int kPBytes = kRows * kKv * 2;  // 8-row groups of 2048 bytes
+  static constexpr int kBoxBytes = 8 * D * 2;      // one 8-position TMA box, both spans
+  static constexpr int kQOff = 0;
+  static constexpr int kKOff = kQOff + kQBytes;
+  static constexpr int kVOff = kKOff + 2 * kKvBytes;
+  static constexpr int kPhOff = kVOff + 2 * kKvBytes;
+  static constexpr int kPlOff = kPhOff + kPBytes;
+  static constexpr int kBarOff = kPlOff + kPBytes;
+  static constexpr int kNumBars = 16;
+  static constexpr int kInfoOff = kBarOff + kNumBars * 8;  // [tmem base, abort, tile count, rounds]
+  static constexpr int kMaxMine = 64;                      // rounds of the sorted schedule
+  static constexpr int kMineOff = kInfoOff + 32;
+  static constexpr int kSmemBytes = kMineOff + kMaxMine * 8 + 1024;  // + 1 KB alignment
+  // the sorted schedule's scratch (histogram of costs, tile list) lives in the key ring before
+  // the first copy
+  static constexpr int kMaxBins = 2048;  // costs 0 .. 2047 (16-position steps)
+  static constexpr int kMaxList = 4096;  // (sequence, tile) pairs
+  static constexpr int kTmemCols = 512;  // S0 [0, 128), S1 [128, 256), O [256, 256 + D)
+  static_assert(D == 64 || D == 128, "head_dim 64 or 128");
+  static_assert(G == 1 || G == 2 || G == 4 || G == 8, "1, 2, 4 or 8 query heads per kv head");
+  static_assert(BS % 8 == 0, "block size a multiple of the 8-position box");
+  static_assert((kMaxBins + kMaxList) * 4 <= 2 * kKvBytes, "schedule scratch fits the key ring");
+  static_assert(kSmemBytes <= 232448, "shared memory of one CTA");
+};
+
+// Warp-cooperative: the sequence holding tile y of the step (tiles ordered by sequence, then
+// position) and the tile's index within it; s = -1 when y is past the last tile.
+template <int TOK>
+__device__ __forceinline__ void locate_tile_tc(const PrefillArgs &a, long long y, int &s_out,
+                                               int &tau_out) {
+  const int lane = threadIdx.x & 31;
+  long long running = 0;
+  for (int base = 0; base < a.num_seqs; base += 32) {
+    const int s = base + lane;
+    int cnt = 0;
+    if (s < a.num_seqs) {
+      const int q_len = __ldg(a.query_start + s + 1) - __ldg(a.query_start + s);
+      cnt = q_len > 0 ? (q_len + TOK - 1) / TOK : 0;
+    }
+    long long incl = cnt;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const long long v = __shfl_up_sync(FULL_MASK, incl, off);
+      if (lane >= off) incl += v;
+    }
+    const long long total = __shfl_sync(FULL_MASK, incl, 31);
+    if (running + total > y) {
+      const bool hit = running + incl - cnt <= y && y < running + incl;
+      const int src = __ffs(__ballot_sync(FULL_MASK, hit)) - 1;
+      s_out = base + src;
+      tau_out = (int)(y - running - __shfl_sync(FULL_MASK, incl - cnt, src));
+      return;
+    }
+    running += total;
+  }
+  s_out = -1;
+  tau_out = 0;
+}
+
+// The per-tile quantities every role derives the same way.
+struct TcTile {
+  int s, tau, kvh;
+  int q0, q_len, L;
+  int tok0, ntok, pos0, n_kv;
+  bool valid;
+};
+
+// Two 16-bit terms of a pair of weights: hi = round(p), lo = round(p - hi).
+template <bool kBf16>
+__device__ __forceinline__ void split2(float x, float y, uint32_t &hi, uint32_t &lo) {
+  if constexpr (kBf16) {
+    const __nv_bfloat162 h = __floats2bfloat162_rn(x, y);
+    const float2 hf = __bfloat1622float2(h);
+    const __nv_bfloat162 l = __floats2bfloat162_rn(x - hf.x, y - hf.y);
+    hi = *reinterpret_cast<const uint32_t *>(&h);
+    lo = *reinterpret_cast<const uint32_t *>(&l);
+  } else {
+    const __half2 h = __floats2half2_rn(x, y);
+    const float2 hf = __half22float2(h);
+    const __half2 l = __floats2half2_rn(x - hf.x, y - hf.y);
+    hi = *reinterpret_cast<const uint32_t *>(&h);
+    lo = *reinterpret_cast<const uint32_t *>(&l);
+  }
+}
+
+template <typename T, int D, int BS, int G>
+__global__ void __launch_bounds__(PrefillTcTraits<D, BS, G>::kThreads, 1)
+    paged_prefill_tc_kernel(const PrefillArgs a, const __grid_constant__ TmaMaps maps) {
+  using Tr = PrefillTcTraits<D, BS, G>;
+  constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  unsigned char *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + Tr::kBarOff);
+  uint64_t *k_full = bars + 0, *k_empty = bars + 2, *v_full = bars + 4, *v_empty = bars + 6;
+  uint64_t *s_full = bars + 8, *s_free = bars + 10;
+  uint64_t *p_ready = bars + 12, *o_done = bars + 13, *q_ready = bars + 14, *fin = bars + 15;
+  volatile int *info = reinterpret_cast<volatile int *>(smem + Tr::kInfoOff);
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + Tr::kInfoOff);
+  int2 *mine = reinterpret_cast<int2 *>(smem + Tr::kMineOff);
+
+  const int tid = threadIdx.x;
+  const int lane = tid & 31;
+  const int wid = tid >> 5;
+  const int Hkv = a.num_kv_heads;
+  const int max_len = a.max_blocks * BS;
+
+  if (tid == 0) {
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(k_full + i, 1);
+      mbar_init(k_empty + i, 1);
+      mbar_init(v_full + i, 1);
+      mbar_init(v_empty + i, 1);
+      mbar_init(s_full + i, 1);
+      mbar_init(s_free + i, 128);
+    }
+    mbar_init(p_ready, 128);
+    mbar_init(o_done, 1);
+    mbar_init(q_ready, 128);
+    mbar_init(fin, 1);
+    fence_barrier_init();
+    info[1] = 0;
+    info[2] = 0;
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&maps.k)) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&maps.v)) : "memory");
+  }
+  if (wid == 5) {
+    tc::alloc(tmem_slot, Tr::kTmemCols);
+    tc::relinquish();
+  }
+
+  // ---- the longest-first schedule (scratch in the key ring) ----
+  int *bins = reinterpret_cast<int *>(smem + Tr::kKOff);
+  int *list = bins + Tr::kMaxBins;
+  const int nbins = (max_len + 15) / 16 + 1;
+  bool sorted = nbins <= Tr::kMaxBins && a.num_seqs < (1 << 19);
+  if (sorted)
+    for (int i = tid; i < nbins; i += Tr::kThreads) bins[i] = 0;
+  __syncthreads();
+  auto seq_tiles = [&](int sq, int &len_out, int &q_out) {
+    const int q0s = __ldg(a.query_start + sq);
+    const int qn = __ldg(a.query_start + sq + 1) - q0s;
+    const int raw = __ldg(a.context_lens + sq);
+    const int Ls = raw < 0 ? 0 : (raw > max_len ? max_len : raw);
+    len_out = Ls;
+    q_out = qn;
+    if (qn > Ls || q0s < 0 || (long long)q0s + qn > a.num_tokens) return -1;  // invalid
+    return qn > 0 ? (qn + Tr::kTokens - 1) / Tr::kTokens : 0;
+  };
+  auto tile_cost = [&](int Ls, int qn, int t) {
+    const int last = min((t + 1) * Tr::kTokens, qn);  // tokens up to this tile's last one
+    return (Ls - qn + last + 15) / 16;
+  };
+  if (sorted) {
+    for (int sq = tid; sq < a.num_seqs; sq += Tr::kThreads) {
+      int Ls, qn;
+      const int nt = seq_tiles(sq, Ls, qn);
+      if (nt < 0) {
+        // new tokens outside the context, or query rows outside the query tensor: report
+        set_error(a.err, PA_DEVERR_CONTEXT_LEN);
+        continue;
+      }
+      for (int t = 0; t < nt && t < Tr::kMaxList; ++t) atomicAdd(bins + tile_cost(Ls, qn, t), 1);
+      atomicAdd((int *)info + 2, nt);
+    }
+  }
+  __syncthreads();
+  const int ntiles = sorted ? info[2] : 0;
+  const long long total = (long long)ntiles * Hkv;
+  sorted = sorted && ntiles <= Tr::kMaxList && total <= (long long)Tr::kMaxMine * gridDim.x;
+  if (sorted && wid == 0) {
+    // bins[c] <- number of tiles costing more than c: where the tiles of cost c start
+    const int seg = (nbins + 31) / 32;
+    const int hi = nbins - 1 - lane * seg;  // this lane's costs: hi, hi-1, .., hi-seg+1
+    int sum = 0;
+    for (int i = 0; i < seg; ++i)
+      if (hi - i >= 0) sum += bins[hi - i];
+    int incl = sum;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int v = __shfl_up_sync(FULL_MASK, incl, off);
+      if (lane >= off) incl += v;
+    }
+    int run = incl - sum;
+    for (int i = 0; i < seg; ++i)
+      if (hi - i >= 0) {
+        const int n = bins[hi - i];
+        bins[hi - i] = run;
+        run += n;
+      }
+  }
+  __syncthreads();
+  if (sorted) {
+    for (int sq = tid; sq < a.num_seqs; sq += Tr::kThreads) {
+      int Ls, qn;
+      const int nt = seq_tiles(sq, Ls, qn);
+      for (int t = 0; t < nt; ++t) list[atomicAdd(bins + tile_cost(Ls, qn, t), 1)] = (sq << 12) | t;
+    }
+  }
+  __syncthreads();
+  if (sorted && tid < Tr::kMaxMine) {
+    const long long r = tid;
+    const long long k = r * gridDim.x + ((r & 1) ? (long long)gridDim.x - 1 - blockIdx.x : (long long)blockIdx.x);
+    if (k < total) mine[r] = make_int2(list[k / Hkv], (int)(k % Hkv));
+  }
+  if (tid == 0) {
+    // every round but the last is full; in the last one this CTA's position depends on the
+    // direction of the snake
+    long long rounds = 0;
+    if (sorted) {
+      const long long full = total / gridDim.x, rem = total % gridDim.x;
+      const long long at = (full & 1) ? (long long)gridDim.x - 1 - blockIdx.x : (long long)blockIdx.x;
+      rounds = full + (at < rem ? 1 : 0);
+    }
+    info[3] = (int)rounds;
+  }
+  // the scratch is overwritten by copies from here on
+  fence_proxy_async_smem();
+  tc::fence_before();
+  __syncthreads();
+  tc::fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const int my_rounds = info[3];
+
+  // The tile of round `round` (whole warp calls it); false when this CTA has no more tiles.
+  auto next_tile = [&](long long round, TcTile &t) -> bool {
+    if (sorted) {
+      if (round >= my_rounds) return false;
+      const int2 e = mine[round];
+      t.s = e.x >> 12;
+      t.tau = e.x & 4095;
+      t.kvh = e.y;
+    } else {
+      const long long x = blockIdx.x + round * gridDim.x;
+      int ls, lt;
+      locate_tile_tc<Tr::kTokens>(a, x / Hkv, ls, lt);
+      if (ls < 0) return false;
+      t.s = ls;
+      t.tau = lt;
+      t.kvh = (int)(x % Hkv);
+    }
+    t.q0 = __ldg(a.query_start + t.s);
+    t.q_len = __ldg(a.query_start + t.s + 1) - t.q0;
+    const int raw = __ldg(a.context_lens + t.s);
+    t.L = raw < 0 ? 0 : (raw > max_len ? max_len : raw);
+    t.valid = !(t.q_len > t.L || t.q0 < 0 || (long long)t.q0 + t.q_len > a.num_tokens);
+    t.tok0 = t.tau * Tr::kTokens;
+    t.ntok = min(Tr::kTokens, t.q_len - t.tok0);
+    t.pos0 = t.L - t.q_len + t.tok0;
+    t.n_kv = t.valid ? (t.pos0 + t.ntok + Tr::kKv - 1) / Tr::kKv : 0;
+    return true;
+  };
+  // A bounded wait that also gives up once another role has aborted.
+  auto wait = [&](uint64_t *bar, uint32_t parity) -> bool {
+    if (mbar_try_wait(bar, parity)) return true;
+    const long long t0 = clock64();
+    for (;;) {
+      if (mbar_try_wait(bar, parity)) return true;
+      if (info[1] != 0) return false;
+      if (clock64() - t0 > a.wait_cycles) {
+        set_error(a.err, PA_DEVERR_TIMEOUT);
+        info[1] = 1;
+        return false;
+      }
+    }
+  };
+
+  const uint32_t q_s = smem_u32(smem + Tr::kQOff);
+  const uint32_t k_s = smem_u32(smem + Tr::kKOff);
+  const uint32_t v_s = smem_u32(smem + Tr::kVOff);
+  const uint32_t ph_s = smem_u32(smem + Tr::kPhOff);
+  const uint32_t pl_s = smem_u32(smem + Tr::kPlOff);
+
+  if (wid == 4) {
+    // ================= producer: key and value tiles by TMA =================
+    long long kv_base = 0;
+    long long k_issued = 0, v_issued = 0;
+    bool ok = true;
+    TcTile t;
+    for (long long round = 0; ok && next_tile(round, t); ++round) {
+      if (!t.valid) {
+        if (lane == 0 && t.tau == 0 && t.kvh == 0) set_error(a.err, PA_DEVERR_CONTEXT_LEN);
+        continue;
+      }
+      if (lane == 0) {
+        const int32_t *row = a.block_tables + (long long)t.s * a.bt_s;
+        for (int j = 0; j < t.n_kv && ok; ++j) {
+          const long long it = kv_base + j;
+          const int b = (int)(it & 1);
+          const long long use = it >> 1;
+          const int p0 = j * Tr::kKv;
+          const int pend = min(p0 + Tr::kKv, t.L);
+          const uint32_t bytes = (uint32_t)((pend - p0 + 7) / 8) * Tr::kBoxBytes;
+          for (int which = 0; which < 2 && ok; ++which) {
+            uint64_t *full = which ? v_full + b : k_full + b;
+            uint64_t *empty = which ? v_empty + b : k_empty + b;
+            if (use >= 1 && !wait(empty, (uint32_t)((use - 1) & 1))) {
+              ok = false;
+              break;
+            }
+            mbar_arrive_expect_tx(full, bytes);
+            const uint32_t dst = (which ? v_s : k_s) + b * Tr::kKvBytes;
+            const CUtensorMap *map = which ? &maps.v : &maps.k;
+            for (int p = p0; p < pend; p += BS) {
+              int blk = __ldg(row + p / BS);
+              if (blk < 0 || (long long)blk >= a.num_blocks) {
+                set_error(a.err, PA_DEVERR_BLOCK_ID);
+                blk = 0;
+              }
+              for (int y = 0; y < BS && p + y < pend; y += 8)
+                tma_load_tile(dst + ((p + y - p0) / 8) * Tr::kBoxBytes, map, y, t.kvh, blk, full);
+            }
+            if (which) ++v_issued; else ++k_issued;
+          }
+        }
+      }
+      ok = __shfl_sync(FULL_MASK, ok ? 1 : 0, 0) != 0;
+      kv_base += t.n_kv;
+    }
+    if (lane == 0 && !ok) {
+      // let the copies in flight land before the CTA leaves
+      for (long long i = k_issued > 2 ? k_issued - 2 : 0; i < k_issued; ++i)
+        mbar_wait_bounded(k_full + (i & 1), (uint32_t)((i >> 1) & 1), a.wait_cycles);
+      for (long long i = v_issued > 2 ? v_issued - 2 : 0; i < v_issued; ++i)
+        mbar_wait_bounded(v_full + (i & 1), (uint32_t)((i >> 1) & 1), a.wait_cycles);
+    }
+  } else if (wid == 5) {
+    // ================= MMA issue =================
+    constexpr uint32_t kIdS = tc::idesc_f16(kBf16, 128, Tr::kKv, false);
+    constexpr uint32_t kIdO = tc::idesc_f16(kBf16, 128, D, true);
+    long long kv_base = 0;
+    long long qt = 0;
+    bool ok = true;
+    TcTile t;
+    auto pv = [&](int j) -> bool {
+      const long long it = kv_base + j;
+      const int b = (int)(it & 1);
+      if (!wait(p_ready, (uint32_t)(it & 1)) || !wait(v_full + b, (uint32_t)((it >> 1) & 1))) return false;
+      tc::fence_after();
+      const uint32_t vb = v_s + b * Tr::kKvBytes;
+#pragma unroll
+      for (int kt = 0; kt < Tr::kKv / 16; ++kt) {
+        const uint64_t vd = tc::smem_desc(vb + kt * 2 * Tr::kGroup, 1024, Tr::kGroup);
+        const uint32_t poff = (kt >> 2) * 1024 + (kt & 3) * 32;
+        tc::mma(tmem + 256, tc::smem_desc(ph_s + poff, 16, 2048), vd, kIdO, (j > 0 || kt > 0) ? 1u : 0u);
+        tc::mma(tmem + 256, tc::smem_desc(pl_s + poff, 16, 2048), vd, kIdO, 1u);
+      }
+      tc::commit(o_done);
+      tc::commit(v_empty + b);
+      return true;
+    };
+    for (long long round = 0; ok && next_tile(round, t); ++round) {
+      if (!t.valid) continue;
+      if (lane == 0) {
+        ok = wait(q_ready, (uint32_t)(qt & 1));
+        tc::fence_after();
+        for (int j = 0; j < t.n_kv && ok; ++j) {
+          const long long it = kv_base + j;
+          const int b = (int)(it & 1);
+          const long long use = it >> 1;
+          if (!wait(k_full + b, (uint32_t)(use & 1)) ||
+              (use >= 1 && !wait(s_free + b, (uint32_t)((use - 1) & 1)))) {
+            ok = false;
+            break;
+          }
+          tc::fence_after();
+          const uint32_t kb = k_s + b * Tr::kKvBytes;
+#pragma unroll
+          for (int ks = 0; ks < D / 16; ++ks) {
+            const uint32_t off = (ks >> 2) * 1024 + (ks & 3) * 32;
+            tc::mma(tmem + 128 * b, tc::smem_desc(q_s + off, 16, Tr::kGroup),
+                    tc::smem_desc(kb + off, 16, Tr::kGroup), kIdS, ks > 0 ? 1u : 0u);
+          }
+          tc::commit(s_full + b);
+          tc::commit(k_empty + b);
+          if (j > 0) ok = pv(j - 1);
+        }
+        if (ok) ok = pv(t.n_kv - 1);
+      }
+      ok = __shfl_sync(FULL_MASK, ok ? 1 : 0, 0) != 0;
+      kv_base += t.n_kv;
+      ++qt;
+    }
+    if (lane == 0) {
+      // every MMA issued has completed before tensor memory is released
+      tc::commit(fin);
+      mbar_wait_bounded(fin, 0, a.wait_cycles);
+    }
+    __syncwarp();
+  } else {
+    // ================= softmax, one thread per row =================
+    const int r = tid;  // row = tensor-memory lane
+    const int lt = r / G, hh = r % G;
+    const uint32_t lane_base = tc::taddr(tmem, 32 * wid, 0);
+    const uint32_t q_row = q_s + (r >> 3) * Tr::kGroup + (r & 7) * 128;
+    const uint32_t p_row = (r >> 3) * 2048 + (r & 7) * 128;
+    long long kv_base = 0;
+    bool ok = true;
+    TcTile t;
+    for (long long round = 0; ok && next_tile(round, t); ++round) {
+      if (!t.valid) continue;
+      const bool row_ok = lt < t.ntok;
+      const int prow = row_ok ? t.pos0 + lt : -1;
+      // ---- the tile's query rows into shared memory (swizzled, zero rows past the tile) ----
+      {
+        const uint4 *src = reinterpret_cast<const uint4 *>(
+            static_cast<const T *>(a.query) + (long long)(t.q0 + t.tok0 + (row_ok ? lt : 0)) * a.q_t +
+            (long long)(t.kvh * G + hh) * a.q_h);
+#pragma unroll
+        for (int c = 0; c < D / 8; ++c) {
+          const uint4 v = row_ok ? __ldg(src + c) : make_uint4(0u, 0u, 0u, 0u);
+          const uint32_t dst = q_row + (c >> 3) * 1024 + (((c & 7) ^ (r & 7)) << 4);
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(v.x), "r"(v.y),
+                       "r"(v.z), "r"(v.w)
+                       : "memory");
+        }
+        fence_proxy_async_smem();
+        mbar_arrive(q_ready);
+      }
+      float m_ref = -INFINITY, l_sum = 0.f;
+      for (int j = 0; j < t.n_kv; ++j) {
+        const long long it = kv_base + j;
+        const int b = (int)(it & 1);
+        if (!__all_sync(FULL_MASK, wait(s_full + b, (uint32_t)((it >> 1) & 1)))) {
+          ok = false;
+          break;
+        }
+        tc::fence_after();
+        // ---- mask, maximum in base 2 (S read 32 columns at a time) ----
+        const int c_lim = prow - j * Tr::kKv;  // columns 0 .. c_lim are visible to this row
+        const uint32_t s_addr = lane_base + 128 * b;
+        float hi_raw = -INFINITY, lo_raw = INFINITY;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          uint32_t sr[32];
+          tc::ld32x32(s_addr + 32 * q, sr);
+#pragma unroll
+          for (int c = 0; c < 32; ++c) {
+            const float v = 32 * q + c <= c_lim ? __uint_as_float(sr[c]) : NAN;
+            hi_raw = fmaxf(hi_raw, v);  // fmaxf / fminf skip the NaN of masked columns
+            lo_raw = fminf(lo_raw, v);
+          }
+        }
+        // the largest scaled logit (the scale may be negative); -inf when nothing is visible
+        const float mx = c_lim < 0 ? -INFINITY : (a.scale_log2 >= 0.f ? hi_raw : lo_raw) * a.scale_log2;
+        float alpha = 1.f;
+        bool rescale = false;
+        if (mx > m_ref + 8.f) {
+          alpha = m_ref == -INFINITY ? 0.f : fast_exp2(m_ref - mx);
+          rescale = j > 0;
+          m_ref = mx;
+          l_sum *= alpha;
+        }
+        // ---- weights and their two 16-bit terms (S read again; every lane of the warp takes
+        // part in the tensor-memory loads, rows with nothing visible get zero weights) ----
+        uint32_t hp[64], lp[64];
+        const float nm = m_ref == -INFINITY ? 0.f : -m_ref;
+        __syncwarp();
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          uint32_t sr[32];
+          tc::ld32x32(s_addr + 32 * q, sr);
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const int c0 = 32 * q + 2 * i;
+            float p0 = fast_exp2(fmaf(__uint_as_float(sr[2 * i]), a.scale_log2, nm));
+            float p1 = fast_exp2(fmaf(__uint_as_float(sr[2 * i + 1]), a.scale_log2, nm));
+            p0 = c0 <= c_lim ? p0 : 0.f;
+            p1 = c0 + 1 <= c_lim ? p1 : 0.f;
+            l_sum += p0 + p1;
+            split2<kBf16>(p0, p1, hp[16 * q + i], lp[16 * q + i]);
+          }
+        }
+        tc::fence_before();
+        mbar_arrive(s_free + b);
+        // ---- O += P V of the previous kv tile must be done before P and O are touched ----
+        if (j > 0 && !__all_sync(FULL_MASK, wait(o_done, (uint32_t)((it - 1) & 1)))) {
+          ok = false;
+          break;
+        }
+        if (__any_sync(FULL_MASK, rescale)) {
+          tc::fence_after();
+          const float f = rescale ? alpha : 1.f;
+#pragma unroll
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t o[32];
+            tc::ld32x32(lane_base + 256 + 32 * c, o);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * f);
+            tc::st32x32(lane_base + 256 + 32 * c, o);
+          }
+        }
+        if (j == t.n_kv - 1 && (j + 1) * Tr::kKv > t.L) {
+          // positions past the context may hold anything (NaN included) and would meet a zero
+          // weight in the MMA: zero the value rows there once their copy has landed
+          if (!__all_sync(FULL_MASK, wait(v_full + b, (uint32_t)((it >> 1) & 1)))) {
+            ok = false;
+            break;
+          }
+          if (r >= t.L - j * Tr::kKv) {
+            const uint32_t vrow = v_s + b * Tr::kKvBytes + (r >> 3) * Tr::kGroup + (r & 7) * 128;
+#pragma unroll
+            for (int h = 0; h < Tr::kSpans; ++h)
+#pragma unroll
+              for (int c = 0; c < 8; ++c)
+                asm volatile("st.shared.v4.b32 [%0], {%1, %1, %1, %1};" ::"r"(vrow + h * 1024 + c * 16),
+                             "r"(0u)
+                             : "memory");
+          }
+        }
+        // ---- P (hi, lo) into shared memory, swizzled like the operand tiles ----
+#pragma unroll
+        for (int c = 0; c < 16; ++c) {
+          const uint32_t off = p_row + (c >> 3) * 1024 + (((c & 7) ^ (r & 7)) << 4);
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(ph_s + off), "r"(hp[4 * c]),
+                       "r"(hp[4 * c + 1]), "r"(hp[4 * c + 2]), "r"(hp[4 * c + 3])
+                       : "memory");
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(pl_s + off), "r"(lp[4 * c]),
+                       "r"(lp[4 * c + 1]), "r"(lp[4 * c + 2]), "r"(lp[4 * c + 3])
+                       : "memory");
+        }
+        fence_proxy_async_smem();
+        tc::fence_before();
+        mbar_arrive(p_ready);
+      }
+      if (!ok) break;
+      // ---- epilogue: O / l of the valid rows ----
+      const long long last = kv_base + t.n_kv - 1;
+      if (!__all_sync(FULL_MASK, wait(o_done, (uint32_t)(last & 1)))) {
+        ok = false;
+        break;
+      }
+      tc::fence_after();
+      const float inv = row_ok ? 1.f / l_sum : 0.f;
+      const long long ob = (long long)(t.q0 + t.tok0 + (row_ok ? lt : 0)) * a.out_t +
+                           (long long)(t.kvh * G + hh) * a.out_h;
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t o[32];
+        __syncwarp();
+        tc::ld32x32(lane_base + 256 + 32 * c, o);
+        if (!row_ok) {
+        } else if (a.out_dtype == PA_F32) {
+          float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(a.out) + ob + 32 * c);
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            dst[i] = make_float4(__uint_as_float(o[4 * i]) * inv, __uint_as_float(o[4 * i + 1]) * inv,
+                                 __uint_as_float(o[4 * i + 2]) * inv, __uint_as_float(o[4 * i + 3]) * inv);
+        } else {
+          uint4 *dst = reinterpret_cast<uint4 *>(static_cast<T *>(a.out) + ob + 32 * c);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            uint32_t w[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float x0 = __uint_as_float(o[8 * i + 2 * e]) * inv;
+              const float x1 = __uint_as_float(o[8 * i + 2 * e + 1]) * inv;
+              if constexpr (kBf16) {
+                const __nv_bfloat162 h = __floats2bfloat162_rn(x0, x1);
+                w[e] = *reinterpret_cast<const uint32_t *>(&h);
+              } else {
+                const __half2 h = __floats2half2_rn(x0, x1);
+                w[e] = *reinterpret_cast<const uint32_t *>(&h);
+              }
+            }
+            dst[i] = make_uint4(w[0], w[1], w[2], w[3]);
+          }
+        }
+      }
+      kv_base += t.n_kv;
+    }
+  }
+
+  // ---- teardown: every role done, tensor memory released by the warp that allocated it ----
+  tc::fence_before();
+  __syncthreads();
+  if (wid == 5) {
+    tc::fence_after();
+    tc::dealloc(tmem, Tr::kTmemCols);
+  }
+}
+
+template <typename T, int D, int BS, int G>
+cudaError_t launch_prefill_tc(const PrefillArgs &a, const TmaMaps *maps, int num_ctas, cudaStream_t st) {
+  using Tr = PrefillTcTraits<D, BS, G>;
+  paged_prefill_tc_kernel<T, D, BS, G><<<num_ctas, Tr::kThreads, Tr::kSmemBytes, st>>>(a, *maps);
+  return cudaGetLastError();
+}
+
+template <typename T, int D, int BS, int G>
+bool make_prefill_tc(PrefillKernel *k) {
+  using Tr = PrefillTcTraits<D, BS, G>;
+  static bool configured[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
+  if (!configured[dev]) {
+    if (cudaFuncSetAttribute(paged_prefill_tc_kernel<T, D, BS, G>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             Tr::kSmemBytes) != cudaSuccess)
+      return false;
+    configured[dev] = true;
+  }
+  k->launch = &launch_prefill_tc<T, D, BS, G>;
+  k->kernel = reinterpret_cast<const void *>(&paged_prefill_tc_kernel<T, D, BS, G>);
+  k->threads_per_cta = Tr::kThreads;
+  k->smem_bytes = Tr::kSmemBytes;
+  k->tokens_per_tile = Tr::kTokens;
+  k->tma_rows = 8;
+  return true;
+}
+
+// Tables over head_dim {64, 128} x block_size {8, 16, 32} x group {1, 2, 4, 8}.
+template <typename T>
+bool prefill_tc_table(int head_dim, int block_size, int group, PrefillKernel *k) {
+#define PA_CASE(DD, BB, GG) \
+  if (head_dim == DD && block_size == BB && group == GG) return make_prefill_tc<T, DD, BB, GG>(k);
+#define PA_GROUPS(DD, BB) PA_CASE(DD, BB, 1) PA_CASE(DD, BB, 2) PA_CASE(DD, BB, 4) PA_CASE(DD, BB, 8)
+  PA_GROUPS(64, 8)
+  PA_GROUPS(64, 16)
+  PA_GROUPS(64, 32)
+  PA_GROUPS(128, 8)
+  PA_GROUPS(128, 16)
+  PA_GROUPS(128, 32)
+#undef PA_GROUPS
+#undef PA_CASE
+  return false;
+}
+
+}  // namespace pa
