@@ -292,6 +292,15 @@ uint64_t g_map_clock = 0;
 // The cache as a 5-D tensor (64 elements, block_size rows, head_dim / 64 column halves, kv heads,
 // blocks) read in 128-byte swizzled boxes of 64 x `rows` x head_dim/64: one box brings a whole
 // (rows x head_dim) tile, laid out in shared memory as [half][row][128 bytes].
+// rows == 0 asks for the grouped view instead (caches whose blocks are kv heads x rows x
+// head_dim contiguous, see grouped_view_ok): 64 elements, 8 rows, head_dim / 64 halves,
+// block_size / 8 row groups, blocks x kv heads; one box brings a whole (block, kv head) tile laid
+// out as [group of 8 rows][half][row][128 bytes], the operand layout of the tensor-core MMAs.
+bool grouped_view_ok(const pa_tensor *t) {
+  return t->stride[3] == 1 && t->stride[2] == t->shape[3] && t->stride[0] == t->shape[1] * t->stride[1] &&
+         t->shape[2] % 8 == 0;
+}
+
 int cache_map(const pa_tensor *t, int rows, CUtensorMap *out) {
   MapKey key;
   key.ptr = t->data;
@@ -312,11 +321,23 @@ int cache_map(const pa_tensor *t, int rows, CUtensorMap *out) {
   const cuuint64_t e = (cuuint64_t)elt_size(t->dtype);
   const cuuint64_t per128 = 128 / e;  // elements in one 128-byte swizzle span
   const cuuint64_t spans = (cuuint64_t)t->shape[3] / per128;
-  const cuuint64_t dims[5] = {per128, (cuuint64_t)t->shape[2], spans, (cuuint64_t)t->shape[1],
-                              (cuuint64_t)t->shape[0]};
-  const cuuint64_t strides[4] = {(cuuint64_t)t->stride[2] * e, 128, (cuuint64_t)t->stride[1] * e,
-                                 (cuuint64_t)t->stride[0] * e};
-  const cuuint32_t box[5] = {(cuuint32_t)per128, (cuuint32_t)rows, (cuuint32_t)spans, 1, 1};
+  cuuint64_t dims[5] = {per128, (cuuint64_t)t->shape[2], spans, (cuuint64_t)t->shape[1],
+                        (cuuint64_t)t->shape[0]};
+  cuuint64_t strides[4] = {(cuuint64_t)t->stride[2] * e, 128, (cuuint64_t)t->stride[1] * e,
+                           (cuuint64_t)t->stride[0] * e};
+  cuuint32_t box[5] = {(cuuint32_t)per128, (cuuint32_t)rows, (cuuint32_t)spans, 1, 1};
+  if (rows == 0) {
+    const cuuint64_t row_bytes = (cuuint64_t)t->shape[3] * e;
+    const cuuint64_t g[5] = {per128, 8, spans, (cuuint64_t)t->shape[2] / 8,
+                             (cuuint64_t)(t->shape[0] * t->shape[1])};
+    const cuuint64_t st[4] = {row_bytes, 128, 8 * row_bytes, (cuuint64_t)t->stride[1] * e};
+    const cuuint32_t bx[5] = {(cuuint32_t)per128, 8, (cuuint32_t)spans, (cuuint32_t)(t->shape[2] / 8), 1};
+    for (int i = 0; i < 5; ++i) {
+      dims[i] = g[i];
+      box[i] = bx[i];
+    }
+    for (int i = 0; i < 4; ++i) strides[i] = st[i];
+  }
   const cuuint32_t estr[5] = {1, 1, 1, 1, 1};
   CUtensorMap map;
   const CUtensorMapDataType type = t->dtype == PA_FP8_E4M3 ? CU_TENSOR_MAP_DATA_TYPE_UINT8
@@ -336,6 +357,27 @@ int cache_map(const pa_tensor *t, int rows, CUtensorMap *out) {
   }
   g_maps.push_back(MapEntry{key, map, ++g_map_clock});
   *out = map;
+  return PA_OK;
+}
+
+// The prefill's query rows [tokens, heads, head_dim] as a 4-D tensor (64 elements, heads,
+// tokens, head_dim / 64 halves) read in 128-byte swizzled boxes of 64 x G heads x 128/G tokens x
+// halves: one box brings a tile's 128 rows (token-major, head fastest) laid out span-major,
+// [half][row][128 bytes].  Tokens past the tensor read as zeros.
+int query_map(const pa_tensor *q, int G, CUtensorMap *out) {
+  if (!g_encode_tiled) return fail(PA_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
+  const cuuint64_t e = 2;
+  const cuuint64_t spans = (cuuint64_t)q->shape[2] / 64;
+  const cuuint64_t dims[4] = {64, (cuuint64_t)q->shape[1], (cuuint64_t)q->shape[0], spans};
+  const cuuint64_t strides[3] = {(cuuint64_t)q->stride[1] * e, (cuuint64_t)q->stride[0] * e, 128};
+  const cuuint32_t box[4] = {64, (cuuint32_t)G, (cuuint32_t)(128 / G), (cuuint32_t)spans};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  const CUtensorMapDataType type = q->dtype == PA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                                       : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+  const CUresult r = g_encode_tiled(out, type, 4, q->data, dims, strides, box, estr,
+                                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(PA_ERR_LAYOUT, "cuTensorMapEncodeTiled failed for the query (%d)", (int)r);
   return PA_OK;
 }
 
@@ -868,8 +910,12 @@ int pa_prefill(const pa_tensor *out, const pa_tensor *query, const pa_tensor *ke
                                        : pa::prefill_kernel_f16(D, block_size, G, &k);
   if (!got)
     return fail(PA_ERR_CUDA, "could not prepare the prefill kernel: %s", cudaGetErrorString(cudaGetLastError()));
-  pa::TmaMaps maps;
-  if ((rc = cache_map(key_cache, k.tma_rows, &maps.k)) || (rc = cache_map(value_cache, k.tma_rows, &maps.v)))
+  pa::PrefillMaps maps;
+  // one box per (block, kv head) tile when the caches allow the grouped view, else 8-row boxes
+  const bool grouped = grouped_view_ok(key_cache) && grouped_view_ok(value_cache);
+  const int rows = grouped ? 0 : k.tma_rows;
+  if ((rc = cache_map(key_cache, rows, &maps.k)) || (rc = cache_map(value_cache, rows, &maps.v)) ||
+      (rc = query_map(query, G, &maps.q)))
     return rc;
   // enough CTAs for every tile of any split of T tokens among S sequences, at most one wave
   const int64_t tiles = ((T + k.tokens_per_tile - 1) / k.tokens_per_tile + S) * num_kv_heads;
@@ -899,6 +945,7 @@ int pa_prefill(const pa_tensor *out, const pa_tensor *query, const pa_tensor *ke
   a.scale_log2 = (float)((double)scale * 1.4426950408889634);
   a.err = ds->err;
   a.wait_cycles = test_hooks().wait_cycles;
+  a.grouped_maps = grouped ? 1 : 0;
   cudaError_t e = k.launch(a, &maps, ctas, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? PA_OK : cuda_fail(e, "prefill launch");
 }

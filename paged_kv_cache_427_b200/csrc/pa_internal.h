@@ -145,10 +145,18 @@ struct PrefillArgs {
   float scale_log2;
   unsigned int *err;
   long long wait_cycles;
+  int grouped_maps;  // 1: the maps are the grouped view (one box per block and kv head)
+};
+
+// The prefill's tensor maps: the caches (grouped view, or 8-row boxes) and the query rows.
+struct PrefillMaps {
+  CUtensorMap k;
+  CUtensorMap v;
+  CUtensorMap q;
 };
 
 struct PrefillKernel {
-  cudaError_t (*launch)(const PrefillArgs &, const TmaMaps *, int num_ctas, cudaStream_t);
+  cudaError_t (*launch)(const PrefillArgs &, const PrefillMaps *, int num_ctas, cudaStream_t);
   const void *kernel;
   int threads_per_cta;
   int smem_bytes;

@@ -12,18 +12,21 @@
 // A tile is 128 query rows of one (sequence, kv head): 128 / G new tokens times the G query
 // heads that read that kv head (head fastest), one row per tensor-memory lane.  The context is
 // walked in kv tiles of 128 positions.  One persistent CTA per SM, six warps:
-//   * warp 4 (one lane) streams the key and value tiles of 128 positions through two-slot rings
-//     by TMA: 8-position boxes of the paged cache (both 64-element spans of the head, 128-byte
-//     swizzle) placed one after another, which is the operand layout of the MMAs;
+//   * warp 4 streams the tile's query rows (one 4-D box, loaded as soon as the previous tile's
+//     last S = QK^T is done, so it overlaps that tile's end) and the key and value tiles of 128
+//     positions through two-slot rings by TMA: one box per (block, kv head) tile of the paged
+//     cache, 128-byte swizzle, in 8-row groups placed one after another, which is the operand
+//     layout of the MMAs; the lanes issue the boxes of a kv tile together;
 //   * warp 5 (one lane) issues the MMAs: S = Q K^T (M = 128 rows, N = 128 positions, K = head
 //     dim) into one of two S buffers in tensor memory, and O += P V (N = head dim, K = 128
 //     positions) into the O accumulator, P split into two 16-bit terms (hi + lo) as in the
 //     decode kernels so the weights keep about 16 significant bits;
-//   * warps 0-3 (one thread per row) copy the tile's query rows into shared memory, read S from
-//     tensor memory, apply the causal mask (which also hides positions past the context), keep
-//     the online softmax per row in base 2 with a lazy reference maximum (moved only when a
-//     logit passes it by 2^8, when O is rescaled in tensor memory), write P to shared memory and
-//     finally read O, divide by the row sums and store the rows.
+//   * warps 0-3 (one thread per row) read S from tensor memory, apply the causal mask (which
+//     also hides positions past the context), keep the online softmax per row in base 2 with a
+//     lazy reference maximum (moved only when a logit passes it by 2^8, when O is rescaled in
+//     tensor memory), write P to shared memory and finally read O, divide by the row sums and
+//     store the rows.  (P read by the MMA from tensor memory instead measured slower: the
+//     softmax warps' tensor-memory loads then wait behind the MMA's operand reads.)
 // The MMA warp issues S of kv tile j + 1 before O += P V of tile j, so the tensor cores compute
 // the next scores while the softmax warps work on the current ones.  Barriers between the roles
 // are mbarriers (copies: transaction bytes; MMAs: tcgen05.commit; threads: arrival counts);
@@ -55,13 +58,13 @@ struct PrefillTcTraits {
   static constexpr int kKvBytes = kKv * D * 2;
   static constexpr int kPBytes = kRows * kKv * 2;  // 8-row groups of 2048 bytes
   static constexpr int kBoxBytes = 8 * D * 2;      // one 8-position TMA box, both spans
-  static constexpr int kQOff = 0;
+  static constexpr int kQOff = 0;                  // query rows, span-major
   static constexpr int kKOff = kQOff + kQBytes;
   static constexpr int kVOff = kKOff + 2 * kKvBytes;
   static constexpr int kPhOff = kVOff + 2 * kKvBytes;
   static constexpr int kPlOff = kPhOff + kPBytes;
   static constexpr int kBarOff = kPlOff + kPBytes;
-  static constexpr int kNumBars = 16;
+  static constexpr int kNumBars = 20;
   static constexpr int kInfoOff = kBarOff + kNumBars * 8;  // [tmem base, abort, tile count, rounds]
   static constexpr int kMaxMine = 64;                      // rounds of the sorted schedule
   static constexpr int kMineOff = kInfoOff + 32;
@@ -140,7 +143,7 @@ __device__ __forceinline__ void split2(float x, float y, uint32_t &hi, uint32_t 
 
 template <typename T, int D, int BS, int G>
 __global__ void __launch_bounds__(PrefillTcTraits<D, BS, G>::kThreads, 1)
-    paged_prefill_tc_kernel(const PrefillArgs a, const __grid_constant__ TmaMaps maps) {
+    paged_prefill_tc_kernel(const PrefillArgs a, const __grid_constant__ PrefillMaps maps) {
   using Tr = PrefillTcTraits<D, BS, G>;
   constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -148,7 +151,8 @@ __global__ void __launch_bounds__(PrefillTcTraits<D, BS, G>::kThreads, 1)
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + Tr::kBarOff);
   uint64_t *k_full = bars + 0, *k_empty = bars + 2, *v_full = bars + 4, *v_empty = bars + 6;
   uint64_t *s_full = bars + 8, *s_free = bars + 10;
-  uint64_t *p_ready = bars + 12, *o_done = bars + 13, *q_ready = bars + 14, *fin = bars + 15;
+  uint64_t *q_full = bars + 12, *q_empty = bars + 13;
+  uint64_t *p_ready = bars + 16, *o_done = bars + 17, *fin = bars + 18;
   volatile int *info = reinterpret_cast<volatile int *>(smem + Tr::kInfoOff);
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + Tr::kInfoOff);
   int2 *mine = reinterpret_cast<int2 *>(smem + Tr::kMineOff);
@@ -168,15 +172,17 @@ __global__ void __launch_bounds__(PrefillTcTraits<D, BS, G>::kThreads, 1)
       mbar_init(s_full + i, 1);
       mbar_init(s_free + i, 128);
     }
+    mbar_init(q_full, 1);
+    mbar_init(q_empty, 1);
     mbar_init(p_ready, 128);
     mbar_init(o_done, 1);
-    mbar_init(q_ready, 128);
     mbar_init(fin, 1);
     fence_barrier_init();
     info[1] = 0;
     info[2] = 0;
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&maps.k)) : "memory");
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&maps.v)) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&maps.q)) : "memory");
   }
   if (wid == 5) {
     tc::alloc(tmem_slot, Tr::kTmemCols);
@@ -327,7 +333,7 @@ __global__ void __launch_bounds__(PrefillTcTraits<D, BS, G>::kThreads, 1)
 
   if (wid == 4) {
     // ================= producer: key and value tiles by TMA =================
-    long long kv_base = 0;
+    long long kv_base = 0, qt = 0;
     long long k_issued = 0, v_issued = 0;
     bool ok = true;
     TcTile t;
@@ -336,43 +342,89 @@ __global__ void __launch_bounds__(PrefillTcTraits<D, BS, G>::kThreads, 1)
         if (lane == 0 && t.tau == 0 && t.kvh == 0) set_error(a.err, PA_DEVERR_CONTEXT_LEN);
         continue;
       }
-      if (lane == 0) {
-        const int32_t *row = a.block_tables + (long long)t.s * a.bt_s;
-        for (int j = 0; j < t.n_kv && ok; ++j) {
-          const long long it = kv_base + j;
-          const int b = (int)(it & 1);
-          const long long use = it >> 1;
-          const int p0 = j * Tr::kKv;
-          const int pend = min(p0 + Tr::kKv, t.L);
-          const uint32_t bytes = (uint32_t)((pend - p0 + 7) / 8) * Tr::kBoxBytes;
-          for (int which = 0; which < 2 && ok; ++which) {
-            uint64_t *full = which ? v_full + b : k_full + b;
-            uint64_t *empty = which ? v_empty + b : k_empty + b;
-            if (use >= 1 && !wait(empty, (uint32_t)((use - 1) & 1))) {
-              ok = false;
-              break;
-            }
-            mbar_arrive_expect_tx(full, bytes);
-            const uint32_t dst = (which ? v_s : k_s) + b * Tr::kKvBytes;
-            const CUtensorMap *map = which ? &maps.v : &maps.k;
-            for (int p = p0; p < pend; p += BS) {
-              int blk = __ldg(row + p / BS);
-              if (blk < 0 || (long long)blk >= a.num_blocks) {
-                set_error(a.err, PA_DEVERR_BLOCK_ID);
-                blk = 0;
-              }
-              for (int y = 0; y < BS && p + y < pend; y += 8)
-                tma_load_tile(dst + ((p + y - p0) / 8) * Tr::kBoxBytes, map, y, t.kvh, blk, full);
-            }
-            if (which) ++v_issued; else ++k_issued;
+      {
+        // the tile's query rows: tokens q0 + tok0 .. + 128/G of heads kvh*G .. + G (rows past
+        // the tensor read as zeros, rows of the next sequence are computed and dropped), once
+        // the previous tile's S = QK^T are all done
+        bool q_ok = true;
+        if (lane == 0) {
+          q_ok = qt < 1 || wait(q_empty, (uint32_t)((qt - 1) & 1));
+          if (q_ok) {
+            mbar_arrive_expect_tx(q_full, Tr::kQBytes);
+            tma_load_4d(q_s, &maps.q, 0, t.kvh * G, t.q0 + t.tok0, 0, q_full);
           }
         }
+        if (__shfl_sync(FULL_MASK, q_ok ? 1 : 0, 0) == 0) {
+          ok = false;
+          break;
+        }
+        ++qt;
+      }
+      // Block ids of a kv tile: lane i holds the tile's i-th block (at most 16 blocks).  The
+      // ids of tile j + 1 are fetched before the waits of tile j, so their latency is hidden.
+      const int32_t *row = a.block_tables + (long long)t.s * a.bt_s;
+      auto fetch_ids = [&](int j) {
+        const int p0 = j * Tr::kKv;
+        const int nblk = (min(p0 + Tr::kKv, t.L) - p0 + BS - 1) / BS;
+        int blk = 0;
+        if (lane < nblk) {
+          blk = __ldg(row + p0 / BS + lane);
+          if (blk < 0 || (long long)blk >= a.num_blocks) {
+            set_error(a.err, PA_DEVERR_BLOCK_ID);
+            blk = 0;
+          }
+        }
+        return blk;
+      };
+      int cur = fetch_ids(0);
+      for (int j = 0; j < t.n_kv && ok; ++j) {
+        const int nxt = j + 1 < t.n_kv ? fetch_ids(j + 1) : 0;
+        const long long it = kv_base + j;
+        const int b = (int)(it & 1);
+        const long long use = it >> 1;
+        const int p0 = j * Tr::kKv;
+        const int pend = min(p0 + Tr::kKv, t.L);
+        const int nblk = (pend - p0 + BS - 1) / BS;
+        const uint32_t bytes = (uint32_t)(a.grouped_maps ? nblk * (BS / 8) : (pend - p0 + 7) / 8) * Tr::kBoxBytes;
+        for (int which = 0; which < 2; ++which) {
+          uint64_t *full = which ? v_full + b : k_full + b;
+          uint64_t *empty = which ? v_empty + b : k_empty + b;
+          bool w_ok = true;
+          if (lane == 0) {
+            w_ok = use < 1 || wait(empty, (uint32_t)((use - 1) & 1));
+            if (w_ok) mbar_arrive_expect_tx(full, bytes);
+          }
+          if (__shfl_sync(FULL_MASK, w_ok ? 1 : 0, 0) == 0) {
+            ok = false;
+            break;
+          }
+          const uint32_t dst = (which ? v_s : k_s) + b * Tr::kKvBytes;
+          const CUtensorMap *map = which ? &maps.v : &maps.k;
+          if (a.grouped_maps) {
+            // lane i copies the tile's i-th (block, kv head) tile, rows past the context
+            // included: the copies of one kv tile are issued together
+            if (lane < nblk)
+              tma_load_tile(dst + (lane * BS / 8) * Tr::kBoxBytes, map, 0, 0, cur * Hkv + t.kvh, full);
+          } else {
+            for (int bi = 0; bi < nblk; ++bi) {
+              const int blk = __shfl_sync(FULL_MASK, cur, bi);
+              if (lane == 0) {
+                const int p = p0 + bi * BS;
+                for (int y = 0; y < BS && p + y < pend; y += 8)
+                  tma_load_tile(dst + ((p + y - p0) / 8) * Tr::kBoxBytes, map, y, t.kvh, blk, full);
+              }
+            }
+          }
+          if (which) ++v_issued; else ++k_issued;
+        }
+        cur = nxt;
       }
       ok = __shfl_sync(FULL_MASK, ok ? 1 : 0, 0) != 0;
       kv_base += t.n_kv;
     }
     if (lane == 0 && !ok) {
       // let the copies in flight land before the CTA leaves
+      if (qt > 0) mbar_wait_bounded(q_full, (uint32_t)((qt - 1) & 1), a.wait_cycles);
       for (long long i = k_issued > 2 ? k_issued - 2 : 0; i < k_issued; ++i)
         mbar_wait_bounded(k_full + (i & 1), (uint32_t)((i >> 1) & 1), a.wait_cycles);
       for (long long i = v_issued > 2 ? v_issued - 2 : 0; i < v_issued; ++i)
@@ -405,8 +457,9 @@ __global__ void __launch_bounds__(PrefillTcTraits<D, BS, G>::kThreads, 1)
     };
     for (long long round = 0; ok && next_tile(round, t); ++round) {
       if (!t.valid) continue;
+      const uint32_t qbuf = q_s;
       if (lane == 0) {
-        ok = wait(q_ready, (uint32_t)(qt & 1));
+        ok = wait(q_full, (uint32_t)(qt & 1));
         tc::fence_after();
         for (int j = 0; j < t.n_kv && ok; ++j) {
           const long long it = kv_base + j;
@@ -421,12 +474,15 @@ __global__ void __launch_bounds__(PrefillTcTraits<D, BS, G>::kThreads, 1)
           const uint32_t kb = k_s + b * Tr::kKvBytes;
 #pragma unroll
           for (int ks = 0; ks < D / 16; ++ks) {
-            const uint32_t off = (ks >> 2) * 1024 + (ks & 3) * 32;
-            tc::mma(tmem + 128 * b, tc::smem_desc(q_s + off, 16, Tr::kGroup),
-                    tc::smem_desc(kb + off, 16, Tr::kGroup), kIdS, ks > 0 ? 1u : 0u);
+            // query rows span-major (128 rows of a 64-element span, then the next span), keys
+            // in 8-row groups of both spans
+            const uint32_t inner = (ks & 3) * 32;
+            tc::mma(tmem + 128 * b, tc::smem_desc(qbuf + (ks >> 2) * (Tr::kRows * 128) + inner, 16, 1024),
+                    tc::smem_desc(kb + (ks >> 2) * 1024 + inner, 16, Tr::kGroup), kIdS, ks > 0 ? 1u : 0u);
           }
           tc::commit(s_full + b);
           tc::commit(k_empty + b);
+          if (j == t.n_kv - 1) tc::commit(q_empty);
           if (j > 0) ok = pv(j - 1);
         }
         if (ok) ok = pv(t.n_kv - 1);
@@ -446,7 +502,6 @@ __global__ void __launch_bounds__(PrefillTcTraits<D, BS, G>::kThreads, 1)
     const int r = tid;  // row = tensor-memory lane
     const int lt = r / G, hh = r % G;
     const uint32_t lane_base = tc::taddr(tmem, 32 * wid, 0);
-    const uint32_t q_row = q_s + (r >> 3) * Tr::kGroup + (r & 7) * 128;
     const uint32_t p_row = (r >> 3) * 2048 + (r & 7) * 128;
     long long kv_base = 0;
     bool ok = true;
@@ -455,22 +510,6 @@ __global__ void __launch_bounds__(PrefillTcTraits<D, BS, G>::kThreads, 1)
       if (!t.valid) continue;
       const bool row_ok = lt < t.ntok;
       const int prow = row_ok ? t.pos0 + lt : -1;
-      // ---- the tile's query rows into shared memory (swizzled, zero rows past the tile) ----
-      {
-        const uint4 *src = reinterpret_cast<const uint4 *>(
-            static_cast<const T *>(a.query) + (long long)(t.q0 + t.tok0 + (row_ok ? lt : 0)) * a.q_t +
-            (long long)(t.kvh * G + hh) * a.q_h);
-#pragma unroll
-        for (int c = 0; c < D / 8; ++c) {
-          const uint4 v = row_ok ? __ldg(src + c) : make_uint4(0u, 0u, 0u, 0u);
-          const uint32_t dst = q_row + (c >> 3) * 1024 + (((c & 7) ^ (r & 7)) << 4);
-          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(v.x), "r"(v.y),
-                       "r"(v.z), "r"(v.w)
-                       : "memory");
-        }
-        fence_proxy_async_smem();
-        mbar_arrive(q_ready);
-      }
       float m_ref = -INFINITY, l_sum = 0.f;
       for (int j = 0; j < t.n_kv; ++j) {
         const long long it = kv_base + j;
@@ -480,50 +519,62 @@ __global__ void __launch_bounds__(PrefillTcTraits<D, BS, G>::kThreads, 1)
           break;
         }
         tc::fence_after();
-        // ---- mask, maximum in base 2 (S read 32 columns at a time) ----
+        // ---- weights in base 2 against the row's reference maximum, and their two 16-bit
+        // terms.  S is read 32 columns at a time, the next load in flight while the current
+        // columns are processed; every lane of the warp takes part in the loads. ----
         const int c_lim = prow - j * Tr::kKv;  // columns 0 .. c_lim are visible to this row
         const uint32_t s_addr = lane_base + 128 * b;
-        float hi_raw = -INFINITY, lo_raw = INFINITY;
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          uint32_t sr[32];
-          tc::ld32x32(s_addr + 32 * q, sr);
-#pragma unroll
-          for (int c = 0; c < 32; ++c) {
-            const float v = 32 * q + c <= c_lim ? __uint_as_float(sr[c]) : NAN;
-            hi_raw = fmaxf(hi_raw, v);  // fmaxf / fminf skip the NaN of masked columns
-            lo_raw = fminf(lo_raw, v);
-          }
-        }
-        // the largest scaled logit (the scale may be negative); -inf when nothing is visible
-        const float mx = c_lim < 0 ? -INFINITY : (a.scale_log2 >= 0.f ? hi_raw : lo_raw) * a.scale_log2;
-        float alpha = 1.f;
-        bool rescale = false;
-        if (mx > m_ref + 8.f) {
-          alpha = m_ref == -INFINITY ? 0.f : fast_exp2(m_ref - mx);
-          rescale = j > 0;
-          m_ref = mx;
-          l_sum *= alpha;
-        }
-        // ---- weights and their two 16-bit terms (S read again; every lane of the warp takes
-        // part in the tensor-memory loads, rows with nothing visible get zero weights) ----
         uint32_t hp[64], lp[64];
-        const float nm = m_ref == -INFINITY ? 0.f : -m_ref;
-        __syncwarp();
+        // t = logit * scale_log2 - m_ref for visible columns, -inf elsewhere; returns the row's
+        // largest t and fills hp / lp with 2^t (when exps) and the sum of the weights in l_t
+        auto pass = [&](float nm, bool exps, float &l_t) -> float {
+          float tmax = -INFINITY;
+          l_t = 0.f;
+          auto chunk = [&](const uint32_t(&r)[32], int q) {
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          uint32_t sr[32];
-          tc::ld32x32(s_addr + 32 * q, sr);
+            for (int i = 0; i < 16; ++i) {
+              const int c0 = 32 * q + 2 * i;
+              const float t0 = c0 <= c_lim ? fmaf(__uint_as_float(r[2 * i]), a.scale_log2, nm) : -INFINITY;
+              const float t1 = c0 + 1 <= c_lim ? fmaf(__uint_as_float(r[2 * i + 1]), a.scale_log2, nm) : -INFINITY;
+              tmax = fmaxf(tmax, fmaxf(t0, t1));
+              if (exps) {
+                const float p0 = fast_exp2(t0), p1 = fast_exp2(t1);
+                l_t += p0 + p1;
+                split2<kBf16>(p0, p1, hp[16 * q + i], lp[16 * q + i]);
+              }
+            }
+          };
+          // the whole row in one load: under the MMAs' own tensor-memory traffic, one long
+          // load costs less than four shorter ones in a chain
+          __syncwarp();
+          uint32_t sr[128];
+          tc::ld32x128(s_addr, sr);
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const int c0 = 32 * q + 2 * i;
-            float p0 = fast_exp2(fmaf(__uint_as_float(sr[2 * i]), a.scale_log2, nm));
-            float p1 = fast_exp2(fmaf(__uint_as_float(sr[2 * i + 1]), a.scale_log2, nm));
-            p0 = c0 <= c_lim ? p0 : 0.f;
-            p1 = c0 + 1 <= c_lim ? p1 : 0.f;
-            l_sum += p0 + p1;
-            split2<kBf16>(p0, p1, hp[16 * q + i], lp[16 * q + i]);
+          for (int q = 0; q < 4; ++q) chunk(*reinterpret_cast<const uint32_t(*)[32]>(sr + 32 * q), q);
+          return tmax;
+        };
+        float l_t, alpha = 1.f;
+        bool rescale = false;
+        if (j == 0) {
+          // first kv tile: the maximum first, then the weights
+          const float mx = pass(0.f, false, l_t);
+          m_ref = mx;
+          pass(m_ref == -INFINITY ? 0.f : -m_ref, true, l_t);
+          l_sum = l_t;
+        } else {
+          // later tiles: weights against the current reference; a row whose logits pass it by
+          // more than 2^8 moves its reference and takes the pass again
+          const float tmax = pass(m_ref == -INFINITY ? 0.f : -m_ref, true, l_t);
+          const bool move = tmax > 8.f;
+          if (__any_sync(FULL_MASK, move)) {
+            if (move) {
+              alpha = fast_exp2(-tmax);
+              rescale = true;
+              m_ref += tmax;
+            }
+            pass(m_ref == -INFINITY ? 0.f : -m_ref, true, l_t);
           }
+          l_sum = l_sum * alpha + l_t;
         }
         tc::fence_before();
         mbar_arrive(s_free + b);
@@ -561,6 +612,7 @@ __global__ void __launch_bounds__(PrefillTcTraits<D, BS, G>::kThreads, 1)
                              "r"(0u)
                              : "memory");
           }
+          fence_proxy_async_smem();
         }
         // ---- P (hi, lo) into shared memory, swizzled like the operand tiles ----
 #pragma unroll
@@ -635,7 +687,7 @@ __global__ void __launch_bounds__(PrefillTcTraits<D, BS, G>::kThreads, 1)
 }
 
 template <typename T, int D, int BS, int G>
-cudaError_t launch_prefill_tc(const PrefillArgs &a, const TmaMaps *maps, int num_ctas, cudaStream_t st) {
+cudaError_t launch_prefill_tc(const PrefillArgs &a, const PrefillMaps *maps, int num_ctas, cudaStream_t st) {
   using Tr = PrefillTcTraits<D, BS, G>;
   paged_prefill_tc_kernel<T, D, BS, G><<<num_ctas, Tr::kThreads, Tr::kSmemBytes, st>>>(a, *maps);
   return cudaGetLastError();

@@ -74,6 +74,39 @@ def test_prefill_configurations(oracle, dtype, D, bs, hq, hkv):
     assert_no_device_error()
 
 
+def _scale_keys_by_position(b, factor):
+    """Multiply the key of position t of every sequence by factor(t), in the cache and in the
+    new tokens' rows, re-rounded to the storage type."""
+    dt, bs = b.dtype, b.block_size
+    kc = W.decode_to_f64(b.key_cache, dt)
+    key = W.decode_to_f64(b.key, dt)
+    for s in range(b.num_seqs):
+        L = int(b.context_lens[s])
+        q0, q1 = int(b.query_start[s]), int(b.query_start[s + 1])
+        for t in range(L - (q1 - q0)):
+            kc[b.block_tables[s, t // bs], :, t % bs, :] *= factor(t)
+        for j in range(q1 - q0):
+            key[q0 + j] *= factor(L - (q1 - q0) + j)
+    b.key_cache = W.encode(kc, dt)
+    b.key = W.encode(key, dt)
+
+
+def test_prefill_growing_logits_move_the_reference(oracle):
+    """Keys that grow with the position make every later kv tile's logits pass the row's
+    reference maximum by far more than 2^8, so the kernel rescales O in tensor memory and takes
+    the weights' pass again on almost every tile; the result must not change."""
+    require_gpu()
+    b = W.build_prefill_batch("pfgrow", [700, 390, 260], [300, 390, 5], num_heads=32,
+                              num_kv_heads=8, head_dim=128, block_size=16, dtype="bf16",
+                              seed=W.BASE_SEED + 745)
+    _scale_keys_by_position(b, lambda t: 1.0 + t / 8.0)
+    ref, _, _ = _oracle(oracle, b)
+    st = PrefillStep(b)
+    assert_close(st.run("f32"), ref, "bf16", "prefill growing logits")
+    assert_bf16_output(st.run("bf16"), ref, "prefill growing logits bf16 out")
+    assert_no_device_error()
+
+
 def test_prefill_chunked_workload_sampled(oracle):
     """The full-size chunked-prefill step on the GPU; the oracle recomputes three of its
     sequences (their rows of the output)."""
