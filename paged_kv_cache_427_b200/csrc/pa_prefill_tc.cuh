@@ -11,26 +11,28 @@
 //
 // A tile is 128 query rows of one (sequence, kv head): 128 / G new tokens times the G query
 // heads that read that kv head (head fastest), one row per tensor-memory lane.  The context is
-// walked in kv tiles of 128 positions.  One persistent CTA per SM, six warps:
-//   * warp 4 streams the tile's query rows (one 4-D box, loaded as soon as the previous tile's
-//     last S = QK^T is done, so it overlaps that tile's end) and the key and value tiles of 128
-//     positions through two-slot rings by TMA: one box per (block, kv head) tile of the paged
-//     cache, 128-byte swizzle, in 8-row groups placed one after another, which is the operand
-//     layout of the MMAs; the lanes issue the boxes of a kv tile together;
-//   * warp 5 (one lane) issues the MMAs: S = Q K^T (M = 128 rows, N = 128 positions, K = head
-//     dim) into one of two S buffers in tensor memory, and O += P V (N = head dim, K = 128
+// walked in kv tiles of 64 positions.  One persistent CTA per SM, ten warps:
+//   * warp 8 streams the tile's query rows (one 4-D box, loaded as soon as the previous tile's
+//     last S = QK^T is done, so it overlaps that tile's end) and the key and value tiles through
+//     three-slot rings by TMA: one box per (block, kv head) tile of the paged cache, 128-byte
+//     swizzle, in 8-row groups placed one after another, which is the operand layout of the
+//     MMAs; the lanes issue the boxes of a kv tile together;
+//   * warp 9 (one lane) issues the MMAs: S = Q K^T (M = 128 rows, N = 64 positions, K = head
+//     dim) into one of two S buffers in tensor memory, and O += P V (N = head dim, K = 64
 //     positions) into the O accumulator, P split into two 16-bit terms (hi + lo) as in the
 //     decode kernels so the weights keep about 16 significant bits;
-//   * warps 0-3 (one thread per row) read S from tensor memory, apply the causal mask (which
-//     also hides positions past the context), keep the online softmax per row in base 2 with a
-//     lazy reference maximum (moved only when a logit passes it by 2^8, when O is rescaled in
-//     tensor memory), write P to shared memory and finally read O, divide by the row sums and
-//     store the rows.  (P read by the MMA from tensor memory instead measured slower: the
-//     softmax warps' tensor-memory loads then wait behind the MMA's operand reads.)
-// The MMA warp issues S of kv tile j + 1 before O += P V of tile j, so the tensor cores compute
-// the next scores while the softmax warps work on the current ones.  Barriers between the roles
-// are mbarriers (copies: transaction bytes; MMAs: tcgen05.commit; threads: arrival counts);
-// every wait is bounded and a timeout sets an error bit and winds the CTA down.
+//   * warps 0-7 run the softmax, two threads per row: warp w reads tensor-memory lanes
+//     32 (w % 4) .. + 31 and columns 32 (w / 4) .. + 31 of S.  Each thread masks its columns
+//     causally (which also hides positions past the context), keeps the online softmax of its
+//     half of the row in base 2 against a reference maximum the two halves share (exchanged
+//     through shared memory; moved only when a logit passes it by 2^8, when O is rescaled in
+//     tensor memory) and writes its part of P to one of two P buffers in shared memory; at the
+//     end of the tile the halves add their row sums and each stores half of the row of O / l.
+// The MMA warp issues S of kv tile j + 1 before O += P V of tile j, and P has two buffers, so
+// the tensor cores compute the next scores and the previous products while the softmax warps
+// work on the current scores.  Barriers between the roles are mbarriers (copies: transaction
+// bytes; MMAs: tcgen05.commit; threads: arrival counts); every wait is bounded and a timeout sets
+// an error bit and winds the CTA down.
 //
 // Tiles differ in cost (a tile's causal prefix), so they are spread longest first: every CTA
 // builds the same list of (sequence, tile) pairs sorted by cost (a histogram of costs in shared
@@ -48,36 +50,42 @@ namespace pa {
 
 template <int D, int BS, int G>
 struct PrefillTcTraits {
-  static constexpr int kThreads = 192;
+  static constexpr int kSoftmaxWarps = 8;
+  static constexpr int kSoftmaxThreads = kSoftmaxWarps * 32;
+  static constexpr int kProducerWarp = 8;
+  static constexpr int kMmaWarp = 9;
+  static constexpr int kThreads = 320;
   static constexpr int kRows = 128;             // query rows of a tile (MMA M)
   static constexpr int kTokens = kRows / G;     // new tokens of a tile
-  static constexpr int kKv = 128;               // context positions of a kv tile
+  static constexpr int kKv = 64;                // context positions of a kv tile
+  static constexpr int kCols = kKv / 2;         // S columns per softmax thread
   static constexpr int kSpans = D / 64;
-  static constexpr int kGroup = kSpans * 1024;  // bytes between 8-row groups of Q, K, V tiles
-  static constexpr int kQBytes = kRows * D * 2;
+  static constexpr int kGroup = kSpans * 1024;  // bytes between 8-row groups of K, V tiles
+  static constexpr int kQBytes = kRows * D * 2; // span-major: 128 rows of a span, then the next
   static constexpr int kKvBytes = kKv * D * 2;
-  static constexpr int kPBytes = kRows * kKv * 2;  // 8-row groups of 2048 bytes
-  static constexpr int kBoxBytes = 8 * D * 2;      // one 8-position TMA box, both spans
-  static constexpr int kQOff = 0;                  // query rows, span-major
+  static constexpr int kPBytes = kRows * kKv * 2;  // one term of P: 8-row groups of 1 KB
+  static constexpr int kBoxBytes = 8 * D * 2;      // 8 positions, both spans
+  static constexpr int kQOff = 0;
   static constexpr int kKOff = kQOff + kQBytes;
-  static constexpr int kVOff = kKOff + 2 * kKvBytes;
-  static constexpr int kPhOff = kVOff + 2 * kKvBytes;
-  static constexpr int kPlOff = kPhOff + kPBytes;
-  static constexpr int kBarOff = kPlOff + kPBytes;
-  static constexpr int kNumBars = 20;
+  static constexpr int kStages = 3;             // key and value rings
+  static constexpr int kVOff = kKOff + kStages * kKvBytes;
+  static constexpr int kPOff = kVOff + kStages * kKvBytes;  // two buffers of (hi, lo)
+  static constexpr int kBarOff = kPOff + 4 * kPBytes;
+  static constexpr int kNumBars = 28;
   static constexpr int kInfoOff = kBarOff + kNumBars * 8;  // [tmem base, abort, tile count, rounds]
+  static constexpr int kXchOff = kInfoOff + 32;            // float [2 parities][2 halves][128 rows]
   static constexpr int kMaxMine = 64;                      // rounds of the sorted schedule
-  static constexpr int kMineOff = kInfoOff + 32;
+  static constexpr int kMineOff = kXchOff + 2 * 2 * kRows * 4;
   static constexpr int kSmemBytes = kMineOff + kMaxMine * 8 + 1024;  // + 1 KB alignment
-  // the sorted schedule's scratch (histogram of costs, tile list) lives in the key ring before
-  // the first copy
+  // the sorted schedule's scratch (histogram of costs, tile list) lives in the key and value
+  // rings before the first copy
   static constexpr int kMaxBins = 2048;  // costs 0 .. 2047 (16-position steps)
   static constexpr int kMaxList = 4096;  // (sequence, tile) pairs
-  static constexpr int kTmemCols = 512;  // S0 [0, 128), S1 [128, 256), O [256, 256 + D)
+  static constexpr int kTmemCols = 256;  // S0 [0, 64), S1 [64, 128), O [128, 128 + D)
   static_assert(D == 64 || D == 128, "head_dim 64 or 128");
   static_assert(G == 1 || G == 2 || G == 4 || G == 8, "1, 2, 4 or 8 query heads per kv head");
-  static_assert(BS % 8 == 0, "block size a multiple of the 8-position box");
-  static_assert((kMaxBins + kMaxList) * 4 <= 2 * kKvBytes, "schedule scratch fits the key ring");
+  static_assert(BS % 8 == 0 && kKv % BS == 0, "block size a multiple of the 8-position box");
+  static_assert((kMaxBins + kMaxList) * 4 <= 2 * kStages * kKvBytes, "schedule scratch fits the rings");
   static_assert(kSmemBytes <= 232448, "shared memory of one CTA");
 };
 
@@ -149,10 +157,11 @@ __global__ void __launch_bounds__(PrefillTcTraits<D, BS, G>::kThreads, 1)
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + Tr::kBarOff);
-  uint64_t *k_full = bars + 0, *k_empty = bars + 2, *v_full = bars + 4, *v_empty = bars + 6;
-  uint64_t *s_full = bars + 8, *s_free = bars + 10;
-  uint64_t *q_full = bars + 12, *q_empty = bars + 13;
-  uint64_t *p_ready = bars + 16, *o_done = bars + 17, *fin = bars + 18;
+  // rings of kStages slots (key, value tiles) and of two (S, P buffers)
+  uint64_t *k_full = bars + 0, *k_empty = bars + 3, *v_full = bars + 6, *v_empty = bars + 9;
+  uint64_t *s_full = bars + 12, *s_free = bars + 14, *p_ready = bars + 16, *pv_done = bars + 18;
+  uint64_t *q_full = bars + 20, *q_empty = bars + 21, *fin = bars + 22;
+  uint64_t *xbar = bars + 23;  // per row quarter: the exchanges between its two softmax warps
   volatile int *info = reinterpret_cast<volatile int *>(smem + Tr::kInfoOff);
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + Tr::kInfoOff);
   int2 *mine = reinterpret_cast<int2 *>(smem + Tr::kMineOff);
@@ -164,19 +173,22 @@ __global__ void __launch_bounds__(PrefillTcTraits<D, BS, G>::kThreads, 1)
   const int max_len = a.max_blocks * BS;
 
   if (tid == 0) {
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < Tr::kStages; ++i) {
       mbar_init(k_full + i, 1);
       mbar_init(k_empty + i, 1);
       mbar_init(v_full + i, 1);
       mbar_init(v_empty + i, 1);
+    }
+    for (int i = 0; i < 2; ++i) {
       mbar_init(s_full + i, 1);
-      mbar_init(s_free + i, 128);
+      mbar_init(s_free + i, Tr::kSoftmaxThreads);
+      mbar_init(p_ready + i, Tr::kSoftmaxThreads);
+      mbar_init(pv_done + i, 1);
     }
     mbar_init(q_full, 1);
     mbar_init(q_empty, 1);
-    mbar_init(p_ready, 128);
-    mbar_init(o_done, 1);
     mbar_init(fin, 1);
+    for (int i = 0; i < 4; ++i) mbar_init(xbar + i, 64);
     fence_barrier_init();
     info[1] = 0;
     info[2] = 0;
@@ -184,7 +196,7 @@ __global__ void __launch_bounds__(PrefillTcTraits<D, BS, G>::kThreads, 1)
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&maps.v)) : "memory");
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&maps.q)) : "memory");
   }
-  if (wid == 5) {
+  if (wid == Tr::kMmaWarp) {
     tc::alloc(tmem_slot, Tr::kTmemCols);
     tc::relinquish();
   }
@@ -328,11 +340,10 @@ __global__ void __launch_bounds__(PrefillTcTraits<D, BS, G>::kThreads, 1)
   const uint32_t q_s = smem_u32(smem + Tr::kQOff);
   const uint32_t k_s = smem_u32(smem + Tr::kKOff);
   const uint32_t v_s = smem_u32(smem + Tr::kVOff);
-  const uint32_t ph_s = smem_u32(smem + Tr::kPhOff);
-  const uint32_t pl_s = smem_u32(smem + Tr::kPlOff);
+  const uint32_t p_s = smem_u32(smem + Tr::kPOff);  // P buffer b: hi at + 2b kPBytes, lo after it
 
-  if (wid == 4) {
-    // ================= producer: key and value tiles by TMA =================
+  if (wid == Tr::kProducerWarp) {
+    // ================= producer: query rows, key and value tiles by TMA =================
     long long kv_base = 0, qt = 0;
     long long k_issued = 0, v_issued = 0;
     bool ok = true;
@@ -380,8 +391,8 @@ __global__ void __launch_bounds__(PrefillTcTraits<D, BS, G>::kThreads, 1)
       for (int j = 0; j < t.n_kv && ok; ++j) {
         const int nxt = j + 1 < t.n_kv ? fetch_ids(j + 1) : 0;
         const long long it = kv_base + j;
-        const int b = (int)(it & 1);
-        const long long use = it >> 1;
+        const int b = (int)(it % Tr::kStages);
+        const long long use = it / Tr::kStages;
         const int p0 = j * Tr::kKv;
         const int pend = min(p0 + Tr::kKv, t.L);
         const int nblk = (pend - p0 + BS - 1) / BS;
@@ -425,12 +436,13 @@ __global__ void __launch_bounds__(PrefillTcTraits<D, BS, G>::kThreads, 1)
     if (lane == 0 && !ok) {
       // let the copies in flight land before the CTA leaves
       if (qt > 0) mbar_wait_bounded(q_full, (uint32_t)((qt - 1) & 1), a.wait_cycles);
-      for (long long i = k_issued > 2 ? k_issued - 2 : 0; i < k_issued; ++i)
-        mbar_wait_bounded(k_full + (i & 1), (uint32_t)((i >> 1) & 1), a.wait_cycles);
-      for (long long i = v_issued > 2 ? v_issued - 2 : 0; i < v_issued; ++i)
-        mbar_wait_bounded(v_full + (i & 1), (uint32_t)((i >> 1) & 1), a.wait_cycles);
+      constexpr int S = Tr::kStages;
+      for (long long i = k_issued > S ? k_issued - S : 0; i < k_issued; ++i)
+        mbar_wait_bounded(k_full + (int)(i % S), (uint32_t)((i / S) & 1), a.wait_cycles);
+      for (long long i = v_issued > S ? v_issued - S : 0; i < v_issued; ++i)
+        mbar_wait_bounded(v_full + (int)(i % S), (uint32_t)((i / S) & 1), a.wait_cycles);
     }
-  } else if (wid == 5) {
+  } else if (wid == Tr::kMmaWarp) {
     // ================= MMA issue =================
     constexpr uint32_t kIdS = tc::idesc_f16(kBf16, 128, Tr::kKv, false);
     constexpr uint32_t kIdO = tc::idesc_f16(kBf16, 128, D, true);
@@ -440,19 +452,22 @@ __global__ void __launch_bounds__(PrefillTcTraits<D, BS, G>::kThreads, 1)
     TcTile t;
     auto pv = [&](int j) -> bool {
       const long long it = kv_base + j;
-      const int b = (int)(it & 1);
-      if (!wait(p_ready, (uint32_t)(it & 1)) || !wait(v_full + b, (uint32_t)((it >> 1) & 1))) return false;
+      const int b = (int)(it & 1);               // P buffer
+      const int vs = (int)(it % Tr::kStages);    // value slot
+      if (!wait(p_ready + b, (uint32_t)((it >> 1) & 1)) ||
+          !wait(v_full + vs, (uint32_t)((it / Tr::kStages) & 1)))
+        return false;
       tc::fence_after();
-      const uint32_t vb = v_s + b * Tr::kKvBytes;
+      const uint32_t vb = v_s + vs * Tr::kKvBytes;
+      const uint32_t ph = p_s + 2 * b * Tr::kPBytes, pl = ph + Tr::kPBytes;
 #pragma unroll
       for (int kt = 0; kt < Tr::kKv / 16; ++kt) {
         const uint64_t vd = tc::smem_desc(vb + kt * 2 * Tr::kGroup, 1024, Tr::kGroup);
-        const uint32_t poff = (kt >> 2) * 1024 + (kt & 3) * 32;
-        tc::mma(tmem + 256, tc::smem_desc(ph_s + poff, 16, 2048), vd, kIdO, (j > 0 || kt > 0) ? 1u : 0u);
-        tc::mma(tmem + 256, tc::smem_desc(pl_s + poff, 16, 2048), vd, kIdO, 1u);
+        tc::mma(tmem + 128, tc::smem_desc(ph + kt * 32, 16, 1024), vd, kIdO, (j > 0 || kt > 0) ? 1u : 0u);
+        tc::mma(tmem + 128, tc::smem_desc(pl + kt * 32, 16, 1024), vd, kIdO, 1u);
       }
-      tc::commit(o_done);
-      tc::commit(v_empty + b);
+      tc::commit(pv_done + b);
+      tc::commit(v_empty + vs);
       return true;
     };
     for (long long round = 0; ok && next_tile(round, t); ++round) {
@@ -463,25 +478,25 @@ __global__ void __launch_bounds__(PrefillTcTraits<D, BS, G>::kThreads, 1)
         tc::fence_after();
         for (int j = 0; j < t.n_kv && ok; ++j) {
           const long long it = kv_base + j;
-          const int b = (int)(it & 1);
-          const long long use = it >> 1;
-          if (!wait(k_full + b, (uint32_t)(use & 1)) ||
-              (use >= 1 && !wait(s_free + b, (uint32_t)((use - 1) & 1)))) {
+          const int b = (int)(it & 1);              // S buffer
+          const int ks_ = (int)(it % Tr::kStages);  // key slot
+          if (!wait(k_full + ks_, (uint32_t)((it / Tr::kStages) & 1)) ||
+              (it >= 2 && !wait(s_free + b, (uint32_t)(((it >> 1) - 1) & 1)))) {
             ok = false;
             break;
           }
           tc::fence_after();
-          const uint32_t kb = k_s + b * Tr::kKvBytes;
+          const uint32_t kb = k_s + ks_ * Tr::kKvBytes;
 #pragma unroll
           for (int ks = 0; ks < D / 16; ++ks) {
             // query rows span-major (128 rows of a 64-element span, then the next span), keys
             // in 8-row groups of both spans
             const uint32_t inner = (ks & 3) * 32;
-            tc::mma(tmem + 128 * b, tc::smem_desc(qbuf + (ks >> 2) * (Tr::kRows * 128) + inner, 16, 1024),
+            tc::mma(tmem + Tr::kKv * b, tc::smem_desc(qbuf + (ks >> 2) * (Tr::kRows * 128) + inner, 16, 1024),
                     tc::smem_desc(kb + (ks >> 2) * 1024 + inner, 16, Tr::kGroup), kIdS, ks > 0 ? 1u : 0u);
           }
           tc::commit(s_full + b);
-          tc::commit(k_empty + b);
+          tc::commit(k_empty + ks_);
           if (j == t.n_kv - 1) tc::commit(q_empty);
           if (j > 0) ok = pv(j - 1);
         }
@@ -498,11 +513,25 @@ __global__ void __launch_bounds__(PrefillTcTraits<D, BS, G>::kThreads, 1)
     }
     __syncwarp();
   } else {
-    // ================= softmax, one thread per row =================
-    const int r = tid;  // row = tensor-memory lane
+    // ================= softmax, two threads per row =================
+    const int quarter = wid & 3, half = wid >> 2;
+    const int r = 32 * quarter + lane;  // row = tensor-memory lane
     const int lt = r / G, hh = r % G;
-    const uint32_t lane_base = tc::taddr(tmem, 32 * wid, 0);
-    const uint32_t p_row = (r >> 3) * 2048 + (r & 7) * 128;
+    const uint32_t lane_base = tc::taddr(tmem, 32 * quarter, 0);
+    const uint32_t p_row = (r >> 3) * 1024 + (r & 7) * 128;
+    float *xch = reinterpret_cast<float *>(smem + Tr::kXchOff);  // [parity][half][row]
+    // The two threads of a row swap a value through shared memory; the two warps of a row
+    // quarter meet at their own mbarrier (bounded wait), exchanges alternate between two slots.
+    long long nx = 0;  // exchanges so far (the same count in both warps of a quarter)
+    auto swap_with_other_half = [&](float mine_v, float &other) -> bool {
+      float *xs = xch + (nx & 1) * 2 * Tr::kRows;
+      xs[half * Tr::kRows + r] = mine_v;
+      mbar_arrive(xbar + quarter);
+      const bool got = __all_sync(FULL_MASK, wait(xbar + quarter, (uint32_t)(nx & 1)));
+      other = xs[(half ^ 1) * Tr::kRows + r];
+      ++nx;
+      return got;
+    };
     long long kv_base = 0;
     bool ok = true;
     TcTile t;
@@ -510,7 +539,7 @@ __global__ void __launch_bounds__(PrefillTcTraits<D, BS, G>::kThreads, 1)
       if (!t.valid) continue;
       const bool row_ok = lt < t.ntok;
       const int prow = row_ok ? t.pos0 + lt : -1;
-      float m_ref = -INFINITY, l_sum = 0.f;
+      float m_ref = -INFINITY, l_part = 0.f;
       for (int j = 0; j < t.n_kv; ++j) {
         const long long it = kv_base + j;
         const int b = (int)(it & 1);
@@ -519,52 +548,74 @@ __global__ void __launch_bounds__(PrefillTcTraits<D, BS, G>::kThreads, 1)
           break;
         }
         tc::fence_after();
-        // ---- weights in base 2 against the row's reference maximum, and their two 16-bit
-        // terms.  S is read 32 columns at a time, the next load in flight while the current
-        // columns are processed; every lane of the warp takes part in the loads. ----
-        const int c_lim = prow - j * Tr::kKv;  // columns 0 .. c_lim are visible to this row
-        const uint32_t s_addr = lane_base + 128 * b;
-        uint32_t hp[64], lp[64];
-        // t = logit * scale_log2 - m_ref for visible columns, -inf elsewhere; returns the row's
-        // largest t and fills hp / lp with 2^t (when exps) and the sum of the weights in l_t
+        uint32_t sr[Tr::kCols];
+        tc::ld32x32(lane_base + Tr::kKv * b + Tr::kCols * half, sr);
+        tc::fence_before();
+        mbar_arrive(s_free + b);
+        // P buffer b was last read by O += P V two kv tiles ago
+        if (it >= 2 && !__all_sync(FULL_MASK, wait(pv_done + b, (uint32_t)(((it >> 1) - 1) & 1)))) {
+          ok = false;
+          break;
+        }
+        const int c_lim = prow - j * Tr::kKv - Tr::kCols * half;  // this thread's visible columns
+        const uint32_t ph = p_s + 2 * b * Tr::kPBytes + p_row, pl = ph + Tr::kPBytes;
+        // t = logit * scale_log2 + nm on the visible columns (-inf elsewhere); returns the
+        // largest t; with exps writes 2^t as two 16-bit terms to P and their sum to l_t
         auto pass = [&](float nm, bool exps, float &l_t) -> float {
           float tmax = -INFINITY;
           l_t = 0.f;
-          auto chunk = [&](const uint32_t(&r)[32], int q) {
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              const int c0 = 32 * q + 2 * i;
-              const float t0 = c0 <= c_lim ? fmaf(__uint_as_float(r[2 * i]), a.scale_log2, nm) : -INFINITY;
-              const float t1 = c0 + 1 <= c_lim ? fmaf(__uint_as_float(r[2 * i + 1]), a.scale_log2, nm) : -INFINITY;
+          for (int c = 0; c < Tr::kCols / 8; ++c) {
+            uint32_t hw[4], lw[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const int c0 = 8 * c + 2 * i;
+              const float t0 = c0 <= c_lim ? fmaf(__uint_as_float(sr[c0]), a.scale_log2, nm) : -INFINITY;
+              const float t1 = c0 + 1 <= c_lim ? fmaf(__uint_as_float(sr[c0 + 1]), a.scale_log2, nm) : -INFINITY;
               tmax = fmaxf(tmax, fmaxf(t0, t1));
               if (exps) {
                 const float p0 = fast_exp2(t0), p1 = fast_exp2(t1);
                 l_t += p0 + p1;
-                split2<kBf16>(p0, p1, hp[16 * q + i], lp[16 * q + i]);
+                split2<kBf16>(p0, p1, hw[i], lw[i]);
               }
             }
-          };
-          // the whole row in one load: under the MMAs' own tensor-memory traffic, one long
-          // load costs less than four shorter ones in a chain
-          __syncwarp();
-          uint32_t sr[128];
-          tc::ld32x128(s_addr, sr);
-#pragma unroll
-          for (int q = 0; q < 4; ++q) chunk(*reinterpret_cast<const uint32_t(*)[32]>(sr + 32 * q), q);
+            if (exps) {
+              const uint32_t off = (((Tr::kCols / 8) * half + c) ^ (r & 7)) << 4;
+              asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(ph + off), "r"(hw[0]),
+                           "r"(hw[1]), "r"(hw[2]), "r"(hw[3])
+                           : "memory");
+              asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(pl + off), "r"(lw[0]),
+                           "r"(lw[1]), "r"(lw[2]), "r"(lw[3])
+                           : "memory");
+            }
+          }
           return tmax;
+        };
+        // the row's largest t over both halves
+        auto row_max = [&](float mine_t, float &both) -> bool {
+          float other;
+          const bool got = swap_with_other_half(mine_t, other);
+          both = fmaxf(mine_t, other);
+          return got;
         };
         float l_t, alpha = 1.f;
         bool rescale = false;
         if (j == 0) {
           // first kv tile: the maximum first, then the weights
-          const float mx = pass(0.f, false, l_t);
-          m_ref = mx;
+          if (!row_max(pass(0.f, false, l_t), m_ref)) {
+            ok = false;
+            break;
+          }
           pass(m_ref == -INFINITY ? 0.f : -m_ref, true, l_t);
-          l_sum = l_t;
+          l_part = l_t;
         } else {
           // later tiles: weights against the current reference; a row whose logits pass it by
-          // more than 2^8 moves its reference and takes the pass again
-          const float tmax = pass(m_ref == -INFINITY ? 0.f : -m_ref, true, l_t);
+          // more than 2^8 moves its reference (both halves alike) and takes the pass again
+          float tmax;
+          if (!row_max(pass(m_ref == -INFINITY ? 0.f : -m_ref, true, l_t), tmax)) {
+            ok = false;
+            break;
+          }
           const bool move = tmax > 8.f;
           if (__any_sync(FULL_MASK, move)) {
             if (move) {
@@ -574,36 +625,37 @@ __global__ void __launch_bounds__(PrefillTcTraits<D, BS, G>::kThreads, 1)
             }
             pass(m_ref == -INFINITY ? 0.f : -m_ref, true, l_t);
           }
-          l_sum = l_sum * alpha + l_t;
+          l_part = l_part * alpha + l_t;
         }
-        tc::fence_before();
-        mbar_arrive(s_free + b);
-        // ---- O += P V of the previous kv tile must be done before P and O are touched ----
-        if (j > 0 && !__all_sync(FULL_MASK, wait(o_done, (uint32_t)((it - 1) & 1)))) {
-          ok = false;
-          break;
-        }
-        if (__any_sync(FULL_MASK, rescale)) {
+        // O of rows whose reference moved is rescaled (by the first half's warps) once the
+        // previous O += P V is done
+        if (half == 0 && __any_sync(FULL_MASK, rescale)) {
+          const long long pit = it - 1;
+          if (!__all_sync(FULL_MASK, wait(pv_done + (int)(pit & 1), (uint32_t)((pit >> 1) & 1)))) {
+            ok = false;
+            break;
+          }
           tc::fence_after();
           const float f = rescale ? alpha : 1.f;
 #pragma unroll
           for (int c = 0; c < D / 32; ++c) {
             uint32_t o[32];
-            tc::ld32x32(lane_base + 256 + 32 * c, o);
+            tc::ld32x32(lane_base + 128 + 32 * c, o);
 #pragma unroll
             for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * f);
-            tc::st32x32(lane_base + 256 + 32 * c, o);
+            tc::st32x32(lane_base + 128 + 32 * c, o);
           }
         }
-        if (j == t.n_kv - 1 && (j + 1) * Tr::kKv > t.L) {
+        if (half == 0 && j == t.n_kv - 1 && (j + 1) * Tr::kKv > t.L) {
           // positions past the context may hold anything (NaN included) and would meet a zero
           // weight in the MMA: zero the value rows there once their copy has landed
-          if (!__all_sync(FULL_MASK, wait(v_full + b, (uint32_t)((it >> 1) & 1)))) {
+          const int vs = (int)(it % Tr::kStages);
+          if (!__all_sync(FULL_MASK, wait(v_full + vs, (uint32_t)((it / Tr::kStages) & 1)))) {
             ok = false;
             break;
           }
-          if (r >= t.L - j * Tr::kKv) {
-            const uint32_t vrow = v_s + b * Tr::kKvBytes + (r >> 3) * Tr::kGroup + (r & 7) * 128;
+          if (r < Tr::kKv && r >= t.L - j * Tr::kKv) {
+            const uint32_t vrow = v_s + vs * Tr::kKvBytes + (r >> 3) * Tr::kGroup + (r & 7) * 128;
 #pragma unroll
             for (int h = 0; h < Tr::kSpans; ++h)
 #pragma unroll
@@ -612,39 +664,34 @@ __global__ void __launch_bounds__(PrefillTcTraits<D, BS, G>::kThreads, 1)
                              "r"(0u)
                              : "memory");
           }
-          fence_proxy_async_smem();
-        }
-        // ---- P (hi, lo) into shared memory, swizzled like the operand tiles ----
-#pragma unroll
-        for (int c = 0; c < 16; ++c) {
-          const uint32_t off = p_row + (c >> 3) * 1024 + (((c & 7) ^ (r & 7)) << 4);
-          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(ph_s + off), "r"(hp[4 * c]),
-                       "r"(hp[4 * c + 1]), "r"(hp[4 * c + 2]), "r"(hp[4 * c + 3])
-                       : "memory");
-          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(pl_s + off), "r"(lp[4 * c]),
-                       "r"(lp[4 * c + 1]), "r"(lp[4 * c + 2]), "r"(lp[4 * c + 3])
-                       : "memory");
         }
         fence_proxy_async_smem();
         tc::fence_before();
-        mbar_arrive(p_ready);
+        mbar_arrive(p_ready + b);
       }
       if (!ok) break;
-      // ---- epilogue: O / l of the valid rows ----
+      // ---- epilogue: the halves add their sums; each stores half of the row of O / l ----
+      float l_other;
+      if (!swap_with_other_half(l_part, l_other)) {
+        ok = false;
+        break;
+      }
+      const float l_row = l_part + l_other;
       const long long last = kv_base + t.n_kv - 1;
-      if (!__all_sync(FULL_MASK, wait(o_done, (uint32_t)(last & 1)))) {
+      if (!__all_sync(FULL_MASK, wait(pv_done + (int)(last & 1), (uint32_t)((last >> 1) & 1)))) {
         ok = false;
         break;
       }
       tc::fence_after();
-      const float inv = row_ok ? 1.f / l_sum : 0.f;
+      const float inv = row_ok ? 1.f / l_row : 0.f;
       const long long ob = (long long)(t.q0 + t.tok0 + (row_ok ? lt : 0)) * a.out_t +
                            (long long)(t.kvh * G + hh) * a.out_h;
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
+      for (int c2 = 0; c2 < D / 64; ++c2) {
+        const int c = (D / 64) * half + c2;  // 32-column chunk of O
         uint32_t o[32];
         __syncwarp();
-        tc::ld32x32(lane_base + 256 + 32 * c, o);
+        tc::ld32x32(lane_base + 128 + 32 * c, o);
         if (!row_ok) {
         } else if (a.out_dtype == PA_F32) {
           float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(a.out) + ob + 32 * c);
@@ -680,7 +727,7 @@ __global__ void __launch_bounds__(PrefillTcTraits<D, BS, G>::kThreads, 1)
   // ---- teardown: every role done, tensor memory released by the warp that allocated it ----
   tc::fence_before();
   __syncthreads();
-  if (wid == 5) {
+  if (wid == Tr::kMmaWarp) {
     tc::fence_after();
     tc::dealloc(tmem, Tr::kTmemCols);
   }
