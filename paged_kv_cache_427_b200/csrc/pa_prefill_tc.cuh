@@ -11,10 +11,11 @@
 //
 // A tile is 128 query rows of one (sequence, kv head): 128 / G new tokens times the G query
 // heads that read that kv head (head fastest), one row per tensor-memory lane.  The context is
-// walked in kv tiles of 64 positions.  One persistent CTA per SM, ten warps:
+// walked in kv tiles of 64 positions.  One persistent CTA per SM, eleven warps:
 //   * warp 8 streams the tile's query rows (one 4-D box, loaded as soon as the previous tile's
-//     last S = QK^T is done, so it overlaps that tile's end) and the key and value tiles through
-//     three-slot rings by TMA: one box per (block, kv head) tile of the paged cache, 128-byte
+//     last S = QK^T is done, so it overlaps that tile's end) and the key tiles, warp 10 the
+//     value tiles (so keys run ahead of the values, which free later), through three-slot rings
+//     by TMA: one box per (block, kv head) tile of the paged cache, 128-byte
 //     swizzle, in 8-row groups placed one after another, which is the operand layout of the
 //     MMAs; the lanes issue the boxes of a kv tile together;
 //   * warp 9 (one lane) issues the MMAs: S = Q K^T (M = 128 rows, N = 64 positions, K = head
@@ -52,9 +53,10 @@ template <int D, int BS, int G>
 struct PrefillTcTraits {
   static constexpr int kSoftmaxWarps = 8;
   static constexpr int kSoftmaxThreads = kSoftmaxWarps * 32;
-  static constexpr int kProducerWarp = 8;
+  static constexpr int kProducerWarp = 8;  // query rows and key tiles
   static constexpr int kMmaWarp = 9;
-  static constexpr int kThreads = 320;
+  static constexpr int kValueWarp = 10;    // value tiles
+  static constexpr int kThreads = 352;
   static constexpr int kRows = 128;             // query rows of a tile (MMA M)
   static constexpr int kTokens = kRows / G;     // new tokens of a tile
   static constexpr int kKv = 64;                // context positions of a kv tile
@@ -342,8 +344,9 @@ __global__ void __launch_bounds__(PrefillTcTraits<D, BS, G>::kThreads, 1)
   const uint32_t v_s = smem_u32(smem + Tr::kVOff);
   const uint32_t p_s = smem_u32(smem + Tr::kPOff);  // P buffer b: hi at + 2b kPBytes, lo after it
 
-  if (wid == Tr::kProducerWarp) {
-    // ================= producer: query rows, key and value tiles by TMA =================
+  if (wid == Tr::kProducerWarp || wid == Tr::kValueWarp) {
+    // ======= producers: query rows and key tiles (warp 8), value tiles (warp 10), by TMA =======
+    const int which = wid == Tr::kValueWarp ? 1 : 0;
     long long kv_base = 0, qt = 0;
     long long k_issued = 0, v_issued = 0;
     bool ok = true;
@@ -353,7 +356,7 @@ __global__ void __launch_bounds__(PrefillTcTraits<D, BS, G>::kThreads, 1)
         if (lane == 0 && t.tau == 0 && t.kvh == 0) set_error(a.err, PA_DEVERR_CONTEXT_LEN);
         continue;
       }
-      {
+      if (which == 0) {
         // the tile's query rows: tokens q0 + tok0 .. + 128/G of heads kvh*G .. + G (rows past
         // the tensor read as zeros, rows of the next sequence are computed and dropped), once
         // the previous tile's S = QK^T are all done
@@ -397,7 +400,7 @@ __global__ void __launch_bounds__(PrefillTcTraits<D, BS, G>::kThreads, 1)
         const int pend = min(p0 + Tr::kKv, t.L);
         const int nblk = (pend - p0 + BS - 1) / BS;
         const uint32_t bytes = (uint32_t)(a.grouped_maps ? nblk * (BS / 8) : (pend - p0 + 7) / 8) * Tr::kBoxBytes;
-        for (int which = 0; which < 2; ++which) {
+        {
           uint64_t *full = which ? v_full + b : k_full + b;
           uint64_t *empty = which ? v_empty + b : k_empty + b;
           bool w_ok = true;
@@ -407,7 +410,7 @@ __global__ void __launch_bounds__(PrefillTcTraits<D, BS, G>::kThreads, 1)
           }
           if (__shfl_sync(FULL_MASK, w_ok ? 1 : 0, 0) == 0) {
             ok = false;
-            break;
+            continue;
           }
           const uint32_t dst = (which ? v_s : k_s) + b * Tr::kKvBytes;
           const CUtensorMap *map = which ? &maps.v : &maps.k;
