@@ -27,11 +27,13 @@
 //     causally (which also hides positions past the context), keeps the online softmax of its
 //     half of the row in base 2 against a reference maximum the two halves share (exchanged
 //     through shared memory; moved only when a logit passes it by 2^8, when O is rescaled in
-//     tensor memory) and writes its part of P to one of two P buffers in shared memory; at the
-//     end of the tile the halves add their row sums and each stores half of the row of O / l.
-// The MMA warp issues S of kv tile j + 1 before O += P V of tile j, and P has two buffers, so
-// the tensor cores compute the next scores and the previous products while the softmax warps
-// work on the current scores.  Barriers between the roles are mbarriers (copies: transaction
+//     tensor memory) and writes its part of P into tensor memory over the S it came from, where
+//     the MMA reads it as the A operand; at the end of the tile the halves add their row sums
+//     and each stores half of the row of O / l.
+// The MMA warp issues S of kv tile j + 1 before O += P V of tile j, and S / P has two buffers,
+// so the tensor cores compute the next scores and the previous products while the softmax warps
+// work on the current scores.  Keeping Q, K, V as the only shared-memory operands (and P out of
+// shared memory) leaves the shared-memory bandwidth to the MMAs' operand reads.  Barriers between the roles are mbarriers (copies: transaction
 // bytes; MMAs: tcgen05.commit; threads: arrival counts); every wait is bounded and a timeout sets
 // an error bit and winds the CTA down.
 //
@@ -65,14 +67,12 @@ struct PrefillTcTraits {
   static constexpr int kGroup = kSpans * 1024;  // bytes between 8-row groups of K, V tiles
   static constexpr int kQBytes = kRows * D * 2; // span-major: 128 rows of a span, then the next
   static constexpr int kKvBytes = kKv * D * 2;
-  static constexpr int kPBytes = kRows * kKv * 2;  // one term of P: 8-row groups of 1 KB
   static constexpr int kBoxBytes = 8 * D * 2;      // 8 positions, both spans
   static constexpr int kQOff = 0;
   static constexpr int kKOff = kQOff + kQBytes;
   static constexpr int kStages = 3;             // key and value rings
   static constexpr int kVOff = kKOff + kStages * kKvBytes;
-  static constexpr int kPOff = kVOff + kStages * kKvBytes;  // two buffers of (hi, lo)
-  static constexpr int kBarOff = kPOff + 4 * kPBytes;
+  static constexpr int kBarOff = kVOff + kStages * kKvBytes;
   static constexpr int kNumBars = 28;
   static constexpr int kInfoOff = kBarOff + kNumBars * 8;  // [tmem base, abort, tile count, rounds]
   static constexpr int kXchOff = kInfoOff + 32;            // float [2 parities][2 halves][128 rows]
@@ -83,7 +83,10 @@ struct PrefillTcTraits {
   // rings before the first copy
   static constexpr int kMaxBins = 2048;  // costs 0 .. 2047 (16-position steps)
   static constexpr int kMaxList = 4096;  // (sequence, tile) pairs
-  static constexpr int kTmemCols = 256;  // S0 [0, 64), S1 [64, 128), O [128, 128 + D)
+  // tensor memory: S0 [0, 64), S1 [64, 128), O [128, 128 + D).  P of a kv tile replaces its S:
+  // hi terms of positions 0..63 in the buffer's columns 0..31, lo terms in 32..63 (two 16-bit
+  // values per column, the A operand of O += P V)
+  static constexpr int kTmemCols = 256;
   static_assert(D == 64 || D == 128, "head_dim 64 or 128");
   static_assert(G == 1 || G == 2 || G == 4 || G == 8, "1, 2, 4 or 8 query heads per kv head");
   static_assert(BS % 8 == 0 && kKv % BS == 0, "block size a multiple of the 8-position box");
@@ -342,7 +345,6 @@ __global__ void __launch_bounds__(PrefillTcTraits<D, BS, G>::kThreads, 1)
   const uint32_t q_s = smem_u32(smem + Tr::kQOff);
   const uint32_t k_s = smem_u32(smem + Tr::kKOff);
   const uint32_t v_s = smem_u32(smem + Tr::kVOff);
-  const uint32_t p_s = smem_u32(smem + Tr::kPOff);  // P buffer b: hi at + 2b kPBytes, lo after it
 
   if (wid == Tr::kProducerWarp || wid == Tr::kValueWarp) {
     // ======= producers: query rows and key tiles (warp 8), value tiles (warp 10), by TMA =======
@@ -462,12 +464,12 @@ __global__ void __launch_bounds__(PrefillTcTraits<D, BS, G>::kThreads, 1)
         return false;
       tc::fence_after();
       const uint32_t vb = v_s + vs * Tr::kKvBytes;
-      const uint32_t ph = p_s + 2 * b * Tr::kPBytes, pl = ph + Tr::kPBytes;
+      const uint32_t pt = tmem + Tr::kKv * b;  // P over S buffer b
 #pragma unroll
       for (int kt = 0; kt < Tr::kKv / 16; ++kt) {
         const uint64_t vd = tc::smem_desc(vb + kt * 2 * Tr::kGroup, 1024, Tr::kGroup);
-        tc::mma(tmem + 128, tc::smem_desc(ph + kt * 32, 16, 1024), vd, kIdO, (j > 0 || kt > 0) ? 1u : 0u);
-        tc::mma(tmem + 128, tc::smem_desc(pl + kt * 32, 16, 1024), vd, kIdO, 1u);
+        tc::mma_ts(tmem + 128, pt + 8 * kt, vd, kIdO, (j > 0 || kt > 0) ? 1u : 0u);
+        tc::mma_ts(tmem + 128, pt + 32 + 8 * kt, vd, kIdO, 1u);
       }
       tc::commit(pv_done + b);
       tc::commit(v_empty + vs);
@@ -521,7 +523,6 @@ __global__ void __launch_bounds__(PrefillTcTraits<D, BS, G>::kThreads, 1)
     const int r = 32 * quarter + lane;  // row = tensor-memory lane
     const int lt = r / G, hh = r % G;
     const uint32_t lane_base = tc::taddr(tmem, 32 * quarter, 0);
-    const uint32_t p_row = (r >> 3) * 1024 + (r & 7) * 128;
     float *xch = reinterpret_cast<float *>(smem + Tr::kXchOff);  // [parity][half][row]
     // The two threads of a row swap a value through shared memory; the two warps of a row
     // quarter meet at their own mbarrier (bounded wait), exchanges alternate between two slots.
@@ -555,41 +556,23 @@ __global__ void __launch_bounds__(PrefillTcTraits<D, BS, G>::kThreads, 1)
         tc::ld32x32(lane_base + Tr::kKv * b + Tr::kCols * half, sr);
         tc::fence_before();
         mbar_arrive(s_free + b);
-        // P buffer b was last read by O += P V two kv tiles ago
-        if (it >= 2 && !__all_sync(FULL_MASK, wait(pv_done + b, (uint32_t)(((it >> 1) - 1) & 1)))) {
-          ok = false;
-          break;
-        }
         const int c_lim = prow - j * Tr::kKv - Tr::kCols * half;  // this thread's visible columns
-        const uint32_t ph = p_s + 2 * b * Tr::kPBytes + p_row, pl = ph + Tr::kPBytes;
         // t = logit * scale_log2 + nm on the visible columns (-inf elsewhere); returns the
-        // largest t; with exps writes 2^t as two 16-bit terms to P and their sum to l_t
+        // largest t; with exps leaves 2^t as two 16-bit terms in hw / lw, their sum in l_t
+        uint32_t hw[Tr::kCols / 2], lw[Tr::kCols / 2];
         auto pass = [&](float nm, bool exps, float &l_t) -> float {
           float tmax = -INFINITY;
           l_t = 0.f;
 #pragma unroll
-          for (int c = 0; c < Tr::kCols / 8; ++c) {
-            uint32_t hw[4], lw[4];
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              const int c0 = 8 * c + 2 * i;
-              const float t0 = c0 <= c_lim ? fmaf(__uint_as_float(sr[c0]), a.scale_log2, nm) : -INFINITY;
-              const float t1 = c0 + 1 <= c_lim ? fmaf(__uint_as_float(sr[c0 + 1]), a.scale_log2, nm) : -INFINITY;
-              tmax = fmaxf(tmax, fmaxf(t0, t1));
-              if (exps) {
-                const float p0 = fast_exp2(t0), p1 = fast_exp2(t1);
-                l_t += p0 + p1;
-                split2<kBf16>(p0, p1, hw[i], lw[i]);
-              }
-            }
+          for (int i = 0; i < Tr::kCols / 2; ++i) {
+            const int c0 = 2 * i;
+            const float t0 = c0 <= c_lim ? fmaf(__uint_as_float(sr[c0]), a.scale_log2, nm) : -INFINITY;
+            const float t1 = c0 + 1 <= c_lim ? fmaf(__uint_as_float(sr[c0 + 1]), a.scale_log2, nm) : -INFINITY;
+            tmax = fmaxf(tmax, fmaxf(t0, t1));
             if (exps) {
-              const uint32_t off = (((Tr::kCols / 8) * half + c) ^ (r & 7)) << 4;
-              asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(ph + off), "r"(hw[0]),
-                           "r"(hw[1]), "r"(hw[2]), "r"(hw[3])
-                           : "memory");
-              asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(pl + off), "r"(lw[0]),
-                           "r"(lw[1]), "r"(lw[2]), "r"(lw[3])
-                           : "memory");
+              const float p0 = fast_exp2(t0), p1 = fast_exp2(t1);
+              l_t += p0 + p1;
+              split2<kBf16>(p0, p1, hw[i], lw[i]);
             }
           }
           return tmax;
@@ -630,6 +613,9 @@ __global__ void __launch_bounds__(PrefillTcTraits<D, BS, G>::kThreads, 1)
           }
           l_part = l_part * alpha + l_t;
         }
+        // P over S in tensor memory (both halves have read their S: they met at the exchange)
+        tc::st32x16x2(lane_base + Tr::kKv * b + (Tr::kCols / 2) * half, hw,
+                      lane_base + Tr::kKv * b + Tr::kKv / 2 + (Tr::kCols / 2) * half, lw);
         // O of rows whose reference moved is rescaled (by the first half's warps) once the
         // previous O += P V is done
         if (half == 0 && __any_sync(FULL_MASK, rescale)) {
@@ -667,8 +653,8 @@ __global__ void __launch_bounds__(PrefillTcTraits<D, BS, G>::kThreads, 1)
                              "r"(0u)
                              : "memory");
           }
+          fence_proxy_async_smem();
         }
-        fence_proxy_async_smem();
         tc::fence_before();
         mbar_arrive(p_ready + b);
       }

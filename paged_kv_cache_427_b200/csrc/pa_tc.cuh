@@ -52,6 +52,18 @@ __device__ __forceinline__ void mma(uint32_t d_tmem, uint64_t a_desc, uint64_t b
       : "memory");
 }
 
+// The same with A in tensor memory (lane i = row i, two 16-bit elements of the contraction per
+// 32-bit column, the lower k in the low half), B described in shared memory.
+__device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                       uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}"
+      ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 // One arrival on `bar` once every tcgen05 operation this thread issued before has completed.
 __device__ __forceinline__ void commit(uint64_t *bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
@@ -118,6 +130,28 @@ __device__ __forceinline__ void st32x32(uint32_t taddr, const uint32_t (&r)[32])
       : "memory");
 }
 
+
+// Two stores of 16 consecutive 32-bit columns each (a at taddr0, b at taddr1), waited for.
+__device__ __forceinline__ void st32x16x2(uint32_t taddr0, const uint32_t (&a)[16], uint32_t taddr1,
+                                         const uint32_t (&b)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {"
+      "%2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, %17"
+      "};\n\t"
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%1], {"
+      "%18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32, %33"
+      "};\n\t"
+      "tcgen05.wait::st.sync.aligned;"
+      :
+      : "r"(taddr0), "r"(taddr1),
+        "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(a[4]), "r"(a[5]), "r"(a[6]), "r"(a[7]),
+        "r"(a[8]), "r"(a[9]), "r"(a[10]), "r"(a[11]), "r"(a[12]), "r"(a[13]), "r"(a[14]),
+        "r"(a[15]),
+        "r"(b[0]), "r"(b[1]), "r"(b[2]), "r"(b[3]), "r"(b[4]), "r"(b[5]), "r"(b[6]), "r"(b[7]),
+        "r"(b[8]), "r"(b[9]), "r"(b[10]), "r"(b[11]), "r"(b[12]), "r"(b[13]), "r"(b[14]),
+        "r"(b[15])
+      : "memory");
+}
 
 }  // namespace tc
 }  // namespace pa
