@@ -11,31 +11,31 @@
 //
 // A tile is 128 query rows of one (sequence, kv head): 128 / G new tokens times the G query
 // heads that read that kv head (head fastest), one row per tensor-memory lane.  The context is
-// walked in kv tiles of 64 positions.  One persistent CTA per SM, eleven warps:
+// walked in kv tiles of 128 positions.  One persistent CTA per SM, eleven warps:
 //   * warp 8 streams the tile's query rows (one 4-D box, loaded as soon as the previous tile's
 //     last S = QK^T is done, so it overlaps that tile's end) and the key tiles, warp 10 the
-//     value tiles (so keys run ahead of the values, which free later), through three-slot rings
-//     by TMA: one box per (block, kv head) tile of the paged cache, 128-byte
-//     swizzle, in 8-row groups placed one after another, which is the operand layout of the
-//     MMAs; the lanes issue the boxes of a kv tile together;
-//   * warp 9 (one lane) issues the MMAs: S = Q K^T (M = 128 rows, N = 64 positions, K = head
-//     dim) into one of two S buffers in tensor memory, and O += P V (N = head dim, K = 64
+//     value tiles (so keys run ahead of the values, which free later), through two-slot rings
+//     by TMA: one box per (block, kv head) tile of the paged cache, 128-byte swizzle, in 8-row
+//     groups placed one after another, which is the operand layout of the MMAs; the lanes issue
+//     the boxes of a kv tile together;
+//   * warp 9 (one lane) issues the MMAs: S = Q K^T (M = 128 rows, N = 128 positions, K = head
+//     dim) into one of two S buffers in tensor memory, and O += P V (N = head dim, K = 128
 //     positions) into the O accumulator, P split into two 16-bit terms (hi + lo) as in the
 //     decode kernels so the weights keep about 16 significant bits;
 //   * warps 0-7 run the softmax, two threads per row: warp w reads tensor-memory lanes
-//     32 (w % 4) .. + 31 and columns 32 (w / 4) .. + 31 of S.  Each thread masks its columns
-//     causally (which also hides positions past the context), keeps the online softmax of its
-//     half of the row in base 2 against a reference maximum the two halves share (exchanged
-//     through shared memory; moved only when a logit passes it by 2^8, when O is rescaled in
-//     tensor memory) and writes its part of P into tensor memory over the S it came from, where
-//     the MMA reads it as the A operand; at the end of the tile the halves add their row sums
-//     and each stores half of the row of O / l.
+//     32 (w % 4) .. + 31 and the half w / 4 of the kv tile's columns of S.  Each thread masks
+//     its columns causally (which also hides positions past the context), keeps the online
+//     softmax of its half of the row in base 2 against a reference maximum the two halves
+//     share (exchanged through shared memory; moved only when a logit passes it by 2^8, when O
+//     is rescaled in tensor memory) and writes its part of P into tensor memory over its own S
+//     columns, where the MMA reads it as the A operand; at the end of the tile the halves add
+//     their row sums and each stores half of the row of O / l.
 // The MMA warp issues S of kv tile j + 1 before O += P V of tile j, and S / P has two buffers,
 // so the tensor cores compute the next scores and the previous products while the softmax warps
-// work on the current scores.  Keeping Q, K, V as the only shared-memory operands (and P out of
-// shared memory) leaves the shared-memory bandwidth to the MMAs' operand reads.  Barriers between the roles are mbarriers (copies: transaction
-// bytes; MMAs: tcgen05.commit; threads: arrival counts); every wait is bounded and a timeout sets
-// an error bit and winds the CTA down.
+// work on the current scores.  Q, K and V are the only shared-memory operands, which leaves the
+// shared-memory bandwidth to the MMAs' operand reads.  Barriers between the roles are mbarriers
+// (copies: transaction bytes; MMAs: tcgen05.commit; threads: arrival counts); every wait is
+// bounded and a timeout sets an error bit and winds the CTA down.
 //
 // Tiles differ in cost (a tile's causal prefix), so they are spread longest first: every CTA
 // builds the same list of (sequence, tile) pairs sorted by cost (a histogram of costs in shared
@@ -61,7 +61,7 @@ struct PrefillTcTraits {
   static constexpr int kThreads = 352;
   static constexpr int kRows = 128;             // query rows of a tile (MMA M)
   static constexpr int kTokens = kRows / G;     // new tokens of a tile
-  static constexpr int kKv = 64;                // context positions of a kv tile
+  static constexpr int kKv = 128;               // context positions of a kv tile
   static constexpr int kCols = kKv / 2;         // S columns per softmax thread
   static constexpr int kSpans = D / 64;
   static constexpr int kGroup = kSpans * 1024;  // bytes between 8-row groups of K, V tiles
@@ -70,7 +70,7 @@ struct PrefillTcTraits {
   static constexpr int kBoxBytes = 8 * D * 2;      // 8 positions, both spans
   static constexpr int kQOff = 0;
   static constexpr int kKOff = kQOff + kQBytes;
-  static constexpr int kStages = 3;             // key and value rings
+  static constexpr int kStages = 2;             // key and value rings
   static constexpr int kVOff = kKOff + kStages * kKvBytes;
   static constexpr int kBarOff = kVOff + kStages * kKvBytes;
   static constexpr int kNumBars = 28;
@@ -83,10 +83,11 @@ struct PrefillTcTraits {
   // rings before the first copy
   static constexpr int kMaxBins = 2048;  // costs 0 .. 2047 (16-position steps)
   static constexpr int kMaxList = 4096;  // (sequence, tile) pairs
-  // tensor memory: S0 [0, 64), S1 [64, 128), O [128, 128 + D).  P of a kv tile replaces its S:
-  // hi terms of positions 0..63 in the buffer's columns 0..31, lo terms in 32..63 (two 16-bit
-  // values per column, the A operand of O += P V)
-  static constexpr int kTmemCols = 256;
+  // tensor memory: S0 [0, kKv), S1 [kKv, 2 kKv), O [2 kKv, 2 kKv + D).  P of a kv tile replaces
+  // its S: each softmax half's kCols columns hold the hi terms of its positions (two 16-bit
+  // values per column, the A operand of O += P V), then the lo terms
+  static constexpr int kOCol = 2 * kKv;
+  static constexpr int kTmemCols = kOCol + D <= 256 ? 256 : 512;
   static_assert(D == 64 || D == 128, "head_dim 64 or 128");
   static_assert(G == 1 || G == 2 || G == 4 || G == 8, "1, 2, 4 or 8 query heads per kv head");
   static_assert(BS % 8 == 0 && kKv % BS == 0, "block size a multiple of the 8-position box");
@@ -464,12 +465,15 @@ __global__ void __launch_bounds__(PrefillTcTraits<D, BS, G>::kThreads, 1)
         return false;
       tc::fence_after();
       const uint32_t vb = v_s + vs * Tr::kKvBytes;
-      const uint32_t pt = tmem + Tr::kKv * b;  // P over S buffer b
 #pragma unroll
       for (int kt = 0; kt < Tr::kKv / 16; ++kt) {
         const uint64_t vd = tc::smem_desc(vb + kt * 2 * Tr::kGroup, 1024, Tr::kGroup);
-        tc::mma_ts(tmem + 128, pt + 8 * kt, vd, kIdO, (j > 0 || kt > 0) ? 1u : 0u);
-        tc::mma_ts(tmem + 128, pt + 32 + 8 * kt, vd, kIdO, 1u);
+        // positions 16 kt .. + 15 belong to the softmax half h, offset o within it: their hi
+        // terms sit at column kCols h + o / 2 of S buffer b, the lo terms kCols / 2 further
+        const int h = (16 * kt) / Tr::kCols, o = 16 * kt - h * Tr::kCols;
+        const uint32_t pc = tmem + Tr::kKv * b + Tr::kCols * h + o / 2;
+        tc::mma_ts(tmem + Tr::kOCol, pc, vd, kIdO, (j > 0 || kt > 0) ? 1u : 0u);
+        tc::mma_ts(tmem + Tr::kOCol, pc + Tr::kCols / 2, vd, kIdO, 1u);
       }
       tc::commit(pv_done + b);
       tc::commit(v_empty + vs);
@@ -552,10 +556,9 @@ __global__ void __launch_bounds__(PrefillTcTraits<D, BS, G>::kThreads, 1)
           break;
         }
         tc::fence_after();
-        uint32_t sr[Tr::kCols];
-        tc::ld32x32(lane_base + Tr::kKv * b + Tr::kCols * half, sr);
-        tc::fence_before();
-        mbar_arrive(s_free + b);
+        // this thread's S columns and, later, its P: the hi terms of its kCols positions in the
+        // first kCols / 2 of its columns, the lo terms in the rest
+        const uint32_t my_cols = lane_base + Tr::kKv * b + Tr::kCols * half;
         const int c_lim = prow - j * Tr::kKv - Tr::kCols * half;  // this thread's visible columns
         // t = logit * scale_log2 + nm on the visible columns (-inf elsewhere); returns the
         // largest t; with exps leaves 2^t as two 16-bit terms in hw / lw, their sum in l_t
@@ -564,15 +567,21 @@ __global__ void __launch_bounds__(PrefillTcTraits<D, BS, G>::kThreads, 1)
           float tmax = -INFINITY;
           l_t = 0.f;
 #pragma unroll
-          for (int i = 0; i < Tr::kCols / 2; ++i) {
-            const int c0 = 2 * i;
-            const float t0 = c0 <= c_lim ? fmaf(__uint_as_float(sr[c0]), a.scale_log2, nm) : -INFINITY;
-            const float t1 = c0 + 1 <= c_lim ? fmaf(__uint_as_float(sr[c0 + 1]), a.scale_log2, nm) : -INFINITY;
-            tmax = fmaxf(tmax, fmaxf(t0, t1));
-            if (exps) {
-              const float p0 = fast_exp2(t0), p1 = fast_exp2(t1);
-              l_t += p0 + p1;
-              split2<kBf16>(p0, p1, hw[i], lw[i]);
+          for (int q = 0; q < Tr::kCols / 32; ++q) {
+            uint32_t sr[32];
+            __syncwarp();
+            tc::ld32x32(my_cols + 32 * q, sr);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const int c0 = 32 * q + 2 * i;
+              const float t0 = c0 <= c_lim ? fmaf(__uint_as_float(sr[2 * i]), a.scale_log2, nm) : -INFINITY;
+              const float t1 = c0 + 1 <= c_lim ? fmaf(__uint_as_float(sr[2 * i + 1]), a.scale_log2, nm) : -INFINITY;
+              tmax = fmaxf(tmax, fmaxf(t0, t1));
+              if (exps) {
+                const float p0 = fast_exp2(t0), p1 = fast_exp2(t1);
+                l_t += p0 + p1;
+                split2<kBf16>(p0, p1, hw[16 * q + i], lw[16 * q + i]);
+              }
             }
           }
           return tmax;
@@ -586,6 +595,12 @@ __global__ void __launch_bounds__(PrefillTcTraits<D, BS, G>::kThreads, 1)
         };
         float l_t, alpha = 1.f;
         bool rescale = false;
+        // S may be released once both passes that can read it are behind: the first tile reads
+        // it twice (maximum, then weights), a later one once, and a second time on a move
+        auto release_s = [&]() {
+          tc::fence_before();
+          mbar_arrive(s_free + b);
+        };
         if (j == 0) {
           // first kv tile: the maximum first, then the weights
           if (!row_max(pass(0.f, false, l_t), m_ref)) {
@@ -613,9 +628,12 @@ __global__ void __launch_bounds__(PrefillTcTraits<D, BS, G>::kThreads, 1)
           }
           l_part = l_part * alpha + l_t;
         }
-        // P over S in tensor memory (both halves have read their S: they met at the exchange)
-        tc::st32x16x2(lane_base + Tr::kKv * b + (Tr::kCols / 2) * half, hw,
-                      lane_base + Tr::kKv * b + Tr::kKv / 2 + (Tr::kCols / 2) * half, lw);
+        // P over this thread's own S columns in tensor memory
+        release_s();
+#pragma unroll
+        for (int g = 0; g < Tr::kCols / 32; ++g)
+          tc::st32x16x2(my_cols + 16 * g, *reinterpret_cast<const uint32_t(*)[16]>(hw + 16 * g),
+                        my_cols + Tr::kCols / 2 + 16 * g, *reinterpret_cast<const uint32_t(*)[16]>(lw + 16 * g));
         // O of rows whose reference moved is rescaled (by the first half's warps) once the
         // previous O += P V is done
         if (half == 0 && __any_sync(FULL_MASK, rescale)) {
@@ -629,10 +647,10 @@ __global__ void __launch_bounds__(PrefillTcTraits<D, BS, G>::kThreads, 1)
 #pragma unroll
           for (int c = 0; c < D / 32; ++c) {
             uint32_t o[32];
-            tc::ld32x32(lane_base + 128 + 32 * c, o);
+            tc::ld32x32(lane_base + Tr::kOCol + 32 * c, o);
 #pragma unroll
             for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * f);
-            tc::st32x32(lane_base + 128 + 32 * c, o);
+            tc::st32x32(lane_base + Tr::kOCol + 32 * c, o);
           }
         }
         if (half == 0 && j == t.n_kv - 1 && (j + 1) * Tr::kKv > t.L) {
@@ -680,7 +698,7 @@ __global__ void __launch_bounds__(PrefillTcTraits<D, BS, G>::kThreads, 1)
         const int c = (D / 64) * half + c2;  // 32-column chunk of O
         uint32_t o[32];
         __syncwarp();
-        tc::ld32x32(lane_base + 128 + 32 * c, o);
+        tc::ld32x32(lane_base + Tr::kOCol + 32 * c, o);
         if (!row_ok) {
         } else if (a.out_dtype == PA_F32) {
           float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(a.out) + ob + 32 * c);
