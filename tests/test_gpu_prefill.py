@@ -74,6 +74,37 @@ def test_prefill_configurations(oracle, dtype, D, bs, hq, hkv):
     assert_no_device_error()
 
 
+def test_prefill_caches_with_padded_blocks(oracle):
+    """Caches whose blocks hold more kv-head slots than the view passed in (a block stride that
+    is not num_kv_heads x the head stride) cannot use the one-box-per-tile view of the cache;
+    the kernel then reads 8-row boxes.  Same results as the contiguous caches."""
+    require_gpu()
+    b = W.build_prefill_batch("pfpad", [300, 77, 16, 1, 200], [300, 13, 16, 1, 64], num_heads=32,
+                              num_kv_heads=8, head_dim=128, block_size=16, dtype="bf16",
+                              seed=W.BASE_SEED + 746)
+    ref, kc, vc = _oracle(oracle, b)
+    st = PrefillStep(b)
+    nb, hkv, bs, d = st.key_cache.shape
+
+    def padded(t):
+        big = torch.full((nb, hkv + 1, bs, d), float("nan"), dtype=t.dtype, device=t.device)
+        big[:, :hkv] = t
+        return big[:, :hkv]
+
+    kpad, vpad = padded(st.key_cache), padded(st.value_cache)
+    assert kpad.stride(0) != hkv * kpad.stride(1)
+    for dt in ("f32", "bf16"):
+        out = torch.full(st.query.shape, float("nan"), dtype=TORCH_DTYPE[dt], device="cuda")
+        pa.pa_prefill(out, st.query, kpad, vpad, st.tables, st.lens, st.qs, b.scale, b.block_size,
+                      b.num_kv_heads)
+        got = to_host(out, dt)
+        if dt == "f32":
+            assert_close(got, ref, "bf16", "prefill padded-block caches")
+        else:
+            assert np.array_equal(got, st.run("bf16")), "padded-block caches change the bf16 output"
+    assert_no_device_error()
+
+
 def _scale_keys_by_position(b, factor):
     """Multiply the key of position t of every sequence by factor(t), in the cache and in the
     new tokens' rows, re-rounded to the storage type."""
