@@ -171,3 +171,94 @@ def test_status_constants_match_header():
         text = f.read()
     for name, value in re.findall(r"\b(PA_ERR_[A-Z_]+)\s*=\s*(-\d+)", text):
         assert getattr(pa, name) == int(value), name
+
+
+def _prefill_args(S=3, T=40, Hq=8, Hkv=2, D=128, bs=16, NB=32, MB=8, dt=pa.PA_BF16, out_dt=None,
+                  q_data=0x10000, qs_len=None):
+    return dict(out=_t([T, Hq, D], out_dt if out_dt is not None else dt),
+                query=_t([T, Hq, D], dt, data=q_data),
+                kc=_t([NB, Hkv, bs, D], dt), vc=_t([NB, Hkv, bs, D], dt),
+                bt=_t([S, MB], pa.PA_I32), cl=_t([S], pa.PA_I32),
+                qs=_t([qs_len if qs_len is not None else S + 1], pa.PA_I32))
+
+
+def _prefill(lib, a, bs=16, hkv=2, scale=0.1):
+    r = ctypes.byref
+    return lib.pa_prefill(r(a["out"]), r(a["query"]), r(a["kc"]), r(a["vc"]), r(a["bt"]), r(a["cl"]),
+                          r(a["qs"]), scale, bs, hkv, None)
+
+
+@pytest.mark.parametrize("case,expect", [
+    (dict(D=96), -4),                        # head_dim not built
+    (dict(bs=64), -4),                       # block_size not built
+    (dict(Hq=24, Hkv=2), -4),                # group of 12 not built
+    (dict(Hq=7, Hkv=2), -2),                 # heads not a multiple of kv heads
+    (dict(dt=pa.PA_F32), -4),                # prefill is built for 16-bit caches
+    (dict(out_dt=pa.PA_F16), -3),            # out neither fp32 nor the cache type
+    (dict(qs_len=3), -2),                    # query_start needs S + 1 entries
+    (dict(q_data=0x10008), -7),              # query misaligned
+])
+def test_prefill_rejects_bad_arguments_before_cuda(lib, case, expect):
+    kw = dict(case)
+    a = _prefill_args(**kw)
+    assert _prefill(lib, a, bs=kw.get("bs", 16), hkv=kw.get("Hkv", 2)) == expect
+    assert pa.pa_last_error()
+
+
+def test_prefill_rejects_mismatches(lib):
+    a = _prefill_args()
+    assert _prefill(lib, a, bs=8) == -2           # block_size disagrees with the cache
+    assert _prefill(lib, a, hkv=4) == -2          # num_kv_heads disagrees with the cache
+    assert _prefill(lib, a, scale=float("inf")) == -1
+    b = _prefill_args()
+    b["query"] = _t([40, 8, 128], pa.PA_F16)
+    assert _prefill(lib, b) == -3                 # query of another type than the caches
+    c = _prefill_args()
+    c["qs"] = _t([4], pa.PA_I64)
+    assert _prefill(lib, c) == -3                 # query_start must be int32
+    d = _prefill_args()
+    d["out"] = _t([39, 8, 128], pa.PA_BF16)
+    assert _prefill(lib, d) == -2                 # out like the query
+    assert _prefill(lib, _prefill_args(T=0)) == 0  # no new tokens: nothing to do
+
+
+def test_swap_blocks_rejects_bad_arguments(lib):
+    r = ctypes.byref
+    dev_k, dev_v = _t([32, 2, 16, 128], pa.PA_BF16), _t([32, 2, 16, 128], pa.PA_BF16)
+    host_k, host_v = _t([64, 2, 16, 128], pa.PA_BF16), _t([64, 2, 16, 128], pa.PA_BF16)
+    other = _t([64, 2, 8, 128], pa.PA_BF16)
+    pairs = _t([3, 2], pa.PA_I64)
+    assert lib.pa_swap_blocks(r(dev_k), r(dev_v), r(other), r(other), r(pairs), None) == -2
+    assert lib.pa_swap_blocks(r(dev_k), r(dev_v), r(host_k), r(host_v), r(_t([3, 2], pa.PA_I32)), None) == -3
+    assert lib.pa_swap_blocks(r(dev_k), r(dev_v), r(host_k), r(host_v), r(_t([3, 3], pa.PA_I64)), None) == -2
+    assert lib.pa_swap_blocks(r(dev_k), r(dev_v), r(host_k), r(host_v), r(_t([0, 2], pa.PA_I64)), None) == 0
+
+
+def test_fp8_entry_points_reject_bad_arguments(lib):
+    r = ctypes.byref
+    kc8, vc8 = _t([32, 2, 16, 128], pa.PA_FP8_E4M3), _t([32, 2, 16, 128], pa.PA_FP8_E4M3)
+    key = _t([5, 2, 128], pa.PA_BF16)
+    slots = _t([5], pa.PA_I64)
+    ks, vs = _t([2], pa.PA_F32), _t([2], pa.PA_F32)
+    w = lambda k=key, kc=kc8, s1=ks, s2=vs: lib.pa_reshape_and_cache_fp8(r(k), r(k), r(kc), r(kc), r(slots),
+                                                                         r(s1), r(s2), None)
+    assert w(s1=_t([2], pa.PA_F16)) == -3                         # scales must be fp32
+    assert w(s1=_t([3], pa.PA_F32), s2=_t([3], pa.PA_F32)) == -2   # one scale per kv head
+    assert w(kc=_t([32, 2, 16, 128], pa.PA_BF16)) == -3            # the caches must be FP8
+    # the 16-bit entry points refuse FP8 caches, whose values need their scales
+    a = _decode_args()
+    a["kc"], a["vc"] = kc8, vc8
+    assert _decode(lib, a) == -3
+    S, Hq = 4, 8
+
+    def dec(q_dt=pa.PA_BF16, s1=ks, flags=0, kc=kc8, D=128):
+        o, q = _t([S, Hq, D], pa.PA_F32), _t([S, Hq, D], q_dt)
+        bt, cl = _t([S, 4], pa.PA_I32), _t([S], pa.PA_I32)
+        return lib.pa_decode_fp8(r(o), r(q), r(kc), r(kc), r(bt), r(cl), r(s1), r(vs), 0.1, 16, 2, 0,
+                                 flags, None, 0, None)
+
+    assert dec(q_dt=pa.PA_F32) == -3                   # the query must be bf16 or fp16
+    assert dec(s1=_t([2], pa.PA_F16)) == -3            # scales must be fp32
+    assert dec(flags=pa.PA_DECODE_CUDA_CORES) == -4    # FP8 is read by the tensor-core kernel only
+    assert dec(kc=_t([32, 2, 16, 64], pa.PA_FP8_E4M3), D=64) == -4  # head_dim 64 is not built
+    assert pa.pa_last_error()
