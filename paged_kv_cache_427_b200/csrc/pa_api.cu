@@ -297,8 +297,9 @@ uint64_t g_map_clock = 0;
 // block_size / 8 row groups, blocks x kv heads; one box brings a whole (block, kv head) tile laid
 // out as [group of 8 rows][half][row][128 bytes], the operand layout of the tensor-core MMAs.
 bool grouped_view_ok(const pa_tensor *t) {
+  // (block, kv head) pairs are one coordinate of the view, a 32-bit TMA coordinate
   return t->stride[3] == 1 && t->stride[2] == t->shape[3] && t->stride[0] == t->shape[1] * t->stride[1] &&
-         t->shape[2] % 8 == 0;
+         t->shape[2] % 8 == 0 && t->shape[0] * t->shape[1] <= 0x7fffffff;
 }
 
 int cache_map(const pa_tensor *t, int rows, CUtensorMap *out) {
