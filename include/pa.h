@@ -214,11 +214,17 @@ PA_API int pa_decode_fp8(const pa_tensor *out, const pa_tensor *query, const pa_
  *   query_start: [S + 1] int32, non-decreasing from 0; block_tables [S, max_blocks];
  *   context_lens [S].  Caches bf16 or fp16 (fp32 / FP8: PA_ERR_UNSUPPORTED), head_dim 64 or
  *   128, block_size 8/16/32, 1/2/4/8 query heads per kv head.
+ *   query and out need a contiguous head_dim and 16-byte aligned data and token/head strides
+ *   (PA_ERR_LAYOUT otherwise).
  * A sequence with q_len > context_len, or whose rows fall outside [0, T), sets
- * PA_DEVERR_CONTEXT_LEN and its rows are not written.  Rows of tokens past query_start[S] are not written.  One kernel: a persistent grid
- * of 4-warp CTAs, each taking tiles of 64 query rows (64/G tokens x G heads) of one (sequence,
- * kv head) and streaming that sequence's K/V tiles up to the tile's last position through a
- * TMA ring; the tensor cores (mma.sync) compute S = QK^T and O = PV with P kept to ~16 bits.
+ * PA_DEVERR_CONTEXT_LEN and its rows are not written.  Rows of tokens past query_start[S] are
+ * not written.  Asynchronous on `stream`; every tensor is the caller's and stays so.
+ * One kernel on the fifth-generation tensor cores: a persistent grid, one CTA per SM, each
+ * taking tiles of 128 query rows (128/G tokens x G heads) of one (sequence, kv head) and
+ * streaming that sequence's K/V tiles up to the tile's last position by TMA; tcgen05 MMAs
+ * compute S = QK^T and O = PV into tensor memory, with P kept to ~16 bits (two bf16/fp16
+ * terms).  Caches whose blocks are kv heads x rows x head_dim contiguous are read one
+ * (block, kv head) tile per copy, other layouts in 8-row copies.
  */
 PA_API int pa_prefill(const pa_tensor *out, const pa_tensor *query, const pa_tensor *key_cache,
                       const pa_tensor *value_cache, const pa_tensor *block_tables,
