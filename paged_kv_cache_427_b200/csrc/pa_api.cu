@@ -16,6 +16,7 @@
 
 #include "pa.h"
 #include "pa_internal.h"
+#include "pa_prefill_internal.h"
 
 namespace {
 

@@ -97,16 +97,6 @@ __device__ __forceinline__ void tma_load_tile(uint32_t dst, const CUtensorMap *m
       : "memory");
 }
 
-// One box of a 4-D tensor map (the prefill's query rows) into shared memory.
-__device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap *map, int c0, int c1, int c2,
-                                            int c3, uint64_t *bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes "
-      "[%0], [%1, {%2, %3, %4, %5}], [%6];" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(smem_u32(bar))
-      : "memory");
-}
-
 // Prefetch one box of the 5-D cache view into L2 (no shared memory, no completion to wait for).
 __device__ __forceinline__ void tma_prefetch_tile(const CUtensorMap *map, int y, int z, int w) {
   asm volatile(

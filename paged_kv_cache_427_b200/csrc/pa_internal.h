@@ -125,48 +125,6 @@ struct CacheWriteFp8Args {
 
 cudaError_t launch_reshape_and_cache_fp8(const CacheWriteFp8Args &a, int num_sms, cudaStream_t st);
 
-// Causal attention of a step's new tokens (prefill): query row r = query_start[s] + j is
-// token j of sequence s's q_len new tokens, at position context_len - q_len + j.
-struct PrefillArgs {
-  void *out;
-  int out_dtype;
-  int64_t out_t, out_h;  // elements
-  const void *query;
-  int64_t q_t, q_h;      // elements
-  const int32_t *block_tables;
-  int64_t bt_s;
-  const int32_t *context_lens;
-  const int32_t *query_start;
-  int num_seqs;
-  int num_kv_heads;
-  int max_blocks;
-  int64_t num_blocks;
-  int64_t num_tokens;   // query rows
-  float scale_log2;
-  unsigned int *err;
-  long long wait_cycles;
-  int grouped_maps;  // 1: the maps are the grouped view (one box per block and kv head)
-};
-
-// The prefill's tensor maps: the caches (grouped view, or 8-row boxes) and the query rows.
-struct PrefillMaps {
-  CUtensorMap k;
-  CUtensorMap v;
-  CUtensorMap q;
-};
-
-struct PrefillKernel {
-  cudaError_t (*launch)(const PrefillArgs &, const PrefillMaps *, int num_ctas, cudaStream_t);
-  const void *kernel;
-  int threads_per_cta;
-  int smem_bytes;
-  int tokens_per_tile;  // query tokens of one tile (128 rows / query heads per kv head)
-  int tma_rows;
-};
-
-bool prefill_kernel_bf16(int head_dim, int block_size, int group, PrefillKernel *k);
-bool prefill_kernel_f16(int head_dim, int block_size, int group, PrefillKernel *k);
-
 // Tensor-core decode for FP8 E4M3 caches with a bf16 or fp16 query (head_dim 128 only).
 bool decode_kernel_fp8(int q_dtype, int head_dim, int block_size, int group, DecodeKernel *k);
 
