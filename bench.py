@@ -322,6 +322,19 @@ def make_batch(name: str) -> W.PagedBatch:
     return W.workload(name)
 
 
+def max_over_ranks(vals, device=None) -> list:
+    """Element-wise maximum of `vals` over the ranks of the default process group (each rank's
+    times: the slowest rank's count); the values unchanged outside a multi-rank group."""
+    import torch
+    import torch.distributed as dist
+
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return [float(v) for v in vals]
+    t = torch.tensor([float(v) for v in vals], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
 def run_ours(args, b: W.PagedBatch, config: dict, rank: int, world: int, local_rank: int):
     import torch
     import torch.distributed as dist
@@ -548,12 +561,8 @@ def run_ours(args, b: W.PagedBatch, config: dict, rank: int, world: int, local_r
         del graphs
     clocks = sampler.stop()
 
-    if world > 1:
-        t = torch.tensor([elapsed_ms, e2e_ms, float(np.mean(decode_ms))], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        elapsed_ms, e2e_ms, dec_mean = t.tolist()
-    else:
-        dec_mean = float(np.mean(decode_ms))
+    elapsed_ms, e2e_ms, dec_mean = max_over_ranks([elapsed_ms, e2e_ms, float(np.mean(decode_ms))],
+                                                  device=dev)
     flags = pa.pa_get_device_error(clear=True)
     if rank != 0:
         return
