@@ -194,15 +194,17 @@ class ClockSampler:
 # the oracle (CPU baseline and reference arm)
 # ----------------------------------------------------------------------------------------------
 
-def oracle_sample_run(b: W.PagedBatch, budget_s: float, orc):
+def oracle_sample_run(b: W.PagedBatch, budget_s: float, orc, num_threads: int = 0):
     """Time the oracle's step on the first n sequences, n grown until one run takes about
-    budget_s.  Returns (seconds, n, algorithmic bytes of the sample, attended tokens)."""
+    budget_s (num_threads 0: all the oracle's OpenMP threads).  Returns (seconds, n,
+    algorithmic bytes of the sample, attended tokens)."""
     kc, vc = b.key_cache, b.value_cache
     n = 1
     while True:
         sub = W.sub_batch(b, np.arange(n))
         t0 = time.perf_counter()
-        orc.decode(sub["query"], kc, vc, sub["block_tables"], sub["context_lens"], b.scale, b.dtype)
+        orc.decode(sub["query"], kc, vc, sub["block_tables"], sub["context_lens"], b.scale, b.dtype,
+                   num_threads=num_threads)
         dt = time.perf_counter() - t0
         if dt >= budget_s or n == b.num_seqs:
             break
@@ -217,11 +219,16 @@ def cpu_baseline(b: W.PagedBatch, budget_s: float = 10.0):
 
     orc = oracle.load()
     dt, n, nbytes, toks = oracle_sample_run(b, budget_s, orc)
+    # the same oracle on one thread, over a sample of a fifth of the time
+    dt1, n1, nbytes1, toks1 = oracle_sample_run(b, budget_s / 5, orc, num_threads=1)
     return {"value": round(nbytes / dt / 1e9, 4), "unit": "GB/s", "cores": orc.max_threads(),
             "kind": "oracle",
             "sample": f"oracle decode (fp64, OpenMP) of the first {n} of {b.num_seqs} sequences "
                       f"({toks} attended tokens), one run of {dt:.2f} s",
-            "attended_tokens_per_s": round(toks / dt, 1)}
+            "attended_tokens_per_s": round(toks / dt, 1),
+            "one_thread": {"value": round(nbytes1 / dt1 / 1e9, 4), "unit": "GB/s", "cores": 1,
+                           "sample": f"the first {n1} sequences ({toks1} attended tokens), one run "
+                                     f"of {dt1:.2f} s"}}
 
 
 def cpu_baseline_fp8(b: W.PagedBatch, kc8, vc8, ks, vs, budget_s: float = 10.0):
