@@ -174,6 +174,23 @@ def test_prefill_single_tokens_match_decode():
     assert_close(got, to_host(out, "f32"), "bf16", "prefill vs decode")
 
 
+def test_prefill_many_small_sequences_use_the_unsorted_schedule(oracle):
+    """More (sequence, tile) pairs than the kernel's shared tile list holds (4,096): every CTA
+    then takes tiles in sequence order, each warp locating its tile by a scan of query_start.
+    4,200 sequences of one to three new tokens on short contexts, one query head per kv head."""
+    require_gpu()
+    rng = np.random.default_rng(W.BASE_SEED + 747)
+    S = 4200
+    ql = rng.integers(1, 4, S)
+    lens = ql + rng.integers(0, 40, S)
+    b = W.build_prefill_batch("pfmany", lens.tolist(), ql.tolist(), num_heads=2, num_kv_heads=2,
+                              head_dim=64, block_size=16, dtype="bf16", seed=W.BASE_SEED + 748)
+    ref, _, _ = _oracle(oracle, b)
+    st = PrefillStep(b)
+    assert_close(st.run("f32"), ref, "bf16", "prefill, unsorted schedule")
+    assert_no_device_error()
+
+
 def test_prefill_more_new_tokens_than_context_is_flagged():
     require_gpu()
     b = W.build_prefill_batch("pfbad", [40, 40], [10, 10], num_heads=8, num_kv_heads=2,
