@@ -72,3 +72,16 @@ def test_reference_arm_under_torchrun_prints_once():
     assert len(lines) == 1
     line = json.loads(lines[0])
     assert line["impl"] == "reference" and line["value"] > 0
+
+
+@pytest.mark.timeout(600)
+def test_reference_arm_of_a_prefill_workload_times_the_prefill_oracle():
+    """The reference arm reports the arm's own metric: TFLOP/s of the oracle's prefill for the
+    chunked-prefill workload."""
+    cmd = [sys.executable, "bench.py", "--impl", "reference", "--workload", "chunked_prefill",
+           "--steps", "1", "--warmup", "3"]
+    res = subprocess.run(cmd, cwd=ROOT, capture_output=True, text=True, timeout=560)
+    assert res.returncode == 0, res.stderr[-2000:]
+    line = json.loads([l for l in res.stdout.splitlines() if l.startswith("{")][-1])
+    assert line["impl"] == "reference" and line["unit"] == "TFLOP/s"
+    assert line["metric"].startswith("paged prefill attention") and line["value"] > 0
