@@ -331,9 +331,126 @@ def run_reference_prefill(args, b: W.PagedBatch, config: dict):
     print(json.dumps(line), flush=True)
 
 
+def run_reference_fp8(args, b: W.PagedBatch, config: dict):
+    """The reference arm of `--kv fp8`: the workload's pool quantised by the oracle with the
+    same per-kv-head scales as the CUDA arm (largest magnitude of the head's rows / 240), then
+    per step the oracle's FP8 cache write and decode of the first n sequences."""
+    import oracle
+
+    orc = oracle.load()
+    steps, warmup = args.steps, args.warmup
+    bs = b.block_size
+    used = []
+    for s in range(b.num_seqs):
+        t = np.arange(max(int(b.context_lens[s]) - 1, 0))
+        used.append(b.block_tables[s, t // bs].astype(np.int64) * bs + t % bs)
+    used = np.unique(np.concatenate(used))
+    rows_k = b.key_cache[used // bs, :, used % bs, :]
+    rows_v = b.value_cache[used // bs, :, used % bs, :]
+
+    def head_scales(rows, new):
+        x = W.decode_to_f64(np.concatenate([rows, new]), b.dtype)
+        return np.maximum(np.abs(x).max(axis=(0, 2)) / 240.0, 1e-8).astype(np.float32)
+
+    ks, vs = head_scales(rows_k, b.key), head_scales(rows_v, b.value)
+    kc8 = np.full(b.key_cache.shape, 0x7f, dtype=np.uint8)
+    vc8 = np.full(b.value_cache.shape, 0x7f, dtype=np.uint8)
+    orc.reshape_and_cache_fp8(rows_k, rows_v, b.dtype, kc8, vc8, used, ks, vs)
+    per_step = max(0.005, 120.0 / max(1, steps + warmup))
+    n = 1
+    while True:
+        sub = W.sub_batch(b, np.arange(n))
+        t0 = time.perf_counter()
+        orc.decode(sub["query"], kc8, vc8, sub["block_tables"], sub["context_lens"], b.scale, "fp8",
+                   q_dtype=b.dtype, k_scale=ks, v_scale=vs)
+        dt = time.perf_counter() - t0
+        if dt >= per_step or n == b.num_seqs:
+            break
+        n = min(b.num_seqs, max(n + 1, int(n * min(8.0, per_step / max(dt, 1e-4)))))
+
+    def step():
+        orc.reshape_and_cache_fp8(b.key[:n], b.value[:n], b.dtype, kc8, vc8, b.slot_mapping[:n], ks, vs)
+        orc.decode(sub["query"], kc8, vc8, sub["block_tables"], sub["context_lens"], b.scale, "fp8",
+                   q_dtype=b.dtype, k_scale=ks, v_scale=vs)
+
+    for _ in range(warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(steps):
+        step()
+    dt = (time.perf_counter() - t0) / max(1, steps)
+    sb = W.PagedBatch(**{**b.__dict__, "query": sub["query"], "block_tables": sub["block_tables"],
+                          "context_lens": sub["context_lens"]})
+    step_bytes = (decode_bytes(sb, ELT[b.dtype], unique=False, kv_elt=1)
+                  + n * b.num_kv_heads * b.head_dim * (ELT[b.dtype] + 1) * 2 + n * 8)
+    value = step_bytes / dt / 1e9
+    toks = int(sub["context_lens"].sum())
+    line = {"impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s",
+            "n_gpus": args.gpus, "steps": steps, "warmup": warmup, "ms_per_step": round(dt * 1e3, 4),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": dict(config, kv_dtype="fp8_e4m3",
+                                                kv_scales="per kv head: max |x| / 240"),
+            "attended_tokens_per_s": round(toks / dt, 1),
+            "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": orc.max_threads(),
+                             "kind": "oracle",
+                             "sample": f"each step: oracle FP8 cache write + decode of the first {n} of "
+                                       f"{b.num_seqs} sequences ({toks} attended tokens)"},
+            "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def run_reference_swap(args, b: W.PagedBatch, config: dict):
+    """The reference arm of `--swap`: the oracle moves every block the batch uses from the
+    pool to a second pool (scattered ids) and back, timed on the host."""
+    import oracle
+
+    orc = oracle.load()
+    ids = []
+    for s in range(b.num_seqs):
+        ids.extend(b.block_tables[s, :-(-int(b.context_lens[s]) // b.block_size)].tolist())
+    ids = np.array(sorted(set(ids)), np.int64)
+    n = len(ids)
+    rng = np.random.default_rng(0)
+    host_ids = rng.permutation(n).astype(np.int64)
+    hk = np.empty((n,) + b.key_cache.shape[1:], dtype=b.key_cache.dtype)
+    hv = np.empty_like(hk)
+    kc, vc = b.key_cache.copy(), b.value_cache.copy()
+    out_pairs = np.stack([ids, host_ids], 1)
+    in_pairs = np.stack([host_ids, rng.permutation(ids)], 1)
+    block_bytes = int(np.prod(b.key_cache.shape[1:])) * ELT[b.dtype] * 2
+    total = n * block_bytes
+
+    def step():
+        orc.swap_blocks(kc, vc, hk, hv, out_pairs, b.dtype)
+        orc.swap_blocks(hk, hv, kc, vc, in_pairs, b.dtype)
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    dt = (time.perf_counter() - t0) / max(1, args.steps)
+    value = 2 * total / dt / 1e9  # both directions per step
+    line = {"impl": "reference", "metric": "block swap GB/s (device <-> pinned host, pa_swap_blocks)",
+            "value": round(value, 4), "unit": "GB/s", "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(dt * 1e3, 4), "higher_is_better": True,
+            "dtype": b.dtype, "data": "synthetic",
+            "config": dict(config, swapped_blocks=n, bytes_per_direction=total),
+            "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+                             "sample": f"each step: all {n} blocks out and back, host memory"},
+            "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
 def run_reference(args, b: W.PagedBatch, config: dict):
     if b.query_start is not None:
         return run_reference_prefill(args, b, config)
+    if args.swap:
+        return run_reference_swap(args, b, config)
+    if args.kv == "fp8":
+        return run_reference_fp8(args, b, config)
     import oracle
 
     orc = oracle.load()

@@ -85,3 +85,17 @@ def test_reference_arm_of_a_prefill_workload_times_the_prefill_oracle():
     line = json.loads([l for l in res.stdout.splitlines() if l.startswith("{")][-1])
     assert line["impl"] == "reference" and line["unit"] == "TFLOP/s"
     assert line["metric"].startswith("paged prefill attention") and line["value"] > 0
+
+
+@pytest.mark.timeout(600)
+@pytest.mark.parametrize("extra,unit", [(["--kv", "fp8"], "GB/s"), (["--swap"], "GB/s")])
+def test_reference_arm_of_fp8_and_swap_runs_the_matching_oracle(extra, unit):
+    cmd = [sys.executable, "bench.py", "--impl", "reference", "--steps", "1", "--warmup", "3"] + extra
+    res = subprocess.run(cmd, cwd=ROOT, capture_output=True, text=True, timeout=560)
+    assert res.returncode == 0, res.stderr[-2000:]
+    line = json.loads([l for l in res.stdout.splitlines() if l.startswith("{")][-1])
+    assert line["impl"] == "reference" and line["unit"] == unit and line["value"] > 0
+    if "--swap" in extra:
+        assert line["metric"].startswith("block swap")
+    else:
+        assert line["config"]["kv_dtype"] == "fp8_e4m3"
