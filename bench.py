@@ -105,31 +105,49 @@ def hbm_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-DECODE_SOURCES = ("pa_decode_mma.cuh", "pa_decode_common.cuh", "pa_decode.cuh", "pa_device.cuh",
-                  "pa_internal.h", "pa_decode_bf16_d128.cu")
+def bf16_peak():
+    """Dense bf16 tensor rate: the burst figure (a kernel timed alone per launch)."""
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["bf16_tflops"]), "measured"
+    except Exception:
+        return 1590.0, "fallback"
 
 
-def kernel_sources_digest() -> str:
-    """Digest of the files the 16-bit decode kernels are compiled from (device code and the
-    argument block), not the host-side API or the other kernels."""
+# The files each kernel's device code is compiled from (its traffic record is void once any
+# of them changes).
+KERNEL_SOURCES = {
+    "decode": ("pa_decode_mma.cuh", "pa_decode_common.cuh", "pa_decode.cuh", "pa_device.cuh",
+               "pa_internal.h", "pa_decode_bf16_d128.cu"),
+    "decode_fp8": ("pa_decode_mma.cuh", "pa_decode_common.cuh", "pa_decode.cuh", "pa_device.cuh",
+                   "pa_internal.h", "pa_decode_fp8_bf16q.cu"),
+    "prefill": ("pa_prefill_tc.cuh", "pa_tc.cuh", "pa_device.cuh", "pa_prefill_internal.h",
+                "pa_prefill_bf16.cu"),
+}
+
+
+def kernel_sources_digest(kernel: str = "decode") -> str:
+    """Digest of the files a kernel is compiled from (device code and its argument block),
+    not the host-side API or the other kernels."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "paged_kv_cache_427_b200", "csrc")
     for f in sorted(os.listdir(csrc)):
-        if f in DECODE_SOURCES:
+        if f in KERNEL_SOURCES[kernel]:
             with open(os.path.join(csrc, f), "rb") as fh:
                 h.update(f.encode() + fh.read())
     return h.hexdigest()[:16]
 
 
-def recorded_traffic(workload: str):
-    """DRAM bytes per decode launch from the committed ncu summary, if it was taken on the
-    current kernel sources; else None."""
+def recorded_traffic(key: str, kernel: str = "decode"):
+    """DRAM bytes per launch from the committed ncu summary (profiles/traffic.json, keyed by
+    workload, ':fp8' for the FP8 cache), if it was taken on the current kernel sources; else
+    None."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(path) as f:
             rec = json.load(f)
-        entry = rec.get(workload)
-        if entry and entry.get("sources") == kernel_sources_digest():
+        entry = rec.get(key)
+        if entry and entry.get("sources") == kernel_sources_digest(kernel):
             return float(entry["dram_bytes_per_launch"])
     except Exception:
         pass
@@ -212,7 +230,7 @@ def oracle_sample_run(b: W.PagedBatch, budget_s: float, orc, num_threads: int = 
         n = min(b.num_seqs, max(n + 1, int(n * min(8.0, budget_s / max(dt, 1e-4)))))
     sb = W.PagedBatch(**{**b.__dict__, "query": sub["query"], "block_tables": sub["block_tables"],
                           "context_lens": sub["context_lens"]})
-    return dt, n, decode_bytes(sb, ELT[b.dtype], unique=False), int(sub["context_lens"].sum())
+    return dt, n, decode_bytes(sb, ELT[b.dtype], unique=True), int(sub["context_lens"].sum())
 
 
 def cpu_baseline(b: W.PagedBatch, budget_s: float = 10.0):
@@ -249,7 +267,7 @@ def cpu_baseline_fp8(b: W.PagedBatch, kc8, vc8, ks, vs, budget_s: float = 10.0):
         n = min(b.num_seqs, max(n + 1, int(n * min(8.0, budget_s / max(dt, 1e-4)))))
     sb = W.PagedBatch(**{**b.__dict__, "query": sub["query"], "block_tables": sub["block_tables"],
                           "context_lens": sub["context_lens"]})
-    nbytes = decode_bytes(sb, ELT[b.dtype], unique=False, kv_elt=1)
+    nbytes = decode_bytes(sb, ELT[b.dtype], unique=True, kv_elt=1)
     toks = int(sub["context_lens"].sum())
     return {"value": round(nbytes / dt / 1e9, 4), "unit": "GB/s", "cores": orc.max_threads(),
             "kind": "oracle",
@@ -381,7 +399,7 @@ def run_reference_fp8(args, b: W.PagedBatch, config: dict):
     dt = (time.perf_counter() - t0) / max(1, steps)
     sb = W.PagedBatch(**{**b.__dict__, "query": sub["query"], "block_tables": sub["block_tables"],
                           "context_lens": sub["context_lens"]})
-    step_bytes = (decode_bytes(sb, ELT[b.dtype], unique=False, kv_elt=1)
+    step_bytes = (decode_bytes(sb, ELT[b.dtype], unique=True, kv_elt=1)
                   + n * b.num_kv_heads * b.head_dim * (ELT[b.dtype] + 1) * 2 + n * 8)
     value = step_bytes / dt / 1e9
     toks = int(sub["context_lens"].sum())
@@ -509,9 +527,204 @@ def max_over_ranks(vals, device=None) -> list:
     return t.tolist()
 
 
-def run_ours(args, b: W.PagedBatch, config: dict, rank: int, world: int, local_rank: int):
+# ----------------------------------------------------------------------------------------------
+# timing helpers
+# ----------------------------------------------------------------------------------------------
+
+def launch_stats(ms) -> dict:
+    """Mean, median and minimum of per-launch CUDA-event durations (ms in, us out)."""
+    us = np.asarray(ms, dtype=np.float64) * 1e3
+    return {"mean_launch_us": round(float(us.mean()), 3),
+            "median_launch_us": round(float(np.median(us)), 3),
+            "min_launch_us": round(float(us.min()), 3), "launches": int(us.size)}
+
+
+def launch_count(args) -> int:
+    """Launches timed one by one for the roofline: at least 50, at most 500."""
+    return max(50, min(args.steps, 500))
+
+
+def pool_rotations(args, attended: int) -> int:
+    """Copies of the KV pool that consecutive steps rotate over, enough that one step's
+    attended bytes push the previous step's rows out of L2 before they are read again."""
+    return args.rotations or max(2, min(8, math.ceil(3 * L2_BYTES / max(attended, 1)) + 1))
+
+
+def dev_tensor(a, dt, dev):
+    """Device tensor with the bytes of host array `a` (bf16 held as uint16 patterns)."""
     import torch
-    import torch.distributed as dist
+
+    a = np.ascontiguousarray(a)
+    if dt == "bf16":
+        return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(dev)
+    return torch.from_numpy(a).to(dev)
+
+
+def run_steps(step, n: int, stream, first: int = 0) -> float:
+    """n steps with nothing between the launches, one event pair around them: total ms."""
+    import torch
+
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for i in range(first, first + n):
+        step(i)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1)
+
+
+def run_launches(step, n: int) -> list:
+    """n steps with an event pair around each step's main kernel: per-launch ms."""
+    import torch
+
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(n)]
+    torch.cuda.synchronize()
+    for i in range(n):
+        step(i, evs[i])
+    torch.cuda.synchronize()
+    return [s.elapsed_time(e) for s, e in evs]
+
+
+def soak(step, seconds: float, per_round: int = 200):
+    """Untimed load, so the clock sampler sees the GPU busy and clocks settle."""
+    import torch
+
+    t0, i = time.perf_counter(), 0
+    while time.perf_counter() - t0 < seconds:
+        for _ in range(per_round):
+            step(i)
+            i += 1
+        torch.cuda.synchronize()
+
+
+def hbm_roofline(alg_bytes: int, launch_ms, kernel: str, traffic, probe=None) -> dict:
+    peak, src = hbm_peak()
+    st = launch_stats(launch_ms)
+    achieved = alg_bytes / (st["mean_launch_us"] * 1e-6) / 1e9
+    r = {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak, "unit": "GB/s",
+         "frac": round(achieved / peak, 4), "traffic": traffic, "kernel": kernel,
+         "peak_source": src, "algorithmic_bytes_per_launch": int(alg_bytes), **st,
+         "achieved_at_median": round(alg_bytes / (st["median_launch_us"] * 1e-6) / 1e9, 2),
+         "launch_timing": "CUDA events around each launch on its stream, in a timed region of "
+                          "its own after the step region"}
+    if traffic:
+        r["traffic_over_algorithmic"] = round(traffic / alg_bytes, 4)
+    if probe:
+        best = max(probe["ld_GBps"], probe["bulk_GBps"])
+        r["read_probe_GBps"] = best
+        r["frac_of_read_probe"] = round(achieved / best, 4)
+    return r
+
+
+def read_probe(dev, nbytes: int = 4 << 30, reps: int = 10) -> dict | None:
+    """Read-only HBM bandwidth of this GPU: pa_hbm_read_probe over a buffer of `nbytes` (32x
+    L2), both modes, median of `reps` launches after 3 warm-up launches."""
+    import torch
+
+    import paged_kv_cache_427_b200 as pa
+
+    try:
+        buf = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+        buf.view(torch.int32).random_()
+        sink = torch.zeros(4, dtype=torch.int32, device=dev)
+        res = {}
+        for mode, key in ((0, "ld_GBps"), (1, "bulk_GBps")):
+            for _ in range(3):
+                pa.pa_hbm_read_probe(buf, mode, sink)
+            evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                   for _ in range(reps)]
+            for e0, e1 in evs:
+                e0.record()
+                pa.pa_hbm_read_probe(buf, mode, sink)
+                e1.record()
+            torch.cuda.synchronize()
+            ms = float(np.median([a.elapsed_time(b) for a, b in evs]))
+            res[key] = round(nbytes / (ms * 1e-3) / 1e9, 1)
+        if int(sink[1].item()) != 0:
+            return None
+        del buf
+        torch.cuda.empty_cache()
+        res.update({"bytes": nbytes, "reps": reps,
+                    "how": "pa_hbm_read_probe: each byte read once; ld = 16-byte loads from 2048 "
+                           "threads per SM, bulk = 32 KB bulk copies into a 6-slot shared-memory "
+                           "ring per SM; median of the CUDA-event launch times"})
+        return res
+    except Exception as exc:  # the probe is evidence beside the numbers, never a reason to fail
+        print(f"warning: read probe failed: {exc}", file=sys.stderr)
+        return None
+
+
+def timeline_summary(recs, chunk_bytes: int) -> dict:
+    """Per-launch summary of decode timelines (pa_set_decode_timeline records, one array per
+    launch), medians over the launches.  Times are us after the first worker warp started."""
+    import paged_kv_cache_427_b200 as pa
+
+    per = []
+    sm_done = []
+    for rec in recs:
+        r = rec.reshape(-1, pa.TIMELINE_WORDS).astype(np.int64)
+        r = r[r[:, pa.TL_START] > 0]  # warps of this launch
+        live = r[:, pa.TL_CHUNKS] > 0
+        if not live.any():
+            continue
+        o = r[:, pa.TL_START].min()
+        us = lambda c: (r[live, c] - o) / 1e3  # noqa: E731
+        done = np.maximum(r[live, pa.TL_DONE], r[live, pa.TL_MERGED]) - o
+        done = done / 1e3
+        first, last = us(pa.TL_FIRST), us(pa.TL_LAST)
+        span = np.maximum(last - first, 1e-3)
+        rates = r[live, pa.TL_CHUNKS] * chunk_bytes / (span * 1e-6) / 1e9
+        end = float(done.max())
+        per.append({"end_us": end,
+                    "issue_us_p50": float(np.median(us(pa.TL_ISSUE))),
+                    "first_tile_us_p10": float(np.percentile(first, 10)),
+                    "first_tile_us_p50": float(np.median(first)),
+                    "first_tile_us_p90": float(np.percentile(first, 90)),
+                    "last_tile_us_p50": float(np.median(last)),
+                    "done_us_p10": float(np.percentile(done, 10)),
+                    "done_us_p50": float(np.median(done)),
+                    "done_us_p90": float(np.percentile(done, 90)),
+                    "tail_us": end - float(np.median(done)),
+                    "sum_of_warp_rates_GBps": float(rates.sum())})
+        sms = r[live, pa.TL_SM]
+        d = {}
+        for smv, dv in zip(sms, done):
+            d[int(smv)] = max(d.get(int(smv), 0.0), float(dv))
+        sm_done.append(d)
+    if not per:
+        return {}
+    out = {k: round(float(np.median([p[k] for p in per])), 2) for k in per[0]}
+    # do the same SMs finish last in every launch?  rank correlation of the SMs' finish times
+    common = sorted(set.intersection(*[set(d) for d in sm_done])) if sm_done else []
+    if len(sm_done) > 1 and len(common) > 2:
+        ranks = [np.argsort(np.argsort([d[k] for k in common])) for d in sm_done]
+        cs = [float(np.corrcoef(ranks[i], ranks[i + 1])[0, 1]) for i in range(len(ranks) - 1)]
+        out["sm_finish_rank_corr"] = round(float(np.mean(cs)), 3)
+        fin = np.array([[d[k] for k in common] for d in sm_done])
+        out["sm_finish_us_min_p50_max"] = [round(float(x), 2) for x in
+                                           (np.median(fin.min(1)), np.median(np.median(fin, 1)),
+                                            np.median(fin.max(1)))]
+    out["launches"] = len(per)
+    out["how"] = ("pa_set_decode_timeline: globaltimer per worker warp at start, first tile "
+                  "landed, last tile consumed, done (merges included); times after the first "
+                  "warp started; medians over the launches")
+    return out
+
+
+# ----------------------------------------------------------------------------------------------
+# the CUDA path
+# ----------------------------------------------------------------------------------------------
+
+def run_decode(args, b: W.PagedBatch, config: dict, rank: int = 0, world: int = 1,
+               local_rank: int = 0, full: bool = True, probe: dict | None = None) -> dict | None:
+    """The decode step of one workload: the cache write (plus the copy-on-write block copies
+    where the batch has them), then the decode launched to overlap the write.  Timed regions:
+    K steps with nothing between launches (`value`); per-launch events around the decode (the
+    roofline); with `full`, also the step as a CUDA graph, end to end from pinned host memory,
+    the CPU baseline and the timeline.  Returns rank 0's line (None on the other ranks)."""
+    import torch
 
     import paged_kv_cache_427_b200 as pa
 
@@ -520,25 +733,18 @@ def run_ours(args, b: W.PagedBatch, config: dict, rank: int, world: int, local_r
     tdt = {"bf16": torch.bfloat16, "f16": torch.float16, "f32": torch.float32}[b.dtype]
     out_dtype = tdt
 
-    def dev_t(a, dt=None):
-        if dt == "bf16":
-            return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
-        return torch.from_numpy(np.ascontiguousarray(a)).to(dev)
-
-    # rotating pools: enough copies that each step's attended bytes push the previous step's
-    # rows out of L2 before they are read again
-    att = attended_bytes(b)
-    rot = args.rotations or max(2, min(8, math.ceil(3 * L2_BYTES / max(att, 1)) + 1))
-    kc0 = dev_t(b.key_cache, b.dtype)
-    vc0 = dev_t(b.value_cache, b.dtype)
+    rot = pool_rotations(args, attended_bytes(b))
+    kc0 = dev_tensor(b.key_cache, b.dtype, dev)
+    vc0 = dev_tensor(b.value_cache, b.dtype, dev)
     pools = [(kc0, vc0)] + [(kc0.clone(), vc0.clone()) for _ in range(rot - 1)]
-    q = dev_t(b.query, b.dtype)
-    key = dev_t(b.key, b.dtype)
-    value = dev_t(b.value, b.dtype)
-    slots = dev_t(b.slot_mapping)
-    tables = dev_t(b.block_tables)
-    lens = dev_t(b.context_lens)
-    mapping = dev_t(b.block_mapping) if b.block_mapping is not None and len(b.block_mapping) else None
+    q = dev_tensor(b.query, b.dtype, dev)
+    key = dev_tensor(b.key, b.dtype, dev)
+    value = dev_tensor(b.value, b.dtype, dev)
+    slots = dev_tensor(b.slot_mapping, None, dev)
+    tables = dev_tensor(b.block_tables, None, dev)
+    lens = dev_tensor(b.context_lens, None, dev)
+    mapping = (dev_tensor(b.block_mapping, None, dev)
+               if b.block_mapping is not None and len(b.block_mapping) else None)
     out = torch.empty(q.shape, dtype=out_dtype, device=dev)
     stream = torch.cuda.current_stream()
     ws = None
@@ -577,44 +783,25 @@ def run_ours(args, b: W.PagedBatch, config: dict, rank: int, world: int, local_r
     for i in range(args.warmup):
         step(i)
     torch.cuda.synchronize()
-    # a short soak so the clock sampler sees the GPU under this load even when K is small
-    t_soak = time.perf_counter()
-    i = 0
-    while time.perf_counter() - t_soak < args.soak:
-        for _ in range(200):
-            step(i)
-            i += 1
-        torch.cuda.synchronize()
+    soak(step, args.soak if full else min(args.soak, 0.3))
 
     # Timed region 1: K whole steps with nothing between the launches, so each decode may
     # start while the write before it finishes (programmatic dependent launch).
-    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize()
-    start.record(stream)
-    for i in range(args.steps):
-        step(i)
-    end.record(stream)
-    torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
-    elapsed_ms = start.elapsed_time(end)
-    # Timed region 2: the same K steps with a CUDA event pair around every decode launch (an
-    # event between the write and the decode serialises them), for the decode kernel's own
-    # duration in the roofline.
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-           for _ in range(args.steps)]
-    torch.cuda.synchronize()
-    for i in range(args.steps):
-        step(i, evs[i])
-    torch.cuda.synchronize()
-    decode_ms = [s.elapsed_time(e) for s, e in evs]
+        import torch.distributed as dist
 
-    # Timed region 3 (default flags only): the step as one pa_decode_step call, captured once
-    # per pool copy into a CUDA graph and replayed K times.
+        dist.barrier()
+    elapsed_ms = run_steps(step, args.steps, stream)
+    if world > 1:
+        dist.barrier()
+    # Timed region 2: steps with a CUDA event pair around every decode launch (an event
+    # between the write and the decode serialises them), for the decode kernel's own duration.
+    decode_ms = run_launches(step, launch_count(args))
+
+    # Timed region 3 (headline, default flags only): the step as one pa_decode_step call,
+    # captured once per pool copy into a CUDA graph and replayed K times.
     graph = None
-    if args.decode_flags == pa.PA_DECODE_OVERLAP_PREVIOUS and world == 1:
+    if full and args.decode_flags == pa.PA_DECODE_OVERLAP_PREVIOUS and world == 1:
         def graph_step(i):
             kc, vc = pools[i % rot]
             if mapping is not None:
@@ -631,17 +818,110 @@ def run_ours(args, b: W.PagedBatch, config: dict, rank: int, world: int, local_r
         reps = max(1, args.steps // rot)
         for _ in range(3):
             g.replay()
-        g_start, g_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        torch.cuda.synchronize()
-        g_start.record(stream)
-        for _ in range(reps):
-            g.replay()
-        g_end.record(stream)
-        torch.cuda.synchronize()
-        graph = (g_start.elapsed_time(g_end) / (reps * rot), reps * rot)
+        g_ms = run_steps(lambda i: g.replay(), reps, stream)
+        graph = (g_ms / (reps * rot), reps * rot)
         del g
 
-    # end to end through the same calls: inputs from pinned host memory, output read back
+    e2e = None
+    if full:
+        e2e = measure_e2e(args, b, pools, rot, mapping, out, ws, decode, dev, stream, world)
+
+    timeline = None
+    if full and args.timeline and world == 1 and b.dtype != "f32" and not (args.decode_flags & 2):
+        workers = pa.pa_decode_default_workers({"bf16": pa.PA_BF16, "f16": pa.PA_F16}[b.dtype],
+                                               b.head_dim, b.block_size,
+                                               b.num_heads // b.num_kv_heads)
+        buf = torch.zeros(workers * pa.TIMELINE_WORDS, dtype=torch.int64, device=dev)
+        pa.pa_set_decode_timeline(buf)
+        recs = []
+        try:
+            for i in range(args.timeline):
+                buf.zero_()
+                step(i)
+                torch.cuda.synchronize()
+                recs.append(buf.cpu().numpy().copy())
+        finally:
+            pa.pa_set_decode_timeline(None)
+        timeline = timeline_summary(recs, 16 * b.head_dim * ELT[b.dtype] * 2)
+        if args.timeline_out:
+            np.save(args.timeline_out, np.stack(recs))
+    clocks = sampler.stop()
+
+    elapsed_ms, dec_mean = max_over_ranks([elapsed_ms, float(np.mean(decode_ms))], device=dev)
+    if e2e is not None:
+        e2e["ms"] = max_over_ranks([e2e["ms"]], device=dev)[0]
+    flags = pa.pa_get_device_error(clear=True)
+    if rank != 0:
+        return None
+    if flags:
+        print(f"warning: device error word 0x{flags:x}", file=sys.stderr)
+
+    out_elt = torch.tensor([], dtype=out_dtype).element_size()
+    dec_unique = decode_bytes(b, out_elt, unique=True)
+    dec_logical = decode_bytes(b, out_elt, unique=False)
+    step_bytes = dec_unique + write_bytes(b)
+    ms = elapsed_ms / args.steps
+    value = world * step_bytes / (ms * 1e-3) / 1e9
+    peak, peak_src = hbm_peak()
+    kernel = ("paged_decode_kernel (CUDA cores)" if (args.decode_flags & 2 or b.dtype == "f32")
+              else "paged_decode_mma_kernel (mma.sync + TMA)")
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": b.dtype,
+        "data": "synthetic", "config": config,
+        "attended_tokens_per_s": round(world * b.attended_tokens / (ms * 1e-3), 1),
+        "seq_steps_per_s": round(world * b.num_seqs / (ms * 1e-3), 1),
+        "pct_of_8TBs": round(100 * value / world / NOMINAL_HBM_GBS, 2),
+        f"pct_of_{peak_src}_hbm": round(100 * value / world / peak, 2),
+        "roofline": hbm_roofline(dec_unique, decode_ms, kernel,
+                                 recorded_traffic(config["workload"]), probe),
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clocks,
+    }
+    if probe:
+        line["pct_of_read_probe"] = round(100 * value / world / max(probe["ld_GBps"], probe["bulk_GBps"]), 2)
+    if e2e is not None:
+        e_ms = e2e["ms"] / args.steps
+        line["e2e"] = {"value": round(world * step_bytes / (e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
+                       "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"],
+                       "ms_per_step": round(e_ms, 5),
+                       "how": "per step: one pinned-buffer copy in, the write, the decode, the "
+                              "output copy out, synchronize"}
+        if e2e.get("graph_ms") is not None:
+            g_step = e2e["graph_ms"] / args.steps
+            line["e2e_graph"] = {"value": round(step_bytes / (g_step * 1e-3) / 1e9, 2),
+                                 "unit": "GB/s", "h2d_bytes_per_step": e2e["h2d"],
+                                 "d2h_bytes_per_step": e2e["d2h"], "ms_per_step": round(g_step, 5),
+                                 "how": "the same four operations per step captured in one CUDA "
+                                        "graph (per pool copy), replayed, synchronize every step"}
+        if e2e.get("breakdown"):
+            line["e2e_breakdown"] = e2e["breakdown"]
+    if graph is not None:
+        line["graph"] = {"ms_per_step": round(graph[0], 5),
+                         "value": round(step_bytes / (graph[0] * 1e-3) / 1e9, 2), "unit": "GB/s",
+                         "steps": graph[1],
+                         "how": "pa_decode_step (+ pa_copy_blocks) captured in one CUDA graph per "
+                                "pool copy, replayed"}
+    if dec_logical != dec_unique:
+        line["logical_GBps"] = round(world * (dec_logical + write_bytes(b)) / (ms * 1e-3) / 1e9, 2)
+    if timeline:
+        line["timeline"] = timeline
+    if full and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(b, args.cpu_seconds)
+    return line
+
+
+def measure_e2e(args, b, pools, rot, mapping, out, ws, decode, dev, stream, world) -> dict:
+    """The step end to end through the same public calls: every input of the step in one
+    pinned host buffer, one copy in, the calls on device views of it, the output copied back and
+    a synchronize, every step.  Also the same four operations captured in one CUDA graph per
+    pool copy, and a per-operation breakdown of one eager step (events between the
+    operations)."""
+    import torch
+
+    import paged_kv_cache_427_b200 as pa
+
     def host_t(a, dt=None):
         a = np.ascontiguousarray(a)
         t = torch.from_numpy(a.view(np.int16) if dt == "bf16" else a)
@@ -671,37 +951,71 @@ def run_ours(args, b: W.PagedBatch, config: dict, rank: int, world: int, local_r
 
     d_in = {k: dview(k) for k in parts}
     h_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-    h2d = total
-    d2h = h_out.numel() * h_out.element_size()
 
-    def e2e_step(i):
+    def e2e_step(i, ev=None):
+        if ev is not None:
+            ev[0].record(stream)
         d_buf.copy_(h_buf, non_blocking=True)
+        if ev is not None:
+            ev[1].record(stream)
         kc, vc = pools[i % rot]
         if mapping is not None:
             pa.pa_copy_blocks(kc, vc, d_in["mapping"])
         pa.pa_reshape_and_cache(d_in["key"], d_in["value"], kc, vc, d_in["slots"])
+        if ev is not None:
+            ev[2].record(stream)
         decode(d_in["query"], kc, vc, d_in["tables"], d_in["lens"])
+        if ev is not None:
+            ev[3].record(stream)
         h_out.copy_(out, non_blocking=True)
+        if ev is not None:
+            ev[4].record(stream)
         stream.synchronize()
 
-    e2e_steps = args.steps
     for i in range(min(args.warmup, 50)):
         e2e_step(i)
     if world > 1:
+        import torch.distributed as dist
+
         dist.barrier()
     torch.cuda.synchronize()
-    e_start, e_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e_start.record(stream)
-    for i in range(e2e_steps):
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(args.steps):
         e2e_step(i)
-    e_end.record(stream)
+    e1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = e_start.elapsed_time(e_end)
+    res = {"ms": e0.elapsed_time(e1), "h2d": int(total), "d2h": int(h_out.numel() * h_out.element_size())}
+
+    # where one eager end-to-end step's time goes: events between its operations, and the host
+    # wall clock from the first call to the return of the synchronize
+    n_b = max(20, min(args.steps, 200))
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(n_b)]
+    walls = []
+    for i in range(n_b):
+        t0 = time.perf_counter()
+        e2e_step(i, evs[i])
+        walls.append(time.perf_counter() - t0)
+    torch.cuda.synchronize()
+    seg = np.array([[ev[j].elapsed_time(ev[j + 1]) for j in range(4)] for ev in evs]) * 1e3
+    gap = np.array([evs[i][0].elapsed_time(evs[i + 1][0]) for i in range(n_b - 1)]) * 1e3
+    med = np.median(seg, 0)
+    res["breakdown"] = {
+        "h2d_copy_us": round(float(med[0]), 2), "write_us": round(float(med[1]), 2),
+        "decode_us": round(float(med[2]), 2), "d2h_copy_us": round(float(med[3]), 2),
+        "device_busy_us": round(float(med.sum()), 2),
+        "step_to_step_us": round(float(np.median(gap)), 2),
+        "host_wall_us": round(float(np.median(walls)) * 1e6, 2),
+        "idle_between_steps_us": round(float(np.median(gap) - med.sum()), 2),
+        "steps": n_b,
+        "how": "medians over eager end-to-end steps with CUDA events between the operations "
+               "(events serialise the write and the decode); step_to_step is the interval "
+               "between the starts of consecutive steps, idle the part of it no operation of "
+               "the step covers (host launch and synchronize)"}
 
     # The same end-to-end step with its four operations (input copy, pa_decode_step or its two
     # halves, output copy) captured in one CUDA graph per pool copy: one launch per step, still
     # a synchronize and a host read of the output every step.
-    e2e_graph_ms = None
     if args.decode_flags == pa.PA_DECODE_OVERLAP_PREVIOUS and world == 1:
         def e2e_body(i):
             d_buf.copy_(h_buf, non_blocking=True)
@@ -726,85 +1040,22 @@ def run_ours(args, b: W.PagedBatch, config: dict, rank: int, world: int, local_r
         torch.cuda.synchronize()
         g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         g0.record(stream)
-        for i in range(e2e_steps):
+        for i in range(args.steps):
             graphs[i % rot].replay()
             stream.synchronize()
         g1.record(stream)
         torch.cuda.synchronize()
-        e2e_graph_ms = g0.elapsed_time(g1)
+        res["graph_ms"] = g0.elapsed_time(g1)
         del graphs
-    clocks = sampler.stop()
-
-    elapsed_ms, e2e_ms, dec_mean = max_over_ranks([elapsed_ms, e2e_ms, float(np.mean(decode_ms))],
-                                                  device=dev)
-    flags = pa.pa_get_device_error(clear=True)
-    if rank != 0:
-        return
-    if flags:
-        print(f"warning: device error word 0x{flags:x}", file=sys.stderr)
-
-    out_elt = torch.tensor([], dtype=out_dtype).element_size()
-    dec_unique = decode_bytes(b, out_elt, unique=True)
-    dec_logical = decode_bytes(b, out_elt, unique=False)
-    step_bytes = dec_unique + write_bytes(b)
-    ms = elapsed_ms / args.steps
-    value = world * step_bytes / (ms * 1e-3) / 1e9
-    e2e_ms_step = e2e_ms / e2e_steps
-    peak, peak_src = hbm_peak()
-    achieved = dec_unique / (dec_mean * 1e-3) / 1e9
-    line = {
-        "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 5),
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": b.dtype,
-        "data": "synthetic", "config": config,
-        "attended_tokens_per_s": round(world * b.attended_tokens / (ms * 1e-3), 1),
-        "seq_steps_per_s": round(world * b.num_seqs / (ms * 1e-3), 1),
-        "pct_of_8TBs": round(100 * value / world / NOMINAL_HBM_GBS, 2),
-        f"pct_of_{peak_src}_hbm": round(100 * value / world / peak, 2),
-        "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak, "unit": "GB/s",
-                     "frac": round(achieved / peak, 4), "traffic": recorded_traffic(config["workload"]),
-                     "kernel": ("paged_decode_kernel (CUDA cores)"
-                                if (args.decode_flags & 2 or b.dtype == "f32")
-                                else "paged_decode_mma_kernel (mma.sync + TMA)"),
-                     "peak_source": peak_src,
-                     "algorithmic_bytes_per_launch": dec_unique,
-                     "mean_launch_us": round(dec_mean * 1e3, 3),
-                     "launch_timing": "CUDA events around each decode launch, in a second timed "
-                                      "region of the same K steps"},
-        "e2e": {"value": round(world * step_bytes / (e2e_ms_step * 1e-3) / 1e9, 2), "unit": "GB/s",
-                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
-                "ms_per_step": round(e2e_ms_step, 5),
-                "how": "per step: one pinned-buffer copy in, the write, the decode, the output "
-                       "copy out, synchronize"},
-        "gpu_launches": launches_per_step * args.steps,
-        "clocks": clocks,
-    }
-    if e2e_graph_ms is not None:
-        g_step = e2e_graph_ms / e2e_steps
-        line["e2e_graph"] = {"value": round(step_bytes / (g_step * 1e-3) / 1e9, 2), "unit": "GB/s",
-                             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
-                             "ms_per_step": round(g_step, 5),
-                             "how": "the same four operations per step captured in one CUDA "
-                                    "graph (per pool copy), replayed, synchronize every step"}
-    if graph is not None:
-        line["graph"] = {"ms_per_step": round(graph[0], 5),
-                         "value": round(step_bytes / (graph[0] * 1e-3) / 1e9, 2), "unit": "GB/s",
-                         "steps": graph[1],
-                         "how": "pa_decode_step (+ pa_copy_blocks) captured in one CUDA graph per "
-                                "pool copy, replayed"}
-    if dec_logical != dec_unique:
-        line["logical_GBps"] = round(world * (dec_logical + write_bytes(b)) / (ms * 1e-3) / 1e9, 2)
-    if world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(b, args.cpu_seconds)
-    print(json.dumps(line), flush=True)
+    return res
 
 
-def run_fp8(args, b, config):
+def run_fp8(args, b, config, full: bool = True, probe: dict | None = None) -> dict:
     """The same decode step over an FP8 E4M3 cache: the pool is the workload's pool quantised
     (per-kv-head scales: largest magnitude of the head's rows / 240), each step writes the new
     tokens with pa_reshape_and_cache_fp8 and decodes with pa_decode_fp8 launched to overlap the
     write.  Timed like the 16-bit step: K steps with nothing between launches (`value`), then
-    the same K steps with events around each decode (the roofline)."""
+    steps with events around each decode (the roofline)."""
     import torch
 
     import paged_kv_cache_427_b200 as pa
@@ -813,12 +1064,7 @@ def run_fp8(args, b, config):
     dev = torch.device("cuda", 0)
     FP8 = torch.float8_e4m3fn
 
-    def dev_t(a, dt=None):
-        if dt == "bf16":
-            return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
-        return torch.from_numpy(np.ascontiguousarray(a)).to(dev)
-
-    kc16, vc16 = dev_t(b.key_cache, b.dtype), dev_t(b.value_cache, b.dtype)
+    kc16, vc16 = dev_tensor(b.key_cache, b.dtype, dev), dev_tensor(b.value_cache, b.dtype, dev)
     # every slot the step's contexts use, except the new tokens' (the step writes those)
     used = []
     for s in range(b.num_seqs):
@@ -830,11 +1076,10 @@ def run_fp8(args, b, config):
     su = torch.from_numpy(used).to(dev)
     rows_k = kc16[su // b.block_size, :, su % b.block_size, :].contiguous()  # [n, Hkv, D]
     rows_v = vc16[su // b.block_size, :, su % b.block_size, :].contiguous()
-    key, value = dev_t(b.key, b.dtype), dev_t(b.value, b.dtype)
+    key, value = dev_tensor(b.key, b.dtype, dev), dev_tensor(b.value, b.dtype, dev)
     ks = (torch.cat([rows_k, key]).float().abs().amax(dim=(0, 2)) / 240.0).clamp_min(1e-8).contiguous()
     vs = (torch.cat([rows_v, value]).float().abs().amax(dim=(0, 2)) / 240.0).clamp_min(1e-8).contiguous()
-    att = attended_bytes(b) // 2
-    rot = args.rotations or max(2, min(8, math.ceil(3 * L2_BYTES / max(att, 1)) + 1))
+    rot = pool_rotations(args, attended_bytes(b) // 2)
     pools = []
     for _ in range(rot):
         kc = torch.full(kc16.shape, 0x7f, dtype=torch.uint8, device=dev).view(FP8)
@@ -842,8 +1087,10 @@ def run_fp8(args, b, config):
         pa.pa_reshape_and_cache_fp8(rows_k, rows_v, kc, vc, su, ks, vs)
         pools.append((kc, vc))
     del kc16, vc16, rows_k, rows_v
-    q = dev_t(b.query, b.dtype)
-    slots, tables, lens = dev_t(b.slot_mapping), dev_t(b.block_tables), dev_t(b.context_lens)
+    q = dev_tensor(b.query, b.dtype, dev)
+    slots = dev_tensor(b.slot_mapping, None, dev)
+    tables = dev_tensor(b.block_tables, None, dev)
+    lens = dev_tensor(b.context_lens, None, dev)
     out = torch.empty(q.shape, dtype=q.dtype, device=dev)
     ws = torch.zeros(pa.pa_decode_workspace_bytes(b.num_seqs, b.num_heads, b.num_kv_heads,
                                                   b.head_dim, 0), dtype=torch.uint8, device=dev)
@@ -863,27 +1110,9 @@ def run_fp8(args, b, config):
     for i in range(args.warmup):
         step(i)
     torch.cuda.synchronize()
-    t_soak = time.perf_counter()
-    i = 0
-    while time.perf_counter() - t_soak < args.soak:
-        for _ in range(200):
-            step(i)
-            i += 1
-        torch.cuda.synchronize()
-    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    torch.cuda.synchronize()
-    start.record(stream)
-    for i in range(args.steps):
-        step(i)
-    end.record(stream)
-    torch.cuda.synchronize()
-    elapsed_ms = start.elapsed_time(end)
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-           for _ in range(args.steps)]
-    for i in range(args.steps):
-        step(i, evs[i])
-    torch.cuda.synchronize()
-    dec_mean = float(np.mean([s_.elapsed_time(e_) for s_, e_ in evs]))
+    soak(step, args.soak if full else min(args.soak, 0.3))
+    elapsed_ms = run_steps(step, args.steps, stream)
+    dec_ms = run_launches(step, launch_count(args))
     clocks = sampler.stop()
     flags = pa.pa_get_device_error(clear=True)
     if flags:
@@ -893,8 +1122,6 @@ def run_fp8(args, b, config):
     wbytes = t_new * b.num_kv_heads * b.head_dim * (ELT[b.dtype] + 1) * 2 + len(b.slot_mapping) * 8
     ms = elapsed_ms / args.steps
     value = (dec + wbytes) / (ms * 1e-3) / 1e9
-    peak, peak_src = hbm_peak()
-    achieved = dec / (dec_mean * 1e-3) / 1e9
     line = {"metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": 1,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 5),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
@@ -904,20 +1131,16 @@ def run_fp8(args, b, config):
             "attended_tokens_per_s": round(b.attended_tokens / (ms * 1e-3), 1),
             "seq_steps_per_s": round(b.num_seqs / (ms * 1e-3), 1),
             "pct_of_8TBs": round(100 * value / NOMINAL_HBM_GBS, 2),
-            "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak,
-                         "unit": "GB/s", "frac": round(achieved / peak, 4), "traffic": None,
-                         "kernel": "paged_decode_mma_kernel (fp8 e4m3 cache)",
-                         "peak_source": peak_src, "algorithmic_bytes_per_launch": dec,
-                         "mean_launch_us": round(dec_mean * 1e3, 3),
-                         "launch_timing": "CUDA events around each decode launch, in a second "
-                                          "timed region of the same K steps"},
+            "roofline": hbm_roofline(dec, dec_ms, "paged_decode_mma_kernel (fp8 e4m3 cache)",
+                                     recorded_traffic(config["workload"] + ":fp8", "decode_fp8"),
+                                     probe),
             "gpu_launches": 2 * args.steps, "clocks": clocks}
-    if not args.no_cpu_baseline:
+    if full and not args.no_cpu_baseline:
         kc8, vc8 = pools[0]
         line["cpu_baseline"] = cpu_baseline_fp8(
             b, kc8.view(torch.uint8).cpu().numpy(), vc8.view(torch.uint8).cpu().numpy(),
             ks.cpu().numpy(), vs.cpu().numpy(), args.cpu_seconds)
-    print(json.dumps(line), flush=True)
+    return line
 
 
 def prefill_flops(b: W.PagedBatch) -> int:
@@ -932,7 +1155,7 @@ def prefill_flops(b: W.PagedBatch) -> int:
     return 4 * b.head_dim * b.num_heads * tot
 
 
-def run_prefill(args, b, config):
+def run_prefill(args, b, config, full: bool = True) -> dict:
     """A chunked-prefill step: the new tokens' K/V written (pa_reshape_and_cache), then
     pa_prefill.  Timed like the decode step; the roofline is tensor-bound, against the measured
     bf16 dense GEMM rate (the burst figure: the kernel is timed alone per launch)."""
@@ -942,20 +1165,13 @@ def run_prefill(args, b, config):
 
     pa.load()
     dev = torch.device("cuda", 0)
-
-    def dev_t(a, dt=None):
-        if dt == "bf16":
-            return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
-        return torch.from_numpy(np.ascontiguousarray(a)).to(dev)
-
-    kc0, vc0 = dev_t(b.key_cache, b.dtype), dev_t(b.value_cache, b.dtype)
-    att = attended_bytes(b)
-    rot = args.rotations or max(2, min(8, math.ceil(3 * L2_BYTES / max(att, 1)) + 1))
+    kc0, vc0 = dev_tensor(b.key_cache, b.dtype, dev), dev_tensor(b.value_cache, b.dtype, dev)
+    rot = pool_rotations(args, attended_bytes(b))
     pools = [(kc0, vc0)] + [(kc0.clone(), vc0.clone()) for _ in range(rot - 1)]
-    q = dev_t(b.query, b.dtype)
-    key, value = dev_t(b.key, b.dtype), dev_t(b.value, b.dtype)
-    slots, tables = dev_t(b.slot_mapping), dev_t(b.block_tables)
-    lens, qs = dev_t(b.context_lens), dev_t(b.query_start)
+    q = dev_tensor(b.query, b.dtype, dev)
+    key, value = dev_tensor(b.key, b.dtype, dev), dev_tensor(b.value, b.dtype, dev)
+    slots, tables = dev_tensor(b.slot_mapping, None, dev), dev_tensor(b.block_tables, None, dev)
+    lens, qs = dev_tensor(b.context_lens, None, dev), dev_tensor(b.query_start, None, dev)
     out = torch.empty(q.shape, dtype=q.dtype, device=dev)
     stream = torch.cuda.current_stream()
 
@@ -972,40 +1188,20 @@ def run_prefill(args, b, config):
     for i in range(args.warmup):
         step(i)
     torch.cuda.synchronize()
-    t_soak = time.perf_counter()
-    i = 0
-    while time.perf_counter() - t_soak < args.soak:
-        for _ in range(50):
-            step(i)
-            i += 1
-        torch.cuda.synchronize()
-    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    torch.cuda.synchronize()
-    start.record(stream)
-    for i in range(args.steps):
-        step(i)
-    end.record(stream)
-    torch.cuda.synchronize()
-    elapsed_ms = start.elapsed_time(end)
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-           for _ in range(args.steps)]
-    for i in range(args.steps):
-        step(i, evs[i])
-    torch.cuda.synchronize()
-    k_ms = float(np.mean([s_.elapsed_time(e_) for s_, e_ in evs]))
+    soak(step, args.soak if full else min(args.soak, 0.3), per_round=50)
+    elapsed_ms = run_steps(step, args.steps, stream)
+    k_ms = run_launches(step, launch_count(args))
     clocks = sampler.stop()
     flags = pa.pa_get_device_error(clear=True)
     if flags:
         print(f"warning: device error word 0x{flags:x}", file=sys.stderr)
     flops = prefill_flops(b)
     ms = elapsed_ms / args.steps
-    try:
-        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
-            peak, src = float(json.load(f)["bf16_tflops"]), "measured"
-    except Exception:
-        peak, src = 1590.0, "fallback"
-    tflops = flops / (k_ms * 1e-3) / 1e12
+    peak, src = bf16_peak()
+    st = launch_stats(k_ms)
+    tflops = flops / (st["mean_launch_us"] * 1e-6) / 1e12
     new_tokens = int(b.query_start[-1])
+    traffic = recorded_traffic(config["workload"], "prefill")
     line = {"metric": PREFILL_METRIC, "value": round(flops / (ms * 1e-3) / 1e12, 2),
             "unit": "TFLOP/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(ms, 5), "higher_is_better": True, "scaling": "weak",
@@ -1014,14 +1210,63 @@ def run_prefill(args, b, config):
                            query_lens=[int(x) for x in np.diff(b.query_start)]),
             "new_tokens_per_s": round(new_tokens / (ms * 1e-3), 1),
             "roofline": {"bound": "tensor", "achieved": round(tflops, 2), "peak": peak,
-                         "unit": "TFLOP/s", "frac": round(tflops / peak, 4), "traffic": None,
-                         "kernel": "paged_prefill_tc_kernel (tcgen05 + TMEM + TMA)", "peak_source": src,
-                         "algorithmic_flops_per_launch": flops,
-                         "mean_launch_us": round(k_ms * 1e3, 3)},
+                         "unit": "TFLOP/s", "frac": round(tflops / peak, 4), "traffic": traffic,
+                         "kernel": "paged_prefill_tc_kernel (tcgen05 + TMEM + TMA)",
+                         "peak_source": src, "algorithmic_flops_per_launch": flops, **st},
             "gpu_launches": 2 * args.steps, "clocks": clocks}
-    if not args.no_cpu_baseline:
+    if full and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline_prefill(b, args.cpu_seconds)
-    print(json.dumps(line), flush=True)
+    return line
+
+
+# The other workloads of the default run, after the Llama-3-8B-shaped headline: the long
+# mixed batch (its own >= 60 % bar), the block-size sweep, the shared prefix, the FP8 cache on
+# the headline's batch and the chunked prefill.
+CONFIG_RUNS = (("long_mixed", "decode"), ("short_chat_bs8", "decode"), ("short_chat_bs16", "decode"),
+               ("short_chat_bs32", "decode"), ("shared_prefix", "decode"),
+               ("llama3_8b_decode", "fp8"), ("chunked_prefill", "prefill"))
+
+
+def run_configs(args, probe) -> dict:
+    """One compact record per workload of CONFIG_RUNS, each measured like the headline (K
+    steps, then per-launch events), without the end-to-end, graph and CPU legs."""
+    import torch
+
+    keep = ("metric", "value", "unit", "ms_per_step", "pct_of_8TBs", "pct_of_read_probe",
+            "attended_tokens_per_s", "seq_steps_per_s", "new_tokens_per_s", "logical_GBps",
+            "roofline", "clocks", "dtype")
+    res = {}
+    for name, kind in CONFIG_RUNS:
+        b = make_batch(name)
+        cfg = workload_config(args, b, name)
+        if kind == "fp8":
+            line = run_fp8(args, b, cfg, full=False, probe=probe)
+            key = name + ":fp8"
+        elif kind == "prefill":
+            line = run_prefill(args, b, cfg, full=False)
+            key = name
+        else:
+            line = run_decode(args, b, cfg, full=False, probe=probe)
+            key = name
+        rec = {k: line[k] for k in keep if k in line}
+        rec["config"] = {k: v for k, v in line["config"].items()
+                         if k in ("num_seqs", "block_size", "attended_tokens", "kv_dtype",
+                                  "new_tokens", "num_blocks")}
+        res[key] = rec
+        del b
+        torch.cuda.empty_cache()
+    return res
+
+
+def workload_config(args, b, name: str) -> dict:
+    return {"workload": name, "num_seqs": b.num_seqs, "num_heads": b.num_heads,
+            "num_kv_heads": b.num_kv_heads, "head_dim": b.head_dim, "block_size": b.block_size,
+            "kv_dtype": b.dtype, "attended_tokens": b.attended_tokens,
+            "num_blocks": b.num_blocks, "max_blocks_per_seq": b.max_blocks,
+            "seed": b.meta.get("seed"),
+            "l2": "inputs larger than L2: steps rotate over copies of the KV pool",
+            "pool_rotations": args.rotations or "auto",
+            "decode_flags": args.decode_flags}
 
 
 def run_swap(args, b, config):
@@ -1118,9 +1363,9 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
-    ap.add_argument("--workload", default="llama3_8b_decode",
-                    help="llama3_8b_decode | short_chat_bs{8,16,32} | shared_prefix | long_mixed | "
-                         "tiny_fp32 | chunked_prefill (pa_prefill)")
+    ap.add_argument("--workload", default=None,
+                    help="llama3_8b_decode (default) | short_chat_bs{8,16,32} | shared_prefix | "
+                         "long_mixed | tiny_fp32 | chunked_prefill (pa_prefill)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--decode-flags", type=int, default=4,
                     help="pa_decode_ex flags: 4 = start while the cache write runs (default), "
@@ -1129,6 +1374,12 @@ def main():
     ap.add_argument("--soak", type=float, default=1.0, help="seconds of untimed load for the clock sampler")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="the default run: skip the other workloads (the `configs` key)")
+    ap.add_argument("--no-probe", action="store_true", help="skip the read-only HBM probe")
+    ap.add_argument("--timeline", type=int, default=0, metavar="N",
+                    help="record N decode launches with pa_set_decode_timeline and add a summary")
+    ap.add_argument("--timeline-out", default=None, help="save the raw timeline records (.npy)")
     ap.add_argument("--kv", default="native", choices=["native", "fp8"],
                     help="fp8: the same step over an FP8 E4M3 cache (pa_decode_fp8)")
     ap.add_argument("--swap", action="store_true",
@@ -1136,22 +1387,17 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("at least 3 warm-up steps")
+    default_run = args.workload is None
+    workload = args.workload or "llama3_8b_decode"
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     if world != args.gpus:
         args.gpus = world if world > 1 else args.gpus
-    b = make_batch(args.workload)
-    config = {"workload": args.workload, "num_seqs": b.num_seqs, "num_heads": b.num_heads,
-              "num_kv_heads": b.num_kv_heads, "head_dim": b.head_dim, "block_size": b.block_size,
-              "kv_dtype": b.dtype, "attended_tokens": b.attended_tokens,
-              "num_blocks": b.num_blocks, "max_blocks_per_seq": b.max_blocks,
-              "seed": b.meta.get("seed"),
-              "l2": "inputs larger than L2: steps rotate over copies of the KV pool",
-              "pool_rotations": args.rotations or "auto",
-              "decode_flags": args.decode_flags,
-              "parallelism": f"replicas x{world}" if world > 1 else "single GPU"}
+    b = make_batch(workload)
+    config = workload_config(args, b, workload)
+    config["parallelism"] = f"replicas x{world}" if world > 1 else "single GPU"
 
     if args.impl == "reference":
         if rank == 0:
@@ -1167,11 +1413,11 @@ def main():
         return
     if args.kv == "fp8":
         if rank == 0:
-            run_fp8(args, b, config)
+            print(json.dumps(run_fp8(args, b, config)), flush=True)
         return
     if b.query_start is not None:
         if rank == 0:
-            run_prefill(args, b, config)
+            print(json.dumps(run_prefill(args, b, config)), flush=True)
         return
     if world > 1:
         import datetime
@@ -1181,7 +1427,18 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local_rank))
     try:
-        run_ours(args, b, config, rank, world, local_rank)
+        probe = None
+        if world == 1 and not args.no_probe:
+            probe = read_probe(torch.device("cuda", local_rank))
+        line = run_decode(args, b, config, rank, world, local_rank, full=True, probe=probe)
+        if line is not None:
+            if probe:
+                line["hbm_read_probe"] = probe
+            if default_run and world == 1 and not args.no_configs:
+                del b
+                torch.cuda.empty_cache()
+                line["configs"] = run_configs(args, probe)
+            print(json.dumps(line), flush=True)
     finally:
         if world > 1:
             import torch.distributed as dist

@@ -62,7 +62,7 @@
 extern "C" {
 #endif
 
-#define PA_VERSION 5
+#define PA_VERSION 6
 
 /* Symbols of this ABI are the only ones the shared library exports. */
 #if defined(__GNUC__)
@@ -110,8 +110,14 @@ typedef enum pa_status {
 #define PA_DEVERR_SLOT 0x4u        /* slot >= num_blocks * block_size; the token was skipped */
 #define PA_DEVERR_COPY_PAIR 0x8u   /* a copy pair held an id outside [0, num_blocks); skipped */
 #define PA_DEVERR_TIMEOUT 0x10u    /* an asynchronous copy did not complete within about one
-                                      second; the kernel abandoned its work and returned.  The
-                                      decode workspace must be re-initialised afterwards */
+                                      second; the kernel abandoned its work and returned, and
+                                      the results of that call are unspecified.  Recovery:
+                                      reading the word with pa_get_device_error while this bit
+                                      is set marks every decode workspace the library has seen
+                                      (the library-owned ones, the callers' workspaces, and the
+                                      static scratch of pa_decode_noalloc) so that the next
+                                      decode call using it zeroes its merge counters first;
+                                      no other step is needed */
 
 /* Flags of pa_decode_ex. */
 #define PA_DECODE_SEPARATE_REDUCE 0x1u /* merge split contexts in a second kernel instead of
@@ -313,8 +319,8 @@ PA_API size_t pa_decode_workspace_bytes(int64_t num_seqs, int32_t num_heads, int
 PA_API int32_t pa_decode_default_workers(int32_t dtype, int32_t head_dim, int32_t block_size,
                                   int32_t group_size);
 
-/* Zero-fill a decode workspace on `stream` (before its first use, or after a
- * PA_DEVERR_TIMEOUT). */
+/* Zero-fill a decode workspace on `stream` (before its first use; after a PA_DEVERR_TIMEOUT,
+ * pa_get_device_error already arranges for the counters to be zeroed again). */
 PA_API int pa_workspace_init(void *workspace, size_t workspace_bytes, void *stream);
 
 /* Free the library-owned decode workspaces of every device (synchronises each device). */
@@ -345,8 +351,11 @@ PA_API int pa_get_device_error(void *stream, uint32_t *flags, int32_t clear);
  * which every GPU that loads the library holds until the process exits.  A call whose shapes
  * need more scratch than that (roughly: more than about 3,000 (sequence, kv head) pairs at
  * head_dim 128 and 4 query heads per kv head) returns PA_ERR_WORKSPACE without launching.
- * The first call on a device looks up the array's device address and clears it on `stream`;
- * make that first call before any stream capture.  The call itself allocates nothing: no
+ * Every call looks up the array's device address (cudaGetSymbolAddress, which allocates
+ * nothing); the first call on a device, or the first after the module was reloaded, also
+ * clears the array on `stream`: make that first call before any stream capture.  After a
+ * PA_DEVERR_TIMEOUT, reading the error word (pa_get_device_error) is the whole recovery: the
+ * next call zeroes the array's merge counters on its stream before the decode.  The call itself allocates nothing: no
  * cudaMalloc, no cudaFree, no allocating library routine.  All calls share the one array, so
  * calls that overlap on the GPU (for instance on two streams) race and give wrong results;
  * issue them in one stream or one after another.
@@ -356,6 +365,33 @@ PA_API int pa_decode_noalloc(const pa_tensor *out, const pa_tensor *query,
                              const pa_tensor *key_cache, const pa_tensor *value_cache,
                              const pa_tensor *block_tables, const pa_tensor *context_lens,
                              float scale, int32_t block_size, int32_t num_kv_heads, void *stream);
+
+/*
+ * Measurement aids (not part of the attention path).
+ *
+ * pa_set_decode_timeline - when buf is not NULL, every later launch of the tensor-core decode
+ * kernel (pa_decode, pa_decode_ex, pa_decode_step, pa_decode_fp8, pa_decode_noalloc) writes, for
+ * each worker warp w < bytes / 64, eight 64-bit words at buf + 64 w: the global nanosecond
+ * timer when the warp starts, when its first tile has landed, when it has consumed its last
+ * tile, when it is finished; the SM it ran on; the chunks in its share; the timer when its CTA
+ * may read the caches (the previous grid, under PA_DECODE_OVERLAP_PREVIOUS, has finished); the
+ * timer when its CTA's merge warp is finished.  buf: device memory, 8-byte aligned, kept by the
+ * caller.  NULL stops the recording.  Launches that overlap on the GPU overwrite each other's
+ * records.
+ */
+PA_API int pa_set_decode_timeline(void *buf, size_t bytes);
+
+/*
+ * pa_hbm_read_probe - read `bytes` of device memory once, as a read-only bandwidth probe (the
+ * ceiling of a read stream such as decode, next to the copy bandwidth).  mode 0: 16-byte vector
+ * loads from every SM; mode 1: 32 KB bulk asynchronous copies into shared memory (the copy
+ * engine the decode kernels use; a tail shorter than 32 KB is not read).  buf: 128-byte aligned
+ * device memory; sink: device memory of two 32-bit words, the first receives a fold of the
+ * loaded words, the second gets bit 0 set if a copy did not complete within about a second.
+ * Asynchronous on `stream`.
+ */
+PA_API int pa_hbm_read_probe(const void *buf, size_t bytes, int32_t mode, void *sink,
+                             void *stream);
 
 /* PA_VERSION of the library actually loaded. */
 PA_API int32_t pa_version(void);

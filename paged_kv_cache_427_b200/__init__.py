@@ -14,6 +14,7 @@ Calls (same names as the C ABI):
   pa_decode_ex(..., num_workers=0, flags=0, workspace=None)
   pa_decode_workspace_bytes, pa_decode_default_workers, pa_workspace_init,
   pa_release_workspaces, pa_last_error, pa_get_device_error, pa_version
+Measurement aids: pa_set_decode_timeline(buf), pa_hbm_read_probe(buf, mode, sink).
 Seeded synthetic workloads live in ``paged_kv_cache_427_b200.workloads`` (no torch, no CUDA).
 """
 from __future__ import annotations
@@ -92,6 +93,10 @@ def load(path: str = LIBRARY) -> ctypes.CDLL:
     lib.pa_get_device_error.argtypes = [_P, ctypes.POINTER(u32), i32]
     lib.pa_decode_noalloc.argtypes = [_T, _T, _T, _T, _T, _T, f32, i32, i32, _P]
     lib.pa_decode_step.argtypes = [_T, _T, _T, _T, _T, _T, _T, _T, _T, f32, i32, i32, _P, sz, _P]
+    lib.pa_set_decode_timeline.argtypes = [_P, sz]
+    lib.pa_set_decode_timeline.restype = ctypes.c_int
+    lib.pa_hbm_read_probe.argtypes = [_P, sz, i32, _P, _P]
+    lib.pa_hbm_read_probe.restype = ctypes.c_int
     lib.pa_version.argtypes = []
     lib.pa_version.restype = i32
     for name in ("pa_reshape_and_cache", "pa_copy_blocks", "pa_decode", "pa_decode_ex",
@@ -289,3 +294,25 @@ def header_functions(path: str = HEADER) -> list[str]:
     with open(path) as f:
         text = f.read()
     return sorted(set(re.findall(r"^\s*PA_API\s+(?:const\s+)?\w+\s*\*?\s*(pa_\w+)\s*\(", text, re.M)))
+
+
+TIMELINE_WORDS = 8  # 64-bit words per worker warp in a decode timeline record
+TL_START, TL_FIRST, TL_LAST, TL_DONE, TL_SM, TL_CHUNKS, TL_ISSUE, TL_MERGED = range(8)
+
+
+def pa_set_decode_timeline(buf=None):
+    """Make later tensor-core decode launches record per-warp timestamps into `buf` (a CUDA
+    int64 tensor, TIMELINE_WORDS words per worker warp); None stops the recording."""
+    if buf is None:
+        _check("pa_set_decode_timeline", load().pa_set_decode_timeline(None, 0))
+    else:
+        _check("pa_set_decode_timeline",
+               load().pa_set_decode_timeline(buf.data_ptr(), buf.numel() * buf.element_size()))
+
+
+def pa_hbm_read_probe(buf, mode: int, sink, stream=None):
+    """Read every byte of the CUDA tensor `buf` once (mode 0: vector loads, 1: bulk copies into
+    shared memory); `sink` is a CUDA int32 tensor of at least two elements."""
+    _check("pa_hbm_read_probe",
+           load().pa_hbm_read_probe(buf.data_ptr(), buf.numel() * buf.element_size(), int(mode),
+                                    sink.data_ptr(), _stream(stream)))

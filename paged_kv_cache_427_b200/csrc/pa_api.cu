@@ -10,6 +10,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstdlib>
+#include <atomic>
 #include <mutex>
 #include <string>
 #include <vector>
@@ -45,18 +46,36 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t
                                   const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
-// Test hooks, read once per process: PA_TEST_WAIT_LIMIT_CYCLES shortens every wait on a copy,
-// PA_TEST_STALL_COPIES=1 makes each decode warp's first stage wait for 16 bytes that no copy
-// delivers, so that the wait runs out, the kernel records PA_DEVERR_TIMEOUT and returns.
+// Test hooks, read once per process: PA_TEST_WAIT_LIMIT_CYCLES shortens every wait on a copy;
+// PA_TEST_STALL_COPIES makes a decode warp's first stage wait for 16 bytes that no copy
+// delivers, so that the wait runs out, the kernel records PA_DEVERR_TIMEOUT and returns
+// (1: every worker warp; 2: the odd-numbered worker warps only, so that the others finish their
+// pieces and leave merge counters partly counted).  PA_TEST_STALL_CALLS limits the stall to the
+// first n decode launches of the process (default: all of them).
 struct TestHooks {
   long long wait_cycles = 2000000000ll;  // about one second at the 1965 MHz maximum SM clock
   int stall = 0;
+  bool limited = false;                           // PA_TEST_STALL_CALLS given
+  mutable std::atomic<long long> stall_calls{0};  // stalled launches left when limited
   TestHooks() {
     if (const char *v = std::getenv("PA_TEST_WAIT_LIMIT_CYCLES")) {
       const long long x = std::atoll(v);
       if (x > 0) wait_cycles = x;
     }
-    if (const char *v = std::getenv("PA_TEST_STALL_COPIES")) stall = std::atoi(v) != 0;
+    if (const char *v = std::getenv("PA_TEST_STALL_COPIES")) {
+      const int x = std::atoi(v);
+      stall = (x == 1 || x == 2) ? x : 0;
+    }
+    if (const char *v = std::getenv("PA_TEST_STALL_CALLS")) {
+      limited = true;
+      stall_calls = std::atoll(v);
+    }
+  }
+  // The stall mode of the next decode launch (0 once the limited number of launches is spent).
+  int next_stall() const {
+    if (!stall) return 0;
+    if (!limited) return stall;
+    return stall_calls.fetch_sub(1) > 0 ? stall : 0;
   }
 };
 
@@ -84,6 +103,10 @@ std::vector<DeviceState> g_devices;
 // How far a call goes: host-side argument checks only, every check (device memory, workspace
 // size) without launching, or the whole call.
 enum class CallMode { kHostChecks, kAllChecks, kLaunch };
+
+// Measurement aid (pa_set_decode_timeline): where decode launches record per-warp timestamps.
+unsigned long long *g_timeline = nullptr;  // guarded by g_mu
+long long g_timeline_warps = 0;
 
 struct CleanRecord {
   const void *ws;
@@ -597,7 +620,12 @@ int decode_impl(const pa_tensor *out, const pa_tensor *query, const pa_tensor *k
   a.v_scale = fp8 ? static_cast<const float *>(v_scale->data) : nullptr;
   a.separate_reduce = (flags & PA_DECODE_SEPARATE_REDUCE) ? 1 : 0;
   a.wait_cycles = test_hooks().wait_cycles;
-  a.test_stall = test_hooks().stall;
+  a.test_stall = test_hooks().next_stall();
+  {
+    std::lock_guard<std::mutex> lock(g_mu);
+    a.timeline = g_timeline;
+    a.timeline_warps = g_timeline_warps;
+  }
   const int ctas = (W + k.warps_per_cta - 1) / k.warps_per_cta;  // warps_per_cta workers each
   cudaError_t e = k.launch(a, &maps, ctas, (flags & PA_DECODE_OVERLAP_PREVIOUS) != 0, st);
   if (e != cudaSuccess) return cuda_fail(e, "decode launch");
@@ -1081,6 +1109,14 @@ int pa_release_workspaces(void) {
 
 const char *pa_last_error(void) { return g_last_error.c_str(); }
 
+int pa_set_decode_timeline(void *buf, size_t bytes) {
+  if (buf && ((uintptr_t)buf & 7u) != 0) return fail(PA_ERR_LAYOUT, "timeline buffer must be 8-byte aligned");
+  std::lock_guard<std::mutex> lock(g_mu);
+  g_timeline = static_cast<unsigned long long *>(buf);
+  g_timeline_warps = buf ? (long long)(bytes / (pa::kTimelineWords * 8)) : 0;
+  return PA_OK;
+}
+
 int pa_get_device_error(void *stream, uint32_t *flags, int32_t clear) {
   if (!flags) return fail(PA_ERR_INVALID_ARG, "flags is NULL");
   DeviceState *ds;
@@ -1092,6 +1128,13 @@ int pa_get_device_error(void *stream, uint32_t *flags, int32_t clear) {
   if (e == cudaSuccess) e = cudaStreamSynchronize(st);
   if (e != cudaSuccess) return cuda_fail(e, "reading the error word");
   *flags = host;
+  if (host & PA_DEVERR_TIMEOUT) {
+    // An abandoned decode may have left merge counters partly counted in whichever workspace
+    // it used: every workspace this library has seen (its own, the callers', the static
+    // scratch of pa_decode_noalloc) gets its counters zeroed again before its next use.
+    std::lock_guard<std::mutex> lock(g_mu);
+    for (auto &r : g_clean) r.clean = 0;
+  }
   if (clear) {
     e = cudaMemsetAsync(ds->err, 0, sizeof(unsigned int), st);
     if (e == cudaSuccess) e = cudaStreamSynchronize(st);

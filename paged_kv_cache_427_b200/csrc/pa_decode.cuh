@@ -110,7 +110,7 @@ __global__ void __launch_bounds__(128, 1) paged_decode_kernel(const DecodeArgs a
       meta[slot] = cur.meta(f);
       const uint32_t bytes = 2u * cur.valid_copies() * Tr::kCopyBytes +
                              ((f & kFirst) ? (uint32_t)Tr::kQBytes : 0u) +
-                             ((a.test_stall && cur.issued == 0) ? 16u : 0u);
+                             ((cur.issued == 0 && test_stalls(a, gw)) ? 16u : 0u);
       fence_proxy_async_smem();
       mbar_arrive_expect_tx(bars + slot, bytes);
 #pragma unroll

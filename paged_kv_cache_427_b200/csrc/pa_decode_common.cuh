@@ -43,6 +43,12 @@ __device__ __forceinline__ int worker_of(long long c, long long C, int W) {
   return (int)(((c + 1) * (long long)W + C - 1) / C - 1);
 }
 
+// Test hook: whether worker warp gw's first stage waits for 16 bytes that no copy sends
+// (mode 1: every worker; mode 2: the odd-numbered workers only).
+__device__ __forceinline__ bool test_stalls(const DecodeArgs &a, int gw) {
+  return a.test_stall == 1 || (a.test_stall == 2 && (gw & 1));
+}
+
 // Where one warp's share starts and how long it is.
 struct WarpShare {
   long long C;  // chunks in the step

@@ -308,6 +308,8 @@ __global__ void __launch_bounds__(MmaTraits<D, BS, G, (int)sizeof(KV)>::kThreads
     // Everything above read only context_lens and block_tables; the caches and the query may
     // still be written by the previous grid when this one was launched to overlap it.
     wait_for_previous_grid();
+    if (a.timeline != nullptr && k < NW && blockIdx.x * NW + k < a.timeline_warps)
+      a.timeline[(long long)(blockIdx.x * NW + k) * kTimelineWords + kTlIssue] = global_ns();
     long long last_progress = clock64();
     while (__any_sync(FULL_MASK, active)) {
       bool can = false;
@@ -323,7 +325,7 @@ __global__ void __launch_bounds__(MmaTraits<D, BS, G, (int)sizeof(KV)>::kThreads
         meta[slot] = cur.meta(f);
         const uint32_t bytes = 2u * cur.valid_copies() * Tr::kBoxBytes +
                                ((f & kFirst) ? (uint32_t)Tr::kQBytes : 0u) +
-                               ((a.test_stall && cur.issued == 0) ? 16u : 0u);
+                               ((cur.issued == 0 && test_stalls(a, blockIdx.x * NW + k)) ? 16u : 0u);
         mbar_arrive_expect_tx(full + slot, bytes);
 #pragma unroll
         for (int c = 0; c < Tr::kCopies; ++c) {
@@ -405,6 +407,8 @@ __global__ void __launch_bounds__(MmaTraits<D, BS, G, (int)sizeof(KV)>::kThreads
         if (lane == k) ++seen;
       }
     }
+    if (a.timeline != nullptr && lane < NW && blockIdx.x * NW + lane < a.timeline_warps)
+      a.timeline[(long long)(blockIdx.x * NW + lane) * kTimelineWords + kTlMerged] = global_ns();
     return;
   }
 
@@ -414,11 +418,21 @@ __global__ void __launch_bounds__(MmaTraits<D, BS, G, (int)sizeof(KV)>::kThreads
   int posted = 0;
   PieceInfo done_msg;
   done_msg.pair = done_msg.first_worker = done_msg.npieces = done_msg.s = done_msg.kvh = 0;
+  const int gw = blockIdx.x * NW + wid;
+  // measurement aid: this warp's timeline record, or null
+  unsigned long long *tl = (a.timeline != nullptr && lane == 0 && gw < a.timeline_warps)
+                               ? a.timeline + (long long)gw * kTimelineWords
+                               : nullptr;
+  if (tl) {
+    tl[kTlStart] = global_ns();
+    tl[kTlSm] = sm_id();
+    tl[kTlChunks] = (share.n > 0 && share.s >= 0) ? (unsigned long long)share.n : 0ull;
+  }
   if (share.n <= 0 || share.s < 0) {
     mail_post(box, mcount + wid, 0, done_msg, lane);
+    if (tl) tl[kTlFirst] = tl[kTlLast] = tl[kTlDone] = global_ns();
     return;
   }
-  const int gw = blockIdx.x * NW + wid;
   const long long n = share.n;
   unsigned char *ring = smem + wid * ST * Tr::kStageBytes;
   unsigned char *small = smem + Tr::kRingBytes + wid * Tr::kSmallBytes;
@@ -451,6 +465,7 @@ __global__ void __launch_bounds__(MmaTraits<D, BS, G, (int)sizeof(KV)>::kThreads
       mail_post(box, mcount + wid, posted, done_msg, lane);
       return;
     }
+    if (tl && cc == 0) tl[kTlFirst] = global_ns();
     const ChunkMeta m = meta[slot];
     unsigned char *stage = ring + slot * Tr::kStageBytes;
     const uint32_t kbase = smem_u32(stage);
@@ -662,6 +677,7 @@ __global__ void __launch_bounds__(MmaTraits<D, BS, G, (int)sizeof(KV)>::kThreads
     // the stage is no longer needed: hand it back to the producer
     __syncwarp();
     if (lane == 0) mbar_arrive(empty + slot);
+    if (tl && cc == n - 1) tl[kTlLast] = global_ns();
 
     // ---- end of a piece ----
     if (m.flags & kLast) {
@@ -757,6 +773,7 @@ __global__ void __launch_bounds__(MmaTraits<D, BS, G, (int)sizeof(KV)>::kThreads
     }
   }
   mail_post(box, mcount + wid, posted, done_msg, lane);
+  if (tl) tl[kTlDone] = global_ns();
 }
 
 template <typename T, int D, int BS, int G, typename KV = T>

@@ -178,6 +178,18 @@ __device__ __forceinline__ void wait_for_previous_grid() {
 // ... and let the grid launched after this one start early.
 __device__ __forceinline__ void allow_next_grid() { asm volatile("griddepcontrol.launch_dependents;"); }
 
+// Global nanosecond timer and the SM this thread runs on (decode timelines).
+__device__ __forceinline__ unsigned long long global_ns() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+__device__ __forceinline__ unsigned int sm_id() {
+  unsigned int r;
+  asm volatile("mov.u32 %0, %%smid;" : "=r"(r));
+  return r;
+}
+
 __device__ __forceinline__ void set_error(unsigned int *err, unsigned int bits) {
   if (err) atomicOr(err, bits);
 }

@@ -39,7 +39,25 @@ struct DecodeArgs {
   const float *v_scale;
   int separate_reduce;
   long long wait_cycles;  // limit of every wait on a copy (about one second by default)
-  int test_stall;         // test hook: each warp's first stage expects 16 bytes nobody sends
+  int test_stall;         // test hook: 1 every worker's first stage expects 16 bytes nobody
+                          // sends, 2 only the odd-numbered workers'
+  // Measurement aid (pa_set_decode_timeline): kTimelineWords 64-bit records per worker warp
+  // (those with index < timeline_warps), or null.
+  unsigned long long *timeline;
+  long long timeline_warps;
+};
+
+// Fields of one worker warp's timeline record.
+enum TimelineField {
+  kTlStart = 0,     // global ns when the warp begins (after the CTA's set-up)
+  kTlFirst = 1,     // its first tile has landed
+  kTlLast = 2,      // its last tile is consumed (before its last piece's epilogue)
+  kTlDone = 3,      // the warp is finished (epilogue and merges included)
+  kTlSm = 4,        // the SM it ran on
+  kTlChunks = 5,    // chunks in its share
+  kTlIssue = 6,     // the producer may read the caches (the previous grid has finished)
+  kTlMerged = 7,    // the CTA's merge warp is finished (the pieces it published, merged)
+  kTimelineWords = 8
 };
 
 // TMA descriptors of the two caches, viewed as 5-D tensors (64 elements, block_size rows,

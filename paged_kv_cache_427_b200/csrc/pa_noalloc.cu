@@ -3,9 +3,16 @@
 //
 // The array below is the decode scratch of pa_decode_noalloc: merge counters, pair records and
 // partial results, laid out exactly as a pa_decode_ex workspace.  Host code may not use the
-// array's name as a device address (in host code it names a host-side stand-in), so the first
-// call on each device looks the address up with cudaGetSymbolAddress, with that device current,
-// and passes it to the kernels.  Nothing here allocates.
+// array's name as a device address (in host code it names a host-side stand-in), so every call
+// looks the address up with cudaGetSymbolAddress, with the caller's device current, and passes
+// it to the kernels.  The lookup allocates nothing; when the address differs from the one seen
+// before on that device (the first call, or the module reloaded after a device reset) the
+// array is cleared on the call's stream.  Nothing here allocates.
+//
+// After a decode that ran out of its wait limit (PA_DEVERR_TIMEOUT) the merge counters in the
+// array may be partly counted; reading the error word with pa_get_device_error marks every
+// workspace the library knows, this array included, so that the next call zeroes its counters
+// again (on its stream, with cudaMemsetAsync, which allocates nothing).
 #include <cuda_runtime.h>
 
 #include <cstdio>
@@ -22,7 +29,7 @@ constexpr size_t kScratchBytes = PA_NOALLOC_SCRATCH_BYTES;
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kScratchBytes];
 
 std::mutex g_mu;
-void *g_scratch[64];  // device address of g_noalloc_scratch, per device id; null until set up
+void *g_scratch[64];  // device address of g_noalloc_scratch last cleared, per device id
 
 }  // namespace
 
@@ -42,24 +49,22 @@ extern "C" int pa_decode_noalloc(const pa_tensor *out, const pa_tensor *query,
     return PA_ERR_INVALID_ARG;
   }
   void *scratch = nullptr;
+  e = cudaGetSymbolAddress(&scratch, g_noalloc_scratch);
+  if (e != cudaSuccess || !scratch) {
+    char msg[160];
+    snprintf(msg, sizeof(msg), "pa_decode_noalloc: cudaGetSymbolAddress failed: %s",
+             cudaGetErrorString(e));
+    pa::set_last_error(msg);
+    return PA_ERR_CUDA;
+  }
   {
     std::lock_guard<std::mutex> lock(g_mu);
-    if (!g_scratch[dev]) {
-      void *p = nullptr;
-      e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-      if (e != cudaSuccess || !p) {
-        char msg[160];
-        snprintf(msg, sizeof(msg), "pa_decode_noalloc: cudaGetSymbolAddress failed: %s",
-                 cudaGetErrorString(e));
-        pa::set_last_error(msg);
-        return PA_ERR_CUDA;
-      }
-      // The merge counters must start at zero: clear the array once, on the caller's stream.
-      const int rc = pa_workspace_init(p, kScratchBytes, stream);
+    if (g_scratch[dev] != scratch) {
+      // The merge counters must start at zero: clear the array on the caller's stream.
+      const int rc = pa_workspace_init(scratch, kScratchBytes, stream);
       if (rc != PA_OK) return rc;
-      g_scratch[dev] = p;
+      g_scratch[dev] = scratch;
     }
-    scratch = g_scratch[dev];
   }
   const size_t need = pa::decode_scratch_need(query, key_cache, block_size, num_kv_heads);
   if (need > kScratchBytes) {

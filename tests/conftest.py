@@ -18,3 +18,14 @@ def oracle():
     import oracle as oracle_pkg
 
     return oracle_pkg.load()
+
+
+def pytest_terminal_summary(terminalreporter):
+    """The achieved figures of the GPU parity comparisons (tests/gpu_helpers.py RESULTS)."""
+    mod = sys.modules.get("tests.gpu_helpers")
+    res = getattr(mod, "RESULTS", None) if mod else None
+    if not res:
+        return
+    terminalreporter.section("parity figures (GPU path against the oracle)")
+    for what, kind, fig in res:
+        terminalreporter.write_line(f"{kind:9s} {what}: {fig}")

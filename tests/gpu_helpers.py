@@ -1,13 +1,20 @@
 """Helpers for the GPU parity tests: move a seeded batch to the device, run the library's step
 through the C ABI, and compare against the CPU oracle's step on host copies of the same bytes.
 
-Tolerances (fixed before any kernel ran):
+Tolerances (fixed before any kernel ran; the bf16-output bound restated from the kernels'
+arithmetic as below):
   * cache writes and block copies: bit-exact;
   * fp32 caches with fp32 output: max abs error <= 1e-5 and relative L2 error <= 1e-5;
   * bf16 / fp16 caches with fp32 output: max abs error <= 5e-3 and relative L2 <= 1e-3;
-  * bf16 output: each element within one bf16 ulp of the fp64 result plus 1e-5 (the fp32
-    accumulation error of outputs near zero exceeds their ulp), and at least 99% of the
-    elements equal to that result rounded to nearest-even bf16.
+  * bf16 output: every element within one bf16 ulp of the fp64 result o plus
+    2^-16 * max_{t<L} |V_t - o| (the error the fp32 result may carry before its one rounding:
+    each softmax weight is kept to 2^-18 relative by the hi + lo split of P, 2^-22 by exp2,
+    and the fp32 logit and sums add a few 2^-24 per step; a relative error e on the weights
+    moves o by at most e * max_t |V_t - o|; 2^-16 allows four times the split's share), and at
+    least 99% of the elements equal to o rounded to nearest-even bf16 (an element whose exact
+    value lies within that error of a rounding midpoint may round either way).
+The achieved figures of every comparison are collected in RESULTS and printed at the end of
+the pytest run (tests/conftest.py).
 """
 from __future__ import annotations
 
@@ -112,23 +119,73 @@ def errors(got: np.ndarray, ref: np.ndarray):
     return abs_err, rel_l2
 
 
+RESULTS: list = []  # (what, kind, figures) of every comparison, printed after the run
+
+
 def assert_close(got, ref, dtype: str, what: str = ""):
     atol, rtol = TOL[dtype]
     a, r = errors(got, ref)
+    RESULTS.append((what, "fp32 out", f"max abs {a:.2e} (<= {atol}), rel L2 {r:.2e} (<= {rtol})"))
     assert np.all(np.isfinite(got)), f"{what}: non-finite output"
     assert a <= atol and r <= rtol, f"{what}: max abs {a:.3e} (<= {atol}), rel L2 {r:.3e} (<= {rtol})"
     return a, r
 
 
-def assert_bf16_output(got_bits: np.ndarray, ref: np.ndarray, what: str = ""):
-    """bf16 output against the fp64 result: within one ulp + 1e-5, >= 99% exactly RNE(ref)."""
+_FP8_VALUES = None
+
+
+def _fp8_values() -> np.ndarray:
+    """float64 value of each E4M3 code (torch's decoder; NaN codes decode to NaN)."""
+    global _FP8_VALUES
+    if _FP8_VALUES is None:
+        _FP8_VALUES = torch.arange(256, dtype=torch.uint8).view(torch.float8_e4m3fn).double().numpy()
+    return _FP8_VALUES
+
+
+def value_spread(vc: np.ndarray, dtype: str, block_tables, context_lens, ref: np.ndarray,
+                 block_size: int, row_seq=None, v_scale=None) -> np.ndarray:
+    """max over the context (t < L) of |V_t[d] - o[d]| for every output element, ref's shape.
+    vc: the value cache after the step's write, as stored (dtype "bf16", "f16", "f32" or "fp8"
+    codes with per-kv-head v_scale); row_seq[r]: the sequence of output row r (default: row s is
+    sequence s).  For a prefill row the context up to its position is part of t < L, so the
+    spread over t < L bounds it."""
+    rows_n, hq, d = ref.shape
+    hkv = vc.shape[1]
+    g = hq // hkv
+    row_seq = np.arange(rows_n) if row_seq is None else np.asarray(row_seq)
+    out = np.zeros(ref.shape, dtype=np.float64)
+    for s in np.unique(row_seq):
+        L = int(context_lens[s])
+        rows = np.nonzero(row_seq == s)[0]
+        if L <= 0 or rows.size == 0:
+            continue
+        t = np.arange(L)
+        v = vc[block_tables[s, t // block_size], :, t % block_size, :]  # [L, Hkv, D]
+        if dtype == "fp8":
+            v = _fp8_values()[v] * np.asarray(v_scale, np.float64)[None, :, None]
+        else:
+            v = W.decode_to_f64(v, dtype)
+        vmax = np.repeat(v.max(0), g, axis=0)  # [Hq, D]
+        vmin = np.repeat(v.min(0), g, axis=0)
+        o = ref[rows]
+        out[rows] = np.maximum(np.abs(vmax - o), np.abs(vmin - o))
+    return out
+
+
+def assert_bf16_output(got_bits: np.ndarray, ref: np.ndarray, what: str, spread: np.ndarray):
+    """bf16 output against the fp64 result o: |got - o| <= ulp(o) + 2^-16 * spread element by
+    element (spread from value_spread), and >= 99% of the elements exactly RNE(o)."""
     got = W.bf16_bits_to_f32(got_bits).astype(np.float64)
     rne = W.f32_to_bf16_bits(ref.astype(np.float32))
     mag = np.maximum(np.abs(ref), 2.0 ** -126)
     ulp = 2.0 ** (np.floor(np.log2(mag)) - 7)
-    worst = float(np.max((np.abs(got - ref) - 1e-5) / ulp))
-    assert np.all(np.abs(got - ref) <= ulp + 1e-5), f"{what}: bf16 output off by {worst:.2f} ulp + 1e-5"
-    same = float(np.mean(got_bits == rne))
+    bound = ulp + 2.0 ** -16 * spread
+    err = np.abs(got - ref)
+    worst = float(np.max(err / bound)) if err.size else 0.0
+    same = float(np.mean(got_bits == rne)) if err.size else 1.0
+    RESULTS.append((what, "bf16 out", f"{100 * same:.3f}% equal RNE(oracle) (>= 99%), largest "
+                                      f"error {worst:.3f} of its bound (<= 1)"))
+    assert np.all(err <= bound), f"{what}: bf16 output error {worst:.3f} times its bound"
     assert same >= 0.99, f"{what}: only {same:.4f} of bf16 outputs equal RNE(oracle)"
     return same
 

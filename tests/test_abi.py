@@ -31,6 +31,36 @@ def test_every_declared_function_is_exported(lib):
                 and not s.startswith("_init") and not s.startswith("_fini")]
 
 
+# The boundary's calls as first proposed (name: what it does) and the exported calls that
+# provide each; the argument changes are documented beside each declaration in include/pa.h.
+PROPOSED_TO_PROVIDED = {
+    "pa_reshape_and_cache": ["pa_reshape_and_cache"],
+    "pa_decode": ["pa_decode"],
+    # partition_size became num_workers + flags (the split is by bytes over warps, stream-K)
+    "pa_decode_ex": ["pa_decode_ex"],
+    # sized by sequences, heads, head_dim and warps instead of table width and partition size
+    "pa_decode_workspace_bytes": ["pa_decode_workspace_bytes", "pa_decode_default_workers"],
+    "pa_copy_blocks": ["pa_copy_blocks"],
+    "pa_last_error": ["pa_last_error"],
+    # gained a `clear` argument
+    "pa_get_device_error": ["pa_get_device_error"],
+    # freeing the library-owned workspaces
+    "pa_shutdown": ["pa_release_workspaces"],
+    # zero-filling a caller workspace before its first use
+    "(workspace set-up)": ["pa_workspace_init"],
+}
+
+
+def test_every_proposed_call_is_provided(lib):
+    out = subprocess.run(["nm", "-D", "--defined-only", pa.LIBRARY], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(re.findall(r"\sT\s(pa_\w+)$", out, re.M))
+    declared = set(pa.header_functions())
+    for proposed, provided in PROPOSED_TO_PROVIDED.items():
+        for name in provided:
+            assert name in exported and name in declared, f"{proposed}: {name} not provided"
+
+
 def test_version_matches_header(lib):
     with open(pa.HEADER) as f:
         v = int(re.search(r"#define PA_VERSION (\d+)", f.read()).group(1))

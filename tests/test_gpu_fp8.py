@@ -10,6 +10,7 @@ import torch
 import paged_kv_cache_427_b200 as pa
 from paged_kv_cache_427_b200 import workloads as W
 from tests.gpu_helpers import (assert_bf16_output, assert_close, assert_no_device_error,
+                               value_spread,
                                require_gpu, to_host, to_torch)
 
 pytestmark = pytest.mark.gpu
@@ -156,7 +157,9 @@ def test_fp8_decode(llama_fp8, workers, flags):
     out = fb.decode("f32", workers, flags)
     assert_close(out, ref, "bf16", f"fp8 W={workers} flags={flags}")
     outb = fb.decode("bf16", workers, flags)
-    assert_bf16_output(outb, ref, f"fp8 bf16 out W={workers}")
+    spread = value_spread(fb.ovc, "fp8", fb.b.block_tables, fb.b.context_lens, ref,
+                          fb.b.block_size, v_scale=fb.vs)
+    assert_bf16_output(outb, ref, f"fp8 bf16 out W={workers} flags={flags}", spread)
     assert_no_device_error()
 
 

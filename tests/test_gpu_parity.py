@@ -1,8 +1,8 @@
 """Parity of the CUDA path (through the C ABI) with the CPU oracle on the same seeded inputs.
 
 Cache writes and block copies must match bit for bit; attention must meet the tolerances in
-tests/gpu_helpers.py.  Small cases compare every output; the full-size workloads compare the
-whole cache and sampled sequences (the oracle decodes only those).
+tests/gpu_helpers.py.  Every test compares every output row with the oracle, the full-size
+workloads included.
 """
 import numpy as np
 import pytest
@@ -12,7 +12,7 @@ import paged_kv_cache_427_b200 as pa
 from paged_kv_cache_427_b200 import workloads as W
 from tests.gpu_helpers import (DeviceBatch, assert_bf16_output, assert_close,
                                assert_no_device_error, assert_rounded_from, oracle_step,
-                               require_gpu, to_host)
+                               require_gpu, to_host, value_spread)
 
 pytestmark = pytest.mark.gpu
 
@@ -22,6 +22,10 @@ def _gpu():
     require_gpu()
     pa.pa_get_device_error(clear=True)
     yield
+
+
+def _spread(b, vc, ref):
+    return value_spread(vc, b.dtype, b.block_tables, b.context_lens, ref, b.block_size)
 
 
 def _check_caches(db, kc, vc, dtype):
@@ -49,7 +53,7 @@ def test_tiny_fp32(oracle, workers):
 def llama_small(oracle):
     b = W.llama3_8b_decode(num_seqs=12, min_len=1, max_len=300)
     ref, kc, vc = oracle_step(oracle, b)
-    return b, ref, kc, vc
+    return b, ref, kc, vc, _spread(b, vc, ref)
 
 
 @pytest.mark.parametrize("workers,flags", [(None, 0), (1, 0), (7, 0), (33, 0), (512, 0),
@@ -57,20 +61,21 @@ def llama_small(oracle):
                                            (None, 2), (1, 2), (33, 2), (512, 3),
                                            (None, 4), (7, 4), (512, 5), (None, 6)])
 def test_llama_small_workers(llama_small, workers, flags):
-    b, ref, kc, vc = llama_small
+    b, ref, kc, vc, spread = llama_small
     db = DeviceBatch(b)
     db.write()
     _check_caches(db, kc, vc, "bf16")
     out = to_host(db.decode("f32", num_workers=workers, flags=flags), "f32")
     assert_close(out, ref, "bf16", f"W={workers} flags={flags}")
     outb = to_host(db.decode("bf16", num_workers=workers, flags=flags), "bf16")
-    assert_bf16_output(outb, ref, f"bf16 out W={workers}")
+    assert_bf16_output(outb, ref, f"bf16 out W={workers} flags={flags}", spread)
     assert_rounded_from(outb, out, f"bf16 out W={workers}")
     assert_no_device_error()
 
 
 def test_llama_full_size(oracle):
-    """Full Llama-3-8B-shaped step in the launch configuration the benchmark times."""
+    """Full Llama-3-8B-shaped step in the launch configuration the benchmark times; the
+    oracle decodes every one of its 64 sequences."""
     b = W.llama3_8b_decode()
     db = DeviceBatch(b)
     db.write()
@@ -78,12 +83,11 @@ def test_llama_full_size(oracle):
     outb = db.decode("bf16", flags=pa.PA_DECODE_OVERLAP_PREVIOUS)
     out = db.decode("f32")
     torch.cuda.synchronize()
-    lens = b.context_lens
-    seqs = sorted({int(np.argmax(lens)), int(np.argmin(lens)), 0, 1, 31, b.num_seqs - 1})
-    ref, kc, vc = oracle_step(oracle, b, seqs)
+    ref, kc, vc = oracle_step(oracle, b)
     _check_caches(db, kc, vc, "bf16")
-    assert_close(to_host(out, "f32")[seqs], ref, "bf16", "llama full (sampled)")
-    assert_bf16_output(to_host(outb, "bf16")[seqs], ref, "llama full bf16 (sampled)")
+    assert_close(to_host(out, "f32"), ref, "bf16", "llama full (every sequence)")
+    assert_bf16_output(to_host(outb, "bf16"), ref, "llama full bf16 (every sequence)",
+                       _spread(b, vc, ref))
     assert_no_device_error()
 
 
@@ -99,7 +103,7 @@ def test_short_chat_block_sizes(oracle):
         out = to_host(db.decode("f32"), "f32")
         assert_close(out, ref, "bf16", f"short chat bs={bs}")
         outb = to_host(db.decode("bf16"), "bf16")
-        assert_bf16_output(outb, ref, f"short chat bf16 bs={bs}")
+        assert_bf16_output(outb, ref, f"short chat bf16 bs={bs}", _spread(b, vc, ref))
         if ref0 is None:
             ref0 = ref
         assert np.array_equal(ref, ref0), "oracle differs across block sizes"
@@ -116,30 +120,29 @@ def test_shared_prefix(oracle):
     ref, kc, vc = oracle_step(oracle, b)
     _check_caches(db, kc, vc, "bf16")
     assert_close(to_host(db.decode("f32"), "f32"), ref, "bf16", "shared prefix")
-    assert_bf16_output(to_host(db.decode("bf16"), "bf16"), ref, "shared prefix bf16")
+    assert_bf16_output(to_host(db.decode("bf16"), "bf16"), ref, "shared prefix bf16",
+                       _spread(b, vc, ref))
     assert_no_device_error()
 
 
 def test_long_mixed_full_size(oracle):
+    """The long mixed batch at full size (16 contexts of 8k-32k tokens split over many warps,
+    240 short ones); the oracle decodes all 256 sequences."""
     b = W.long_mixed()
     db = DeviceBatch(b)
     db.write()
     out = db.decode("f32")
-    outb = db.decode("bf16")
+    outb = db.decode("bf16", flags=pa.PA_DECODE_OVERLAP_PREVIOUS)
     outs = db.decode("f32", flags=pa.PA_DECODE_SEPARATE_REDUCE)
     outc = db.decode("f32", flags=pa.PA_DECODE_CUDA_CORES)
     torch.cuda.synchronize()
-    lens = b.context_lens
-    longest = list(np.argsort(lens)[-4:])
-    rng = np.random.default_rng(0)
-    short = list(rng.choice(np.where(lens <= 1024)[0], size=8, replace=False))
-    seqs = sorted(int(s) for s in longest + short)
-    ref, kc, vc = oracle_step(oracle, b, seqs)
+    ref, kc, vc = oracle_step(oracle, b)
     _check_caches(db, kc, vc, "bf16")
-    assert_close(to_host(out, "f32")[seqs], ref, "bf16", "long mixed (sampled)")
-    assert_close(to_host(outs, "f32")[seqs], ref, "bf16", "long mixed separate reduce")
-    assert_close(to_host(outc, "f32")[seqs], ref, "bf16", "long mixed CUDA-core kernel")
-    assert_bf16_output(to_host(outb, "bf16")[seqs], ref, "long mixed bf16 (sampled)")
+    assert_close(to_host(out, "f32"), ref, "bf16", "long mixed (every sequence)")
+    assert_close(to_host(outs, "f32"), ref, "bf16", "long mixed separate reduce")
+    assert_close(to_host(outc, "f32"), ref, "bf16", "long mixed CUDA-core kernel")
+    assert_bf16_output(to_host(outb, "bf16"), ref, "long mixed bf16 (every sequence)",
+                       _spread(b, vc, ref))
     assert_no_device_error()
 
 
@@ -212,7 +215,7 @@ def test_configuration_coverage(oracle, dtype, D, bs, hq, hkv):
         if dtype != "f32":
             got = to_host(db.decode(dtype, num_workers=workers, flags=flags), dtype)
             if dtype == "bf16":
-                assert_bf16_output(got, ref, "bf16 out " + what)
+                assert_bf16_output(got, ref, "bf16 out " + what, _spread(b, vc, ref))
             else:
                 assert_close(got.astype(np.float64), ref, dtype, "fp16 out " + what)
     assert_no_device_error()

@@ -2,14 +2,14 @@
 with the oracle (fp32 out within the 16-bit tolerance, 16-bit out against the rounding of the
 fp64 result) on a mixed continuously batched step (whole prompts, prompt chunks on top of a
 prefix, single decode tokens, a sequence with no new token), for every built configuration, on
-the full-size chunked-prefill workload (sampled), and on its error cases."""
+the full-size chunked-prefill workload (every sequence), and on its error cases."""
 import numpy as np
 import pytest
 import torch
 
 import paged_kv_cache_427_b200 as pa
 from paged_kv_cache_427_b200 import workloads as W
-from tests.gpu_helpers import (TORCH_DTYPE, assert_bf16_output, assert_close,
+from tests.gpu_helpers import (TORCH_DTYPE, assert_bf16_output, assert_close, value_spread,
                                assert_no_device_error, require_gpu, to_host, to_torch)
 
 pytestmark = pytest.mark.gpu
@@ -37,6 +37,13 @@ class PrefillStep:
         return to_host(out, out_dtype)
 
 
+def _spread(b, vc, ref):
+    """value_spread for prefill rows: row r belongs to the sequence whose new tokens hold it."""
+    row_seq = np.repeat(np.arange(b.num_seqs), np.diff(b.query_start))
+    return value_spread(vc, b.dtype, b.block_tables, b.context_lens, ref, b.block_size,
+                        row_seq=row_seq)
+
+
 def _oracle(orc, b):
     kc, vc = b.key_cache.copy(), b.value_cache.copy()
     assert orc.reshape_and_cache(b.key, b.value, kc, vc, b.slot_mapping, b.dtype) == 0
@@ -54,7 +61,7 @@ def test_prefill_mixed_batch(oracle):
     assert np.array_equal(to_host(st.key_cache, "bf16"), kc)
     assert np.array_equal(to_host(st.value_cache, "bf16"), vc)
     assert_close(st.run("f32"), ref, "bf16", "prefill mixed batch")
-    assert_bf16_output(st.run("bf16"), ref, "prefill bf16 out")
+    assert_bf16_output(st.run("bf16"), ref, "prefill bf16 out", _spread(b, vc, ref))
     assert_no_device_error()
 
 
@@ -131,31 +138,24 @@ def test_prefill_growing_logits_move_the_reference(oracle):
                               num_kv_heads=8, head_dim=128, block_size=16, dtype="bf16",
                               seed=W.BASE_SEED + 745)
     _scale_keys_by_position(b, lambda t: 1.0 + t / 8.0)
-    ref, _, _ = _oracle(oracle, b)
+    ref, _, vc = _oracle(oracle, b)
     st = PrefillStep(b)
     assert_close(st.run("f32"), ref, "bf16", "prefill growing logits")
-    assert_bf16_output(st.run("bf16"), ref, "prefill growing logits bf16 out")
+    assert_bf16_output(st.run("bf16"), ref, "prefill growing logits bf16 out", _spread(b, vc, ref))
     assert_no_device_error()
 
 
-def test_prefill_chunked_workload_sampled(oracle):
-    """The full-size chunked-prefill step on the GPU; the oracle recomputes three of its
-    sequences (their rows of the output)."""
+def test_prefill_chunked_workload_full_size(oracle):
+    """The full-size chunked-prefill step in the launch configuration the benchmark times;
+    the oracle recomputes every sequence (all 2,048 new tokens of all 32 heads)."""
     require_gpu()
     b = W.chunked_prefill()
     st = PrefillStep(b)
     got = st.run("f32")
-    pick = [0, 3, 6]
-    qs = b.query_start
-    sub = W.build_prefill_batch("sub", b.context_lens[pick], qs[1:][pick] - qs[:-1][pick],
-                                num_heads=32, num_kv_heads=8, head_dim=128, block_size=16,
-                                dtype="bf16", seed=0)  # shapes only
-    rows = np.concatenate([np.arange(qs[s], qs[s + 1]) for s in pick])
-    kc, vc = b.key_cache.copy(), b.value_cache.copy()
-    assert oracle.reshape_and_cache(b.key, b.value, kc, vc, b.slot_mapping, b.dtype) == 0
-    ref = oracle.prefill(b.query[rows], kc, vc, b.block_tables[pick], b.context_lens[pick],
-                         sub.query_start, b.scale, b.dtype)
-    assert_close(got[rows], ref, "bf16", "chunked prefill (sampled sequences)")
+    gotb = st.run("bf16")
+    ref, _, vc = _oracle(oracle, b)
+    assert_close(got, ref, "bf16", "chunked prefill (every sequence)")
+    assert_bf16_output(gotb, ref, "chunked prefill bf16 out (every sequence)", _spread(b, vc, ref))
     assert_no_device_error()
 
 
