@@ -718,12 +718,15 @@ def timeline_summary(recs, chunk_bytes: int) -> dict:
 # ----------------------------------------------------------------------------------------------
 
 def run_decode(args, b: W.PagedBatch, config: dict, rank: int = 0, world: int = 1,
-               local_rank: int = 0, full: bool = True, probe: dict | None = None) -> dict | None:
+               local_rank: int = 0, full: bool = True, probe: dict | None = None,
+               shared: bool = False) -> dict | None:
     """The decode step of one workload: the cache write (plus the copy-on-write block copies
     where the batch has them), then the decode launched to overlap the write.  Timed regions:
     K steps with nothing between launches (`value`); per-launch events around the decode (the
     roofline); with `full`, also the step as a CUDA graph, end to end from pinned host memory,
-    the CPU baseline and the timeline.  Returns rank 0's line (None on the other ranks)."""
+    the CPU baseline and the timeline.  With `shared`, the decode is pa_decode_shared_prefix
+    over the batch's groups (workloads.shared_groups).  Returns rank 0's line (None on the
+    other ranks)."""
     import torch
 
     import paged_kv_cache_427_b200 as pa
@@ -752,11 +755,21 @@ def run_decode(args, b: W.PagedBatch, config: dict, rank: int = 0, world: int = 
         ws = torch.zeros(pa.pa_decode_workspace_bytes(b.num_seqs, b.num_heads, b.num_kv_heads,
                                                       b.head_dim, 0), dtype=torch.uint8, device=dev)
 
-    def decode(qq, kc, vc, tt, ll):
-        if ws is None:
-            pa.pa_decode(out, qq, kc, vc, tt, ll, b.scale, b.block_size, b.num_kv_heads)
+    if shared:
+        g_start, p_lens = (dev_tensor(x, None, dev) for x in W.shared_groups(b))
+        ws_shared = torch.zeros(pa.pa_decode_shared_prefix_workspace_bytes(
+            b.num_seqs, b.num_heads, b.num_kv_heads, b.head_dim, b.max_blocks, b.block_size),
+            dtype=torch.uint8, device=dev)
+
+    def decode(qq, kc, vc, tt, ll, o=None):
+        o = out if o is None else o
+        if shared:
+            pa.pa_decode_shared_prefix(o, qq, kc, vc, tt, ll, g_start, p_lens, b.scale,
+                                       b.block_size, b.num_kv_heads, workspace=ws_shared)
+        elif ws is None:
+            pa.pa_decode(o, qq, kc, vc, tt, ll, b.scale, b.block_size, b.num_kv_heads)
         else:
-            pa.pa_decode_ex(out, qq, kc, vc, tt, ll, b.scale, b.block_size, b.num_kv_heads,
+            pa.pa_decode_ex(o, qq, kc, vc, tt, ll, b.scale, b.block_size, b.num_kv_heads,
                             flags=args.decode_flags, workspace=ws)
 
     def step(i, ev=None):
@@ -770,7 +783,8 @@ def run_decode(args, b: W.PagedBatch, config: dict, rank: int = 0, world: int = 
         if ev is not None:
             ev[1].record(stream)
 
-    launches_per_step = 2 + (1 if mapping is not None else 0) + (1 if args.decode_flags & 1 else 0)
+    launches_per_step = (2 + (1 if mapping is not None else 0) + (1 if args.decode_flags & 1 else 0)
+                         + (1 if shared else 0))
     gpu_uuid = None
     try:
         gpu_uuid = str(torch.cuda.get_device_properties(dev).uuid)
@@ -801,7 +815,7 @@ def run_decode(args, b: W.PagedBatch, config: dict, rank: int = 0, world: int = 
     # Timed region 3 (headline, default flags only): the step as one pa_decode_step call,
     # captured once per pool copy into a CUDA graph and replayed K times.
     graph = None
-    if full and args.decode_flags == pa.PA_DECODE_OVERLAP_PREVIOUS and world == 1:
+    if full and args.decode_flags == pa.PA_DECODE_OVERLAP_PREVIOUS and world == 1 and not shared:
         def graph_step(i):
             kc, vc = pools[i % rot]
             if mapping is not None:
@@ -849,7 +863,7 @@ def run_decode(args, b: W.PagedBatch, config: dict, rank: int = 0, world: int = 
 
     elapsed_ms, dec_mean = max_over_ranks([elapsed_ms, float(np.mean(decode_ms))], device=dev)
     if e2e is not None:
-        e2e["ms"] = max_over_ranks([e2e["ms"]], device=dev)[0]
+        e2e["ms"], e2e["serial_ms"] = max_over_ranks([e2e["ms"], e2e["serial_ms"]], device=dev)
     flags = pa.pa_get_device_error(clear=True)
     if rank != 0:
         return None
@@ -865,6 +879,9 @@ def run_decode(args, b: W.PagedBatch, config: dict, rank: int = 0, world: int = 
     peak, peak_src = hbm_peak()
     kernel = ("paged_decode_kernel (CUDA cores)" if (args.decode_flags & 2 or b.dtype == "f32")
               else "paged_decode_mma_kernel (mma.sync + TMA)")
+    if shared:
+        kernel = ("paged_prefill_tc_kernel shared-prefix pass (tcgen05) + paged_decode_mma_kernel "
+                  "(mma.sync + TMA); launch times cover both")
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 5),
@@ -886,8 +903,16 @@ def run_decode(args, b: W.PagedBatch, config: dict, rank: int = 0, world: int = 
         line["e2e"] = {"value": round(world * step_bytes / (e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
                        "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"],
                        "ms_per_step": round(e_ms, 5),
-                       "how": "per step: one pinned-buffer copy in, the write, the decode, the "
-                              "output copy out, synchronize"}
+                       "how": "per step: one pinned-buffer copy of the step's inputs in (on a copy "
+                              "stream, overlapping the previous step's compute; two buffers), the "
+                              "write, the decode, the output copied out and waited for by the host "
+                              "after the next step is launched"}
+        s_ms = e2e["serial_ms"] / args.steps
+        line["e2e_serial"] = {"value": round(world * step_bytes / (s_ms * 1e-3) / 1e9, 2),
+                              "unit": "GB/s", "h2d_bytes_per_step": e2e["h2d"],
+                              "d2h_bytes_per_step": e2e["d2h"], "ms_per_step": round(s_ms, 5),
+                              "how": "per step: the input copy, the write, the decode, the output "
+                                     "copy, synchronize, nothing overlapped"}
         if e2e.get("graph_ms") is not None:
             g_step = e2e["graph_ms"] / args.steps
             line["e2e_graph"] = {"value": round(step_bytes / (g_step * 1e-3) / 1e9, 2),
@@ -907,6 +932,8 @@ def run_decode(args, b: W.PagedBatch, config: dict, rank: int = 0, world: int = 
         line["logical_GBps"] = round(world * (dec_logical + write_bytes(b)) / (ms * 1e-3) / 1e9, 2)
     if timeline:
         line["timeline"] = timeline
+    if shared:
+        line["decode_call"] = "pa_decode_shared_prefix"
     if full and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(b, args.cpu_seconds)
     return line
@@ -985,7 +1012,61 @@ def measure_e2e(args, b, pools, rot, mapping, out, ws, decode, dev, stream, worl
         e2e_step(i)
     e1.record(stream)
     torch.cuda.synchronize()
-    res = {"ms": e0.elapsed_time(e1), "h2d": int(total), "d2h": int(h_out.numel() * h_out.element_size())}
+    res = {"serial_ms": e0.elapsed_time(e1), "h2d": int(total),
+           "d2h": int(h_out.numel() * h_out.element_size())}
+
+    # Pipelined, as a serving loop runs it: every step still copies its own inputs in and reads
+    # its own result back, but step i's input copy runs on a copy stream while step i-1
+    # computes (two input buffers, two outputs), and the host waits for step i-1's result
+    # after launching step i.
+    copy_stream = torch.cuda.Stream(device=dev)
+    d_bufs = [d_buf, torch.empty_like(d_buf)]
+
+    def views(buf):
+        v = {}
+        for k, t in parts.items():
+            n = t.numel() * t.element_size()
+            v[k] = buf[offs[k]:offs[k] + n].view(t.dtype).view(t.shape)
+        return v
+
+    d_ins = [d_in, views(d_bufs[1])]
+    outs = [out, torch.empty_like(out)]
+    h_outs = [h_out, torch.empty(out.shape, dtype=out.dtype).pin_memory()]
+    ev_in = [torch.cuda.Event(), torch.cuda.Event()]    # input copy of buffer j landed
+    ev_used = [torch.cuda.Event(), torch.cuda.Event()]  # the step on buffer j has read it
+    ev_out = [torch.cuda.Event(), torch.cuda.Event()]   # the result of buffer j is on the host
+
+    def pipe_step(i):
+        j = i % 2
+        with torch.cuda.stream(copy_stream):
+            copy_stream.wait_event(ev_used[j])
+            d_bufs[j].copy_(h_buf, non_blocking=True)
+            ev_in[j].record(copy_stream)
+        stream.wait_event(ev_in[j])
+        kc, vc = pools[i % rot]
+        dj = d_ins[j]
+        if mapping is not None:
+            pa.pa_copy_blocks(kc, vc, dj["mapping"])
+        pa.pa_reshape_and_cache(dj["key"], dj["value"], kc, vc, dj["slots"])
+        decode(dj["query"], kc, vc, dj["tables"], dj["lens"], o=outs[j])
+        ev_used[j].record(stream)
+        h_outs[j].copy_(outs[j], non_blocking=True)
+        ev_out[j].record(stream)
+        if i >= 1:
+            ev_out[1 - j].synchronize()  # step i-1's result is on the host
+
+    for i in range(min(args.warmup, 50)):
+        pipe_step(i)
+    torch.cuda.synchronize()
+    p0, p1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    p0.record(stream)
+    copy_stream.wait_event(p0)  # every copy of the timed region starts after p0
+    for i in range(args.steps):
+        pipe_step(i)
+    p1.record(stream)
+    ev_out[(args.steps - 1) % 2].synchronize()
+    torch.cuda.synchronize()
+    res["ms"] = p0.elapsed_time(p1)
 
     # where one eager end-to-end step's time goes: events between its operations, and the host
     # wall clock from the first call to the return of the synchronize
@@ -1016,7 +1097,7 @@ def measure_e2e(args, b, pools, rot, mapping, out, ws, decode, dev, stream, worl
     # The same end-to-end step with its four operations (input copy, pa_decode_step or its two
     # halves, output copy) captured in one CUDA graph per pool copy: one launch per step, still
     # a synchronize and a host read of the output every step.
-    if args.decode_flags == pa.PA_DECODE_OVERLAP_PREVIOUS and world == 1:
+    if args.decode_flags == pa.PA_DECODE_OVERLAP_PREVIOUS and world == 1 and not args.shared:
         def e2e_body(i):
             d_buf.copy_(h_buf, non_blocking=True)
             kc, vc = pools[i % rot]
@@ -1113,6 +1194,24 @@ def run_fp8(args, b, config, full: bool = True, probe: dict | None = None) -> di
     soak(step, args.soak if full else min(args.soak, 0.3))
     elapsed_ms = run_steps(step, args.steps, stream)
     dec_ms = run_launches(step, launch_count(args))
+    timeline = None
+    if full and args.timeline:
+        workers = pa.pa_decode_default_workers(pa.PA_BF16, b.head_dim, b.block_size,
+                                               b.num_heads // b.num_kv_heads)
+        buf = torch.zeros(max(workers, 1) * 2 * pa.TIMELINE_WORDS, dtype=torch.int64, device=dev)
+        pa.pa_set_decode_timeline(buf)
+        recs = []
+        try:
+            for i in range(args.timeline):
+                buf.zero_()
+                step(i)
+                torch.cuda.synchronize()
+                recs.append(buf.cpu().numpy().copy())
+        finally:
+            pa.pa_set_decode_timeline(None)
+        timeline = timeline_summary(recs, 16 * b.head_dim * 1 * 2)
+        if args.timeline_out:
+            np.save(args.timeline_out, np.stack(recs))
     clocks = sampler.stop()
     flags = pa.pa_get_device_error(clear=True)
     if flags:
@@ -1135,6 +1234,8 @@ def run_fp8(args, b, config, full: bool = True, probe: dict | None = None) -> di
                                      recorded_traffic(config["workload"] + ":fp8", "decode_fp8"),
                                      probe),
             "gpu_launches": 2 * args.steps, "clocks": clocks}
+    if timeline:
+        line["timeline"] = timeline
     if full and not args.no_cpu_baseline:
         kc8, vc8 = pools[0]
         line["cpu_baseline"] = cpu_baseline_fp8(
@@ -1223,8 +1324,9 @@ def run_prefill(args, b, config, full: bool = True) -> dict:
 # mixed batch (its own >= 60 % bar), the block-size sweep, the shared prefix, the FP8 cache on
 # the headline's batch and the chunked prefill.
 CONFIG_RUNS = (("long_mixed", "decode"), ("short_chat_bs8", "decode"), ("short_chat_bs16", "decode"),
-               ("short_chat_bs32", "decode"), ("shared_prefix", "decode"),
-               ("llama3_8b_decode", "fp8"), ("chunked_prefill", "prefill"))
+               ("short_chat_bs32", "decode"), ("shared_prefix", "shared"),
+               ("shared_prefix", "decode"), ("llama3_8b_decode", "fp8"),
+               ("chunked_prefill", "prefill"))
 
 
 def run_configs(args, probe) -> dict:
@@ -1234,7 +1336,7 @@ def run_configs(args, probe) -> dict:
 
     keep = ("metric", "value", "unit", "ms_per_step", "pct_of_8TBs", "pct_of_read_probe",
             "attended_tokens_per_s", "seq_steps_per_s", "new_tokens_per_s", "logical_GBps",
-            "roofline", "clocks", "dtype")
+            "roofline", "clocks", "dtype", "decode_call")
     res = {}
     for name, kind in CONFIG_RUNS:
         b = make_batch(name)
@@ -1245,9 +1347,12 @@ def run_configs(args, probe) -> dict:
         elif kind == "prefill":
             line = run_prefill(args, b, cfg, full=False)
             key = name
+        elif kind == "shared":
+            line = run_decode(args, b, cfg, full=False, probe=probe, shared=True)
+            key = name
         else:
             line = run_decode(args, b, cfg, full=False, probe=probe)
-            key = name
+            key = name + (":pa_decode" if name == "shared_prefix" else "")
         rec = {k: line[k] for k in keep if k in line}
         rec["config"] = {k: v for k, v in line["config"].items()
                          if k in ("num_seqs", "block_size", "attended_tokens", "kv_dtype",
@@ -1380,6 +1485,8 @@ def main():
     ap.add_argument("--timeline", type=int, default=0, metavar="N",
                     help="record N decode launches with pa_set_decode_timeline and add a summary")
     ap.add_argument("--timeline-out", default=None, help="save the raw timeline records (.npy)")
+    ap.add_argument("--shared", action="store_true",
+                    help="decode the workload with pa_decode_shared_prefix over its groups")
     ap.add_argument("--kv", default="native", choices=["native", "fp8"],
                     help="fp8: the same step over an FP8 E4M3 cache (pa_decode_fp8)")
     ap.add_argument("--swap", action="store_true",
@@ -1430,7 +1537,8 @@ def main():
         probe = None
         if world == 1 and not args.no_probe:
             probe = read_probe(torch.device("cuda", local_rank))
-        line = run_decode(args, b, config, rank, world, local_rank, full=True, probe=probe)
+        line = run_decode(args, b, config, rank, world, local_rank, full=True, probe=probe,
+                          shared=args.shared)
         if line is not None:
             if probe:
                 line["hbm_read_probe"] = probe

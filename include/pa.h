@@ -119,6 +119,12 @@ typedef enum pa_status {
                                       decode call using it zeroes its merge counters first;
                                       no other step is needed */
 
+#define PA_DEVERR_PREFIX 0x20u     /* pa_decode_shared_prefix: a group's members disagree on
+                                      their shared prefix (length or physical blocks), or a
+                                      prefix is not a whole number of blocks; such a sequence
+                                      is decoded over its whole context instead where it can
+                                      be, otherwise its result is unspecified */
+
 /* Flags of pa_decode_ex. */
 #define PA_DECODE_SEPARATE_REDUCE 0x1u /* merge split contexts in a second kernel instead of
                                           in the last warp to finish each (sequence, kv head) */
@@ -365,6 +371,48 @@ PA_API int pa_decode_noalloc(const pa_tensor *out, const pa_tensor *query,
                              const pa_tensor *key_cache, const pa_tensor *value_cache,
                              const pa_tensor *block_tables, const pa_tensor *context_lens,
                              float scale, int32_t block_size, int32_t num_kv_heads, void *stream);
+
+/*
+ * pa_decode_shared_prefix - pa_decode for a batch whose sequences come in groups that share a
+ * prompt prefix stored once: several sequences' block tables name the same physical blocks
+ * ([P2] 4.1, parallel sampling and shared prompts; [P3] 2.2, shared prompt pages).  Same
+ * result as pa_decode (within the same tolerances); the shared prefix is read once per kv head
+ * for all members instead of once per member.
+ *   group_start  [num_groups + 1] int32, non-decreasing from 0: group g is the consecutive
+ *                sequences group_start[g] .. group_start[g+1] - 1 (a sequence in no group is a
+ *                group of one).
+ *   prefix_lens  [num_seqs] int32: the number of leading positions sequence s shares with the
+ *                other members of its group; equal within a group, a multiple of block_size,
+ *                and every member's block-table entries for those positions equal the first
+ *                member's.  0 = nothing shared.
+ * Two kernels on `stream`: the prefix pass computes, on the fifth-generation tensor cores,
+ * every member's query rows (128 rows = 128 / G members x G heads per tile) against its group's
+ * prefix, read once through the first member's block table, in items of 256 positions, and
+ * stores partial results (O / l, running maximum, sum); the decode kernel then walks each
+ * sequence's positions prefix_lens[s] .. L-1 and merges its pieces with the prefix partials by
+ * the log-sum-exp rule.  A sequence with prefix_lens[s] >= L is decoded over its whole context.
+ * Disagreements (a member's prefix length or blocks differ from the first member's, a prefix
+ * not a multiple of block_size) set PA_DEVERR_PREFIX.  Caches bf16 or fp16 (otherwise
+ * PA_ERR_UNSUPPORTED); head_dim, block_size and group sizes as for pa_prefill; out fp32 or the
+ * caches' type.  workspace: device memory of at least pa_decode_shared_prefix_workspace_bytes
+ * bytes, 256-byte aligned, zeroed before its first use (pa_workspace_init), or NULL for a
+ * library-owned one (as for pa_decode).  The decode starts as a programmatic dependent of the
+ * prefix pass; the prefix pass itself starts after the kernel before it on `stream`.
+ */
+PA_API int pa_decode_shared_prefix(const pa_tensor *out, const pa_tensor *query,
+                                   const pa_tensor *key_cache, const pa_tensor *value_cache,
+                                   const pa_tensor *block_tables, const pa_tensor *context_lens,
+                                   const pa_tensor *group_start, const pa_tensor *prefix_lens,
+                                   float scale, int32_t block_size, int32_t num_kv_heads,
+                                   void *workspace, size_t workspace_bytes, void *stream);
+
+/* Bytes of workspace pa_decode_shared_prefix needs (0 on invalid arguments): the decode
+ * workspace of pa_decode_ex plus the prefix pass's partial results for prefixes of up to
+ * max_blocks_per_seq * block_size positions. */
+PA_API size_t pa_decode_shared_prefix_workspace_bytes(int64_t num_seqs, int32_t num_heads,
+                                                      int32_t num_kv_heads, int32_t head_dim,
+                                                      int64_t max_blocks_per_seq,
+                                                      int32_t block_size);
 
 /*
  * Measurement aids (not part of the attention path).

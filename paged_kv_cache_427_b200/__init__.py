@@ -36,6 +36,7 @@ PA_DEVERR_CONTEXT_LEN = 0x2
 PA_DEVERR_SLOT = 0x4
 PA_DEVERR_COPY_PAIR = 0x8
 PA_DEVERR_TIMEOUT = 0x10
+PA_DEVERR_PREFIX = 0x20
 PA_NOALLOC_SCRATCH_BYTES = 8 * 1024 * 1024
 PA_ERR_INVALID_ARG = -1
 PA_ERR_SHAPE = -2
@@ -93,6 +94,10 @@ def load(path: str = LIBRARY) -> ctypes.CDLL:
     lib.pa_get_device_error.argtypes = [_P, ctypes.POINTER(u32), i32]
     lib.pa_decode_noalloc.argtypes = [_T, _T, _T, _T, _T, _T, f32, i32, i32, _P]
     lib.pa_decode_step.argtypes = [_T, _T, _T, _T, _T, _T, _T, _T, _T, f32, i32, i32, _P, sz, _P]
+    lib.pa_decode_shared_prefix.argtypes = [_T, _T, _T, _T, _T, _T, _T, _T, f32, i32, i32, _P, sz, _P]
+    lib.pa_decode_shared_prefix.restype = ctypes.c_int
+    lib.pa_decode_shared_prefix_workspace_bytes.argtypes = [i64, i32, i32, i32, i64, i32]
+    lib.pa_decode_shared_prefix_workspace_bytes.restype = sz
     lib.pa_set_decode_timeline.argtypes = [_P, sz]
     lib.pa_set_decode_timeline.restype = ctypes.c_int
     lib.pa_hbm_read_probe.argtypes = [_P, sz, i32, _P, _P]
@@ -294,6 +299,28 @@ def header_functions(path: str = HEADER) -> list[str]:
     with open(path) as f:
         text = f.read()
     return sorted(set(re.findall(r"^\s*PA_API\s+(?:const\s+)?\w+\s*\*?\s*(pa_\w+)\s*\(", text, re.M)))
+
+
+def pa_decode_shared_prefix(out, query, key_cache, value_cache, block_tables, context_lens,
+                            group_start, prefix_lens, scale, block_size, num_kv_heads,
+                            workspace=None, stream=None):
+    """pa_decode for groups of consecutive sequences sharing a prompt prefix (group_start
+    [num_groups + 1] int32, prefix_lens [num_seqs] int32); see include/pa.h."""
+    lib = load()
+    d = [describe(x) for x in (out, query, key_cache, value_cache, block_tables, context_lens,
+                               group_start, prefix_lens)]
+    ws_ptr = workspace.data_ptr() if workspace is not None else None
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check("pa_decode_shared_prefix",
+           lib.pa_decode_shared_prefix(*[ctypes.byref(x) for x in d], ctypes.c_float(scale),
+                                       block_size, num_kv_heads, ws_ptr, ws_bytes, _stream(stream)))
+
+
+def pa_decode_shared_prefix_workspace_bytes(num_seqs, num_heads, num_kv_heads, head_dim,
+                                            max_blocks_per_seq, block_size) -> int:
+    return int(load().pa_decode_shared_prefix_workspace_bytes(num_seqs, num_heads, num_kv_heads,
+                                                              head_dim, max_blocks_per_seq,
+                                                              block_size))
 
 
 TIMELINE_WORDS = 8  # 64-bit words per worker warp in a decode timeline record

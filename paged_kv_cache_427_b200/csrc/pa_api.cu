@@ -439,16 +439,105 @@ WsLayout ws_layout(int64_t S, int Hq, int Hkv, int D, int W) {
   return L;
 }
 
+// Shared-prefix pass: items of kPrefixItemTokens positions; its partial results follow the
+// decode workspace: pre_ml [S*Hq*splits*2] f32 | pre_o [S*Hq*splits*D] f32.
+constexpr int kPrefixItemTokens = 256;  // two kv tiles of 128 positions
+
+struct PrefixLayout {
+  size_t pre_ml, pre_o, total;
+  int splits;
+};
+
+PrefixLayout prefix_layout(size_t start, int64_t S, int Hq, int D, int64_t max_blocks,
+                           int block_size) {
+  PrefixLayout P;
+  const int64_t max_len = max_blocks * block_size;
+  P.splits = (int)((max_len + kPrefixItemTokens - 1) / kPrefixItemTokens);
+  if (P.splits < 1) P.splits = 1;
+  const size_t slots = (size_t)S * (size_t)Hq * (size_t)P.splits;
+  P.pre_ml = align256(start);
+  P.pre_o = P.pre_ml + align256(slots * 2 * 4);
+  P.total = P.pre_o + align256(slots * (size_t)D * 4);
+  return P;
+}
+
+// The prefix pass of pa_decode_shared_prefix: the prefill kernel over every group's members
+// (their decode queries as consecutive query rows) and its shared prefix, storing partial
+// results for the decode to merge.
+int launch_prefix_pass(const pa::DecodeArgs &d, const pa_tensor *query, const pa_tensor *key_cache,
+                       const pa_tensor *value_cache, const pa_tensor *group_start,
+                       const CacheShape &cs, int D, int G, int block_size, DeviceState *ds,
+                       cudaStream_t st) {
+  int rc;
+  pa::PrefillKernel k;
+  const bool got = cs.dtype == PA_BF16 ? pa::prefill_kernel_bf16(D, block_size, G, &k)
+                                       : pa::prefill_kernel_f16(D, block_size, G, &k);
+  if (!got)
+    return fail(PA_ERR_CUDA, "could not prepare the prefix pass: %s", cudaGetErrorString(cudaGetLastError()));
+  pa::PrefillMaps maps;
+  const pa_tensor *kc = key_cache, *vc = value_cache;
+  const bool grouped = grouped_view_ok(kc) && grouped_view_ok(vc);
+  const int rows = grouped ? 0 : k.tma_rows;
+  if ((rc = cache_map(kc, rows, &maps.k)) || (rc = cache_map(vc, rows, &maps.v)) ||
+      (rc = query_map(query, G, &maps.q)))
+    return rc;
+  const int64_t S = d.num_seqs;
+  const int64_t NG = group_start->shape[0] - 1;
+  if (NG <= 0) return PA_OK;
+  // items: every row tile of every group, for every kv head and prefix item (a bound: the
+  // groups' sizes and prefixes are device values)
+  const int64_t items = ((S + k.tokens_per_tile - 1) / k.tokens_per_tile + NG) * d.num_kv_heads *
+                        (int64_t)d.pre_splits;
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k.kernel, k.threads_per_cta,
+                                                    k.smem_bytes) != cudaSuccess || per_sm < 1) {
+    cudaGetLastError();
+    per_sm = 1;
+  }
+  const int64_t wave = (int64_t)per_sm * ds->num_sms;
+  const int ctas = (int)(items < wave ? items : wave);
+  pa::PrefillArgs a = {};
+  a.out = nullptr;
+  a.out_dtype = PA_F32;
+  a.query = query->data;
+  a.q_t = query->stride[0];
+  a.q_h = query->stride[1];
+  a.block_tables = d.block_tables;
+  a.bt_s = d.bt_s;
+  a.context_lens = d.context_lens;
+  a.query_start = nullptr;
+  a.num_seqs = d.num_seqs;
+  a.num_kv_heads = d.num_kv_heads;
+  a.max_blocks = d.max_blocks;
+  a.num_blocks = d.num_blocks;
+  a.num_tokens = S;
+  a.scale_log2 = d.scale_log2;
+  a.err = d.err;
+  a.wait_cycles = d.wait_cycles;
+  a.grouped_maps = grouped ? 1 : 0;
+  a.group_start = static_cast<const int32_t *>(group_start->data);
+  a.prefix_lens = d.prefix_lens;
+  a.num_groups = (int)NG;
+  a.pre_kv = kPrefixItemTokens / 128;
+  a.pre_splits = d.pre_splits;
+  a.pre_o = const_cast<float *>(d.pre_o);
+  a.pre_ml = const_cast<float *>(d.pre_ml);
+  cudaError_t e = k.launch(a, &maps, ctas, st);
+  return e == cudaSuccess ? PA_OK : cuda_fail(e, "prefix pass launch");
+}
+
 int decode_impl(const pa_tensor *out, const pa_tensor *query, const pa_tensor *key_cache,
                 const pa_tensor *value_cache, const pa_tensor *block_tables,
                 const pa_tensor *context_lens, float scale, int32_t block_size,
                 int32_t num_kv_heads, int32_t num_workers, uint32_t flags, void *workspace,
                 size_t workspace_bytes, bool library_workspace, void *stream,
                 CallMode mode = CallMode::kLaunch, const pa_tensor *k_scale = nullptr,
-                const pa_tensor *v_scale = nullptr) {
+                const pa_tensor *v_scale = nullptr, const pa_tensor *group_start = nullptr,
+                const pa_tensor *prefix_lens = nullptr) {
   int rc;
   CacheShape cs;
   const bool fp8 = k_scale != nullptr;
+  const bool shared = group_start != nullptr;
   if ((rc = check_caches(key_cache, value_cache, &cs, fp8))) return rc;
   if (fp8 && cs.dtype != PA_FP8_E4M3) return fail(PA_ERR_DTYPE, "pa_decode_fp8 needs fp8_e4m3 caches");
   if ((rc = check_tensor(query, "query", 3)) || (rc = check_tensor(out, "out", 3)) ||
@@ -511,10 +600,27 @@ int decode_impl(const pa_tensor *out, const pa_tensor *query, const pa_tensor *k
   if (S > 0x7fffffff || block_tables->shape[1] * block_size > 0x7fffffff)
     return fail(PA_ERR_SHAPE, "too many sequences or too long a block table");
   if (!std::isfinite(scale)) return fail(PA_ERR_INVALID_ARG, "scale must be finite");
+  if (shared) {
+    if (!prefix_lens) return fail(PA_ERR_INVALID_ARG, "prefix_lens is required");
+    if ((rc = check_tensor(group_start, "group_start", 1)) || (rc = check_tensor(prefix_lens, "prefix_lens", 1)))
+      return rc;
+    if (group_start->dtype != PA_I32 || prefix_lens->dtype != PA_I32)
+      return fail(PA_ERR_DTYPE, "group_start and prefix_lens must be int32");
+    if (group_start->shape[0] < 1 || prefix_lens->shape[0] != S)
+      return fail(PA_ERR_SHAPE, "group_start needs num_groups + 1 entries and prefix_lens one per sequence");
+    if ((group_start->stride[0] != 1 && group_start->shape[0] > 1) || (prefix_lens->stride[0] != 1 && S > 1))
+      return fail(PA_ERR_LAYOUT, "group_start and prefix_lens must be contiguous");
+    if (cs.dtype != PA_BF16 && cs.dtype != PA_F16)
+      return fail(PA_ERR_UNSUPPORTED, "shared prefixes are built for bf16 and fp16 caches");
+    if (group_start->shape[0] - 1 > 0x7fffffff) return fail(PA_ERR_SHAPE, "too many groups");
+  }
   if (S == 0 || mode == CallMode::kHostChecks) return PA_OK;
   DeviceState *ds;
   int dev;
   if ((rc = device_state(&ds, &dev))) return rc;
+  if (shared && ((rc = check_device_memory(group_start, "group_start", dev)) ||
+                 (rc = check_device_memory(prefix_lens, "prefix_lens", dev))))
+    return rc;
   if ((rc = check_device_memory(key_cache, "key_cache", dev)) ||
       (rc = check_device_memory(value_cache, "value_cache", dev)) ||
       (rc = check_device_memory(query, "query", dev)) || (rc = check_device_memory(out, "out", dev)) ||
@@ -541,17 +647,19 @@ int decode_impl(const pa_tensor *out, const pa_tensor *query, const pa_tensor *k
   const double chunks = (double)S * num_kv_heads * ((double)block_tables->shape[1] * block_size / k.chunk_tokens + 1);
   if (chunks * (double)W > 4.0e18) return fail(PA_ERR_SHAPE, "step too large for the work split");
   const WsLayout L = ws_layout(S, (int)Hq, num_kv_heads, D, W);
+  const PrefixLayout PL = prefix_layout(L.total, S, (int)Hq, D, block_tables->shape[1], block_size);
+  const size_t need = shared ? PL.total : L.total;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (mode == CallMode::kAllChecks) {  // everything a launch would check, nothing launched
-    if (!library_workspace && (!workspace || workspace_bytes < L.total))
-      return fail(PA_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", L.total, workspace_bytes);
+    if (!library_workspace && (!workspace || workspace_bytes < need))
+      return fail(PA_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", need, workspace_bytes);
     if (!library_workspace && ((uintptr_t)workspace & 255u) != 0)
       return fail(PA_ERR_WORKSPACE, "workspace must be 256-byte aligned");
     return PA_OK;
   }
   if (library_workspace) {
     std::lock_guard<std::mutex> lock(g_mu);
-    if (ds->ws_bytes < L.total) {
+    if (ds->ws_bytes < need) {
       cudaError_t e;
       if (ds->ws) {
         e = cudaDeviceSynchronize();
@@ -561,7 +669,7 @@ int decode_impl(const pa_tensor *out, const pa_tensor *query, const pa_tensor *k
         ds->ws = nullptr;
         ds->ws_bytes = 0;
       }
-      const size_t want = L.total + L.total / 4;
+      const size_t want = need + need / 4;
       e = cudaMalloc(&ds->ws, want);
       if (e != cudaSuccess) return cuda_fail(e, "cudaMalloc(decode workspace)");
       e = cudaMemsetAsync(ds->ws, 0, want, st);
@@ -572,8 +680,8 @@ int decode_impl(const pa_tensor *out, const pa_tensor *query, const pa_tensor *k
     workspace = ds->ws;
     workspace_bytes = ds->ws_bytes;
   } else {
-    if (!workspace || workspace_bytes < L.total)
-      return fail(PA_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", L.total, workspace_bytes);
+    if (!workspace || workspace_bytes < need)
+      return fail(PA_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", need, workspace_bytes);
     if (((uintptr_t)workspace & 255u) != 0) return fail(PA_ERR_WORKSPACE, "workspace must be 256-byte aligned");
   }
   {
@@ -588,7 +696,7 @@ int decode_impl(const pa_tensor *out, const pa_tensor *query, const pa_tensor *k
     rec.clean = counter_bytes;
   }
 
-  pa::DecodeArgs a;
+  pa::DecodeArgs a = {};
   a.out = out->data;
   a.out_dtype = out->dtype;
   a.out_s = out->stride[0];
@@ -626,8 +734,20 @@ int decode_impl(const pa_tensor *out, const pa_tensor *query, const pa_tensor *k
     a.timeline = g_timeline;
     a.timeline_warps = g_timeline_warps;
   }
+  bool overlap = (flags & PA_DECODE_OVERLAP_PREVIOUS) != 0;
+  if (shared) {
+    a.prefix_lens = static_cast<const int32_t *>(prefix_lens->data);
+    a.pre_ml = reinterpret_cast<float *>(ws + PL.pre_ml);
+    a.pre_o = reinterpret_cast<float *>(ws + PL.pre_o);
+    a.pre_splits = PL.splits;
+    a.pre_kv_tokens = kPrefixItemTokens;
+    if ((rc = launch_prefix_pass(a, query, key_cache, value_cache, group_start, cs, D, G,
+                                 block_size, ds, st)))
+      return rc;
+    overlap = true;  // the decode's prologue runs while the prefix pass finishes
+  }
   const int ctas = (W + k.warps_per_cta - 1) / k.warps_per_cta;  // warps_per_cta workers each
-  cudaError_t e = k.launch(a, &maps, ctas, (flags & PA_DECODE_OVERLAP_PREVIOUS) != 0, st);
+  cudaError_t e = k.launch(a, &maps, ctas, overlap, st);
   if (e != cudaSuccess) return cuda_fail(e, "decode launch");
   if (a.separate_reduce) {
     e = k.launch_reduce(a, st);
@@ -955,7 +1075,7 @@ int pa_prefill(const pa_tensor *out, const pa_tensor *query, const pa_tensor *ke
     per_sm = 1;
   const int64_t wave = (int64_t)per_sm * ds->num_sms;
   const int ctas = (int)(tiles < wave ? tiles : wave);
-  pa::PrefillArgs a;
+  pa::PrefillArgs a = {};
   a.out = out->data;
   a.out_dtype = out->dtype;
   a.out_t = out->stride[0];
@@ -1054,6 +1174,28 @@ int pa_decode_ex(const pa_tensor *out, const pa_tensor *query, const pa_tensor *
   return decode_impl(out, query, key_cache, value_cache, block_tables, context_lens, scale,
                      block_size, num_kv_heads, num_workers, flags, workspace, workspace_bytes,
                      false, stream);
+}
+
+int pa_decode_shared_prefix(const pa_tensor *out, const pa_tensor *query, const pa_tensor *key_cache,
+                            const pa_tensor *value_cache, const pa_tensor *block_tables,
+                            const pa_tensor *context_lens, const pa_tensor *group_start,
+                            const pa_tensor *prefix_lens, float scale, int32_t block_size,
+                            int32_t num_kv_heads, void *workspace, size_t workspace_bytes,
+                            void *stream) {
+  if (!group_start) return fail(PA_ERR_INVALID_ARG, "group_start is required");
+  return decode_impl(out, query, key_cache, value_cache, block_tables, context_lens, scale,
+                     block_size, num_kv_heads, 0, 0u, workspace, workspace_bytes,
+                     workspace == nullptr, stream, CallMode::kLaunch, nullptr, nullptr,
+                     group_start, prefix_lens);
+}
+
+size_t pa_decode_shared_prefix_workspace_bytes(int64_t num_seqs, int32_t num_heads,
+                                               int32_t num_kv_heads, int32_t head_dim,
+                                               int64_t max_blocks_per_seq, int32_t block_size) {
+  if (max_blocks_per_seq < 0 || block_size <= 0) return 0;
+  const size_t base = pa_decode_workspace_bytes(num_seqs, num_heads, num_kv_heads, head_dim, 0);
+  if (base == 0) return 0;
+  return prefix_layout(base, num_seqs, num_heads, head_dim, max_blocks_per_seq, block_size).total;
 }
 
 size_t pa_decode_workspace_bytes(int64_t num_seqs, int32_t num_heads, int32_t num_kv_heads,

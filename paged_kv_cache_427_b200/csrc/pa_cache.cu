@@ -17,8 +17,10 @@ namespace pa {
 
 // One thread per 16-byte piece of one (token, kv head) row, keys and values together.
 __global__ void __launch_bounds__(256) reshape_and_cache_kernel(CacheWriteArgs a) {
-  // A decode launched to overlap this grid may start now; it waits for this grid's writes
-  // before it reads the caches.
+  // Launched as a programmatic dependent of the kernel before it: wait for that kernel (and its
+  // memory) before touching anything.  Then a decode launched to overlap this grid may start;
+  // it waits for this grid's writes before it reads the caches.
+  wait_for_previous_grid();
   allow_next_grid();
   const int vec_per_row = a.row_bytes >> 4;
   const int64_t total = a.num_tokens * a.num_kv_heads * vec_per_row;
@@ -49,6 +51,8 @@ __global__ void __launch_bounds__(256) reshape_and_cache_kernel(CacheWriteArgs a
 // and destination caches may be the same tensors (copy-on-write) or live in different memory
 // (swap between device memory and pinned host memory mapped into the device's address space).
 __global__ void __launch_bounds__(256) copy_blocks_kernel(CopyBlocksArgs a) {
+  wait_for_previous_grid();  // launched as a programmatic dependent, as the write kernel
+  allow_next_grid();
   const int vec_per_tile = a.tile_bytes >> 4;
   const int64_t total = a.num_pairs * a.num_kv_heads * vec_per_tile;
   for (int64_t idx = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; idx < total;
@@ -106,6 +110,7 @@ __device__ __forceinline__ void load_row16(const char *p, float (&f)[16]) {
 // Each element is divided by its head's scale in fp32 (IEEE division) before the conversion.
 template <typename S>
 __global__ void __launch_bounds__(256) reshape_and_cache_fp8_kernel(CacheWriteFp8Args a) {
+  wait_for_previous_grid();  // launched as a programmatic dependent, as the 16-bit write
   allow_next_grid();
   const int vec_per_row = a.head_dim >> 4;
   const int64_t total = a.num_tokens * a.num_kv_heads * vec_per_row;
@@ -146,31 +151,43 @@ static int grid_for(int64_t items, int num_sms) {
   return (int)(blocks < 1 ? 1 : (blocks > cap ? cap : blocks));
 }
 
+// Launch as a programmatic dependent of the kernel before it on `st`: the grid may become
+// resident while that kernel finishes (its launch latency hidden behind that kernel's last
+// CTAs); every thread waits for that kernel and its memory before it reads or writes anything.
+template <typename A>
+cudaError_t launch_dependent(void (*kernel)(A), int grid, cudaStream_t st, const A &a) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(256);
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, a);
+}
+
 cudaError_t launch_reshape_and_cache(const CacheWriteArgs &a, int num_sms, cudaStream_t st) {
   const int64_t items = a.num_tokens * a.num_kv_heads * (a.row_bytes / 16);
   if (items == 0) return cudaSuccess;
-  reshape_and_cache_kernel<<<grid_for(items, num_sms), 256, 0, st>>>(a);
-  return cudaGetLastError();
+  return launch_dependent(reshape_and_cache_kernel, grid_for(items, num_sms), st, a);
 }
 
 cudaError_t launch_copy_blocks(const CopyBlocksArgs &a, int num_sms, cudaStream_t st) {
   const int64_t items = a.num_pairs * a.num_kv_heads * (a.tile_bytes / 16);
   if (items == 0) return cudaSuccess;
-  copy_blocks_kernel<<<grid_for(items, num_sms), 256, 0, st>>>(a);
-  return cudaGetLastError();
+  return launch_dependent(copy_blocks_kernel, grid_for(items, num_sms), st, a);
 }
 
 cudaError_t launch_reshape_and_cache_fp8(const CacheWriteFp8Args &a, int num_sms, cudaStream_t st) {
   const int64_t items = a.num_tokens * a.num_kv_heads * (a.head_dim / 16);
   if (items == 0) return cudaSuccess;
   const int grid = grid_for(items, num_sms);
-  if (a.src_dtype == PA_F32)
-    reshape_and_cache_fp8_kernel<float><<<grid, 256, 0, st>>>(a);
-  else if (a.src_dtype == PA_BF16)
-    reshape_and_cache_fp8_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(a);
-  else
-    reshape_and_cache_fp8_kernel<__half><<<grid, 256, 0, st>>>(a);
-  return cudaGetLastError();
+  if (a.src_dtype == PA_F32) return launch_dependent(reshape_and_cache_fp8_kernel<float>, grid, st, a);
+  if (a.src_dtype == PA_BF16)
+    return launch_dependent(reshape_and_cache_fp8_kernel<__nv_bfloat16>, grid, st, a);
+  return launch_dependent(reshape_and_cache_fp8_kernel<__half>, grid, st, a);
 }
 
 }  // namespace pa

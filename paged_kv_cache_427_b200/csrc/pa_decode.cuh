@@ -85,7 +85,7 @@ __global__ void __launch_bounds__(128, 1) paged_decode_kernel(const DecodeArgs a
   const int max_len = a.max_blocks * BS;
 
   WarpShare share;
-  if (!split_prologue<CH, Tr::kWarps, G, D>(a, max_len, share)) return;
+  if (!split_prologue<CH, Tr::kWarps, G, D, BS>(a, max_len, share)) return;
   const int gw = blockIdx.x * Tr::kWarps + wid;
 
   unsigned char *wsm = smem + wid * Tr::kWarpBytes;
@@ -307,7 +307,9 @@ __global__ void __launch_bounds__(128, 1) paged_decode_kernel(const DecodeArgs a
       }
       if (a.separate_reduce && piece_at_start && lane == 0)
         a.pair_meta[m.pair] = make_int2(m.first_worker, m.npieces);
-      if (m.npieces == 1) {
+      // a (sequence, kv head) inside one share is written directly, unless it has partial
+      // results of a shared prefix to merge with
+      if (m.npieces == 1 && (a.prefix_lens == nullptr || prefix_pieces<BS>(a, m.s, max_len) == 0)) {
         if (r == 0) {
           const int out_elt = a.out_dtype == PA_F32 ? 4 : 2;
 #pragma unroll
@@ -345,7 +347,7 @@ __global__ void __launch_bounds__(128, 1) paged_decode_kernel(const DecodeArgs a
             if (lane == h) ml = make_float2(mh[h], lh[h]);
           *reinterpret_cast<float2 *>(a.part_ml + (seg * G + lane) * 2) = ml;
         }
-        finish_piece<G, D>(a, m, lane);
+        finish_piece<G, D, BS>(a, m, lane);
       }
     }
     __syncwarp();

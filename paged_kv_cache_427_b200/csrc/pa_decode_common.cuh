@@ -43,6 +43,32 @@ __device__ __forceinline__ int worker_of(long long c, long long C, int W) {
   return (int)(((c + 1) * (long long)W + C - 1) / C - 1);
 }
 
+// The first position the decode reads of sequence s, whose context holds len positions: its
+// shared prefix when the shared-prefix pass covered it (0 < prefix < len, a multiple of the block
+// size, within the pass's items), else 0 (the whole context is decoded here).  A prefix that is
+// not a multiple of the block size or needs more items than the workspace holds is reported.
+template <int BS>
+__device__ __forceinline__ int decode_start(const DecodeArgs &a, int s, int len) {
+  if (a.prefix_lens == nullptr) return 0;
+  const int p = __ldg(a.prefix_lens + s);
+  if (p <= 0 || p >= len) return 0;
+  if (p % BS != 0 || (p + a.pre_kv_tokens - 1) / a.pre_kv_tokens > a.pre_splits) {
+    set_error(a.err, PA_DEVERR_PREFIX);
+    return 0;
+  }
+  return p;
+}
+
+// The number of prefix-pass partial results sequence s merges (0 without a shared prefix).
+template <int BS>
+__device__ __forceinline__ int prefix_pieces(const DecodeArgs &a, int s, int max_len) {
+  if (a.prefix_lens == nullptr) return 0;
+  const int raw = __ldg(a.context_lens + s);
+  const int len = raw < 0 ? 0 : (raw > max_len ? max_len : raw);
+  const int p = decode_start<BS>(a, s, len);
+  return p > 0 ? (p + a.pre_kv_tokens - 1) / a.pre_kv_tokens : 0;
+}
+
 // Test hook: whether worker warp gw's first stage waits for 16 bytes that no copy sends
 // (mode 1: every worker; mode 2: the odd-numbered workers only).
 __device__ __forceinline__ bool test_stalls(const DecodeArgs &a, int gw) {
@@ -79,7 +105,7 @@ __device__ __forceinline__ long long warp_sum(long long x) {
 // 32 sequences at a time.  No shared memory and no block-wide barrier, so warps start as soon
 // as they are scheduled.  Warp gw also flags bad lengths (warp 0) and zeroes the rows of empty
 // contexts s with s % (warps launched) == gw.  Returns false when this warp has no work.
-template <int CH, int kWarps, int G, int D>
+template <int CH, int kWarps, int G, int D, int BS>
 __device__ __forceinline__ bool split_prologue(const DecodeArgs &a, int max_len, WarpShare &ws) {
   const int lane = threadIdx.x & 31;
   const int gw = blockIdx.x * kWarps + (threadIdx.x >> 5);
@@ -96,7 +122,7 @@ __device__ __forceinline__ bool split_prologue(const DecodeArgs &a, int max_len,
       if (len == 0 && s % launched == gw)
         zero_rows<D>(static_cast<char *>(a.out) + (long long)s * a.out_s * (a.out_dtype == PA_F32 ? 4 : 2),
                      a.out_h, a.out_dtype, Hkv * G);
-      mine += (len + CH - 1) / CH;
+      mine += (len - decode_start<BS>(a, s, len) + CH - 1) / CH;
     }
   }
   const long long C = warp_sum(mine) * Hkv;
@@ -109,7 +135,8 @@ __device__ __forceinline__ bool split_prologue(const DecodeArgs &a, int max_len,
   long long running = 0;
   for (int base = 0; base < S; base += 32) {
     const int s = base + lane;
-    const int len = s < S ? clamp_len(__ldg(a.context_lens + s), max_len) : 0;
+    const int full = s < S ? clamp_len(__ldg(a.context_lens + s), max_len) : 0;
+    const int len = s < S ? full - decode_start<BS>(a, s, full) : 0;  // positions decoded here
     const long long cnt = (long long)((len + CH - 1) / CH) * Hkv;
     long long incl = cnt;
 #pragma unroll
@@ -137,6 +164,7 @@ __device__ __forceinline__ bool split_prologue(const DecodeArgs &a, int max_len,
 template <int CH, int BS, int COPIES, int COPY_ROWS>
 struct ChunkCursor {
   int s, len, nch, kvh, i, next_len;
+  int start, next_start;  // first decoded position of the sequence (its shared prefix, or 0)
   long long base;  // global index of chunk 0 of the current (sequence, kv head)
   int first_worker, npieces;
   long long issued, n, C;
@@ -147,7 +175,7 @@ struct ChunkCursor {
 #pragma unroll
     for (int k = 0; k < COPIES; ++k) {
       const int t = i * CH + k * COPY_ROWS;
-      blk[k] = (t < len) ? __ldg(a.block_tables + (long long)s * a.bt_s + t / BS) : 0;
+      blk[k] = (t < len) ? __ldg(a.block_tables + (long long)s * a.bt_s + (start + t) / BS) : 0;
     }
   }
 
@@ -166,13 +194,25 @@ struct ChunkCursor {
     issued = 0;
     s = ws.s;
     len = ws.len;
+    start = decode_start<BS>(a, s, clamp_len(__ldg(a.context_lens + s), max_len));
     nch = (len + CH - 1) / CH;
     kvh = ws.rem / nch;
     i = ws.rem % nch;
     base = ws.g0 - ws.rem + (long long)kvh * nch;
-    next_len = (s + 1 < S) ? clamp_len(__ldg(a.context_lens + s + 1), max_len) : 0;
+    load_next(a);
     fetch_blocks(a);
     pieces();
+  }
+
+  // Decoded length and start of sequence s + 1.
+  __device__ __forceinline__ void load_next(const DecodeArgs &a) {
+    next_len = 0;
+    next_start = 0;
+    if (s + 1 < S) {
+      const int full = clamp_len(__ldg(a.context_lens + s + 1), max_len);
+      next_start = decode_start<BS>(a, s + 1, full);
+      next_len = full - next_start;
+    }
   }
 
   __device__ __forceinline__ int flags() const {
@@ -215,12 +255,15 @@ struct ChunkCursor {
         kvh = 0;
         ++s;
         len = next_len;
+        start = next_start;
         while (len == 0 && s + 1 < S) {
           ++s;
-          len = clamp_len(__ldg(a.context_lens + s), max_len);
+          const int full = clamp_len(__ldg(a.context_lens + s), max_len);
+          start = decode_start<BS>(a, s, full);
+          len = full - start;
         }
         nch = (len + CH - 1) / CH;
-        next_len = (s + 1 < S) ? clamp_len(__ldg(a.context_lens + s + 1), max_len) : 0;
+        load_next(a);
       }
       pieces();
     }
@@ -229,13 +272,28 @@ struct ChunkCursor {
 };
 
 // Merge the pieces (o, m, l) of one (sequence, kv head) and write its G output rows.  Called by
-// a whole warp; pieces live in workspace slots pair + first_worker + k, k < npieces.  Loads are
-// issued for many pieces at once (lane k fetches piece k's (m, l); then 4 pieces' outputs per
-// round) so a merge costs a few memory round trips, not two per piece.  m is in base-2 units.
+// a whole warp; pieces live in workspace slots pair + first_worker + k, k < npieces, followed by
+// the npre partial results of the shared-prefix pass (slots of the query head, item k - npieces).
+// Loads are issued for many pieces at once (lane k fetches piece k's (m, l); then 4 pieces'
+// outputs per round) so a merge costs a few memory round trips, not two per piece.  m is in
+// base-2 units.
 template <int G, int D>
 __device__ __forceinline__ void merge_pieces(const DecodeArgs &a, int pair, int first_worker,
-                                             int npieces, int s, int kvh, int lane) {
+                                             int npieces, int s, int kvh, int lane, int npre = 0) {
   const long long seg0 = (long long)pair + first_worker;
+  const long long pre0 = ((long long)s * a.num_kv_heads + kvh) * G;  // first query head's slots
+  const int total = npieces + npre;
+  // (m, l) and output of piece k for head h
+  auto ml_of = [&](int k, int h) -> const float2 * {
+    return k < npieces
+               ? reinterpret_cast<const float2 *>(a.part_ml + ((seg0 + k) * G + h) * 2)
+               : reinterpret_cast<const float2 *>(a.pre_ml + ((pre0 + h) * a.pre_splits + (k - npieces)) * 2);
+  };
+  auto o_of = [&](int k, int h) -> const float4 * {
+    return k < npieces
+               ? reinterpret_cast<const float4 *>(a.part_o + ((seg0 + k) * G + h) * D)
+               : reinterpret_cast<const float4 *>(a.pre_o + ((pre0 + h) * a.pre_splits + (k - npieces)) * D);
+  };
   const bool active = lane < D / 4;  // lane j handles dims [4j, 4j+4) of every head
   float M[G], den[G];
   float4 num[G];
@@ -245,8 +303,8 @@ __device__ __forceinline__ void merge_pieces(const DecodeArgs &a, int pair, int 
     den[h] = 0.f;
     num[h] = make_float4(0.f, 0.f, 0.f, 0.f);
   }
-  for (int base = 0; base < npieces; base += 32) {
-    const int cnt = npieces - base < 32 ? npieces - base : 32;
+  for (int base = 0; base < total; base += 32) {
+    const int cnt = total - base < 32 ? total - base : 32;
     // lane k < cnt: (m, l) of piece base + k for every head
     float mk[G], lk[G];
 #pragma unroll
@@ -257,7 +315,7 @@ __device__ __forceinline__ void merge_pieces(const DecodeArgs &a, int pair, int 
     if (lane < cnt) {
 #pragma unroll
       for (int h = 0; h < G; ++h) {
-        const float2 ml = __ldcg(reinterpret_cast<const float2 *>(a.part_ml + ((seg0 + base + lane) * G + h) * 2));
+        const float2 ml = __ldcg(ml_of(base + lane, h));
         mk[h] = ml.x;
         lk[h] = ml.y;
       }
@@ -292,9 +350,8 @@ __device__ __forceinline__ void merge_pieces(const DecodeArgs &a, int pair, int 
       for (int u = 0; u < U; ++u)
 #pragma unroll
         for (int h = 0; h < G; ++h)
-          x[u][h] = (active && k + u < cnt)
-                        ? __ldcg(reinterpret_cast<const float4 *>(a.part_o + ((seg0 + base + k + u) * G + h) * D) + lane)
-                        : make_float4(0.f, 0.f, 0.f, 0.f);
+          x[u][h] = (active && k + u < cnt) ? __ldcg(o_of(base + k + u, h) + lane)
+                                            : make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
       for (int u = 0; u < U; ++u)
 #pragma unroll
@@ -335,6 +392,25 @@ __device__ __forceinline__ void merge_pieces(const DecodeArgs &a, int pair, int 
   }
 }
 
+#ifndef PA_TICKET_ACQREL
+#define PA_TICKET_ACQREL 0  // 1: merge tickets by one acquire-release atomic, no separate fences
+#endif
+
+// Take a ticket of a merge counter.  With PA_TICKET_ACQREL the atomic has acquire-release
+// semantics at GPU scope: the release orders the warp's stores of its piece (made visible to
+// lane 0 by the warp barrier before it) before the increment, and the acquire orders the loads
+// of the other pieces after it for the warp that takes the last ticket: one round trip in
+// place of a fence followed by an atomic and a second fence.  Called by lane 0.
+__device__ __forceinline__ unsigned int ticket_add(unsigned int *counter) {
+#if PA_TICKET_ACQREL
+  unsigned int old;
+  asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;" : "=r"(old) : "l"(counter) : "memory");
+  return old;
+#else
+  return atomicAdd(counter, 1u);
+#endif
+}
+
 // What a worker needs to take a split piece's ticket after its (o, m, l) are stored.
 struct PieceInfo {
   int pair, first_worker, npieces, s, kvh;
@@ -342,31 +418,36 @@ struct PieceInfo {
 
 // Take the ticket of a published piece and merge when it is the last of its (sequence, kv
 // head).  The caller has made the piece's stores visible GPU-wide.  Called by a whole warp.
-template <int G, int D>
+template <int G, int D, int BS>
 __device__ __forceinline__ void take_ticket(const DecodeArgs &a, const PieceInfo &p, int lane) {
   unsigned int ticket = 0;
-  if (lane == 0) ticket = atomicAdd(a.counters + p.pair, 1u);
+  __syncwarp();
+  if (lane == 0) ticket = ticket_add(a.counters + p.pair);
   ticket = __shfl_sync(FULL_MASK, ticket, 0);
   if (ticket == (unsigned int)(p.npieces - 1)) {
-    __threadfence();
-    merge_pieces<G, D>(a, p.pair, p.first_worker, p.npieces, p.s, p.kvh, lane);
+    if (!PA_TICKET_ACQREL) __threadfence();
+    __syncwarp();
+    merge_pieces<G, D>(a, p.pair, p.first_worker, p.npieces, p.s, p.kvh, lane,
+                       prefix_pieces<BS>(a, p.s, a.max_blocks * BS));
     if (lane == 0) a.counters[p.pair] = 0u;
   }
 }
 
 // After a piece's (o, m, l) are stored: publish them, take a ticket, and merge when this is the
 // last piece of its (sequence, kv head).  Called by a whole warp.
-template <int G, int D>
+template <int G, int D, int BS>
 __device__ __forceinline__ void finish_piece(const DecodeArgs &a, const ChunkMeta &m, int lane) {
   if (a.separate_reduce) return;
-  __threadfence();
+  if (!PA_TICKET_ACQREL) __threadfence();
   __syncwarp();
   unsigned int ticket = 0;
-  if (lane == 0) ticket = atomicAdd(a.counters + m.pair, 1u);
+  if (lane == 0) ticket = ticket_add(a.counters + m.pair);
   ticket = __shfl_sync(FULL_MASK, ticket, 0);
   if (ticket == (unsigned int)(m.npieces - 1)) {
-    __threadfence();
-    merge_pieces<G, D>(a, m.pair, m.first_worker, m.npieces, m.s, m.kvh, lane);
+    if (!PA_TICKET_ACQREL) __threadfence();
+    __syncwarp();
+    merge_pieces<G, D>(a, m.pair, m.first_worker, m.npieces, m.s, m.kvh, lane,
+                       prefix_pieces<BS>(a, m.s, a.max_blocks * BS));
     if (lane == 0) a.counters[m.pair] = 0u;
   }
 }

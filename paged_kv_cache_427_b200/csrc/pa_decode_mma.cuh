@@ -123,6 +123,16 @@ __device__ __forceinline__ bool mbar_test(uint64_t *bar, uint32_t parity) {
   return done != 0;
 }
 
+#ifndef PA_DECODE_STAGES
+#define PA_DECODE_STAGES 2  // stages per worker, 16-bit caches
+#endif
+#ifndef PA_EARLY_ISSUE
+#define PA_EARLY_ISSUE 0  // issue the first stages before the previous grid has finished
+#endif
+#ifndef PA_FP8_MAX_STAGES
+#define PA_FP8_MAX_STAGES 5  // most stages per worker, FP8 caches
+#endif
+
 // KVB: bytes per cache element (2: bf16/fp16, 1: FP8 E4M3).  The query is 16-bit either way.
 template <int D, int BS, int G, int KVB = 2>
 struct MmaTraits {
@@ -140,7 +150,13 @@ struct MmaTraits {
   // in flight than HBM needs to run at full rate; the longer queues only raise the latency
   // every worker sees and widen the spread of finishing times (measured: the Llama-shaped
   // decode 60 -> 58 us, the long mixed batch 275 -> 259 us).
-  static constexpr int kStages = KVB == 2 ? 2 : 3;  // FP8 stages hold half the bytes
+  // FP8 stages hold half the bytes, so a worker needs more of them for the same bytes in flight:
+  // as many as keep two CTAs per SM (about 110 KB of shared memory each), at most kMaxFp8Stages.
+  static constexpr int kMaxFp8Stages = PA_FP8_MAX_STAGES;
+  static constexpr int kFp8Stages = (110 * 1024) / (kWorkers * kStageBytes) < kMaxFp8Stages
+                                        ? (110 * 1024) / (kWorkers * kStageBytes)
+                                        : kMaxFp8Stages;
+  static constexpr int kStages = KVB == 2 ? PA_DECODE_STAGES : kFp8Stages;
   static constexpr int kRingBytes = kWorkers * kStages * kStageBytes;
   static constexpr int kPbufBytes = 2 * 8 * 16 * 2;    // [hi, lo][8 heads][16 tokens]
   static constexpr int kMetaOff = 0;
@@ -244,7 +260,7 @@ __global__ void __launch_bounds__(MmaTraits<D, BS, G, (int)sizeof(KV)>::kThreads
     }
     WarpShare ws;
     ws.n = 0;
-    const bool has = split_prologue<16, NW, G, D>(a, max_len, ws);
+    const bool has = split_prologue<16, NW, G, D, BS>(a, max_len, ws);
     if (lane == 0) {
       ShareRecord r;
       r.s = has ? ws.s : -1;
@@ -303,6 +319,51 @@ __global__ void __launch_bounds__(MmaTraits<D, BS, G, (int)sizeof(KV)>::kThreads
         }
       }
     }
+    // One stage of this lane's worker: the chunk's key and value boxes, plus the group's query
+    // rows when a new (sequence, kv head) starts, all counted on the stage's full barrier.
+    auto issue = [&](int slot) {
+      const int f = cur.flags();
+      unsigned char *stage = ring + slot * Tr::kStageBytes;
+      meta[slot] = cur.meta(f);
+      const uint32_t bytes = 2u * cur.valid_copies() * Tr::kBoxBytes +
+                             ((f & kFirst) ? (uint32_t)Tr::kQBytes : 0u) +
+                             ((cur.issued == 0 && test_stalls(a, blockIdx.x * NW + k)) ? 16u : 0u);
+      mbar_arrive_expect_tx(full + slot, bytes);
+#pragma unroll
+      for (int c = 0; c < Tr::kCopies; ++c) {
+        const int t = cur.i * 16 + c * Tr::kBoxRows;
+        if (t < cur.len) {
+          int blk = cur.blk[c];
+          if (blk < 0 || (long long)blk >= a.num_blocks) {
+            set_error(a.err, PA_DEVERR_BLOCK_ID);
+            blk = 0;
+          }
+          const uint32_t off = c * Tr::kBoxBytes;
+          tma_load_tile(smem_u32(stage + off), &maps.k, t % BS, cur.kvh, blk, full + slot);
+          tma_load_tile(smem_u32(stage + Tr::kTileBytes + off), &maps.v, t % BS, cur.kvh, blk,
+                        full + slot);
+        }
+      }
+      if (f & kFirst) {
+        const char *q = static_cast<const char *>(a.query) +
+                        ((long long)cur.s * a.q_s + (long long)cur.kvh * G * a.q_h) * 2;
+        if (a.q_heads_contiguous) {
+          bulk_copy_g2s(stage + 2 * Tr::kTileBytes, q, Tr::kQBytes, full + slot);
+        } else {
+#pragma unroll
+          for (int h = 0; h < G; ++h)
+            bulk_copy_g2s(stage + 2 * Tr::kTileBytes + h * D * 2, q + (long long)h * a.q_h * 2,
+                          D * 2, full + slot);
+        }
+      }
+      cur.advance(a);
+      if (cur.issued >= cur.n) active = false;
+    };
+#if PA_EARLY_ISSUE
+    // The first stages of chunks that end before the sequence's last position: the grid before
+    // this one writes only that position of each sequence (the step's new token).
+    while (active && cur.issued < ST && (cur.i + 1) * 16 < cur.len) issue((int)(cur.issued % ST));
+#endif
     // A grid launched after this one (the separate merge) may start now and wait for us.
     if (lane == 0) allow_next_grid();
     // Everything above read only context_lens and block_tables; the caches and the query may
@@ -319,44 +380,7 @@ __global__ void __launch_bounds__(MmaTraits<D, BS, G, (int)sizeof(KV)>::kThreads
         can = cur.issued < ST ||
               mbar_test(empty + slot, (uint32_t)(((cur.issued / ST) - 1) & 1));
       }
-      if (can) {
-        const int f = cur.flags();
-        unsigned char *stage = ring + slot * Tr::kStageBytes;
-        meta[slot] = cur.meta(f);
-        const uint32_t bytes = 2u * cur.valid_copies() * Tr::kBoxBytes +
-                               ((f & kFirst) ? (uint32_t)Tr::kQBytes : 0u) +
-                               ((cur.issued == 0 && test_stalls(a, blockIdx.x * NW + k)) ? 16u : 0u);
-        mbar_arrive_expect_tx(full + slot, bytes);
-#pragma unroll
-        for (int c = 0; c < Tr::kCopies; ++c) {
-          const int t = cur.i * 16 + c * Tr::kBoxRows;
-          if (t < cur.len) {
-            int blk = cur.blk[c];
-            if (blk < 0 || (long long)blk >= a.num_blocks) {
-              set_error(a.err, PA_DEVERR_BLOCK_ID);
-              blk = 0;
-            }
-            const uint32_t off = c * Tr::kBoxBytes;
-            tma_load_tile(smem_u32(stage + off), &maps.k, t % BS, cur.kvh, blk, full + slot);
-            tma_load_tile(smem_u32(stage + Tr::kTileBytes + off), &maps.v, t % BS, cur.kvh, blk,
-                          full + slot);
-          }
-        }
-        if (f & kFirst) {
-          const char *q = static_cast<const char *>(a.query) +
-                          ((long long)cur.s * a.q_s + (long long)cur.kvh * G * a.q_h) * 2;
-          if (a.q_heads_contiguous) {
-            bulk_copy_g2s(stage + 2 * Tr::kTileBytes, q, Tr::kQBytes, full + slot);
-          } else {
-#pragma unroll
-            for (int h = 0; h < G; ++h)
-              bulk_copy_g2s(stage + 2 * Tr::kTileBytes + h * D * 2, q + (long long)h * a.q_h * 2,
-                            D * 2, full + slot);
-          }
-        }
-        cur.advance(a);
-        if (cur.issued >= cur.n) active = false;
-      }
+      if (can) issue(slot);
       if (__any_sync(FULL_MASK, can)) {
         last_progress = clock64();
       } else {
@@ -400,9 +424,9 @@ __global__ void __launch_bounds__(MmaTraits<D, BS, G, (int)sizeof(KV)>::kThreads
         if (p.npieces == 0) {
           if (lane == k) fin = true;
         } else {
-          __threadfence();
+          if (!PA_TICKET_ACQREL) __threadfence();
           __syncwarp();
-          take_ticket<G, D>(a, p, lane);
+          take_ticket<G, D, BS>(a, p, lane);
         }
         if (lane == k) ++seen;
       }
@@ -694,7 +718,9 @@ __global__ void __launch_bounds__(MmaTraits<D, BS, G, (int)sizeof(KV)>::kThreads
       }
       if (a.separate_reduce && piece_at_start && lane == 0)
         a.pair_meta[m.pair] = make_int2(m.first_worker, m.npieces);
-      if (m.npieces == 1) {
+      // a (sequence, kv head) inside one share is written directly, unless it has partial
+      // results of a shared prefix to merge with
+      if (m.npieces == 1 && (a.prefix_lens == nullptr || prefix_pieces<BS>(a, m.s, max_len) == 0)) {
         const int out_elt = a.out_dtype == PA_F32 ? 4 : 2;
         char *row0 = static_cast<char *>(a.out) +
                      ((long long)m.s * a.out_s + (long long)(m.kvh * G + h0) * a.out_h) * out_elt;
@@ -766,7 +792,7 @@ __global__ void __launch_bounds__(MmaTraits<D, BS, G, (int)sizeof(KV)>::kThreads
           } else {
             // the share's last piece: nothing is left to overlap the fence with, and the four
             // workers publish their last pieces in parallel rather than through one merge warp
-            finish_piece<G, D>(a, m, lane);
+            finish_piece<G, D, BS>(a, m, lane);
           }
         }
       }

@@ -45,6 +45,16 @@ struct DecodeArgs {
   // (those with index < timeline_warps), or null.
   unsigned long long *timeline;
   long long timeline_warps;
+  // Shared prefixes (pa_decode_shared_prefix), or null: sequence s decodes only positions
+  // prefix_lens[s] .. L-1 when 0 < prefix_lens[s] < L and prefix_lens[s] is a multiple of the
+  // block size (otherwise its whole context), and merges the pre_splits partial results
+  // (pre_o, pre_ml, laid out as in the prefill's shared-prefix pass) that the prefix pass left
+  // for its first ceil(ceil(prefix / pre_kv_tokens)) items.
+  const int32_t *prefix_lens;
+  const float *pre_o;
+  const float *pre_ml;
+  int pre_splits;
+  int pre_kv_tokens;  // positions per prefix item
 };
 
 // Fields of one worker warp's timeline record.

@@ -27,6 +27,19 @@ struct PrefillArgs {
   unsigned int *err;
   long long wait_cycles;
   int grouped_maps;  // 1: the maps are the grouped view (one box per block and kv head)
+  // Shared-prefix pass (pa_decode_shared_prefix) when pre_o is not null: the query rows are the
+  // decode queries of consecutive sequences (query_start unused), group g's members are
+  // sequences group_start[g] .. group_start[g+1]-1, and every member's rows attend, with no
+  // causal limit, to positions 0 .. P-1 of the group's shared prefix, P = prefix_lens of the
+  // first member, read through the first member's block table.  The work is cut into items
+  // of pre_kv kv tiles; item sigma of (member, head) stores O / l and (m, l), m in base 2.
+  const int32_t *group_start;  // [num_groups + 1]
+  const int32_t *prefix_lens;  // [num_seqs]
+  int num_groups;
+  int pre_kv;                  // kv tiles (128 positions) per item
+  int pre_splits;              // item slots per (sequence, query head)
+  float *pre_o;                // [num_seqs][num_heads][pre_splits][head_dim]
+  float *pre_ml;               // [num_seqs][num_heads][pre_splits][2]
 };
 
 // The prefill's tensor maps: the caches (grouped view, or 8-row boxes) and the query rows.

@@ -146,7 +146,66 @@ struct TcTile {
   int q0, q_len, L;
   int tok0, ntok, pos0, n_kv;
   bool valid;
+  int j0;          // first kv tile of the item (0 unless the shared-prefix pass splits the range)
+  int slot;        // the item's slot among a (sequence, head)'s partial results (prefix pass)
+  bool noncausal;  // every row sees positions 0 .. L-1 (prefix pass)
 };
+
+// Shared-prefix pass: the prefix length of group g (that of its first member, clamped to the
+// block table) and its members; 0 members when the group is malformed.
+__device__ __forceinline__ void prefix_group(const PrefillArgs &a, int g, int max_len, int &first,
+                                             int &members, int &P) {
+  first = __ldg(a.group_start + g);
+  const int end = __ldg(a.group_start + g + 1);
+  members = end - first;
+  P = 0;
+  if (first < 0 || members < 0 || (long long)end > a.num_tokens) {
+    members = 0;
+    return;
+  }
+  if (members > 0) {
+    const int raw = __ldg(a.prefix_lens + first);
+    P = raw < 0 ? 0 : (raw > max_len ? max_len : raw);
+  }
+}
+
+// Warp-cooperative: the group holding item y of the shared-prefix pass (items ordered by
+// group, then kv head, row tile, split) and y's index within the group; g = -1 past the end.
+template <int TOK, int KV>
+__device__ __forceinline__ void locate_prefix_item(const PrefillArgs &a, int max_len, long long y,
+                                                   int &g_out, long long &rem_out) {
+  const int lane = threadIdx.x & 31;
+  long long running = 0;
+  for (int base = 0; base < a.num_groups; base += 32) {
+    const int g = base + lane;
+    long long cnt = 0;
+    if (g < a.num_groups) {
+      int first, members, P;
+      prefix_group(a, g, max_len, first, members, P);
+      if (members > 0 && P > 0) {
+        const int splits = ((P + KV - 1) / KV + a.pre_kv - 1) / a.pre_kv;
+        cnt = (long long)((members + TOK - 1) / TOK) * a.num_kv_heads * splits;
+      }
+    }
+    long long incl = cnt;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const long long v = __shfl_up_sync(FULL_MASK, incl, off);
+      if (lane >= off) incl += v;
+    }
+    const long long total = __shfl_sync(FULL_MASK, incl, 31);
+    if (running + total > y) {
+      const bool hit = running + incl - cnt <= y && y < running + incl;
+      const int src = __ffs(__ballot_sync(FULL_MASK, hit)) - 1;
+      g_out = base + src;
+      rem_out = y - running - __shfl_sync(FULL_MASK, incl - cnt, src);
+      return;
+    }
+    running += total;
+  }
+  g_out = -1;
+  rem_out = 0;
+}
 
 // Two 16-bit terms of a pair of weights: hi = round(p), lo = round(p - hi).
 template <bool kBf16>
@@ -217,12 +276,16 @@ __global__ void __launch_bounds__(PrefillTcTraits<D, BS, G>::kThreads, 1)
     tc::alloc(tmem_slot, Tr::kTmemCols);
     tc::relinquish();
   }
+  // a grid launched after this one to overlap it (the decode after the shared-prefix pass)
+  // may start: it reads nothing this grid writes before it waits for this grid to finish
+  if (tid == 0) allow_next_grid();
 
   // ---- the longest-first schedule (scratch in the key ring) ----
   int *bins = reinterpret_cast<int *>(smem + Tr::kKOff);
   int *list = bins + Tr::kMaxBins;
   const int nbins = (max_len + 15) / 16 + 1;
-  bool sorted = nbins <= Tr::kMaxBins && a.num_seqs < (1 << 19);
+  const bool prefix_pass = a.pre_o != nullptr;
+  bool sorted = !prefix_pass && nbins <= Tr::kMaxBins && a.num_seqs < (1 << 19);
   if (sorted)
     for (int i = tid; i < nbins; i += Tr::kThreads) bins[i] = 0;
   __syncthreads();
@@ -313,6 +376,36 @@ __global__ void __launch_bounds__(PrefillTcTraits<D, BS, G>::kThreads, 1)
 
   // The tile of round `round` (whole warp calls it); false when this CTA has no more tiles.
   auto next_tile = [&](long long round, TcTile &t) -> bool {
+    t.j0 = 0;
+    t.slot = 0;
+    t.noncausal = false;
+    if (prefix_pass) {
+      int g;
+      long long rem;
+      locate_prefix_item<Tr::kTokens, Tr::kKv>(a, max_len, blockIdx.x + round * gridDim.x, g, rem);
+      if (g < 0) return false;
+      int first, members, P;
+      prefix_group(a, g, max_len, first, members, P);
+      const int kv_tiles = (P + Tr::kKv - 1) / Tr::kKv;
+      const int splits = (kv_tiles + a.pre_kv - 1) / a.pre_kv;
+      const int row_tiles = (members + Tr::kTokens - 1) / Tr::kTokens;
+      t.slot = (int)(rem % splits);
+      rem /= splits;
+      t.tau = (int)(rem % row_tiles);
+      t.kvh = (int)(rem / row_tiles);
+      t.s = first;  // the prefix is read through the first member's block table
+      t.q0 = first;
+      t.q_len = members;
+      t.L = P;
+      t.valid = t.slot < a.pre_splits;
+      t.tok0 = t.tau * Tr::kTokens;
+      t.ntok = min(Tr::kTokens, members - t.tok0);
+      t.pos0 = 0;
+      t.j0 = t.slot * a.pre_kv;
+      t.n_kv = t.valid ? min(a.pre_kv, kv_tiles - t.j0) : 0;
+      t.noncausal = true;
+      return true;
+    }
     if (sorted) {
       if (round >= my_rounds) return false;
       const int2 e = mine[round];
@@ -367,8 +460,27 @@ __global__ void __launch_bounds__(PrefillTcTraits<D, BS, G>::kThreads, 1)
     TcTile t;
     for (long long round = 0; ok && next_tile(round, t); ++round) {
       if (!t.valid) {
-        if (lane == 0 && t.tau == 0 && t.kvh == 0) set_error(a.err, PA_DEVERR_CONTEXT_LEN);
+        if (lane == 0 && t.tau == 0 && t.kvh == 0)
+          set_error(a.err, t.noncausal ? PA_DEVERR_PREFIX : PA_DEVERR_CONTEXT_LEN);
         continue;
+      }
+      if (t.noncausal && which == 1 && t.kvh == 0) {
+        // shared-prefix pass: the members of this tile must name the first member's prefix
+        // length and, over this item's positions, its physical blocks (kv head 0's items check)
+        const int32_t *row0 = a.block_tables + (long long)t.s * a.bt_s;
+        const int b0 = t.j0 * Tr::kKv / BS;
+        const int b1 = (min((t.j0 + t.n_kv) * Tr::kKv, t.L) + BS - 1) / BS;
+        bool bad = false;
+        for (int m = t.tok0 + lane; m < t.tok0 + t.ntok; m += 32) {
+          const int sq = t.q0 + m;
+          if (sq == t.s) continue;
+          if (__ldg(a.prefix_lens + sq) != __ldg(a.prefix_lens + t.s)) bad = true;
+          const int32_t *row = a.block_tables + (long long)sq * a.bt_s;
+          for (int b = b0; b < b1; ++b)
+            if (__ldg(row + b) != __ldg(row0 + b)) bad = true;
+        }
+        if (bad) set_error(a.err, PA_DEVERR_PREFIX);
+        if (lane == 0 && t.L % BS != 0) set_error(a.err, PA_DEVERR_PREFIX);
       }
       if (which == 0) {
         // the tile's query rows: tokens q0 + tok0 .. + 128/G of heads kvh*G .. + G (rows past
@@ -392,7 +504,7 @@ __global__ void __launch_bounds__(PrefillTcTraits<D, BS, G>::kThreads, 1)
       // ids of tile j + 1 are fetched before the waits of tile j, so their latency is hidden.
       const int32_t *row = a.block_tables + (long long)t.s * a.bt_s;
       auto fetch_ids = [&](int j) {
-        const int p0 = j * Tr::kKv;
+        const int p0 = (t.j0 + j) * Tr::kKv;
         const int nblk = (min(p0 + Tr::kKv, t.L) - p0 + BS - 1) / BS;
         int blk = 0;
         if (lane < nblk) {
@@ -410,7 +522,7 @@ __global__ void __launch_bounds__(PrefillTcTraits<D, BS, G>::kThreads, 1)
         const long long it = kv_base + j;
         const int b = (int)(it % Tr::kStages);
         const long long use = it / Tr::kStages;
-        const int p0 = j * Tr::kKv;
+        const int p0 = (t.j0 + j) * Tr::kKv;
         const int pend = min(p0 + Tr::kKv, t.L);
         const int nblk = (pend - p0 + BS - 1) / BS;
         const uint32_t bytes = (uint32_t)(a.grouped_maps ? nblk * (BS / 8) : (pend - p0 + 7) / 8) * Tr::kBoxBytes;
@@ -557,7 +669,7 @@ __global__ void __launch_bounds__(PrefillTcTraits<D, BS, G>::kThreads, 1)
     for (long long round = 0; ok && next_tile(round, t); ++round) {
       if (!t.valid) continue;
       const bool row_ok = lt < t.ntok;
-      const int prow = row_ok ? t.pos0 + lt : -1;
+      const int prow = row_ok ? (t.noncausal ? t.L - 1 : t.pos0 + lt) : -1;
       float m_ref = -INFINITY, l_part = 0.f;
       for (int j = 0; j < t.n_kv; ++j) {
         const long long it = kv_base + j;
@@ -570,7 +682,8 @@ __global__ void __launch_bounds__(PrefillTcTraits<D, BS, G>::kThreads, 1)
         // this thread's S columns and, later, its P: the hi terms of its kCols positions in the
         // first kCols / 2 of its columns, the lo terms in the rest
         const uint32_t my_cols = lane_base + Tr::kKv * b + Tr::kCols * half;
-        const int c_lim = prow - j * Tr::kKv - Tr::kCols * half;  // this thread's visible columns
+        const int jj = t.j0 + j;  // the kv tile's index in the context
+        const int c_lim = prow - jj * Tr::kKv - Tr::kCols * half;  // this thread's visible columns
         // t = logit * scale_log2 + nm on the visible columns (-inf elsewhere); returns the
         // largest t; with exps leaves 2^t as two 16-bit terms in hw / lw, their sum in l_t
         uint32_t hw[Tr::kCols / 2], lw[Tr::kCols / 2];
@@ -664,7 +777,7 @@ __global__ void __launch_bounds__(PrefillTcTraits<D, BS, G>::kThreads, 1)
             tc::st32x32(lane_base + Tr::kOCol + 32 * c, o);
           }
         }
-        if (half == 0 && j == t.n_kv - 1 && (j + 1) * Tr::kKv > t.L) {
+        if (half == 0 && j == t.n_kv - 1 && (jj + 1) * Tr::kKv > t.L) {
           // positions past the context may hold anything (NaN included) and would meet a zero
           // weight in the MMA: zero the value rows there once their copy has landed
           const int vs = (int)(it % Tr::kStages);
@@ -672,7 +785,7 @@ __global__ void __launch_bounds__(PrefillTcTraits<D, BS, G>::kThreads, 1)
             ok = false;
             break;
           }
-          if (r < Tr::kKv && r >= t.L - j * Tr::kKv) {
+          if (r < Tr::kKv && r >= t.L - jj * Tr::kKv) {
             const uint32_t vrow = v_s + vs * Tr::kKvBytes + (r >> 3) * Tr::kGroup + (r & 7) * 128;
 #pragma unroll
             for (int h = 0; h < Tr::kSpans; ++h)
@@ -702,6 +815,30 @@ __global__ void __launch_bounds__(PrefillTcTraits<D, BS, G>::kThreads, 1)
       }
       tc::fence_after();
       const float inv = row_ok ? 1.f / l_row : 0.f;
+      if (prefix_pass) {
+        // this item's partial result of (member sequence, query head): O / l and (m, l); the
+        // tensor-memory loads are warp-wide, only the stores depend on the row
+        const long long slot = ((long long)(t.q0 + t.tok0 + (row_ok ? lt : 0)) * (Hkv * G) +
+                                t.kvh * G + hh) * a.pre_splits + t.slot;
+        float *dst = a.pre_o + slot * D;
+#pragma unroll
+        for (int c2 = 0; c2 < D / 64; ++c2) {
+          const int c = (D / 64) * half + c2;
+          uint32_t o[32];
+          __syncwarp();
+          tc::ld32x32(lane_base + Tr::kOCol + 32 * c, o);
+          if (row_ok) {
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+              reinterpret_cast<float4 *>(dst + 32 * c)[i] =
+                  make_float4(__uint_as_float(o[4 * i]) * inv, __uint_as_float(o[4 * i + 1]) * inv,
+                              __uint_as_float(o[4 * i + 2]) * inv, __uint_as_float(o[4 * i + 3]) * inv);
+          }
+        }
+        if (row_ok && half == 0) *reinterpret_cast<float2 *>(a.pre_ml + slot * 2) = make_float2(m_ref, l_row);
+        kv_base += t.n_kv;
+        continue;
+      }
       const long long ob = (long long)(t.q0 + t.tok0 + (row_ok ? lt : 0)) * a.out_t +
                            (long long)(t.kvh * G + hh) * a.out_h;
 #pragma unroll

@@ -427,6 +427,17 @@ def shared_prefix(num_groups: int = 32, group_size: int = 4, prefix_len: int = 1
                             "group_size": group_size, "fill": fill})
 
 
+def shared_groups(b: PagedBatch):
+    """The batch's prefix sharing for pa_decode_shared_prefix: (group_start [num_groups + 1],
+    prefix_lens [num_seqs]) int32.  The shared-prefix batch is one group whose members share
+    its whole-block system prompt; any other batch is one group per sequence sharing nothing."""
+    S = b.num_seqs
+    if "prefix_len" in b.meta:
+        return (np.array([0, S], dtype=np.int32),
+                np.full(S, int(b.meta["prefix_len"]), dtype=np.int32))
+    return np.arange(S + 1, dtype=np.int32), np.zeros(S, dtype=np.int32)
+
+
 def workload(name: str, **kw) -> PagedBatch:
     """Build a workload by name: tiny_fp32, llama3_8b_decode, short_chat_bs{8,16,32},
     shared_prefix, long_mixed."""

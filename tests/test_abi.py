@@ -292,3 +292,39 @@ def test_fp8_entry_points_reject_bad_arguments(lib):
     assert dec(flags=pa.PA_DECODE_CUDA_CORES) == -4    # FP8 is read by the tensor-core kernel only
     assert dec(kc=_t([32, 2, 16, 64], pa.PA_FP8_E4M3), D=64) == -4  # head_dim 64 is not built
     assert pa.pa_last_error()
+
+
+def _shared_call(lib, a, gs, pl, bs=16, hkv=2):
+    r = ctypes.byref
+    return lib.pa_decode_shared_prefix(r(a["out"]), r(a["query"]), r(a["kc"]), r(a["vc"]),
+                                       r(a["bt"]), r(a["cl"]), r(gs) if gs is not None else None,
+                                       r(pl), 0.1, bs, hkv, None, 0, None)
+
+
+def test_shared_prefix_rejects_bad_arguments_before_cuda(lib):
+    a = _decode_args()  # 4 sequences
+    gs, pl = _t([2], pa.PA_I32), _t([4], pa.PA_I32)
+    assert _shared_call(lib, a, None, pl) == -1                           # no group_start
+    assert _shared_call(lib, a, _t([2], pa.PA_I64), pl) == -3             # group_start not int32
+    assert _shared_call(lib, a, gs, _t([3], pa.PA_I32)) == -2             # not one per sequence
+    assert _shared_call(lib, a, _t([0], pa.PA_I32), pl) == -2             # no entries at all
+    assert _shared_call(lib, a, gs, _t([4], pa.PA_I32, stride=[2])) == -7  # not contiguous
+    assert _shared_call(lib, _decode_args(dt=pa.PA_F32), gs, pl) == -4    # fp32 caches
+    assert _shared_call(lib, a, gs, pl, bs=8) == -2                       # block_size disagrees
+    assert pa.pa_last_error()
+
+
+def test_shared_prefix_workspace_bytes(lib):
+    # the decode workspace at the largest default worker count, then (m, l) and O / l of every
+    # (sequence, query head) and 256-position prefix item, each region rounded up to 256 bytes
+    def up(x):
+        return (x + 255) // 256 * 256
+
+    S, Hq, Hkv, D, MB, bs = 8, 32, 8, 128, 40, 16
+    base = pa.pa_decode_workspace_bytes(S, Hq, Hkv, D, 0)
+    if base == 0:  # no device: the default worker count is unknown, nothing to check
+        assert pa.pa_decode_shared_prefix_workspace_bytes(S, Hq, Hkv, D, MB, bs) == 0
+        return
+    splits = (MB * bs + 255) // 256
+    expect = up(base) + up(S * Hq * splits * 2 * 4) + up(S * Hq * splits * D * 4)
+    assert pa.pa_decode_shared_prefix_workspace_bytes(S, Hq, Hkv, D, MB, bs) == expect

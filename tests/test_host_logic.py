@@ -104,3 +104,4 @@ def test_default_run_measures_every_config():
               "chunked_prefill"):
         assert n in names
     assert ("llama3_8b_decode", "fp8") in bench.CONFIG_RUNS
+    assert ("shared_prefix", "shared") in bench.CONFIG_RUNS
