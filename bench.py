@@ -772,10 +772,25 @@ def run_decode(args, b: W.PagedBatch, config: dict, rank: int = 0, world: int = 
             pa.pa_decode_ex(o, qq, kc, vc, tt, ll, b.scale, b.block_size, b.num_kv_heads,
                             flags=args.decode_flags, workspace=ws)
 
+    # The whole step through pa_decode_step when the default flags apply (one kernel when each
+    # sequence brings one new token: the write and the decode fused), else the write and the
+    # decode as two calls.
+    whole_step = (args.decode_flags == pa.PA_DECODE_OVERLAP_PREVIOUS and not shared
+                  and b.dtype != "f32")
+    fused = whole_step and len(b.slot_mapping) == b.num_seqs
+
     def step(i, ev=None):
         kc, vc = pools[i % rot]
         if mapping is not None:
             pa.pa_copy_blocks(kc, vc, mapping)
+        if whole_step:
+            if ev is not None:
+                ev[0].record(stream)
+            pa.pa_decode_step(key, value, kc, vc, slots, out, q, tables, lens, b.scale,
+                              b.block_size, b.num_kv_heads, workspace=ws)
+            if ev is not None:
+                ev[1].record(stream)
+            return
         pa.pa_reshape_and_cache(key, value, kc, vc, slots)
         if ev is not None:
             ev[0].record(stream)
@@ -783,8 +798,8 @@ def run_decode(args, b: W.PagedBatch, config: dict, rank: int = 0, world: int = 
         if ev is not None:
             ev[1].record(stream)
 
-    launches_per_step = (2 + (1 if mapping is not None else 0) + (1 if args.decode_flags & 1 else 0)
-                         + (1 if shared else 0))
+    launches_per_step = ((1 if fused else 2) + (1 if mapping is not None else 0)
+                         + (1 if args.decode_flags & 1 else 0) + (1 if shared else 0))
     gpu_uuid = None
     try:
         gpu_uuid = str(torch.cuda.get_device_properties(dev).uuid)
@@ -879,6 +894,10 @@ def run_decode(args, b: W.PagedBatch, config: dict, rank: int = 0, world: int = 
     peak, peak_src = hbm_peak()
     kernel = ("paged_decode_kernel (CUDA cores)" if (args.decode_flags & 2 or b.dtype == "f32")
               else "paged_decode_mma_kernel (mma.sync + TMA)")
+    if fused:
+        kernel = ("paged_decode_mma_kernel (mma.sync + TMA), fused step: the cache write inside "
+                  "the same kernel")
+    roof_bytes = dec_unique + (write_bytes(b) if fused else 0)
     if shared:
         kernel = ("paged_prefill_tc_kernel shared-prefix pass (tcgen05) + paged_decode_mma_kernel "
                   "(mma.sync + TMA); launch times cover both")
@@ -891,7 +910,7 @@ def run_decode(args, b: W.PagedBatch, config: dict, rank: int = 0, world: int = 
         "seq_steps_per_s": round(world * b.num_seqs / (ms * 1e-3), 1),
         "pct_of_8TBs": round(100 * value / world / NOMINAL_HBM_GBS, 2),
         f"pct_of_{peak_src}_hbm": round(100 * value / world / peak, 2),
-        "roofline": hbm_roofline(dec_unique, decode_ms, kernel,
+        "roofline": hbm_roofline(roof_bytes, decode_ms, kernel,
                                  recorded_traffic(config["workload"]), probe),
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks,
@@ -934,6 +953,8 @@ def run_decode(args, b: W.PagedBatch, config: dict, rank: int = 0, world: int = 
         line["timeline"] = timeline
     if shared:
         line["decode_call"] = "pa_decode_shared_prefix"
+    elif whole_step:
+        line["decode_call"] = "pa_decode_step" + (" (fused: one kernel)" if fused else "")
     if full and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(b, args.cpu_seconds)
     return line

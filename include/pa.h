@@ -134,8 +134,8 @@ typedef enum pa_status {
 #define PA_DECODE_OVERLAP_PREVIOUS 0x4u /* let the decode kernel start while the kernel launched
                                           just before it on `stream` is still running
                                           (programmatic dependent launch): it reads context_lens
-                                          and block_tables and zeroes the out rows of empty
-                                          contexts before it waits for that kernel, and reads
+                                          and block_tables, and may zero the out rows of empty
+                                          contexts, before it waits for that kernel; it reads
                                           the caches and the query only after.  Use it only when
                                           that kernel writes none of context_lens, block_tables
                                           and out, e.g. right after pa_reshape_and_cache */
@@ -158,16 +158,26 @@ PA_API int pa_reshape_and_cache(const pa_tensor *key, const pa_tensor *value,
  * pa_decode_step - one whole decode step: pa_reshape_and_cache(key, value, key_cache,
  * value_cache, slot_mapping) followed by pa_decode_ex(out, query, key_cache, value_cache,
  * block_tables, context_lens, ..., num_workers = 0, PA_DECODE_OVERLAP_PREVIOUS, workspace),
- * i.e. the write side of [P2] 4.1 and the attention of [P4] 2.2.2 for the same step.  The
- * decode is launched as a programmatic dependent of the write: its prologue (context_lens,
- * block_tables, the split of the work) runs while the write finishes, and it reads the caches
- * only after.  Both halves are validated before either is launched, so a refused call launches
- * nothing.  workspace: as for pa_decode_ex, or NULL for the library-owned one of pa_decode.
+ * i.e. the write side of [P2] 4.1 and the attention of [P4] 2.2.2 for the same step.
+ * One new token per sequence (key->shape[0] == number of sequences) in bf16 or f16 caches:
+ * the step is ONE kernel.  Token s is sequence s's position context_lens[s] - 1; the kernel
+ * stores it into slot slot_mapping[s] and, for that position, attends to the rows of key and
+ * value themselves, so no part of the decode waits for the store.  A slot that is not that
+ * position under block_tables (or a token of an empty context) is still stored as asked and
+ * sets PA_DEVERR_SLOT; out rows of empty contexts are zeroed.  Any other shape (several
+ * tokens per sequence, fp32 caches): two kernels, the write and then the decode, launched as
+ * a programmatic dependent of the write: its prologue (context_lens, block_tables, the split
+ * of the work) runs while the write finishes, and it reads the caches only after.  Both
+ * halves are validated before either is launched, so a refused call launches nothing.
+ * In both forms the decode waits for the kernel launched before it on `stream` before it
+ * reads the caches or the query (programmatic dependent launch, as under
+ * PA_DECODE_OVERLAP_PREVIOUS, with the same rule for what that kernel may write).
+ * workspace: as for pa_decode_ex, or NULL for the library-owned one of pa_decode.
  * With a caller workspace initialised beforehand (pa_workspace_init) the call allocates
  * nothing and can be captured into a CUDA graph (one graph node per kernel, the programmatic
  * dependency kept as a graph edge); the graph is valid as long as the tensors it was captured
  * with stay where they are.  Errors as for the two calls; on PA_ERR_CUDA from the decode launch
- * the cache write may already have been launched.
+ * of the two-kernel form the cache write may already have been launched.
  */
 PA_API int pa_decode_step(const pa_tensor *key, const pa_tensor *value,
                           const pa_tensor *key_cache, const pa_tensor *value_cache,

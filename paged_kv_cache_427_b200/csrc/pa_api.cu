@@ -533,7 +533,7 @@ int decode_impl(const pa_tensor *out, const pa_tensor *query, const pa_tensor *k
                 size_t workspace_bytes, bool library_workspace, void *stream,
                 CallMode mode = CallMode::kLaunch, const pa_tensor *k_scale = nullptr,
                 const pa_tensor *v_scale = nullptr, const pa_tensor *group_start = nullptr,
-                const pa_tensor *prefix_lens = nullptr) {
+                const pa_tensor *prefix_lens = nullptr, const pa::CacheWriteArgs *step = nullptr) {
   int rc;
   CacheShape cs;
   const bool fp8 = k_scale != nullptr;
@@ -735,6 +735,10 @@ int decode_impl(const pa_tensor *out, const pa_tensor *query, const pa_tensor *k
     a.timeline_warps = g_timeline_warps;
   }
   bool overlap = (flags & PA_DECODE_OVERLAP_PREVIOUS) != 0;
+  if (step) {
+    a.fused = 1;
+    a.step = *step;
+  }
   if (shared) {
     a.prefix_lens = static_cast<const int32_t *>(prefix_lens->data);
     a.pre_ml = reinterpret_cast<float *>(ws + PL.pre_ml);
@@ -792,7 +796,7 @@ namespace {
 
 int write_impl(const pa_tensor *key, const pa_tensor *value, const pa_tensor *key_cache,
                const pa_tensor *value_cache, const pa_tensor *slot_mapping, void *stream,
-               CallMode mode) {
+               CallMode mode, pa::CacheWriteArgs *prepared = nullptr) {
   int rc;
   CacheShape cs;
   if ((rc = check_caches(key_cache, value_cache, &cs))) return rc;
@@ -841,6 +845,7 @@ int write_impl(const pa_tensor *key, const pa_tensor *value, const pa_tensor *ke
   a.num_slots = cs.num_blocks * cs.block_size;
   a.err = ds->err;
   if (a.row_bytes % 16 != 0) return fail(PA_ERR_UNSUPPORTED, "head_dim * element size must be a multiple of 16 bytes");
+  if (prepared) *prepared = a;
   if (mode == CallMode::kAllChecks) return PA_OK;
   cudaError_t err = pa::launch_reshape_and_cache(a, ds->num_sms, static_cast<cudaStream_t>(stream));
   return err == cudaSuccess ? PA_OK : cuda_fail(err, "reshape_and_cache launch");
@@ -1131,6 +1136,27 @@ int pa_decode_step(const pa_tensor *key, const pa_tensor *value, const pa_tensor
                    int32_t num_kv_heads, void *workspace, size_t workspace_bytes, void *stream) {
   const bool lib_ws = workspace == nullptr;
   int rc;
+  // One new token per sequence in 16-bit caches: one kernel for the whole step, which writes
+  // the caches and decodes with token s as sequence s's position L-1 (read from key / value,
+  // so the decode never waits for the write).  Otherwise: the write kernel, then the decode.
+  const bool fused = key && query && context_lens && key_cache && key->ndim == 3 &&
+                     context_lens->ndim == 1 && key->shape[0] == context_lens->shape[0] &&
+                     (key_cache->dtype == PA_BF16 || key_cache->dtype == PA_F16);
+  if (fused) {
+    pa::CacheWriteArgs w;
+    for (CallMode m : {CallMode::kHostChecks, CallMode::kAllChecks})
+      if ((rc = write_impl(key, value, key_cache, value_cache, slot_mapping, stream, m, &w)) ||
+          (rc = decode_impl(out, query, key_cache, value_cache, block_tables, context_lens, scale,
+                            block_size, num_kv_heads, 0, PA_DECODE_OVERLAP_PREVIOUS, workspace,
+                            workspace_bytes, lib_ws, stream, m)))
+        return rc;
+    if (key->shape[0] > 0)
+      return decode_impl(out, query, key_cache, value_cache, block_tables, context_lens, scale,
+                         block_size, num_kv_heads, 0, PA_DECODE_OVERLAP_PREVIOUS, workspace,
+                         workspace_bytes, lib_ws, stream, CallMode::kLaunch, nullptr, nullptr,
+                         nullptr, nullptr, &w);
+    return PA_OK;
+  }
   // both halves are checked (host-side checks of both first) before either is launched
   for (CallMode m : {CallMode::kHostChecks, CallMode::kAllChecks})
     if ((rc = write_impl(key, value, key_cache, value_cache, slot_mapping, stream, m)) ||

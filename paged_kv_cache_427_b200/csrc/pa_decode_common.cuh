@@ -23,6 +23,10 @@
 #include "pa_device.cuh"
 #include "pa_internal.h"
 
+#ifndef PA_MERGE_PREFETCH
+#define PA_MERGE_PREFETCH 0  // 1: a merge loads its first pieces' outputs with their (m, l)
+#endif
+
 namespace pa {
 
 // Per-stage description written by the issuing lane before the stage's barrier arrives.
@@ -33,6 +37,7 @@ struct ChunkMeta {
 constexpr int kFirst = 1;      // first chunk of this warp's piece of a (sequence, kv head)
 constexpr int kLast = 2;       // last chunk of the piece
 constexpr int kPairStart = 4;  // chunk 0 of the (sequence, kv head)
+constexpr int kNewRow = 8;     // fused step: the chunk holds position L-1, the step's new token
 
 __device__ __forceinline__ int clamp_len(int len, int max_len) {
   return len < 0 ? 0 : (len > max_len ? max_len : len);
@@ -41,6 +46,44 @@ __device__ __forceinline__ int clamp_len(int len, int max_len) {
 // The warp whose share [floor(w*C/W), floor((w+1)*C/W)) contains chunk c.
 __device__ __forceinline__ int worker_of(long long c, long long C, int W) {
   return (int)(((c + 1) * (long long)W + C - 1) / C - 1);
+}
+
+// Fused decode step: thread `tid` of `nthreads` moves its 16-byte pieces of the step's new
+// key and value rows into their cache slots (as the cache write kernel does), and checks that
+// token s is sequence s's position L-1, which the decode reads from the new rows directly: a
+// slot that differs sets PA_DEVERR_SLOT.
+template <int BS>
+__device__ __forceinline__ void fused_cache_write(const DecodeArgs &a, int max_len, int tid,
+                                                  int nthreads) {
+  const CacheWriteArgs &w = a.step;
+  const int vec_per_row = w.row_bytes >> 4;
+  const int64_t total = w.num_tokens * w.num_kv_heads * vec_per_row;
+  for (int64_t idx = tid; idx < total; idx += nthreads) {
+    const int v = (int)(idx % vec_per_row);
+    const int64_t th = idx / vec_per_row;
+    const int h = (int)(th % w.num_kv_heads);
+    const int64_t t = th / w.num_kv_heads;
+    const int64_t slot = __ldg(w.slots + t);
+    if (h == 0 && v == 0) {
+      const int len = clamp_len(__ldg(a.context_lens + t), max_len);
+      int64_t expect = -1;
+      if (len > 0) {
+        const int blk = __ldg(a.block_tables + t * a.bt_s + (len - 1) / BS);
+        expect = (int64_t)blk * BS + (len - 1) % BS;
+      }
+      if (slot != expect) set_error(a.err, PA_DEVERR_SLOT);
+    }
+    if (slot < 0) continue;
+    if (slot >= w.num_slots) {
+      if (h == 0 && v == 0) set_error(a.err, PA_DEVERR_SLOT);
+      continue;
+    }
+    const int64_t dst = (slot / w.block_size) * w.c_blk + h * w.c_head + (slot % w.block_size) * w.row_bytes + v * 16;
+    const uint4 kv = __ldg(reinterpret_cast<const uint4 *>(w.key + t * w.k_tok + h * w.k_head) + v);
+    const uint4 vv = __ldg(reinterpret_cast<const uint4 *>(w.value + t * w.v_tok + h * w.v_head) + v);
+    *reinterpret_cast<uint4 *>(w.key_cache + dst) = kv;
+    *reinterpret_cast<uint4 *>(w.value_cache + dst) = vv;
+  }
 }
 
 // The first position the decode reads of sequence s, whose context holds len positions: its
@@ -105,7 +148,7 @@ __device__ __forceinline__ long long warp_sum(long long x) {
 // 32 sequences at a time.  No shared memory and no block-wide barrier, so warps start as soon
 // as they are scheduled.  Warp gw also flags bad lengths (warp 0) and zeroes the rows of empty
 // contexts s with s % (warps launched) == gw.  Returns false when this warp has no work.
-template <int CH, int kWarps, int G, int D, int BS>
+template <int CH, int kWarps, int G, int D, int BS, bool kZeroEmpty = true>
 __device__ __forceinline__ bool split_prologue(const DecodeArgs &a, int max_len, WarpShare &ws) {
   const int lane = threadIdx.x & 31;
   const int gw = blockIdx.x * kWarps + (threadIdx.x >> 5);
@@ -119,7 +162,7 @@ __device__ __forceinline__ bool split_prologue(const DecodeArgs &a, int max_len,
       const int raw = __ldg(a.context_lens + s);
       const int len = clamp_len(raw, max_len);
       if (raw != len && gw == 0) set_error(a.err, PA_DEVERR_CONTEXT_LEN);
-      if (len == 0 && s % launched == gw)
+      if (kZeroEmpty && len == 0 && s % launched == gw)
         zero_rows<D>(static_cast<char *>(a.out) + (long long)s * a.out_s * (a.out_dtype == PA_F32 ? 4 : 2),
                      a.out_h, a.out_dtype, Hkv * G);
       mine += (len - decode_start<BS>(a, s, len) + CH - 1) / CH;
@@ -303,8 +346,19 @@ __device__ __forceinline__ void merge_pieces(const DecodeArgs &a, int pair, int 
     den[h] = 0.f;
     num[h] = make_float4(0.f, 0.f, 0.f, 0.f);
   }
+  // outputs: U pieces per round (U*G float4 in flight per lane), loads issued together
+  constexpr int U = G >= 8 ? 1 : 8 / G;
   for (int base = 0; base < total; base += 32) {
     const int cnt = total - base < 32 ? total - base : 32;
+#if PA_MERGE_PREFETCH
+    // the first round's outputs do not depend on the weights: load them with the (m, l)
+    float4 x0[U][G];
+#pragma unroll
+    for (int u = 0; u < U; ++u)
+#pragma unroll
+      for (int h = 0; h < G; ++h)
+        x0[u][h] = (active && u < cnt) ? __ldcg(o_of(base + u, h) + lane) : make_float4(0.f, 0.f, 0.f, 0.f);
+#endif
     // lane k < cnt: (m, l) of piece base + k for every head
     float mk[G], lk[G];
 #pragma unroll
@@ -342,16 +396,24 @@ __device__ __forceinline__ void merge_pieces(const DecodeArgs &a, int pair, int 
       den[h] += ws;
       mk[h] = w;  // reuse: the weight of piece base + lane
     }
-    // outputs: U pieces per round (U*G float4 in flight per lane), loads issued together
-    constexpr int U = G >= 8 ? 1 : 8 / G;
     for (int k = 0; k < cnt; k += U) {
       float4 x[U][G];
+#if PA_MERGE_PREFETCH
+      if (k == 0) {
 #pragma unroll
-      for (int u = 0; u < U; ++u)
+        for (int u = 0; u < U; ++u)
 #pragma unroll
-        for (int h = 0; h < G; ++h)
-          x[u][h] = (active && k + u < cnt) ? __ldcg(o_of(base + k + u, h) + lane)
-                                            : make_float4(0.f, 0.f, 0.f, 0.f);
+          for (int h = 0; h < G; ++h) x[u][h] = x0[u][h];
+      } else
+#endif
+      {
+#pragma unroll
+        for (int u = 0; u < U; ++u)
+#pragma unroll
+          for (int h = 0; h < G; ++h)
+            x[u][h] = (active && k + u < cnt) ? __ldcg(o_of(base + k + u, h) + lane)
+                                              : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
 #pragma unroll
       for (int u = 0; u < U; ++u)
 #pragma unroll
@@ -393,7 +455,7 @@ __device__ __forceinline__ void merge_pieces(const DecodeArgs &a, int pair, int 
 }
 
 #ifndef PA_TICKET_ACQREL
-#define PA_TICKET_ACQREL 0  // 1: merge tickets by one acquire-release atomic, no separate fences
+#define PA_TICKET_ACQREL 1  // 0: a fence, then a relaxed atomic, then a fence
 #endif
 
 // Take a ticket of a merge counter.  With PA_TICKET_ACQREL the atomic has acquire-release

@@ -143,7 +143,10 @@ struct MmaTraits {
   static constexpr int kBoxBytes = kBoxRows * D * KVB;  // one box: [block][row][128 B]
   static constexpr int kTileBytes = 16 * D * KVB;       // key (or value) bytes of a chunk
   static constexpr int kQBytes = G * D * 2;
-  static constexpr int kStageBytes = 2 * kTileBytes + (kQBytes + 1023) / 1024 * 1024;
+  // a fused decode step's new key and value rows of the chunk holding position L-1 (16-bit)
+  static constexpr int kNewBytes = KVB == 2 ? 2 * D * 2 : 0;
+  static constexpr int kNewOff = 2 * kTileBytes + kQBytes;
+  static constexpr int kStageBytes = 2 * kTileBytes + (kQBytes + kNewBytes + 1023) / 1024 * 1024;
   static constexpr int kWorkers = 4;                    // consumer warps
   static constexpr int kThreads = (kWorkers + 2) * 32;  // + one producer and one merge warp
   // Two stages per worker: one being computed, one in flight.  A third stage puts more bytes
@@ -260,7 +263,7 @@ __global__ void __launch_bounds__(MmaTraits<D, BS, G, (int)sizeof(KV)>::kThreads
     }
     WarpShare ws;
     ws.n = 0;
-    const bool has = split_prologue<16, NW, G, D, BS>(a, max_len, ws);
+    const bool has = split_prologue<16, NW, G, D, BS, false>(a, max_len, ws);
     if (lane == 0) {
       ShareRecord r;
       r.s = has ? ws.s : -1;
@@ -322,11 +325,14 @@ __global__ void __launch_bounds__(MmaTraits<D, BS, G, (int)sizeof(KV)>::kThreads
     // One stage of this lane's worker: the chunk's key and value boxes, plus the group's query
     // rows when a new (sequence, kv head) starts, all counted on the stage's full barrier.
     auto issue = [&](int slot) {
-      const int f = cur.flags();
+      // fused step: the chunk holding position L-1 also brings that position's new rows
+      const bool new_row = !kFp8 && a.fused && cur.i == cur.nch - 1;
+      const int f = cur.flags() | (new_row ? kNewRow : 0);
       unsigned char *stage = ring + slot * Tr::kStageBytes;
       meta[slot] = cur.meta(f);
       const uint32_t bytes = 2u * cur.valid_copies() * Tr::kBoxBytes +
                              ((f & kFirst) ? (uint32_t)Tr::kQBytes : 0u) +
+                             (new_row ? (uint32_t)(2 * D * 2) : 0u) +
                              ((cur.issued == 0 && test_stalls(a, blockIdx.x * NW + k)) ? 16u : 0u);
       mbar_arrive_expect_tx(full + slot, bytes);
 #pragma unroll
@@ -343,6 +349,14 @@ __global__ void __launch_bounds__(MmaTraits<D, BS, G, (int)sizeof(KV)>::kThreads
           tma_load_tile(smem_u32(stage + Tr::kTileBytes + off), &maps.v, t % BS, cur.kvh, blk,
                         full + slot);
         }
+      }
+      if (new_row) {
+        bulk_copy_g2s(stage + Tr::kNewOff,
+                      a.step.key + (long long)cur.s * a.step.k_tok + (long long)cur.kvh * a.step.k_head,
+                      D * 2, full + slot);
+        bulk_copy_g2s(stage + Tr::kNewOff + D * 2,
+                      a.step.value + (long long)cur.s * a.step.v_tok + (long long)cur.kvh * a.step.v_head,
+                      D * 2, full + slot);
       }
       if (f & kFirst) {
         const char *q = static_cast<const char *>(a.query) +
@@ -397,6 +411,19 @@ __global__ void __launch_bounds__(MmaTraits<D, BS, G, (int)sizeof(KV)>::kThreads
 
   if (wid == NW + 1) {
     // ================================ merge warp ================================
+    // First, once the grid before this one (when it was launched to overlap it) has finished:
+    // the out rows of empty contexts are zeroed, and in a fused decode step this grid's share
+    // of the step's cache write is done.
+    wait_for_previous_grid();
+    {
+      const int launched_lanes = gridDim.x * 32;
+      const int out_elt = a.out_dtype == PA_F32 ? 4 : 2;
+      for (int s = blockIdx.x * 32 + lane; s < a.num_seqs; s += launched_lanes)
+        if (clamp_len(__ldg(a.context_lens + s), max_len) == 0)
+          zero_rows<D>(static_cast<char *>(a.out) + (long long)s * a.out_s * out_elt, a.out_h,
+                       a.out_dtype, a.num_kv_heads * G);
+      if (a.fused) fused_cache_write<BS>(a, max_len, blockIdx.x * 32 + lane, launched_lanes);
+    }
     // Lane k follows worker k's mailbox.  For each split piece the warp makes the piece's
     // stores visible GPU-wide, takes the ticket of its (sequence, kv head) and, when the piece
     // is the last one there, merges all of them; the workers never stall on a GPU-wide fence.
@@ -492,6 +519,23 @@ __global__ void __launch_bounds__(MmaTraits<D, BS, G, (int)sizeof(KV)>::kThreads
     if (tl && cc == 0) tl[kTlFirst] = global_ns();
     const ChunkMeta m = meta[slot];
     unsigned char *stage = ring + slot * Tr::kStageBytes;
+    if constexpr (!kFp8) {
+      if (m.flags & kNewRow) {
+        // fused step: position L-1 is this step's new token, read from the step's key and
+        // value rather than the cache (which this kernel writes concurrently); put its rows into
+        // the tiles at row (L-1) % 16, in the tiles' swizzled layout
+        constexpr int kPieces = D * 2 / 16;  // 16-byte pieces of a row
+        const int r = (m.len - 1) & 15;
+        if (lane < 2 * kPieces) {
+          const int which = lane / kPieces, c = lane % kPieces;
+          const uint4 v = *reinterpret_cast<const uint4 *>(stage + Tr::kNewOff + which * D * 2 + c * 16);
+          *reinterpret_cast<uint4 *>(stage + which * Tr::kTileBytes + tile_offset<Tr>(r, c / 8) +
+                                     (((c % 8) ^ (r & 7)) << 4)) = v;
+          fence_proxy_async_smem();  // before the stage is copied into again
+        }
+        __syncwarp();
+      }
+    }
     const uint32_t kbase = smem_u32(stage);
     const uint32_t vbase = kbase + Tr::kTileBytes;
     if (m.flags & kFirst) {

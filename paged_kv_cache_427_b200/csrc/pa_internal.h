@@ -9,6 +9,22 @@
 
 namespace pa {
 
+struct CacheWriteArgs {
+  const char *key;
+  const char *value;
+  int64_t k_tok, k_head, v_tok, v_head;  // bytes
+  char *key_cache;
+  char *value_cache;
+  int64_t c_blk, c_head;  // bytes
+  int row_bytes;
+  const int64_t *slots;
+  int64_t num_tokens;
+  int num_kv_heads;
+  int block_size;
+  int64_t num_slots;
+  unsigned int *err;
+};
+
 // Everything a decode launch needs, already validated.  Strides are in elements.
 struct DecodeArgs {
   void *out;
@@ -55,6 +71,12 @@ struct DecodeArgs {
   const float *pre_ml;
   int pre_splits;
   int pre_kv_tokens;  // positions per prefix item
+  // Fused decode step (pa_decode_step with one new token per sequence), when fused != 0: the
+  // kernel also performs this cache write (its merge warps, after the previous grid), and reads
+  // position L-1 of sequence s from the new token s (step.key / step.value) instead of the
+  // cache, so that the decode never waits for the write.
+  int fused;
+  CacheWriteArgs step;
 };
 
 // Fields of one worker warp's timeline record.
@@ -97,21 +119,6 @@ bool decode_kernel_f32(int head_dim, int block_size, int group, bool tensor_core
 bool decode_kernel_bf16(int head_dim, int block_size, int group, bool tensor_cores, DecodeKernel *k);
 bool decode_kernel_f16(int head_dim, int block_size, int group, bool tensor_cores, DecodeKernel *k);
 
-struct CacheWriteArgs {
-  const char *key;
-  const char *value;
-  int64_t k_tok, k_head, v_tok, v_head;  // bytes
-  char *key_cache;
-  char *value_cache;
-  int64_t c_blk, c_head;  // bytes
-  int row_bytes;
-  const int64_t *slots;
-  int64_t num_tokens;
-  int num_kv_heads;
-  int block_size;
-  int64_t num_slots;
-  unsigned int *err;
-};
 
 // Whole-block copies from one pair of caches to another (the same pair for copy-on-write,
 // device and pinned host memory for swapping).
