@@ -23,10 +23,6 @@
 #include "pa_device.cuh"
 #include "pa_internal.h"
 
-#ifndef PA_MERGE_PREFETCH
-#define PA_MERGE_PREFETCH 0  // 1: a merge loads its first pieces' outputs with their (m, l)
-#endif
-
 namespace pa {
 
 // Per-stage description written by the issuing lane before the stage's barrier arrives.
@@ -317,10 +313,10 @@ struct ChunkCursor {
 // Merge the pieces (o, m, l) of one (sequence, kv head) and write its G output rows.  Called by
 // a whole warp; pieces live in workspace slots pair + first_worker + k, k < npieces, followed by
 // the npre partial results of the shared-prefix pass (slots of the query head, item k - npieces).
-// Loads are issued for many pieces at once (lane k fetches piece k's (m, l); then 4 pieces'
-// outputs per round) so a merge costs a few memory round trips, not two per piece.  m is in
-// base-2 units.
-template <int G, int D>
+// Loads are issued for many pieces at once (lane k fetches piece k's (m, l); the outputs of
+// several pieces per round) so a merge costs a few memory round trips, not two per piece.  m is
+// in base-2 units.
+template <int G, int D, int U = (G >= 8 ? 1 : 16 / G)>
 __device__ __forceinline__ void merge_pieces(const DecodeArgs &a, int pair, int first_worker,
                                              int npieces, int s, int kvh, int lane, int npre = 0) {
   const long long seg0 = (long long)pair + first_worker;
@@ -346,19 +342,20 @@ __device__ __forceinline__ void merge_pieces(const DecodeArgs &a, int pair, int 
     den[h] = 0.f;
     num[h] = make_float4(0.f, 0.f, 0.f, 0.f);
   }
-  // outputs: U pieces per round (U*G float4 in flight per lane), loads issued together
-  constexpr int U = G >= 8 ? 1 : 8 / G;
-  for (int base = 0; base < total; base += 32) {
-    const int cnt = total - base < 32 ? total - base : 32;
-#if PA_MERGE_PREFETCH
-    // the first round's outputs do not depend on the weights: load them with the (m, l)
-    float4 x0[U][G];
+  // Outputs: U pieces per round (U*G float4 in flight per lane), loads issued together.  The
+  // first round of each group of 32 pieces is issued with the group's (m, l), since the outputs
+  // do not depend on the weights: a merge of up to U pieces costs one memory round trip.
+  float4 x[U][G];
+  auto load_round = [&](int first, int cnt) {
 #pragma unroll
     for (int u = 0; u < U; ++u)
 #pragma unroll
       for (int h = 0; h < G; ++h)
-        x0[u][h] = (active && u < cnt) ? __ldcg(o_of(base + u, h) + lane) : make_float4(0.f, 0.f, 0.f, 0.f);
-#endif
+        x[u][h] = (active && u < cnt) ? __ldcg(o_of(first + u, h) + lane) : make_float4(0.f, 0.f, 0.f, 0.f);
+  };
+  for (int base = 0; base < total; base += 32) {
+    const int cnt = total - base < 32 ? total - base : 32;
+    load_round(base, cnt);
     // lane k < cnt: (m, l) of piece base + k for every head
     float mk[G], lk[G];
 #pragma unroll
@@ -397,23 +394,7 @@ __device__ __forceinline__ void merge_pieces(const DecodeArgs &a, int pair, int 
       mk[h] = w;  // reuse: the weight of piece base + lane
     }
     for (int k = 0; k < cnt; k += U) {
-      float4 x[U][G];
-#if PA_MERGE_PREFETCH
-      if (k == 0) {
-#pragma unroll
-        for (int u = 0; u < U; ++u)
-#pragma unroll
-          for (int h = 0; h < G; ++h) x[u][h] = x0[u][h];
-      } else
-#endif
-      {
-#pragma unroll
-        for (int u = 0; u < U; ++u)
-#pragma unroll
-          for (int h = 0; h < G; ++h)
-            x[u][h] = (active && k + u < cnt) ? __ldcg(o_of(base + k + u, h) + lane)
-                                              : make_float4(0.f, 0.f, 0.f, 0.f);
-      }
+      if (k > 0) load_round(base + k, cnt - k);
 #pragma unroll
       for (int u = 0; u < U; ++u)
 #pragma unroll
@@ -484,33 +465,36 @@ template <int G, int D, int BS>
 __device__ __forceinline__ void take_ticket(const DecodeArgs &a, const PieceInfo &p, int lane) {
   unsigned int ticket = 0;
   __syncwarp();
-  if (lane == 0) ticket = ticket_add(a.counters + p.pair);
+  // a single piece has only shared-prefix partial results to merge with: no ticket
+  if (p.npieces > 1 && lane == 0) ticket = ticket_add(a.counters + p.pair);
   ticket = __shfl_sync(FULL_MASK, ticket, 0);
   if (ticket == (unsigned int)(p.npieces - 1)) {
     if (!PA_TICKET_ACQREL) __threadfence();
     __syncwarp();
     merge_pieces<G, D>(a, p.pair, p.first_worker, p.npieces, p.s, p.kvh, lane,
                        prefix_pieces<BS>(a, p.s, a.max_blocks * BS));
-    if (lane == 0) a.counters[p.pair] = 0u;
+    if (lane == 0 && p.npieces > 1) a.counters[p.pair] = 0u;
   }
 }
 
 // After a piece's (o, m, l) are stored: publish them, take a ticket, and merge when this is the
-// last piece of its (sequence, kv head).  Called by a whole warp.
-template <int G, int D, int BS>
+// last piece of its (sequence, kv head), U pieces per round.  Called by a whole warp.  A single
+// piece (merged with shared-prefix partial results only) takes no ticket.
+template <int G, int D, int BS, int U = (G >= 8 ? 1 : 16 / G)>
 __device__ __forceinline__ void finish_piece(const DecodeArgs &a, const ChunkMeta &m, int lane) {
   if (a.separate_reduce) return;
+  const unsigned int others = (unsigned int)(m.npieces - 1);
   if (!PA_TICKET_ACQREL) __threadfence();
   __syncwarp();
-  unsigned int ticket = 0;
-  if (lane == 0) ticket = ticket_add(a.counters + m.pair);
+  unsigned int ticket = others;
+  if (others > 0 && lane == 0) ticket = ticket_add(a.counters + m.pair);
   ticket = __shfl_sync(FULL_MASK, ticket, 0);
-  if (ticket == (unsigned int)(m.npieces - 1)) {
+  if (ticket == others) {
     if (!PA_TICKET_ACQREL) __threadfence();
     __syncwarp();
-    merge_pieces<G, D>(a, m.pair, m.first_worker, m.npieces, m.s, m.kvh, lane,
-                       prefix_pieces<BS>(a, m.s, a.max_blocks * BS));
-    if (lane == 0) a.counters[m.pair] = 0u;
+    merge_pieces<G, D, U>(a, m.pair, m.first_worker, m.npieces, m.s, m.kvh, lane,
+                          prefix_pieces<BS>(a, m.s, a.max_blocks * BS));
+    if (lane == 0 && others > 0) a.counters[m.pair] = 0u;
   }
 }
 

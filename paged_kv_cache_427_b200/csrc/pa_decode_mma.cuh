@@ -469,6 +469,7 @@ __global__ void __launch_bounds__(MmaTraits<D, BS, G, (int)sizeof(KV)>::kThreads
   int posted = 0;
   PieceInfo done_msg;
   done_msg.pair = done_msg.first_worker = done_msg.npieces = done_msg.s = done_msg.kvh = 0;
+  ChunkMeta last_piece = {};  // the share's last piece when it is split (npieces > 0)
   const int gw = blockIdx.x * NW + wid;
   // measurement aid: this warp's timeline record, or null
   unsigned long long *tl = (a.timeline != nullptr && lane == 0 && gw < a.timeline_warps)
@@ -804,6 +805,7 @@ __global__ void __launch_bounds__(MmaTraits<D, BS, G, (int)sizeof(KV)>::kThreads
       } else {
         const long long seg = (long long)m.pair + gw;
         float *o0 = a.part_o + (seg * G + h0) * D;
+        float2 *ml0 = reinterpret_cast<float2 *>(a.part_ml) + seg * G + h0;
         float *o1 = o0 + D;
 #pragma unroll
         for (int mt = 0; mt < Tr::kMTiles; ++mt) {
@@ -818,8 +820,8 @@ __global__ void __launch_bounds__(MmaTraits<D, BS, G, (int)sizeof(KV)>::kThreads
           }
         }
         if (g == 0) {
-          if (h0 < G) *reinterpret_cast<float2 *>(a.part_ml + (seg * G + h0) * 2) = make_float2(m0, t0);
-          if (h1 < G) *reinterpret_cast<float2 *>(a.part_ml + (seg * G + h1) * 2) = make_float2(m1, t1);
+          if (h0 < G) ml0[0] = make_float2(m0, t0);
+          if (h1 < G) ml0[1] = make_float2(m1, t1);
         }
         if (!a.separate_reduce) {
           PieceInfo p;
@@ -828,20 +830,25 @@ __global__ void __launch_bounds__(MmaTraits<D, BS, G, (int)sizeof(KV)>::kThreads
           p.npieces = m.npieces;
           p.s = m.s;
           p.kvh = m.kvh;
-          if (cc < n - 1 && posted < Tr::kMboxEntries - 1) {
+          if (cc == n - 1) {
+            // the share's last piece: published after the loop (nothing is left to overlap it
+            // with), by this warp, so the four workers publish their last pieces in parallel
+            // rather than through one merge warp
+            last_piece = m;
+          } else if (posted < Tr::kMboxEntries - 1) {
             // a piece that ends inside the share: the merge warp publishes it while this warp
             // goes on with its next piece
             mail_post(box, mcount + wid, posted, p, lane);
             ++posted;
           } else {
-            // the share's last piece: nothing is left to overlap the fence with, and the four
-            // workers publish their last pieces in parallel rather than through one merge warp
-            finish_piece<G, D, BS>(a, m, lane);
+            finish_piece<G, D, BS, 1>(a, m, lane);  // mailbox full (rare): small merge rounds
           }
         }
       }
     }
   }
+  // the loop's registers are free here: the merge takes its large rounds
+  if (last_piece.npieces > 0) finish_piece<G, D, BS>(a, last_piece, lane);
   mail_post(box, mcount + wid, posted, done_msg, lane);
   if (tl) tl[kTlDone] = global_ns();
 }
