@@ -112,27 +112,46 @@ def load(path: str = LIBRARY) -> ctypes.CDLL:
     return lib
 
 
-def _torch_dtype_code(t) -> int:
-    import torch
+_DTYPE_CODES: dict = {}
 
-    codes = {torch.float32: PA_F32, torch.bfloat16: PA_BF16, torch.float16: PA_F16,
-             torch.int32: PA_I32, torch.int64: PA_I64, torch.float8_e4m3fn: PA_FP8_E4M3}
-    if t.dtype not in codes:
+
+def _torch_dtype_code(t) -> int:
+    if not _DTYPE_CODES:
+        import torch
+
+        _DTYPE_CODES.update({torch.float32: PA_F32, torch.bfloat16: PA_BF16,
+                             torch.float16: PA_F16, torch.int32: PA_I32, torch.int64: PA_I64,
+                             torch.float8_e4m3fn: PA_FP8_E4M3})
+    code = _DTYPE_CODES.get(t.dtype)
+    if code is None:
         raise TypeError(f"unsupported tensor dtype {t.dtype}")
-    return codes[t.dtype]
+    return code
+
+
+# A descriptor holds only the address, dtype, shape and strides, so one built for the same four
+# values is the same descriptor whatever tensor they came from: descriptors are kept and reused
+# (a decode loop passes the same buffers every step; building a ctypes structure costs
+# microseconds of host time per tensor).
+_DESCRIPTORS: dict = {}
+_DESCRIPTORS_MAX = 4096
 
 
 def describe(t) -> PaTensor:
-    """pa_tensor descriptor of a torch tensor (no copy; the tensor must outlive the call)."""
-    d = PaTensor()
-    d.data = t.data_ptr()
-    d.dtype = _torch_dtype_code(t)
-    d.ndim = t.dim()
+    """pa_tensor descriptor of a torch tensor (no copy; the tensor must outlive the call).  The
+    descriptor is shared by every tensor with the same address, dtype, shape and strides: do not
+    modify it."""
+    key = (t.data_ptr(), t.dtype, t.shape, t.stride())
+    d = _DESCRIPTORS.get(key)
+    if d is not None:
+        return d
     if t.dim() > 5:
         raise ValueError("at most 5 dimensions")
-    for i, (n, s) in enumerate(zip(t.shape, t.stride())):
-        d.shape[i] = n
-        d.stride[i] = s
+    shape = (ctypes.c_int64 * 5)(*t.shape)
+    stride = (ctypes.c_int64 * 5)(*t.stride())
+    d = PaTensor(t.data_ptr(), _torch_dtype_code(t), t.dim(), shape, stride)
+    if len(_DESCRIPTORS) >= _DESCRIPTORS_MAX:
+        _DESCRIPTORS.clear()
+    _DESCRIPTORS[key] = d
     return d
 
 

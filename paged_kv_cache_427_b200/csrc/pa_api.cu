@@ -41,6 +41,7 @@ int cuda_fail(cudaError_t e, const char *what) {
 }
 
 typedef CUresult (*MemGetAddressRangeFn)(CUdeviceptr *, size_t *, CUdeviceptr);
+typedef CUresult (*PointerGetAttributesFn)(unsigned int, CUpointer_attribute *, void **, CUdeviceptr);
 typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
                                   const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
                                   const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
@@ -101,8 +102,9 @@ std::vector<DeviceState> g_devices;
 // counters.  For each workspace the library remembers how many leading bytes are known to hold
 // zero counters and zeroes the rest (on the call's stream) before a call that needs more.
 // How far a call goes: host-side argument checks only, every check (device memory, workspace
-// size) without launching, or the whole call.
-enum class CallMode { kHostChecks, kAllChecks, kLaunch };
+// size) without launching, the whole call, or the launch of a call whose every check has just
+// passed with the same arguments (its device-memory queries are not repeated).
+enum class CallMode { kHostChecks, kAllChecks, kLaunch, kLaunchChecked };
 
 // Measurement aid (pa_set_decode_timeline): where decode launches record per-warp timestamps.
 unsigned long long *g_timeline = nullptr;  // guarded by g_mu
@@ -122,6 +124,7 @@ CleanRecord &clean_record(const void *ws) {
   return g_clean.back();
 }
 MemGetAddressRangeFn g_mem_range = nullptr;
+PointerGetAttributesFn g_ptr_attrs = nullptr;
 EncodeTiledFn g_encode_tiled = nullptr;
 bool g_mem_range_tried = false;
 
@@ -148,6 +151,11 @@ int device_state(DeviceState **out, int *dev_out) {
             cudaSuccess &&
         q == cudaDriverEntryPointSuccess)
       g_mem_range = reinterpret_cast<MemGetAddressRangeFn>(fn);
+    fn = nullptr;
+    if (cudaGetDriverEntryPoint("cuPointerGetAttributes", &fn, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_ptr_attrs = reinterpret_cast<PointerGetAttributesFn>(fn);
     fn = nullptr;
     if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) ==
             cudaSuccess &&
@@ -218,6 +226,31 @@ int check_device_memory(const pa_tensor *t, const char *name, int dev) {
   const uint64_t ext = extent_bytes(t);
   if (ext == 0) return PA_OK;
   if (!t->data) return fail(PA_ERR_INVALID_ARG, "%s: NULL data pointer", name);
+  const uint64_t p = (uint64_t)(uintptr_t)t->data;
+  if (g_ptr_attrs) {
+    // One driver query for the memory type, the device, managed or not and the allocation's
+    // range (a pointer the driver does not know comes back with type 0).
+    CUmemorytype type = (CUmemorytype)0;
+    int ordinal = -1;
+    CUdeviceptr start = 0;
+    size_t size = 0;
+    unsigned int managed = 0;  // the driver writes a one-byte bool into the low byte
+    CUpointer_attribute which[5] = {CU_POINTER_ATTRIBUTE_MEMORY_TYPE, CU_POINTER_ATTRIBUTE_DEVICE_ORDINAL,
+                                    CU_POINTER_ATTRIBUTE_RANGE_START_ADDR, CU_POINTER_ATTRIBUTE_RANGE_SIZE,
+                                    CU_POINTER_ATTRIBUTE_IS_MANAGED};
+    void *data[5] = {&type, &ordinal, &start, &size, &managed};
+    if (g_ptr_attrs(5, which, data, (CUdeviceptr)(uintptr_t)t->data) == CUDA_SUCCESS) {
+      const bool is_managed = (managed & 0xffu) != 0;
+      if (type != CU_MEMORYTYPE_DEVICE && type != CU_MEMORYTYPE_UNIFIED && !is_managed)
+        return fail(PA_ERR_LAYOUT, "%s: not device memory", name);
+      if (!is_managed && type == CU_MEMORYTYPE_DEVICE && ordinal != dev)
+        return fail(PA_ERR_LAYOUT, "%s: lives on device %d, current device is %d", name, ordinal, dev);
+      if (size > 0 && p + ext > (uint64_t)start + size)
+        return fail(PA_ERR_LAYOUT, "%s: addresses %llu bytes but its allocation ends after %llu", name,
+                    (unsigned long long)ext, (unsigned long long)((uint64_t)start + size - p));
+      return PA_OK;
+    }
+  }
   cudaPointerAttributes attr;
   cudaError_t e = cudaPointerGetAttributes(&attr, t->data);
   if (e != cudaSuccess) {
@@ -232,7 +265,6 @@ int check_device_memory(const pa_tensor *t, const char *name, int dev) {
     CUdeviceptr base = 0;
     size_t size = 0;
     // When the driver cannot name the allocation the pointer check above stands alone.
-    const uint64_t p = (uint64_t)(uintptr_t)t->data;
     if (g_mem_range(&base, &size, (CUdeviceptr)(uintptr_t)t->data) == CUDA_SUCCESS &&
         p + ext > (uint64_t)base + size)
       return fail(PA_ERR_LAYOUT, "%s: addresses %llu bytes but its allocation ends after %llu", name,
@@ -407,13 +439,29 @@ int query_map(const pa_tensor *q, int G, CUtensorMap *out) {
 }
 
 // Warps of one full wave of the device for a kernel (CTAs per SM x SMs x warps per CTA).
+// The occupancy query is asked once per kernel and device (it costs host time on every call).
 int default_workers(const pa::DecodeKernel &k, int num_sms) {
+  struct Occ {
+    const void *kernel;
+    int dev, per_sm;
+  };
+  static std::vector<Occ> known;  // guarded by g_mu
+  int dev = 0;
+  cudaGetDevice(&dev);
+  {
+    std::lock_guard<std::mutex> lock(g_mu);
+    for (const Occ &o : known)
+      if (o.kernel == k.kernel && o.dev == dev) return o.per_sm * num_sms * k.warps_per_cta;
+  }
   int per_sm = 0;
   if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k.kernel, k.threads_per_cta,
                                                     k.smem_bytes) != cudaSuccess ||
       per_sm < 1) {
     cudaGetLastError();
     per_sm = 1;
+  } else {
+    std::lock_guard<std::mutex> lock(g_mu);
+    known.push_back(Occ{k.kernel, dev, per_sm});
   }
   return per_sm * num_sms * k.warps_per_cta;
 }
@@ -618,6 +666,7 @@ int decode_impl(const pa_tensor *out, const pa_tensor *query, const pa_tensor *k
   DeviceState *ds;
   int dev;
   if ((rc = device_state(&ds, &dev))) return rc;
+  if (mode != CallMode::kLaunchChecked) {
   if (shared && ((rc = check_device_memory(group_start, "group_start", dev)) ||
                  (rc = check_device_memory(prefix_lens, "prefix_lens", dev))))
     return rc;
@@ -630,6 +679,7 @@ int decode_impl(const pa_tensor *out, const pa_tensor *query, const pa_tensor *k
   if (fp8 && ((rc = check_device_memory(k_scale, "k_scale", dev)) ||
               (rc = check_device_memory(v_scale, "v_scale", dev))))
     return rc;
+  }
 
   pa::DecodeKernel k;
   const bool tensor_cores = cs.dtype != PA_F32 && !(flags & PA_DECODE_CUDA_CORES);
@@ -820,10 +870,11 @@ int write_impl(const pa_tensor *key, const pa_tensor *value, const pa_tensor *ke
   DeviceState *ds;
   int dev;
   if ((rc = device_state(&ds, &dev))) return rc;
-  if ((rc = check_device_memory(key_cache, "key_cache", dev)) ||
-      (rc = check_device_memory(value_cache, "value_cache", dev)) ||
-      (rc = check_device_memory(key, "key", dev)) || (rc = check_device_memory(value, "value", dev)) ||
-      (rc = check_device_memory(slot_mapping, "slot_mapping", dev)))
+  if (mode != CallMode::kLaunchChecked &&
+      ((rc = check_device_memory(key_cache, "key_cache", dev)) ||
+       (rc = check_device_memory(value_cache, "value_cache", dev)) ||
+       (rc = check_device_memory(key, "key", dev)) || (rc = check_device_memory(value, "value", dev)) ||
+       (rc = check_device_memory(slot_mapping, "slot_mapping", dev))))
     return rc;
   const size_t e = elt_size(cs.dtype);
   pa::CacheWriteArgs a;
@@ -1153,8 +1204,8 @@ int pa_decode_step(const pa_tensor *key, const pa_tensor *value, const pa_tensor
     if (key->shape[0] > 0)
       return decode_impl(out, query, key_cache, value_cache, block_tables, context_lens, scale,
                          block_size, num_kv_heads, 0, PA_DECODE_OVERLAP_PREVIOUS, workspace,
-                         workspace_bytes, lib_ws, stream, CallMode::kLaunch, nullptr, nullptr,
-                         nullptr, nullptr, &w);
+                         workspace_bytes, lib_ws, stream, CallMode::kLaunchChecked, nullptr,
+                         nullptr, nullptr, nullptr, &w);
     return PA_OK;
   }
   // both halves are checked (host-side checks of both first) before either is launched
@@ -1164,11 +1215,12 @@ int pa_decode_step(const pa_tensor *key, const pa_tensor *value, const pa_tensor
                           block_size, num_kv_heads, 0, PA_DECODE_OVERLAP_PREVIOUS, workspace,
                           workspace_bytes, lib_ws, stream, m)))
       return rc;
-  if ((rc = write_impl(key, value, key_cache, value_cache, slot_mapping, stream, CallMode::kLaunch)))
+  if ((rc = write_impl(key, value, key_cache, value_cache, slot_mapping, stream,
+                      CallMode::kLaunchChecked)))
     return rc;
   return decode_impl(out, query, key_cache, value_cache, block_tables, context_lens, scale,
                      block_size, num_kv_heads, 0, PA_DECODE_OVERLAP_PREVIOUS, workspace,
-                     workspace_bytes, lib_ws, stream);
+                     workspace_bytes, lib_ws, stream, CallMode::kLaunchChecked);
 }
 
 int pa_copy_blocks(const pa_tensor *key_cache, const pa_tensor *value_cache,
