@@ -1154,10 +1154,10 @@ def measure_e2e(args, b, pools, rot, mapping, out, ws, decode, dev, stream, worl
 
 def run_fp8(args, b, config, full: bool = True, probe: dict | None = None) -> dict:
     """The same decode step over an FP8 E4M3 cache: the pool is the workload's pool quantised
-    (per-kv-head scales: largest magnitude of the head's rows / 240), each step writes the new
-    tokens with pa_reshape_and_cache_fp8 and decodes with pa_decode_fp8 launched to overlap the
-    write.  Timed like the 16-bit step: K steps with nothing between launches (`value`), then
-    steps with events around each decode (the roofline)."""
+    (per-kv-head scales: largest magnitude of the head's rows / 240), and each step is one
+    pa_decode_step_fp8 call (one kernel: the new tokens quantised into the caches, and the
+    decode).  Timed like the 16-bit step: K steps with nothing between launches (`value`), then
+    steps with events around each call (the roofline)."""
     import torch
 
     import paged_kv_cache_427_b200 as pa
@@ -1200,11 +1200,10 @@ def run_fp8(args, b, config, full: bool = True, probe: dict | None = None) -> di
 
     def step(i, ev=None):
         kc, vc = pools[i % rot]
-        pa.pa_reshape_and_cache_fp8(key, value, kc, vc, slots, ks, vs)
         if ev is not None:
             ev[0].record(stream)
-        pa.pa_decode_fp8(out, q, kc, vc, tables, lens, ks, vs, b.scale, b.block_size,
-                         b.num_kv_heads, 0, pa.PA_DECODE_OVERLAP_PREVIOUS, ws)
+        pa.pa_decode_step_fp8(key, value, kc, vc, slots, ks, vs, out, q, tables, lens, b.scale,
+                              b.block_size, b.num_kv_heads, workspace=ws)
         if ev is not None:
             ev[1].record(stream)
 
@@ -1251,10 +1250,11 @@ def run_fp8(args, b, config, full: bool = True, probe: dict | None = None) -> di
             "attended_tokens_per_s": round(b.attended_tokens / (ms * 1e-3), 1),
             "seq_steps_per_s": round(b.num_seqs / (ms * 1e-3), 1),
             "pct_of_8TBs": round(100 * value / NOMINAL_HBM_GBS, 2),
-            "roofline": hbm_roofline(dec, dec_ms, "paged_decode_mma_kernel (fp8 e4m3 cache)",
+            "roofline": hbm_roofline(dec, dec_ms, "paged_decode_mma_kernel (fp8 e4m3 cache), fused "
+                                     "step: the quantising cache write inside the same kernel",
                                      recorded_traffic(config["workload"] + ":fp8", "decode_fp8"),
                                      probe),
-            "gpu_launches": 2 * args.steps, "clocks": clocks}
+            "gpu_launches": args.steps, "clocks": clocks}
     if timeline:
         line["timeline"] = timeline
     if full and not args.no_cpu_baseline:
@@ -1335,7 +1335,7 @@ def run_prefill(args, b, config, full: bool = True) -> dict:
                          "unit": "TFLOP/s", "frac": round(tflops / peak, 4), "traffic": traffic,
                          "kernel": "paged_prefill_tc_kernel (tcgen05 + TMEM + TMA)",
                          "peak_source": src, "algorithmic_flops_per_launch": flops, **st},
-            "gpu_launches": 2 * args.steps, "clocks": clocks}
+            "gpu_launches": args.steps, "clocks": clocks}
     if full and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline_prefill(b, args.cpu_seconds)
     return line

@@ -62,7 +62,7 @@
 extern "C" {
 #endif
 
-#define PA_VERSION 6
+#define PA_VERSION 7
 
 /* Symbols of this ABI are the only ones the shared library exports. */
 #if defined(__GNUC__)
@@ -223,6 +223,28 @@ PA_API int pa_decode_fp8(const pa_tensor *out, const pa_tensor *query, const pa_
                          const pa_tensor *v_scale, float scale, int32_t block_size,
                          int32_t num_kv_heads, int32_t num_workers, uint32_t flags,
                          void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * pa_decode_step_fp8 - one whole decode step over FP8 caches: pa_reshape_and_cache_fp8(key,
+ * value, key_cache, value_cache, slot_mapping, k_scale, v_scale) followed by pa_decode_fp8(out,
+ * query, ..., num_workers = 0, PA_DECODE_OVERLAP_PREVIOUS, workspace), as pa_decode_step is for
+ * 16-bit caches.  One new token per sequence (key->shape[0] == number of sequences) whose
+ * key/value have the query's 16-bit type: ONE kernel.  Token s is sequence s's position
+ * context_lens[s] - 1; the kernel quantises it into slot slot_mapping[s] (codes identical to
+ * pa_reshape_and_cache_fp8's) and attends to those same codes for that position, so no part of
+ * the decode waits for the write; a slot that is not that position is stored as asked and sets
+ * PA_DEVERR_SLOT.  Any other shape or an fp32 key/value: two kernels, the write and then the
+ * decode launched to overlap it.  Both halves are validated before either is launched.
+ * workspace as for pa_decode_fp8 (NULL: the library-owned one).  Errors as for the two calls.
+ */
+PA_API int pa_decode_step_fp8(const pa_tensor *key, const pa_tensor *value,
+                              const pa_tensor *key_cache, const pa_tensor *value_cache,
+                              const pa_tensor *slot_mapping, const pa_tensor *k_scale,
+                              const pa_tensor *v_scale, const pa_tensor *out,
+                              const pa_tensor *query, const pa_tensor *block_tables,
+                              const pa_tensor *context_lens, float scale, int32_t block_size,
+                              int32_t num_kv_heads, void *workspace, size_t workspace_bytes,
+                              void *stream);
 
 /*
  * pa_prefill - causal attention of a step's new tokens (a prompt, or a chunk of one, of each

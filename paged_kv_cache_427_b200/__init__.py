@@ -94,6 +94,8 @@ def load(path: str = LIBRARY) -> ctypes.CDLL:
     lib.pa_get_device_error.argtypes = [_P, ctypes.POINTER(u32), i32]
     lib.pa_decode_noalloc.argtypes = [_T, _T, _T, _T, _T, _T, f32, i32, i32, _P]
     lib.pa_decode_step.argtypes = [_T, _T, _T, _T, _T, _T, _T, _T, _T, f32, i32, i32, _P, sz, _P]
+    lib.pa_decode_step_fp8.argtypes = [_T] * 11 + [f32, i32, i32, _P, sz, _P]
+    lib.pa_decode_step_fp8.restype = ctypes.c_int
     lib.pa_decode_shared_prefix.argtypes = [_T, _T, _T, _T, _T, _T, _T, _T, f32, i32, i32, _P, sz, _P]
     lib.pa_decode_shared_prefix.restype = ctypes.c_int
     lib.pa_decode_shared_prefix_workspace_bytes.argtypes = [i64, i32, i32, i32, i64, i32]
@@ -249,6 +251,21 @@ def pa_decode_ex(out, query, key_cache, value_cache, block_tables, context_lens,
     _check("pa_decode_ex", lib.pa_decode_ex(*[ctypes.byref(x) for x in d], float(scale),
                                             int(block_size), int(num_kv_heads), int(num_workers),
                                             int(flags), ws_ptr, ws_bytes, _stream(stream)))
+
+
+def pa_decode_step_fp8(key, value, key_cache, value_cache, slot_mapping, k_scale, v_scale, out,
+                       query, block_tables, context_lens, scale, block_size, num_kv_heads,
+                       workspace=None, stream=None):
+    """One whole step over FP8 caches: the quantising cache write and the decode, one kernel
+    when each sequence brings one token in the query's type (see include/pa.h)."""
+    lib = load()
+    d = [describe(x) for x in (key, value, key_cache, value_cache, slot_mapping, k_scale, v_scale,
+                               out, query, block_tables, context_lens)]
+    ws_ptr = workspace.data_ptr() if workspace is not None else None
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check("pa_decode_step_fp8", lib.pa_decode_step_fp8(*[ctypes.byref(x) for x in d], float(scale),
+                                                        int(block_size), int(num_kv_heads), ws_ptr,
+                                                        ws_bytes, _stream(stream)))
 
 
 def pa_decode_step(key, value, key_cache, value_cache, slot_mapping, out, query, block_tables,

@@ -979,7 +979,8 @@ int copy_blocks_impl(const pa_tensor *src_k, const pa_tensor *src_v, const pa_te
 
 int write_fp8_impl(const pa_tensor *key, const pa_tensor *value, const pa_tensor *key_cache,
                    const pa_tensor *value_cache, const pa_tensor *slot_mapping,
-                   const pa_tensor *k_scale, const pa_tensor *v_scale, void *stream) {
+                   const pa_tensor *k_scale, const pa_tensor *v_scale, void *stream,
+                   CallMode mode = CallMode::kLaunch, pa::CacheWriteArgs *prepared = nullptr) {
   int rc;
   CacheShape cs;
   if ((rc = check_caches(key_cache, value_cache, &cs, true))) return rc;
@@ -1008,18 +1009,43 @@ int write_fp8_impl(const pa_tensor *key, const pa_tensor *value, const pa_tensor
   if (!aligned16(key->data) || !aligned16(value->data) || !strides16(key, 2) || !strides16(value, 2))
     return fail(PA_ERR_LAYOUT, "key/value: data and token/head strides must be 16-byte aligned");
   if (cs.head_dim % 16 != 0) return fail(PA_ERR_UNSUPPORTED, "FP8 caches: head_dim must be a multiple of 16");
-  if (T == 0) return PA_OK;
+  if (T == 0 || mode == CallMode::kHostChecks) return PA_OK;
   DeviceState *ds;
   int dev;
   if ((rc = device_state(&ds, &dev))) return rc;
-  if ((rc = check_device_memory(key_cache, "key_cache", dev)) ||
-      (rc = check_device_memory(value_cache, "value_cache", dev)) ||
-      (rc = check_device_memory(key, "key", dev)) || (rc = check_device_memory(value, "value", dev)) ||
-      (rc = check_device_memory(slot_mapping, "slot_mapping", dev)) ||
-      (rc = check_device_memory(k_scale, "k_scale", dev)) ||
-      (rc = check_device_memory(v_scale, "v_scale", dev)))
+  if (mode != CallMode::kLaunchChecked &&
+      ((rc = check_device_memory(key_cache, "key_cache", dev)) ||
+       (rc = check_device_memory(value_cache, "value_cache", dev)) ||
+       (rc = check_device_memory(key, "key", dev)) || (rc = check_device_memory(value, "value", dev)) ||
+       (rc = check_device_memory(slot_mapping, "slot_mapping", dev)) ||
+       (rc = check_device_memory(k_scale, "k_scale", dev)) ||
+       (rc = check_device_memory(v_scale, "v_scale", dev))))
     return rc;
   const size_t se = elt_size(key->dtype);
+  if (prepared) {
+    // the same write done by the fused decode step (16-bit key/value rows, codes of head_dim
+    // bytes per cache row)
+    pa::CacheWriteArgs w;
+    w.key = static_cast<const char *>(key->data);
+    w.value = static_cast<const char *>(value->data);
+    w.k_tok = key->stride[0] * (int64_t)se;
+    w.k_head = key->stride[1] * (int64_t)se;
+    w.v_tok = value->stride[0] * (int64_t)se;
+    w.v_head = value->stride[1] * (int64_t)se;
+    w.key_cache = static_cast<char *>(key_cache->data);
+    w.value_cache = static_cast<char *>(value_cache->data);
+    w.c_blk = key_cache->stride[0];
+    w.c_head = key_cache->stride[1];
+    w.row_bytes = cs.head_dim;
+    w.slots = static_cast<const int64_t *>(slot_mapping->data);
+    w.num_tokens = T;
+    w.num_kv_heads = cs.num_kv_heads;
+    w.block_size = cs.block_size;
+    w.num_slots = cs.num_blocks * cs.block_size;
+    w.err = ds->err;
+    *prepared = w;
+  }
+  if (mode == CallMode::kAllChecks) return PA_OK;
   pa::CacheWriteFp8Args a;
   a.key = static_cast<const char *>(key->data);
   a.value = static_cast<const char *>(value->data);
@@ -1178,6 +1204,44 @@ int pa_decode_fp8(const pa_tensor *out, const pa_tensor *query, const pa_tensor 
 int pa_reshape_and_cache(const pa_tensor *key, const pa_tensor *value, const pa_tensor *key_cache,
                          const pa_tensor *value_cache, const pa_tensor *slot_mapping, void *stream) {
   return write_impl(key, value, key_cache, value_cache, slot_mapping, stream, CallMode::kLaunch);
+}
+
+int pa_decode_step_fp8(const pa_tensor *key, const pa_tensor *value, const pa_tensor *key_cache,
+                       const pa_tensor *value_cache, const pa_tensor *slot_mapping,
+                       const pa_tensor *k_scale, const pa_tensor *v_scale, const pa_tensor *out,
+                       const pa_tensor *query, const pa_tensor *block_tables,
+                       const pa_tensor *context_lens, float scale, int32_t block_size,
+                       int32_t num_kv_heads, void *workspace, size_t workspace_bytes,
+                       void *stream) {
+  if (!k_scale || !v_scale) return fail(PA_ERR_INVALID_ARG, "k_scale and v_scale are required");
+  const bool lib_ws = workspace == nullptr;
+  int rc;
+  // One new token per sequence, in the query's 16-bit type: one kernel, which quantises the
+  // token into the caches and into its tiles as position L-1.  Otherwise the write kernel, then
+  // the decode launched to overlap it.
+  const bool fused = key && query && context_lens && key->ndim == 3 && context_lens->ndim == 1 &&
+                     key->shape[0] == context_lens->shape[0] && key->dtype == query->dtype;
+  pa::CacheWriteArgs w;
+  for (CallMode m : {CallMode::kHostChecks, CallMode::kAllChecks})
+    if ((rc = write_fp8_impl(key, value, key_cache, value_cache, slot_mapping, k_scale, v_scale,
+                             stream, m, fused ? &w : nullptr)) ||
+        (rc = decode_impl(out, query, key_cache, value_cache, block_tables, context_lens, scale,
+                          block_size, num_kv_heads, 0, PA_DECODE_OVERLAP_PREVIOUS, workspace,
+                          workspace_bytes, lib_ws, stream, m, k_scale, v_scale)))
+      return rc;
+  if (fused) {
+    if (key->shape[0] == 0) return PA_OK;
+    return decode_impl(out, query, key_cache, value_cache, block_tables, context_lens, scale,
+                       block_size, num_kv_heads, 0, PA_DECODE_OVERLAP_PREVIOUS, workspace,
+                       workspace_bytes, lib_ws, stream, CallMode::kLaunchChecked, k_scale,
+                       v_scale, nullptr, nullptr, &w);
+  }
+  if ((rc = write_fp8_impl(key, value, key_cache, value_cache, slot_mapping, k_scale, v_scale,
+                           stream, CallMode::kLaunchChecked)))
+    return rc;
+  return decode_impl(out, query, key_cache, value_cache, block_tables, context_lens, scale,
+                     block_size, num_kv_heads, 0, PA_DECODE_OVERLAP_PREVIOUS, workspace,
+                     workspace_bytes, lib_ws, stream, CallMode::kLaunchChecked, k_scale, v_scale);
 }
 
 int pa_decode_step(const pa_tensor *key, const pa_tensor *value, const pa_tensor *key_cache,

@@ -76,36 +76,6 @@ __global__ void __launch_bounds__(256) copy_blocks_kernel(CopyBlocksArgs a) {
   }
 }
 
-// Two fp32 values -> two FP8 E4M3 codes (round to nearest even, saturated to +-448, NaN kept),
-// x0 in the low byte.
-__device__ __forceinline__ uint16_t f32x2_to_fp8x2(float x0, float x1) {
-  uint16_t r;
-  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(x1), "f"(x0));
-  return r;
-}
-
-template <typename S>
-__device__ __forceinline__ void load_row16(const char *p, float (&f)[16]) {
-  if constexpr (sizeof(S) == 4) {
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const uint4 v = __ldg(reinterpret_cast<const uint4 *>(p) + i);
-      f[4 * i] = __uint_as_float(v.x);
-      f[4 * i + 1] = __uint_as_float(v.y);
-      f[4 * i + 2] = __uint_as_float(v.z);
-      f[4 * i + 3] = __uint_as_float(v.w);
-    }
-  } else {
-#pragma unroll
-    for (int i = 0; i < 2; ++i) {
-      float g[8];
-      Elem<S>::unpack(__ldg(reinterpret_cast<const uint4 *>(p) + i), g);
-#pragma unroll
-      for (int j = 0; j < 8; ++j) f[8 * i + j] = g[j];
-    }
-  }
-}
-
 // One thread per 16 codes (16 elements) of one (token, kv head) row, keys and values together.
 // Each element is divided by its head's scale in fp32 (IEEE division) before the conversion.
 template <typename S>
@@ -129,19 +99,10 @@ __global__ void __launch_bounds__(256) reshape_and_cache_fp8_kernel(CacheWriteFp
     const int64_t dst = (slot / a.block_size) * a.c_blk + h * a.c_head +
                         (slot % a.block_size) * a.head_dim + v * 16;
     const float ks = __ldg(a.k_scale + h), vs = __ldg(a.v_scale + h);
-    float fk[16], fv[16];
-    load_row16<S>(a.key + t * a.k_tok + h * a.k_head + (int64_t)v * 16 * sizeof(S), fk);
-    load_row16<S>(a.value + t * a.v_tok + h * a.v_head + (int64_t)v * 16 * sizeof(S), fv);
-    uint32_t ck[4], cv[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      ck[i] = (uint32_t)f32x2_to_fp8x2(__fdiv_rn(fk[4 * i], ks), __fdiv_rn(fk[4 * i + 1], ks)) |
-              ((uint32_t)f32x2_to_fp8x2(__fdiv_rn(fk[4 * i + 2], ks), __fdiv_rn(fk[4 * i + 3], ks)) << 16);
-      cv[i] = (uint32_t)f32x2_to_fp8x2(__fdiv_rn(fv[4 * i], vs), __fdiv_rn(fv[4 * i + 1], vs)) |
-              ((uint32_t)f32x2_to_fp8x2(__fdiv_rn(fv[4 * i + 2], vs), __fdiv_rn(fv[4 * i + 3], vs)) << 16);
-    }
-    *reinterpret_cast<uint4 *>(a.key_cache + dst) = make_uint4(ck[0], ck[1], ck[2], ck[3]);
-    *reinterpret_cast<uint4 *>(a.value_cache + dst) = make_uint4(cv[0], cv[1], cv[2], cv[3]);
+    *reinterpret_cast<uint4 *>(a.key_cache + dst) =
+        fp8_codes16<S>(a.key + t * a.k_tok + h * a.k_head + (int64_t)v * 16 * sizeof(S), ks);
+    *reinterpret_cast<uint4 *>(a.value_cache + dst) =
+        fp8_codes16<S>(a.value + t * a.v_tok + h * a.v_head + (int64_t)v * 16 * sizeof(S), vs);
   }
 }
 

@@ -82,6 +82,44 @@ __device__ __forceinline__ void fused_cache_write(const DecodeArgs &a, int max_l
   }
 }
 
+// The same for FP8 E4M3 caches: token s's 16-bit rows (element type S) are quantised with the
+// cache write's arithmetic (fp8_codes16), so the codes match what that kernel would store.
+// w.row_bytes is the cache row (head_dim codes).
+template <typename S, int BS>
+__device__ __forceinline__ void fused_cache_write_fp8(const DecodeArgs &a, int max_len, int tid,
+                                                      int nthreads) {
+  const CacheWriteArgs &w = a.step;
+  const int vec_per_row = w.row_bytes >> 4;  // 16 codes per item
+  const int64_t total = w.num_tokens * w.num_kv_heads * vec_per_row;
+  for (int64_t idx = tid; idx < total; idx += nthreads) {
+    const int v = (int)(idx % vec_per_row);
+    const int64_t th = idx / vec_per_row;
+    const int h = (int)(th % w.num_kv_heads);
+    const int64_t t = th / w.num_kv_heads;
+    const int64_t slot = __ldg(w.slots + t);
+    if (h == 0 && v == 0) {
+      const int len = clamp_len(__ldg(a.context_lens + t), max_len);
+      int64_t expect = -1;
+      if (len > 0) {
+        const int blk = __ldg(a.block_tables + t * a.bt_s + (len - 1) / BS);
+        expect = (int64_t)blk * BS + (len - 1) % BS;
+      }
+      if (slot != expect) set_error(a.err, PA_DEVERR_SLOT);
+    }
+    if (slot < 0) continue;
+    if (slot >= w.num_slots) {
+      if (h == 0 && v == 0) set_error(a.err, PA_DEVERR_SLOT);
+      continue;
+    }
+    const int64_t dst = (slot / w.block_size) * w.c_blk + h * w.c_head + (slot % w.block_size) * w.row_bytes + v * 16;
+    const int64_t src = (int64_t)v * 16 * (int64_t)sizeof(S);
+    *reinterpret_cast<uint4 *>(w.key_cache + dst) =
+        fp8_codes16<S>(w.key + t * w.k_tok + h * w.k_head + src, __ldg(a.k_scale + h));
+    *reinterpret_cast<uint4 *>(w.value_cache + dst) =
+        fp8_codes16<S>(w.value + t * w.v_tok + h * w.v_head + src, __ldg(a.v_scale + h));
+  }
+}
+
 // The first position the decode reads of sequence s, whose context holds len positions: its
 // shared prefix when the shared-prefix pass covered it (0 < prefix < len, a multiple of the block
 // size, within the pass's items), else 0 (the whole context is decoded here).  A prefix that is

@@ -143,8 +143,9 @@ struct MmaTraits {
   static constexpr int kBoxBytes = kBoxRows * D * KVB;  // one box: [block][row][128 B]
   static constexpr int kTileBytes = 16 * D * KVB;       // key (or value) bytes of a chunk
   static constexpr int kQBytes = G * D * 2;
-  // a fused decode step's new key and value rows of the chunk holding position L-1 (16-bit)
-  static constexpr int kNewBytes = KVB == 2 ? 2 * D * 2 : 0;
+  // a fused decode step's new key and value rows of the chunk holding position L-1 (16-bit,
+  // the query's type; quantised in shared memory for FP8 caches)
+  static constexpr int kNewBytes = 2 * D * 2;
   static constexpr int kNewOff = 2 * kTileBytes + kQBytes;
   static constexpr int kStageBytes = 2 * kTileBytes + (kQBytes + kNewBytes + 1023) / 1024 * 1024;
   static constexpr int kWorkers = 4;                    // consumer warps
@@ -326,7 +327,7 @@ __global__ void __launch_bounds__(MmaTraits<D, BS, G, (int)sizeof(KV)>::kThreads
     // rows when a new (sequence, kv head) starts, all counted on the stage's full barrier.
     auto issue = [&](int slot) {
       // fused step: the chunk holding position L-1 also brings that position's new rows
-      const bool new_row = !kFp8 && a.fused && cur.i == cur.nch - 1;
+      const bool new_row = a.fused && cur.i == cur.nch - 1;
       const int f = cur.flags() | (new_row ? kNewRow : 0);
       unsigned char *stage = ring + slot * Tr::kStageBytes;
       meta[slot] = cur.meta(f);
@@ -422,7 +423,12 @@ __global__ void __launch_bounds__(MmaTraits<D, BS, G, (int)sizeof(KV)>::kThreads
         if (clamp_len(__ldg(a.context_lens + s), max_len) == 0)
           zero_rows<D>(static_cast<char *>(a.out) + (long long)s * a.out_s * out_elt, a.out_h,
                        a.out_dtype, a.num_kv_heads * G);
-      if (a.fused) fused_cache_write<BS>(a, max_len, blockIdx.x * 32 + lane, launched_lanes);
+      if (a.fused) {
+        if constexpr (kFp8)
+          fused_cache_write_fp8<T, BS>(a, max_len, blockIdx.x * 32 + lane, launched_lanes);
+        else
+          fused_cache_write<BS>(a, max_len, blockIdx.x * 32 + lane, launched_lanes);
+      }
     }
     // Lane k follows worker k's mailbox.  For each split piece the warp makes the piece's
     // stores visible GPU-wide, takes the ticket of its (sequence, kv head) and, when the piece
@@ -520,7 +526,24 @@ __global__ void __launch_bounds__(MmaTraits<D, BS, G, (int)sizeof(KV)>::kThreads
     if (tl && cc == 0) tl[kTlFirst] = global_ns();
     const ChunkMeta m = meta[slot];
     unsigned char *stage = ring + slot * Tr::kStageBytes;
-    if constexpr (!kFp8) {
+    if constexpr (kFp8) {
+      if (m.flags & kNewRow) {
+        // fused step over FP8 caches: the new token's 16-bit rows quantised as the cache write
+        // quantises them (fp8_codes8), into row (L-1) % 16 of the FP8 tiles: lane l takes
+        // elements 8 (l % 16) .. + 7 of the key (l < 16) or value row, which land in half
+        // l % 2 of 16-byte piece (l % 16) / 2 of the swizzled row
+        static_assert(D == 128, "FP8 rows of one 128-byte span");
+        const int r = (m.len - 1) & 15;
+        const int which = lane >> 4, j = lane & 15;
+        float f[8];
+        Elem<T>::unpack(*reinterpret_cast<const uint4 *>(stage + Tr::kNewOff + which * D * 2 + j * 16), f);
+        const uint2 codes = fp8_codes8(f, __ldg((which ? a.v_scale : a.k_scale) + m.kvh));
+        *reinterpret_cast<uint2 *>(stage + which * Tr::kTileBytes + tile_offset<Tr>(r, 0) +
+                                   ((((j >> 1) ^ (r & 7)) << 4) | ((j & 1) << 3))) = codes;
+        fence_proxy_async_smem();  // before the stage is copied into again
+        __syncwarp();
+      }
+    } else {
       if (m.flags & kNewRow) {
         // fused step: position L-1 is this step's new token, read from the step's key and
         // value rather than the cache (which this kernel writes concurrently); put its rows into

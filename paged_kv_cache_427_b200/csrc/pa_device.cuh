@@ -65,6 +65,49 @@ struct Elem<__half> {
   }
 };
 
+// ------------------------------------------------------------------------------------------
+// FP8 E4M3 cache codes.  A value x of kv head h is stored as code(x / scale[h]): the division in
+// fp32 (IEEE, round to nearest), the conversion rounding to nearest even and saturating to
+// +-448 (NaN kept).  The cache write kernel and the fused decode step both quantise with these,
+// so a position holds the same code whichever of them wrote it.
+// ------------------------------------------------------------------------------------------
+// Two fp32 values -> two codes, x0 in the low byte.
+__device__ __forceinline__ uint16_t f32x2_to_fp8x2(float x0, float x1) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(x1), "f"(x0));
+  return r;
+}
+
+// Eight values -> eight codes (element i in byte i).
+__device__ __forceinline__ uint2 fp8_codes8(const float (&f)[8], float scale) {
+  uint32_t w[2];
+#pragma unroll
+  for (int i = 0; i < 2; ++i)
+    w[i] = (uint32_t)f32x2_to_fp8x2(__fdiv_rn(f[4 * i], scale), __fdiv_rn(f[4 * i + 1], scale)) |
+           ((uint32_t)f32x2_to_fp8x2(__fdiv_rn(f[4 * i + 2], scale), __fdiv_rn(f[4 * i + 3], scale)) << 16);
+  return make_uint2(w[0], w[1]);
+}
+
+// Sixteen consecutive elements of type S at p (16-byte aligned) -> sixteen codes.
+template <typename S>
+__device__ __forceinline__ uint4 fp8_codes16(const char *p, float scale) {
+  float a[8], b[8];
+  if constexpr (sizeof(S) == 4) {
+    float g[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      Elem<float>::unpack(__ldg(reinterpret_cast<const uint4 *>(p) + i), g);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) (i < 2 ? a[4 * i + j] : b[4 * (i - 2) + j]) = g[j];
+    }
+  } else {
+    Elem<S>::unpack(__ldg(reinterpret_cast<const uint4 *>(p)), a);
+    Elem<S>::unpack(__ldg(reinterpret_cast<const uint4 *>(p) + 1), b);
+  }
+  const uint2 lo = fp8_codes8(a, scale), hi = fp8_codes8(b, scale);
+  return make_uint4(lo.x, lo.y, hi.x, hi.y);
+}
+
 // Store n (= 4 or 8) fp32 values to `dst` in the given output element type, as 16-byte
 // vectors (dst is 16-byte aligned).
 __device__ __forceinline__ void store_row_piece(void *dst, int out_dtype, const float *v, int n) {
