@@ -489,6 +489,13 @@ WsLayout ws_layout(int64_t S, int Hq, int Hkv, int D, int W) {
 
 // Shared-prefix pass: items of kPrefixItemTokens positions; its partial results follow the
 // decode workspace: pre_ml [S*Hq*splits*2] f32 | pre_o [S*Hq*splits*D] f32.
+#ifndef PA_PIECE_COST_16
+#define PA_PIECE_COST_16 1  // split cost of a (sequence, kv head) start, 16-bit caches (chunks)
+#endif
+#ifndef PA_PIECE_COST_FP8
+#define PA_PIECE_COST_FP8 3  // the same, FP8 caches
+#endif
+
 constexpr int kPrefixItemTokens = 256;  // two kv tiles of 128 positions
 
 struct PrefixLayout {
@@ -693,8 +700,14 @@ int decode_impl(const pa_tensor *out, const pa_tensor *query, const pa_tensor *k
       return rc;
   }
   const int W = num_workers > 0 ? num_workers : default_workers(k, ds->num_sms);
-  // worker_of() multiplies a chunk index by W in 64 bits
-  const double chunks = (double)S * num_kv_heads * ((double)block_tables->shape[1] * block_size / k.chunk_tokens + 1);
+  // The split's cost of a (sequence, kv head) start, in chunks: what a warp spends once per
+  // piece (query rows, partial result, ticket, merge).  Per-warp timings of the Llama-shaped
+  // step put it near one chunk's time with 16-bit caches and two to three with FP8 (whose
+  // chunks take less time); the settings are the fastest measured (1 vs 0 and 2; 3 vs 0 and 2).
+  const int piece_cost = k.tma_rows > 0 ? (fp8 ? PA_PIECE_COST_FP8 : PA_PIECE_COST_16) : 0;
+  // worker_of() multiplies a position by W in 64 bits
+  const double chunks = (double)S * num_kv_heads *
+                        ((double)block_tables->shape[1] * block_size / k.chunk_tokens + 1 + piece_cost);
   if (chunks * (double)W > 4.0e18) return fail(PA_ERR_SHAPE, "step too large for the work split");
   const WsLayout L = ws_layout(S, (int)Hq, num_kv_heads, D, W);
   const PrefixLayout PL = prefix_layout(L.total, S, (int)Hq, D, block_tables->shape[1], block_size);
@@ -768,6 +781,7 @@ int decode_impl(const pa_tensor *out, const pa_tensor *query, const pa_tensor *k
   a.num_blocks = cs.num_blocks;
   a.scale_log2 = (float)((double)scale * 1.4426950408889634);
   a.num_workers = W;
+  a.piece_cost = piece_cost;
   char *ws = static_cast<char *>(workspace);
   a.counters = reinterpret_cast<unsigned int *>(ws + L.counters);
   a.pair_meta = reinterpret_cast<int2 *>(ws + L.pair_meta);

@@ -12,12 +12,15 @@
 // 4.1 and [P4] 2.2.1.
 //
 // Work split (B200 design, not from the sources): the step's work is the list of chunks
-// (sequence, kv head, a fixed number of key rows) in sequence-major order, C chunks in all.  A
-// persistent grid of W warps gives warp w the chunks [floor(wC/W), floor((w+1)C/W)) (W is
-// clamped to C so that no share is empty).  No launch size depends on context lengths and every
-// warp moves the same number of bytes, whatever the mix of lengths.  A (sequence, kv head)
-// inside one share is written directly; otherwise each share's piece stores (o, m, l) in the
-// workspace and the last piece to finish (atomic ticket, no waiting) merges them.
+// (sequence, kv head, a fixed number of key rows) in sequence-major order, C chunks in all.
+// Every chunk costs one unit and every (sequence, kv head) a further `alpha` units at its start
+// (what a warp spends once per piece: loading the query rows, storing and merging a partial
+// result), so chunk c of pair p = s * Hkv + kvh sits at position pos(c) = c + alpha * (p + 1) of
+// T = C + alpha * S * Hkv positions.  A persistent grid of W warps gives warp w the chunks with
+// positions in [floor(wT/W), floor((w+1)T/W)) (W clamped to C): equal cost per warp, whatever the
+// mix of lengths, and no launch size depends on context lengths.  A (sequence, kv head) inside
+// one share is written directly; otherwise each share's piece stores (o, m, l) in the workspace
+// and the last piece to finish (atomic ticket, no waiting) merges them.
 #pragma once
 
 #include "pa_device.cuh"
@@ -39,9 +42,9 @@ __device__ __forceinline__ int clamp_len(int len, int max_len) {
   return len < 0 ? 0 : (len > max_len ? max_len : len);
 }
 
-// The warp whose share [floor(w*C/W), floor((w+1)*C/W)) contains chunk c.
-__device__ __forceinline__ int worker_of(long long c, long long C, int W) {
-  return (int)(((c + 1) * (long long)W + C - 1) / C - 1);
+// The warp whose share of positions [floor(w*T/W), floor((w+1)*T/W)) contains position x.
+__device__ __forceinline__ int worker_of(long long x, long long T, int W) {
+  return (int)(((x + 1) * (long long)W + T - 1) / T - 1);
 }
 
 // Fused decode step: thread `tid` of `nthreads` moves its 16-byte pieces of the step's new
@@ -154,9 +157,10 @@ __device__ __forceinline__ bool test_stalls(const DecodeArgs &a, int gw) {
 
 // Where one warp's share starts and how long it is.
 struct WarpShare {
-  long long C;  // chunks in the step
+  long long T;  // positions of the split: the step's chunks plus alpha per (sequence, kv head)
   int W;        // effective number of workers
-  long long g0, n;
+  int alpha;    // positions per (sequence, kv head) start
+  long long g0, n;  // first chunk (index in the chunk list) and number of chunks
   int s, rem, len;  // first chunk: sequence, index among that sequence's Hkv*nch chunks, length
 };
 
@@ -178,10 +182,11 @@ __device__ __forceinline__ long long warp_sum(long long x) {
 }
 
 // Warp-level prologue: every warp counts the step's chunks itself (reading context_lens
-// coalesced), takes its share, and finds the sequence holding its first chunk with a scan over
-// 32 sequences at a time.  No shared memory and no block-wide barrier, so warps start as soon
-// as they are scheduled.  Warp gw also flags bad lengths (warp 0) and zeroes the rows of empty
-// contexts s with s % (warps launched) == gw.  Returns false when this warp has no work.
+// coalesced), takes its share of positions, and finds the first chunk at or after each end of it
+// with a scan over 32 sequences at a time.  No shared memory and no block-wide barrier, so warps
+// start as soon as they are scheduled.  Warp gw also flags bad lengths (warp 0) and zeroes the
+// rows of empty contexts s with s % (warps launched) == gw.  Returns false when this warp has no
+// chunk.
 template <int CH, int kWarps, int G, int D, int BS, bool kZeroEmpty = true>
 __device__ __forceinline__ bool split_prologue(const DecodeArgs &a, int max_len, WarpShare &ws) {
   const int lane = threadIdx.x & 31;
@@ -189,6 +194,7 @@ __device__ __forceinline__ bool split_prologue(const DecodeArgs &a, int max_len,
   const int launched = gridDim.x * kWarps;
   const int S = a.num_seqs;
   const int Hkv = a.num_kv_heads;
+  const int alpha = a.piece_cost;
   long long mine = 0;
   for (int base = 0; base < S; base += 32) {
     const int s = base + lane;
@@ -203,36 +209,67 @@ __device__ __forceinline__ bool split_prologue(const DecodeArgs &a, int max_len,
     }
   }
   const long long C = warp_sum(mine) * Hkv;
+  const long long T = C + (long long)alpha * S * Hkv;
   const int W = (int)(C < (long long)a.num_workers ? C : (long long)a.num_workers);
-  ws.C = C;
+  ws.T = T;
   ws.W = W;
+  ws.alpha = alpha;
   if (W == 0 || gw >= W) return false;
-  ws.g0 = (long long)gw * C / W;
-  ws.n = (long long)(gw + 1) * C / W - ws.g0;  // >= 1 because W <= C
-  long long running = 0;
-  for (int base = 0; base < S; base += 32) {
+  // the first chunk at or after position x0 (this share's start) and x1 (the next share's)
+  const long long x0 = (long long)gw * T / W, x1 = (long long)(gw + 1) * T / W;
+  long long c1 = C;
+  bool found0 = false, found1 = false;
+  long long run_cnt = 0, run_cost = 0;
+  for (int base = 0; base < S && !found1; base += 32) {
     const int s = base + lane;
     const int full = s < S ? clamp_len(__ldg(a.context_lens + s), max_len) : 0;
     const int len = s < S ? full - decode_start<BS>(a, s, full) : 0;  // positions decoded here
-    const long long cnt = (long long)((len + CH - 1) / CH) * Hkv;
-    long long incl = cnt;
+    const int nch = (len + CH - 1) / CH;
+    const long long cnt = (long long)nch * Hkv;
+    const long long cost = s < S ? (long long)(nch + alpha) * Hkv : 0;
+    long long incl_cnt = cnt, incl_cost = cost;
 #pragma unroll
     for (int off = 1; off < 32; off <<= 1) {
-      const long long y = __shfl_up_sync(FULL_MASK, incl, off);
-      if (lane >= off) incl += y;
+      const long long y = __shfl_up_sync(FULL_MASK, incl_cnt, off);
+      const long long z = __shfl_up_sync(FULL_MASK, incl_cost, off);
+      if (lane >= off) {
+        incl_cnt += y;
+        incl_cost += z;
+      }
     }
-    const long long tile_total = __shfl_sync(FULL_MASK, incl, 31);
-    if (running + tile_total > ws.g0) {
-      const bool hit = (running + incl - cnt <= ws.g0) && (ws.g0 < running + incl);
-      const int src = __ffs(__ballot_sync(FULL_MASK, hit)) - 1;
-      ws.s = base + src;
-      ws.rem = (int)(ws.g0 - running - __shfl_sync(FULL_MASK, incl - cnt, src));
-      ws.len = __shfl_sync(FULL_MASK, len, src);
-      return true;
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      if (j == 0 ? found0 : found1) continue;
+      const long long x = j == 0 ? x0 : x1;
+      // the first sequence with a chunk whose positions end after x
+      const bool hit = nch > 0 && run_cost + incl_cost > x;
+      const unsigned int hits = __ballot_sync(FULL_MASK, hit);
+      if (hits == 0u) continue;
+      const int src = __ffs(hits) - 1;
+      const long long seq_cost0 = run_cost + __shfl_sync(FULL_MASK, incl_cost - cost, src);
+      const long long seq_cnt0 = run_cnt + __shfl_sync(FULL_MASK, incl_cnt - cnt, src);
+      const int hn = __shfl_sync(FULL_MASK, nch, src);
+      const long long r = x > seq_cost0 ? x - seq_cost0 : 0;  // x may lie in an empty sequence before
+      const int kvh = (int)(r / (hn + alpha));
+      const int off = (int)(r - (long long)kvh * (hn + alpha));
+      const int rem = kvh * hn + (off < alpha ? 0 : off - alpha);
+      if (j == 0) {
+        found0 = true;
+        ws.s = base + src;
+        ws.rem = rem;
+        ws.len = __shfl_sync(FULL_MASK, len, src);
+        ws.g0 = seq_cnt0 + rem;
+      } else {
+        found1 = true;
+        c1 = seq_cnt0 + rem;
+      }
     }
-    running += tile_total;
+    run_cnt += __shfl_sync(FULL_MASK, incl_cnt, 31);
+    run_cost += __shfl_sync(FULL_MASK, incl_cost, 31);
   }
-  return false;  // not reached: g0 < C always lies in some sequence
+  if (!found0) return false;  // no chunk lies at or after this share's start
+  ws.n = c1 - ws.g0;
+  return ws.n > 0;
 }
 
 // Walks one warp's share chunk by chunk in issue order.  Every lane keeps the same state.
@@ -244,8 +281,8 @@ struct ChunkCursor {
   int start, next_start;  // first decoded position of the sequence (its shared prefix, or 0)
   long long base;  // global index of chunk 0 of the current (sequence, kv head)
   int first_worker, npieces;
-  long long issued, n, C;
-  int W, S, Hkv, max_len;
+  long long issued, n, T;
+  int W, alpha, S, Hkv, max_len;
   int blk[COPIES];
 
   __device__ __forceinline__ void fetch_blocks(const DecodeArgs &a) {
@@ -256,17 +293,21 @@ struct ChunkCursor {
     }
   }
 
+  // The warps whose shares hold the current (sequence, kv head): chunk c of pair p lies at
+  // position c + alpha * (p + 1).
   __device__ __forceinline__ void pieces() {
-    first_worker = worker_of(base, C, W);
-    npieces = worker_of(base + nch - 1, C, W) - first_worker + 1;
+    const long long shift = (long long)alpha * ((long long)s * Hkv + kvh + 1);
+    first_worker = worker_of(base + shift, T, W);
+    npieces = worker_of(base + nch - 1 + shift, T, W) - first_worker + 1;
   }
 
   __device__ __forceinline__ void init(const DecodeArgs &a, const WarpShare &ws, int max_len_) {
     S = a.num_seqs;
     Hkv = a.num_kv_heads;
     max_len = max_len_;
-    C = ws.C;
+    T = ws.T;
     W = ws.W;
+    alpha = ws.alpha;
     n = ws.n;
     issued = 0;
     s = ws.s;

@@ -248,7 +248,7 @@ __global__ void __launch_bounds__(MmaTraits<D, BS, G, (int)sizeof(KV)>::kThreads
   ShareRecord *shares = reinterpret_cast<ShareRecord *>(smem + Tr::kShareOff);
   MailEntry *mbox = reinterpret_cast<MailEntry *>(smem + Tr::kMboxOff);
   unsigned int *mcount = reinterpret_cast<unsigned int *>(smem + Tr::kMcountOff);
-  long long *step_C = reinterpret_cast<long long *>(smem + Tr::kShareOff + NW * 32);
+  long long *step_T = reinterpret_cast<long long *>(smem + Tr::kShareOff + NW * 32);
   int *step_W = reinterpret_cast<int *>(smem + Tr::kShareOff + NW * 32 + 8);
 
   // ---- set-up: barriers, then every worker finds its share and publishes it ----
@@ -276,7 +276,7 @@ __global__ void __launch_bounds__(MmaTraits<D, BS, G, (int)sizeof(KV)>::kThreads
       shares[wid] = r;
       mcount[wid] = 0u;
       if (wid == 0) {
-        *step_C = ws.C;
+        *step_T = ws.T;
         *step_W = ws.W;
       }
     }
@@ -301,7 +301,8 @@ __global__ void __launch_bounds__(MmaTraits<D, BS, G, (int)sizeof(KV)>::kThreads
       const ShareRecord r = shares[k];
       if (r.n > 0 && r.s >= 0) {
         WarpShare ws;
-        ws.C = *step_C;
+        ws.T = *step_T;
+        ws.alpha = a.piece_cost;
         ws.W = *step_W;
         ws.g0 = r.g0;
         ws.n = r.n;

@@ -45,6 +45,7 @@ struct DecodeArgs {
   int64_t num_blocks;
   float scale_log2;  // scale * log2(e): logits are kept in base-2 units
   int num_workers;   // warps sharing the work
+  int piece_cost;    // the split's cost of a (sequence, kv head) start, in chunks (see the split)
   // workspace (see pa_api.cu for the layout)
   unsigned int *counters;
   int2 *pair_meta;
