@@ -495,8 +495,17 @@ WsLayout ws_layout(int64_t S, int Hq, int Hkv, int D, int W) {
 #ifndef PA_PIECE_COST_FP8
 #define PA_PIECE_COST_FP8 3  // the same, FP8 caches
 #endif
+#ifndef PA_PIECE_COST_SHARED
+#define PA_PIECE_COST_SHARED 8  // the same, shared-prefix decode (each piece also merges the
+                                // prefix pass's partial results)
+#endif
 
-constexpr int kPrefixItemTokens = 256;  // two kv tiles of 128 positions
+#ifndef PA_PREFIX_ITEM_TOKENS
+#define PA_PREFIX_ITEM_TOKENS 256
+#endif
+// Positions of one prefix-pass item (a multiple of the prefill kernel's 128-position kv tile):
+// each item leaves one partial result per (member, query head) for the decode to merge.
+constexpr int kPrefixItemTokens = PA_PREFIX_ITEM_TOKENS;
 
 struct PrefixLayout {
   size_t pre_ml, pre_o, total;
@@ -704,7 +713,10 @@ int decode_impl(const pa_tensor *out, const pa_tensor *query, const pa_tensor *k
   // piece (query rows, partial result, ticket, merge).  Per-warp timings of the Llama-shaped
   // step put it near one chunk's time with 16-bit caches and two to three with FP8 (whose
   // chunks take less time); the settings are the fastest measured (1 vs 0 and 2; 3 vs 0 and 2).
-  const int piece_cost = k.tma_rows > 0 ? (fp8 ? PA_PIECE_COST_FP8 : PA_PIECE_COST_16) : 0;
+  const int piece_cost = k.tma_rows == 0 ? 0
+                         : shared       ? PA_PIECE_COST_SHARED
+                         : fp8          ? PA_PIECE_COST_FP8
+                                        : PA_PIECE_COST_16;
   // worker_of() multiplies a position by W in 64 bits
   const double chunks = (double)S * num_kv_heads *
                         ((double)block_tables->shape[1] * block_size / k.chunk_tokens + 1 + piece_cost);

@@ -464,24 +464,6 @@ __global__ void __launch_bounds__(PrefillTcTraits<D, BS, G>::kThreads, 1)
           set_error(a.err, t.noncausal ? PA_DEVERR_PREFIX : PA_DEVERR_CONTEXT_LEN);
         continue;
       }
-      if (t.noncausal && which == 1 && t.kvh == 0) {
-        // shared-prefix pass: the members of this tile must name the first member's prefix
-        // length and, over this item's positions, its physical blocks (kv head 0's items check)
-        const int32_t *row0 = a.block_tables + (long long)t.s * a.bt_s;
-        const int b0 = t.j0 * Tr::kKv / BS;
-        const int b1 = (min((t.j0 + t.n_kv) * Tr::kKv, t.L) + BS - 1) / BS;
-        bool bad = false;
-        for (int m = t.tok0 + lane; m < t.tok0 + t.ntok; m += 32) {
-          const int sq = t.q0 + m;
-          if (sq == t.s) continue;
-          if (__ldg(a.prefix_lens + sq) != __ldg(a.prefix_lens + t.s)) bad = true;
-          const int32_t *row = a.block_tables + (long long)sq * a.bt_s;
-          for (int b = b0; b < b1; ++b)
-            if (__ldg(row + b) != __ldg(row0 + b)) bad = true;
-        }
-        if (bad) set_error(a.err, PA_DEVERR_PREFIX);
-        if (lane == 0 && t.L % BS != 0) set_error(a.err, PA_DEVERR_PREFIX);
-      }
       if (which == 0) {
         // the tile's query rows: tokens q0 + tok0 .. + 128/G of heads kvh*G .. + G (rows past
         // the tensor read as zeros, rows of the next sequence are computed and dropped), once
@@ -560,6 +542,25 @@ __global__ void __launch_bounds__(PrefillTcTraits<D, BS, G>::kThreads, 1)
         cur = nxt;
       }
       ok = __shfl_sync(FULL_MASK, ok ? 1 : 0, 0) != 0;
+      if (t.noncausal && which == 1 && t.kvh == 0) {
+        // shared-prefix pass: the members of this tile must name the first member's prefix
+        // length and, over this item's positions, its physical blocks (kv head 0's items check,
+        // once their value copies are issued: the check only reports)
+        const int32_t *row0 = a.block_tables + (long long)t.s * a.bt_s;
+        const int b0 = t.j0 * Tr::kKv / BS;
+        const int b1 = (min((t.j0 + t.n_kv) * Tr::kKv, t.L) + BS - 1) / BS;
+        bool bad = false;
+        for (int m = t.tok0 + lane; m < t.tok0 + t.ntok; m += 32) {
+          const int sq = t.q0 + m;
+          if (sq == t.s) continue;
+          if (__ldg(a.prefix_lens + sq) != __ldg(a.prefix_lens + t.s)) bad = true;
+          const int32_t *row = a.block_tables + (long long)sq * a.bt_s;
+          for (int b = b0; b < b1; ++b)
+            if (__ldg(row + b) != __ldg(row0 + b)) bad = true;
+        }
+        if (bad) set_error(a.err, PA_DEVERR_PREFIX);
+        if (lane == 0 && t.L % BS != 0) set_error(a.err, PA_DEVERR_PREFIX);
+      }
       kv_base += t.n_kv;
     }
     if (lane == 0 && !ok) {
