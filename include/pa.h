@@ -330,9 +330,10 @@ PA_API int pa_decode(const pa_tensor *out, const pa_tensor *query, const pa_tens
 
 /*
  * pa_decode_ex - pa_decode with caller-chosen parallel split and caller-owned workspace.
- *   num_workers   number of warps that split the step's work, each taking an equal share of
- *                 the (sequence, kv head, 16-row chunk) list; 0 = one full wave of the device.
- *                 1 computes every sequence in a single warp (no merging at all).
+ *   num_workers   number of warps that split the step's work, each taking a contiguous share
+ *                 of the (sequence, kv head, 16-row chunk) list of equal cost (a chunk costs
+ *                 one, each (sequence, kv head) start a few more); 0 = one full wave of the
+ *                 device.  1 computes every sequence in a single warp (no merging at all).
  *   flags         0 or PA_DECODE_SEPARATE_REDUCE.
  *   workspace     device memory of at least pa_decode_workspace_bytes(...) bytes, 256-byte
  *                 aligned, zero-filled before its first use (pa_workspace_init).  Every call

@@ -97,6 +97,25 @@ __device__ __forceinline__ void tma_load_tile(uint32_t dst, const CUtensorMap *m
       : "memory");
 }
 
+// The same with an L2 cache policy (createpolicy): the decode streams every key and value tile
+// once, so its copies are marked evict-first and leave L2 to what the launch reads again (the
+// pieces' partial results, the block tables, the queries).
+__device__ __forceinline__ void tma_load_tile_hint(uint32_t dst, const CUtensorMap *map, int y, int z,
+                                                   int w, uint64_t *bar, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.5d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint "
+      "[%0], [%1, {%2, %3, %4, %5, %6}], [%7], %8;" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(0), "r"(y), "r"(0), "r"(z), "r"(w),
+      "r"(smem_u32(bar)), "l"(policy)
+      : "memory");
+}
+
+__device__ __forceinline__ uint64_t l2_evict_first_policy() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+
 // Prefetch one box of the 5-D cache view into L2 (no shared memory, no completion to wait for).
 __device__ __forceinline__ void tma_prefetch_tile(const CUtensorMap *map, int y, int z, int w) {
   asm volatile(
@@ -324,6 +343,7 @@ __global__ void __launch_bounds__(MmaTraits<D, BS, G, (int)sizeof(KV)>::kThreads
         }
       }
     }
+    const uint64_t stream_policy = l2_evict_first_policy();
     // One stage of this lane's worker: the chunk's key and value boxes, plus the group's query
     // rows when a new (sequence, kv head) starts, all counted on the stage's full barrier.
     auto issue = [&](int slot) {
@@ -347,9 +367,10 @@ __global__ void __launch_bounds__(MmaTraits<D, BS, G, (int)sizeof(KV)>::kThreads
             blk = 0;
           }
           const uint32_t off = c * Tr::kBoxBytes;
-          tma_load_tile(smem_u32(stage + off), &maps.k, t % BS, cur.kvh, blk, full + slot);
-          tma_load_tile(smem_u32(stage + Tr::kTileBytes + off), &maps.v, t % BS, cur.kvh, blk,
-                        full + slot);
+          tma_load_tile_hint(smem_u32(stage + off), &maps.k, t % BS, cur.kvh, blk, full + slot,
+                             stream_policy);
+          tma_load_tile_hint(smem_u32(stage + Tr::kTileBytes + off), &maps.v, t % BS, cur.kvh, blk,
+                             full + slot, stream_policy);
         }
       }
       if (new_row) {
