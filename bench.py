@@ -124,6 +124,8 @@ KERNEL_SOURCES = {
     "prefill": ("pa_prefill_tc.cuh", "pa_tc.cuh", "pa_device.cuh", "pa_prefill_internal.h",
                 "pa_prefill_bf16.cu"),
 }
+# the shared-prefix cascade: the prefill kernel's prefix pass and the decode kernel
+KERNEL_SOURCES["shared"] = tuple(sorted(set(KERNEL_SOURCES["decode"]) | set(KERNEL_SOURCES["prefill"])))
 
 
 def kernel_sources_digest(kernel: str = "decode") -> str:
@@ -911,7 +913,8 @@ def run_decode(args, b: W.PagedBatch, config: dict, rank: int = 0, world: int = 
         "pct_of_8TBs": round(100 * value / world / NOMINAL_HBM_GBS, 2),
         f"pct_of_{peak_src}_hbm": round(100 * value / world / peak, 2),
         "roofline": hbm_roofline(roof_bytes, decode_ms, kernel,
-                                 recorded_traffic(config["workload"]), probe),
+                                 recorded_traffic(config["workload"] + (":shared" if shared else ""),
+                                                  "shared" if shared else "decode"), probe),
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks,
     }
