@@ -73,6 +73,12 @@ __device__ __forceinline__ void fp8x4_to_f16x2(uint32_t w, uint32_t &lo, uint32_
       : "r"(w));
 }
 
+__device__ __forceinline__ void ldmatrix_x2(uint32_t &r0, uint32_t &r1, uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0,%1}, [%2];"
+               : "=r"(r0), "=r"(r1)
+               : "r"(addr));
+}
+
 __device__ __forceinline__ void ldmatrix_x4(uint32_t (&r)[4], uint32_t addr) {
   asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
                : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
@@ -524,6 +530,14 @@ __global__ void __launch_bounds__(MmaTraits<D, BS, G, (int)sizeof(KV)>::kThreads
   const int g = lane >> 2;  // fragment row group
   const int c = lane & 3;   // fragment column pair
   const int h0 = 2 * c, h1 = 2 * c + 1;  // heads of this lane's logits / output columns
+  // With G <= 4 the MMAs' 8 head columns have room for P's lo term: column n of P carries the
+  // hi term of head n for n < 4 and the lo term of head n - 4 for n >= 4, so one P.V MMA per V
+  // fragment does both terms.  The query columns follow (column n holds head n % 4, zero past
+  // G): lanes c and c + 2 compute the same logits, and the two halves of O are added where a
+  // piece ends.
+  constexpr bool kPackLo = G <= 4;
+  const int qh = kPackLo ? (g & 3) : g;     // query head of MMA column g
+  const bool lo_lane = kPackLo && c >= 2;  // this lane's columns hold lo terms
   const int lm = lane >> 3;  // which 8x8 matrix this lane addresses for ldmatrix
   const int lr = lane & 7;   // row within it
   uint32_t qb[Tr::kKSteps][2];
@@ -598,7 +612,7 @@ __global__ void __launch_bounds__(MmaTraits<D, BS, G, (int)sizeof(KV)>::kThreads
           const int base = 32 * (ks >> 1) + 16 * (ks & 1) + 4 * c;
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            qv[ks][e] = g < G ? Elem<T>::to_float(q[g * D + base + e]) : 0.f;
+            qv[ks][e] = qh < G ? Elem<T>::to_float(q[qh * D + base + e]) : 0.f;
             mx = fmaxf(mx, fabsf(qv[ks][e]));
           }
         }
@@ -623,9 +637,9 @@ __global__ void __launch_bounds__(MmaTraits<D, BS, G, (int)sizeof(KV)>::kThreads
       } else {
 #pragma unroll
         for (int ks = 0; ks < Tr::kKSteps; ++ks) {
-          if (g < G) {
-            qb[ks][0] = *reinterpret_cast<const uint32_t *>(qs + (g * D + 16 * ks + 2 * c) * 2);
-            qb[ks][1] = *reinterpret_cast<const uint32_t *>(qs + (g * D + 16 * ks + 8 + 2 * c) * 2);
+          if (qh < G) {
+            qb[ks][0] = *reinterpret_cast<const uint32_t *>(qs + (qh * D + 16 * ks + 2 * c) * 2);
+            qb[ks][1] = *reinterpret_cast<const uint32_t *>(qs + (qh * D + 16 * ks + 8 + 2 * c) * 2);
           } else {
             qb[ks][0] = 0u;
             qb[ks][1] = 0u;
@@ -714,7 +728,22 @@ __global__ void __launch_bounds__(MmaTraits<D, BS, G, (int)sizeof(KV)>::kThreads
     const float p2 = fast_exp2(s[2] - m0), p3 = fast_exp2(s[3] - m1);
     l0 += p0 + p2;
     l1 += p1 + p3;
-    {
+    uint32_t pf[4];  // B fragments: hi (tokens 0-7, 8-15), lo (tokens 0-7, 8-15)
+    if constexpr (kPackLo) {
+      // P transposed to [column][token]: this lane's columns take the hi or the lo terms
+      uint16_t *pb = reinterpret_cast<uint16_t *>(pbuf);
+      uint16_t hi, lo;
+      M::split(p0, hi, lo);
+      pb[h0 * 16 + g] = lo_lane ? lo : hi;
+      M::split(p1, hi, lo);
+      pb[h1 * 16 + g] = lo_lane ? lo : hi;
+      M::split(p2, hi, lo);
+      pb[h0 * 16 + g + 8] = lo_lane ? lo : hi;
+      M::split(p3, hi, lo);
+      pb[h1 * 16 + g + 8] = lo_lane ? lo : hi;
+      __syncwarp();
+      ldmatrix_x2(pf[0], pf[1], smem_u32(pbuf) + lr * 32 + (lm & 1) * 16);
+    } else {
       // P transposed to [hi|lo][head][token] for the B operand of P.V
       uint16_t *pb = reinterpret_cast<uint16_t *>(pbuf);
       uint16_t hi, lo;
@@ -730,10 +759,9 @@ __global__ void __launch_bounds__(MmaTraits<D, BS, G, (int)sizeof(KV)>::kThreads
       M::split(p3, hi, lo);
       pb[h1 * 16 + g + 8] = hi;
       pb[128 + h1 * 16 + g + 8] = lo;
+      __syncwarp();
+      ldmatrix_x4(pf, smem_u32(pbuf) + (lm >> 1) * 256 + lr * 32 + (lm & 1) * 16);
     }
-    __syncwarp();
-    uint32_t pf[4];  // B fragments: hi (tokens 0-7, 8-15), lo (tokens 0-7, 8-15)
-    ldmatrix_x4(pf, smem_u32(pbuf) + (lm >> 1) * 256 + lr * 32 + (lm & 1) * 16);
 
     // ---- P.V on tensor cores: o[mt] = O^T[dim 16mt+g | +8][head 2c | 2c+1] (FP8 caches:
     // dims 16mt+2g | 16mt+2g+1) ----
@@ -765,7 +793,7 @@ __global__ void __launch_bounds__(MmaTraits<D, BS, G, (int)sizeof(KV)>::kThreads
               if (mask_hi8) { vf[2] &= 0x0000ffffu; vf[3] &= 0x0000ffffu; }
             }
             M::mma(o[2 * mp + t2], vf, pf[0], pf[1]);
-            M::mma(o[2 * mp + t2], vf, pf[2], pf[3]);
+            if constexpr (!kPackLo) M::mma(o[2 * mp + t2], vf, pf[2], pf[3]);
           }
         }
       } else {
@@ -784,7 +812,7 @@ __global__ void __launch_bounds__(MmaTraits<D, BS, G, (int)sizeof(KV)>::kThreads
           if (mask_hi8) { vf[2] &= 0x0000ffffu; vf[3] &= 0x0000ffffu; }
         }
         M::mma(o[mt], vf, pf[0], pf[1]);
-        M::mma(o[mt], vf, pf[2], pf[3]);
+        if constexpr (!kPackLo) M::mma(o[mt], vf, pf[2], pf[3]);
       }
       }
     }
@@ -795,6 +823,13 @@ __global__ void __launch_bounds__(MmaTraits<D, BS, G, (int)sizeof(KV)>::kThreads
 
     // ---- end of a piece ----
     if (m.flags & kLast) {
+      if constexpr (kPackLo) {
+        // lane c (c < 2) adds lane c + 2's lo columns to its hi ones
+#pragma unroll
+        for (int mt = 0; mt < Tr::kMTiles; ++mt)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) o[mt][e] += __shfl_xor_sync(FULL_MASK, o[mt][e], 2);
+      }
       float t0 = l0, t1 = l1;
 #pragma unroll
       for (int off = 4; off < 32; off <<= 1) {
