@@ -44,6 +44,14 @@ struct MmaType<__nv_bfloat16> {
     hi = *reinterpret_cast<const uint16_t *>(&h);
     lo = *reinterpret_cast<const uint16_t *>(&l);
   }
+  // (x, y) -> packed hi and lo terms, x in the lower half of each
+  static __device__ __forceinline__ void split2(float x, float y, uint32_t &hi, uint32_t &lo) {
+    const __nv_bfloat162 h = __floats2bfloat162_rn(x, y);
+    const float2 hf = __bfloat1622float2(h);
+    const __nv_bfloat162 l = __floats2bfloat162_rn(x - hf.x, y - hf.y);
+    hi = *reinterpret_cast<const uint32_t *>(&h);
+    lo = *reinterpret_cast<const uint32_t *>(&l);
+  }
   static constexpr CUtensorMapDataType kTmaType = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
 };
 template <>
@@ -61,6 +69,13 @@ struct MmaType<__half> {
     hi = *reinterpret_cast<const uint16_t *>(&h);
     lo = *reinterpret_cast<const uint16_t *>(&l);
   }
+  static __device__ __forceinline__ void split2(float x, float y, uint32_t &hi, uint32_t &lo) {
+    const __half2 h = __floats2half2_rn(x, y);
+    const float2 hf = __half22float2(h);
+    const __half2 l = __floats2half2_rn(x - hf.x, y - hf.y);
+    hi = *reinterpret_cast<const uint32_t *>(&h);
+    lo = *reinterpret_cast<const uint32_t *>(&l);
+  }
   static constexpr CUtensorMapDataType kTmaType = CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
 };
 
@@ -73,10 +88,12 @@ __device__ __forceinline__ void fp8x4_to_f16x2(uint32_t w, uint32_t &lo, uint32_
       : "r"(w));
 }
 
-__device__ __forceinline__ void ldmatrix_x2(uint32_t &r0, uint32_t &r1, uint32_t addr) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0,%1}, [%2];"
-               : "=r"(r0), "=r"(r1)
-               : "r"(addr));
+// Transpose of an 8x8 matrix of 16-bit values held by the warp (lane l: row l / 4, columns
+// 2 (l % 4) and + 1, the lower column in the lower half) into the same layout.
+__device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x) {
+  uint32_t y;
+  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
+  return y;
 }
 
 __device__ __forceinline__ void ldmatrix_x4(uint32_t (&r)[4], uint32_t addr) {
@@ -187,12 +204,10 @@ struct MmaTraits {
                                         : kMaxFp8Stages;
   static constexpr int kStages = KVB == 2 ? PA_DECODE_STAGES : kFp8Stages;
   static constexpr int kRingBytes = kWorkers * kStages * kStageBytes;
-  static constexpr int kPbufBytes = 2 * 8 * 16 * 2;    // [hi, lo][8 heads][16 tokens]
   static constexpr int kMetaOff = 0;
   static constexpr int kFullOff = kStages * 32;
   static constexpr int kEmptyOff = kFullOff + kStages * 8;
-  static constexpr int kPbufOff = (kEmptyOff + kStages * 8 + 127) / 128 * 128;
-  static constexpr int kSmallBytes = kPbufOff + kPbufBytes;
+  static constexpr int kSmallBytes = (kEmptyOff + kStages * 8 + 127) / 128 * 128;
   static constexpr int kShareOff = kRingBytes + kWorkers * kSmallBytes;
   static constexpr int kMboxEntries = 4;                // split pieces (at most 2) + done
   static constexpr int kMboxOff = kShareOff + kWorkers * 32 + 16;
@@ -525,7 +540,6 @@ __global__ void __launch_bounds__(MmaTraits<D, BS, G, (int)sizeof(KV)>::kThreads
   const ChunkMeta *meta = reinterpret_cast<const ChunkMeta *>(small + Tr::kMetaOff);
   uint64_t *full = reinterpret_cast<uint64_t *>(small + Tr::kFullOff);
   uint64_t *empty = reinterpret_cast<uint64_t *>(small + Tr::kEmptyOff);
-  unsigned char *pbuf = small + Tr::kPbufOff;
 
   const int g = lane >> 2;  // fragment row group
   const int c = lane & 3;   // fragment column pair
@@ -547,9 +561,9 @@ __global__ void __launch_bounds__(MmaTraits<D, BS, G, (int)sizeof(KV)>::kThreads
   // logit scale of this lane's two heads (base 2) and the output scale (FP8 value scale)
   float sc0 = a.scale_log2, sc1 = a.scale_log2, vsc = 1.f;
 
+  int slot = 0;         // cc % ST
+  uint32_t parity = 0;  // (cc / ST) & 1
   for (long long cc = 0; cc < n; ++cc) {
-    const int slot = (int)(cc % ST);
-    const uint32_t parity = (uint32_t)((cc / ST) & 1);
     // (one verdict for the whole warp: the paths below are warp-synchronous)
     if (!__all_sync(FULL_MASK, mbar_wait_bounded(full + slot, parity, a.wait_cycles))) {
       // a copy never completed: record it, let the copies that may be in flight land, stop.
@@ -689,10 +703,10 @@ __global__ void __launch_bounds__(MmaTraits<D, BS, G, (int)sizeof(KV)>::kThreads
             M::mma(sa, af, qb[ks][0], qb[ks][1]);
         }
       }
-      s[0] = (sa[0] + sb[0]) * sc0;
-      s[1] = (sa[1] + sb[1]) * sc1;
-      s[2] = (sa[2] + sb[2]) * sc0;
-      s[3] = (sa[3] + sb[3]) * sc1;
+      s[0] = sa[0] + sb[0];  // logits before their scale
+      s[1] = sa[1] + sb[1];
+      s[2] = sa[2] + sb[2];
+      s[3] = sa[3] + sb[3];
     }
     const int tok0 = m.chunk * 16;
     const bool tail = tok0 + 16 > m.len;
@@ -701,10 +715,13 @@ __global__ void __launch_bounds__(MmaTraits<D, BS, G, (int)sizeof(KV)>::kThreads
       if (tok0 + g + 8 >= m.len) s[2] = s[3] = -INFINITY;
     }
 
-    // ---- online softmax: the reference maximum moves only when some logit passes it by
-    // more than 8 (base 2); only then are the chunk maxima gathered across lanes ----
-    float cm0 = fmaxf(s[0], s[2]), cm1 = fmaxf(s[1], s[3]);
-    if (__any_sync(FULL_MASK, (cm0 > m0 + 8.f) || (cm1 > m1 + 8.f))) {
+    // ---- online softmax in base 2: t = logit * scale - m is the exponent of a weight against
+    // the reference maximum m, which moves only when some t passes 8 (m = -inf, a piece's start,
+    // gives t = +inf); only then are the chunk maxima gathered across lanes ----
+    float t[4] = {fmaf(s[0], sc0, -m0), fmaf(s[1], sc1, -m1), fmaf(s[2], sc0, -m0),
+                  fmaf(s[3], sc1, -m1)};
+    if (__any_sync(FULL_MASK, fmaxf(t[0], t[2]) > 8.f || fmaxf(t[1], t[3]) > 8.f)) {
+      float cm0 = fmaxf(s[0] * sc0, s[2] * sc0), cm1 = fmaxf(s[1] * sc1, s[3] * sc1);
 #pragma unroll
       for (int off = 4; off < 32; off <<= 1) {
         cm0 = fmaxf(cm0, __shfl_xor_sync(FULL_MASK, cm0, off));
@@ -723,44 +740,32 @@ __global__ void __launch_bounds__(MmaTraits<D, BS, G, (int)sizeof(KV)>::kThreads
         o[mt][2] *= a0;
         o[mt][3] *= a1;
       }
+      t[0] = fmaf(s[0], sc0, -m0);
+      t[1] = fmaf(s[1], sc1, -m1);
+      t[2] = fmaf(s[2], sc0, -m0);
+      t[3] = fmaf(s[3], sc1, -m1);
     }
-    const float p0 = fast_exp2(s[0] - m0), p1 = fast_exp2(s[1] - m1);
-    const float p2 = fast_exp2(s[2] - m0), p3 = fast_exp2(s[3] - m1);
+    const float p0 = fast_exp2(t[0]), p1 = fast_exp2(t[1]);
+    const float p2 = fast_exp2(t[2]), p3 = fast_exp2(t[3]);
     l0 += p0 + p2;
     l1 += p1 + p3;
-    uint32_t pf[4];  // B fragments: hi (tokens 0-7, 8-15), lo (tokens 0-7, 8-15)
-    if constexpr (kPackLo) {
-      // P transposed to [column][token]: this lane's columns take the hi or the lo terms
-      uint16_t *pb = reinterpret_cast<uint16_t *>(pbuf);
-      uint16_t hi, lo;
-      M::split(p0, hi, lo);
-      pb[h0 * 16 + g] = lo_lane ? lo : hi;
-      M::split(p1, hi, lo);
-      pb[h1 * 16 + g] = lo_lane ? lo : hi;
-      M::split(p2, hi, lo);
-      pb[h0 * 16 + g + 8] = lo_lane ? lo : hi;
-      M::split(p3, hi, lo);
-      pb[h1 * 16 + g + 8] = lo_lane ? lo : hi;
-      __syncwarp();
-      ldmatrix_x2(pf[0], pf[1], smem_u32(pbuf) + lr * 32 + (lm & 1) * 16);
-    } else {
-      // P transposed to [hi|lo][head][token] for the B operand of P.V
-      uint16_t *pb = reinterpret_cast<uint16_t *>(pbuf);
-      uint16_t hi, lo;
-      M::split(p0, hi, lo);
-      pb[h0 * 16 + g] = hi;
-      pb[128 + h0 * 16 + g] = lo;
-      M::split(p1, hi, lo);
-      pb[h1 * 16 + g] = hi;
-      pb[128 + h1 * 16 + g] = lo;
-      M::split(p2, hi, lo);
-      pb[h0 * 16 + g + 8] = hi;
-      pb[128 + h0 * 16 + g + 8] = lo;
-      M::split(p3, hi, lo);
-      pb[h1 * 16 + g + 8] = hi;
-      pb[128 + h1 * 16 + g + 8] = lo;
-      __syncwarp();
-      ldmatrix_x4(pf, smem_u32(pbuf) + (lm >> 1) * 256 + lr * 32 + (lm & 1) * 16);
+    // P as the B operand of P.V, in registers: each lane packs its two columns of token rows g
+    // and g + 8 (a C fragment), and movmatrix transposes each 8x8 block into the B fragment
+    // (tokens 2c, 2c+1 | 2c+8, 2c+9 of column g)
+    uint32_t pf[4];  // hi (tokens 0-7, 8-15), lo (tokens 0-7, 8-15); with kPackLo pf[0..1] only
+    {
+      uint32_t h01, l01, h23, l23;
+      M::split2(p0, p1, h01, l01);
+      M::split2(p2, p3, h23, l23);
+      if constexpr (kPackLo) {
+        pf[0] = movmatrix_trans(lo_lane ? l01 : h01);
+        pf[1] = movmatrix_trans(lo_lane ? l23 : h23);
+      } else {
+        pf[0] = movmatrix_trans(h01);
+        pf[1] = movmatrix_trans(h23);
+        pf[2] = movmatrix_trans(l01);
+        pf[3] = movmatrix_trans(l23);
+      }
     }
 
     // ---- P.V on tensor cores: o[mt] = O^T[dim 16mt+g | +8][head 2c | 2c+1] (FP8 caches:
@@ -925,6 +930,10 @@ __global__ void __launch_bounds__(MmaTraits<D, BS, G, (int)sizeof(KV)>::kThreads
           }
         }
       }
+    }
+    if (++slot == ST) {
+      slot = 0;
+      parity ^= 1u;
     }
   }
   // the loop's registers are free here: the merge takes its large rounds
