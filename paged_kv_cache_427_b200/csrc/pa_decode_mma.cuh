@@ -769,12 +769,17 @@ __global__ void __launch_bounds__(MmaTraits<D, BS, G, (int)sizeof(KV)>::kThreads
     }
 
     // ---- P.V on tensor cores: o[mt] = O^T[dim 16mt+g | +8][head 2c | 2c+1] (FP8 caches:
-    // dims 16mt+2g | 16mt+2g+1) ----
-    {
-      const bool mask_lo = tail && (tok0 + 2 * c >= m.len);
-      const bool mask_hi = tail && (tok0 + 2 * c + 1 >= m.len);
-      const bool mask_lo8 = tail && (tok0 + 2 * c + 8 >= m.len);
-      const bool mask_hi8 = tail && (tok0 + 2 * c + 9 >= m.len);
+    // dims 16mt+2g | 16mt+2g+1).  Value rows past the context may hold anything (NaN included)
+    // and are zeroed: only a sequence's last chunk has such rows, so that case has its own copy
+    // of the loop and the others carry no masking ----
+    auto pv = [&](auto masked) {
+      constexpr bool kMasked = decltype(masked)::value;
+      // tokens 2c, 2c+1 (the halves of vf[0], vf[1]) and 2c+8, 2c+9 (vf[2], vf[3])
+      uint32_t m01 = 0xffffffffu, m89 = 0xffffffffu;
+      if constexpr (kMasked) {
+        m01 = (tok0 + 2 * c >= m.len ? 0u : 0x0000ffffu) | (tok0 + 2 * c + 1 >= m.len ? 0u : 0xffff0000u);
+        m89 = (tok0 + 2 * c + 8 >= m.len ? 0u : 0x0000ffffu) | (tok0 + 2 * c + 9 >= m.len ? 0u : 0xffff0000u);
+      }
       if constexpr (kFp8) {
         // ldmatrix.trans of 16-bit pairs: matrix j (tokens 8(j&1).., 16-byte chunk 2mp + (j>>1))
         // gives each lane tokens 2c, 2c+1 of dims 2g, 2g+1; a byte permute regroups them by dim
@@ -791,36 +796,39 @@ __global__ void __launch_bounds__(MmaTraits<D, BS, G, (int)sizeof(KV)>::kThreads
             uint32_t vf[4];
             fp8x4_to_f16x2(__byte_perm(r[2 * t2], 0u, 0x3120u), vf[0], vf[1]);
             fp8x4_to_f16x2(__byte_perm(r[2 * t2 + 1], 0u, 0x3120u), vf[2], vf[3]);
-            if (tail) {
-              if (mask_lo) { vf[0] &= 0xffff0000u; vf[1] &= 0xffff0000u; }
-              if (mask_hi) { vf[0] &= 0x0000ffffu; vf[1] &= 0x0000ffffu; }
-              if (mask_lo8) { vf[2] &= 0xffff0000u; vf[3] &= 0xffff0000u; }
-              if (mask_hi8) { vf[2] &= 0x0000ffffu; vf[3] &= 0x0000ffffu; }
+            if constexpr (kMasked) {
+              vf[0] &= m01;
+              vf[1] &= m01;
+              vf[2] &= m89;
+              vf[3] &= m89;
             }
             M::mma(o[2 * mp + t2], vf, pf[0], pf[1]);
             if constexpr (!kPackLo) M::mma(o[2 * mp + t2], vf, pf[2], pf[3]);
           }
         }
       } else {
-      const int row = ((lm >> 1) << 3) | lr;  // token row of the V tile
+        const int row = ((lm >> 1) << 3) | lr;  // token row of the V tile
 #pragma unroll
-      for (int mt = 0; mt < Tr::kMTiles; ++mt) {
-        const int c16g = (mt << 1) | (lm & 1);
-        const uint32_t addr = vbase + tile_offset<Tr>(row, c16g >> 3) + (((c16g & 7) ^ lr) << 4);
-        uint32_t vf[4];
-        ldmatrix_x4_trans(vf, addr);
-        if (tail) {
-          // rows past the context may hold anything (NaN included): zero them
-          if (mask_lo) { vf[0] &= 0xffff0000u; vf[1] &= 0xffff0000u; }
-          if (mask_hi) { vf[0] &= 0x0000ffffu; vf[1] &= 0x0000ffffu; }
-          if (mask_lo8) { vf[2] &= 0xffff0000u; vf[3] &= 0xffff0000u; }
-          if (mask_hi8) { vf[2] &= 0x0000ffffu; vf[3] &= 0x0000ffffu; }
+        for (int mt = 0; mt < Tr::kMTiles; ++mt) {
+          const int c16g = (mt << 1) | (lm & 1);
+          const uint32_t addr = vbase + tile_offset<Tr>(row, c16g >> 3) + (((c16g & 7) ^ lr) << 4);
+          uint32_t vf[4];
+          ldmatrix_x4_trans(vf, addr);
+          if constexpr (kMasked) {
+            vf[0] &= m01;
+            vf[1] &= m01;
+            vf[2] &= m89;
+            vf[3] &= m89;
+          }
+          M::mma(o[mt], vf, pf[0], pf[1]);
+          if constexpr (!kPackLo) M::mma(o[mt], vf, pf[2], pf[3]);
         }
-        M::mma(o[mt], vf, pf[0], pf[1]);
-        if constexpr (!kPackLo) M::mma(o[mt], vf, pf[2], pf[3]);
       }
-      }
-    }
+    };
+    if (tail)
+      pv(std::true_type{});
+    else
+      pv(std::false_type{});
     // the stage is no longer needed: hand it back to the producer
     __syncwarp();
     if (lane == 0) mbar_arrive(empty + slot);
