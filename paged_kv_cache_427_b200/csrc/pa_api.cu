@@ -678,6 +678,10 @@ int decode_impl(const pa_tensor *out, const pa_tensor *query, const pa_tensor *k
       return fail(PA_ERR_UNSUPPORTED, "shared prefixes are built for bf16 and fp16 caches");
     if (group_start->shape[0] - 1 > 0x7fffffff) return fail(PA_ERR_SHAPE, "too many groups");
   }
+  // a worker counts its share's chunks in 32 bits: at most 2e9 chunks of 16 positions a step
+  // (counting each (sequence, kv head) start at the largest piece cost)
+  if ((double)S * num_kv_heads * ((double)block_tables->shape[1] * block_size / 16 + 1 + PA_PIECE_COST_SHARED) > 2.0e9)
+    return fail(PA_ERR_SHAPE, "step too large for the work split");
   if (S == 0 || mode == CallMode::kHostChecks) return PA_OK;
   DeviceState *ds;
   int dev;
@@ -717,10 +721,11 @@ int decode_impl(const pa_tensor *out, const pa_tensor *query, const pa_tensor *k
                          : shared       ? PA_PIECE_COST_SHARED
                          : fp8          ? PA_PIECE_COST_FP8
                                         : PA_PIECE_COST_16;
-  // worker_of() multiplies a position by W in 64 bits
+  // worker_of() multiplies a position by W in 64 bits; a worker counts its share's chunks in 32
   const double chunks = (double)S * num_kv_heads *
                         ((double)block_tables->shape[1] * block_size / k.chunk_tokens + 1 + piece_cost);
-  if (chunks * (double)W > 4.0e18) return fail(PA_ERR_SHAPE, "step too large for the work split");
+  if (chunks * (double)W > 4.0e18 || chunks > 2.0e9)
+    return fail(PA_ERR_SHAPE, "step too large for the work split");
   const WsLayout L = ws_layout(S, (int)Hq, num_kv_heads, D, W);
   const PrefixLayout PL = prefix_layout(L.total, S, (int)Hq, D, block_tables->shape[1], block_size);
   const size_t need = shared ? PL.total : L.total;

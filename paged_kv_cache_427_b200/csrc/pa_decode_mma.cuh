@@ -52,6 +52,12 @@ struct MmaType<__nv_bfloat16> {
     hi = *reinterpret_cast<const uint32_t *>(&h);
     lo = *reinterpret_cast<const uint32_t *>(&l);
   }
+  static __device__ __forceinline__ uint32_t term2(float x, float y, float sel) {
+    const __nv_bfloat162 h = __floats2bfloat162_rn(x, y);
+    const float2 hf = __bfloat1622float2(h);
+    const __nv_bfloat162 r = __floats2bfloat162_rn(fmaf(-sel, hf.x, x), fmaf(-sel, hf.y, y));
+    return *reinterpret_cast<const uint32_t *>(&r);
+  }
   static constexpr CUtensorMapDataType kTmaType = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
 };
 template <>
@@ -75,6 +81,13 @@ struct MmaType<__half> {
     const __half2 l = __floats2half2_rn(x - hf.x, y - hf.y);
     hi = *reinterpret_cast<const uint32_t *>(&h);
     lo = *reinterpret_cast<const uint32_t *>(&l);
+  }
+  // (x, y) -> their packed hi terms (sel = 0) or lo terms (sel = 1), as split2 gives them
+  static __device__ __forceinline__ uint32_t term2(float x, float y, float sel) {
+    const __half2 h = __floats2half2_rn(x, y);
+    const float2 hf = __half22float2(h);
+    const __half2 r = __floats2half2_rn(fmaf(-sel, hf.x, x), fmaf(-sel, hf.y, y));
+    return *reinterpret_cast<const uint32_t *>(&r);
   }
   static constexpr CUtensorMapDataType kTmaType = CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
 };
@@ -535,6 +548,7 @@ __global__ void __launch_bounds__(MmaTraits<D, BS, G, (int)sizeof(KV)>::kThreads
     return;
   }
   const long long n = share.n;
+  const int ni = (int)n;  // below 2^31: the host bounds a step's chunks
   unsigned char *ring = smem + wid * ST * Tr::kStageBytes;
   unsigned char *small = smem + Tr::kRingBytes + wid * Tr::kSmallBytes;
   const ChunkMeta *meta = reinterpret_cast<const ChunkMeta *>(small + Tr::kMetaOff);
@@ -551,7 +565,7 @@ __global__ void __launch_bounds__(MmaTraits<D, BS, G, (int)sizeof(KV)>::kThreads
   // piece ends.
   constexpr bool kPackLo = G <= 4;
   const int qh = kPackLo ? (g & 3) : g;     // query head of MMA column g
-  const bool lo_lane = kPackLo && c >= 2;  // this lane's columns hold lo terms
+  const float lo_sel = (kPackLo && c >= 2) ? 1.f : 0.f;  // this lane's columns hold lo terms
   const int lm = lane >> 3;  // which 8x8 matrix this lane addresses for ldmatrix
   const int lr = lane & 7;   // row within it
   uint32_t qb[Tr::kKSteps][2];
@@ -563,7 +577,7 @@ __global__ void __launch_bounds__(MmaTraits<D, BS, G, (int)sizeof(KV)>::kThreads
 
   int slot = 0;         // cc % ST
   uint32_t parity = 0;  // (cc / ST) & 1
-  for (long long cc = 0; cc < n; ++cc) {
+  for (int cc = 0; cc < ni; ++cc) {
     // (one verdict for the whole warp: the paths below are warp-synchronous)
     if (!__all_sync(FULL_MASK, mbar_wait_bounded(full + slot, parity, a.wait_cycles))) {
       // a copy never completed: record it, let the copies that may be in flight land, stop.
@@ -753,19 +767,17 @@ __global__ void __launch_bounds__(MmaTraits<D, BS, G, (int)sizeof(KV)>::kThreads
     // and g + 8 (a C fragment), and movmatrix transposes each 8x8 block into the B fragment
     // (tokens 2c, 2c+1 | 2c+8, 2c+9 of column g)
     uint32_t pf[4];  // hi (tokens 0-7, 8-15), lo (tokens 0-7, 8-15); with kPackLo pf[0..1] only
-    {
+    if constexpr (kPackLo) {
+      pf[0] = movmatrix_trans(M::term2(p0, p1, lo_sel));
+      pf[1] = movmatrix_trans(M::term2(p2, p3, lo_sel));
+    } else {
       uint32_t h01, l01, h23, l23;
       M::split2(p0, p1, h01, l01);
       M::split2(p2, p3, h23, l23);
-      if constexpr (kPackLo) {
-        pf[0] = movmatrix_trans(lo_lane ? l01 : h01);
-        pf[1] = movmatrix_trans(lo_lane ? l23 : h23);
-      } else {
-        pf[0] = movmatrix_trans(h01);
-        pf[1] = movmatrix_trans(h23);
-        pf[2] = movmatrix_trans(l01);
-        pf[3] = movmatrix_trans(l23);
-      }
+      pf[0] = movmatrix_trans(h01);
+      pf[1] = movmatrix_trans(h23);
+      pf[2] = movmatrix_trans(l01);
+      pf[3] = movmatrix_trans(l23);
     }
 
     // ---- P.V on tensor cores: o[mt] = O^T[dim 16mt+g | +8][head 2c | 2c+1] (FP8 caches:
@@ -832,7 +844,7 @@ __global__ void __launch_bounds__(MmaTraits<D, BS, G, (int)sizeof(KV)>::kThreads
     // the stage is no longer needed: hand it back to the producer
     __syncwarp();
     if (lane == 0) mbar_arrive(empty + slot);
-    if (tl && cc == n - 1) tl[kTlLast] = global_ns();
+    if (tl && cc == ni - 1) tl[kTlLast] = global_ns();
 
     // ---- end of a piece ----
     if (m.flags & kLast) {
@@ -923,7 +935,7 @@ __global__ void __launch_bounds__(MmaTraits<D, BS, G, (int)sizeof(KV)>::kThreads
           p.npieces = m.npieces;
           p.s = m.s;
           p.kvh = m.kvh;
-          if (cc == n - 1) {
+          if (cc == ni - 1) {
             // the share's last piece: published after the loop (nothing is left to overlap it
             // with), by this warp, so the four workers publish their last pieces in parallel
             // rather than through one merge warp

@@ -148,6 +148,17 @@ def test_decode_rejects_mismatches(lib):
     assert _decode(lib, e) == -2                 # one context length per sequence
 
 
+def test_decode_rejects_a_step_too_large_for_the_work_split(lib):
+    # 16 sequences x 2 kv heads x 2^31 - 16 positions: 2^32 chunks of 16 positions, past the
+    # 2e9 a worker's 32-bit chunk count allows (each table alone is within its own bound)
+    mb = (2**31 - 16) // 16
+    a = _decode_args(S=16, Hq=4, Hkv=2, MB=mb)
+    assert _decode(lib, a) == -2
+    assert "too large" in pa.pa_last_error()
+    ok = _decode_args(S=16, Hq=4, Hkv=2, MB=mb // 64)  # 2^26 chunks: passes this check
+    assert _decode(lib, ok) != -2
+
+
 def test_zero_sequences_is_a_no_op(lib):
     a = _decode_args(S=0)
     assert _decode(lib, a) == 0
