@@ -638,9 +638,12 @@ __global__ void __launch_bounds__(MmaTraits<D, BS, G, (int)sizeof(KV)>::kThreads
 #pragma unroll
         for (int ks = 0; ks < Tr::kKSteps; ++ks) {
           const int base = 32 * (ks >> 1) + 16 * (ks & 1) + 4 * c;
+          // the 4 dims in one 8-byte load
+          const uint2 u = qh < G ? *reinterpret_cast<const uint2 *>(q + qh * D + base) : make_uint2(0u, 0u);
+          const T *e4 = reinterpret_cast<const T *>(&u);
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            qv[ks][e] = qh < G ? Elem<T>::to_float(q[qh * D + base + e]) : 0.f;
+            qv[ks][e] = Elem<T>::to_float(e4[e]);
             mx = fmaxf(mx, fabsf(qv[ks][e]));
           }
         }
@@ -875,37 +878,39 @@ __global__ void __launch_bounds__(MmaTraits<D, BS, G, (int)sizeof(KV)>::kThreads
         char *row0 = static_cast<char *>(a.out) +
                      ((long long)m.s * a.out_s + (long long)(m.kvh * G + h0) * a.out_h) * out_elt;
         char *row1 = row0 + (long long)a.out_h * out_elt;
+        // dims d0, d1 of one output row: adjacent with FP8 caches (one 8- or 4-byte store)
+        auto put = [&](char *row, int d0, int d1, float x, float y) {
+          if (a.out_dtype == PA_F32) {
+            float *r = reinterpret_cast<float *>(row);
+            if constexpr (kFp8) {
+              *reinterpret_cast<float2 *>(r + d0) = make_float2(x, y);
+            } else {
+              r[d0] = x;
+              r[d1] = y;
+            }
+          } else if (a.out_dtype == PA_BF16) {
+            __nv_bfloat16 *r = reinterpret_cast<__nv_bfloat16 *>(row);
+            if constexpr (kFp8) {
+              *reinterpret_cast<__nv_bfloat162 *>(r + d0) = __floats2bfloat162_rn(x, y);
+            } else {
+              r[d0] = __float2bfloat16_rn(x);
+              r[d1] = __float2bfloat16_rn(y);
+            }
+          } else {
+            __half *r = reinterpret_cast<__half *>(row);
+            if constexpr (kFp8) {
+              *reinterpret_cast<__half2 *>(r + d0) = __floats2half2_rn(x, y);
+            } else {
+              r[d0] = __float2half_rn(x);
+              r[d1] = __float2half_rn(y);
+            }
+          }
+        };
 #pragma unroll
         for (int mt = 0; mt < Tr::kMTiles; ++mt) {
           const int d0 = kFp8 ? 16 * mt + 2 * g : 16 * mt + g, d1 = kFp8 ? d0 + 1 : d0 + 8;
-          if (a.out_dtype == PA_F32) {
-            if (h0 < G) {
-              reinterpret_cast<float *>(row0)[d0] = o[mt][0] * inv0;
-              reinterpret_cast<float *>(row0)[d1] = o[mt][2] * inv0;
-            }
-            if (h1 < G) {
-              reinterpret_cast<float *>(row1)[d0] = o[mt][1] * inv1;
-              reinterpret_cast<float *>(row1)[d1] = o[mt][3] * inv1;
-            }
-          } else if (a.out_dtype == PA_BF16) {
-            if (h0 < G) {
-              reinterpret_cast<__nv_bfloat16 *>(row0)[d0] = __float2bfloat16_rn(o[mt][0] * inv0);
-              reinterpret_cast<__nv_bfloat16 *>(row0)[d1] = __float2bfloat16_rn(o[mt][2] * inv0);
-            }
-            if (h1 < G) {
-              reinterpret_cast<__nv_bfloat16 *>(row1)[d0] = __float2bfloat16_rn(o[mt][1] * inv1);
-              reinterpret_cast<__nv_bfloat16 *>(row1)[d1] = __float2bfloat16_rn(o[mt][3] * inv1);
-            }
-          } else {
-            if (h0 < G) {
-              reinterpret_cast<__half *>(row0)[d0] = __float2half_rn(o[mt][0] * inv0);
-              reinterpret_cast<__half *>(row0)[d1] = __float2half_rn(o[mt][2] * inv0);
-            }
-            if (h1 < G) {
-              reinterpret_cast<__half *>(row1)[d0] = __float2half_rn(o[mt][1] * inv1);
-              reinterpret_cast<__half *>(row1)[d1] = __float2half_rn(o[mt][3] * inv1);
-            }
-          }
+          if (h0 < G) put(row0, d0, d1, o[mt][0] * inv0, o[mt][2] * inv0);
+          if (h1 < G) put(row1, d0, d1, o[mt][1] * inv1, o[mt][3] * inv1);
         }
       } else {
         const long long seg = (long long)m.pair + gw;
@@ -915,13 +920,18 @@ __global__ void __launch_bounds__(MmaTraits<D, BS, G, (int)sizeof(KV)>::kThreads
 #pragma unroll
         for (int mt = 0; mt < Tr::kMTiles; ++mt) {
           const int d0 = kFp8 ? 16 * mt + 2 * g : 16 * mt + g, d1 = kFp8 ? d0 + 1 : d0 + 8;
-          if (h0 < G) {
-            o0[d0] = o[mt][0] * inv0;
-            o0[d1] = o[mt][2] * inv0;
-          }
-          if (h1 < G) {
-            o1[d0] = o[mt][1] * inv1;
-            o1[d1] = o[mt][3] * inv1;
+          if constexpr (kFp8) {
+            if (h0 < G) *reinterpret_cast<float2 *>(o0 + d0) = make_float2(o[mt][0] * inv0, o[mt][2] * inv0);
+            if (h1 < G) *reinterpret_cast<float2 *>(o1 + d0) = make_float2(o[mt][1] * inv1, o[mt][3] * inv1);
+          } else {
+            if (h0 < G) {
+              o0[d0] = o[mt][0] * inv0;
+              o0[d1] = o[mt][2] * inv0;
+            }
+            if (h1 < G) {
+              o1[d0] = o[mt][1] * inv1;
+              o1[d1] = o[mt][3] * inv1;
+            }
           }
         }
         if (g == 0) {
