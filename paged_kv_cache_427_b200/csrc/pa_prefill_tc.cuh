@@ -688,7 +688,11 @@ __global__ void __launch_bounds__(PrefillTcTraits<D, BS, G>::kThreads, 1)
         // t = logit * scale_log2 + nm on the visible columns (-inf elsewhere); returns the
         // largest t; with exps leaves 2^t as two 16-bit terms in hw / lw, their sum in l_t
         uint32_t hw[Tr::kCols / 2], lw[Tr::kCols / 2];
-        auto pass = [&](float nm, bool exps, float &l_t) -> float {
+        // Only kv tiles that reach past a row's position need the causal mask; when every row
+        // of the warp sees all of its columns the pass runs without it
+        const bool unmasked = __all_sync(FULL_MASK, c_lim >= Tr::kCols - 1);
+        auto pass_as = [&](auto masked, float nm, bool exps, float &l_t) -> float {
+          constexpr bool kMasked = decltype(masked)::value;
           float tmax = -INFINITY;
           l_t = 0.f;
 #pragma unroll
@@ -699,8 +703,12 @@ __global__ void __launch_bounds__(PrefillTcTraits<D, BS, G>::kThreads, 1)
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
               const int c0 = 32 * q + 2 * i;
-              const float t0 = c0 <= c_lim ? fmaf(__uint_as_float(sr[2 * i]), a.scale_log2, nm) : -INFINITY;
-              const float t1 = c0 + 1 <= c_lim ? fmaf(__uint_as_float(sr[2 * i + 1]), a.scale_log2, nm) : -INFINITY;
+              float t0 = fmaf(__uint_as_float(sr[2 * i]), a.scale_log2, nm);
+              float t1 = fmaf(__uint_as_float(sr[2 * i + 1]), a.scale_log2, nm);
+              if constexpr (kMasked) {
+                t0 = c0 <= c_lim ? t0 : -INFINITY;
+                t1 = c0 + 1 <= c_lim ? t1 : -INFINITY;
+              }
               tmax = fmaxf(tmax, fmaxf(t0, t1));
               if (exps) {
                 const float p0 = fast_exp2(t0), p1 = fast_exp2(t1);
@@ -710,6 +718,9 @@ __global__ void __launch_bounds__(PrefillTcTraits<D, BS, G>::kThreads, 1)
             }
           }
           return tmax;
+        };
+        auto pass = [&](float nm, bool exps, float &l_t) -> float {
+          return unmasked ? pass_as(std::false_type{}, nm, exps, l_t) : pass_as(std::true_type{}, nm, exps, l_t);
         };
         // the row's largest t over both halves
         auto row_max = [&](float mine_t, float &both) -> bool {
