@@ -525,18 +525,39 @@ PrefixLayout prefix_layout(size_t start, int64_t S, int Hq, int D, int64_t max_b
   return P;
 }
 
+#ifndef PA_PREFIX_SM_DIVISOR
+#define PA_PREFIX_SM_DIVISOR 1
+#endif
+// The prefix pass runs on at most 1/PA_PREFIX_SM_DIVISOR of the SMs (its persistent CTAs take
+// the items in rounds); the decode, launched to overlap it, streams the suffixes on whatever SMs
+// are free and waits for the pass only to merge.  Each item is a chain of dependent hand-offs,
+// so fewer CTAs lengthen the pass more than the decode gains: on the 128-sequence shared-prefix
+// batch the cascade took 64.0 us with every SM, 69.1 / 75.5 / 94.2 us with a third, a quarter,
+// a sixth (the decode then sized to the SMs left).
+int prefix_pass_ctas(int64_t S, int64_t NG, int num_kv_heads, int splits, int tokens_per_tile,
+                     int num_sms) {
+  if (NG <= 0) return 0;
+  const int64_t items = ((S + tokens_per_tile - 1) / tokens_per_tile + NG) * num_kv_heads * (int64_t)splits;
+  int64_t cap = num_sms / PA_PREFIX_SM_DIVISOR;
+  if (cap < 1) cap = 1;
+  return (int)(items < cap ? items : cap);
+}
+
+bool prefix_pass_kernel(const CacheShape &cs, int D, int G, int block_size, pa::PrefillKernel *k) {
+  return cs.dtype == PA_BF16 ? pa::prefill_kernel_bf16(D, block_size, G, k)
+                             : pa::prefill_kernel_f16(D, block_size, G, k);
+}
+
 // The prefix pass of pa_decode_shared_prefix: the prefill kernel over every group's members
 // (their decode queries as consecutive query rows) and its shared prefix, storing partial
-// results for the decode to merge.
+// results for the decode to merge, on `ctas` persistent CTAs.
 int launch_prefix_pass(const pa::DecodeArgs &d, const pa_tensor *query, const pa_tensor *key_cache,
                        const pa_tensor *value_cache, const pa_tensor *group_start,
-                       const CacheShape &cs, int D, int G, int block_size, DeviceState *ds,
+                       const CacheShape &cs, int D, int G, int block_size, int ctas,
                        cudaStream_t st) {
   int rc;
   pa::PrefillKernel k;
-  const bool got = cs.dtype == PA_BF16 ? pa::prefill_kernel_bf16(D, block_size, G, &k)
-                                       : pa::prefill_kernel_f16(D, block_size, G, &k);
-  if (!got)
+  if (!prefix_pass_kernel(cs, D, G, block_size, &k))
     return fail(PA_ERR_CUDA, "could not prepare the prefix pass: %s", cudaGetErrorString(cudaGetLastError()));
   pa::PrefillMaps maps;
   const pa_tensor *kc = key_cache, *vc = value_cache;
@@ -547,19 +568,7 @@ int launch_prefix_pass(const pa::DecodeArgs &d, const pa_tensor *query, const pa
     return rc;
   const int64_t S = d.num_seqs;
   const int64_t NG = group_start->shape[0] - 1;
-  if (NG <= 0) return PA_OK;
-  // items: every row tile of every group, for every kv head and prefix item (a bound: the
-  // groups' sizes and prefixes are device values)
-  const int64_t items = ((S + k.tokens_per_tile - 1) / k.tokens_per_tile + NG) * d.num_kv_heads *
-                        (int64_t)d.pre_splits;
-  int per_sm = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k.kernel, k.threads_per_cta,
-                                                    k.smem_bytes) != cudaSuccess || per_sm < 1) {
-    cudaGetLastError();
-    per_sm = 1;
-  }
-  const int64_t wave = (int64_t)per_sm * ds->num_sms;
-  const int ctas = (int)(items < wave ? items : wave);
+  if (NG <= 0 || ctas <= 0) return PA_OK;
   pa::PrefillArgs a = {};
   a.out = nullptr;
   a.out_dtype = PA_F32;
@@ -712,7 +721,20 @@ int decode_impl(const pa_tensor *out, const pa_tensor *query, const pa_tensor *k
     if ((rc = cache_map(key_cache, k.tma_rows, &maps.k)) || (rc = cache_map(value_cache, k.tma_rows, &maps.v)))
       return rc;
   }
-  const int W = num_workers > 0 ? num_workers : default_workers(k, ds->num_sms);
+  // shared prefixes: the SMs the prefix pass leaves to the decode
+  int prefix_ctas = 0;
+  if (shared) {
+    pa::PrefillKernel pk;
+    if (!prefix_pass_kernel(cs, D, G, block_size, &pk))
+      return fail(PA_ERR_CUDA, "could not prepare the prefix pass: %s", cudaGetErrorString(cudaGetLastError()));
+    const int64_t max_len = block_tables->shape[1] * block_size;
+    const int splits = (int)((max_len + kPrefixItemTokens - 1) / kPrefixItemTokens);
+    prefix_ctas = prefix_pass_ctas(S, group_start->shape[0] - 1, num_kv_heads, splits < 1 ? 1 : splits,
+                                   pk.tokens_per_tile, ds->num_sms);
+  }
+  // (the decode is sized to the SMs left when the pass takes at most half of them)
+  const int decode_sms = k.tma_rows > 0 && 2 * prefix_ctas <= ds->num_sms ? ds->num_sms - prefix_ctas : ds->num_sms;
+  const int W = num_workers > 0 ? num_workers : default_workers(k, decode_sms);
   // The split's cost of a (sequence, kv head) start, in chunks: what a warp spends once per
   // piece (query rows, partial result, ticket, merge).  Per-warp timings of the Llama-shaped
   // step put it near one chunk's time with 16-bit caches and two to three with FP8 (whose
@@ -827,9 +849,12 @@ int decode_impl(const pa_tensor *out, const pa_tensor *query, const pa_tensor *k
     a.pre_splits = PL.splits;
     a.pre_kv_tokens = kPrefixItemTokens;
     if ((rc = launch_prefix_pass(a, query, key_cache, value_cache, group_start, cs, D, G,
-                                 block_size, ds, st)))
+                                 block_size, prefix_ctas, st)))
       return rc;
-    overlap = true;  // the decode's prologue runs while the prefix pass finishes
+    overlap = true;  // the decode runs while the prefix pass does
+    // the tensor-core decode streams at once (the pass is stream-ordered after the caches'
+    // writers) and waits for the pass only before merging its partial results
+    a.prefix_overlap = k.tma_rows > 0 ? 1 : 0;
   }
   const int ctas = (W + k.warps_per_cta - 1) / k.warps_per_cta;  // warps_per_cta workers each
   cudaError_t e = k.launch(a, &maps, ctas, overlap, st);

@@ -550,8 +550,9 @@ __device__ __forceinline__ void take_ticket(const DecodeArgs &a, const PieceInfo
   if (ticket == (unsigned int)(p.npieces - 1)) {
     if (!PA_TICKET_ACQREL) __threadfence();
     __syncwarp();
-    merge_pieces<G, D>(a, p.pair, p.first_worker, p.npieces, p.s, p.kvh, lane,
-                       prefix_pieces<BS>(a, p.s, a.max_blocks * BS));
+    const int npre = prefix_pieces<BS>(a, p.s, a.max_blocks * BS);
+    if (npre > 0) wait_for_previous_grid();  // the prefix pass's partial results are complete
+    merge_pieces<G, D>(a, p.pair, p.first_worker, p.npieces, p.s, p.kvh, lane, npre);
     if (lane == 0 && p.npieces > 1) a.counters[p.pair] = 0u;
   }
 }
@@ -571,8 +572,9 @@ __device__ __forceinline__ void finish_piece(const DecodeArgs &a, const ChunkMet
   if (ticket == others) {
     if (!PA_TICKET_ACQREL) __threadfence();
     __syncwarp();
-    merge_pieces<G, D, U>(a, m.pair, m.first_worker, m.npieces, m.s, m.kvh, lane,
-                          prefix_pieces<BS>(a, m.s, a.max_blocks * BS));
+    const int npre = prefix_pieces<BS>(a, m.s, a.max_blocks * BS);
+    if (npre > 0) wait_for_previous_grid();  // the prefix pass's partial results are complete
+    merge_pieces<G, D, U>(a, m.pair, m.first_worker, m.npieces, m.s, m.kvh, lane, npre);
     if (lane == 0 && others > 0) a.counters[m.pair] = 0u;
   }
 }

@@ -438,8 +438,9 @@ __global__ void __launch_bounds__(MmaTraits<D, BS, G, (int)sizeof(KV)>::kThreads
     // A grid launched after this one (the separate merge) may start now and wait for us.
     if (lane == 0) allow_next_grid();
     // Everything above read only context_lens and block_tables; the caches and the query may
-    // still be written by the previous grid when this one was launched to overlap it.
-    wait_for_previous_grid();
+    // still be written by the previous grid when this one was launched to overlap it (not when
+    // that grid is the shared-prefix pass: see prefix_overlap).
+    if (!a.prefix_overlap) wait_for_previous_grid();
     if (a.timeline != nullptr && k < NW && blockIdx.x * NW + k < a.timeline_warps)
       a.timeline[(long long)(blockIdx.x * NW + k) * kTimelineWords + kTlIssue] = global_ns();
     long long last_progress = clock64();
@@ -463,6 +464,7 @@ __global__ void __launch_bounds__(MmaTraits<D, BS, G, (int)sizeof(KV)>::kThreads
         __nanosleep(64);
       }
     }
+    if (a.prefix_overlap) wait_for_previous_grid();  // this grid completes after the prefix pass
     return;
   }
 
@@ -470,8 +472,8 @@ __global__ void __launch_bounds__(MmaTraits<D, BS, G, (int)sizeof(KV)>::kThreads
     // ================================ merge warp ================================
     // First, once the grid before this one (when it was launched to overlap it) has finished:
     // the out rows of empty contexts are zeroed, and in a fused decode step this grid's share
-    // of the step's cache write is done.
-    wait_for_previous_grid();
+    // of the step's cache write is done.  The shared-prefix pass writes neither.
+    if (!a.prefix_overlap || a.fused) wait_for_previous_grid();
     {
       const int launched_lanes = gridDim.x * 32;
       const int out_elt = a.out_dtype == PA_F32 ? 4 : 2;

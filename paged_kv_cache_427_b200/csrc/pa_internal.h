@@ -72,6 +72,11 @@ struct DecodeArgs {
   const float *pre_ml;
   int pre_splits;
   int pre_kv_tokens;  // positions per prefix item
+  // The grid before this one is the prefix pass, launched in stream order after every writer of
+  // this grid's inputs: the decode streams at once and waits for that grid only before a merge
+  // that reads its partial results (and before its producer exits, so that this grid cannot
+  // complete first).
+  int prefix_overlap;
   // Fused decode step (pa_decode_step with one new token per sequence), when fused != 0: the
   // kernel also performs this cache write (its merge warps, after the previous grid), and reads
   // position L-1 of sequence s from the new token s (step.key / step.value) instead of the
