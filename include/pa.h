@@ -420,7 +420,7 @@ PA_API int pa_decode_noalloc(const pa_tensor *out, const pa_tensor *query,
  *                member's.  0 = nothing shared.
  * Two kernels on `stream`: the prefix pass computes, on the fifth-generation tensor cores,
  * every member's query rows (128 rows = 128 / G members x G heads per tile) against its group's
- * prefix, read once through the first member's block table, in items of 256 positions, and
+ * prefix, read once through the first member's block table, in items of 512 positions, and
  * stores partial results (O / l, running maximum, sum); the decode kernel then walks each
  * sequence's positions prefix_lens[s] .. L-1 and merges its pieces with the prefix partials by
  * the log-sum-exp rule.  A sequence with prefix_lens[s] >= L is decoded over its whole context.

@@ -501,10 +501,13 @@ WsLayout ws_layout(int64_t S, int Hq, int Hkv, int D, int W) {
 #endif
 
 #ifndef PA_PREFIX_ITEM_TOKENS
-#define PA_PREFIX_ITEM_TOKENS 256
+#define PA_PREFIX_ITEM_TOKENS 512
 #endif
 // Positions of one prefix-pass item (a multiple of the prefill kernel's 128-position kv tile):
-// each item leaves one partial result per (member, query head) for the decode to merge.
+// each item leaves one partial result per (member, query head) for the decode to merge.  On the
+// 128-sequence shared-prefix batch (1024-position prompt) the cascade took 64.1 us with items of
+// 256 positions, 63.0 with 512 (half the CTAs, each over four kv tiles, leave SMs to the decode
+// sooner, and each merge takes two prefix pieces instead of four), 67.7 with 1024.
 constexpr int kPrefixItemTokens = PA_PREFIX_ITEM_TOKENS;
 
 struct PrefixLayout {

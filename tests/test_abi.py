@@ -327,7 +327,7 @@ def test_shared_prefix_rejects_bad_arguments_before_cuda(lib):
 
 def test_shared_prefix_workspace_bytes(lib):
     # the decode workspace at the largest default worker count, then (m, l) and O / l of every
-    # (sequence, query head) and 256-position prefix item, each region rounded up to 256 bytes
+    # (sequence, query head) and 512-position prefix item, each region rounded up to 256 bytes
     def up(x):
         return (x + 255) // 256 * 256
 
@@ -336,6 +336,6 @@ def test_shared_prefix_workspace_bytes(lib):
     if base == 0:  # no device: the default worker count is unknown, nothing to check
         assert pa.pa_decode_shared_prefix_workspace_bytes(S, Hq, Hkv, D, MB, bs) == 0
         return
-    splits = (MB * bs + 255) // 256
+    splits = (MB * bs + 511) // 512
     expect = up(base) + up(S * Hq * splits * 2 * 4) + up(S * Hq * splits * D * 4)
     assert pa.pa_decode_shared_prefix_workspace_bytes(S, Hq, Hkv, D, MB, bs) == expect
