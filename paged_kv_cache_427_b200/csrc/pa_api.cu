@@ -496,9 +496,12 @@ WsLayout ws_layout(int64_t S, int Hq, int Hkv, int D, int W) {
 #define PA_PIECE_COST_FP8 3  // the same, FP8 caches
 #endif
 #ifndef PA_PIECE_COST_SHARED
-#define PA_PIECE_COST_SHARED 8  // the same, shared-prefix decode (each piece also merges the
+#define PA_PIECE_COST_SHARED 2  // the same, shared-prefix decode (each piece also merges the
                                 // prefix pass's partial results)
 #endif
+constexpr int kMaxPieceCost = PA_PIECE_COST_16 > PA_PIECE_COST_FP8
+                                  ? (PA_PIECE_COST_16 > PA_PIECE_COST_SHARED ? PA_PIECE_COST_16 : PA_PIECE_COST_SHARED)
+                                  : (PA_PIECE_COST_FP8 > PA_PIECE_COST_SHARED ? PA_PIECE_COST_FP8 : PA_PIECE_COST_SHARED);
 
 #ifndef PA_PREFIX_ITEM_TOKENS
 #define PA_PREFIX_ITEM_TOKENS 512
@@ -692,7 +695,7 @@ int decode_impl(const pa_tensor *out, const pa_tensor *query, const pa_tensor *k
   }
   // a worker counts its share's chunks in 32 bits: at most 2e9 chunks of 16 positions a step
   // (counting each (sequence, kv head) start at the largest piece cost)
-  if ((double)S * num_kv_heads * ((double)block_tables->shape[1] * block_size / 16 + 1 + PA_PIECE_COST_SHARED) > 2.0e9)
+  if ((double)S * num_kv_heads * ((double)block_tables->shape[1] * block_size / 16 + 1 + kMaxPieceCost) > 2.0e9)
     return fail(PA_ERR_SHAPE, "step too large for the work split");
   if (S == 0 || mode == CallMode::kHostChecks) return PA_OK;
   DeviceState *ds;
