@@ -490,10 +490,10 @@ WsLayout ws_layout(int64_t S, int Hq, int Hkv, int D, int W) {
 // Shared-prefix pass: items of kPrefixItemTokens positions; its partial results follow the
 // decode workspace: pre_ml [S*Hq*splits*2] f32 | pre_o [S*Hq*splits*D] f32.
 #ifndef PA_PIECE_COST_16
-#define PA_PIECE_COST_16 1  // split cost of a (sequence, kv head) start, 16-bit caches (chunks)
+#define PA_PIECE_COST_16 2  // split cost of a (sequence, kv head) start, 16-bit caches (chunks)
 #endif
 #ifndef PA_PIECE_COST_FP8
-#define PA_PIECE_COST_FP8 3  // the same, FP8 caches
+#define PA_PIECE_COST_FP8 4  // the same, FP8 caches
 #endif
 #ifndef PA_PIECE_COST_SHARED
 #define PA_PIECE_COST_SHARED 2  // the same, shared-prefix decode (each piece also merges the
@@ -744,7 +744,8 @@ int decode_impl(const pa_tensor *out, const pa_tensor *query, const pa_tensor *k
   // The split's cost of a (sequence, kv head) start, in chunks: what a warp spends once per
   // piece (query rows, partial result, ticket, merge).  Per-warp timings of the Llama-shaped
   // step put it near one chunk's time with 16-bit caches and two to three with FP8 (whose
-  // chunks take less time); the settings are the fastest measured (1 vs 0 and 2; 3 vs 0 and 2).
+  // chunks take less time); once the workers' per-chunk chain was cut, the fastest measured
+  // became 2 for 16-bit caches (against 0, 1, 3) and 4 for FP8 (against 2, 3).
   const int piece_cost = k.tma_rows == 0 ? 0
                          : shared       ? PA_PIECE_COST_SHARED
                          : fp8          ? PA_PIECE_COST_FP8
