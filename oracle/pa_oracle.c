@@ -42,8 +42,9 @@
  * kernel decides the code in).
  *
  * FP8 KV cache ([P2] 4.3 lists FP8 E4M3, 8-bit floating point, ~50 % memory, as a supported
- * storage format; using it for the KV cache with one fp32 scale per kv head is this build's
- * reading): the cache holds code(x / scale[h]) and the attention reads decode(code) * scale[h].
+ * storage format; applying it to the KV cache with one fp32 scale per kv head is a reading of
+ * that passage, which states no scaling): the cache holds code(x / scale[h]) and the attention
+ * reads decode(code) * scale[h].
  * E4M3: 1 sign bit, 4 exponent bits (bias 7), 3 fraction bits; exponent 0 is subnormal
  * (m * 2^-9); S.1111.111 is NaN; no infinities; the largest finite magnitude is 448.
  */
