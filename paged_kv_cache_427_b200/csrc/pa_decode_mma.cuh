@@ -11,13 +11,16 @@
 //   * q.K: mma.sync m16n8k16 with the 16 tokens as M, the query heads of the GQA group as N
 //     (padded to 8 with zeros) and head_dim as K; A comes from the key tile by ldmatrix, B (the
 //     group's query rows) is loaded once per piece into registers.  Products of two 16-bit
-//     values are exact in the fp32 accumulator; the scale is applied to the fp32 result.
+//     values are exact in the fp32 accumulator; the scale is applied to the fp32 result, in the
+//     same FFMA that subtracts the running maximum.
 //   * softmax: base-2 logits, per-head chunk maxima over 8 lanes by shuffles, the running
 //     maximum moved only when a chunk exceeds it by more than 2^8 (weights stay <= 256).
 //   * P.V: mma.sync with head_dim as M (V tile read transposed by ldmatrix.trans), the tokens as
 //     K and the heads as N.  P is split into two 16-bit terms (P = hi + lo, hi = round(P),
 //     lo = round(P - hi)) so the weights keep about 16 significant bits: one 16-bit rounding of P
-//     alone would cost ~2^-9 relative error per weight.
+//     alone would cost ~2^-9 relative error per weight.  With at most 4 heads per kv head the lo
+//     terms ride in the MMA's unused head columns (one MMA per V fragment for both terms).  P
+//     reaches the B operand in registers: movmatrix.trans of each lane's packed C fragment.
 // Warp specialization keeps the copies off the critical path: four worker warps per CTA
 // consume chunks from their own rings, one producer warp issues all copies (see the kernel).
 #pragma once
