@@ -927,8 +927,9 @@ def run_decode(args, b: W.PagedBatch, config: dict, rank: int = 0, world: int = 
                        "ms_per_step": round(e_ms, 5),
                        "how": "per step: one pinned-buffer copy of the step's inputs in (on a copy "
                               "stream, overlapping the previous step's compute; two buffers), the "
-                              "write, the decode, the output copied out and waited for by the host "
-                              "after the next step is launched"}
+                              "write, the decode, the output copied out (on a second copy stream, "
+                              "overlapping the next step's compute; two outputs) and waited for by "
+                              "the host after the next step is launched"}
         s_ms = e2e["serial_ms"] / args.steps
         line["e2e_serial"] = {"value": round(world * step_bytes / (s_ms * 1e-3) / 1e9, 2),
                               "unit": "GB/s", "h2d_bytes_per_step": e2e["h2d"],
@@ -1041,9 +1042,11 @@ def measure_e2e(args, b, pools, rot, mapping, out, ws, decode, dev, stream, worl
 
     # Pipelined, as a serving loop runs it: every step still copies its own inputs in and reads
     # its own result back, but step i's input copy runs on a copy stream while step i-1
-    # computes (two input buffers, two outputs), and the host waits for step i-1's result
-    # after launching step i.
+    # computes (two input buffers, two outputs), step i-1's result goes back on a second copy
+    # stream while step i computes, and the host waits for step i-1's result after launching
+    # step i.
     copy_stream = torch.cuda.Stream(device=dev)
+    d2h_stream = torch.cuda.Stream(device=dev)
     d_bufs = [d_buf, torch.empty_like(d_buf)]
 
     def views(buf):
@@ -1067,6 +1070,7 @@ def measure_e2e(args, b, pools, rot, mapping, out, ws, decode, dev, stream, worl
             d_bufs[j].copy_(h_buf, non_blocking=True)
             ev_in[j].record(copy_stream)
         stream.wait_event(ev_in[j])
+        stream.wait_event(ev_out[j])  # outs[j]'s previous result (step i-2) has left the device
         kc, vc = pools[i % rot]
         dj = d_ins[j]
         if mapping is not None:
@@ -1074,8 +1078,10 @@ def measure_e2e(args, b, pools, rot, mapping, out, ws, decode, dev, stream, worl
         pa.pa_reshape_and_cache(dj["key"], dj["value"], kc, vc, dj["slots"])
         decode(dj["query"], kc, vc, dj["tables"], dj["lens"], o=outs[j])
         ev_used[j].record(stream)
-        h_outs[j].copy_(outs[j], non_blocking=True)
-        ev_out[j].record(stream)
+        with torch.cuda.stream(d2h_stream):
+            d2h_stream.wait_event(ev_used[j])
+            h_outs[j].copy_(outs[j], non_blocking=True)
+            ev_out[j].record(d2h_stream)
         if i >= 1:
             ev_out[1 - j].synchronize()  # step i-1's result is on the host
 
@@ -1085,8 +1091,10 @@ def measure_e2e(args, b, pools, rot, mapping, out, ws, decode, dev, stream, worl
     p0, p1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     p0.record(stream)
     copy_stream.wait_event(p0)  # every copy of the timed region starts after p0
+    d2h_stream.wait_event(p0)
     for i in range(args.steps):
         pipe_step(i)
+    stream.wait_event(ev_out[(args.steps - 1) % 2])  # the region ends with the last result out
     p1.record(stream)
     ev_out[(args.steps - 1) % 2].synchronize()
     torch.cuda.synchronize()
