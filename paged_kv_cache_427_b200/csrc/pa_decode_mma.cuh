@@ -40,14 +40,8 @@ struct MmaType<__nv_bfloat16> {
         : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
   }
-  // p -> (hi, lo) as 16-bit patterns with hi + lo ~= p to about 16 significant bits
-  static __device__ __forceinline__ void split(float p, uint16_t &hi, uint16_t &lo) {
-    const __nv_bfloat16 h = __float2bfloat16_rn(p);
-    const __nv_bfloat16 l = __float2bfloat16_rn(p - __bfloat162float(h));
-    hi = *reinterpret_cast<const uint16_t *>(&h);
-    lo = *reinterpret_cast<const uint16_t *>(&l);
-  }
-  // (x, y) -> packed hi and lo terms, x in the lower half of each
+  // (x, y) -> packed hi and lo terms (hi = round(p), lo = round(p - hi): hi + lo keeps about 16
+  // significant bits of p), x in the lower half of each
   static __device__ __forceinline__ void split2(float x, float y, uint32_t &hi, uint32_t &lo) {
     const __nv_bfloat162 h = __floats2bfloat162_rn(x, y);
     const float2 hf = __bfloat1622float2(h);
@@ -55,6 +49,7 @@ struct MmaType<__nv_bfloat16> {
     hi = *reinterpret_cast<const uint32_t *>(&h);
     lo = *reinterpret_cast<const uint32_t *>(&l);
   }
+  // (x, y) -> their packed hi terms (sel = 0) or lo terms (sel = 1), as split2 gives them
   static __device__ __forceinline__ uint32_t term2(float x, float y, float sel) {
     const __nv_bfloat162 h = __floats2bfloat162_rn(x, y);
     const float2 hf = __bfloat1622float2(h);
@@ -71,12 +66,6 @@ struct MmaType<__half> {
         "{%8,%9}, {%0,%1,%2,%3};"
         : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-  }
-  static __device__ __forceinline__ void split(float p, uint16_t &hi, uint16_t &lo) {
-    const __half h = __float2half_rn(p);
-    const __half l = __float2half_rn(p - __half2float(h));
-    hi = *reinterpret_cast<const uint16_t *>(&h);
-    lo = *reinterpret_cast<const uint16_t *>(&l);
   }
   static __device__ __forceinline__ void split2(float x, float y, uint32_t &hi, uint32_t &lo) {
     const __half2 h = __floats2half2_rn(x, y);
